@@ -1,0 +1,376 @@
+"""Pins of the CPU oracle to things other than itself (runs without a GPU).
+
+* T1  capacity >= sequence length reduces to exact causal attention (the paper,
+      §A.5.2: "for N <= N_C our method reduces to standard training"), checked
+      against an independently written dense softmax from scipy, including the
+      accumulated H2O scores = column sums of the full causal weight matrix.
+* T2  invariants: each softmax row sums to one, so the summed weights of a chunk
+      add up to S * q_g per KV head; weights are >= 0; a new slot gets no
+      weight from rows before its own token (the mask of §A.1).
+* T3  slot selection vs brute force over all subsets on tiny caches, tie-heavy.
+* T4  the hand-derived four-slot toy in tests/golden/h2o_toy_4slot.json.
+* T5  quantization closed forms: exact round trips, error <= scale / 2,
+      hand-packed int4 bytes.
+* T6  attention closed forms: one visible slot gives y = v and lse = logit;
+      zero queries give the mean of the visible values.
+* planted mistakes: altered copies of oracle functions must fail the pins.
+"""
+
+import itertools
+import json
+import math
+import os
+from fractions import Fraction
+
+import numpy as np
+import pytest
+from scipy.special import logsumexp, softmax
+
+import oracle
+from oracle import EMPTY_POS, OracleCache, attend_head, quantize_rows, select_slots
+from oracle import h2o_oracle as ho
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
+
+
+def _frac(s):
+    return float(Fraction(s))
+
+
+# ----------------------------------------------------------------------------
+# Independent textbook attention (T1).
+# ----------------------------------------------------------------------------
+def textbook_causal(Q, K, V):
+    """Q: [Hq, N, d], K/V: [Hk, N, d] float64; plain causal softmax attention.
+    Returns Y [Hq, N, d], LSE [Hq, N], M [Hq, N, N] (rows i, columns j)."""
+    Hq, N, d = Q.shape
+    q_g = Hq // K.shape[0]
+    Y = np.zeros_like(Q)
+    L = np.zeros((Hq, N))
+    M = np.zeros((Hq, N, N))
+    tri = np.triu(np.ones((N, N), bool), k=1)  # j > i is in the future
+    for h in range(Hq):
+        g = h // q_g
+        logits = np.einsum("id,jd->ij", Q[h], K[g]) / np.sqrt(d)
+        logits[tri] = -np.inf
+        M[h] = softmax(logits, axis=1)
+        L[h] = logsumexp(logits, axis=1)
+        Y[h] = np.einsum("ij,jd->id", M[h], V[g])
+    return Y, L, M
+
+
+def run_chunks(cache, Q, K, V, sizes):
+    """Feed [B,H,N,d] arrays through the oracle in chunks of the given sizes.
+    Returns per-chunk (P, S, y, lse, w, wq, slots) and folds the last w in."""
+    out = []
+    P = 0
+    w_prev = None
+    for S in sizes:
+        slots = cache.evict_insert(w_prev, K[:, :, P:P + S], V[:, :, P:P + S], S, P)
+        y, lse, w, wq = cache.attend(Q[:, :, P:P + S], S, P)
+        out.append((P, S, y, lse, w, wq, slots))
+        w_prev = w
+        P += S
+    cache.evict_insert(w_prev, None, None, 0, P)
+    return out
+
+
+def _rand(rng, shape, scale=1.0):
+    return (rng.standard_normal(shape) * scale).astype(np.float32)
+
+
+# ----------------------------------------------------------------------------
+# T1
+# ----------------------------------------------------------------------------
+@pytest.mark.parametrize("sizes,capacity", [([8, 8, 5, 13, 6], 48), ([40], 40), ([1] * 12, 12)])
+def test_t1_no_eviction_equals_textbook_causal(sizes, capacity):
+    rng = np.random.default_rng(7)
+    B, Hq, Hk, d = 2, 4, 2, 16
+    N = sum(sizes)
+    Q = _rand(rng, (B, Hq, N, d))
+    K = _rand(rng, (B, Hk, N, d))
+    V = _rand(rng, (B, Hk, N, d))
+    cache = OracleCache(B, Hq, Hk, d, capacity, "f32")
+    res = run_chunks(cache, Q, K, V, sizes)
+    for b in range(B):
+        Yt, Lt, Mt = textbook_causal(Q[b].astype(np.float64), K[b].astype(np.float64),
+                                     V[b].astype(np.float64))
+        for (P, S, y, lse, w, wq, slots) in res:
+            np.testing.assert_allclose(y[b], Yt[:, P:P + S], rtol=1e-12, atol=1e-12)
+            np.testing.assert_allclose(lse[b], Lt[:, P:P + S], rtol=1e-12, atol=1e-12)
+            # slots fill left to right: token t sits in slot t
+            np.testing.assert_array_equal(slots[b], np.broadcast_to(np.arange(P, P + S), slots[b].shape))
+            # per-head summed weights over this chunk's rows = column sums of M
+            colsum = Mt[:, P:P + S, :].sum(axis=1)  # [Hq, N]
+            np.testing.assert_allclose(wq[b][:, :N], colsum, rtol=1e-12, atol=1e-13)
+        # cumulative H2O score = full-sequence column sums summed over each group
+        full = Mt.sum(axis=1).reshape(Hk, Hq // Hk, N).sum(axis=1)
+        np.testing.assert_allclose(cache.scores[b][:, :N], full, rtol=2e-6, atol=1e-6)
+        assert np.all(cache.scores[b][:, N:] == 0)
+
+
+# ----------------------------------------------------------------------------
+# T2
+# ----------------------------------------------------------------------------
+def _evicting_run(kv="f32", seed=3, d=32, capacity=24, sizes=(8, 8, 8, 8, 5, 8, 3, 8)):
+    rng = np.random.default_rng(seed)
+    B, Hq, Hk = 2, 6, 2
+    N = sum(sizes)
+    Q = _rand(rng, (B, Hq, N, d))
+    K = _rand(rng, (B, Hk, N, d))
+    K[:, :, ::7] *= 4  # a few heavy hitters
+    V = _rand(rng, (B, Hk, N, d))
+    cache = OracleCache(B, Hq, Hk, d, capacity, kv)
+    return cache, run_chunks(cache, Q, K, V, list(sizes)), (Q, K, V)
+
+
+def test_t2_weight_invariants():
+    cache, res, (Q, K, V) = _evicting_run()
+    q_g = cache.q_g
+    for (P, S, y, lse, w, wq, slots) in res:
+        assert np.all(w >= 0) and np.all(wq >= 0)
+        np.testing.assert_allclose(w.sum(axis=-1), S * q_g, rtol=1e-12)
+        np.testing.assert_allclose(wq.sum(axis=-1), S, rtol=1e-12)
+        np.testing.assert_allclose(
+            w, wq.reshape(w.shape[0], w.shape[1], q_g, -1).sum(axis=2), rtol=1e-12, atol=1e-15)
+
+
+def test_t2_new_slot_invisible_to_earlier_rows():
+    # With the chunk's keys written, rows 0..k-1 must put zero weight on the
+    # slot that holds token P+k.
+    rng = np.random.default_rng(11)
+    B, Hq, Hk, d, cap, S = 1, 2, 1, 8, 10, 4
+    cache = OracleCache(B, Hq, Hk, d, cap, "f32")
+    P = 0
+    w_prev = None
+    for c in range(5):
+        k = _rand(rng, (B, Hk, S, d))
+        v = _rand(rng, (B, Hk, S, d))
+        q = _rand(rng, (B, Hq, S, d))
+        slots = cache.evict_insert(w_prev, k, v, S, P)
+        y, lse, w, wq = cache.attend(q, S, P)
+        for kk in range(1, S):
+            _, _, w_trunc, _ = cache.attend(q[:, :, :kk], kk, P)
+            assert w_trunc[0, 0, slots[0, 0, kk]] == 0.0
+        assert w[0, 0, slots[0, 0, S - 1]] > 0
+        w_prev = w
+        P += S
+
+
+# ----------------------------------------------------------------------------
+# T3
+# ----------------------------------------------------------------------------
+def brute_force_select(scores, token_pos, n_new):
+    """Search every subset of size n_new for the one whose members all rank
+    before every non-member under (occupied?, score, slot)."""
+    n = len(scores)
+
+    def key(j):
+        occ = token_pos[j] != EMPTY_POS
+        return (occ, float(scores[j]) if occ else 0.0, j)
+
+    hits = []
+    for sub in itertools.combinations(range(n), n_new):
+        rest = [j for j in range(n) if j not in sub]
+        if all(key(a) < key(b) for a in sub for b in rest):
+            hits.append(list(sub))
+    assert len(hits) == 1
+    return np.array(hits[0])
+
+
+def test_t3_selection_brute_force():
+    rng = np.random.default_rng(5)
+    for trial in range(400):
+        n = int(rng.integers(1, 9))
+        s = int(rng.integers(0, n + 1))
+        scores = rng.integers(0, 3, n).astype(np.float32)  # many ties
+        if trial % 3 == 0:
+            scores = scores + rng.random(n).astype(np.float32)
+        tp = np.arange(n, dtype=np.int64)
+        n_empty = int(rng.integers(0, n + 1)) if trial % 4 == 0 else 0
+        if n_empty:
+            tp[n - n_empty:] = EMPTY_POS
+        got = select_slots(scores, tp, s)
+        np.testing.assert_array_equal(got, brute_force_select(scores, tp, s))
+
+
+def test_t3_documented_example():
+    scores = np.array([2, 1, 1, 1, 3], np.float32)
+    np.testing.assert_array_equal(select_slots(scores, np.arange(5), 2), [1, 2])
+
+
+# ----------------------------------------------------------------------------
+# T4
+# ----------------------------------------------------------------------------
+def _toy_run(Hq):
+    with open(os.path.join(GOLDEN, "h2o_toy_4slot.json")) as f:
+        toy = json.load(f)
+    cache = OracleCache(1, Hq, 1, 2, 4, "f32")
+    rng = np.random.default_rng(0)
+    w_prev = None
+    results = []
+    for ch in toy["chunks"]:
+        P = ch["P"]
+        toks = np.array([P, P + 1])
+        v = np.stack([toks, 10 - toks], axis=-1).astype(np.float32)[None, None]
+        k = _rand(rng, (1, 1, 2, 2))
+        if w_prev is not None:
+            pre = (cache.scores + w_prev.astype(np.float32))[0, 0]
+        else:
+            pre = cache.scores[0, 0].copy()
+        slots = cache.evict_insert(w_prev, k, v, 2, P)
+        y, lse, w, wq = cache.attend(np.zeros((1, Hq, 2, 2), np.float32), 2, P)
+        results.append((ch, pre, slots, y, lse, w))
+        w_prev = w
+    return results
+
+
+def test_t4_hand_derived_toy():
+    for ch, pre, slots, y, lse, w in _toy_run(1):
+        np.testing.assert_allclose(pre, [_frac(s) for s in ch["scores_before_select"]], rtol=1e-6)
+        np.testing.assert_array_equal(slots[0, 0], ch["slots"])
+        np.testing.assert_allclose(w[0, 0], [_frac(s) for s in ch["w"]], rtol=1e-14, atol=1e-15)
+        exp_lse = [math.log(int(s[4:-1])) for s in ch["lse"]]
+        np.testing.assert_allclose(lse[0, 0], exp_lse, rtol=1e-14, atol=1e-15)
+        np.testing.assert_allclose(y[0, 0], [[_frac(a) for a in r] for r in ch["y"]], rtol=1e-14)
+
+
+def test_t4_gqa_copy_doubles_weights():
+    one = _toy_run(1)
+    two = _toy_run(2)
+    for (ch, _, s1, _, _, w1), (_, _, s2, y2, _, w2) in zip(one, two):
+        np.testing.assert_array_equal(s1, s2)
+        np.testing.assert_allclose(w2, 2 * w1, rtol=1e-15)
+        np.testing.assert_allclose(y2[0, 0], y2[0, 1])
+
+
+# ----------------------------------------------------------------------------
+# T5
+# ----------------------------------------------------------------------------
+@pytest.mark.parametrize("kind", ["i8", "i4"])
+def test_t5_exact_round_trip(kind):
+    qmax = oracle.QMAX[kind]
+    rng = np.random.default_rng(2)
+    for sigma in [2.0 ** -3, 2.0 ** -7, 0.5, 2.0 ** 4]:
+        k = rng.integers(-qmax, qmax + 1, size=(16, 8))
+        k[:, 0] = qmax * np.where(rng.random(16) < 0.5, -1, 1)  # max |k| = qmax
+        x = (k * sigma).astype(np.float32)
+        codes, scales = quantize_rows(x, kind)
+        np.testing.assert_array_equal(scales.astype(np.float64), sigma)
+        np.testing.assert_array_equal(codes, k)
+        np.testing.assert_array_equal(oracle.dequantize_rows(codes, scales), x)
+
+
+@pytest.mark.parametrize("kind", ["i8", "i4"])
+def test_t5_error_bound_and_zero_rows(kind):
+    rng = np.random.default_rng(3)
+    x = (rng.standard_normal((200, 128)) * rng.choice([0.01, 1, 40], (200, 1))).astype(np.float32)
+    x[5] = 0.0
+    codes, scales = quantize_rows(x, kind)
+    assert np.all(codes[5] == 0) and scales[5] == 0
+    err = np.abs(oracle.dequantize_rows(codes, scales) - x)
+    assert np.all(err <= scales.astype(np.float64)[:, None] / 2 * (1 + 1e-3) + 1e-30)
+    assert np.all(np.abs(codes) <= oracle.QMAX[kind])
+
+
+def test_t5_int4_packing_by_hand():
+    codes = np.array([[1, -1, 7, -8, 0, 3]], np.int8)
+    packed = oracle.pack_int4(codes)
+    # low nibble = even element: (1 | 0xF<<4), (7 | 0x8<<4), (0 | 3<<4)
+    np.testing.assert_array_equal(packed, [[0xF1, 0x87, 0x30]])
+    np.testing.assert_array_equal(oracle.unpack_int4(packed), codes)
+
+
+def test_t5_scale_rounding_by_hand():
+    # absmax 1.0 over qmax 127: float32(1/127) rounded to fp16 is 0x2008
+    x = np.array([[1.0, -0.5, 0.25, 0.0]], np.float32)
+    codes, scales = quantize_rows(x, "i8")
+    assert scales.view(np.uint16)[0] == 0x2008
+    s = float(np.float16(scales[0]))
+    np.testing.assert_array_equal(codes[0], [round(1.0 / s), round(-0.5 / s), round(0.25 / s), 0])
+
+
+# ----------------------------------------------------------------------------
+# T6
+# ----------------------------------------------------------------------------
+def test_t6_single_visible_slot_and_uniform_queries():
+    rng = np.random.default_rng(9)
+    d, n = 8, 6
+    K = rng.standard_normal((n, d))
+    V = rng.standard_normal((n, d))
+    tp = np.array([3, 50, 51, EMPTY_POS, 52, 53])
+    q = rng.standard_normal((1, d))
+    y, lse, m = attend_head(q, K, V, tp, 3)  # only slot 0 (token 3) visible
+    np.testing.assert_allclose(y[0], V[0], rtol=1e-15)
+    np.testing.assert_allclose(lse[0], q[0] @ K[0] / np.sqrt(d), rtol=1e-14)
+    np.testing.assert_array_equal(m[0], [1, 0, 0, 0, 0, 0])
+    # zero queries: mean of the visible values, lse = log(#visible)
+    y, lse, m = attend_head(np.zeros((3, d)), K, V, tp, 50)
+    np.testing.assert_allclose(y[0], V[:2].mean(0), rtol=1e-14)
+    np.testing.assert_allclose(y[1], V[:3].mean(0), rtol=1e-14)
+    np.testing.assert_allclose(y[2], V[[0, 1, 2, 4]].mean(0), rtol=1e-14)
+    np.testing.assert_allclose(lse, np.log([2, 3, 4]), rtol=1e-14)
+
+
+def test_t6_lse_matches_library_logsumexp():
+    rng = np.random.default_rng(4)
+    d, n, S, P = 16, 40, 7, 30
+    K = rng.standard_normal((n, d)) * 3
+    V = rng.standard_normal((n, d))
+    tp = rng.permutation(n) + 2
+    q = rng.standard_normal((S, d))
+    y, lse, m = attend_head(q, K, V, tp, P)
+    for i in range(S):
+        vis = tp <= P + i
+        a = q[i] @ K[vis].T / np.sqrt(d)
+        np.testing.assert_allclose(lse[i], logsumexp(a), rtol=1e-13)
+        np.testing.assert_allclose(m[i, vis], softmax(a), rtol=1e-12)
+
+
+# ----------------------------------------------------------------------------
+# Planted mistakes must fail the pins.
+# ----------------------------------------------------------------------------
+def _t1_passes():
+    try:
+        test_t1_no_eviction_equals_textbook_causal([8, 8, 5, 13, 6], 48)
+        test_t4_hand_derived_toy()
+        test_t6_single_visible_slot_and_uniform_queries()
+        return True
+    except AssertionError:
+        return False
+
+
+def test_planted_mistakes_are_caught(monkeypatch):
+    assert _t1_passes()
+    good = ho.attend_head
+
+    def off_by_one_mask(q, keys, values, token_pos, P):
+        return good(q, keys, values, token_pos - 1, P)
+
+    def no_scale(q, keys, values, token_pos, P):
+        return good(np.asarray(q) * np.sqrt(q.shape[-1]), keys, values, token_pos, P)
+
+    for bad in (off_by_one_mask, no_scale):
+        monkeypatch.setattr(ho, "attend_head", bad)
+        assert not _t1_passes(), bad.__name__
+        monkeypatch.setattr(ho, "attend_head", good)
+
+    good_sel = ho.select_slots
+
+    def ties_to_highest(scores, token_pos, n_new):
+        r = good_sel(scores[::-1].copy(), token_pos[::-1].copy(), n_new)
+        return np.sort(len(scores) - 1 - r)
+
+    monkeypatch.setattr(ho, "select_slots", ties_to_highest)
+    with pytest.raises(AssertionError):
+        test_t3_selection_brute_force_with(ho.select_slots)
+
+
+def test_t3_selection_brute_force_with(sel=select_slots):
+    rng = np.random.default_rng(8)
+    for _ in range(200):
+        n = int(rng.integers(2, 8))
+        s = int(rng.integers(1, n))
+        scores = rng.integers(0, 2, n).astype(np.float32)
+        tp = np.arange(n)
+        np.testing.assert_array_equal(sel(scores, tp, s), brute_force_select(scores, tp, s))
