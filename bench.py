@@ -1,0 +1,451 @@
+#!/usr/bin/env python3
+"""Benchmark: chunked cache attention + summed weights + H2O eviction.
+
+One step = one sequence of one attention layer pushed through the whole hot
+path, chunk by chunk (h2o_evict_insert, then attn_chunk_with_scoresum), plus the
+final fold of the last chunk's weights.  Default workload: the Qwen3-4B-shaped
+layer at 128K tokens (batch 1, 32 query / 8 KV heads, head_dim 128, bf16, a
+32768-slot cache, chunks of 1024).  Metric: tokens per second over all ranks.
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--config 128k|64k|int8|int4stack]
+  python bench.py --impl reference ...   # the CPU oracle on the host cores
+
+Under torchrun each rank runs its own layer (seed + rank): the path has no
+exchange step, so scaling is weak and no collective runs on the data path.
+"""
+
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import numpy as np  # noqa: E402
+import torch  # noqa: E402
+
+from h2o_kv_cache_attn_b200.configs import SHORT  # noqa: E402
+
+METRIC = "chunked cache-attention+scoresum tokens/s; % BF16 tensor peak; evict µs/chunk"
+UNIT = "tokens/s"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+def peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return d, "measured"
+    return FALLBACK_PEAKS, "fallback"
+
+
+# --------------------------------------------------------------------------- #
+def dist_init():
+    ws = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if ws > 1:
+        import datetime
+
+        import torch.distributed as dist
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    return ws, rank, local
+
+
+def barrier(ws):
+    if ws > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def max_over_ranks(x, ws):
+    if ws == 1:
+        return x
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+class ClockSampler:
+    """nvidia-smi samples of SM clock and throttle reasons during the timed region."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index):
+        self.gpu = gpu_index
+        self.proc = None
+        self.lines = []
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "200"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.t = threading.Thread(target=self._read, daemon=True)
+            self.t.start()
+        except (FileNotFoundError, OSError):
+            self.proc = None
+        return self
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def __exit__(self, *a):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+
+    def summary(self):
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            parts = [p.strip() for p in ln.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                mx = float(parts[2])
+            except ValueError:
+                continue
+            for n, v in zip(names, parts[5:9]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": mx,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+# --------------------------------------------------------------------------- #
+def kernel_source_hash():
+    h = hashlib.sha256()
+    csrc = os.path.join(ROOT, "h2o_kv_cache_attn_b200", "csrc")
+    for f in sorted(os.listdir(csrc)):
+        with open(os.path.join(csrc, f), "rb") as fh:
+            h.update(f.encode() + fh.read())
+    return h.hexdigest()[:16]
+
+
+def recorded_traffic(kernel_name):
+    """DRAM bytes per launch from the committed ncu summary, if it was taken on
+    the current kernel sources (else None)."""
+    p = os.path.join(ROOT, "profiles", "dram_traffic.json")
+    if not os.path.exists(p):
+        return None
+    with open(p) as f:
+        d = json.load(f)
+    e = d.get(kernel_name)
+    if not e or e.get("source_hash") != kernel_source_hash():
+        return None
+    return e.get("bytes_per_launch")
+
+
+def alg_flops_chunk(wl, n_valid, S):
+    """Algorithmic attention FLOPs of one chunk: QK^T and PV over the valid
+    slots, 4 * B * H_q * S * n_valid * d."""
+    return 4.0 * wl.B * wl.Hq * S * n_valid * wl.d
+
+
+def exec_flops_chunk(wl, n_valid, S):
+    """Executed tensor FLOPs: the score-sum pass recomputes QK^T once more."""
+    return 6.0 * wl.B * wl.Hq * S * n_valid * wl.d
+
+
+def evict_bytes_chunk(wl, S):
+    """Algorithmic HBM bytes of one evict/insert call: scores read+write and
+    w_prev read (3 * 4 * N_C), new K/V read (2 * S * d * 2), stored K/V rows and
+    scales written, token_pos and slot list written, per (b, h_k)."""
+    row = {"f32": wl.d * 4, "bf16": wl.d * 2, "i8": wl.d, "i4": wl.d // 2}[wl.kv_dtype]
+    sc = 2 if wl.kv_dtype in ("i8", "i4") else 0
+    per = 3 * 4 * wl.capacity + 2 * S * wl.d * 2 + 2 * S * (row + sc) + 2 * S * 4
+    return per * wl.B * wl.Hk
+
+
+# --------------------------------------------------------------------------- #
+def run_ours(args, wl, ws, rank, local):
+    from h2o_kv_cache_attn_b200 import binding as hb
+    from h2o_kv_cache_attn_b200.runner import LayerRunner
+    from h2o_kv_cache_attn_b200.synth import ChunkSource
+
+    hb.load()  # raises if the CUDA library is missing
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    stream = torch.cuda.current_stream(dev)
+    src = ChunkSource(wl, layer=rank, device=dev)
+    chunks = [src.chunk(c) for c in range(wl.n_chunks)]
+    runner = LayerRunner(wl, dev, with_wq=False, with_lse=False)
+    n_valid = [min(wl.capacity, (c + 1) * wl.chunk) for c in range(wl.n_chunks)]
+
+    def one_step(events=None):
+        runner.reset()
+        for c, (q, k, v) in enumerate(chunks):
+            S = q.shape[2]
+            if events is not None:
+                e0, e1, e2 = (torch.cuda.Event(enable_timing=True) for _ in range(3))
+                e0.record(stream)
+            runner.cache.evict_insert(runner.w_prev(), k, v, S, runner.P, None)
+            if events is not None:
+                e1.record(stream)
+            runner.cache.attend(q, S, runner.P, runner.y if S == wl.chunk else torch.empty_like(q),
+                                None, runner.w_cur(), None)
+            if events is not None:
+                e2.record(stream)
+                events.append((c, e0, e1, e2))
+            runner.chunk_index += 1
+            runner.P += S
+        runner.finish()
+
+    for _ in range(args.warmup):
+        one_step()
+    torch.cuda.synchronize()
+    barrier(ws)
+    torch.cuda.synchronize()
+    events = []
+    with ClockSampler(local) as clk:
+        t0 = torch.cuda.Event(enable_timing=True)
+        t1 = torch.cuda.Event(enable_timing=True)
+        t0.record(stream)
+        for _ in range(args.steps):
+            one_step(events)
+        t1.record(stream)
+        torch.cuda.synchronize()
+    barrier(ws)
+    torch.cuda.synchronize()
+    ms_total = max_over_ranks(t0.elapsed_time(t1), ws)
+    ms_step = ms_total / args.steps
+    tokens_step = wl.B * wl.seq_len
+    value = tokens_step * ws * args.steps / (ms_total / 1e3)
+
+    # per-call durations inside the timed region
+    ev_ms, at_ms, at_flops_exec, at_flops_alg = [], [], 0.0, 0.0
+    evict_full_ms = []
+    for (c, e0, e1, e2) in events:
+        ev = e0.elapsed_time(e1)
+        at = e1.elapsed_time(e2)
+        ev_ms.append(ev)
+        at_ms.append(at)
+        S = wl.chunk_len(c)
+        at_flops_exec += exec_flops_chunk(wl, n_valid[c], S)
+        at_flops_alg += alg_flops_chunk(wl, n_valid[c], S)
+        if n_valid[c] == wl.capacity and c * wl.chunk >= wl.capacity:
+            evict_full_ms.append(ev)
+    at_total_s = sum(at_ms) / 1e3
+    pk, pk_kind = peaks()
+    tc_peak = pk.get("bf16_tflops_sustained", pk["bf16_tflops"])
+    tflops_exec = at_flops_exec / at_total_s / 1e12
+    tflops_alg = at_flops_alg / at_total_s / 1e12
+    evict_us = statistics.median(evict_full_ms) * 1e3 if evict_full_ms else None
+    evict_gbs = evict_bytes_chunk(wl, wl.chunk) / (evict_us * 1e-6) / 1e9 if evict_us else None
+    tc_used = bool(runner.cache.shape.head_dim == 128 and wl.kv_dtype != "f32" and _tc_enabled())
+    n_launches_attn = 1 if tc_used else 2
+    launches_per_step = wl.n_chunks * (2 + n_launches_attn) + 1
+    per_launch_flops = at_flops_exec / len(at_ms)
+    per_launch_ms = sum(at_ms) / len(at_ms)
+    if tc_used:
+        roof = {"bound": "tensor", "achieved": round(tflops_exec, 2), "peak": tc_peak,
+                "unit": "TFLOP/s", "frac": round(tflops_exec / tc_peak, 4),
+                "traffic": recorded_traffic("attn_tc"),
+                "kernel": "attention (one fused launch per chunk)",
+                "flops_per_launch": per_launch_flops, "avg_launch_ms": round(per_launch_ms, 4),
+                "peak_kind": f"{pk_kind} bf16 sustained"}
+    else:
+        fma_peak = 148 * 128 * 2 * 1.965e9 / 1e12
+        roof = {"bound": "alu", "achieved": round(tflops_exec, 2), "peak": round(fma_peak, 1),
+                "unit": "TFLOP/s", "frac": round(tflops_exec / fma_peak, 4),
+                "traffic": recorded_traffic("attn_simt"),
+                "kernel": "attention, CUDA-core path (2 launches per chunk)",
+                "flops_per_launch": per_launch_flops, "avg_launch_ms": round(per_launch_ms, 4),
+                "peak_kind": "derived: 148 SMs x 128 FP32 FMA/clk x 2 x 1965 MHz"}
+    extra = {"pct_bf16_peak_exec": round(100 * tflops_exec / tc_peak, 2),
+             "pct_bf16_peak_alg": round(100 * tflops_alg / tc_peak, 2),
+             "evict_us_per_chunk": round(evict_us, 2) if evict_us else None,
+             "evict_gbs": round(evict_gbs, 1) if evict_gbs else None,
+             "evict_frac_hbm": round(evict_gbs / pk["hbm_gbs"], 4) if evict_gbs else None,
+             "attn_ms_per_step": round(sum(at_ms) / args.steps, 3),
+             "evict_ms_per_step": round(sum(ev_ms) / args.steps, 3)}
+    clocks = clk.summary()
+    res = dict(value=value, ms_step=ms_step, roof=roof, extra=extra, clocks=clocks,
+               launches=launches_per_step * args.steps)
+
+    # ---- end to end through the public API, host buffers ----------------------
+    host = [(q.cpu().pin_memory(), k.cpu().pin_memory(), v.cpu().pin_memory()) for (q, k, v) in chunks]
+    del chunks
+    q_d = torch.empty_like(host[0][0], device=dev)
+    k_d = torch.empty_like(host[0][1], device=dev)
+    v_d = torch.empty_like(host[0][2], device=dev)
+    y_h = torch.empty(host[0][0].shape, dtype=host[0][0].dtype).pin_memory()
+    w_h = torch.empty((wl.B, wl.Hk, wl.capacity), dtype=torch.float32).pin_memory()
+    h2d = sum(t.numel() * t.element_size() for ch in host for t in ch)
+    d2h = wl.n_chunks * (y_h.numel() * y_h.element_size() + w_h.numel() * w_h.element_size())
+
+    def e2e_step():
+        runner.reset()
+        for c, (qh, kh, vh) in enumerate(host):
+            S = qh.shape[2]
+            qd, kd, vd = (q_d, k_d, v_d) if S == wl.chunk else (torch.empty_like(qh, device=dev),
+                                                               torch.empty_like(kh, device=dev),
+                                                               torch.empty_like(vh, device=dev))
+            qd.copy_(qh, non_blocking=True)
+            kd.copy_(kh, non_blocking=True)
+            vd.copy_(vh, non_blocking=True)
+            y, _, w, _, _ = runner.step(qd, kd, vd)
+            if S == wl.chunk:
+                y_h.copy_(y, non_blocking=True)
+            w_h.copy_(w, non_blocking=True)
+        runner.finish()
+
+    e2e_step()
+    torch.cuda.synchronize()
+    barrier(ws)
+    torch.cuda.synchronize()
+    t0 = torch.cuda.Event(enable_timing=True)
+    t1 = torch.cuda.Event(enable_timing=True)
+    t0.record(stream)
+    for _ in range(args.steps):
+        e2e_step()
+    t1.record(stream)
+    torch.cuda.synchronize()
+    barrier(ws)
+    ms_e2e = max_over_ranks(t0.elapsed_time(t1), ws)
+    res["e2e"] = {"value": tokens_step * ws * args.steps / (ms_e2e / 1e3), "unit": UNIT,
+                  "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h}
+    res["tc_used"] = tc_used
+    return res
+
+
+def _tc_enabled():
+    try:
+        from h2o_kv_cache_attn_b200 import binding as hb
+        lib = hb.load()
+        return hasattr(lib, "h2okv_tc_enabled") and bool(lib.h2okv_tc_enabled())
+    except Exception:
+        return False
+
+
+# --------------------------------------------------------------------------- #
+def oracle_sample(wl, groups=1, chunk=None, layer=0):
+    """Time the CPU oracle on one steady-state eviction chunk for `groups` of the
+    B*H_k (batch row, KV head) groups; extrapolate to tokens/s of the whole
+    workload (every group, one chunk of S tokens per group per chunk)."""
+    import oracle
+    from h2o_kv_cache_attn_b200.synth import ChunkSource
+
+    if chunk is None:
+        chunk = -(-wl.capacity // wl.chunk) + 1  # the second eviction chunk
+    src = ChunkSource(wl, layer, "cpu")
+    q, k, v = src.chunk(chunk)
+    q, k, v = (t.float().numpy() for t in (q, k, v))
+    rng = np.random.default_rng(1)
+    S = q.shape[2]
+    P = chunk * wl.chunk
+    # a full cache of earlier tokens with random scores (the sample's state)
+    oc = oracle.OracleCache(1, wl.q_g, 1, wl.d, wl.capacity, wl.kv_dtype)
+    kk = rng.standard_normal((1, 1, wl.capacity, wl.d)).astype(np.float32)
+    vv = rng.standard_normal((1, 1, wl.capacity, wl.d)).astype(np.float32)
+    oc.evict_insert(None, kk, vv, wl.capacity, P - wl.capacity)
+    oc.scores[:] = rng.random(oc.scores.shape).astype(np.float32)
+    w_prev = rng.random((1, 1, wl.capacity)).astype(np.float32)
+    t0 = time.perf_counter()
+    for gi in range(groups):
+        b, g = divmod(gi, wl.Hk)
+        oc.evict_insert(w_prev, k[b:b + 1, g:g + 1], v[b:b + 1, g:g + 1], S, P)
+        oc.attend(q[b:b + 1, g * wl.q_g:(g + 1) * wl.q_g], S, P)
+    dt = time.perf_counter() - t0
+    n_groups = wl.B * wl.Hk * wl.layers
+    chunk_s = dt / groups * n_groups
+    tokens_per_s = wl.B * S / chunk_s
+    try:
+        import threadpoolctl
+        info = threadpoolctl.threadpool_info()
+        cores = max((i.get("num_threads", 1) for i in info), default=1)
+    except Exception:
+        cores = os.cpu_count()
+    return {"value": tokens_per_s, "unit": UNIT, "cores": cores, "kind": "oracle",
+            "sample": (f"one steady-state eviction chunk (S={S}, P={P}) for {groups} of "
+                       f"{n_groups} (batch, KV-head) groups, float64 numpy oracle; "
+                       f"{dt:.2f} s measured, extrapolated to all groups"),
+            "seconds": dt}
+
+
+# --------------------------------------------------------------------------- #
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=5)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--config", default="128k", choices=sorted(SHORT))
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    wl = SHORT[args.config]
+    if args.warmup < 3:
+        print("warning: --warmup < 3; using 3", file=sys.stderr)
+        args.warmup = 3
+    ws = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+
+    config = {"workload": wl.name, "batch": wl.B, "q_heads": wl.Hq, "kv_heads": wl.Hk,
+              "head_dim": wl.d, "cache_slots": wl.capacity, "seq_len": wl.seq_len,
+              "chunk": wl.chunk, "kv_dtype": wl.kv_dtype, "layers_per_rank": 1,
+              "parallelism": f"independent layers x{ws} (no collective)",
+              "l2": "inputs larger than L2 (cache buffers + chunk inputs > 126 MB per step)"}
+
+    if args.impl == "reference":
+        if rank != 0:
+            return 0
+        vals = []
+        for s in range(args.warmup + args.steps):
+            r = oracle_sample(wl, groups=1)
+            if s >= args.warmup:
+                vals.append(r)
+        value = statistics.median(v["value"] for v in vals)
+        line = {"impl": "reference", "metric": METRIC, "value": value, "unit": UNIT,
+                "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+                "ms_per_step": wl.B * wl.seq_len / value * 1e3, "higher_is_better": True,
+                "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+                "data": "synthetic (seeded, recipe of the workload)", "config": config,
+                "cpu_baseline": {k: vals[-1][k] for k in ("kind", "cores", "sample")} | {"value": value},
+                "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+        print(json.dumps(line))
+        return 0
+
+    ws, rank, local = dist_init()
+    res = run_ours(args, wl, ws, rank, local)
+    cpu = None
+    if rank == 0 and ws == 1 and not args.no_cpu_baseline:
+        cpu = oracle_sample(wl, groups=1)
+        cpu.pop("seconds", None)
+    if rank == 0:
+        line = {"metric": METRIC, "value": res["value"], "unit": UNIT, "n_gpus": ws,
+                "steps": args.steps, "warmup": args.warmup, "ms_per_step": res["ms_step"],
+                "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+                "dtype": "f32" if wl.q_dtype == "f32" else "bf16",
+                "data": "synthetic (seeded N(0,1), 1% heavy-hitter keys x4, bf16)", "config": config,
+                "roofline": res["roof"], "cpu_baseline": cpu, "e2e": res["e2e"],
+                "gpu_launches": res["launches"], "clocks": res["clocks"], **res["extra"]}
+        print(json.dumps(line))
+    if ws > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,74 @@
+// Internal declarations shared by the library's translation units.
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_fp16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "h2okv.h"
+
+namespace h2okv {
+
+constexpr int32_t kEmptyPos = INT32_MAX;
+constexpr int kMaxHeadDim = 256;
+constexpr int kMaxCapacity = 65536;
+
+// Workspace carve-up of one cache (all offsets 256-byte aligned).
+struct WorkspaceLayout {
+  size_t slot_list;    // int32 [B*Hk*max_chunk]: chosen slots, ascending per (b, h_k)
+  size_t sel_keys;     // uint32 [B*Hk*N_C]: selection keys when they do not fit in shared memory
+  size_t lse2;         // float [B*Hq*max_chunk]: base-2 log-sum-exp per query row
+  size_t part_ml;      // float2 [splits*B*Hq*rows_pad]: split-KV partial (max, sum) for pass 1
+  size_t part_w;       // float [B*Hq*row_tiles*N_C]: per-row-tile summed weights (tensor-core path)
+  size_t part_o;       // float [splits*B*Hq*rows_pad*d]: split-KV partial outputs (tensor-core path)
+  size_t total;
+};
+
+struct TcPlan {          // launch plan of the tensor-core path
+  bool enabled;
+  int tiles_per_head;    // ceil(max_chunk / 128)
+  int max_splits;        // key splits the workspace is sized for
+};
+
+}  // namespace h2okv
+
+struct h2okv_cache {
+  h2okv_cache_desc desc;
+  h2okv_cache_buffers bufs;
+  int32_t n_filled;
+  size_t row_bytes;  // bytes of one stored key/value row
+  h2okv::WorkspaceLayout ws;
+  h2okv::TcPlan tc;
+};
+
+namespace h2okv {
+
+// Error reporting (thread-local message).
+int set_error(int code, const char *fmt, ...);
+int check_launch(const char *what);
+
+inline size_t kv_row_bytes(int kv_dtype, int d) {
+  switch (kv_dtype) {
+    case H2OKV_F32: return (size_t)d * 4;
+    case H2OKV_BF16: return (size_t)d * 2;
+    case H2OKV_I8: return (size_t)d;
+    case H2OKV_I4: return (size_t)d / 2;
+  }
+  return 0;
+}
+
+// ---- launchers (return H2OKV_OK or an error code) -------------------------
+int launch_init_cache(h2okv_cache *c, cudaStream_t st);
+int launch_evict_insert(h2okv_cache *c, const float *w_prev, const void *k_new, const void *v_new,
+                        int S, int64_t P, int32_t *slots_out, cudaStream_t st);
+int launch_quantize(int kv_dtype, const __nv_bfloat16 *x, int64_t n_rows, int d, void *codes,
+                    __half *scales, cudaStream_t st);
+int launch_attn_simt(h2okv_cache *c, const void *q, int S, int64_t P, void *y, float *lse,
+                     float *w, float *wq, cudaStream_t st);
+bool tc_path_supported(const h2okv_cache_desc &d);
+int launch_attn_tc(h2okv_cache *c, const void *q, int S, int64_t P, void *y, float *lse, float *w,
+                   float *wq, cudaStream_t st);
+void tc_plan(const h2okv_cache_desc &d, TcPlan *plan);
+
+}  // namespace h2okv

@@ -159,12 +159,18 @@ def attend_head(q: np.ndarray, keys: np.ndarray, values: np.ndarray,
     rows = P + np.arange(S, dtype=np.int64)[:, None]
     masked = rows < token_pos.astype(np.int64)[None, :]
     a = np.where(masked, -np.inf, a)
+    seen = ~np.all(masked, axis=1)
     amax = np.max(a, axis=1, keepdims=True)
+    amax = np.where(seen[:, None], amax, 0.0)
     e = np.exp(a - amax)
     total = np.sum(e, axis=1, keepdims=True)
-    m = e / total
+    # A row with no visible slot (only possible if the chunk's own keys were not
+    # inserted first) has an empty softmax: by convention it gets zero weights,
+    # y = 0 and lse = -inf.
+    m = e / np.where(seen[:, None], total, 1.0)
     y = m @ v
-    lse = (amax + np.log(total))[:, 0]
+    with np.errstate(divide="ignore"):
+        lse = (amax + np.log(total))[:, 0]
     return y, lse, m
 
 

@@ -312,6 +312,15 @@ def test_t6_single_visible_slot_and_uniform_queries():
     np.testing.assert_allclose(lse, np.log([2, 3, 4]), rtol=1e-14)
 
 
+def test_row_without_visible_slot_convention():
+    d = 4
+    K = np.ones((3, d))
+    V = np.ones((3, d))
+    y, lse, m = attend_head(np.ones((2, d)), K, V, np.array([5, EMPTY_POS, 9]), 4)
+    assert lse[0] == -np.inf and np.all(y[0] == 0) and np.all(m[0] == 0)
+    assert lse[1] == 2.0 and m[1, 0] == 1.0  # q.k / sqrt(d) = 4 / 2
+
+
 def test_t6_lse_matches_library_logsumexp():
     rng = np.random.default_rng(4)
     d, n, S, P = 16, 40, 7, 30
