@@ -173,9 +173,9 @@ def test_error_paths_leave_device_usable(cuda_device):
         hb.attn_chunk_with_scoresum(run.cache.handle, q, 0, 0, run.y, None, run.w[0])
     with pytest.raises(hb.H2OKVError):
         hb.attn_chunk_with_scoresum(run.cache.handle, q, 33, 0, run.y, None, run.w[0])
-    run.step(q, k, v)
+    y, lse, w, wq, slots = run.step(q, k, v)
     torch.cuda.synchronize()
-    assert abs(float(run.w_cur().sum()) - 32 * wl.q_g * wl.B * wl.Hk) < 1e-2
+    assert abs(float(w.sum()) - 32 * wl.q_g * wl.B * wl.Hk) < 1e-2
 
 
 # ---------------------------------------------------------------------------
