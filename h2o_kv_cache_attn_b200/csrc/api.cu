@@ -80,6 +80,8 @@ static void layout(const h2okv_cache_desc &d, const TcPlan &tc, WorkspaceLayout 
   if (d.capacity > kSmemKeyCap) off = align256(off + B * Hk * NC * 4);
   ws->lse2 = off;
   off = align256(off + B * Hq * S * 4);
+  ws->status = off;
+  off = align256(off + 4);
   ws->part_ml = ws->part_w = ws->part_o = off;
   if (tc.enabled) {
     const size_t rows_pad = (size_t)tc.tiles_per_head * 128;
@@ -156,6 +158,8 @@ int kv_cache_create(const h2okv_cache_desc *desc, const h2okv_cache_buffers *buf
   c->n_filled = 0;
   c->row_bytes = kv_row_bytes(desc->kv_dtype, desc->head_dim);
   tc_plan(*desc, &c->tc);
+  c->tc.maps_ready = false;
+  c->wait_timeout_ns = kDefaultWaitTimeoutNs;
   layout(*desc, c->tc, &c->ws);
   rc = launch_init_cache(c, (cudaStream_t)stream);
   if (rc) {
@@ -172,6 +176,28 @@ int kv_cache_reset(h2okv_cache *c, void *stream) {
   int rc = launch_init_cache(c, (cudaStream_t)stream);
   if (rc) return rc;
   c->n_filled = 0;
+  return H2OKV_OK;
+}
+
+int kv_cache_device_status(h2okv_cache *c, int32_t *status, void *stream) {
+  g_err[0] = 0;
+  if (!c || !status) return set_error(H2OKV_ERR_INVALID_ARG, "NULL argument");
+  cudaStream_t st = (cudaStream_t)stream;
+  int32_t *dev = reinterpret_cast<int32_t *>(reinterpret_cast<uint8_t *>(c->bufs.workspace) +
+                                             c->ws.status);
+  int32_t v = 0;
+  if (cudaMemcpyAsync(&v, dev, 4, cudaMemcpyDeviceToHost, st) != cudaSuccess ||
+      cudaMemsetAsync(dev, 0, 4, st) != cudaSuccess || cudaStreamSynchronize(st) != cudaSuccess)
+    return set_error(H2OKV_ERR_CUDA, "reading the device status word failed: %s",
+                     cudaGetErrorString(cudaGetLastError()));
+  *status = v;
+  return H2OKV_OK;
+}
+
+int kv_cache_set_wait_timeout(h2okv_cache *c, uint64_t timeout_ns) {
+  g_err[0] = 0;
+  if (!c) return set_error(H2OKV_ERR_INVALID_ARG, "cache is NULL");
+  c->wait_timeout_ns = timeout_ns;
   return H2OKV_OK;
 }
 

@@ -273,6 +273,9 @@ __global__ void init_kernel(int32_t *__restrict__ token_pos, float *__restrict__
 
 int launch_init_cache(h2okv_cache *c, cudaStream_t st) {
   const size_t n = (size_t)c->desc.batch * c->desc.n_kv_heads * c->desc.capacity;
+  if (cudaMemsetAsync(reinterpret_cast<uint8_t *>(c->bufs.workspace) + c->ws.status, 0, 4, st) !=
+      cudaSuccess)
+    return set_error(H2OKV_ERR_CUDA, "cudaMemsetAsync(status) failed");
   const int blocks = (int)((n + 255) / 256 < 4096 ? (n + 255) / 256 : 4096);
   init_kernel<<<blocks, 256, 0, st>>>(c->bufs.token_pos, c->bufs.scores, n);
   return check_launch("init_kernel");

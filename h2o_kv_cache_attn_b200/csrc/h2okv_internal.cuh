@@ -22,6 +22,7 @@ struct WorkspaceLayout {
   size_t part_ml;      // float2 [splits*B*Hq*rows_pad]: split-KV partial (max, sum) for pass 1
   size_t part_w;       // float [B*Hq*row_tiles*N_C]: per-row-tile summed weights (tensor-core path)
   size_t part_o;       // float [splits*B*Hq*rows_pad*d]: split-KV partial outputs (tensor-core path)
+  size_t status;       // int32: device status word (0 = ok, else an H2OKV_ERR_* code)
   size_t total;
 };
 
@@ -29,7 +30,12 @@ struct TcPlan {          // launch plan of the tensor-core path
   bool enabled;
   int tiles_per_head;    // ceil(max_chunk / 128)
   int max_splits;        // key splits the workspace is sized for
+  bool maps_ready;       // k_map / v_map encoded
+  alignas(64) unsigned char k_map[128];  // CUtensorMap over keys
+  alignas(64) unsigned char v_map[128];  // CUtensorMap over values
 };
+
+constexpr uint64_t kDefaultWaitTimeoutNs = 2000000000ull;  // bounded device waits
 
 }  // namespace h2okv
 
@@ -40,6 +46,7 @@ struct h2okv_cache {
   size_t row_bytes;  // bytes of one stored key/value row
   h2okv::WorkspaceLayout ws;
   h2okv::TcPlan tc;
+  uint64_t wait_timeout_ns;
 };
 
 namespace h2okv {

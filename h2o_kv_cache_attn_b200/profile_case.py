@@ -1,0 +1,64 @@
+"""A short, steady-state run of the hot path for profiler captures.
+
+``python -m h2o_kv_cache_attn_b200.profile_case [--config 128k] [--iters 3]``
+
+Fills one layer's cache directly (every slot occupied, random keys, values and
+scores), then runs ``--iters`` eviction chunks (h2o_evict_insert followed by
+attn_chunk_with_scoresum).  Only a handful of launches precede the measured
+ones, so a profiler can capture e.g. the second attention launch of a full
+128K-token / 32768-slot layer with the cache larger than L2.
+"""
+
+from __future__ import annotations
+
+import argparse
+
+import torch
+
+from .configs import SHORT
+from .runner import LayerRunner
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--config", default="128k", choices=sorted(SHORT))
+    ap.add_argument("--iters", type=int, default=3)
+    args = ap.parse_args()
+    wl = SHORT[args.config]
+    dev = torch.device("cuda:0")
+    g = torch.Generator(device=dev)
+    g.manual_seed(wl.seed)
+    run = LayerRunner(wl, dev, with_wq=False, with_lse=False)
+    c = run.cache
+    if wl.kv_dtype in ("bf16", "f32"):
+        c.keys.copy_(torch.randn(c.keys.shape, generator=g, device=dev))
+        c.values.copy_(torch.randn(c.values.shape, generator=g, device=dev))
+    else:
+        c.keys.copy_(torch.randint(-100, 100, c.keys.shape, generator=g, device=dev).to(c.keys.dtype))
+        c.values.copy_(torch.randint(-100, 100, c.values.shape, generator=g, device=dev).to(c.values.dtype))
+        c.k_scales.fill_(0.01)
+        c.v_scales.fill_(0.01)
+    c.token_pos.copy_(torch.arange(wl.capacity, dtype=torch.int32, device=dev).expand_as(c.token_pos))
+    c.scores.copy_(torch.rand(c.scores.shape, generator=g, device=dev))
+    c.set_fill(wl.capacity)
+    qt = torch.float32 if wl.q_dtype == "f32" else torch.bfloat16
+    kvt = torch.float32 if wl.kv_dtype == "f32" else torch.bfloat16
+    S = wl.chunk
+    q = torch.randn((wl.B, wl.Hq, S, wl.d), generator=g, device=dev).to(qt)
+    k = torch.randn((wl.B, wl.Hk, S, wl.d), generator=g, device=dev).to(kvt)
+    v = torch.randn((wl.B, wl.Hk, S, wl.d), generator=g, device=dev).to(kvt)
+    run.P = wl.capacity
+    run.chunk_index = 1  # the cache is full: the first w_prev is the zero buffer
+    for _ in range(args.iters):
+        run.step(q, k, v)
+    torch.cuda.synchronize()
+    w = run.last[2]
+    total = float(w.sum())
+    expect = wl.B * wl.Hk * S * wl.q_g
+    print(f"profile_case {wl.name}: {args.iters} chunks, sum(w) = {total:.1f} (expect {expect})")
+    if abs(total - expect) > 1e-3 * expect:
+        raise SystemExit("summed weights do not add up")
+
+
+if __name__ == "__main__":
+    main()

@@ -126,6 +126,19 @@ H2OKV_API int kv_cache_destroy(h2okv_cache *cache);
 H2OKV_API int kv_cache_get_fill(const h2okv_cache *cache, int32_t *n_filled);
 H2OKV_API int kv_cache_set_fill(h2okv_cache *cache, int32_t n_filled);
 
+/* Device status of a cache: the tensor-core kernels bound every wait on
+ * another warp or on a copy; when a wait exceeds the cache's limit the kernel
+ * stops early, drains its own copies and matrix operations, frees its tensor
+ * memory and records H2OKV_ERR_TIMEOUT here (outputs of that call are then
+ * undefined).  This call synchronizes `stream`, returns the recorded status
+ * (0 = ok) in *status and clears it. */
+H2OKV_API int kv_cache_device_status(h2okv_cache *cache, int32_t *status, void *stream);
+
+/* Limit of each bounded device-side wait, in nanoseconds (default 2 s).  A
+ * limit of 0 makes the first wait that does not complete at once give up:
+ * use it only to exercise the timeout path. */
+H2OKV_API int kv_cache_set_wait_timeout(h2okv_cache *cache, uint64_t timeout_ns);
+
 /* Quantize n_rows rows of head_dim bf16 values (the 8/4-bit cache format, §2 /
  * §A.10; the paper gives only the bit width, the scheme is):
  *   scale = fp16_rn(min(absmax / qmax, 65504)), qmax = 127 (I8) or 7 (I4);
