@@ -17,11 +17,13 @@ from .binding import (  # noqa: F401
     h2okv_last_error,
     kv_cache_create,
     kv_cache_destroy,
+    kv_cache_device_status,
     kv_cache_get_fill,
     kv_cache_quantize,
     kv_cache_query_sizes,
     kv_cache_reset,
     kv_cache_set_fill,
+    kv_cache_set_wait_timeout,
     lib_path,
     load,
 )

@@ -24,7 +24,8 @@ EMPTY_POS = 2**31 - 1
 BUF_NAMES = ("keys", "values", "k_scales", "v_scales", "token_pos", "scores", "workspace")
 EXPORTED = ("kv_cache_query_sizes", "kv_cache_create", "kv_cache_reset", "kv_cache_destroy",
             "kv_cache_get_fill", "kv_cache_set_fill", "kv_cache_quantize", "h2o_evict_insert",
-            "attn_chunk_with_scoresum", "h2okv_last_error", "h2okv_abi_version")
+            "attn_chunk_with_scoresum", "kv_cache_device_status", "kv_cache_set_wait_timeout",
+            "h2okv_last_error", "h2okv_abi_version")
 
 
 class H2OKVError(RuntimeError):
@@ -75,6 +76,8 @@ def load() -> ctypes.CDLL:
         "kv_cache_quantize": (ctypes.c_int, [i32, vp, i64, i32, vp, vp, vp]),
         "h2o_evict_insert": (ctypes.c_int, [vp, vp, vp, vp, i32, i64, vp, vp]),
         "attn_chunk_with_scoresum": (ctypes.c_int, [vp, vp, i32, i64, vp, vp, vp, vp, vp]),
+        "kv_cache_device_status": (ctypes.c_int, [vp, ctypes.POINTER(i32), vp]),
+        "kv_cache_set_wait_timeout": (ctypes.c_int, [vp, ctypes.c_uint64]),
         "h2okv_last_error": (ctypes.c_char_p, []),
         "h2okv_abi_version": (i32, []),
     }
@@ -157,6 +160,17 @@ def attn_chunk_with_scoresum(handle, q, S: int, P: int, y_out, lse_out, w_out, w
     _check(load().attn_chunk_with_scoresum(handle, _ptr(q), int(S), int(P), _ptr(y_out),
                                            _ptr(lse_out), _ptr(w_out), _ptr(wq_out),
                                            _stream(stream)))
+
+
+def kv_cache_device_status(handle, stream=None) -> int:
+    """Read and clear the device status word (0 = ok, else an error code)."""
+    v = ctypes.c_int32()
+    _check(load().kv_cache_device_status(handle, ctypes.byref(v), _stream(stream)))
+    return v.value
+
+
+def kv_cache_set_wait_timeout(handle, timeout_ns: int):
+    _check(load().kv_cache_set_wait_timeout(handle, int(timeout_ns)))
 
 
 def h2okv_last_error() -> str:

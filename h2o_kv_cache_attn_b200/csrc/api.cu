@@ -30,9 +30,6 @@ int check_launch(const char *what) {
 
 static size_t align256(size_t x) { return (x + 255) & ~(size_t)255; }
 
-// Selection keys live in shared memory up to this many slots.
-constexpr int kSmemKeyCap = 53248;
-
 static int validate_desc(const h2okv_cache_desc *d) {
   if (!d) return set_error(H2OKV_ERR_INVALID_ARG, "desc is NULL");
   if (d->batch < 1 || d->n_kv_heads < 1 || d->n_q_heads < 1)
@@ -71,13 +68,9 @@ static int validate_desc(const h2okv_cache_desc *d) {
 }
 
 static void layout(const h2okv_cache_desc &d, const TcPlan &tc, WorkspaceLayout *ws) {
-  const size_t B = d.batch, Hk = d.n_kv_heads, Hq = d.n_q_heads, NC = d.capacity,
-               S = d.max_chunk, D = d.head_dim;
+  const size_t B = d.batch, Hq = d.n_q_heads, NC = d.capacity, S = d.max_chunk,
+               D = d.head_dim;
   size_t off = 0;
-  ws->slot_list = off;
-  off = align256(off + B * Hk * S * 4);
-  ws->sel_keys = off;
-  if (d.capacity > kSmemKeyCap) off = align256(off + B * Hk * NC * 4);
   ws->lse2 = off;
   off = align256(off + B * Hq * S * 4);
   ws->status = off;
@@ -252,6 +245,8 @@ int h2o_evict_insert(h2okv_cache *c, const float *w_prev, const void *k_new, con
                      (long long)P);
   if (S > 0 && (!k_new || !v_new))
     return set_error(H2OKV_ERR_INVALID_ARG, "k_new and v_new are required when S > 0");
+  if (misaligned(k_new, 16) || misaligned(v_new, 16) || misaligned(w_prev, 4))
+    return set_error(H2OKV_ERR_INVALID_ARG, "k_new and v_new must be 16-byte aligned");
   if (S == 0 && !w_prev) return H2OKV_OK;
   int rc = launch_evict_insert(c, w_prev, k_new, v_new, S, P, slots_out, (cudaStream_t)stream);
   if (rc) return rc;

@@ -50,14 +50,16 @@ constexpr uint32_t OFF_K0 = OFF_Q + kTileBytes;
 constexpr uint32_t OFF_V0 = OFF_K0 + kTileBytes;
 constexpr uint32_t OFF_K1 = OFF_V0 + kTileBytes;
 constexpr uint32_t OFF_V1 = OFF_K1 + kTileBytes;
-constexpr uint32_t OFF_P = OFF_V1 + kTileBytes;
-constexpr uint32_t OFF_TP = OFF_P + kTileBytes;        // int32 [2][BN]
+constexpr uint32_t OFF_P0 = OFF_V1 + kTileBytes;
+constexpr uint32_t OFF_P1 = OFF_P0 + kTileBytes;
+constexpr uint32_t OFF_TP = OFF_P1 + kTileBytes;       // int32 [2][BN]
 constexpr uint32_t OFF_TPMAX = OFF_TP + 2 * BN * 4;    // int32 [2] (+pad)
 constexpr uint32_t OFF_LSE = OFF_TPMAX + 16;           // float [BM]
 constexpr uint32_t OFF_BAR = OFF_LSE + BM * 4;         // uint64 barriers
-constexpr int NBAR = 13;
+constexpr int NBAR = 15;
 constexpr uint32_t OFF_TMEM = OFF_BAR + NBAR * 8;
 constexpr uint32_t kSmemBytes = OFF_TMEM + 16 + 1024;  // + alignment slack
+static_assert(kSmemBytes <= 232448, "shared memory budget");
 
 constexpr uint32_t kTmemCols = 512;  // S buffers at 0 and 128, O at 256
 constexpr uint32_t IDESC_K_MAJOR = idesc_bf16_f32(128, 128, false, false);
@@ -75,7 +77,7 @@ struct TcParams {
 };
 
 enum { B_Q = 0, B_FULL0, B_FULL1, B_EMPTY0, B_EMPTY1, B_SFULL0, B_SFULL1, B_SFREE0, B_SFREE1,
-       B_PFULL, B_PFREE, B_OFULL, B_DRAIN };
+       B_PFULL0, B_PFULL1, B_PFREE0, B_PFREE1, B_OFULL, B_DRAIN };
 
 // K-major SW128 operand (rows x 128 columns as two 64-column halves): k-step ks
 // (16 columns) starts 32 bytes further inside a half.
@@ -138,8 +140,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     mbar_init(&bar[B_SFULL1], 1);
     mbar_init(&bar[B_SFREE0], 4);
     mbar_init(&bar[B_SFREE1], 4);
-    mbar_init(&bar[B_PFULL], 4);
-    mbar_init(&bar[B_PFREE], 1);
+    mbar_init(&bar[B_PFULL0], 4);
+    mbar_init(&bar[B_PFULL1], 4);
+    mbar_init(&bar[B_PFREE0], 1);
+    mbar_init(&bar[B_PFREE1], 1);
     mbar_init(&bar[B_OFULL], 1);
     mbar_init(&bar[B_DRAIN], 1);
     fence_mbar_init();
@@ -212,7 +216,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   } else if (warp == 1) {
     // ------------------------------------------------------------------ MMA issuer
     if (lane == 0) {
-      const uint32_t q_addr = sbase + OFF_Q, p_addr = sbase + OFF_P;
+      const uint32_t q_addr = sbase + OFF_Q;
       if (!mbar_wait(&bar[B_Q], 0, lim)) fail(p, aborted);
       tc_fence_after();
       // phase A: S = Q K^T
@@ -249,15 +253,17 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (!aborted && !issue_st(0)) fail(p, aborted);
       for (int kt = 0; kt < n_kt && !aborted; ++kt) {
         if (kt + 1 < n_kt && !issue_st(kt + 1)) { fail(p, aborted); break; }
-        if (!mbar_wait(&bar[B_PFULL], kt & 1, lim)) { fail(p, aborted); break; }
+        const int pb = kt & 1;
+        if (!mbar_wait(&bar[B_PFULL0 + pb], (kt >> 1) & 1, lim)) { fail(p, aborted); break; }
         tc_fence_after();
         const int s = (n_kt + kt) & 1;
         const uint32_t v_addr = sbase + (s ? OFF_V1 : OFF_V0);
+        const uint32_t p_addr = sbase + (pb ? OFF_P1 : OFF_P0);
 #pragma unroll
         for (int ks = 0; ks < BN / 16; ++ks)
           mma_bf16_ss(tmem + 256, mnmajor_desc(p_addr, ks), mnmajor_desc(v_addr, ks), IDESC_PV,
                       (kt > 0 || ks > 0) ? 1u : 0u);
-        mma_commit(&bar[B_PFREE]);
+        mma_commit(&bar[B_PFREE0 + pb]);
         mma_commit(&bar[B_EMPTY0 + s]);
       }
       mma_commit(&bar[B_OFULL]);
@@ -274,20 +280,17 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int row_i = i0 + st;
     const int64_t row_lim = (int64_t)p.P + row_i;
     float m = -INFINITY, l = 0.f;
-    uint32_t r[32];
-    float x[BN];
+    uint32_t xr[BN];
     for (int kt = 0; kt < n_kt && !aborted; ++kt) {
       const int u = kt, buf = u & 1, s = kt & 1;
       if (!warp_wait(&bar[B_SFULL0 + buf], (u >> 1) & 1, lim)) { fail(p, aborted); break; }
       if (!warp_wait(&bar[B_FULL0 + s], (kt >> 1) & 1, lim)) { fail(p, aborted); break; }
       tc_fence_after();
-#pragma unroll
-      for (int c = 0; c < 4; ++c) {
-        tmem_ld32(tmem + lane_base + buf * 128 + c * 32, r);
-        tmem_wait_ld();
-#pragma unroll
-        for (int e = 0; e < 32; ++e) x[c * 32 + e] = __uint_as_float(r[e]);
-      }
+      tmem_ld32(tmem + lane_base + buf * 128 + 0, *reinterpret_cast<uint32_t(*)[32]>(xr + 0));
+      tmem_ld32(tmem + lane_base + buf * 128 + 32, *reinterpret_cast<uint32_t(*)[32]>(xr + 32));
+      tmem_ld32(tmem + lane_base + buf * 128 + 64, *reinterpret_cast<uint32_t(*)[32]>(xr + 64));
+      tmem_ld32(tmem + lane_base + buf * 128 + 96, *reinterpret_cast<uint32_t(*)[32]>(xr + 96));
+      tmem_wait_ld();
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&bar[B_SFREE0 + buf]);
@@ -295,18 +298,26 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (!all_visible) {
 #pragma unroll
         for (int e = 0; e < BN; ++e)
-          if ((int64_t)tp_s[s * BN + e] > row_lim) x[e] = -INFINITY;
+          if ((int64_t)tp_s[s * BN + e] > row_lim) xr[e] = __float_as_uint(-INFINITY);
       }
       __syncwarp();
       if (lane == 0) mbar_arrive(&bar[B_EMPTY0 + s]);
-      float mx = -INFINITY;
+      // row max with 8 independent chains
+      float mx8[8];
 #pragma unroll
-      for (int e = 0; e < BN; ++e) mx = fmaxf(mx, x[e]);
+      for (int q = 0; q < 8; ++q) mx8[q] = __uint_as_float(xr[q]);
+#pragma unroll
+      for (int e = 8; e < BN; ++e) mx8[e & 7] = fmaxf(mx8[e & 7], __uint_as_float(xr[e]));
+      const float mx = fmaxf(fmaxf(fmaxf(mx8[0], mx8[1]), fmaxf(mx8[2], mx8[3])),
+                             fmaxf(fmaxf(mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7])));
       const float m_new = fmaxf(m, mx * c2);
       if (m_new == -INFINITY) continue;
-      float sum = 0.f;
+      float sm8[8];
 #pragma unroll
-      for (int e = 0; e < BN; ++e) sum += ex2(fmaf(x[e], c2, -m_new));
+      for (int q = 0; q < 8; ++q) sm8[q] = 0.f;
+#pragma unroll
+      for (int e = 0; e < BN; ++e) sm8[e & 7] += ex2(fmaf(__uint_as_float(xr[e]), c2, -m_new));
+      const float sum = ((sm8[0] + sm8[1]) + (sm8[2] + sm8[3])) + ((sm8[4] + sm8[5]) + (sm8[6] + sm8[7]));
       l = l * ex2(m - m_new) + sum;
       m = m_new;
     }
@@ -318,55 +329,64 @@ __global__ void __launch_bounds__(kThreads, 1)
     // phase B
     const int rmax = min(BM, p.S - i0);
     float *pw = p.part_w + ((size_t)bhq * p.tiles + t) * p.N_C;
-    const uint32_t p_row = sbase + OFF_P + (st >> 3) * 1024 + (st & 7) * 128;
+    const uint32_t p_row = (st >> 3) * 1024 + (st & 7) * 128;
+    uint32_t r[32];
     for (int kt = 0; kt < n_kt && !aborted; ++kt) {
-      const int u = n_kt + kt, buf = u & 1, it = n_kt + kt, s = it & 1;
+      const int u = n_kt + kt, buf = u & 1, it = n_kt + kt, s = it & 1, pb = kt & 1;
       if (!warp_wait(&bar[B_SFULL0 + buf], (u >> 1) & 1, lim)) { fail(p, aborted); break; }
       if (!warp_wait(&bar[B_FULL0 + s], (it >> 1) & 1, lim)) { fail(p, aborted); break; }
+      // P buffer pb was last read by the P V product of tile kt - 2
+      if (kt >= 2 && !warp_wait(&bar[B_PFREE0 + pb], ((kt >> 1) - 1) & 1, lim)) {
+        fail(p, aborted);
+        break;
+      }
       tc_fence_after();
       const int64_t tpj = tp_s[s * BN + st];
       __syncwarp();
       if (lane == 0) mbar_arrive(&bar[B_EMPTY0 + s]);
-      // visible rows r of this tile: tpj <= P + i0 + r
+      // visible rows r of this tile: tpj <= P + i0 + r, r < rmax
       const int64_t rm = tpj - (int64_t)p.P - i0;
       const int rmin = rm <= 0 ? 0 : (rm >= BM ? BM : (int)rm);
-      float colsum = 0.f;
-      uint32_t pk[BM / 2];
+      const bool full = __all_sync(0xffffffffu, rmin == 0 && rmax == BM);
+      const uint32_t p_buf = sbase + (pb ? OFF_P1 : OFF_P0) + p_row;
+      float cs8[8];
+#pragma unroll
+      for (int q = 0; q < 8; ++q) cs8[q] = 0.f;
 #pragma unroll
       for (int c = 0; c < 4; ++c) {
         tmem_ld32(tmem + lane_base + buf * 128 + c * 32, r);
         tmem_wait_ld();
+        uint32_t pk[16];
 #pragma unroll
         for (int e = 0; e < 32; e += 2) {
           const int r0 = c * 32 + e;
           float p0 = ex2(fmaf(__uint_as_float(r[e]), c2, -lse_s[r0]));
           float p1 = ex2(fmaf(__uint_as_float(r[e + 1]), c2, -lse_s[r0 + 1]));
-          p0 = (r0 >= rmin && r0 < rmax) ? p0 : 0.f;
-          p1 = (r0 + 1 >= rmin && r0 + 1 < rmax) ? p1 : 0.f;
-          colsum += p0 + p1;
-          pk[r0 >> 1] = pack_bf16x2(p0, p1);
+          if (!full) {
+            p0 = (r0 >= rmin && r0 < rmax) ? p0 : 0.f;
+            p1 = (r0 + 1 >= rmin && r0 + 1 < rmax) ? p1 : 0.f;
+          }
+          cs8[(e >> 1) & 7] += p0 + p1;
+          pk[e >> 1] = pack_bf16x2(p0, p1);
         }
-      }
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&bar[B_SFREE0 + buf]);
-      if (kt > 0 && !warp_wait(&bar[B_PFREE], (kt - 1) & 1, lim)) { fail(p, aborted); break; }
-      // P[row][slot] as the MN-major A operand: slot = K index (row of 128 B within
-      // an 8-slot atom), rows = M index (64 per block, 16-byte chunks swizzled).
+        // rows 32c .. 32c+31 = M block c/2, 16-byte chunks (c%2)*4 .. +3 of this slot's K row
 #pragma unroll
-      for (int mb = 0; mb < 2; ++mb) {
-#pragma unroll
-        for (int cc = 0; cc < 8; ++cc) {
-          const int base = mb * 32 + cc * 4;  // index into pk (2 rows per entry)
-          const uint32_t addr = p_row + mb * kHalfBytes + ((cc ^ (st & 7)) << 4);
-          asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(pk[base]),
-                       "r"(pk[base + 1]), "r"(pk[base + 2]), "r"(pk[base + 3])
+        for (int q = 0; q < 4; ++q) {
+          const int cc = (c & 1) * 4 + q;
+          const uint32_t addr = p_buf + (c >> 1) * kHalfBytes + ((cc ^ (st & 7)) << 4);
+          asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(pk[4 * q]),
+                       "r"(pk[4 * q + 1]), "r"(pk[4 * q + 2]), "r"(pk[4 * q + 3])
                        : "memory");
         }
       }
+      tc_fence_before();
       fence_proxy_async_smem();
       __syncwarp();
-      if (lane == 0) mbar_arrive(&bar[B_PFULL]);
+      if (lane == 0) {
+        mbar_arrive(&bar[B_SFREE0 + buf]);
+        mbar_arrive(&bar[B_PFULL0 + pb]);
+      }
+      const float colsum = ((cs8[0] + cs8[1]) + (cs8[2] + cs8[3])) + ((cs8[4] + cs8[5]) + (cs8[6] + cs8[7]));
       const int j = kt * BN + st;
       if (j < p.N_C) pw[j] = colsum;
     }

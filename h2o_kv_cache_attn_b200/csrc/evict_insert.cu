@@ -4,25 +4,34 @@
 // §A.5.3 keys' = scatter(keys, index, key_new)), plus the 8/4-bit row
 // quantizer used on insert.
 //
-// Two kernels per call:
-//   select_kernel  one CTA per (b, h_k): scores += w_prev, then the S slots to
-//                  overwrite -- empty slots first, then the smallest (score,
-//                  slot) pairs -- by a 4-pass 8-bit radix select on
-//                  order-preserving uint32 keys held in shared memory, and a
-//                  block scan in slot order that lists the chosen slots
-//                  ascending (token k -> k-th smallest slot);
-//   scatter_kernel one warp per (b, h_k, k): copies (or quantizes) the new key
-//                  and value rows into their slots.
+// One launch per call: evict_kernel runs a thread-block cluster of CL CTAs per
+// (b, h_k).  Each CTA holds a contiguous slice of the N_C slots in registers
+// (IPT consecutive slots per thread) and
+//   1. folds w_prev into the float32 scores and forms order-preserving uint32
+//      selection keys (0 for an empty slot, so empty slots come first);
+//   2. finds the S-th smallest key with a 4-pass, 8-bit radix select: each CTA
+//      builds a 256-bin histogram of its slice, the cluster sums them through
+//      distributed shared memory, every CTA picks the same bin;
+//   3. lists the chosen slots in slot order (token k -> k-th smallest slot):
+//      a block scan plus a cluster prefix of per-CTA counts gives each chosen
+//      slot its position; the slot of position k is sent to CTA k % CL;
+//   4. copies (or quantizes) the new key/value rows k = rank, rank + CL, ...
+//      into their slots.
+// While the cache is still filling (n_filled + S <= N_C) the slots are
+// n_filled + k and steps 2-3 are skipped.  No scratch memory in global memory.
 // The quantizer must agree bit for bit with an IEEE float32 reference: it uses
 // correctly rounded division, rintf and __float2half_rn only (this file is
 // never built with fast-math).
+#include <cooperative_groups.h>
+
 #include "h2okv_internal.cuh"
 
 namespace h2okv {
 namespace {
 
-constexpr int kSelThreads = 1024;
-constexpr int kSmemKeyCap = 53248;  // keys held in shared memory up to this capacity
+constexpr int kEvThreads = 256;   // threads per CTA of the eviction kernel
+constexpr int kEvictCluster = 8;  // CTAs per (b, h_k): a portable cluster size
+constexpr int kEvWarps = kEvThreads / 32;
 
 // Unsigned key with the order of the float: -0 and +0 map to the same key;
 // every non-NaN score maps to a key >= 1 so that 0 can mark an empty slot.
@@ -32,7 +41,7 @@ __device__ __forceinline__ uint32_t order_key(float s) {
   return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
 }
 
-// Block-wide exclusive scan of one uint32 per thread (blockDim.x == kSelThreads).
+// Block-wide exclusive scan of one uint32 per thread (blockDim.x == kEvThreads).
 __device__ __forceinline__ uint32_t block_exclusive_scan(uint32_t v, uint32_t *warp_tot,
                                                          uint32_t *total) {
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
@@ -45,141 +54,19 @@ __device__ __forceinline__ uint32_t block_exclusive_scan(uint32_t v, uint32_t *w
   if (lane == 31) warp_tot[warp] = incl;
   __syncthreads();
   if (warp == 0) {
-    uint32_t wv = warp_tot[lane];
+    uint32_t wv = lane < kEvWarps ? warp_tot[lane] : 0u;
     uint32_t wincl = wv;
 #pragma unroll
     for (int o = 1; o < 32; o <<= 1) {
       uint32_t t = __shfl_up_sync(0xffffffffu, wincl, o);
       if (lane >= o) wincl += t;
     }
-    warp_tot[lane] = wincl - wv;
-    if (lane == 31) *total = wincl;
+    if (lane < kEvWarps) warp_tot[lane] = wincl - wv;
+    if (lane == kEvWarps - 1) *total = wincl;
   }
   __syncthreads();
-  uint32_t r = warp_tot[warp] + incl - v;
-  __syncthreads();  // warp_tot is reused by the next call
-  return r;
+  return warp_tot[warp] + incl - v;
 }
-
-// mode 0: accumulate only; 1: fill slots n_filled.. (no occupied slot is
-// touched); 2: generic selection (empty slots first, then lowest scores).
-__global__ void __launch_bounds__(kSelThreads)
-    select_kernel(float *__restrict__ scores, const float *__restrict__ w_prev,
-                  int32_t *__restrict__ token_pos, int N_C, int S, int P, int mode, int n_filled,
-                  int max_chunk, int32_t *__restrict__ slot_list, int32_t *__restrict__ slots_out,
-                  uint32_t *__restrict__ gkeys) {
-  extern __shared__ uint32_t smem_keys[];
-  __shared__ uint32_t hist[256];
-  __shared__ uint32_t warp_tot[32];
-  __shared__ uint32_t s_prefix, s_k, s_total;
-
-  const int bh = blockIdx.x;
-  const size_t base = (size_t)bh * N_C;
-  float *sc = scores + base;
-  const float *wp = w_prev ? w_prev + base : nullptr;
-  int32_t *tp = token_pos + base;
-  uint32_t *keys = gkeys ? gkeys + base : smem_keys;
-  int32_t *list = slot_list + (size_t)bh * max_chunk;
-  int32_t *sout = slots_out ? slots_out + (size_t)bh * S : nullptr;
-  const int tid = threadIdx.x, lane = tid & 31;
-
-  // 1. scores += w_prev (float32), selection keys.
-  for (int j = tid; j < N_C; j += blockDim.x) {
-    float s = sc[j];
-    if (wp) {
-      s = __fadd_rn(s, wp[j]);
-      sc[j] = s;
-    }
-    if (mode == 2) keys[j] = (tp[j] == kEmptyPos) ? 0u : order_key(s);
-  }
-  if (mode == 0) return;
-  __syncthreads();
-  if (mode == 1) {
-    for (int k = tid; k < S; k += blockDim.x) {
-      const int j = n_filled + k;
-      list[k] = j;
-      if (sout) sout[k] = j;
-      tp[j] = P + k;
-      sc[j] = 0.f;
-    }
-    return;
-  }
-
-  // 2. radix select of the S-th smallest key, 8 bits per pass from the top.
-  uint32_t prefix = 0u, pmask = 0u, k = (uint32_t)S;
-  const int n_round = (N_C + kSelThreads - 1) / kSelThreads;
-  for (int shift = 24; shift >= 0; shift -= 8) {
-    for (int i = tid; i < 256; i += blockDim.x) hist[i] = 0u;
-    __syncthreads();
-    for (int r = 0; r < n_round; ++r) {
-      const int j = r * kSelThreads + tid;
-      uint32_t bin = 0xffffffffu;
-      if (j < N_C) {
-        const uint32_t key = keys[j];
-        if ((key & pmask) == prefix) bin = (key >> shift) & 255u;
-      }
-      const uint32_t peers = __match_any_sync(0xffffffffu, bin);
-      if (bin != 0xffffffffu && lane == __ffs(peers) - 1) atomicAdd(&hist[bin], __popc(peers));
-    }
-    __syncthreads();
-    if (tid < 32) {
-      uint32_t loc[8], sum = 0;
-#pragma unroll
-      for (int t = 0; t < 8; ++t) {
-        loc[t] = hist[lane * 8 + t];
-        sum += loc[t];
-      }
-      uint32_t incl = sum;
-#pragma unroll
-      for (int o = 1; o < 32; o <<= 1) {
-        uint32_t v = __shfl_up_sync(0xffffffffu, incl, o);
-        if (lane >= o) incl += v;
-      }
-      const uint32_t excl = incl - sum;
-      if (excl < k && k <= incl) {
-        uint32_t c = excl;
-#pragma unroll
-        for (int t = 0; t < 8; ++t) {
-          if (c + loc[t] >= k) {
-            s_prefix = prefix | ((uint32_t)(lane * 8 + t) << shift);
-            s_k = k - c;
-            break;
-          }
-          c += loc[t];
-        }
-      }
-    }
-    __syncthreads();
-    prefix = s_prefix;
-    k = s_k;
-    pmask |= 255u << shift;
-  }
-  const uint32_t T = prefix, k_eq = k;  // take all keys < T and the first k_eq keys == T
-
-  // 3. slot-ordered listing: pos(j) = #(key < T before j) + min(#(key == T before j), k_eq).
-  uint32_t less_base = 0, eq_base = 0;
-  for (int r = 0; r < n_round; ++r) {
-    const int j = r * kSelThreads + tid;
-    uint32_t key = 0xffffffffu;
-    bool valid = j < N_C;
-    if (valid) key = keys[j];
-    const uint32_t is_less = valid && key < T, is_eq = valid && key == T;
-    const uint32_t ex = block_exclusive_scan((is_less << 16) | is_eq, warp_tot, &s_total);
-    const uint32_t tot = s_total;
-    const uint32_t less_before = less_base + (ex >> 16), eq_before = eq_base + (ex & 0xffffu);
-    if (is_less || (is_eq && eq_before < k_eq)) {
-      const uint32_t pos = less_before + min(eq_before, k_eq);
-      list[pos] = j;
-      if (sout) sout[pos] = j;
-      tp[j] = P + (int)pos;
-      sc[j] = 0.f;
-    }
-    less_base += tot >> 16;
-    eq_base += tot & 0xffffu;
-    __syncthreads();  // s_total is rewritten by the next round
-  }
-}
-
 // ---- row quantizer ------------------------------------------------------------
 // One warp per row of d bf16 values; lane handles element pairs lane, lane+32, ...
 template <int KV>
@@ -218,36 +105,209 @@ __device__ __forceinline__ void quantize_row_warp(const __nv_bfloat16 *__restric
 
 template <int KV>
 __device__ __forceinline__ void copy_row_warp(const void *__restrict__ src, void *__restrict__ dst,
-                                              int d) {
+                                              size_t row_bytes) {
   const int lane = threadIdx.x & 31;
-  const int words = KV == H2OKV_F32 ? d : d / 2;  // 32-bit words per row
-  const uint32_t *s = reinterpret_cast<const uint32_t *>(src);
-  uint32_t *o = reinterpret_cast<uint32_t *>(dst);
-  for (int i = lane; i < words; i += 32) o[i] = s[i];
+  const uint4 *s = reinterpret_cast<const uint4 *>(src);
+  uint4 *o = reinterpret_cast<uint4 *>(dst);
+  for (int i = lane; i < (int)(row_bytes / 16); i += 32) o[i] = s[i];
 }
 
 template <int KV>
-__global__ void __launch_bounds__(256)
-    scatter_kernel(const void *__restrict__ k_new, const void *__restrict__ v_new,
-                   uint8_t *__restrict__ keys, uint8_t *__restrict__ values,
-                   __half *__restrict__ k_scales, __half *__restrict__ v_scales,
-                   const int32_t *__restrict__ slot_list, int n_rows, int S, int max_chunk,
-                   int N_C, int d, size_t row_bytes, size_t in_row_bytes) {
-  const int row = blockIdx.x * 8 + (threadIdx.x >> 5);
-  if (row >= n_rows) return;
-  const int bh = row / S, k = row - bh * S;
-  const int slot = slot_list[(size_t)bh * max_chunk + k];
-  const size_t dst_row = (size_t)bh * N_C + slot;
-  const uint8_t *ksrc = reinterpret_cast<const uint8_t *>(k_new) + (size_t)row * in_row_bytes;
-  const uint8_t *vsrc = reinterpret_cast<const uint8_t *>(v_new) + (size_t)row * in_row_bytes;
+__device__ __forceinline__ void insert_row_warp(const uint8_t *ksrc, const uint8_t *vsrc,
+                                                uint8_t *keys, uint8_t *values, __half *ks,
+                                                __half *vs, size_t dst_row, int d,
+                                                size_t row_bytes) {
   if constexpr (KV == H2OKV_I8 || KV == H2OKV_I4) {
     quantize_row_warp<KV>(reinterpret_cast<const __nv_bfloat16 *>(ksrc), d,
-                          keys + dst_row * row_bytes, k_scales + dst_row);
+                          keys + dst_row * row_bytes, ks + dst_row);
     quantize_row_warp<KV>(reinterpret_cast<const __nv_bfloat16 *>(vsrc), d,
-                          values + dst_row * row_bytes, v_scales + dst_row);
+                          values + dst_row * row_bytes, vs + dst_row);
   } else {
-    copy_row_warp<KV>(ksrc, keys + dst_row * row_bytes, d);
-    copy_row_warp<KV>(vsrc, values + dst_row * row_bytes, d);
+    copy_row_warp<KV>(ksrc, keys + dst_row * row_bytes, row_bytes);
+    copy_row_warp<KV>(vsrc, values + dst_row * row_bytes, row_bytes);
+  }
+}
+
+struct EvictArgs {
+  float *scores;
+  const float *w_prev;
+  int32_t *token_pos;
+  const uint8_t *k_new, *v_new;
+  uint8_t *keys, *values;
+  __half *k_scales, *v_scales;
+  int32_t *slots_out;
+  int N_C, S, P, mode, n_filled, d, slice;
+  size_t row_bytes, in_row_bytes;
+};
+
+// mode 0: fold w_prev only (S = 0); 1: fill slots n_filled.. (no occupied slot is
+// touched); 2: generic choice (empty slots first, then lowest scores).
+template <int KV, int IPT>
+__global__ void __launch_bounds__(kEvThreads) evict_kernel(const EvictArgs a) {
+  namespace cg = cooperative_groups;
+  cg::cluster_group cluster = cg::this_cluster();
+  const int CL = (int)cluster.num_blocks();
+  const int rank = (int)cluster.block_rank();
+  const int bh = blockIdx.x / CL;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+
+  __shared__ uint32_t hist[2][256];
+  __shared__ uint32_t tot_bins[256];
+  __shared__ uint32_t warp_tot[kEvWarps];
+  __shared__ uint32_t s_prefix, s_k, s_total;
+  __shared__ uint32_t cta_less, cta_eq;
+  extern __shared__ int32_t rowslot[];  // [ceil(S / CL)]: slot of chunk row rank + CL * m
+
+  const size_t gbase = (size_t)bh * a.N_C;
+  const int j0 = rank * a.slice + tid * IPT;
+  float sc[IPT];
+  uint32_t key[IPT];
+  bool valid[IPT];
+#pragma unroll
+  for (int i = 0; i < IPT; ++i) {
+    const int j = j0 + i;
+    valid[i] = j < a.N_C;
+    sc[i] = 0.f;
+    key[i] = 0u;
+    if (valid[i]) {
+      float s = a.scores[gbase + j];
+      if (a.w_prev) s = __fadd_rn(s, a.w_prev[gbase + j]);
+      sc[i] = s;
+      if (a.mode == 2) key[i] = (a.token_pos[gbase + j] == kEmptyPos) ? 0u : order_key(s);
+    }
+  }
+
+  if (a.mode != 2) {
+    // fold (and, while filling, the trivial slot choice n_filled + k)
+#pragma unroll
+    for (int i = 0; i < IPT; ++i) {
+      const int j = j0 + i;
+      if (!valid[i]) continue;
+      const int k = j - a.n_filled;
+      if (a.mode == 1 && k >= 0 && k < a.S) {
+        a.scores[gbase + j] = 0.f;
+        a.token_pos[gbase + j] = a.P + k;
+        if (a.slots_out) a.slots_out[(size_t)bh * a.S + k] = j;
+      } else if (a.w_prev) {
+        a.scores[gbase + j] = sc[i];
+      }
+    }
+    if (a.mode == 1) {
+      for (int k = rank + CL * warp; k < a.S; k += CL * kEvWarps) {
+        const size_t row = (size_t)bh * a.S + k;
+        insert_row_warp<KV>(a.k_new + row * a.in_row_bytes, a.v_new + row * a.in_row_bytes,
+                            a.keys, a.values, a.k_scales, a.v_scales, gbase + a.n_filled + k,
+                            a.d, a.row_bytes);
+      }
+    }
+    return;
+  }
+
+  // ---- radix select of the S-th smallest key over the whole cluster --------------
+  uint32_t prefix = 0u, pmask = 0u, kk = (uint32_t)a.S;
+  for (int pass = 0; pass < 4; ++pass) {
+    const int shift = 24 - 8 * pass;
+    uint32_t *h = hist[pass & 1];
+    h[tid] = 0u;
+    __syncthreads();
+#pragma unroll
+    for (int i = 0; i < IPT; ++i) {
+      const uint32_t bin =
+          (valid[i] && (key[i] & pmask) == prefix) ? (key[i] >> shift) & 255u : 0xffffffffu;
+      const uint32_t peers = __match_any_sync(0xffffffffu, bin);
+      if (bin != 0xffffffffu && lane == __ffs(peers) - 1) atomicAdd(&h[bin], __popc(peers));
+    }
+    cluster.sync();  // every CTA's histogram of this pass is complete
+    uint32_t sum = 0u;
+    for (int q = 0; q < CL; ++q) sum += cluster.map_shared_rank(h, q)[tid];
+    tot_bins[tid] = sum;
+    __syncthreads();
+    if (warp == 0) {
+      uint32_t loc[8], lsum = 0;
+#pragma unroll
+      for (int t = 0; t < 8; ++t) {
+        loc[t] = tot_bins[lane * 8 + t];
+        lsum += loc[t];
+      }
+      uint32_t incl = lsum;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const uint32_t v = __shfl_up_sync(0xffffffffu, incl, o);
+        if (lane >= o) incl += v;
+      }
+      const uint32_t excl = incl - lsum;
+      if (excl < kk && kk <= incl) {
+        uint32_t c = excl;
+#pragma unroll
+        for (int t = 0; t < 8; ++t) {
+          if (c + loc[t] >= kk) {
+            s_prefix = prefix | ((uint32_t)(lane * 8 + t) << shift);
+            s_k = kk - c;
+            break;
+          }
+          c += loc[t];
+        }
+      }
+    }
+    __syncthreads();
+    prefix = s_prefix;
+    kk = s_k;
+    pmask |= 255u << shift;
+  }
+  const uint32_t T = prefix, k_eq = kk;  // take every key < T and the first k_eq keys == T
+
+  // ---- chosen slots in slot order ---------------------------------------------------
+  uint32_t nl = 0, ne = 0;
+#pragma unroll
+  for (int i = 0; i < IPT; ++i) {
+    nl += (valid[i] && key[i] < T) ? 1u : 0u;
+    ne += (valid[i] && key[i] == T) ? 1u : 0u;
+  }
+  // per-thread counts <= IPT and per-CTA totals <= kEvThreads * IPT < 65536: pack 16 + 16 bits
+  const uint32_t ex = block_exclusive_scan((nl << 16) | ne, warp_tot, &s_total);
+  if (tid == 0) {
+    cta_less = s_total >> 16;
+    cta_eq = s_total & 0xffffu;
+  }
+  cluster.sync();  // per-CTA totals visible to the cluster
+  uint32_t base_less = 0, base_eq = 0;
+  for (int q = 0; q < rank; ++q) {
+    base_less += *cluster.map_shared_rank(&cta_less, q);
+    base_eq += *cluster.map_shared_rank(&cta_eq, q);
+  }
+  uint32_t less_before = base_less + (ex >> 16), eq_before = base_eq + (ex & 0xffffu);
+#pragma unroll
+  for (int i = 0; i < IPT; ++i) {
+    if (!valid[i]) continue;
+    const int j = j0 + i;
+    bool take = false;
+    uint32_t pos = 0;
+    if (key[i] < T) {
+      take = true;
+      pos = less_before + min(eq_before, k_eq);
+      ++less_before;
+    } else if (key[i] == T) {
+      take = eq_before < k_eq;
+      pos = less_before + eq_before;
+      ++eq_before;
+    }
+    if (take) {
+      sc[i] = 0.f;
+      a.token_pos[gbase + j] = a.P + (int)pos;
+      if (a.slots_out) a.slots_out[(size_t)bh * a.S + pos] = j;
+      int32_t *dst = cluster.map_shared_rank(rowslot, (int)(pos % (uint32_t)CL));
+      dst[pos / (uint32_t)CL] = j;
+    }
+    a.scores[gbase + j] = sc[i];
+  }
+  cluster.sync();  // rowslot lists complete
+
+  // ---- insert the chunk's rows k = rank, rank + CL, ... -----------------------------
+  for (int m = warp; rank + CL * m < a.S; m += kEvWarps) {
+    const int k = rank + CL * m;
+    const size_t row = (size_t)bh * a.S + k;
+    insert_row_warp<KV>(a.k_new + row * a.in_row_bytes, a.v_new + row * a.in_row_bytes, a.keys,
+                        a.values, a.k_scales, a.v_scales, gbase + rowslot[m], a.d, a.row_bytes);
   }
 }
 
@@ -281,59 +341,82 @@ int launch_init_cache(h2okv_cache *c, cudaStream_t st) {
   return check_launch("init_kernel");
 }
 
+template <int KV, int IPT>
+static int launch_evict_t(const EvictArgs &a, int n_groups, int CL, cudaStream_t st) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)(n_groups * CL));
+  cfg.blockDim = dim3(kEvThreads);
+  cfg.dynamicSmemBytes = (size_t)((a.S + CL - 1) / CL) * 4;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = CL;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  if (cfg.dynamicSmemBytes > 48 * 1024) {
+    cudaError_t e = cudaFuncSetAttribute(evict_kernel<KV, IPT>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         (int)cfg.dynamicSmemBytes);
+    if (e != cudaSuccess)
+      return set_error(H2OKV_ERR_CUDA, "cudaFuncSetAttribute(evict_kernel): %s",
+                       cudaGetErrorString(e));
+  }
+  cudaError_t e = cudaLaunchKernelEx(&cfg, evict_kernel<KV, IPT>, a);
+  if (e != cudaSuccess)
+    return set_error(H2OKV_ERR_CUDA, "evict_kernel launch: %s", cudaGetErrorString(e));
+  return check_launch("evict_kernel");
+}
+
+template <int KV>
+static int launch_evict_kv(const EvictArgs &a, int n_groups, int CL, int ipt, cudaStream_t st) {
+  switch (ipt) {
+    case 1: return launch_evict_t<KV, 1>(a, n_groups, CL, st);
+    case 2: return launch_evict_t<KV, 2>(a, n_groups, CL, st);
+    case 4: return launch_evict_t<KV, 4>(a, n_groups, CL, st);
+    case 8: return launch_evict_t<KV, 8>(a, n_groups, CL, st);
+    case 16: return launch_evict_t<KV, 16>(a, n_groups, CL, st);
+    case 32: return launch_evict_t<KV, 32>(a, n_groups, CL, st);
+  }
+  return set_error(H2OKV_ERR_UNSUPPORTED, "capacity too large for the eviction kernel");
+}
+
 int launch_evict_insert(h2okv_cache *c, const float *w_prev, const void *k_new, const void *v_new,
                         int S, int64_t P, int32_t *slots_out, cudaStream_t st) {
   const h2okv_cache_desc &d = c->desc;
-  const int BH = d.batch * d.n_kv_heads;
-  const int mode = S == 0 ? 0 : (c->n_filled + S <= d.capacity ? 1 : 2);
-  uint8_t *ws = reinterpret_cast<uint8_t *>(c->bufs.workspace);
-  int32_t *slot_list = reinterpret_cast<int32_t *>(ws + c->ws.slot_list);
-  uint32_t *gkeys = nullptr;
-  size_t smem = 0;
-  if (mode == 2) {
-    if (d.capacity > kSmemKeyCap)
-      gkeys = reinterpret_cast<uint32_t *>(ws + c->ws.sel_keys);
-    else
-      smem = (size_t)d.capacity * 4;
-  }
-  if (smem > 48 * 1024) {
-    static thread_local int configured_dev = -1;
-    int dev = 0;
-    cudaGetDevice(&dev);
-    if (configured_dev != dev) {
-      cudaError_t e = cudaFuncSetAttribute(select_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                           kSmemKeyCap * 4);
-      if (e != cudaSuccess)
-        return set_error(H2OKV_ERR_CUDA, "cudaFuncSetAttribute(select_kernel): %s",
-                         cudaGetErrorString(e));
-      configured_dev = dev;
-    }
-  }
-  select_kernel<<<BH, kSelThreads, smem, st>>>(c->bufs.scores, w_prev, c->bufs.token_pos,
-                                                d.capacity, S, (int)P, mode, c->n_filled,
-                                                d.max_chunk, slot_list, slots_out, gkeys);
-  int rc = check_launch("select_kernel");
-  if (rc || S == 0) return rc;
-
-  const int n_rows = BH * S;
-  const int blocks = (n_rows + 7) / 8;
-  const size_t in_row = (size_t)d.head_dim * (d.q_dtype == H2OKV_F32 ? 4 : 2);
-  uint8_t *keys = reinterpret_cast<uint8_t *>(c->bufs.keys);
-  uint8_t *vals = reinterpret_cast<uint8_t *>(c->bufs.values);
-  __half *ks = reinterpret_cast<__half *>(c->bufs.k_scales);
-  __half *vs = reinterpret_cast<__half *>(c->bufs.v_scales);
-#define H2OKV_SCATTER(KV)                                                                   \
-  scatter_kernel<KV><<<blocks, 256, 0, st>>>(k_new, v_new, keys, vals, ks, vs, slot_list,  \
-                                             n_rows, S, d.max_chunk, d.capacity, d.head_dim, \
-                                             c->row_bytes, in_row)
+  EvictArgs a;
+  a.scores = c->bufs.scores;
+  a.w_prev = w_prev;
+  a.token_pos = c->bufs.token_pos;
+  a.k_new = reinterpret_cast<const uint8_t *>(k_new);
+  a.v_new = reinterpret_cast<const uint8_t *>(v_new);
+  a.keys = reinterpret_cast<uint8_t *>(c->bufs.keys);
+  a.values = reinterpret_cast<uint8_t *>(c->bufs.values);
+  a.k_scales = reinterpret_cast<__half *>(c->bufs.k_scales);
+  a.v_scales = reinterpret_cast<__half *>(c->bufs.v_scales);
+  a.slots_out = slots_out;
+  a.N_C = d.capacity;
+  a.S = S;
+  a.P = (int)P;
+  a.mode = S == 0 ? 0 : (c->n_filled + S <= d.capacity ? 1 : 2);
+  a.n_filled = c->n_filled;
+  a.d = d.head_dim;
+  a.row_bytes = c->row_bytes;
+  a.in_row_bytes = (size_t)d.head_dim * (d.q_dtype == H2OKV_F32 ? 4 : 2);
+  // cluster size and slots per thread: CL * kEvThreads * IPT >= N_C
+  const int CL = kEvictCluster;
+  int ipt = 1;
+  while ((int64_t)CL * kEvThreads * ipt < d.capacity) ipt *= 2;
+  a.slice = kEvThreads * ipt;
+  const int n_groups = d.batch * d.n_kv_heads;
   switch (d.kv_dtype) {
-    case H2OKV_F32: H2OKV_SCATTER(H2OKV_F32); break;
-    case H2OKV_BF16: H2OKV_SCATTER(H2OKV_BF16); break;
-    case H2OKV_I8: H2OKV_SCATTER(H2OKV_I8); break;
-    case H2OKV_I4: H2OKV_SCATTER(H2OKV_I4); break;
+    case H2OKV_F32: return launch_evict_kv<H2OKV_F32>(a, n_groups, CL, ipt, st);
+    case H2OKV_BF16: return launch_evict_kv<H2OKV_BF16>(a, n_groups, CL, ipt, st);
+    case H2OKV_I8: return launch_evict_kv<H2OKV_I8>(a, n_groups, CL, ipt, st);
+    case H2OKV_I4: return launch_evict_kv<H2OKV_I4>(a, n_groups, CL, ipt, st);
   }
-#undef H2OKV_SCATTER
-  return check_launch("scatter_kernel");
+  return set_error(H2OKV_ERR_UNSUPPORTED, "kv dtype");
 }
 
 int launch_quantize(int kv_dtype, const __nv_bfloat16 *x, int64_t n_rows, int d, void *codes,

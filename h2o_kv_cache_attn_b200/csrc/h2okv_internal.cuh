@@ -16,8 +16,6 @@ constexpr int kMaxCapacity = 65536;
 
 // Workspace carve-up of one cache (all offsets 256-byte aligned).
 struct WorkspaceLayout {
-  size_t slot_list;    // int32 [B*Hk*max_chunk]: chosen slots, ascending per (b, h_k)
-  size_t sel_keys;     // uint32 [B*Hk*N_C]: selection keys when they do not fit in shared memory
   size_t lse2;         // float [B*Hq*max_chunk]: base-2 log-sum-exp per query row
   size_t part_ml;      // float2 [splits*B*Hq*rows_pad]: split-KV partial (max, sum) for pass 1
   size_t part_w;       // float [B*Hq*row_tiles*N_C]: per-row-tile summed weights (tensor-core path)

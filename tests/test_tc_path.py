@@ -33,3 +33,35 @@ CASES = [
 def test_tc_workload_every_chunk(wl, cuda_device):
     run, n = run_and_check(wl, cuda_device)
     assert n == wl.n_chunks
+
+
+def test_forced_wait_timeout_reports_status_and_recovers(cuda_device):
+    """Every device-side wait of the tensor-core kernel is bounded.  With the
+    limit set to 0 the first wait that is not already complete gives up: the
+    kernel drains its own copies and matrix operations, frees its tensor memory
+    and records H2OKV_ERR_TIMEOUT.  The context stays usable and the next call
+    with the default limit is correct again."""
+    import torch
+
+    from h2o_kv_cache_attn_b200 import binding as hb
+    from h2o_kv_cache_attn_b200.runner import LayerRunner
+    from h2o_kv_cache_attn_b200.synth import ChunkSource
+
+    from .harness import check_attend, snapshot, to_np
+
+    wl = tc("timeout", capacity=512, chunk=256, seq_len=512)
+    run = LayerRunner(wl, cuda_device, with_wq=True)
+    q, k, v = (t.to(cuda_device) for t in ChunkSource(wl).chunk(0))
+    run.cache.evict_insert(None, k, v, 256, 0)
+    torch.cuda.synchronize()
+    h = run.cache.handle
+    assert hb.kv_cache_device_status(h) == 0
+    hb.kv_cache_set_wait_timeout(h, 0)
+    hb.attn_chunk_with_scoresum(h, q, 256, 0, run.y, run.lse, run.w[0], run.wq)
+    assert hb.kv_cache_device_status(h) == hb.ERR_TIMEOUT
+    hb.kv_cache_set_wait_timeout(h, 2_000_000_000)
+    hb.attn_chunk_with_scoresum(h, q, 256, 0, run.y, run.lse, run.w[0], run.wq)
+    assert hb.kv_cache_device_status(h) == 0
+    after = snapshot(run.cache)
+    check_attend(wl, after, to_np(q), 256, 0, to_np(run.y), to_np(run.lse), to_np(run.w[0]),
+                 to_np(run.wq), [(0, 0), (0, 1)])
