@@ -3,29 +3,32 @@
 // SDPA plus the attention weights summed over the query axis, returned per KV
 // slot and summed over the q_g query heads of each GQA group).
 //
-// One CTA owns 128 query rows of one head (rows past S are zero-filled by TMA
-// and never written).  It streams the head's KV group twice:
+// One CTA owns two 128-row query tiles (a, b) of one KV group (two row tiles of
+// one head, or the same rows of two heads); rows past S are zero-filled by TMA
+// and never written.  It streams the group's K/V twice, each 128-slot tile once
+// for both query tiles (half the bytes per FLOP of one tile per CTA):
 //
-//   phase A  S = Q K^T per 128-slot tile (tcgen05.mma, M=128 rows, N=128 slots,
-//            K=128, accumulator in TMEM); one softmax thread per row reads its
-//            row with tcgen05.ld and keeps the online max / sum -> base-2 LSE.
-//   phase B  S^T = K Q^T per tile (M=128 slots, N=128 rows): one thread per
+//   phase A  S = Q K^T (tcgen05.mma, M=128 rows, N=128 slots, K=128, fp32 in
+//            TMEM) for a and b; one softmax thread per row keeps the online
+//            max / sum of its rows of a and b -> base-2 log-sum-exp.
+//   phase B  S^T = K Q^T (M=128 slots, N=128 rows) for a and b: one thread per
 //            SLOT reads its 128 logits, forms p = exp2(s*log2e/sqrt(d) - lse2_i)
 //            with the FINAL row LSE, sums them in registers (the slot's summed
-//            weight over this CTA's rows: no atomics, deterministic) and writes
-//            p as bf16 into shared memory (MN-major operand layout); then
-//            O += P V (tcgen05.mma, A = P MN-major, B = V MN-major) in TMEM.
-//            P is already normalised, so O needs no rescaling.
+//            weight over the tile's rows: no atomics, deterministic) and writes
+//            p as bf16 into shared memory (the MN-major A operand), then
+//            O += P V (A = P, B = V, both MN-major).  P is normalised already,
+//            so O needs no rescaling.  TMEM: S^T_a, S^T_b, O_a, O_b.
 //
-// Warp roles (256 threads): warp 0 TMA producer (K/V tiles via
-// cp.async.bulk.tensor, no multicast; token positions via plain loads), warp 1
-// TMEM allocator and single-thread MMA issuer, warps 4-7 softmax / column sums /
-// epilogue (warp 4+q owns TMEM lanes 32q..32q+31).  Two K/V stages and two TMEM
-// S buffers let the MMA of tile kt+1 overlap the softmax of tile kt.  Every
-// wait is bounded; a timeout sets the cache's device status word and the CTA
-// drains its copies and MMAs before freeing TMEM.
+// Warp roles (256 threads): warp 0 TMA producer (K and V tiles through separate
+// two-stage rings via cp.async.bulk.tensor, no multicast; token positions by
+// plain loads), warp 1 TMEM allocator and single-thread MMA issuer, warps 4-7
+// softmax / column sums / epilogue (warp 4+q owns TMEM lanes 32q..32q+31).
+// The MMA issue order PV_a(kt), S^T_a(kt+1), PV_b(kt), S^T_b(kt+1) keeps the
+// tensor pipe busy while the softmax warps work on the other query tile.
+// Every wait is bounded; a timeout sets the cache's device status word and the
+// CTA drains its copies and MMAs before freeing TMEM.
 //
-// Per-(row tile, slot) sums go to a partial buffer; a small reduction kernel
+// Per-(query tile, slot) sums go to a partial buffer; a small reduction kernel
 // sums them in a fixed order into w [B, H_k, N_C] and wq [B, H_q, N_C].
 #include <stdio.h>
 
@@ -37,31 +40,30 @@ namespace {
 
 using namespace ptx;
 
-constexpr int BM = 128;        // query rows per CTA
+constexpr int BM = 128;        // query rows per tile
 constexpr int BN = 128;        // slots per tile
 constexpr int D = 128;         // head dim
 constexpr int kThreads = 256;
 constexpr uint32_t kTileBytes = BM * D * 2;  // 32 KiB (two 64-column swizzled halves)
 constexpr uint32_t kHalfBytes = kTileBytes / 2;
 
-// shared memory carve-up (offsets from a 1024-aligned base)
-constexpr uint32_t OFF_Q = 0;
-constexpr uint32_t OFF_K0 = OFF_Q + kTileBytes;
-constexpr uint32_t OFF_V0 = OFF_K0 + kTileBytes;
-constexpr uint32_t OFF_K1 = OFF_V0 + kTileBytes;
-constexpr uint32_t OFF_V1 = OFF_K1 + kTileBytes;
-constexpr uint32_t OFF_P0 = OFF_V1 + kTileBytes;
-constexpr uint32_t OFF_P1 = OFF_P0 + kTileBytes;
-constexpr uint32_t OFF_TP = OFF_P1 + kTileBytes;       // int32 [2][BN]
-constexpr uint32_t OFF_TPMAX = OFF_TP + 2 * BN * 4;    // int32 [2] (+pad)
-constexpr uint32_t OFF_LSE = OFF_TPMAX + 16;           // float [BM]
-constexpr uint32_t OFF_BAR = OFF_LSE + BM * 4;         // uint64 barriers
-constexpr int NBAR = 15;
+// shared memory carve-up (1024-aligned base)
+constexpr uint32_t OFF_QA = 0;
+constexpr uint32_t OFF_QB = OFF_QA + kTileBytes;
+constexpr uint32_t OFF_K0 = OFF_QB + kTileBytes;
+constexpr uint32_t OFF_K1 = OFF_K0 + kTileBytes;
+constexpr uint32_t OFF_V0 = OFF_K1 + kTileBytes;
+constexpr uint32_t OFF_V1 = OFF_V0 + kTileBytes;
+constexpr uint32_t OFF_P = OFF_V1 + kTileBytes;
+constexpr uint32_t OFF_TP = OFF_P + kTileBytes;        // int32 [2 stages][BN]
+constexpr uint32_t OFF_LSE = OFF_TP + 2 * BN * 4;      // float [2 tiles][BM]
+constexpr uint32_t OFF_BAR = OFF_LSE + 2 * BM * 4;     // uint64 barriers
+constexpr int NBAR = 22;
 constexpr uint32_t OFF_TMEM = OFF_BAR + NBAR * 8;
-constexpr uint32_t kSmemBytes = OFF_TMEM + 16 + 1024;  // + alignment slack
+constexpr uint32_t kSmemBytes = OFF_TMEM + 16;
 static_assert(kSmemBytes <= 232448, "shared memory budget");
 
-constexpr uint32_t kTmemCols = 512;  // S buffers at 0 and 128, O at 256
+constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t IDESC_K_MAJOR = idesc_bf16_f32(128, 128, false, false);
 constexpr uint32_t IDESC_PV = idesc_bf16_f32(128, 128, true, true);
 
@@ -71,13 +73,21 @@ struct TcParams {
   float *lse_out;            // [B*Hq][S] or null
   float *part_w;             // [B*Hq*tiles][N_C]
   int *status;               // device status word (0 = ok)
-  int Hq, Hk, q_g, N_C, S, P, tiles, n_kt;
+  int Hq, Hk, q_g, N_C, S, P, tiles, n_kt, ctas_per_group;
   float scale2;  // log2(e) / sqrt(d)
   unsigned long long timeout_ns;
 };
 
-enum { B_Q = 0, B_FULL0, B_FULL1, B_EMPTY0, B_EMPTY1, B_SFULL0, B_SFULL1, B_SFREE0, B_SFREE1,
-       B_PFULL0, B_PFULL1, B_PFREE0, B_PFREE1, B_OFULL, B_DRAIN };
+enum {
+  B_Q = 0,
+  B_KFULL0, B_KFULL1, B_KEMPTY0, B_KEMPTY1,  // K ring (+ token positions)
+  B_VFULL0, B_VFULL1, B_VEMPTY0, B_VEMPTY1,  // V ring (phase B)
+  B_SFULL0, B_SFULL1, B_SFREE0, B_SFREE1,    // phase A S pair per tile parity
+  B_AFREE,                                   // phase A TMEM fully read
+  B_TFULLA, B_TFULLB, B_TFREEA, B_TFREEB,    // phase B S^T per query tile
+  B_PFULL, B_PFREE,                          // P buffer (uses alternate a, b)
+  B_OFULL, B_DRAIN                           // O complete; MMA drain before TMEM is freed
+};
 
 // K-major SW128 operand (rows x 128 columns as two 64-column halves): k-step ks
 // (16 columns) starts 32 bytes further inside a half.
@@ -107,43 +117,132 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   return *reinterpret_cast<uint32_t *>(&v);
 }
 
+__device__ __forceinline__ void tmem_ld128(uint32_t taddr, uint32_t (&x)[BN]) {
+  tmem_ld32(taddr + 0, *reinterpret_cast<uint32_t(*)[32]>(x + 0));
+  tmem_ld32(taddr + 32, *reinterpret_cast<uint32_t(*)[32]>(x + 32));
+  tmem_ld32(taddr + 64, *reinterpret_cast<uint32_t(*)[32]>(x + 64));
+  tmem_ld32(taddr + 96, *reinterpret_cast<uint32_t(*)[32]>(x + 96));
+  tmem_wait_ld();
+}
+
+// Online (max, sum) update of one row over one 128-slot tile (base-2 units).
+__device__ __forceinline__ void row_update(uint32_t (&x)[BN], bool masked, const int32_t *tp,
+                                           int64_t row_lim, float c2, float &m, float &l) {
+  if (masked) {
+#pragma unroll
+    for (int e = 0; e < BN; ++e)
+      if ((int64_t)tp[e] > row_lim) x[e] = __float_as_uint(-INFINITY);
+  }
+  float mx8[8];
+#pragma unroll
+  for (int q = 0; q < 8; ++q) mx8[q] = __uint_as_float(x[q]);
+#pragma unroll
+  for (int e = 8; e < BN; ++e) mx8[e & 7] = fmaxf(mx8[e & 7], __uint_as_float(x[e]));
+  const float mx = fmaxf(fmaxf(fmaxf(mx8[0], mx8[1]), fmaxf(mx8[2], mx8[3])),
+                         fmaxf(fmaxf(mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7])));
+  const float m_new = fmaxf(m, mx * c2);
+  if (m_new == -INFINITY) return;
+  float sm8[8];
+#pragma unroll
+  for (int q = 0; q < 8; ++q) sm8[q] = 0.f;
+#pragma unroll
+  for (int e = 0; e < BN; ++e) sm8[e & 7] += ex2(fmaf(__uint_as_float(x[e]), c2, -m_new));
+  const float sum = ((sm8[0] + sm8[1]) + (sm8[2] + sm8[3])) + ((sm8[4] + sm8[5]) + (sm8[6] + sm8[7]));
+  l = l * ex2(m - m_new) + sum;
+  m = m_new;
+}
+
+// Phase B for one slot (this thread) and one query tile: normalised p over the
+// tile's 128 rows from S^T in TMEM, packed to bf16 pairs, column sum returned.
+__device__ __forceinline__ float slot_probs(uint32_t taddr, const float *lse, float c2, int rmin,
+                                            int rmax, bool full, uint32_t (&pk)[BM / 2]) {
+  uint32_t r[32];
+  float cs8[8];
+#pragma unroll
+  for (int q = 0; q < 8; ++q) cs8[q] = 0.f;
+#pragma unroll
+  for (int c = 0; c < 4; ++c) {
+    tmem_ld32(taddr + c * 32, r);
+    tmem_wait_ld();
+#pragma unroll
+    for (int e = 0; e < 32; e += 2) {
+      const int r0 = c * 32 + e;
+      float p0 = ex2(fmaf(__uint_as_float(r[e]), c2, -lse[r0]));
+      float p1 = ex2(fmaf(__uint_as_float(r[e + 1]), c2, -lse[r0 + 1]));
+      if (!full) {
+        p0 = (r0 >= rmin && r0 < rmax) ? p0 : 0.f;
+        p1 = (r0 + 1 >= rmin && r0 + 1 < rmax) ? p1 : 0.f;
+      }
+      cs8[(e >> 1) & 7] += p0 + p1;
+      pk[r0 >> 1] = pack_bf16x2(p0, p1);
+    }
+  }
+  return ((cs8[0] + cs8[1]) + (cs8[2] + cs8[3])) + ((cs8[4] + cs8[5]) + (cs8[6] + cs8[7]));
+}
+
+// P[row][slot] as the MN-major A operand: slot = K index (a 128-byte row of an
+// 8-slot atom), rows = M index (64 per block, 16-byte chunks swizzled).
+__device__ __forceinline__ void store_p(uint32_t p_slot_row, int st, const uint32_t (&pk)[BM / 2]) {
+#pragma unroll
+  for (int mb = 0; mb < 2; ++mb) {
+#pragma unroll
+    for (int cc = 0; cc < 8; ++cc) {
+      const int base = mb * 32 + cc * 4;
+      const uint32_t addr = p_slot_row + mb * kHalfBytes + ((cc ^ (st & 7)) << 4);
+      asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(pk[base]),
+                   "r"(pk[base + 1]), "r"(pk[base + 2]), "r"(pk[base + 3])
+                   : "memory");
+    }
+  }
+}
+
 __global__ void __launch_bounds__(kThreads, 1)
     attn_tc_kernel(const __grid_constant__ CUtensorMap q_map,
                    const __grid_constant__ CUtensorMap k_map,
                    const __grid_constant__ CUtensorMap v_map, const TcParams p) {
-  extern __shared__ uint8_t smem_raw[];
-  uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
-                                              ~uintptr_t(1023));
+  extern __shared__ __align__(1024) uint8_t smem[];
   const uint32_t sbase = smem_u32(smem);
+  if (sbase & 1023u) {  // the swizzled operand tiles need a 1024-byte aligned base
+    if (threadIdx.x == 0) atomicExch(p.status, H2OKV_ERR_CUDA);
+    return;
+  }
   int32_t *tp_s = reinterpret_cast<int32_t *>(smem + OFF_TP);
-  int32_t *tpmax_s = reinterpret_cast<int32_t *>(smem + OFF_TPMAX);
   float *lse_s = reinterpret_cast<float *>(smem + OFF_LSE);
   uint64_t *bar = reinterpret_cast<uint64_t *>(smem + OFF_BAR);
   uint32_t *tmem_s = reinterpret_cast<uint32_t *>(smem + OFF_TMEM);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int w = blockIdx.x;
-  const int bhq = w / p.tiles, t = w - bhq * p.tiles;
-  const int b = bhq / p.Hq, h = bhq - b * p.Hq;
-  const int bg = b * p.Hk + h / p.q_g;
-  const int i0 = t * BM;
+  // work: query tiles 2c and 2c+1 of group bg, in (head, row tile) order
+  const int bg = blockIdx.x / p.ctas_per_group;
+  const int c = blockIdx.x - bg * p.ctas_per_group;
+  const int b = bg / p.Hk, g = bg - b * p.Hk;
+  const int n_qt = p.q_g * p.tiles;
+  const int qa = 2 * c, qb = 2 * c + 1;
+  const bool has_b = qb < n_qt;
+  const int hl_a = qa / p.tiles, t_a = qa - hl_a * p.tiles;
+  const int hl_b = has_b ? qb / p.tiles : hl_a, t_b = has_b ? qb - hl_b * p.tiles : t_a;
+  const int bhq_a = b * p.Hq + g * p.q_g + hl_a, bhq_b = b * p.Hq + g * p.q_g + hl_b;
+  const int i0_a = t_a * BM, i0_b = t_b * BM;
   const int n_kt = p.n_kt;
   const uint64_t lim = p.timeout_ns;
 
   if (threadIdx.x == 0) {
     mbar_init(&bar[B_Q], 1);
-    mbar_init(&bar[B_FULL0], 1);
-    mbar_init(&bar[B_FULL1], 1);
-    mbar_init(&bar[B_EMPTY0], 5);  // MMA commit + 4 softmax warps
-    mbar_init(&bar[B_EMPTY1], 5);
-    mbar_init(&bar[B_SFULL0], 1);
-    mbar_init(&bar[B_SFULL1], 1);
-    mbar_init(&bar[B_SFREE0], 4);
-    mbar_init(&bar[B_SFREE1], 4);
-    mbar_init(&bar[B_PFULL0], 4);
-    mbar_init(&bar[B_PFULL1], 4);
-    mbar_init(&bar[B_PFREE0], 1);
-    mbar_init(&bar[B_PFREE1], 1);
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&bar[B_KFULL0 + i], 1);
+      mbar_init(&bar[B_KEMPTY0 + i], 5);  // MMA commit + 4 softmax warps (token positions)
+      mbar_init(&bar[B_VFULL0 + i], 1);
+      mbar_init(&bar[B_VEMPTY0 + i], 1);
+      mbar_init(&bar[B_SFULL0 + i], 1);
+      mbar_init(&bar[B_SFREE0 + i], 4);
+    }
+    mbar_init(&bar[B_AFREE], 4);
+    mbar_init(&bar[B_TFULLA], 1);
+    mbar_init(&bar[B_TFULLB], 1);
+    mbar_init(&bar[B_TFREEA], 4);
+    mbar_init(&bar[B_TFREEB], 4);
+    mbar_init(&bar[B_PFULL], 4);
+    mbar_init(&bar[B_PFREE], 1);
     mbar_init(&bar[B_OFULL], 1);
     mbar_init(&bar[B_DRAIN], 1);
     fence_mbar_init();
@@ -166,64 +265,75 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (warp == 0) {
     // ------------------------------------------------------------------ producer
     if (lane == 0) {
-      mbar_expect_tx(&bar[B_Q], kTileBytes);
-      tma_load_3d(smem + OFF_Q, &q_map, &bar[B_Q], 0, i0, bhq);
-      tma_load_3d(smem + OFF_Q + kHalfBytes, &q_map, &bar[B_Q], 64, i0, bhq);
+      mbar_expect_tx(&bar[B_Q], has_b ? 2 * kTileBytes : kTileBytes);
+      tma_load_3d(smem + OFF_QA, &q_map, &bar[B_Q], 0, i0_a, bhq_a);
+      tma_load_3d(smem + OFF_QA + kHalfBytes, &q_map, &bar[B_Q], 64, i0_a, bhq_a);
+      if (has_b) {
+        tma_load_3d(smem + OFF_QB, &q_map, &bar[B_Q], 0, i0_b, bhq_b);
+        tma_load_3d(smem + OFF_QB + kHalfBytes, &q_map, &bar[B_Q], 64, i0_b, bhq_b);
+      }
       mbar_arrive(&bar[B_Q]);
     }
     const int32_t *tpg = p.token_pos + (size_t)bg * p.N_C;
-    int issued = 0;
+    int k_issued = 0, v_issued = 0;
     for (int it = 0; it < 2 * n_kt && !aborted; ++it) {
       const bool phB = it >= n_kt;
       const int kt = phB ? it - n_kt : it;
       const int s = it & 1, n = it >> 1;
-      if (n > 0 && !warp_wait(&bar[B_EMPTY0 + s], (n - 1) & 1, lim)) {
+      // K tile + token positions
+      if (n > 0 && !warp_wait(&bar[B_KEMPTY0 + s], (n - 1) & 1, lim)) {
         fail(p, aborted);
         break;
       }
       uint8_t *kdst = smem + (s ? OFF_K1 : OFF_K0);
-      uint8_t *vdst = smem + (s ? OFF_V1 : OFF_V0);
       if (lane == 0) {
-        mbar_expect_tx(&bar[B_FULL0 + s], phB ? 2 * kTileBytes : kTileBytes);
-        tma_load_3d(kdst, &k_map, &bar[B_FULL0 + s], 0, kt * BN, bg);
-        tma_load_3d(kdst + kHalfBytes, &k_map, &bar[B_FULL0 + s], 64, kt * BN, bg);
-        if (phB) {
-          tma_load_3d(vdst, &v_map, &bar[B_FULL0 + s], 0, kt * BN, bg);
-          tma_load_3d(vdst + kHalfBytes, &v_map, &bar[B_FULL0 + s], 64, kt * BN, bg);
-        }
+        mbar_expect_tx(&bar[B_KFULL0 + s], kTileBytes);
+        tma_load_3d(kdst, &k_map, &bar[B_KFULL0 + s], 0, kt * BN, bg);
+        tma_load_3d(kdst + kHalfBytes, &k_map, &bar[B_KFULL0 + s], 64, kt * BN, bg);
       }
-      int32_t tmax = INT32_MIN;
 #pragma unroll
       for (int e = lane; e < BN; e += 32) {
         const int j = kt * BN + e;
-        const int32_t v = j < p.N_C ? tpg[j] : kEmptyPos;
-        tp_s[s * BN + e] = v;
-        tmax = max(tmax, v);
+        tp_s[s * BN + e] = j < p.N_C ? tpg[j] : kEmptyPos;
       }
-#pragma unroll
-      for (int o = 16; o > 0; o >>= 1) tmax = max(tmax, __shfl_xor_sync(0xffffffffu, tmax, o));
-      if (lane == 0) tpmax_s[s] = tmax;
       __syncwarp();
-      if (lane == 0) mbar_arrive(&bar[B_FULL0 + s]);
-      issued = it + 1;
+      if (lane == 0) mbar_arrive(&bar[B_KFULL0 + s]);
+      k_issued = it + 1;
+      if (phB) {  // V tile, ring indexed by kt
+        const int vs = kt & 1, vn = kt >> 1;
+        if (vn > 0 && !warp_wait(&bar[B_VEMPTY0 + vs], (vn - 1) & 1, lim)) {
+          fail(p, aborted);
+          break;
+        }
+        uint8_t *vdst = smem + (vs ? OFF_V1 : OFF_V0);
+        if (lane == 0) {
+          mbar_expect_tx(&bar[B_VFULL0 + vs], kTileBytes);
+          tma_load_3d(vdst, &v_map, &bar[B_VFULL0 + vs], 0, kt * BN, bg);
+          tma_load_3d(vdst + kHalfBytes, &v_map, &bar[B_VFULL0 + vs], 64, kt * BN, bg);
+          mbar_arrive(&bar[B_VFULL0 + vs]);
+        }
+        v_issued = kt + 1;
+      }
     }
-    // drain: the last (up to two) issued stage loads must land before exit
+    // drain: the last issued loads must land before exit
     if (lane == 0) {
       mbar_wait(&bar[B_Q], 0, 4000000000ull);
-      for (int it = issued - 1; it >= 0 && it >= issued - 2; --it)
-        mbar_wait(&bar[B_FULL0 + (it & 1)], (it >> 1) & 1, 4000000000ull);
+      for (int it = k_issued - 1; it >= 0 && it >= k_issued - 2; --it)
+        mbar_wait(&bar[B_KFULL0 + (it & 1)], (it >> 1) & 1, 4000000000ull);
+      for (int kt = v_issued - 1; kt >= 0 && kt >= v_issued - 2; --kt)
+        mbar_wait(&bar[B_VFULL0 + (kt & 1)], (kt >> 1) & 1, 4000000000ull);
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------------ MMA issuer
     if (lane == 0) {
-      const uint32_t q_addr = sbase + OFF_Q;
+      const uint32_t qa_addr = sbase + OFF_QA, qb_addr = sbase + OFF_QB, p_addr = sbase + OFF_P;
       if (!mbar_wait(&bar[B_Q], 0, lim)) fail(p, aborted);
       tc_fence_after();
-      // phase A: S = Q K^T
+      // phase A: S_a, S_b = Q_a K^T, Q_b K^T into the column pair of the tile parity
       for (int kt = 0; kt < n_kt && !aborted; ++kt) {
-        const int s = kt & 1, u = kt, buf = u & 1;
-        if (!mbar_wait(&bar[B_FULL0 + s], (kt >> 1) & 1, lim)) { fail(p, aborted); break; }
-        if (u >= 2 && !mbar_wait(&bar[B_SFREE0 + buf], ((u >> 1) - 1) & 1, lim)) {
+        const int s = kt & 1, u = kt & 1;
+        if (!mbar_wait(&bar[B_KFULL0 + s], (kt >> 1) & 1, lim)) { fail(p, aborted); break; }
+        if (kt >= 2 && !mbar_wait(&bar[B_SFREE0 + u], ((kt >> 1) - 1) & 1, lim)) {
           fail(p, aborted);
           break;
         }
@@ -231,40 +341,61 @@ __global__ void __launch_bounds__(kThreads, 1)
         const uint32_t k_addr = sbase + (s ? OFF_K1 : OFF_K0);
 #pragma unroll
         for (int ks = 0; ks < D / 16; ++ks)
-          mma_bf16_ss(tmem + buf * 128, kmajor_desc(q_addr, ks), kmajor_desc(k_addr, ks),
+          mma_bf16_ss(tmem + u * 256, kmajor_desc(qa_addr, ks), kmajor_desc(k_addr, ks),
                       IDESC_K_MAJOR, ks > 0);
-        mma_commit(&bar[B_SFULL0 + buf]);
-        mma_commit(&bar[B_EMPTY0 + s]);
+        if (has_b) {
+#pragma unroll
+          for (int ks = 0; ks < D / 16; ++ks)
+            mma_bf16_ss(tmem + u * 256 + 128, kmajor_desc(qb_addr, ks), kmajor_desc(k_addr, ks),
+                        IDESC_K_MAJOR, ks > 0);
+        }
+        mma_commit(&bar[B_SFULL0 + u]);
+        mma_commit(&bar[B_KEMPTY0 + s]);
       }
-      // phase B: S^T = K Q^T, then O += P V
-      auto issue_st = [&](int kt) -> bool {
-        const int it = n_kt + kt, s = it & 1, u = n_kt + kt, buf = u & 1;
-        if (!mbar_wait(&bar[B_FULL0 + s], (it >> 1) & 1, lim)) return false;
-        if (u >= 2 && !mbar_wait(&bar[B_SFREE0 + buf], ((u >> 1) - 1) & 1, lim)) return false;
+      // every phase A TMEM read is done before phase B reuses the columns
+      if (!aborted && !mbar_wait(&bar[B_AFREE], 0, lim)) fail(p, aborted);
+      tc_fence_after();
+      // phase B.  S^T_x(kt) = K(kt) Q_x^T into columns 0 (a) / 128 (b);
+      // O_x += P_x(kt) V(kt) into columns 256 (a) / 384 (b).
+      auto issue_st = [&](int kt, bool tile_b) -> bool {
+        const int it = n_kt + kt, s = it & 1;
+        if (!tile_b && !mbar_wait(&bar[B_KFULL0 + s], (it >> 1) & 1, lim)) return false;
+        if (kt >= 1 && !mbar_wait(&bar[tile_b ? B_TFREEB : B_TFREEA], (kt - 1) & 1, lim))
+          return false;
         tc_fence_after();
         const uint32_t k_addr = sbase + (s ? OFF_K1 : OFF_K0);
+        const uint32_t q_addr = tile_b ? qb_addr : qa_addr;
 #pragma unroll
         for (int ks = 0; ks < D / 16; ++ks)
-          mma_bf16_ss(tmem + buf * 128, kmajor_desc(k_addr, ks), kmajor_desc(q_addr, ks),
+          mma_bf16_ss(tmem + (tile_b ? 128 : 0), kmajor_desc(k_addr, ks), kmajor_desc(q_addr, ks),
                       IDESC_K_MAJOR, ks > 0);
-        mma_commit(&bar[B_SFULL0 + buf]);
+        mma_commit(&bar[tile_b ? B_TFULLB : B_TFULLA]);
+        if (tile_b || !has_b) mma_commit(&bar[B_KEMPTY0 + s]);  // K(kt) no longer read
         return true;
       };
-      if (!aborted && !issue_st(0)) fail(p, aborted);
-      for (int kt = 0; kt < n_kt && !aborted; ++kt) {
-        if (kt + 1 < n_kt && !issue_st(kt + 1)) { fail(p, aborted); break; }
-        const int pb = kt & 1;
-        if (!mbar_wait(&bar[B_PFULL0 + pb], (kt >> 1) & 1, lim)) { fail(p, aborted); break; }
+      auto issue_pv = [&](int kt, bool tile_b) -> bool {
+        const int use = has_b ? 2 * kt + (tile_b ? 1 : 0) : kt;
+        if (!mbar_wait(&bar[B_PFULL], use & 1, lim)) return false;
+        if (!tile_b && !mbar_wait(&bar[B_VFULL0 + (kt & 1)], (kt >> 1) & 1, lim)) return false;
         tc_fence_after();
-        const int s = (n_kt + kt) & 1;
-        const uint32_t v_addr = sbase + (s ? OFF_V1 : OFF_V0);
-        const uint32_t p_addr = sbase + (pb ? OFF_P1 : OFF_P0);
+        const uint32_t v_addr = sbase + ((kt & 1) ? OFF_V1 : OFF_V0);
 #pragma unroll
         for (int ks = 0; ks < BN / 16; ++ks)
-          mma_bf16_ss(tmem + 256, mnmajor_desc(p_addr, ks), mnmajor_desc(v_addr, ks), IDESC_PV,
-                      (kt > 0 || ks > 0) ? 1u : 0u);
-        mma_commit(&bar[B_PFREE0 + pb]);
-        mma_commit(&bar[B_EMPTY0 + s]);
+          mma_bf16_ss(tmem + (tile_b ? 384 : 256), mnmajor_desc(p_addr, ks),
+                      mnmajor_desc(v_addr, ks), IDESC_PV, (kt > 0 || ks > 0) ? 1u : 0u);
+        mma_commit(&bar[B_PFREE]);
+        if (tile_b || !has_b) mma_commit(&bar[B_VEMPTY0 + (kt & 1)]);  // V(kt) no longer read
+        return true;
+      };
+      if (!aborted && !issue_st(0, false)) fail(p, aborted);
+      if (!aborted && has_b && !issue_st(0, true)) fail(p, aborted);
+      for (int kt = 0; kt < n_kt && !aborted; ++kt) {
+        if (!issue_pv(kt, false)) { fail(p, aborted); break; }
+        if (kt + 1 < n_kt && !issue_st(kt + 1, false)) { fail(p, aborted); break; }
+        if (has_b) {
+          if (!issue_pv(kt, true)) { fail(p, aborted); break; }
+          if (kt + 1 < n_kt && !issue_st(kt + 1, true)) { fail(p, aborted); break; }
+        }
       }
       mma_commit(&bar[B_OFULL]);
       // drain: every MMA issued by this thread completes before TMEM is freed
@@ -274,137 +405,115 @@ __global__ void __launch_bounds__(kThreads, 1)
     __syncwarp();
   } else if (warp >= 4) {
     // ------------------------------------------------------------ softmax / sums
-    const int st = threadIdx.x - 128;  // row (phase A) or slot (phase B) within the tile
+    const int st = threadIdx.x - 128;  // row (phase A) or slot (phase B) within a tile
     const uint32_t lane_base = (uint32_t)(32 * (warp - 4)) << 16;
     const float c2 = p.scale2;
-    const int row_i = i0 + st;
-    const int64_t row_lim = (int64_t)p.P + row_i;
-    float m = -INFINITY, l = 0.f;
-    uint32_t xr[BN];
+    const int64_t lim_a = (int64_t)p.P + i0_a + st, lim_b = (int64_t)p.P + i0_b + st;
+    const int i0_min = min(i0_a, i0_b);
+    float m_a = -INFINITY, l_a = 0.f, m_b = -INFINITY, l_b = 0.f;
+    uint32_t x[BN];
     for (int kt = 0; kt < n_kt && !aborted; ++kt) {
-      const int u = kt, buf = u & 1, s = kt & 1;
-      if (!warp_wait(&bar[B_SFULL0 + buf], (u >> 1) & 1, lim)) { fail(p, aborted); break; }
-      if (!warp_wait(&bar[B_FULL0 + s], (kt >> 1) & 1, lim)) { fail(p, aborted); break; }
+      const int u = kt & 1, s = kt & 1;
+      if (!warp_wait(&bar[B_SFULL0 + u], (kt >> 1) & 1, lim)) { fail(p, aborted); break; }
+      if (!warp_wait(&bar[B_KFULL0 + s], (kt >> 1) & 1, lim)) { fail(p, aborted); break; }
       tc_fence_after();
-      tmem_ld32(tmem + lane_base + buf * 128 + 0, *reinterpret_cast<uint32_t(*)[32]>(xr + 0));
-      tmem_ld32(tmem + lane_base + buf * 128 + 32, *reinterpret_cast<uint32_t(*)[32]>(xr + 32));
-      tmem_ld32(tmem + lane_base + buf * 128 + 64, *reinterpret_cast<uint32_t(*)[32]>(xr + 64));
-      tmem_ld32(tmem + lane_base + buf * 128 + 96, *reinterpret_cast<uint32_t(*)[32]>(xr + 96));
-      tmem_wait_ld();
+      // any slot of this tile invisible to some row of the CTA?
+      const int32_t tpv = max(max(tp_s[s * BN + lane], tp_s[s * BN + lane + 32]),
+                              max(tp_s[s * BN + lane + 64], tp_s[s * BN + lane + 96]));
+      const bool masked = __any_sync(0xffffffffu, (int64_t)tpv > (int64_t)p.P + i0_min);
+      tmem_ld128(tmem + lane_base + u * 256, x);
+      row_update(x, masked, tp_s + s * BN, lim_a, c2, m_a, l_a);
+      if (has_b) {
+        tmem_ld128(tmem + lane_base + u * 256 + 128, x);
+        row_update(x, masked, tp_s + s * BN, lim_b, c2, m_b, l_b);
+      }
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(&bar[B_SFREE0 + buf]);
-      const bool all_visible = (int64_t)tpmax_s[s] <= (int64_t)p.P + i0;
-      if (!all_visible) {
-#pragma unroll
-        for (int e = 0; e < BN; ++e)
-          if ((int64_t)tp_s[s * BN + e] > row_lim) xr[e] = __float_as_uint(-INFINITY);
+      if (lane == 0) {
+        mbar_arrive(&bar[B_SFREE0 + u]);
+        mbar_arrive(&bar[B_KEMPTY0 + s]);
       }
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&bar[B_EMPTY0 + s]);
-      // row max with 8 independent chains
-      float mx8[8];
-#pragma unroll
-      for (int q = 0; q < 8; ++q) mx8[q] = __uint_as_float(xr[q]);
-#pragma unroll
-      for (int e = 8; e < BN; ++e) mx8[e & 7] = fmaxf(mx8[e & 7], __uint_as_float(xr[e]));
-      const float mx = fmaxf(fmaxf(fmaxf(mx8[0], mx8[1]), fmaxf(mx8[2], mx8[3])),
-                             fmaxf(fmaxf(mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7])));
-      const float m_new = fmaxf(m, mx * c2);
-      if (m_new == -INFINITY) continue;
-      float sm8[8];
-#pragma unroll
-      for (int q = 0; q < 8; ++q) sm8[q] = 0.f;
-#pragma unroll
-      for (int e = 0; e < BN; ++e) sm8[e & 7] += ex2(fmaf(__uint_as_float(xr[e]), c2, -m_new));
-      const float sum = ((sm8[0] + sm8[1]) + (sm8[2] + sm8[3])) + ((sm8[4] + sm8[5]) + (sm8[6] + sm8[7]));
-      l = l * ex2(m - m_new) + sum;
-      m = m_new;
     }
-    const float lse2 = (l > 0.f) ? m + lg2(l) : -INFINITY;
-    lse_s[st] = lse2;
-    if (p.lse_out && row_i < p.S) p.lse_out[(size_t)bhq * p.S + row_i] = lse2 * 0.69314718055994531f;
+    __syncwarp();
+    if (lane == 0) mbar_arrive(&bar[B_AFREE]);
+    const float lse2_a = (l_a > 0.f) ? m_a + lg2(l_a) : -INFINITY;
+    const float lse2_b = (l_b > 0.f) ? m_b + lg2(l_b) : -INFINITY;
+    lse_s[st] = lse2_a;
+    lse_s[BM + st] = lse2_b;
+    if (p.lse_out) {
+      if (i0_a + st < p.S) p.lse_out[(size_t)bhq_a * p.S + i0_a + st] = lse2_a * 0.69314718055994531f;
+      if (has_b && i0_b + st < p.S)
+        p.lse_out[(size_t)bhq_b * p.S + i0_b + st] = lse2_b * 0.69314718055994531f;
+    }
     named_bar_sync(1, 128);
 
     // phase B
-    const int rmax = min(BM, p.S - i0);
-    float *pw = p.part_w + ((size_t)bhq * p.tiles + t) * p.N_C;
-    const uint32_t p_row = (st >> 3) * 1024 + (st & 7) * 128;
-    uint32_t r[32];
+    const int rmax_a = min(BM, p.S - i0_a), rmax_b = min(BM, p.S - i0_b);
+    float *pw_a = p.part_w + ((size_t)bhq_a * p.tiles + t_a) * p.N_C;
+    float *pw_b = p.part_w + ((size_t)bhq_b * p.tiles + t_b) * p.N_C;
+    const uint32_t p_row = sbase + OFF_P + (st >> 3) * 1024 + (st & 7) * 128;
+    uint32_t pk[BM / 2];
     for (int kt = 0; kt < n_kt && !aborted; ++kt) {
-      const int u = n_kt + kt, buf = u & 1, it = n_kt + kt, s = it & 1, pb = kt & 1;
-      if (!warp_wait(&bar[B_SFULL0 + buf], (u >> 1) & 1, lim)) { fail(p, aborted); break; }
-      if (!warp_wait(&bar[B_FULL0 + s], (it >> 1) & 1, lim)) { fail(p, aborted); break; }
-      // P buffer pb was last read by the P V product of tile kt - 2
-      if (kt >= 2 && !warp_wait(&bar[B_PFREE0 + pb], ((kt >> 1) - 1) & 1, lim)) {
-        fail(p, aborted);
-        break;
-      }
+      const int it = n_kt + kt, s = it & 1;
+      const int j = kt * BN + st;
+      // ---- tile a
+      if (!warp_wait(&bar[B_TFULLA], kt & 1, lim)) { fail(p, aborted); break; }
+      if (!warp_wait(&bar[B_KFULL0 + s], (it >> 1) & 1, lim)) { fail(p, aborted); break; }
       tc_fence_after();
       const int64_t tpj = tp_s[s * BN + st];
       __syncwarp();
-      if (lane == 0) mbar_arrive(&bar[B_EMPTY0 + s]);
-      // visible rows r of this tile: tpj <= P + i0 + r, r < rmax
-      const int64_t rm = tpj - (int64_t)p.P - i0;
-      const int rmin = rm <= 0 ? 0 : (rm >= BM ? BM : (int)rm);
-      const bool full = __all_sync(0xffffffffu, rmin == 0 && rmax == BM);
-      const uint32_t p_buf = sbase + (pb ? OFF_P1 : OFF_P0) + p_row;
-      float cs8[8];
-#pragma unroll
-      for (int q = 0; q < 8; ++q) cs8[q] = 0.f;
-#pragma unroll
-      for (int c = 0; c < 4; ++c) {
-        tmem_ld32(tmem + lane_base + buf * 128 + c * 32, r);
-        tmem_wait_ld();
-        uint32_t pk[16];
-#pragma unroll
-        for (int e = 0; e < 32; e += 2) {
-          const int r0 = c * 32 + e;
-          float p0 = ex2(fmaf(__uint_as_float(r[e]), c2, -lse_s[r0]));
-          float p1 = ex2(fmaf(__uint_as_float(r[e + 1]), c2, -lse_s[r0 + 1]));
-          if (!full) {
-            p0 = (r0 >= rmin && r0 < rmax) ? p0 : 0.f;
-            p1 = (r0 + 1 >= rmin && r0 + 1 < rmax) ? p1 : 0.f;
-          }
-          cs8[(e >> 1) & 7] += p0 + p1;
-          pk[e >> 1] = pack_bf16x2(p0, p1);
-        }
-        // rows 32c .. 32c+31 = M block c/2, 16-byte chunks (c%2)*4 .. +3 of this slot's K row
-#pragma unroll
-        for (int q = 0; q < 4; ++q) {
-          const int cc = (c & 1) * 4 + q;
-          const uint32_t addr = p_buf + (c >> 1) * kHalfBytes + ((cc ^ (st & 7)) << 4);
-          asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(pk[4 * q]),
-                       "r"(pk[4 * q + 1]), "r"(pk[4 * q + 2]), "r"(pk[4 * q + 3])
-                       : "memory");
-        }
-      }
+      if (lane == 0) mbar_arrive(&bar[B_KEMPTY0 + s]);
+      const int64_t rm_a = tpj - (int64_t)p.P - i0_a, rm_b = tpj - (int64_t)p.P - i0_b;
+      const int rmin_a = rm_a <= 0 ? 0 : (rm_a >= BM ? BM : (int)rm_a);
+      const int rmin_b = rm_b <= 0 ? 0 : (rm_b >= BM ? BM : (int)rm_b);
+      const bool full_a = __all_sync(0xffffffffu, rmin_a == 0 && rmax_a == BM);
+      const float cs_a = slot_probs(tmem + lane_base + 0, lse_s, c2, rmin_a, rmax_a, full_a, pk);
       tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&bar[B_TFREEA]);
+      // P buffer was last read by PV of the previous use (b of kt-1, or a of kt-1)
+      const int use_a = has_b ? 2 * kt : kt;
+      if (use_a > 0 && !warp_wait(&bar[B_PFREE], (use_a - 1) & 1, lim)) { fail(p, aborted); break; }
+      store_p(p_row, st, pk);
       fence_proxy_async_smem();
       __syncwarp();
-      if (lane == 0) {
-        mbar_arrive(&bar[B_SFREE0 + buf]);
-        mbar_arrive(&bar[B_PFULL0 + pb]);
-      }
-      const float colsum = ((cs8[0] + cs8[1]) + (cs8[2] + cs8[3])) + ((cs8[4] + cs8[5]) + (cs8[6] + cs8[7]));
-      const int j = kt * BN + st;
-      if (j < p.N_C) pw[j] = colsum;
+      if (lane == 0) mbar_arrive(&bar[B_PFULL]);
+      if (j < p.N_C) pw_a[j] = cs_a;
+      if (!has_b) continue;
+      // ---- tile b
+      if (!warp_wait(&bar[B_TFULLB], kt & 1, lim)) { fail(p, aborted); break; }
+      tc_fence_after();
+      const bool full_b = __all_sync(0xffffffffu, rmin_b == 0 && rmax_b == BM);
+      const float cs_b =
+          slot_probs(tmem + lane_base + 128, lse_s + BM, c2, rmin_b, rmax_b, full_b, pk);
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&bar[B_TFREEB]);
+      if (!warp_wait(&bar[B_PFREE], (2 * kt) & 1, lim)) { fail(p, aborted); break; }
+      store_p(p_row, st, pk);
+      fence_proxy_async_smem();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&bar[B_PFULL]);
+      if (j < p.N_C) pw_b[j] = cs_b;
     }
     // epilogue: y = O (already normalised)
     if (!aborted && !warp_wait(&bar[B_OFULL], 0, lim)) fail(p, aborted);
     tc_fence_after();
-    if (!aborted) {
-      __nv_bfloat16 *yrow = p.y + ((size_t)bhq * p.S + row_i) * D;
+    for (int tt = 0; tt < (has_b ? 2 : 1) && !aborted; ++tt) {
+      const int i0 = tt ? i0_b : i0_a;
+      const int row_i = i0 + st;
+      __nv_bfloat16 *yrow = p.y + ((size_t)(tt ? bhq_b : bhq_a) * p.S + row_i) * D;
+      uint32_t r[32];
 #pragma unroll
-      for (int c = 0; c < 4; ++c) {
-        tmem_ld32(tmem + lane_base + 256 + c * 32, r);
+      for (int cq = 0; cq < 4; ++cq) {
+        tmem_ld32(tmem + lane_base + 256 + tt * 128 + cq * 32, r);
         tmem_wait_ld();
         if (row_i < p.S) {
           uint32_t o[16];
 #pragma unroll
           for (int e = 0; e < 16; ++e)
             o[e] = pack_bf16x2(__uint_as_float(r[2 * e]), __uint_as_float(r[2 * e + 1]));
-          uint4 *dst = reinterpret_cast<uint4 *>(yrow + c * 32);
+          uint4 *dst = reinterpret_cast<uint4 *>(yrow + cq * 32);
 #pragma unroll
           for (int e = 0; e < 4; ++e)
             dst[e] = make_uint4(o[4 * e], o[4 * e + 1], o[4 * e + 2], o[4 * e + 3]);
@@ -529,9 +638,10 @@ int launch_attn_tc(h2okv_cache *c, const void *q, int S, int64_t P, void *y, flo
   prm.P = (int)P;
   prm.tiles = (S + BM - 1) / BM;
   prm.n_kt = (d.capacity + BN - 1) / BN;
+  prm.ctas_per_group = (prm.q_g * prm.tiles + 1) / 2;
   prm.scale2 = (float)(1.4426950408889634 / 11.313708498984761);  // log2(e) / sqrt(128)
   prm.timeout_ns = c->wait_timeout_ns;
-  const int grid = d.batch * d.n_q_heads * prm.tiles;
+  const int grid = d.batch * d.n_kv_heads * prm.ctas_per_group;
   attn_tc_kernel<<<grid, kThreads, kSmemBytes, st>>>(
       qmap, *reinterpret_cast<const CUtensorMap *>(c->tc.k_map),
       *reinterpret_cast<const CUtensorMap *>(c->tc.v_map), prm);

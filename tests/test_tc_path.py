@@ -26,6 +26,7 @@ CASES = [
     tc("tc_s_eq_capacity", capacity=256, chunk=256, seq_len=768),
     tc("tc_mha_c384_s128", Hq=2, Hk=2, capacity=384, chunk=128, seq_len=1024),
     tc("tc_s100_c700", Hq=4, Hk=1, capacity=700, chunk=100, seq_len=1200, heavy_hitters=False),
+    tc("tc_mha_s300_odd_tiles", Hq=2, Hk=2, capacity=640, chunk=300, seq_len=1500),
 ]
 
 
