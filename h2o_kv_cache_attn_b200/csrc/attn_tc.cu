@@ -19,10 +19,12 @@
 //            O += P V (A = P, B = V, both MN-major).  P is normalised already,
 //            so O needs no rescaling.  TMEM: S^T_a, S^T_b, O_a, O_b.
 //
-// Warp roles (256 threads): warp 0 TMA producer (K and V tiles through separate
+// Warp roles (384 threads): warp 0 TMA producer (K and V tiles through separate
 // two-stage rings via cp.async.bulk.tensor, no multicast; token positions by
 // plain loads), warp 1 TMEM allocator and single-thread MMA issuer, warps 4-7
-// softmax / column sums / epilogue (warp 4+q owns TMEM lanes 32q..32q+31).
+// (tile a) and 8-11 (tile b) softmax / column sums / epilogue (warp w owns
+// TMEM lanes 32(w%4)..32(w%4)+31).  The single P buffer is handed over
+// a(kt) -> b(kt) -> a(kt+1) through per-tile full / free barriers.
 // The MMA issue order PV_a(kt), S^T_a(kt+1), PV_b(kt), S^T_b(kt+1) keeps the
 // tensor pipe busy while the softmax warps work on the other query tile.
 // Every wait is bounded; a timeout sets the cache's device status word and the
@@ -43,7 +45,7 @@ using namespace ptx;
 constexpr int BM = 128;        // query rows per tile
 constexpr int BN = 128;        // slots per tile
 constexpr int D = 128;         // head dim
-constexpr int kThreads = 256;
+constexpr int kThreads = 384;  // 4 control warps + 2 softmax warpgroups
 constexpr uint32_t kTileBytes = BM * D * 2;  // 32 KiB (two 64-column swizzled halves)
 constexpr uint32_t kHalfBytes = kTileBytes / 2;
 
@@ -58,7 +60,7 @@ constexpr uint32_t OFF_P = OFF_V1 + kTileBytes;
 constexpr uint32_t OFF_TP = OFF_P + kTileBytes;        // int32 [2 stages][BN]
 constexpr uint32_t OFF_LSE = OFF_TP + 2 * BN * 4;      // float [2 tiles][BM]
 constexpr uint32_t OFF_BAR = OFF_LSE + 2 * BM * 4;     // uint64 barriers
-constexpr int NBAR = 22;
+constexpr int NBAR = 24;
 constexpr uint32_t OFF_TMEM = OFF_BAR + NBAR * 8;
 constexpr uint32_t kSmemBytes = OFF_TMEM + 16;
 static_assert(kSmemBytes <= 232448, "shared memory budget");
@@ -85,7 +87,7 @@ enum {
   B_SFULL0, B_SFULL1, B_SFREE0, B_SFREE1,    // phase A S pair per tile parity
   B_AFREE,                                   // phase A TMEM fully read
   B_TFULLA, B_TFULLB, B_TFREEA, B_TFREEB,    // phase B S^T per query tile
-  B_PFULL, B_PFREE,                          // P buffer (uses alternate a, b)
+  B_PFULLA, B_PFULLB, B_PFREEA, B_PFREEB,    // P buffer, handed a(kt) -> b(kt) -> a(kt+1)
   B_OFULL, B_DRAIN                           // O complete; MMA drain before TMEM is freed
 };
 
@@ -117,27 +119,20 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   return *reinterpret_cast<uint32_t *>(&v);
 }
 
-__device__ __forceinline__ void tmem_ld128(uint32_t taddr, uint32_t (&x)[BN]) {
-  tmem_ld32(taddr + 0, *reinterpret_cast<uint32_t(*)[32]>(x + 0));
-  tmem_ld32(taddr + 32, *reinterpret_cast<uint32_t(*)[32]>(x + 32));
-  tmem_ld32(taddr + 64, *reinterpret_cast<uint32_t(*)[32]>(x + 64));
-  tmem_ld32(taddr + 96, *reinterpret_cast<uint32_t(*)[32]>(x + 96));
-  tmem_wait_ld();
-}
-
-// Online (max, sum) update of one row over one 128-slot tile (base-2 units).
-__device__ __forceinline__ void row_update(uint32_t (&x)[BN], bool masked, const int32_t *tp,
+// Online (max, sum) update of one row over N slots (base-2 units).
+template <int N>
+__device__ __forceinline__ void row_update(uint32_t (&x)[N], bool masked, const int32_t *tp,
                                            int64_t row_lim, float c2, float &m, float &l) {
   if (masked) {
 #pragma unroll
-    for (int e = 0; e < BN; ++e)
+    for (int e = 0; e < N; ++e)
       if ((int64_t)tp[e] > row_lim) x[e] = __float_as_uint(-INFINITY);
   }
   float mx8[8];
 #pragma unroll
   for (int q = 0; q < 8; ++q) mx8[q] = __uint_as_float(x[q]);
 #pragma unroll
-  for (int e = 8; e < BN; ++e) mx8[e & 7] = fmaxf(mx8[e & 7], __uint_as_float(x[e]));
+  for (int e = 8; e < N; ++e) mx8[e & 7] = fmaxf(mx8[e & 7], __uint_as_float(x[e]));
   const float mx = fmaxf(fmaxf(fmaxf(mx8[0], mx8[1]), fmaxf(mx8[2], mx8[3])),
                          fmaxf(fmaxf(mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7])));
   const float m_new = fmaxf(m, mx * c2);
@@ -146,7 +141,7 @@ __device__ __forceinline__ void row_update(uint32_t (&x)[BN], bool masked, const
 #pragma unroll
   for (int q = 0; q < 8; ++q) sm8[q] = 0.f;
 #pragma unroll
-  for (int e = 0; e < BN; ++e) sm8[e & 7] += ex2(fmaf(__uint_as_float(x[e]), c2, -m_new));
+  for (int e = 0; e < N; ++e) sm8[e & 7] += ex2(fmaf(__uint_as_float(x[e]), c2, -m_new));
   const float sum = ((sm8[0] + sm8[1]) + (sm8[2] + sm8[3])) + ((sm8[4] + sm8[5]) + (sm8[6] + sm8[7]));
   l = l * ex2(m - m_new) + sum;
   m = m_new;
@@ -226,23 +221,26 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int n_kt = p.n_kt;
   const uint64_t lim = p.timeout_ns;
 
+  const int nwg = has_b ? 2 : 1;  // softmax warpgroups with a query tile
   if (threadIdx.x == 0) {
     mbar_init(&bar[B_Q], 1);
     for (int i = 0; i < 2; ++i) {
       mbar_init(&bar[B_KFULL0 + i], 1);
-      mbar_init(&bar[B_KEMPTY0 + i], 5);  // MMA commit + 4 softmax warps (token positions)
+      mbar_init(&bar[B_KEMPTY0 + i], 1 + 4 * nwg);  // MMA commit + softmax warps (token positions)
       mbar_init(&bar[B_VFULL0 + i], 1);
       mbar_init(&bar[B_VEMPTY0 + i], 1);
       mbar_init(&bar[B_SFULL0 + i], 1);
-      mbar_init(&bar[B_SFREE0 + i], 4);
+      mbar_init(&bar[B_SFREE0 + i], 4 * nwg);
     }
-    mbar_init(&bar[B_AFREE], 4);
+    mbar_init(&bar[B_AFREE], 4 * nwg);
     mbar_init(&bar[B_TFULLA], 1);
     mbar_init(&bar[B_TFULLB], 1);
     mbar_init(&bar[B_TFREEA], 4);
     mbar_init(&bar[B_TFREEB], 4);
-    mbar_init(&bar[B_PFULL], 4);
-    mbar_init(&bar[B_PFREE], 1);
+    mbar_init(&bar[B_PFULLA], 4);
+    mbar_init(&bar[B_PFULLB], 4);
+    mbar_init(&bar[B_PFREEA], 1);
+    mbar_init(&bar[B_PFREEB], 1);
     mbar_init(&bar[B_OFULL], 1);
     mbar_init(&bar[B_DRAIN], 1);
     fence_mbar_init();
@@ -374,8 +372,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         return true;
       };
       auto issue_pv = [&](int kt, bool tile_b) -> bool {
-        const int use = has_b ? 2 * kt + (tile_b ? 1 : 0) : kt;
-        if (!mbar_wait(&bar[B_PFULL], use & 1, lim)) return false;
+        if (!mbar_wait(&bar[tile_b ? B_PFULLB : B_PFULLA], kt & 1, lim)) return false;
         if (!tile_b && !mbar_wait(&bar[B_VFULL0 + (kt & 1)], (kt >> 1) & 1, lim)) return false;
         tc_fence_after();
         const uint32_t v_addr = sbase + ((kt & 1) ? OFF_V1 : OFF_V0);
@@ -383,7 +380,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int ks = 0; ks < BN / 16; ++ks)
           mma_bf16_ss(tmem + (tile_b ? 384 : 256), mnmajor_desc(p_addr, ks),
                       mnmajor_desc(v_addr, ks), IDESC_PV, (kt > 0 || ks > 0) ? 1u : 0u);
-        mma_commit(&bar[B_PFREE]);
+        mma_commit(&bar[tile_b ? B_PFREEB : B_PFREEA]);
         if (tile_b || !has_b) mma_commit(&bar[B_VEMPTY0 + (kt & 1)]);  // V(kt) no longer read
         return true;
       };
@@ -403,31 +400,35 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_wait(&bar[B_DRAIN], 0, 4000000000ull);
     }
     __syncwarp();
-  } else if (warp >= 4) {
-    // ------------------------------------------------------------ softmax / sums
-    const int st = threadIdx.x - 128;  // row (phase A) or slot (phase B) within a tile
-    const uint32_t lane_base = (uint32_t)(32 * (warp - 4)) << 16;
+  } else if (warp >= 4 && (warp < 8 || has_b)) {
+    // -------------------------------------------- softmax / sums, one warpgroup per query tile
+    const int wg = (warp - 4) >> 2;  // 0: tile a, 1: tile b
+    const int st = threadIdx.x - 128 * (1 + wg);  // row (phase A) or slot (phase B) in the tile
+    const uint32_t lane_base = (uint32_t)(32 * (warp & 3)) << 16;
     const float c2 = p.scale2;
-    const int64_t lim_a = (int64_t)p.P + i0_a + st, lim_b = (int64_t)p.P + i0_b + st;
-    const int i0_min = min(i0_a, i0_b);
-    float m_a = -INFINITY, l_a = 0.f, m_b = -INFINITY, l_b = 0.f;
-    uint32_t x[BN];
+    const int i0 = wg ? i0_b : i0_a, bhq = wg ? bhq_b : bhq_a, t = wg ? t_b : t_a;
+    const int64_t row_lim = (int64_t)p.P + i0 + st;
+    float m = -INFINITY, l = 0.f;
+    uint32_t x[64];
     for (int kt = 0; kt < n_kt && !aborted; ++kt) {
       const int u = kt & 1, s = kt & 1;
       if (!warp_wait(&bar[B_SFULL0 + u], (kt >> 1) & 1, lim)) { fail(p, aborted); break; }
       if (!warp_wait(&bar[B_KFULL0 + s], (kt >> 1) & 1, lim)) { fail(p, aborted); break; }
       tc_fence_after();
-      // any slot of this tile invisible to some row of the CTA?
+      // any slot of this tile invisible to some row of this query tile?
       const int32_t tpv = max(max(tp_s[s * BN + lane], tp_s[s * BN + lane + 32]),
                               max(tp_s[s * BN + lane + 64], tp_s[s * BN + lane + 96]));
-      const bool masked = __any_sync(0xffffffffu, (int64_t)tpv > (int64_t)p.P + i0_min);
-      tmem_ld128(tmem + lane_base + u * 256, x);
-      row_update(x, masked, tp_s + s * BN, lim_a, c2, m_a, l_a);
-      if (has_b) {
-        tmem_ld128(tmem + lane_base + u * 256 + 128, x);
-        row_update(x, masked, tp_s + s * BN, lim_b, c2, m_b, l_b);
-      }
+      const bool masked = __any_sync(0xffffffffu, (int64_t)tpv > (int64_t)p.P + i0);
+      const uint32_t sa = tmem + lane_base + u * 256 + wg * 128;
+      tmem_ld32(sa, *reinterpret_cast<uint32_t(*)[32]>(x));
+      tmem_ld32(sa + 32, *reinterpret_cast<uint32_t(*)[32]>(x + 32));
+      tmem_wait_ld();
+      row_update<64>(x, masked, tp_s + s * BN, row_lim, c2, m, l);
+      tmem_ld32(sa + 64, *reinterpret_cast<uint32_t(*)[32]>(x));
+      tmem_ld32(sa + 96, *reinterpret_cast<uint32_t(*)[32]>(x + 32));
+      tmem_wait_ld();
       tc_fence_before();
+      row_update<64>(x, masked, tp_s + s * BN + 64, row_lim, c2, m, l);
       __syncwarp();
       if (lane == 0) {
         mbar_arrive(&bar[B_SFREE0 + u]);
@@ -436,77 +437,58 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     __syncwarp();
     if (lane == 0) mbar_arrive(&bar[B_AFREE]);
-    const float lse2_a = (l_a > 0.f) ? m_a + lg2(l_a) : -INFINITY;
-    const float lse2_b = (l_b > 0.f) ? m_b + lg2(l_b) : -INFINITY;
-    lse_s[st] = lse2_a;
-    lse_s[BM + st] = lse2_b;
-    if (p.lse_out) {
-      if (i0_a + st < p.S) p.lse_out[(size_t)bhq_a * p.S + i0_a + st] = lse2_a * 0.69314718055994531f;
-      if (has_b && i0_b + st < p.S)
-        p.lse_out[(size_t)bhq_b * p.S + i0_b + st] = lse2_b * 0.69314718055994531f;
-    }
-    named_bar_sync(1, 128);
+    const float lse2 = (l > 0.f) ? m + lg2(l) : -INFINITY;
+    float *lse_t = lse_s + wg * BM;
+    lse_t[st] = lse2;
+    if (p.lse_out && i0 + st < p.S)
+      p.lse_out[(size_t)bhq * p.S + i0 + st] = lse2 * 0.69314718055994531f;
+    named_bar_sync(1 + wg, 128);
 
     // phase B
-    const int rmax_a = min(BM, p.S - i0_a), rmax_b = min(BM, p.S - i0_b);
-    float *pw_a = p.part_w + ((size_t)bhq_a * p.tiles + t_a) * p.N_C;
-    float *pw_b = p.part_w + ((size_t)bhq_b * p.tiles + t_b) * p.N_C;
+    const int rmax = min(BM, p.S - i0);
+    float *pw = p.part_w + ((size_t)bhq * p.tiles + t) * p.N_C;
     const uint32_t p_row = sbase + OFF_P + (st >> 3) * 1024 + (st & 7) * 128;
     uint32_t pk[BM / 2];
     for (int kt = 0; kt < n_kt && !aborted; ++kt) {
       const int it = n_kt + kt, s = it & 1;
       const int j = kt * BN + st;
-      // ---- tile a
-      if (!warp_wait(&bar[B_TFULLA], kt & 1, lim)) { fail(p, aborted); break; }
+      if (!warp_wait(&bar[wg ? B_TFULLB : B_TFULLA], kt & 1, lim)) { fail(p, aborted); break; }
       if (!warp_wait(&bar[B_KFULL0 + s], (it >> 1) & 1, lim)) { fail(p, aborted); break; }
       tc_fence_after();
       const int64_t tpj = tp_s[s * BN + st];
       __syncwarp();
       if (lane == 0) mbar_arrive(&bar[B_KEMPTY0 + s]);
-      const int64_t rm_a = tpj - (int64_t)p.P - i0_a, rm_b = tpj - (int64_t)p.P - i0_b;
-      const int rmin_a = rm_a <= 0 ? 0 : (rm_a >= BM ? BM : (int)rm_a);
-      const int rmin_b = rm_b <= 0 ? 0 : (rm_b >= BM ? BM : (int)rm_b);
-      const bool full_a = __all_sync(0xffffffffu, rmin_a == 0 && rmax_a == BM);
-      const float cs_a = slot_probs(tmem + lane_base + 0, lse_s, c2, rmin_a, rmax_a, full_a, pk);
+      // visible rows r of this tile: tpj <= P + i0 + r, r < rmax
+      const int64_t rm = tpj - (int64_t)p.P - i0;
+      const int rmin = rm <= 0 ? 0 : (rm >= BM ? BM : (int)rm);
+      const bool full = __all_sync(0xffffffffu, rmin == 0 && rmax == BM);
+      const float cs = slot_probs(tmem + lane_base + wg * 128, lse_t, c2, rmin, rmax, full, pk);
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(&bar[B_TFREEA]);
-      // P buffer was last read by PV of the previous use (b of kt-1, or a of kt-1)
-      const int use_a = has_b ? 2 * kt : kt;
-      if (use_a > 0 && !warp_wait(&bar[B_PFREE], (use_a - 1) & 1, lim)) { fail(p, aborted); break; }
+      if (lane == 0) mbar_arrive(&bar[wg ? B_TFREEB : B_TFREEA]);
+      // the single P buffer goes a(kt) -> b(kt) -> a(kt+1): wait for the previous reader
+      bool ok = true;
+      if (wg == 1)
+        ok = warp_wait(&bar[B_PFREEA], kt & 1, lim);
+      else if (kt > 0)
+        ok = warp_wait(&bar[has_b ? B_PFREEB : B_PFREEA], (kt - 1) & 1, lim);
+      if (!ok) { fail(p, aborted); break; }
       store_p(p_row, st, pk);
       fence_proxy_async_smem();
       __syncwarp();
-      if (lane == 0) mbar_arrive(&bar[B_PFULL]);
-      if (j < p.N_C) pw_a[j] = cs_a;
-      if (!has_b) continue;
-      // ---- tile b
-      if (!warp_wait(&bar[B_TFULLB], kt & 1, lim)) { fail(p, aborted); break; }
-      tc_fence_after();
-      const bool full_b = __all_sync(0xffffffffu, rmin_b == 0 && rmax_b == BM);
-      const float cs_b =
-          slot_probs(tmem + lane_base + 128, lse_s + BM, c2, rmin_b, rmax_b, full_b, pk);
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&bar[B_TFREEB]);
-      if (!warp_wait(&bar[B_PFREE], (2 * kt) & 1, lim)) { fail(p, aborted); break; }
-      store_p(p_row, st, pk);
-      fence_proxy_async_smem();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&bar[B_PFULL]);
-      if (j < p.N_C) pw_b[j] = cs_b;
+      if (lane == 0) mbar_arrive(&bar[wg ? B_PFULLB : B_PFULLA]);
+      if (j < p.N_C) pw[j] = cs;
     }
     // epilogue: y = O (already normalised)
     if (!aborted && !warp_wait(&bar[B_OFULL], 0, lim)) fail(p, aborted);
     tc_fence_after();
-    for (int tt = 0; tt < (has_b ? 2 : 1) && !aborted; ++tt) {
-      const int i0 = tt ? i0_b : i0_a;
+    if (!aborted) {
       const int row_i = i0 + st;
-      __nv_bfloat16 *yrow = p.y + ((size_t)(tt ? bhq_b : bhq_a) * p.S + row_i) * D;
+      __nv_bfloat16 *yrow = p.y + ((size_t)bhq * p.S + row_i) * D;
       uint32_t r[32];
 #pragma unroll
       for (int cq = 0; cq < 4; ++cq) {
-        tmem_ld32(tmem + lane_base + 256 + tt * 128 + cq * 32, r);
+        tmem_ld32(tmem + lane_base + 256 + wg * 128 + cq * 32, r);
         tmem_wait_ld();
         if (row_i < p.S) {
           uint32_t o[16];
