@@ -25,7 +25,7 @@ BUF_NAMES = ("keys", "values", "k_scales", "v_scales", "token_pos", "scores", "w
 EXPORTED = ("kv_cache_query_sizes", "kv_cache_create", "kv_cache_reset", "kv_cache_destroy",
             "kv_cache_get_fill", "kv_cache_set_fill", "kv_cache_quantize", "h2o_evict_insert",
             "attn_chunk_with_scoresum", "kv_cache_device_status", "kv_cache_set_wait_timeout",
-            "h2okv_last_error", "h2okv_abi_version")
+            "attn_chunk_with_scoresum_noalloc", "h2okv_last_error", "h2okv_abi_version")
 
 
 class H2OKVError(RuntimeError):
@@ -78,6 +78,8 @@ def load() -> ctypes.CDLL:
         "attn_chunk_with_scoresum": (ctypes.c_int, [vp, vp, i32, i64, vp, vp, vp, vp, vp]),
         "kv_cache_device_status": (ctypes.c_int, [vp, ctypes.POINTER(i32), vp]),
         "kv_cache_set_wait_timeout": (ctypes.c_int, [vp, ctypes.c_uint64]),
+        "attn_chunk_with_scoresum_noalloc": (ctypes.c_int, [ctypes.POINTER(CacheDesc), vp, vp, vp, vp,
+                                                            vp, vp, i32, i64, vp, vp, vp, vp, vp]),
         "h2okv_last_error": (ctypes.c_char_p, []),
         "h2okv_abi_version": (i32, []),
     }
@@ -171,6 +173,17 @@ def kv_cache_device_status(handle, stream=None) -> int:
 
 def kv_cache_set_wait_timeout(handle, timeout_ns: int):
     _check(load().kv_cache_set_wait_timeout(handle, int(timeout_ns)))
+
+
+def attn_chunk_with_scoresum_noalloc(desc: CacheDesc, keys, values, k_scales, v_scales, token_pos,
+                                     q, S: int, P: int, y_out, lse_out, w_out, wq_out=None,
+                                     stream=None):
+    """Allocation-free attention over caller-owned cache buffers (no handle, no
+    workspace); its scratch is a fixed array inside the library."""
+    _check(load().attn_chunk_with_scoresum_noalloc(
+        ctypes.byref(desc), _ptr(keys), _ptr(values), _ptr(k_scales), _ptr(v_scales),
+        _ptr(token_pos), _ptr(q), int(S), int(P), _ptr(y_out), _ptr(lse_out), _ptr(w_out),
+        _ptr(wq_out), _stream(stream)))
 
 
 def h2okv_last_error() -> str:

@@ -14,6 +14,8 @@
 // g is head g*q_g + r / S, chunk row r % S.
 #include <math.h>
 
+#include <mutex>
+
 #include "h2okv_internal.cuh"
 
 namespace h2okv {
@@ -319,3 +321,112 @@ int launch_attn_simt(h2okv_cache *c, const void *q, int S, int64_t P, void *y, f
 }
 
 }  // namespace h2okv
+
+// ---- allocation-free entry point ---------------------------------------------------
+// Some callers cannot allocate device memory: every byte they use is owned by
+// another allocator (a framework's caching pool, an inference engine's fixed
+// arena), so they cannot size and hand over the per-cache workspace that
+// attn_chunk_with_scoresum needs.  attn_chunk_with_scoresum_noalloc runs the
+// CUDA-core attention above with its only scratch -- one base-2 log-sum-exp per
+// query row -- in a file-scope __device__ array instead.
+namespace h2okv {
+namespace {
+
+// B * H_q * S rows the array holds (1 MiB of float per device).
+constexpr size_t kNoAllocMaxRows = size_t(1) << 18;
+constexpr int kNoAllocMaxDevices = 64;
+
+static __device__ __align__(256) float g_noalloc_lse2[kNoAllocMaxRows];
+
+std::mutex g_noalloc_mu;
+float *g_noalloc_ptr[kNoAllocMaxDevices];
+
+// Device address of the array on the current device.  In host code the array's
+// name is only a host-side stand-in, so its device address is looked up once per
+// device (with that device current) and cached.
+int noalloc_scratch(float **out) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess)
+    return set_error(H2OKV_ERR_CUDA, "cudaGetDevice: %s", cudaGetErrorString(e));
+  if (dev < 0 || dev >= kNoAllocMaxDevices)
+    return set_error(H2OKV_ERR_UNSUPPORTED, "device ordinal %d above %d", dev,
+                     kNoAllocMaxDevices - 1);
+  std::lock_guard<std::mutex> lock(g_noalloc_mu);
+  if (!g_noalloc_ptr[dev]) {
+    void *ptr = nullptr;
+    e = cudaGetSymbolAddress(&ptr, g_noalloc_lse2);
+    if (e != cudaSuccess)
+      return set_error(H2OKV_ERR_CUDA, "cudaGetSymbolAddress(scratch): %s", cudaGetErrorString(e));
+    g_noalloc_ptr[dev] = static_cast<float *>(ptr);
+  }
+  *out = g_noalloc_ptr[dev];
+  return H2OKV_OK;
+}
+
+}  // namespace
+}  // namespace h2okv
+
+extern "C" int attn_chunk_with_scoresum_noalloc(const h2okv_cache_desc *desc, const void *keys,
+                                                const void *values, const void *k_scales,
+                                                const void *v_scales, const int32_t *token_pos,
+                                                const void *q, int32_t S, int64_t P, void *y_out,
+                                                float *lse_out, float *w_out, float *wq_out,
+                                                void *stream) {
+  using namespace h2okv;
+  set_error(H2OKV_OK, "");
+  size_t sizes[H2OKV_NUM_BUFS];
+  int rc = kv_cache_query_sizes(desc, sizes);  // validates the description
+  if (rc) return rc;
+  const bool quant = desc->kv_dtype == H2OKV_I8 || desc->kv_dtype == H2OKV_I4;
+  if (!keys || !values || !token_pos || !q || !y_out || !w_out || (quant && (!k_scales || !v_scales)))
+    return set_error(H2OKV_ERR_INVALID_ARG, "a required buffer is NULL");
+  if (S < 1 || S > desc->max_chunk)
+    return set_error(H2OKV_ERR_INVALID_ARG, "S = %d outside [1, max_chunk %d]", S,
+                     desc->max_chunk);
+  if (P < 0 || P + S >= (int64_t)INT32_MAX)
+    return set_error(H2OKV_ERR_INVALID_ARG, "P = %lld out of range for int32 token positions",
+                     (long long)P);
+  const size_t rows = (size_t)desc->batch * desc->n_q_heads * S;
+  if (rows > kNoAllocMaxRows)
+    return set_error(H2OKV_ERR_INVALID_ARG,
+                     "batch * n_q_heads * S = %zu exceeds the %zu rows of the static scratch", rows,
+                     kNoAllocMaxRows);
+  float *scratch = nullptr;
+  rc = noalloc_scratch(&scratch);
+  if (rc) return rc;
+
+  cudaStream_t st = (cudaStream_t)stream;
+  SimtArgs a;
+  a.q = q;
+  a.keys = reinterpret_cast<const uint8_t *>(keys);
+  a.values = reinterpret_cast<const uint8_t *>(values);
+  a.k_scales = quant ? reinterpret_cast<const __half *>(k_scales) : nullptr;
+  a.v_scales = quant ? reinterpret_cast<const __half *>(v_scales) : nullptr;
+  a.token_pos = token_pos;
+  a.y = y_out;
+  a.lse_out = lse_out;
+  a.lse2 = scratch;  // fully written by pass 1 before pass 2 reads it: no clearing needed
+  a.w = w_out;
+  a.wq = wq_out;
+  a.Hq = desc->n_q_heads;
+  a.Hk = desc->n_kv_heads;
+  a.q_g = desc->n_q_heads / desc->n_kv_heads;
+  a.d = desc->head_dim;
+  a.N_C = desc->capacity;
+  a.S = S;
+  a.P = (int)P;
+  a.row_bytes = kv_row_bytes(desc->kv_dtype, desc->head_dim);
+  a.scale2 = (float)(1.4426950408889634 / sqrt((double)desc->head_dim));
+  const size_t nw = (size_t)desc->batch * desc->n_kv_heads * desc->capacity * 4;
+  if (cudaMemsetAsync(w_out, 0, nw, st) != cudaSuccess ||
+      (wq_out && cudaMemsetAsync(wq_out, 0, nw * a.q_g, st) != cudaSuccess))
+    return set_error(H2OKV_ERR_CUDA, "cudaMemsetAsync of w_out/wq_out failed");
+  if (desc->q_dtype == H2OKV_F32) return run<H2OKV_F32, H2OKV_F32>(a, desc->batch, st);
+  switch (desc->kv_dtype) {
+    case H2OKV_BF16: return run<H2OKV_BF16, H2OKV_BF16>(a, desc->batch, st);
+    case H2OKV_I8: return run<H2OKV_BF16, H2OKV_I8>(a, desc->batch, st);
+    case H2OKV_I4: return run<H2OKV_BF16, H2OKV_I4>(a, desc->batch, st);
+  }
+  return set_error(H2OKV_ERR_UNSUPPORTED, "dtype combination");
+}

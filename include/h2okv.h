@@ -184,6 +184,37 @@ H2OKV_API int attn_chunk_with_scoresum(h2okv_cache *cache, const void *q, int32_
                              void *y_out, float *lse_out, float *w_out, float *wq_out,
                              void *stream);
 
+/* Allocation-free variant of attn_chunk_with_scoresum (the paper has no
+ * counterpart: it is an interface for callers that cannot allocate device
+ * memory).  Some callers own no device allocations of their own -- every byte
+ * they touch belongs to another allocator, such as a framework's caching pool
+ * or an inference engine's fixed arena -- so they cannot provide the per-cache
+ * workspace that kv_cache_create requires.  This call needs neither a handle
+ * nor a workspace: it takes the cache description and buffers directly and
+ * keeps its only scratch (one float32 log-sum-exp per query row) in a
+ * file-scope device array inside the library.  It computes what
+ * attn_chunk_with_scoresum computes, with the same arguments and layouts
+ * (keys/values/scales/token_pos as in h2okv_cache_buffers; q, y_out, lse_out,
+ * w_out, wq_out as in attn_chunk_with_scoresum), on the library's CUDA-core
+ * kernels.
+ *   - Limit: batch * n_q_heads * S <= 262144 rows; larger calls return
+ *     H2OKV_ERR_INVALID_ARG without enqueuing anything.
+ *   - The array (1 MiB) exists on every GPU that loads the library and is held
+ *     until the process exits.
+ *   - The first call on a device looks up the array's device address
+ *     (cudaGetSymbolAddress) with that device current; make that first call
+ *     before any stream capture.
+ *   - Every call on a device shares the one array and leaves the last call's
+ *     contents in it; calls whose work overlaps on the GPU (different streams,
+ *     no ordering between them) race on it and give undefined results.
+ *   - It calls no cudaMalloc, cudaFree or other allocating routine. */
+H2OKV_API int attn_chunk_with_scoresum_noalloc(const h2okv_cache_desc *desc, const void *keys,
+                                               const void *values, const void *k_scales,
+                                               const void *v_scales, const int32_t *token_pos,
+                                               const void *q, int32_t S, int64_t P, void *y_out,
+                                               float *lse_out, float *w_out, float *wq_out,
+                                               void *stream);
+
 /* Message of the last error on this thread ("" if none). */
 H2OKV_API const char *h2okv_last_error(void);
 
