@@ -46,6 +46,11 @@ constexpr int BM = 128;        // query rows per tile
 constexpr int BN = 128;        // slots per tile
 constexpr int D = 128;         // head dim
 constexpr int kThreads = 384;  // 4 control warps + 2 softmax warpgroups
+// Register split between the warpgroups.  The launch allots 168 registers per
+// thread (384 x 168 = 64512); the control warpgroup drops to 88 and the two
+// softmax warpgroups rise to 208: 128 x 88 + 256 x 208 = 64512.
+constexpr int kLaunchRegs = 168, kCtrlRegs = 88, kSoftRegs = 208;
+static_assert(128 * kCtrlRegs + 256 * kSoftRegs == kThreads * kLaunchRegs, "register split");
 constexpr uint32_t kTileBytes = BM * D * 2;  // 32 KiB (two 64-column swizzled halves)
 constexpr uint32_t kHalfBytes = kTileBytes / 2;
 
@@ -151,26 +156,25 @@ __device__ __forceinline__ void row_update(uint32_t (&x)[N], bool masked, const 
 // tile's 128 rows from S^T in TMEM, packed to bf16 pairs, column sum returned.
 __device__ __forceinline__ float slot_probs(uint32_t taddr, const float *lse, float c2, int rmin,
                                             int rmax, bool full, uint32_t (&pk)[BM / 2]) {
-  uint32_t r[32];
+  uint32_t r[BM];
+  tmem_ld32(taddr + 0, *reinterpret_cast<uint32_t(*)[32]>(r + 0));
+  tmem_ld32(taddr + 32, *reinterpret_cast<uint32_t(*)[32]>(r + 32));
+  tmem_ld32(taddr + 64, *reinterpret_cast<uint32_t(*)[32]>(r + 64));
+  tmem_ld32(taddr + 96, *reinterpret_cast<uint32_t(*)[32]>(r + 96));
+  tmem_wait_ld();
   float cs8[8];
 #pragma unroll
   for (int q = 0; q < 8; ++q) cs8[q] = 0.f;
 #pragma unroll
-  for (int c = 0; c < 4; ++c) {
-    tmem_ld32(taddr + c * 32, r);
-    tmem_wait_ld();
-#pragma unroll
-    for (int e = 0; e < 32; e += 2) {
-      const int r0 = c * 32 + e;
-      float p0 = ex2(fmaf(__uint_as_float(r[e]), c2, -lse[r0]));
-      float p1 = ex2(fmaf(__uint_as_float(r[e + 1]), c2, -lse[r0 + 1]));
-      if (!full) {
-        p0 = (r0 >= rmin && r0 < rmax) ? p0 : 0.f;
-        p1 = (r0 + 1 >= rmin && r0 + 1 < rmax) ? p1 : 0.f;
-      }
-      cs8[(e >> 1) & 7] += p0 + p1;
-      pk[r0 >> 1] = pack_bf16x2(p0, p1);
+  for (int e = 0; e < BM; e += 2) {
+    float p0 = ex2(fmaf(__uint_as_float(r[e]), c2, -lse[e]));
+    float p1 = ex2(fmaf(__uint_as_float(r[e + 1]), c2, -lse[e + 1]));
+    if (!full) {
+      p0 = (e >= rmin && e < rmax) ? p0 : 0.f;
+      p1 = (e + 1 >= rmin && e + 1 < rmax) ? p1 : 0.f;
     }
+    cs8[(e >> 1) & 7] += p0 + p1;
+    pk[e >> 1] = pack_bf16x2(p0, p1);
   }
   return ((cs8[0] + cs8[1]) + (cs8[2] + cs8[3])) + ((cs8[4] + cs8[5]) + (cs8[6] + cs8[7]));
 }
@@ -260,6 +264,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   const uint32_t tmem = *tmem_s;
   bool aborted = false;
 
+  if (warp < 4) {
+  reg_dealloc<kCtrlRegs>();
   if (warp == 0) {
     // ------------------------------------------------------------------ producer
     if (lane == 0) {
@@ -400,7 +406,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_wait(&bar[B_DRAIN], 0, 4000000000ull);
     }
     __syncwarp();
-  } else if (warp >= 4 && (warp < 8 || has_b)) {
+  }
+  } else {
+  reg_alloc<kSoftRegs>();
+  if (warp < 8 || has_b) {
     // -------------------------------------------- softmax / sums, one warpgroup per query tile
     const int wg = (warp - 4) >> 2;  // 0: tile a, 1: tile b
     const int st = threadIdx.x - 128 * (1 + wg);  // row (phase A) or slot (phase B) in the tile
@@ -409,7 +418,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int i0 = wg ? i0_b : i0_a, bhq = wg ? bhq_b : bhq_a, t = wg ? t_b : t_a;
     const int64_t row_lim = (int64_t)p.P + i0 + st;
     float m = -INFINITY, l = 0.f;
-    uint32_t x[64];
+    uint32_t x[BN];
     for (int kt = 0; kt < n_kt && !aborted; ++kt) {
       const int u = kt & 1, s = kt & 1;
       if (!warp_wait(&bar[B_SFULL0 + u], (kt >> 1) & 1, lim)) { fail(p, aborted); break; }
@@ -422,13 +431,11 @@ __global__ void __launch_bounds__(kThreads, 1)
       const uint32_t sa = tmem + lane_base + u * 256 + wg * 128;
       tmem_ld32(sa, *reinterpret_cast<uint32_t(*)[32]>(x));
       tmem_ld32(sa + 32, *reinterpret_cast<uint32_t(*)[32]>(x + 32));
-      tmem_wait_ld();
-      row_update<64>(x, masked, tp_s + s * BN, row_lim, c2, m, l);
-      tmem_ld32(sa + 64, *reinterpret_cast<uint32_t(*)[32]>(x));
-      tmem_ld32(sa + 96, *reinterpret_cast<uint32_t(*)[32]>(x + 32));
+      tmem_ld32(sa + 64, *reinterpret_cast<uint32_t(*)[32]>(x + 64));
+      tmem_ld32(sa + 96, *reinterpret_cast<uint32_t(*)[32]>(x + 96));
       tmem_wait_ld();
       tc_fence_before();
-      row_update<64>(x, masked, tp_s + s * BN + 64, row_lim, c2, m, l);
+      row_update<BN>(x, masked, tp_s + s * BN, row_lim, c2, m, l);
       __syncwarp();
       if (lane == 0) {
         mbar_arrive(&bar[B_SFREE0 + u]);
@@ -503,6 +510,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
     }
     tc_fence_before();
+  }
   }
   __syncthreads();
   if (warp == 1) {
@@ -605,6 +613,20 @@ int launch_attn_tc(h2okv_cache *c, const void *q, int S, int64_t P, void *y, flo
       return set_error(H2OKV_ERR_CUDA, "cudaFuncSetAttribute(attn_tc_kernel): %s",
                        cudaGetErrorString(e));
     configured_dev = dev;
+  }
+  static thread_local int checked_dev = -1;
+  if (checked_dev != dev) {
+    cudaFuncAttributes fa;
+    cudaError_t e = cudaFuncGetAttributes(&fa, attn_tc_kernel);
+    if (e != cudaSuccess)
+      return set_error(H2OKV_ERR_CUDA, "cudaFuncGetAttributes(attn_tc_kernel): %s",
+                       cudaGetErrorString(e));
+    // the in-kernel register split assumes exactly this launch allotment
+    if (fa.numRegs != kLaunchRegs)
+      return set_error(H2OKV_ERR_UNSUPPORTED,
+                       "attn_tc_kernel built with %d registers per thread, expected %d", fa.numRegs,
+                       kLaunchRegs);
+    checked_dev = dev;
   }
   TcParams prm;
   prm.token_pos = c->bufs.token_pos;
