@@ -124,6 +124,12 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   return *reinterpret_cast<uint32_t *>(&v);
 }
 
+// Exponentials: in every group of 8 consecutive elements the last kPolyA (phase A)
+// or kPolyB (phase B) go to the FMA-pipe polynomial exp2_poly2, the others to the
+// MUFU ex2 unit, so that neither unit alone bounds the softmax warps.
+constexpr int kPolyA = 4;
+constexpr int kPolyB = 2;
+
 // Online (max, sum) update of one row over N slots (base-2 units).
 template <int N>
 __device__ __forceinline__ void row_update(uint32_t (&x)[N], bool masked, const int32_t *tp,
@@ -142,19 +148,31 @@ __device__ __forceinline__ void row_update(uint32_t (&x)[N], bool masked, const 
                          fmaxf(fmaxf(mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7])));
   const float m_new = fmaxf(m, mx * c2);
   if (m_new == -INFINITY) return;
-  float sm8[8];
+  const float2 c2v = make_float2(c2, c2), negm = make_float2(-m_new, -m_new);
+  float2 acc[4];
 #pragma unroll
-  for (int q = 0; q < 8; ++q) sm8[q] = 0.f;
+  for (int q = 0; q < 4; ++q) acc[q] = make_float2(0.f, 0.f);
 #pragma unroll
-  for (int e = 0; e < N; ++e) sm8[e & 7] += ex2(fmaf(__uint_as_float(x[e]), c2, -m_new));
-  const float sum = ((sm8[0] + sm8[1]) + (sm8[2] + sm8[3])) + ((sm8[4] + sm8[5]) + (sm8[6] + sm8[7]));
-  l = l * ex2(m - m_new) + sum;
+  for (int e = 0; e < N; e += 2) {
+    const float2 a =
+        fma2(make_float2(__uint_as_float(x[e]), __uint_as_float(x[e + 1])), c2v, negm);
+    float2 v;
+    if ((e & 7) >= 8 - kPolyA)
+      v = exp2_poly2(a);
+    else
+      v = make_float2(ex2(a.x), ex2(a.y));
+    acc[(e >> 1) & 3] = add2(acc[(e >> 1) & 3], v);
+  }
+  const float2 s01 = add2(acc[0], acc[1]), s23 = add2(acc[2], acc[3]);
+  const float2 s4 = add2(s01, s23);
+  l = l * ex2(m - m_new) + (s4.x + s4.y);
   m = m_new;
 }
 
 // Phase B for one slot (this thread) and one query tile: normalised p over the
 // tile's 128 rows from S^T in TMEM, packed to bf16 pairs, column sum returned.
-__device__ __forceinline__ float slot_probs(uint32_t taddr, const float *lse, float c2, int rmin,
+// nlse holds -lse2 of the tile's rows.
+__device__ __forceinline__ float slot_probs(uint32_t taddr, const float *nlse, float c2, int rmin,
                                             int rmax, bool full, uint32_t (&pk)[BM / 2]) {
   uint32_t r[BM];
   tmem_ld32(taddr + 0, *reinterpret_cast<uint32_t(*)[32]>(r + 0));
@@ -162,21 +180,29 @@ __device__ __forceinline__ float slot_probs(uint32_t taddr, const float *lse, fl
   tmem_ld32(taddr + 64, *reinterpret_cast<uint32_t(*)[32]>(r + 64));
   tmem_ld32(taddr + 96, *reinterpret_cast<uint32_t(*)[32]>(r + 96));
   tmem_wait_ld();
-  float cs8[8];
+  const float2 c2v = make_float2(c2, c2);
+  float2 acc[4];
 #pragma unroll
-  for (int q = 0; q < 8; ++q) cs8[q] = 0.f;
+  for (int q = 0; q < 4; ++q) acc[q] = make_float2(0.f, 0.f);
 #pragma unroll
   for (int e = 0; e < BM; e += 2) {
-    float p0 = ex2(fmaf(__uint_as_float(r[e]), c2, -lse[e]));
-    float p1 = ex2(fmaf(__uint_as_float(r[e + 1]), c2, -lse[e + 1]));
+    const float2 nl = *reinterpret_cast<const float2 *>(nlse + e);
+    const float2 a = fma2(make_float2(__uint_as_float(r[e]), __uint_as_float(r[e + 1])), c2v, nl);
+    float2 v;
+    if ((e & 7) >= 8 - kPolyB)
+      v = exp2_poly2(a);
+    else
+      v = make_float2(ex2(a.x), ex2(a.y));
     if (!full) {
-      p0 = (e >= rmin && e < rmax) ? p0 : 0.f;
-      p1 = (e + 1 >= rmin && e + 1 < rmax) ? p1 : 0.f;
+      v.x = (e >= rmin && e < rmax) ? v.x : 0.f;
+      v.y = (e + 1 >= rmin && e + 1 < rmax) ? v.y : 0.f;
     }
-    cs8[(e >> 1) & 7] += p0 + p1;
-    pk[e >> 1] = pack_bf16x2(p0, p1);
+    acc[(e >> 1) & 3] = add2(acc[(e >> 1) & 3], v);
+    pk[e >> 1] = pack_bf16x2_int(v.x, v.y);
   }
-  return ((cs8[0] + cs8[1]) + (cs8[2] + cs8[3])) + ((cs8[4] + cs8[5]) + (cs8[6] + cs8[7]));
+  const float2 s01 = add2(acc[0], acc[1]), s23 = add2(acc[2], acc[3]);
+  const float2 s4 = add2(s01, s23);
+  return s4.x + s4.y;
 }
 
 // P[row][slot] as the MN-major A operand: slot = K index (a 128-byte row of an
@@ -445,8 +471,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     __syncwarp();
     if (lane == 0) mbar_arrive(&bar[B_AFREE]);
     const float lse2 = (l > 0.f) ? m + lg2(l) : -INFINITY;
-    float *lse_t = lse_s + wg * BM;
-    lse_t[st] = lse2;
+    float *lse_t = lse_s + wg * BM;  // holds -lse2 of the tile's rows
+    lse_t[st] = -lse2;
     if (p.lse_out && i0 + st < p.S)
       p.lse_out[(size_t)bhq * p.S + i0 + st] = lse2 * 0.69314718055994531f;
     named_bar_sync(1 + wg, 128);

@@ -178,3 +178,55 @@ __device__ __forceinline__ float lg2(float x) {
 
 }  // namespace ptx
 }  // namespace h2okv
+
+namespace h2okv {
+namespace ptx {
+
+// ---- packed float32 pairs (one instruction for two lanes' worth of math) -------------
+__device__ __forceinline__ uint64_t f2_bits(float2 v) {
+  return (uint64_t)__float_as_uint(v.x) | ((uint64_t)__float_as_uint(v.y) << 32);
+}
+__device__ __forceinline__ float2 bits_f2(uint64_t b) {
+  return make_float2(__uint_as_float((uint32_t)b), __uint_as_float((uint32_t)(b >> 32)));
+}
+__device__ __forceinline__ float2 fma2(float2 a, float2 b, float2 c) {
+  uint64_t d;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(f2_bits(a)), "l"(f2_bits(b)), "l"(f2_bits(c)));
+  return bits_f2(d);
+}
+__device__ __forceinline__ float2 add2(float2 a, float2 b) {
+  uint64_t d;
+  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(f2_bits(a)), "l"(f2_bits(b)));
+  return bits_f2(d);
+}
+
+// 2^x for a pair, on the FMA pipe: x = n + f with n = rint(x) (the 1.5 * 2^23
+// rounding constant), f in [-1/2, 1/2]; 2^f by a degree-4 polynomial (near-minimax
+// relative-error fit, exp2_poly_coeffs.py: max relative error 2.7e-6); 2^n by adding
+// n to the exponent field.  Inputs are clamped to [-126, +inf) so the exponent
+// never wraps; results below 2^-126 come out as tiny positives instead of 0.
+__device__ __forceinline__ float2 exp2_poly2(float2 x) {
+  x.x = fmaxf(x.x, -126.f);
+  x.y = fmaxf(x.y, -126.f);
+  const float2 magic = make_float2(12582912.f, 12582912.f);
+  const float2 t = add2(x, magic);
+  const float2 n = add2(t, make_float2(-12582912.f, -12582912.f));
+  const float2 f = fma2(n, make_float2(-1.f, -1.f), x);
+  float2 p = fma2(make_float2(0.009570101276040077f, 0.009570101276040077f), f,
+                  make_float2(0.05591786280274391f, 0.05591786280274391f));
+  p = fma2(p, f, make_float2(0.240247443318367f, 0.240247443318367f));
+  p = fma2(p, f, make_float2(0.6931217908859253f, 0.6931217908859253f));
+  p = fma2(p, f, make_float2(0.9999992847442627f, 0.9999992847442627f));
+  return make_float2(__uint_as_float(__float_as_uint(p.x) + (__float_as_uint(t.x) << 23)),
+                     __uint_as_float(__float_as_uint(p.y) + (__float_as_uint(t.y) << 23)));
+}
+
+// Two non-negative floats to packed bf16 (low half = lo), rounded to nearest with
+// ties away from zero, on the integer pipe.
+__device__ __forceinline__ uint32_t pack_bf16x2_int(float lo, float hi) {
+  const uint32_t a = __float_as_uint(lo) + 0x8000u, b = __float_as_uint(hi) + 0x8000u;
+  return __byte_perm(a, b, 0x7632);
+}
+
+}  // namespace ptx
+}  // namespace h2okv
