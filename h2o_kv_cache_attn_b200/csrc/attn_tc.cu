@@ -25,8 +25,9 @@
 // (tile a) and 8-11 (tile b) softmax / column sums / epilogue (warp w owns
 // TMEM lanes 32(w%4)..32(w%4)+31).  The single P buffer is handed over
 // a(kt) -> b(kt) -> a(kt+1) through per-tile full / free barriers.
-// The MMA issue order PV_a(kt), S^T_a(kt+1), PV_b(kt), S^T_b(kt+1) keeps the
-// tensor pipe busy while the softmax warps work on the other query tile.
+// The MMA issue order S^T_a(kt+1), S^T_b(kt+1), PV_a(kt), PV_b(kt) lets the tensor
+// pipe compute the next logits while the softmax warps turn the current ones
+// into P.
 // Every wait is bounded; a timeout sets the cache's device status word and the
 // CTA drains its copies and MMAs before freeing TMEM.
 //
@@ -127,8 +128,8 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
 // Exponentials: in every group of 8 consecutive elements the last kPolyA (phase A)
 // or kPolyB (phase B) go to the FMA-pipe polynomial exp2_poly2, the others to the
 // MUFU ex2 unit, so that neither unit alone bounds the softmax warps.
-constexpr int kPolyA = 4;
-constexpr int kPolyB = 2;
+constexpr int kPolyA = 0;
+constexpr int kPolyB = 0;
 
 // Online (max, sum) update of one row over N slots (base-2 units).
 template <int N>
@@ -418,13 +419,14 @@ __global__ void __launch_bounds__(kThreads, 1)
       };
       if (!aborted && !issue_st(0, false)) fail(p, aborted);
       if (!aborted && has_b && !issue_st(0, true)) fail(p, aborted);
+      // S^T of the next tile is issued as soon as the softmax warps have read the
+      // current one out of TMEM (long before their P is ready), then the P V
+      // products of the current tile.
       for (int kt = 0; kt < n_kt && !aborted; ++kt) {
-        if (!issue_pv(kt, false)) { fail(p, aborted); break; }
         if (kt + 1 < n_kt && !issue_st(kt + 1, false)) { fail(p, aborted); break; }
-        if (has_b) {
-          if (!issue_pv(kt, true)) { fail(p, aborted); break; }
-          if (kt + 1 < n_kt && !issue_st(kt + 1, true)) { fail(p, aborted); break; }
-        }
+        if (kt + 1 < n_kt && has_b && !issue_st(kt + 1, true)) { fail(p, aborted); break; }
+        if (!issue_pv(kt, false)) { fail(p, aborted); break; }
+        if (has_b && !issue_pv(kt, true)) { fail(p, aborted); break; }
       }
       mma_commit(&bar[B_OFULL]);
       // drain: every MMA issued by this thread completes before TMEM is freed
