@@ -49,33 +49,19 @@ def peaks():
 
 
 # --------------------------------------------------------------------------- #
-def dist_init():
-    ws = int(os.environ.get("WORLD_SIZE", "1"))
-    rank = int(os.environ.get("RANK", "0"))
-    local = int(os.environ.get("LOCAL_RANK", "0"))
-    if ws > 1:
-        import datetime
+from h2o_kv_cache_attn_b200 import dist as hdist  # noqa: E402
 
-        import torch.distributed as dist
-        torch.cuda.set_device(local)
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
-                                device_id=torch.device("cuda", local))
-    return ws, rank, local
+
+def dist_init():
+    return hdist.init("nccl")
 
 
 def barrier(ws):
-    if ws > 1:
-        import torch.distributed as dist
-        dist.barrier()
+    hdist.barrier()
 
 
 def max_over_ranks(x, ws):
-    if ws == 1:
-        return x
-    import torch.distributed as dist
-    t = torch.tensor([x], dtype=torch.float64, device="cuda")
-    dist.all_reduce(t, op=dist.ReduceOp.MAX)
-    return float(t.item())
+    return hdist.max_over_ranks(x)
 
 
 class ClockSampler:
@@ -434,9 +420,7 @@ def main():
                 "roofline": res["roof"], "cpu_baseline": cpu, "e2e": res["e2e"],
                 "gpu_launches": res["launches"], "clocks": res["clocks"], **res["extra"]}
         print(json.dumps(line))
-    if ws > 1:
-        import torch.distributed as dist
-        dist.destroy_process_group()
+    hdist.shutdown()
     return 0
 
 

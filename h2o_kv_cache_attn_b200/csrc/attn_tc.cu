@@ -19,9 +19,10 @@
 //            O += P V (A = P, B = V, both MN-major).  P is normalised already,
 //            so O needs no rescaling.  TMEM: S^T_a, S^T_b, O_a, O_b.
 //
-// Warp roles (384 threads): warp 0 TMA producer (K and V tiles through separate
-// two-stage rings via cp.async.bulk.tensor, no multicast; token positions by
-// plain loads), warp 1 TMEM allocator and single-thread MMA issuer, warps 4-7
+// Warp roles (384 threads): warp 0 loads Q, K tiles (cp.async.bulk.tensor, no
+// multicast) and token positions (1-D bulk copy) through a two-stage ring, warp 2
+// loads V tiles through its own two-stage ring, warp 1 allocates TMEM and issues
+// every MMA from one thread, warps 4-7
 // (tile a) and 8-11 (tile b) softmax / column sums / epilogue (warp w owns
 // TMEM lanes 32(w%4)..32(w%4)+31).  The single P buffer is handed over
 // a(kt) -> b(kt) -> a(kt+1) through per-tile full / free barriers.
@@ -47,6 +48,7 @@ constexpr int BM = 128;        // query rows per tile
 constexpr int BN = 128;        // slots per tile
 constexpr int D = 128;         // head dim
 constexpr int kThreads = 384;  // 4 control warps + 2 softmax warpgroups
+constexpr int kPrefetch = 4;   // K / V tiles requested into L2 this many loads ahead
 // Register split between the warpgroups.  The launch allots 168 registers per
 // thread (384 x 168 = 64512); the control warpgroup drops to 88 and the two
 // softmax warpgroups rise to 208: 128 x 88 + 256 x 208 = 64512.
@@ -82,6 +84,7 @@ struct TcParams {
   float *part_w;             // [B*Hq*tiles][N_C]
   int *status;               // device status word (0 = ok)
   int Hq, Hk, q_g, N_C, S, P, tiles, n_kt, ctas_per_group;
+  int tp_bulk;  // token positions by 1-D bulk copy (N_C % 4 == 0: 16-byte aligned rows)
   float scale2;  // log2(e) / sqrt(d)
   unsigned long long timeout_ns;
 };
@@ -133,13 +136,14 @@ constexpr int kPolyB = 0;
 
 // Online (max, sum) update of one row over N slots (base-2 units).
 template <int N>
-__device__ __forceinline__ void row_update(uint32_t (&x)[N], bool masked, const int32_t *tp,
-                                           int64_t row_lim, float c2, float &m, float &l) {
-  if (masked) {
+__device__ __forceinline__ void row_mask(uint32_t (&x)[N], const int32_t *tp, int64_t row_lim) {
 #pragma unroll
-    for (int e = 0; e < N; ++e)
-      if ((int64_t)tp[e] > row_lim) x[e] = __float_as_uint(-INFINITY);
-  }
+  for (int e = 0; e < N; ++e)
+    if ((int64_t)tp[e] > row_lim) x[e] = __float_as_uint(-INFINITY);
+}
+
+template <int N>
+__device__ __forceinline__ void row_update(const uint32_t (&x)[N], float c2, float &m, float &l) {
   float mx8[8];
 #pragma unroll
   for (int q = 0; q < 8; ++q) mx8[q] = __uint_as_float(x[q]);
@@ -173,14 +177,16 @@ __device__ __forceinline__ void row_update(uint32_t (&x)[N], bool masked, const 
 // Phase B for one slot (this thread) and one query tile: normalised p over the
 // tile's 128 rows from S^T in TMEM, packed to bf16 pairs, column sum returned.
 // nlse holds -lse2 of the tile's rows.
-__device__ __forceinline__ float slot_probs(uint32_t taddr, const float *nlse, float c2, int rmin,
-                                            int rmax, bool full, uint32_t (&pk)[BM / 2]) {
-  uint32_t r[BM];
+__device__ __forceinline__ void tmem_ld128(uint32_t taddr, uint32_t (&r)[BM]) {
   tmem_ld32(taddr + 0, *reinterpret_cast<uint32_t(*)[32]>(r + 0));
   tmem_ld32(taddr + 32, *reinterpret_cast<uint32_t(*)[32]>(r + 32));
   tmem_ld32(taddr + 64, *reinterpret_cast<uint32_t(*)[32]>(r + 64));
   tmem_ld32(taddr + 96, *reinterpret_cast<uint32_t(*)[32]>(r + 96));
   tmem_wait_ld();
+}
+
+__device__ __forceinline__ float slot_probs(const uint32_t (&r)[BM], const float *nlse, float c2,
+                                            int rmin, int rmax, bool full, uint32_t (&pk)[BM / 2]) {
   const float2 c2v = make_float2(c2, c2);
   float2 acc[4];
 #pragma unroll
@@ -294,7 +300,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (warp < 4) {
   reg_dealloc<kCtrlRegs>();
   if (warp == 0) {
-    // ------------------------------------------------------------------ producer
+    // ------------------------------------------------- producer of Q, K and token positions
     if (lane == 0) {
       mbar_expect_tx(&bar[B_Q], has_b ? 2 * kTileBytes : kTileBytes);
       tma_load_3d(smem + OFF_QA, &q_map, &bar[B_Q], 0, i0_a, bhq_a);
@@ -306,54 +312,71 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_arrive(&bar[B_Q]);
     }
     const int32_t *tpg = p.token_pos + (size_t)bg * p.N_C;
-    int k_issued = 0, v_issued = 0;
+    int k_issued = 0;
     for (int it = 0; it < 2 * n_kt && !aborted; ++it) {
-      const bool phB = it >= n_kt;
-      const int kt = phB ? it - n_kt : it;
+      const int kt = it >= n_kt ? it - n_kt : it;
       const int s = it & 1, n = it >> 1;
-      // K tile + token positions
       if (n > 0 && !warp_wait(&bar[B_KEMPTY0 + s], (n - 1) & 1, lim)) {
         fail(p, aborted);
         break;
       }
       uint8_t *kdst = smem + (s ? OFF_K1 : OFF_K0);
+      int32_t *tdst = tp_s + s * BN;
+      const int nv = min(BN, p.N_C - kt * BN);  // slots of this tile inside the cache
       if (lane == 0) {
-        mbar_expect_tx(&bar[B_KFULL0 + s], kTileBytes);
+        mbar_expect_tx(&bar[B_KFULL0 + s], kTileBytes + (p.tp_bulk ? nv * 4 : 0));
         tma_load_3d(kdst, &k_map, &bar[B_KFULL0 + s], 0, kt * BN, bg);
         tma_load_3d(kdst + kHalfBytes, &k_map, &bar[B_KFULL0 + s], 64, kt * BN, bg);
+        if (p.tp_bulk) bulk_load(tdst, tpg + kt * BN, nv * 4, &bar[B_KFULL0 + s]);
+        // bring the K tiles kPrefetch loads ahead into L2 (the ring holds only two)
+        const int ahead = it + kPrefetch;
+        if (ahead < 2 * n_kt) {
+          const int kta = ahead >= n_kt ? ahead - n_kt : ahead;
+          tma_prefetch_l2_3d(&k_map, 0, kta * BN, bg);
+          tma_prefetch_l2_3d(&k_map, 64, kta * BN, bg);
+        }
       }
+      if (p.tp_bulk) {
+        for (int e = nv + lane; e < BN; e += 32) tdst[e] = kEmptyPos;
+      } else {
 #pragma unroll
-      for (int e = lane; e < BN; e += 32) {
-        const int j = kt * BN + e;
-        tp_s[s * BN + e] = j < p.N_C ? tpg[j] : kEmptyPos;
+        for (int e = lane; e < BN; e += 32) tdst[e] = e < nv ? tpg[kt * BN + e] : kEmptyPos;
       }
       __syncwarp();
       if (lane == 0) mbar_arrive(&bar[B_KFULL0 + s]);
       k_issued = it + 1;
-      if (phB) {  // V tile, ring indexed by kt
-        const int vs = kt & 1, vn = kt >> 1;
-        if (vn > 0 && !warp_wait(&bar[B_VEMPTY0 + vs], (vn - 1) & 1, lim)) {
-          fail(p, aborted);
-          break;
-        }
-        uint8_t *vdst = smem + (vs ? OFF_V1 : OFF_V0);
-        if (lane == 0) {
-          mbar_expect_tx(&bar[B_VFULL0 + vs], kTileBytes);
-          tma_load_3d(vdst, &v_map, &bar[B_VFULL0 + vs], 0, kt * BN, bg);
-          tma_load_3d(vdst + kHalfBytes, &v_map, &bar[B_VFULL0 + vs], 64, kt * BN, bg);
-          mbar_arrive(&bar[B_VFULL0 + vs]);
-        }
-        v_issued = kt + 1;
-      }
     }
     // drain: the last issued loads must land before exit
     if (lane == 0) {
       mbar_wait(&bar[B_Q], 0, 4000000000ull);
       for (int it = k_issued - 1; it >= 0 && it >= k_issued - 2; --it)
         mbar_wait(&bar[B_KFULL0 + (it & 1)], (it >> 1) & 1, 4000000000ull);
+    }
+  } else if (warp == 2) {
+    // ------------------------------------------------------------------ producer of V
+    if (lane == 0) {
+      int v_issued = 0;
+      for (int kt = 0; kt < n_kt && !aborted; ++kt) {
+        const int vs = kt & 1, vn = kt >> 1;
+        if (vn > 0 && !mbar_wait(&bar[B_VEMPTY0 + vs], (vn - 1) & 1, lim)) {
+          fail(p, aborted);
+          break;
+        }
+        uint8_t *vdst = smem + (vs ? OFF_V1 : OFF_V0);
+        mbar_expect_tx(&bar[B_VFULL0 + vs], kTileBytes);
+        tma_load_3d(vdst, &v_map, &bar[B_VFULL0 + vs], 0, kt * BN, bg);
+        tma_load_3d(vdst + kHalfBytes, &v_map, &bar[B_VFULL0 + vs], 64, kt * BN, bg);
+        mbar_arrive(&bar[B_VFULL0 + vs]);
+        if (kt + kPrefetch < n_kt) {
+          tma_prefetch_l2_3d(&v_map, 0, (kt + kPrefetch) * BN, bg);
+          tma_prefetch_l2_3d(&v_map, 64, (kt + kPrefetch) * BN, bg);
+        }
+        v_issued = kt + 1;
+      }
       for (int kt = v_issued - 1; kt >= 0 && kt >= v_issued - 2; --kt)
         mbar_wait(&bar[B_VFULL0 + (kt & 1)], (kt >> 1) & 1, 4000000000ull);
     }
+    __syncwarp();
   } else if (warp == 1) {
     // ------------------------------------------------------------------ MMA issuer
     if (lane == 0) {
@@ -462,13 +485,15 @@ __global__ void __launch_bounds__(kThreads, 1)
       tmem_ld32(sa + 64, *reinterpret_cast<uint32_t(*)[32]>(x + 64));
       tmem_ld32(sa + 96, *reinterpret_cast<uint32_t(*)[32]>(x + 96));
       tmem_wait_ld();
+      if (masked) row_mask<BN>(x, tp_s + s * BN, row_lim);
+      // S buffer and K stage (with its token positions) are free once read
       tc_fence_before();
-      row_update<BN>(x, masked, tp_s + s * BN, row_lim, c2, m, l);
       __syncwarp();
       if (lane == 0) {
         mbar_arrive(&bar[B_SFREE0 + u]);
         mbar_arrive(&bar[B_KEMPTY0 + s]);
       }
+      row_update<BN>(x, c2, m, l);
     }
     __syncwarp();
     if (lane == 0) mbar_arrive(&bar[B_AFREE]);
@@ -497,10 +522,13 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int64_t rm = tpj - (int64_t)p.P - i0;
       const int rmin = rm <= 0 ? 0 : (rm >= BM ? BM : (int)rm);
       const bool full = __all_sync(0xffffffffu, rmin == 0 && rmax == BM);
-      const float cs = slot_probs(tmem + lane_base + wg * 128, lse_t, c2, rmin, rmax, full, pk);
+      uint32_t r[BM];
+      tmem_ld128(tmem + lane_base + wg * 128, r);
+      // S^T buffer is free once read: the next tile's logits can be computed meanwhile
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&bar[wg ? B_TFREEB : B_TFREEA]);
+      const float cs = slot_probs(r, lse_t, c2, rmin, rmax, full, pk);
       // the single P buffer goes a(kt) -> b(kt) -> a(kt+1): wait for the previous reader
       bool ok = true;
       if (wg == 1)
@@ -671,6 +699,7 @@ int launch_attn_tc(h2okv_cache *c, const void *q, int S, int64_t P, void *y, flo
   prm.tiles = (S + BM - 1) / BM;
   prm.n_kt = (d.capacity + BN - 1) / BN;
   prm.ctas_per_group = (prm.q_g * prm.tiles + 1) / 2;
+  prm.tp_bulk = (d.capacity % 4 == 0) ? 1 : 0;
   prm.scale2 = (float)(1.4426950408889634 / 11.313708498984761);  // log2(e) / sqrt(128)
   prm.timeout_ns = c->wait_timeout_ns;
   const int grid = d.batch * d.n_kv_heads * prm.ctas_per_group;
