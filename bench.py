@@ -241,9 +241,9 @@ def run_ours(args, wl, ws, rank, local):
     evict_gbs = evict_bytes_chunk(wl, wl.chunk) / (evict_us * 1e-6) / 1e9 if evict_us else None
     # the tensor-core path serves head_dim 128 with a bf16 cache (same rule as the library)
     tc_used = wl.d == 128 and wl.kv_dtype == "bf16" and wl.q_dtype == "bf16"
-    # per chunk: select + scatter, then two attention launches (tc: attention + reduction;
-    # CUDA-core path: two passes); plus the final fold and the reset per step
-    launches_per_step = wl.n_chunks * 4 + 2
+    # per chunk: one eviction launch, then two attention launches (tensor-core path:
+    # attention + reduction; CUDA-core path: two passes); plus the reset and the final fold
+    launches_per_step = wl.n_chunks * 3 + 2
     per_launch_alg = at_flops_alg / len(at_ms)
     per_launch_ms = sum(at_ms) / len(at_ms)
     if tc_used:

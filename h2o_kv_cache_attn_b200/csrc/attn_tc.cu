@@ -19,8 +19,10 @@
 //            O += P V (A = P, B = V, both MN-major).  P is normalised already,
 //            so O needs no rescaling.  TMEM: S^T_a, S^T_b, O_a, O_b.
 //
-// Warp roles (384 threads): warp 0 loads Q, K tiles (cp.async.bulk.tensor, no
-// multicast) and token positions (1-D bulk copy) through a two-stage ring, warp 2
+// Warp roles (384 threads): warp 0 loads Q and K tiles (cp.async.bulk.tensor, no
+// multicast) and turns the slots' token positions into positions relative to the
+// chunk (floats, for arithmetic masking) through a four-stage (phase A) and a
+// two-stage (phase B) ring, warp 2
 // loads V tiles through its own two-stage ring, warp 1 allocates TMEM and issues
 // every MMA from one thread, warps 4-7
 // (tile a) and 8-11 (tile b) softmax / column sums / epilogue (warp w owns
@@ -49,6 +51,8 @@ constexpr int BN = 128;        // slots per tile
 constexpr int D = 128;         // head dim
 constexpr int kThreads = 384;  // 4 control warps + 2 softmax warpgroups
 constexpr int kPrefetch = 4;   // K / V tiles requested into L2 this many loads ahead
+constexpr int kRelFar = 1 << 20;  // relative position of a slot no row of the chunk sees
+constexpr float kMaskBias = 1073741824.f;  // 2^30: subtracted from a masked logit
 // Register split between the warpgroups.  The launch allots 168 registers per
 // thread (384 x 168 = 64512); the control warpgroup drops to 88 and the two
 // softmax warpgroups rise to 208: 128 x 88 + 256 x 208 = 64512.
@@ -68,10 +72,21 @@ constexpr uint32_t OFF_P = OFF_V1 + kTileBytes;
 constexpr uint32_t OFF_TP = OFF_P + kTileBytes;        // int32 [2 stages][BN]
 constexpr uint32_t OFF_LSE = OFF_TP + 2 * BN * 4;      // float [2 tiles][BM]
 constexpr uint32_t OFF_BAR = OFF_LSE + 2 * BM * 4;     // uint64 barriers
-constexpr int NBAR = 24;
+constexpr int kStagesA = 4;  // phase A K ring: slots K0, K1, V0, V1 (V is unused in phase A)
+constexpr int NBAR = 25 + 2 * kStagesA;
 constexpr uint32_t OFF_TMEM = OFF_BAR + NBAR * 8;
 constexpr uint32_t kSmemBytes = OFF_TMEM + 16;
 static_assert(kSmemBytes <= 232448, "shared memory budget");
+
+// phase A stage -> slot; phase A token positions live in the P region (unused in phase A)
+__host__ __device__ constexpr uint32_t slot_a(int a) {
+  return a == 0 ? OFF_K0 : a == 1 ? OFF_K1 : a == 2 ? OFF_V0 : OFF_V1;
+}
+// last phase A tile that used stage a (or -1): the slot is free once that use is released
+__device__ __forceinline__ int last_use_a(int a, int n_kt) {
+  if (a >= n_kt) return -1;
+  return a + ((n_kt - 1 - a) / kStagesA) * kStagesA;
+}
 
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t IDESC_K_MAJOR = idesc_bf16_f32(128, 128, false, false);
@@ -84,20 +99,21 @@ struct TcParams {
   float *part_w;             // [B*Hq*tiles][N_C]
   int *status;               // device status word (0 = ok)
   int Hq, Hk, q_g, N_C, S, P, tiles, n_kt, ctas_per_group;
-  int tp_bulk;  // token positions by 1-D bulk copy (N_C % 4 == 0: 16-byte aligned rows)
   float scale2;  // log2(e) / sqrt(d)
   unsigned long long timeout_ns;
 };
 
 enum {
   B_Q = 0,
-  B_KFULL0, B_KFULL1, B_KEMPTY0, B_KEMPTY1,  // K ring (+ token positions)
+  B_KFULL0, B_KFULL1, B_KEMPTY0, B_KEMPTY1,  // phase B K ring (+ token positions)
   B_VFULL0, B_VFULL1, B_VEMPTY0, B_VEMPTY1,  // V ring (phase B)
   B_SFULL0, B_SFULL1, B_SFREE0, B_SFREE1,    // phase A S pair per tile parity
   B_AFREE,                                   // phase A TMEM fully read
   B_TFULLA, B_TFULLB, B_TFREEA, B_TFREEB,    // phase B S^T per query tile
   B_PFULLA, B_PFULLB, B_PFREEA, B_PFREEB,    // P buffer, handed a(kt) -> b(kt) -> a(kt+1)
-  B_OFULL, B_DRAIN                           // O complete; MMA drain before TMEM is freed
+  B_OFULL, B_DRAIN,                          // O complete; MMA drain before TMEM is freed
+  B_VGO,                                     // every phase A MMA done: V may use slots V0 / V1
+  B_AFULL0, B_AEMPTY0 = B_AFULL0 + kStagesA  // phase A K ring (+ token positions)
 };
 
 // K-major SW128 operand (rows x 128 columns as two 64-column halves): k-step ks
@@ -135,22 +151,36 @@ constexpr int kPolyA = 0;
 constexpr int kPolyB = 0;
 
 // Online (max, sum) update of one row over N slots (base-2 units).
+// Masked logits (slot relative position rel_e > row index ri) drop by 2^30:
+// nm = sat(rel_e - ri) is 1 for a masked slot, 0 for a visible one.
 template <int N>
-__device__ __forceinline__ void row_mask(uint32_t (&x)[N], const int32_t *tp, int64_t row_lim) {
+__device__ __forceinline__ void row_mask(uint32_t (&x)[N], const float *rel, float ri) {
 #pragma unroll
-  for (int e = 0; e < N; ++e)
-    if ((int64_t)tp[e] > row_lim) x[e] = __float_as_uint(-INFINITY);
+  for (int e = 0; e < N; e += 4) {
+    const float4 r4 = *reinterpret_cast<const float4 *>(rel + e);
+    const float rr[4] = {r4.x, r4.y, r4.z, r4.w};
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      const float nm = fma_sat(rr[q], 1.f, -ri);
+      x[e + q] = __float_as_uint(fmaf(nm, -kMaskBias, __uint_as_float(x[e + q])));
+    }
+  }
 }
 
 template <int N>
 __device__ __forceinline__ void row_update(const uint32_t (&x)[N], float c2, float &m, float &l) {
-  float mx8[8];
+  static_assert(N % 16 == 0, "row width");
+  float mx8[8];  // eight independent chains of three-input maxima
 #pragma unroll
-  for (int q = 0; q < 8; ++q) mx8[q] = __uint_as_float(x[q]);
+  for (int q = 0; q < 8; ++q) mx8[q] = fmaxf(__uint_as_float(x[q]), __uint_as_float(x[q + 8]));
 #pragma unroll
-  for (int e = 8; e < N; ++e) mx8[e & 7] = fmaxf(mx8[e & 7], __uint_as_float(x[e]));
-  const float mx = fmaxf(fmaxf(fmaxf(mx8[0], mx8[1]), fmaxf(mx8[2], mx8[3])),
-                         fmaxf(fmaxf(mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7])));
+  for (int e = 16; e < N; e += 16) {
+#pragma unroll
+    for (int q = 0; q < 8; ++q)
+      mx8[q] = fmax3(mx8[q], __uint_as_float(x[e + q]), __uint_as_float(x[e + 8 + q]));
+  }
+  const float mx = fmax3(fmax3(mx8[0], mx8[1], mx8[2]), fmax3(mx8[3], mx8[4], mx8[5]),
+                         fmaxf(mx8[6], mx8[7]));
   const float m_new = fmaxf(m, mx * c2);
   if (m_new == -INFINITY) return;
   const float2 c2v = make_float2(c2, c2), negm = make_float2(-m_new, -m_new);
@@ -187,6 +217,7 @@ __device__ __forceinline__ void tmem_ld128(uint32_t taddr, uint32_t (&r)[BM]) {
 
 __device__ __forceinline__ float slot_probs(const uint32_t (&r)[BM], const float *nlse, float c2,
                                             int rmin, int rmax, bool full, uint32_t (&pk)[BM / 2]) {
+  const float rminf = (float)rmin;
   const float2 c2v = make_float2(c2, c2);
   float2 acc[4];
 #pragma unroll
@@ -194,18 +225,22 @@ __device__ __forceinline__ float slot_probs(const uint32_t (&r)[BM], const float
 #pragma unroll
   for (int e = 0; e < BM; e += 2) {
     const float2 nl = *reinterpret_cast<const float2 *>(nlse + e);
-    const float2 a = fma2(make_float2(__uint_as_float(r[e]), __uint_as_float(r[e + 1])), c2v, nl);
+    float2 a = fma2(make_float2(__uint_as_float(r[e]), __uint_as_float(r[e + 1])), c2v, nl);
+    if (!full) {  // rows before rmin are masked: nm = sat(rmin - row) is 1 there
+      const float2 nm = make_float2(fma_sat(rminf, 1.f, -(float)e), fma_sat(rminf, 1.f, -(float)(e + 1)));
+      a = fma2(nm, make_float2(-kMaskBias, -kMaskBias), a);
+    }
     float2 v;
     if ((e & 7) >= 8 - kPolyB)
       v = exp2_poly2(a);
     else
       v = make_float2(ex2(a.x), ex2(a.y));
-    if (!full) {
-      v.x = (e >= rmin && e < rmax) ? v.x : 0.f;
-      v.y = (e + 1 >= rmin && e + 1 < rmax) ? v.y : 0.f;
+    if (rmax < BM) {  // rows past the chunk (last row tile only)
+      v.x = e < rmax ? v.x : 0.f;
+      v.y = e + 1 < rmax ? v.y : 0.f;
     }
     acc[(e >> 1) & 3] = add2(acc[(e >> 1) & 3], v);
-    pk[e >> 1] = pack_bf16x2_int(v.x, v.y);
+    pk[e >> 1] = pack_bf16x2(v.x, v.y);
   }
   const float2 s01 = add2(acc[0], acc[1]), s23 = add2(acc[2], acc[3]);
   const float2 s4 = add2(s01, s23);
@@ -280,6 +315,11 @@ __global__ void __launch_bounds__(kThreads, 1)
     mbar_init(&bar[B_PFREEB], 1);
     mbar_init(&bar[B_OFULL], 1);
     mbar_init(&bar[B_DRAIN], 1);
+    mbar_init(&bar[B_VGO], 1);
+    for (int i = 0; i < kStagesA; ++i) {
+      mbar_init(&bar[B_AFULL0 + i], 1);
+      mbar_init(&bar[B_AEMPTY0 + i], 1 + 4 * nwg);
+    }
     fence_mbar_init();
   }
   if (warp == 1) {
@@ -312,23 +352,41 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_arrive(&bar[B_Q]);
     }
     const int32_t *tpg = p.token_pos + (size_t)bg * p.N_C;
-    int k_issued = 0;
+    int issued_a = 0, issued_b = 0;
     for (int it = 0; it < 2 * n_kt && !aborted; ++it) {
-      const int kt = it >= n_kt ? it - n_kt : it;
-      const int s = it & 1, n = it >> 1;
-      if (n > 0 && !warp_wait(&bar[B_KEMPTY0 + s], (n - 1) & 1, lim)) {
-        fail(p, aborted);
-        break;
+      const bool phB = it >= n_kt;
+      const int kt = phB ? it - n_kt : it;
+      int stage;
+      uint64_t *full;
+      uint8_t *kdst;
+      int32_t *tdst;
+      if (!phB) {  // phase A: four stages
+        stage = kt % kStagesA;
+        const int n = kt / kStagesA;
+        if (n > 0 && !warp_wait(&bar[B_AEMPTY0 + stage], (n - 1) & 1, lim)) { fail(p, aborted); break; }
+        full = &bar[B_AFULL0 + stage];
+        kdst = smem + slot_a(stage);
+        tdst = reinterpret_cast<int32_t *>(smem + OFF_P) + stage * BN;
+      } else {  // phase B: slots K0 / K1 after their last phase A use
+        stage = kt & 1;
+        bool ok;
+        if (kt < 2) {
+          const int lu = last_use_a(stage, n_kt);
+          ok = lu < 0 || warp_wait(&bar[B_AEMPTY0 + stage], (lu / kStagesA) & 1, lim);
+        } else {
+          ok = warp_wait(&bar[B_KEMPTY0 + stage], ((kt >> 1) - 1) & 1, lim);
+        }
+        if (!ok) { fail(p, aborted); break; }
+        full = &bar[B_KFULL0 + stage];
+        kdst = smem + (stage ? OFF_K1 : OFF_K0);
+        tdst = tp_s + stage * BN;
       }
-      uint8_t *kdst = smem + (s ? OFF_K1 : OFF_K0);
-      int32_t *tdst = tp_s + s * BN;
       const int nv = min(BN, p.N_C - kt * BN);  // slots of this tile inside the cache
       if (lane == 0) {
-        mbar_expect_tx(&bar[B_KFULL0 + s], kTileBytes + (p.tp_bulk ? nv * 4 : 0));
-        tma_load_3d(kdst, &k_map, &bar[B_KFULL0 + s], 0, kt * BN, bg);
-        tma_load_3d(kdst + kHalfBytes, &k_map, &bar[B_KFULL0 + s], 64, kt * BN, bg);
-        if (p.tp_bulk) bulk_load(tdst, tpg + kt * BN, nv * 4, &bar[B_KFULL0 + s]);
-        // bring the K tiles kPrefetch loads ahead into L2 (the ring holds only two)
+        mbar_expect_tx(full, kTileBytes);
+        tma_load_3d(kdst, &k_map, full, 0, kt * BN, bg);
+        tma_load_3d(kdst + kHalfBytes, &k_map, full, 64, kt * BN, bg);
+        // bring the K tiles kPrefetch loads ahead into L2
         const int ahead = it + kPrefetch;
         if (ahead < 2 * n_kt) {
           const int kta = ahead >= n_kt ? ahead - n_kt : ahead;
@@ -336,21 +394,25 @@ __global__ void __launch_bounds__(kThreads, 1)
           tma_prefetch_l2_3d(&k_map, 64, kta * BN, bg);
         }
       }
-      if (p.tp_bulk) {
-        for (int e = nv + lane; e < BN; e += 32) tdst[e] = kEmptyPos;
-      } else {
+      // position of each slot's token relative to the chunk start, as a float:
+      // row i of the chunk sees the slot iff rel <= i (empty / outside slots: 2^20)
 #pragma unroll
-        for (int e = lane; e < BN; e += 32) tdst[e] = e < nv ? tpg[kt * BN + e] : kEmptyPos;
+      for (int e = lane; e < BN; e += 32) {
+        const int64_t t = e < nv ? (int64_t)tpg[kt * BN + e] : (int64_t)kEmptyPos;
+        const int64_t rel = t - (int64_t)p.P;
+        tdst[e] = __float_as_int((float)(rel < -1 ? -1 : (rel > kRelFar ? kRelFar : rel)));
       }
       __syncwarp();
-      if (lane == 0) mbar_arrive(&bar[B_KFULL0 + s]);
-      k_issued = it + 1;
+      if (lane == 0) mbar_arrive(full);
+      if (phB) issued_b = kt + 1; else issued_a = kt + 1;
     }
-    // drain: the last issued loads must land before exit
+    // drain: the last issued loads of both rings must land before exit
     if (lane == 0) {
       mbar_wait(&bar[B_Q], 0, 4000000000ull);
-      for (int it = k_issued - 1; it >= 0 && it >= k_issued - 2; --it)
-        mbar_wait(&bar[B_KFULL0 + (it & 1)], (it >> 1) & 1, 4000000000ull);
+      for (int kt = issued_a - 1; kt >= 0 && kt >= issued_a - kStagesA; --kt)
+        mbar_wait(&bar[B_AFULL0 + kt % kStagesA], (kt / kStagesA) & 1, 4000000000ull);
+      for (int kt = issued_b - 1; kt >= 0 && kt >= issued_b - 2; --kt)
+        mbar_wait(&bar[B_KFULL0 + (kt & 1)], (kt >> 1) & 1, 4000000000ull);
     }
   } else if (warp == 2) {
     // ------------------------------------------------------------------ producer of V
@@ -358,7 +420,13 @@ __global__ void __launch_bounds__(kThreads, 1)
       int v_issued = 0;
       for (int kt = 0; kt < n_kt && !aborted; ++kt) {
         const int vs = kt & 1, vn = kt >> 1;
-        if (vn > 0 && !mbar_wait(&bar[B_VEMPTY0 + vs], (vn - 1) & 1, lim)) {
+        bool ok;
+        if (vn == 0) {  // slots V0 / V1 serve as phase A K stages 2 / 3 until every phase A MMA is done
+          ok = mbar_wait(&bar[B_VGO], 0, lim);
+        } else {
+          ok = mbar_wait(&bar[B_VEMPTY0 + vs], (vn - 1) & 1, lim);
+        }
+        if (!ok) {
           fail(p, aborted);
           break;
         }
@@ -385,14 +453,14 @@ __global__ void __launch_bounds__(kThreads, 1)
       tc_fence_after();
       // phase A: S_a, S_b = Q_a K^T, Q_b K^T into the column pair of the tile parity
       for (int kt = 0; kt < n_kt && !aborted; ++kt) {
-        const int s = kt & 1, u = kt & 1;
-        if (!mbar_wait(&bar[B_KFULL0 + s], (kt >> 1) & 1, lim)) { fail(p, aborted); break; }
+        const int a = kt % kStagesA, u = kt & 1;
+        if (!mbar_wait(&bar[B_AFULL0 + a], (kt / kStagesA) & 1, lim)) { fail(p, aborted); break; }
         if (kt >= 2 && !mbar_wait(&bar[B_SFREE0 + u], ((kt >> 1) - 1) & 1, lim)) {
           fail(p, aborted);
           break;
         }
         tc_fence_after();
-        const uint32_t k_addr = sbase + (s ? OFF_K1 : OFF_K0);
+        const uint32_t k_addr = sbase + slot_a(a);
 #pragma unroll
         for (int ks = 0; ks < D / 16; ++ks)
           mma_bf16_ss(tmem + u * 256, kmajor_desc(qa_addr, ks), kmajor_desc(k_addr, ks),
@@ -404,16 +472,17 @@ __global__ void __launch_bounds__(kThreads, 1)
                         IDESC_K_MAJOR, ks > 0);
         }
         mma_commit(&bar[B_SFULL0 + u]);
-        mma_commit(&bar[B_KEMPTY0 + s]);
+        mma_commit(&bar[B_AEMPTY0 + a]);
       }
+      mma_commit(&bar[B_VGO]);  // phase A K tiles in slots V0 / V1 no longer read
       // every phase A TMEM read is done before phase B reuses the columns
       if (!aborted && !mbar_wait(&bar[B_AFREE], 0, lim)) fail(p, aborted);
       tc_fence_after();
       // phase B.  S^T_x(kt) = K(kt) Q_x^T into columns 0 (a) / 128 (b);
       // O_x += P_x(kt) V(kt) into columns 256 (a) / 384 (b).
       auto issue_st = [&](int kt, bool tile_b) -> bool {
-        const int it = n_kt + kt, s = it & 1;
-        if (!tile_b && !mbar_wait(&bar[B_KFULL0 + s], (it >> 1) & 1, lim)) return false;
+        const int s = kt & 1;
+        if (!tile_b && !mbar_wait(&bar[B_KFULL0 + s], (kt >> 1) & 1, lim)) return false;
         if (kt >= 1 && !mbar_wait(&bar[tile_b ? B_TFREEB : B_TFREEA], (kt - 1) & 1, lim))
           return false;
         tc_fence_after();
@@ -467,39 +536,41 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t lane_base = (uint32_t)(32 * (warp & 3)) << 16;
     const float c2 = p.scale2;
     const int i0 = wg ? i0_b : i0_a, bhq = wg ? bhq_b : bhq_a, t = wg ? t_b : t_a;
-    const int64_t row_lim = (int64_t)p.P + i0 + st;
     float m = -INFINITY, l = 0.f;
     uint32_t x[BN];
     for (int kt = 0; kt < n_kt && !aborted; ++kt) {
-      const int u = kt & 1, s = kt & 1;
+      const int u = kt & 1, a = kt % kStagesA;
       if (!warp_wait(&bar[B_SFULL0 + u], (kt >> 1) & 1, lim)) { fail(p, aborted); break; }
-      if (!warp_wait(&bar[B_KFULL0 + s], (kt >> 1) & 1, lim)) { fail(p, aborted); break; }
+      if (!warp_wait(&bar[B_AFULL0 + a], (kt / kStagesA) & 1, lim)) { fail(p, aborted); break; }
       tc_fence_after();
+      const float *rela = reinterpret_cast<const float *>(smem + OFF_P) + a * BN;
       // any slot of this tile invisible to some row of this query tile?
-      const int32_t tpv = max(max(tp_s[s * BN + lane], tp_s[s * BN + lane + 32]),
-                              max(tp_s[s * BN + lane + 64], tp_s[s * BN + lane + 96]));
-      const bool masked = __any_sync(0xffffffffu, (int64_t)tpv > (int64_t)p.P + i0);
+      const float rv = fmax3(fmaxf(rela[lane], rela[lane + 32]), rela[lane + 64], rela[lane + 96]);
+      const bool masked = __any_sync(0xffffffffu, rv > (float)i0);
       const uint32_t sa = tmem + lane_base + u * 256 + wg * 128;
       tmem_ld32(sa, *reinterpret_cast<uint32_t(*)[32]>(x));
       tmem_ld32(sa + 32, *reinterpret_cast<uint32_t(*)[32]>(x + 32));
       tmem_ld32(sa + 64, *reinterpret_cast<uint32_t(*)[32]>(x + 64));
       tmem_ld32(sa + 96, *reinterpret_cast<uint32_t(*)[32]>(x + 96));
       tmem_wait_ld();
-      if (masked) row_mask<BN>(x, tp_s + s * BN, row_lim);
+      if (masked) row_mask<BN>(x, rela, (float)(i0 + st));
       // S buffer and K stage (with its token positions) are free once read
       tc_fence_before();
       __syncwarp();
       if (lane == 0) {
         mbar_arrive(&bar[B_SFREE0 + u]);
-        mbar_arrive(&bar[B_KEMPTY0 + s]);
+        mbar_arrive(&bar[B_AEMPTY0 + a]);
       }
       row_update<BN>(x, c2, m, l);
     }
     __syncwarp();
     if (lane == 0) mbar_arrive(&bar[B_AFREE]);
-    const float lse2 = (l > 0.f) ? m + lg2(l) : -INFINITY;
+    // masked logits sit 2^30 below the visible ones: a row whose maximum is that
+    // low sees no slot (lse = -inf, no weight, y = 0)
+    const bool seen = l > 0.f && m > -0.5f * kMaskBias * c2;
+    const float lse2 = seen ? m + lg2(l) : -INFINITY;
     float *lse_t = lse_s + wg * BM;  // holds -lse2 of the tile's rows
-    lse_t[st] = -lse2;
+    lse_t[st] = seen ? -lse2 : -kMaskBias;
     if (p.lse_out && i0 + st < p.S)
       p.lse_out[(size_t)bhq * p.S + i0 + st] = lse2 * 0.69314718055994531f;
     named_bar_sync(1 + wg, 128);
@@ -510,17 +581,17 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t p_row = sbase + OFF_P + (st >> 3) * 1024 + (st & 7) * 128;
     uint32_t pk[BM / 2];
     for (int kt = 0; kt < n_kt && !aborted; ++kt) {
-      const int it = n_kt + kt, s = it & 1;
+      const int s = kt & 1;
       const int j = kt * BN + st;
       if (!warp_wait(&bar[wg ? B_TFULLB : B_TFULLA], kt & 1, lim)) { fail(p, aborted); break; }
-      if (!warp_wait(&bar[B_KFULL0 + s], (it >> 1) & 1, lim)) { fail(p, aborted); break; }
+      if (!warp_wait(&bar[B_KFULL0 + s], (kt >> 1) & 1, lim)) { fail(p, aborted); break; }
       tc_fence_after();
-      const int64_t tpj = tp_s[s * BN + st];
+      const float relj = __int_as_float(tp_s[s * BN + st]);
       __syncwarp();
       if (lane == 0) mbar_arrive(&bar[B_KEMPTY0 + s]);
-      // visible rows r of this tile: tpj <= P + i0 + r, r < rmax
-      const int64_t rm = tpj - (int64_t)p.P - i0;
-      const int rmin = rm <= 0 ? 0 : (rm >= BM ? BM : (int)rm);
+      // visible rows r of this tile: relj <= i0 + r, r < rmax
+      const float rmf = fminf(fmaxf(relj - (float)i0, 0.f), (float)BM);
+      const int rmin = (int)rmf;
       const bool full = __all_sync(0xffffffffu, rmin == 0 && rmax == BM);
       uint32_t r[BM];
       tmem_ld128(tmem + lane_base + wg * 128, r);
@@ -699,7 +770,6 @@ int launch_attn_tc(h2okv_cache *c, const void *q, int S, int64_t P, void *y, flo
   prm.tiles = (S + BM - 1) / BM;
   prm.n_kt = (d.capacity + BN - 1) / BN;
   prm.ctas_per_group = (prm.q_g * prm.tiles + 1) / 2;
-  prm.tp_bulk = (d.capacity % 4 == 0) ? 1 : 0;
   prm.scale2 = (float)(1.4426950408889634 / 11.313708498984761);  // log2(e) / sqrt(128)
   prm.timeout_ns = c->wait_timeout_ns;
   const int grid = d.batch * d.n_kv_heads * prm.ctas_per_group;

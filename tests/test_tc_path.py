@@ -66,3 +66,26 @@ def test_forced_wait_timeout_reports_status_and_recovers(cuda_device):
     after = snapshot(run.cache)
     check_attend(wl, after, to_np(q), 256, 0, to_np(run.y), to_np(run.lse), to_np(run.w[0]),
                  to_np(run.wq), [(0, 0), (0, 1)])
+
+
+def test_rows_without_visible_slot(cuda_device):
+    """Attention over a cache that holds none of the chunk's tokens: every row
+    sees nothing, so y = 0, lse = -inf and no weight (the convention of the
+    C ABI), on the tensor-core path."""
+    import numpy as np
+    import torch
+
+    from h2o_kv_cache_attn_b200.runner import LayerRunner
+    from h2o_kv_cache_attn_b200.synth import ChunkSource
+
+    from .harness import to_np
+
+    wl = tc("empty_rows", capacity=384, chunk=200, seq_len=400)
+    run = LayerRunner(wl, cuda_device, with_wq=True)
+    q, _, _ = (t.to(cuda_device) for t in ChunkSource(wl).chunk(0))
+    y = torch.empty_like(q)
+    lse = torch.empty(q.shape[:3], dtype=torch.float32, device=cuda_device)
+    run.cache.attend(q, 200, 0, y, lse, run.w[0], run.wq)
+    torch.cuda.synchronize()
+    assert np.all(to_np(y) == 0) and np.all(np.isneginf(to_np(lse)))
+    assert np.all(to_np(run.w[0]) == 0) and np.all(to_np(run.wq) == 0)
