@@ -154,6 +154,21 @@ int kv_cache_create(const h2okv_cache_desc *desc, const h2okv_cache_buffers *buf
   c->tc.maps_ready = false;
   c->wait_timeout_ns = kDefaultWaitTimeoutNs;
   layout(*desc, c->tc, &c->ws);
+  // The attention kernels read every slot and mask the empty ones arithmetically,
+  // which needs finite values there: start from zeroed rows and scales.
+  {
+    const size_t n_slots = (size_t)desc->batch * desc->n_kv_heads * desc->capacity;
+    cudaStream_t st = (cudaStream_t)stream;
+    bool ok = cudaMemsetAsync(bufs->keys, 0, n_slots * c->row_bytes, st) == cudaSuccess &&
+              cudaMemsetAsync(bufs->values, 0, n_slots * c->row_bytes, st) == cudaSuccess;
+    if (ok && c->bufs.k_scales && c->bufs.v_scales)
+      ok = cudaMemsetAsync(c->bufs.k_scales, 0, n_slots * 2, st) == cudaSuccess &&
+           cudaMemsetAsync(c->bufs.v_scales, 0, n_slots * 2, st) == cudaSuccess;
+    if (!ok) {
+      delete c;
+      return set_error(H2OKV_ERR_CUDA, "cudaMemsetAsync(cache rows) failed");
+    }
+  }
   rc = launch_init_cache(c, (cudaStream_t)stream);
   if (rc) {
     delete c;

@@ -103,31 +103,6 @@ __device__ __forceinline__ void quantize_row_warp(const __nv_bfloat16 *__restric
   }
 }
 
-template <int KV>
-__device__ __forceinline__ void copy_row_warp(const void *__restrict__ src, void *__restrict__ dst,
-                                              size_t row_bytes) {
-  const int lane = threadIdx.x & 31;
-  const uint4 *s = reinterpret_cast<const uint4 *>(src);
-  uint4 *o = reinterpret_cast<uint4 *>(dst);
-  for (int i = lane; i < (int)(row_bytes / 16); i += 32) o[i] = s[i];
-}
-
-template <int KV>
-__device__ __forceinline__ void insert_row_warp(const uint8_t *ksrc, const uint8_t *vsrc,
-                                                uint8_t *keys, uint8_t *values, __half *ks,
-                                                __half *vs, size_t dst_row, int d,
-                                                size_t row_bytes) {
-  if constexpr (KV == H2OKV_I8 || KV == H2OKV_I4) {
-    quantize_row_warp<KV>(reinterpret_cast<const __nv_bfloat16 *>(ksrc), d,
-                          keys + dst_row * row_bytes, ks + dst_row);
-    quantize_row_warp<KV>(reinterpret_cast<const __nv_bfloat16 *>(vsrc), d,
-                          values + dst_row * row_bytes, vs + dst_row);
-  } else {
-    copy_row_warp<KV>(ksrc, keys + dst_row * row_bytes, row_bytes);
-    copy_row_warp<KV>(vsrc, values + dst_row * row_bytes, row_bytes);
-  }
-}
-
 struct EvictArgs {
   float *scores;
   const float *w_prev;
@@ -139,6 +114,147 @@ struct EvictArgs {
   int N_C, S, P, mode, n_filled, d, slice;
   size_t row_bytes, in_row_bytes;
 };
+
+constexpr int kCopyUnroll = 8;   // 16-byte pieces per thread in flight in the row copy
+constexpr int kQuantUnroll = 4;  // rows per lane segment in flight in the row quantizer
+
+// Chunk rows k = rank + CL * m (m = 0 .. n_rows - 1) of this (b, h_k) go to slot slot_of(m).
+// f32 / bf16 caches: the key and value rows are cut into 16-byte pieces spread over the
+// whole CTA (consecutive threads take consecutive pieces of a row), and every thread loads
+// kCopyUnroll pieces before it stores any, so a launch waits on memory a few times in all
+// rather than once per row.
+template <typename SlotOf>
+__device__ __forceinline__ void copy_rows_cta(const EvictArgs &a, size_t bh, int rank, int CL,
+                                              int n_rows, SlotOf slot_of) {
+  const int C = (int)(a.row_bytes / 16);  // 16-byte pieces per row (row_bytes % 16 == 0)
+  const int total = n_rows * 2 * C;
+  const size_t gbase = bh * (size_t)a.N_C;
+  for (int base = threadIdx.x; base < total; base += kEvThreads * kCopyUnroll) {
+    uint4 r[kCopyUnroll];
+    uint4 *dst[kCopyUnroll];
+#pragma unroll
+    for (int u = 0; u < kCopyUnroll; ++u) {
+      const int e = base + u * kEvThreads;
+      dst[u] = nullptr;
+      if (e < total) {
+        const int c = e % C, rest = e / C, t = rest & 1, m = rest >> 1;
+        const size_t row = bh * (size_t)a.S + rank + (size_t)CL * m;
+        const uint8_t *src = (t ? a.v_new : a.k_new) + row * a.in_row_bytes;
+        r[u] = __ldcs(reinterpret_cast<const uint4 *>(src) + c);
+        dst[u] = reinterpret_cast<uint4 *>((t ? a.values : a.keys) +
+                                           (gbase + (size_t)slot_of(m)) * a.row_bytes) + c;
+      }
+    }
+#pragma unroll
+    for (int u = 0; u < kCopyUnroll; ++u)
+      if (dst[u]) *dst[u] = r[u];
+  }
+}
+
+// int8 / int4 caches: one row per segment of L lanes (L = the smallest power of two
+// >= d / 8); lane i of a segment holds elements 8i .. 8i + 7 of the row.  A warp covers
+// 32 / L rows per pass and keeps kQuantUnroll passes in flight.  Per row, the same
+// arithmetic as the per-row quantizer: absmax, IEEE division by qmax, clamp to the fp16
+// range, round to fp16, then rint(x / scale) clamped to [-qmax, qmax].
+template <int KV, typename SlotOf>
+__device__ __forceinline__ void quantize_rows_cta(const EvictArgs &a, size_t bh, int rank, int CL,
+                                                  int n_rows, SlotOf slot_of) {
+  constexpr int qmax = KV == H2OKV_I8 ? 127 : 7;
+  const int G = a.d / 8;
+  int L = 1;
+  while (L < G) L <<= 1;
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int seg = lane / L, li = lane % L, segs = 32 / L;
+  const int items = n_rows * 2;  // (m, t): t = 0 key row, 1 value row
+  const size_t gbase = bh * (size_t)a.N_C;
+  for (int p0 = 0; (p0 * kEvWarps + warp) * segs < items; p0 += kQuantUnroll) {
+    uint4 x[kQuantUnroll];
+    bool ok[kQuantUnroll];
+#pragma unroll
+    for (int u = 0; u < kQuantUnroll; ++u) {
+      const int item = ((p0 + u) * kEvWarps + warp) * segs + seg;
+      ok[u] = item < items && li < G;
+      x[u] = make_uint4(0u, 0u, 0u, 0u);
+      if (ok[u]) {
+        const int t = item & 1, m = item >> 1;
+        const size_t row = bh * (size_t)a.S + rank + (size_t)CL * m;
+        const uint8_t *src = (t ? a.v_new : a.k_new) + row * a.in_row_bytes;
+        x[u] = __ldcs(reinterpret_cast<const uint4 *>(src) + li);
+      }
+    }
+#pragma unroll
+    for (int u = 0; u < kQuantUnroll; ++u) {
+      float v[8];
+      const __nv_bfloat162 *h2 = reinterpret_cast<const __nv_bfloat162 *>(&x[u]);
+      float amax = 0.f;
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        const float2 f = __bfloat1622float2(h2[q]);
+        v[2 * q] = f.x;
+        v[2 * q + 1] = f.y;
+        amax = fmaxf(amax, fmaxf(fabsf(f.x), fabsf(f.y)));
+      }
+      for (int o = L >> 1; o > 0; o >>= 1)
+        amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
+      float r = amax / (float)qmax;  // IEEE division
+      r = fminf(r, 65504.f);
+      const __half hs = __float2half_rn(r);
+      const float s = __half2float(hs);
+      int qc[8];
+#pragma unroll
+      for (int q = 0; q < 8; ++q)
+        qc[q] = s > 0.f ? (int)fminf(fmaxf(rintf(v[q] / s), (float)-qmax), (float)qmax) : 0;
+      if (!ok[u]) continue;
+      const int item = ((p0 + u) * kEvWarps + warp) * segs + seg;
+      const int t = item & 1, m = item >> 1;
+      const size_t drow = gbase + (size_t)slot_of(m);
+      uint8_t *codes = (t ? a.values : a.keys) + drow * a.row_bytes;
+      if (li == 0) (t ? a.v_scales : a.k_scales)[drow] = hs;
+      if (KV == H2OKV_I8) {
+        uint32_t lo = 0u, hi = 0u;
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          lo |= ((uint32_t)(qc[q] & 0xFF)) << (8 * q);
+          hi |= ((uint32_t)(qc[q + 4] & 0xFF)) << (8 * q);
+        }
+        reinterpret_cast<uint2 *>(codes)[li] = make_uint2(lo, hi);
+      } else {
+        uint32_t w = 0u;  // element 2i in the low nibble of byte i
+#pragma unroll
+        for (int q = 0; q < 8; ++q) w |= ((uint32_t)(qc[q] & 0xF)) << (4 * q);
+        reinterpret_cast<uint32_t *>(codes)[li] = w;
+      }
+    }
+  }
+}
+
+template <int KV, typename SlotOf>
+__device__ __forceinline__ void insert_rows_cta(const EvictArgs &a, size_t bh, int rank, int CL,
+                                                SlotOf slot_of) {
+  const int n_rows = rank < a.S ? (a.S - rank + CL - 1) / CL : 0;
+  if constexpr (KV == H2OKV_I8 || KV == H2OKV_I4)
+    quantize_rows_cta<KV>(a, bh, rank, CL, n_rows, slot_of);
+  else
+    copy_rows_cta(a, bh, rank, CL, n_rows, slot_of);
+}
+
+template <int IPT>
+__device__ __forceinline__ void store_slice(float *dst, const float (&v)[IPT],
+                                            const bool (&valid)[IPT], bool vec) {
+  if constexpr (IPT % 4 == 0) {
+    if (vec) {
+#pragma unroll
+      for (int i = 0; i < IPT; i += 4)
+        *reinterpret_cast<float4 *>(dst + i) = make_float4(v[i], v[i + 1], v[i + 2], v[i + 3]);
+      return;
+    }
+  }
+  {
+#pragma unroll
+    for (int i = 0; i < IPT; ++i)
+      if (valid[i]) dst[i] = v[i];
+  }
+}
 
 // mode 0: fold w_prev only (S = 0); 1: fill slots n_filled.. (no occupied slot is
 // touched); 2: generic choice (empty slots first, then lowest scores).
@@ -160,21 +276,53 @@ __global__ void __launch_bounds__(kEvThreads) evict_kernel(const EvictArgs a) {
 
   const size_t gbase = (size_t)bh * a.N_C;
   const int j0 = rank * a.slice + tid * IPT;
-  float sc[IPT];
+  float sc[IPT], wp[IPT];
+  int32_t tp[IPT];
   uint32_t key[IPT];
   bool valid[IPT];
 #pragma unroll
   for (int i = 0; i < IPT; ++i) {
-    const int j = j0 + i;
-    valid[i] = j < a.N_C;
+    valid[i] = j0 + i < a.N_C;
     sc[i] = 0.f;
-    key[i] = 0u;
-    if (valid[i]) {
-      float s = a.scores[gbase + j];
-      if (a.w_prev) s = __fadd_rn(s, a.w_prev[gbase + j]);
-      sc[i] = s;
-      if (a.mode == 2) key[i] = (a.token_pos[gbase + j] == kEmptyPos) ? 0u : order_key(s);
+    wp[i] = 0.f;
+    tp[i] = kEmptyPos;
+  }
+  // 16-byte loads when this thread's slots are whole and aligned, else one by one
+  const bool vec = IPT % 4 == 0 && j0 + IPT <= a.N_C &&
+                   ((reinterpret_cast<uintptr_t>(a.scores + gbase + j0) |
+                     reinterpret_cast<uintptr_t>(a.token_pos + gbase + j0) |
+                     (a.w_prev ? reinterpret_cast<uintptr_t>(a.w_prev + gbase + j0) : 0u)) &
+                    15u) == 0u;
+  bool loaded = false;
+  if constexpr (IPT % 4 == 0) {
+    if (vec) {
+#pragma unroll
+      for (int i = 0; i < IPT; i += 4) {
+        *reinterpret_cast<float4 *>(&sc[i]) =
+            *reinterpret_cast<const float4 *>(a.scores + gbase + j0 + i);
+        if (a.w_prev)
+          *reinterpret_cast<float4 *>(&wp[i]) =
+              __ldcs(reinterpret_cast<const float4 *>(a.w_prev + gbase + j0 + i));
+        if (a.mode == 2)
+          *reinterpret_cast<int4 *>(&tp[i]) =
+              *reinterpret_cast<const int4 *>(a.token_pos + gbase + j0 + i);
+      }
+      loaded = true;
     }
+  }
+  if (!loaded) {
+#pragma unroll
+    for (int i = 0; i < IPT; ++i) {
+      if (!valid[i]) continue;
+      sc[i] = a.scores[gbase + j0 + i];
+      if (a.w_prev) wp[i] = a.w_prev[gbase + j0 + i];
+      if (a.mode == 2) tp[i] = a.token_pos[gbase + j0 + i];
+    }
+  }
+#pragma unroll
+  for (int i = 0; i < IPT; ++i) {
+    if (a.w_prev) sc[i] = __fadd_rn(sc[i], wp[i]);
+    key[i] = (valid[i] && a.mode == 2 && tp[i] != kEmptyPos) ? order_key(sc[i]) : 0u;
   }
 
   if (a.mode != 2) {
@@ -185,20 +333,16 @@ __global__ void __launch_bounds__(kEvThreads) evict_kernel(const EvictArgs a) {
       if (!valid[i]) continue;
       const int k = j - a.n_filled;
       if (a.mode == 1 && k >= 0 && k < a.S) {
-        a.scores[gbase + j] = 0.f;
+        sc[i] = 0.f;
+        if (!a.w_prev) a.scores[gbase + j] = 0.f;
         a.token_pos[gbase + j] = a.P + k;
         if (a.slots_out) a.slots_out[(size_t)bh * a.S + k] = j;
-      } else if (a.w_prev) {
-        a.scores[gbase + j] = sc[i];
       }
     }
+    if (a.w_prev) store_slice<IPT>(a.scores + gbase + j0, sc, valid, vec);
     if (a.mode == 1) {
-      for (int k = rank + CL * warp; k < a.S; k += CL * kEvWarps) {
-        const size_t row = (size_t)bh * a.S + k;
-        insert_row_warp<KV>(a.k_new + row * a.in_row_bytes, a.v_new + row * a.in_row_bytes,
-                            a.keys, a.values, a.k_scales, a.v_scales, gbase + a.n_filled + k,
-                            a.d, a.row_bytes);
-      }
+      const int first = a.n_filled + rank;
+      insert_rows_cta<KV>(a, (size_t)bh, rank, CL, [&](int m) { return first + CL * m; });
     }
     return;
   }
@@ -298,17 +442,12 @@ __global__ void __launch_bounds__(kEvThreads) evict_kernel(const EvictArgs a) {
       int32_t *dst = cluster.map_shared_rank(rowslot, (int)(pos % (uint32_t)CL));
       dst[pos / (uint32_t)CL] = j;
     }
-    a.scores[gbase + j] = sc[i];
   }
+  store_slice<IPT>(a.scores + gbase + j0, sc, valid, vec);
   cluster.sync();  // rowslot lists complete
 
   // ---- insert the chunk's rows k = rank, rank + CL, ... -----------------------------
-  for (int m = warp; rank + CL * m < a.S; m += kEvWarps) {
-    const int k = rank + CL * m;
-    const size_t row = (size_t)bh * a.S + k;
-    insert_row_warp<KV>(a.k_new + row * a.in_row_bytes, a.v_new + row * a.in_row_bytes, a.keys,
-                        a.values, a.k_scales, a.v_scales, gbase + rowslot[m], a.d, a.row_bytes);
-  }
+  insert_rows_cta<KV>(a, (size_t)bh, rank, CL, [&](int m) { return rowslot[m]; });
 }
 
 template <int KV>

@@ -108,13 +108,16 @@ enum {
 H2OKV_API int kv_cache_query_sizes(const h2okv_cache_desc *desc, size_t sizes[H2OKV_NUM_BUFS]);
 
 /* Create a handle over caller-owned buffers and enqueue their initialisation
- * on `stream`: token_pos = INT32_MAX (empty), scores = 0; keys/values/scales
- * are left as they are (empty slots are never read unmasked).  The cache then
- * holds no token (fill level 0).  Writes the handle to *out. */
+ * on `stream`: token_pos = INT32_MAX (empty), scores = 0, keys/values/scales
+ * zero-filled (the attention kernels read every slot and mask empty ones
+ * arithmetically, so every slot must hold finite values; a caller that writes
+ * the buffers directly must keep them finite).  The cache then holds no token
+ * (fill level 0).  Writes the handle to *out. */
 H2OKV_API int kv_cache_create(const h2okv_cache_desc *desc, const h2okv_cache_buffers *bufs,
                     void *stream, h2okv_cache **out);
 
-/* Return the cache to the empty state (as after create). */
+/* Return the cache to the empty state (token_pos and scores as after create;
+ * the rows keep their previous, finite contents). */
 H2OKV_API int kv_cache_reset(h2okv_cache *cache, void *stream);
 
 /* Free the handle (not the caller's buffers).  NULL is accepted. */
