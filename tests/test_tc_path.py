@@ -89,3 +89,41 @@ def test_rows_without_visible_slot(cuda_device):
     torch.cuda.synchronize()
     assert np.all(to_np(y) == 0) and np.all(np.isneginf(to_np(lse)))
     assert np.all(to_np(run.w[0]) == 0) and np.all(to_np(run.wq) == 0)
+
+
+def test_create_clears_nonfinite_rows(cuda_device):
+    """The tensor-core kernels read every slot and mask empty ones
+    arithmetically, so kv_cache_create zero-fills the rows: a cache created over
+    buffers full of NaN gives bit for bit the outputs of one created over zeros."""
+    import numpy as np
+    import torch
+
+    from h2o_kv_cache_attn_b200 import binding as hb
+    from h2o_kv_cache_attn_b200.runner import LayerRunner
+    from h2o_kv_cache_attn_b200.synth import ChunkSource
+
+    from .harness import to_np
+
+    wl = tc("nan_rows", capacity=384, chunk=128, seq_len=256)
+    src = ChunkSource(wl)
+    outs = []
+    for poison in (False, True):
+        run = LayerRunner(wl, cuda_device, with_wq=True)
+        if poison:
+            c = run.cache
+            c.keys.fill_(float("nan"))
+            c.values.fill_(float("nan"))
+            old = c.handle
+            c.handle = hb.kv_cache_create(c._desc, c._bufs, None)
+            hb.kv_cache_destroy(old)
+        res = []
+        for ci in range(wl.n_chunks):
+            q, k, v = (t.to(cuda_device) for t in src.chunk(ci))
+            y, _, w, wq, _ = run.step(q, k, v)
+            torch.cuda.synchronize()
+            res.append((to_np(y).copy(), to_np(w).copy(), to_np(wq).copy()))
+        outs.append(res)
+    for a, b in zip(*outs):
+        assert np.all(np.isfinite(b[0])) and np.all(np.isfinite(b[1]))
+        for x, z in zip(a, b):
+            assert np.array_equal(x, z)
