@@ -241,8 +241,9 @@ def run_ours(args, wl, ws, rank, local):
     tflops_alg = at_flops_alg / at_total_s / 1e12
     evict_us = statistics.median(evict_full_ms) * 1e3 if evict_full_ms else None
     evict_gbs = evict_bytes_chunk(wl, wl.chunk) / (evict_us * 1e-6) / 1e9 if evict_us else None
-    # the tensor-core path serves head_dim 128 with a bf16 cache (same rule as the library)
-    tc_used = wl.d == 128 and wl.kv_dtype == "bf16" and wl.q_dtype == "bf16"
+    # the tensor-core path serves head_dim 128 with a bf16, int8 or int4 cache and bf16
+    # queries (the same rule as the library)
+    tc_used = wl.d == 128 and wl.kv_dtype in ("bf16", "i8", "i4") and wl.q_dtype == "bf16"
     # per chunk: one eviction launch, then two attention launches (tensor-core path:
     # attention + reduction; CUDA-core path: two passes); plus the reset and the final fold
     launches_per_step = wl.n_chunks * 3 + 2

@@ -1,7 +1,8 @@
 // Tensor-core path of chunked cache attention with summed weights for d = 128
-// and a bf16 cache ("Learning how to Forget", §A.1 token-position mask, §A.7
-// SDPA plus the attention weights summed over the query axis, returned per KV
-// slot and summed over the q_g query heads of each GQA group).
+// and a bf16, int8 or int4 cache ("Learning how to Forget", §A.1 token-position
+// mask, §A.7 SDPA plus the attention weights summed over the query axis, returned
+// per KV slot and summed over the q_g query heads of each GQA group; §4 / Table
+// 1 8- and 4-bit caches).
 //
 // One CTA owns two 128-row query tiles (a, b) of one KV group (two row tiles of
 // one head, or the same rows of two heads); rows past S are zero-filled by TMA
@@ -31,12 +32,19 @@
 // The MMA issue order S^T_a(kt+1), S^T_b(kt+1), PV_a(kt), PV_b(kt) lets the tensor
 // pipe compute the next logits while the softmax warps turn the current ones
 // into P.
+// Quantized caches (int8 / int4 codes with one fp16 scale per slot): warps 0, 2
+// and 3 replace the TMA producers and dequantize while they load (see
+// convert_tile): key tiles become exact bf16 integers and the key scale s_j
+// multiplies the logits of slot j (a column scale of S in phase A, a per-thread
+// factor in phase B), so scores and summed weights see the stored keys exactly;
+// value tiles are stored as bf16(code * scale).
 // Every wait is bounded; a timeout sets the cache's device status word and the
 // CTA drains its copies and MMAs before freeing TMEM.
 //
 // Per-(query tile, slot) sums go to a partial buffer; a small reduction kernel
 // sums them in a fixed order into w [B, H_k, N_C] and wq [B, H_q, N_C].
 #include <stdio.h>
+#include <string.h>
 
 #include "h2okv_internal.cuh"
 #include "tc_ptx.cuh"
@@ -71,14 +79,18 @@ constexpr uint32_t OFF_V1 = OFF_V0 + kTileBytes;
 constexpr uint32_t OFF_P = OFF_V1 + kTileBytes;
 constexpr uint32_t OFF_TP = OFF_P + kTileBytes;        // int32 [2 stages][BN]
 constexpr uint32_t OFF_LSE = OFF_TP + 2 * BN * 4;      // float [2 tiles][BM]
-constexpr uint32_t OFF_BAR = OFF_LSE + 2 * BM * 4;     // uint64 barriers
+constexpr uint32_t OFF_KSB = OFF_LSE + 2 * BM * 4;     // fp16 [2 stages][BN] phase B key scales
+constexpr uint32_t OFF_BAR = OFF_KSB + 2 * BN * 2;     // uint64 barriers
 constexpr int kStagesA = 4;  // phase A K ring: slots K0, K1, V0, V1 (V is unused in phase A)
 constexpr int NBAR = 25 + 2 * kStagesA;
 constexpr uint32_t OFF_TMEM = OFF_BAR + NBAR * 8;
 constexpr uint32_t kSmemBytes = OFF_TMEM + 16;
 static_assert(kSmemBytes <= 232448, "shared memory budget");
 
-// phase A stage -> slot; phase A token positions live in the P region (unused in phase A)
+// phase A stage -> slot; phase A token positions (float [kStagesA][BN]) and key
+// scales (float [kStagesA][BN], quantized caches) live in the P region, unused in phase A
+constexpr uint32_t OFF_REL_A = OFF_P;
+constexpr uint32_t OFF_KS_A = OFF_P + kStagesA * BN * 4;
 __host__ __device__ constexpr uint32_t slot_a(int a) {
   return a == 0 ? OFF_K0 : a == 1 ? OFF_K1 : a == 2 ? OFF_V0 : OFF_V1;
 }
@@ -94,6 +106,8 @@ constexpr uint32_t IDESC_PV = idesc_bf16_f32(128, 128, true, true);
 
 struct TcParams {
   const int32_t *token_pos;  // [B*Hk][N_C]
+  const uint8_t *kq, *vq;    // quantized caches: codes [B*Hk][N_C][row bytes]
+  const __half *ksc, *vsc;   // quantized caches: scales [B*Hk][N_C]
   __nv_bfloat16 *y;          // [B*Hq][S][D]
   float *lse_out;            // [B*Hq][S] or null
   float *part_w;             // [B*Hq*tiles][N_C]
@@ -263,6 +277,155 @@ __device__ __forceinline__ void store_p(uint32_t p_slot_row, int st, const uint3
   }
 }
 
+// ---- quantized caches: dequantizing tile loads --------------------------------------
+// 96 converter threads (warps 0, 2, 3) read a 128-slot tile of codes with 16-byte
+// loads (a batch in flight per thread), turn every code into bf16 and store the
+// tile in the swizzled K-major layout the MMA reads (the bytes a TMA load of a
+// bf16 tile would produce: row j at 128 j, 16-byte chunk c at c ^ (j % 8), dims
+// 64..127 in the second 16 KiB half).  A code c becomes a float exactly as the
+// float whose bits are 0x4B0000uu (2^23 + u, u = c + 128 or c + 8 as an unsigned
+// byte) minus 2^23 + 128 (or + 8); |c| <= 127 is exact in bf16.  Value tiles are
+// multiplied by their slot's scale first (exact in float32, one rounding to bf16).
+constexpr int kConvThreads = 96;
+template <int KV>
+struct QTile;
+template <>
+struct QTile<H2OKV_I8> {
+  static constexpr int kRowBytes = D, kChunksPerRow = D / 16;  // 16 codes per 16-byte chunk
+};
+template <>
+struct QTile<H2OKV_I4> {
+  static constexpr int kRowBytes = D / 2, kChunksPerRow = D / 32;  // 32 codes per chunk
+};
+
+__device__ __forceinline__ float offset_byte_float(uint32_t u, uint32_t k) {
+  return __uint_as_float(__byte_perm(u, 0x4B000000u, 0x7440u | k));  // bits 0x4B0000 | byte k
+}
+
+__device__ __forceinline__ void st_shared_v4(uint32_t addr, uint32_t a, uint32_t b, uint32_t c,
+                                             uint32_t d) {
+  asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(a), "r"(b), "r"(c),
+               "r"(d)
+               : "memory");
+}
+
+// 8 int8 codes (element 4i + k in byte k of word i) -> 4 bf16 pairs in element order
+__device__ __forceinline__ void cvt_i8x8(uint32_t w0, uint32_t w1, float2 s2, bool fold,
+                                         uint32_t (&o)[4]) {
+  const float2 off = make_float2(-8388736.f, -8388736.f);  // -(2^23 + 128)
+  const uint32_t ws[2] = {w0 ^ 0x80808080u, w1 ^ 0x80808080u};
+#pragma unroll
+  for (int i = 0; i < 2; ++i) {
+    float2 a = add2(make_float2(offset_byte_float(ws[i], 0), offset_byte_float(ws[i], 1)), off);
+    float2 b = add2(make_float2(offset_byte_float(ws[i], 2), offset_byte_float(ws[i], 3)), off);
+    if (fold) {
+      a = mul2(a, s2);
+      b = mul2(b, s2);
+    }
+    o[2 * i] = pack_bf16x2(a.x, a.y);
+    o[2 * i + 1] = pack_bf16x2(b.x, b.y);
+  }
+}
+
+// 8 int4 codes (element 2k in the low nibble, 2k + 1 in the high nibble of byte k)
+// -> 4 bf16 pairs in element order
+__device__ __forceinline__ void cvt_i4x8(uint32_t w, float2 s2, bool fold, uint32_t (&o)[4]) {
+  const float2 off = make_float2(-8388616.f, -8388616.f);  // -(2^23 + 8)
+  const uint32_t u = w ^ 0x88888888u;
+  const uint32_t lo = u & 0x0F0F0F0Fu, hi = (u >> 4) & 0x0F0F0F0Fu;
+#pragma unroll
+  for (int k = 0; k < 4; ++k) {
+    float2 a = add2(make_float2(offset_byte_float(lo, k), offset_byte_float(hi, k)), off);
+    if (fold) a = mul2(a, s2);
+    o[k] = pack_bf16x2(a.x, a.y);
+  }
+}
+
+// Tile of slots slot0 .. slot0 + 127 (nv of them inside the cache; the rest are
+// written as zeros) into the bf16 operand at shared address dst.
+template <int KV>
+__device__ __forceinline__ void convert_tile(const uint8_t *__restrict__ codes,
+                                             const __half *__restrict__ scales, int slot0, int nv,
+                                             uint32_t dst, bool fold, int ct) {
+  using T = QTile<KV>;
+  constexpr int kChunks = BN * T::kChunksPerRow;
+  constexpr int kPer = (kChunks + kConvThreads - 1) / kConvThreads;
+  constexpr int kBatch = KV == H2OKV_I8 ? 3 : 2;  // loads in flight per thread (register budget of the loader warps)
+#pragma unroll
+  for (int r0 = 0; r0 < kPer; r0 += kBatch) {
+    uint4 w[kBatch];
+    float sc[kBatch];
+#pragma unroll
+    for (int b = 0; b < kBatch; ++b) {
+      const int ch = ct + kConvThreads * (r0 + b);
+      const int j = ch / T::kChunksPerRow, q = ch % T::kChunksPerRow;
+      w[b] = make_uint4(0u, 0u, 0u, 0u);
+      sc[b] = 0.f;
+      if (r0 + b < kPer && ch < kChunks && j < nv) {
+        w[b] = __ldg(reinterpret_cast<const uint4 *>(codes + (size_t)(slot0 + j) * T::kRowBytes) + q);
+        if (fold) sc[b] = __half2float(scales[slot0 + j]);
+      }
+    }
+#pragma unroll
+    for (int b = 0; b < kBatch; ++b) {
+      const int ch = ct + kConvThreads * (r0 + b);
+      if (r0 + b >= kPer || ch >= kChunks) continue;
+      const int j = ch / T::kChunksPerRow, q = ch % T::kChunksPerRow;
+      const uint32_t sw = (uint32_t)(j & 7);
+      const float2 s2 = make_float2(sc[b], sc[b]);
+      uint32_t o[4];
+      if constexpr (KV == H2OKV_I8) {
+        // dims 16q .. 16q + 15: half q / 4, 16-byte chunks 2 (q % 4) and 2 (q % 4) + 1
+        const uint32_t row = dst + (uint32_t)(q >> 2) * kHalfBytes + (uint32_t)j * 128;
+        const uint32_t c0 = 2u * (uint32_t)(q & 3);
+        cvt_i8x8(w[b].x, w[b].y, s2, fold, o);
+        st_shared_v4(row + ((c0 ^ sw) << 4), o[0], o[1], o[2], o[3]);
+        cvt_i8x8(w[b].z, w[b].w, s2, fold, o);
+        st_shared_v4(row + (((c0 + 1) ^ sw) << 4), o[0], o[1], o[2], o[3]);
+      } else {
+        // dims 32q .. 32q + 31: half q / 2, 16-byte chunks 4 (q % 2) .. 4 (q % 2) + 3
+        const uint32_t row = dst + (uint32_t)(q >> 1) * kHalfBytes + (uint32_t)j * 128;
+        const uint32_t c0 = 4u * (uint32_t)(q & 1);
+        const uint32_t ws[4] = {w[b].x, w[b].y, w[b].z, w[b].w};
+#pragma unroll
+        for (int m = 0; m < 4; ++m) {
+          cvt_i4x8(ws[m], s2, fold, o);
+          st_shared_v4(row + (((c0 + m) ^ sw) << 4), o[0], o[1], o[2], o[3]);
+        }
+      }
+    }
+  }
+}
+
+// Key scales times the raw logits of one row (phase A, quantized caches).
+template <int N>
+__device__ __forceinline__ void scale_row(uint32_t (&x)[N], const float *ks) {
+#pragma unroll
+  for (int e = 0; e < N; e += 4) {
+    const float4 k4 = *reinterpret_cast<const float4 *>(ks + e);
+    const float2 a = mul2(make_float2(__uint_as_float(x[e]), __uint_as_float(x[e + 1])),
+                          make_float2(k4.x, k4.y));
+    const float2 b = mul2(make_float2(__uint_as_float(x[e + 2]), __uint_as_float(x[e + 3])),
+                          make_float2(k4.z, k4.w));
+    x[e] = __float_as_uint(a.x);
+    x[e + 1] = __float_as_uint(a.y);
+    x[e + 2] = __float_as_uint(b.x);
+    x[e + 3] = __float_as_uint(b.y);
+  }
+}
+
+// Relative token positions of a tile's slots (float; 2^20 for empty / outside
+// slots), written by the loader threads t = first, first + step, ...
+__device__ __forceinline__ void write_rel(float *dst, const int32_t *tpg, int slot0, int nv, int P,
+                                          int first, int step) {
+  for (int e = first; e < BN; e += step) {
+    const int64_t t = e < nv ? (int64_t)tpg[slot0 + e] : (int64_t)kEmptyPos;
+    const int64_t rel = t - (int64_t)P;
+    dst[e] = (float)(rel < -1 ? -1 : (rel > kRelFar ? kRelFar : rel));
+  }
+}
+
+template <int KV>
 __global__ void __launch_bounds__(kThreads, 1)
     attn_tc_kernel(const __grid_constant__ CUtensorMap q_map,
                    const __grid_constant__ CUtensorMap k_map,
@@ -294,12 +457,14 @@ __global__ void __launch_bounds__(kThreads, 1)
   const uint64_t lim = p.timeout_ns;
 
   const int nwg = has_b ? 2 : 1;  // softmax warpgroups with a query tile
+  // tile-full barriers: one TMA producer (bf16) or the three loader warps (quantized)
+  constexpr uint32_t kFullCount = KV == H2OKV_BF16 ? 1 : kConvThreads / 32;
   if (threadIdx.x == 0) {
     mbar_init(&bar[B_Q], 1);
     for (int i = 0; i < 2; ++i) {
-      mbar_init(&bar[B_KFULL0 + i], 1);
+      mbar_init(&bar[B_KFULL0 + i], kFullCount);
       mbar_init(&bar[B_KEMPTY0 + i], 1 + 4 * nwg);  // MMA commit + softmax warps (token positions)
-      mbar_init(&bar[B_VFULL0 + i], 1);
+      mbar_init(&bar[B_VFULL0 + i], kFullCount);
       mbar_init(&bar[B_VEMPTY0 + i], 1);
       mbar_init(&bar[B_SFULL0 + i], 1);
       mbar_init(&bar[B_SFREE0 + i], 4 * nwg);
@@ -317,7 +482,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     mbar_init(&bar[B_DRAIN], 1);
     mbar_init(&bar[B_VGO], 1);
     for (int i = 0; i < kStagesA; ++i) {
-      mbar_init(&bar[B_AFULL0 + i], 1);
+      mbar_init(&bar[B_AFULL0 + i], kFullCount);
       mbar_init(&bar[B_AEMPTY0 + i], 1 + 4 * nwg);
     }
     fence_mbar_init();
@@ -329,8 +494,10 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
   if (warp == 0 && lane == 0) {
     prefetch_tensormap(&q_map);
-    prefetch_tensormap(&k_map);
-    prefetch_tensormap(&v_map);
+    if (KV == H2OKV_BF16) {
+      prefetch_tensormap(&k_map);
+      prefetch_tensormap(&v_map);
+    }
   }
   __syncthreads();
   tc_fence_after();
@@ -339,6 +506,88 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   if (warp < 4) {
   reg_dealloc<kCtrlRegs>();
+  if (warp == 1) {
+    // ------------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      const uint32_t qa_addr = sbase + OFF_QA, qb_addr = sbase + OFF_QB, p_addr = sbase + OFF_P;
+      if (!mbar_wait(&bar[B_Q], 0, lim)) fail(p, aborted);
+      tc_fence_after();
+      // phase A: S_a, S_b = Q_a K^T, Q_b K^T into the column pair of the tile parity
+      for (int kt = 0; kt < n_kt && !aborted; ++kt) {
+        const int a = kt % kStagesA, u = kt & 1;
+        if (!mbar_wait(&bar[B_AFULL0 + a], (kt / kStagesA) & 1, lim)) { fail(p, aborted); break; }
+        if (kt >= 2 && !mbar_wait(&bar[B_SFREE0 + u], ((kt >> 1) - 1) & 1, lim)) {
+          fail(p, aborted);
+          break;
+        }
+        tc_fence_after();
+        const uint32_t k_addr = sbase + slot_a(a);
+#pragma unroll
+        for (int ks = 0; ks < D / 16; ++ks)
+          mma_bf16_ss(tmem + u * 256, kmajor_desc(qa_addr, ks), kmajor_desc(k_addr, ks),
+                      IDESC_K_MAJOR, ks > 0);
+        if (has_b) {
+#pragma unroll
+          for (int ks = 0; ks < D / 16; ++ks)
+            mma_bf16_ss(tmem + u * 256 + 128, kmajor_desc(qb_addr, ks), kmajor_desc(k_addr, ks),
+                        IDESC_K_MAJOR, ks > 0);
+        }
+        mma_commit(&bar[B_SFULL0 + u]);
+        mma_commit(&bar[B_AEMPTY0 + a]);
+      }
+      mma_commit(&bar[B_VGO]);  // phase A K tiles in slots V0 / V1 no longer read
+      // every phase A TMEM read is done before phase B reuses the columns
+      if (!aborted && !mbar_wait(&bar[B_AFREE], 0, lim)) fail(p, aborted);
+      tc_fence_after();
+      // phase B.  S^T_x(kt) = K(kt) Q_x^T into columns 0 (a) / 128 (b);
+      // O_x += P_x(kt) V(kt) into columns 256 (a) / 384 (b).
+      auto issue_st = [&](int kt, bool tile_b) -> bool {
+        const int s = kt & 1;
+        if (!tile_b && !mbar_wait(&bar[B_KFULL0 + s], (kt >> 1) & 1, lim)) return false;
+        if (kt >= 1 && !mbar_wait(&bar[tile_b ? B_TFREEB : B_TFREEA], (kt - 1) & 1, lim))
+          return false;
+        tc_fence_after();
+        const uint32_t k_addr = sbase + (s ? OFF_K1 : OFF_K0);
+        const uint32_t q_addr = tile_b ? qb_addr : qa_addr;
+#pragma unroll
+        for (int ks = 0; ks < D / 16; ++ks)
+          mma_bf16_ss(tmem + (tile_b ? 128 : 0), kmajor_desc(k_addr, ks), kmajor_desc(q_addr, ks),
+                      IDESC_K_MAJOR, ks > 0);
+        mma_commit(&bar[tile_b ? B_TFULLB : B_TFULLA]);
+        if (tile_b || !has_b) mma_commit(&bar[B_KEMPTY0 + s]);  // K(kt) no longer read
+        return true;
+      };
+      auto issue_pv = [&](int kt, bool tile_b) -> bool {
+        if (!mbar_wait(&bar[tile_b ? B_PFULLB : B_PFULLA], kt & 1, lim)) return false;
+        if (!tile_b && !mbar_wait(&bar[B_VFULL0 + (kt & 1)], (kt >> 1) & 1, lim)) return false;
+        tc_fence_after();
+        const uint32_t v_addr = sbase + ((kt & 1) ? OFF_V1 : OFF_V0);
+#pragma unroll
+        for (int ks = 0; ks < BN / 16; ++ks)
+          mma_bf16_ss(tmem + (tile_b ? 384 : 256), mnmajor_desc(p_addr, ks),
+                      mnmajor_desc(v_addr, ks), IDESC_PV, (kt > 0 || ks > 0) ? 1u : 0u);
+        mma_commit(&bar[tile_b ? B_PFREEB : B_PFREEA]);
+        if (tile_b || !has_b) mma_commit(&bar[B_VEMPTY0 + (kt & 1)]);  // V(kt) no longer read
+        return true;
+      };
+      if (!aborted && !issue_st(0, false)) fail(p, aborted);
+      if (!aborted && has_b && !issue_st(0, true)) fail(p, aborted);
+      // S^T of the next tile is issued as soon as the softmax warps have read the
+      // current one out of TMEM (long before their P is ready), then the P V
+      // products of the current tile.
+      for (int kt = 0; kt < n_kt && !aborted; ++kt) {
+        if (kt + 1 < n_kt && !issue_st(kt + 1, false)) { fail(p, aborted); break; }
+        if (kt + 1 < n_kt && has_b && !issue_st(kt + 1, true)) { fail(p, aborted); break; }
+        if (!issue_pv(kt, false)) { fail(p, aborted); break; }
+        if (has_b && !issue_pv(kt, true)) { fail(p, aborted); break; }
+      }
+      mma_commit(&bar[B_OFULL]);
+      // drain: every MMA issued by this thread completes before TMEM is freed
+      mma_commit(&bar[B_DRAIN]);
+      mbar_wait(&bar[B_DRAIN], 0, 4000000000ull);
+    }
+    __syncwarp();
+  } else if constexpr (KV == H2OKV_BF16) {
   if (warp == 0) {
     // ------------------------------------------------- producer of Q, K and token positions
     if (lane == 0) {
@@ -445,86 +694,96 @@ __global__ void __launch_bounds__(kThreads, 1)
         mbar_wait(&bar[B_VFULL0 + (kt & 1)], (kt >> 1) & 1, 4000000000ull);
     }
     __syncwarp();
-  } else if (warp == 1) {
-    // ------------------------------------------------------------------ MMA issuer
-    if (lane == 0) {
-      const uint32_t qa_addr = sbase + OFF_QA, qb_addr = sbase + OFF_QB, p_addr = sbase + OFF_P;
-      if (!mbar_wait(&bar[B_Q], 0, lim)) fail(p, aborted);
-      tc_fence_after();
-      // phase A: S_a, S_b = Q_a K^T, Q_b K^T into the column pair of the tile parity
-      for (int kt = 0; kt < n_kt && !aborted; ++kt) {
-        const int a = kt % kStagesA, u = kt & 1;
-        if (!mbar_wait(&bar[B_AFULL0 + a], (kt / kStagesA) & 1, lim)) { fail(p, aborted); break; }
-        if (kt >= 2 && !mbar_wait(&bar[B_SFREE0 + u], ((kt >> 1) - 1) & 1, lim)) {
-          fail(p, aborted);
-          break;
-        }
-        tc_fence_after();
-        const uint32_t k_addr = sbase + slot_a(a);
-#pragma unroll
-        for (int ks = 0; ks < D / 16; ++ks)
-          mma_bf16_ss(tmem + u * 256, kmajor_desc(qa_addr, ks), kmajor_desc(k_addr, ks),
-                      IDESC_K_MAJOR, ks > 0);
-        if (has_b) {
-#pragma unroll
-          for (int ks = 0; ks < D / 16; ++ks)
-            mma_bf16_ss(tmem + u * 256 + 128, kmajor_desc(qb_addr, ks), kmajor_desc(k_addr, ks),
-                        IDESC_K_MAJOR, ks > 0);
-        }
-        mma_commit(&bar[B_SFULL0 + u]);
-        mma_commit(&bar[B_AEMPTY0 + a]);
+  }
+  } else {
+    // --------------------------- loaders of quantized tiles (warps 0, 2, 3: 96 threads)
+    const int ct = warp == 0 ? lane : 32 * (warp - 1) + lane;
+    if (warp == 0 && lane == 0) {
+      mbar_expect_tx(&bar[B_Q], has_b ? 2 * kTileBytes : kTileBytes);
+      tma_load_3d(smem + OFF_QA, &q_map, &bar[B_Q], 0, i0_a, bhq_a);
+      tma_load_3d(smem + OFF_QA + kHalfBytes, &q_map, &bar[B_Q], 64, i0_a, bhq_a);
+      if (has_b) {
+        tma_load_3d(smem + OFF_QB, &q_map, &bar[B_Q], 0, i0_b, bhq_b);
+        tma_load_3d(smem + OFF_QB + kHalfBytes, &q_map, &bar[B_Q], 64, i0_b, bhq_b);
       }
-      mma_commit(&bar[B_VGO]);  // phase A K tiles in slots V0 / V1 no longer read
-      // every phase A TMEM read is done before phase B reuses the columns
-      if (!aborted && !mbar_wait(&bar[B_AFREE], 0, lim)) fail(p, aborted);
-      tc_fence_after();
-      // phase B.  S^T_x(kt) = K(kt) Q_x^T into columns 0 (a) / 128 (b);
-      // O_x += P_x(kt) V(kt) into columns 256 (a) / 384 (b).
-      auto issue_st = [&](int kt, bool tile_b) -> bool {
-        const int s = kt & 1;
-        if (!tile_b && !mbar_wait(&bar[B_KFULL0 + s], (kt >> 1) & 1, lim)) return false;
-        if (kt >= 1 && !mbar_wait(&bar[tile_b ? B_TFREEB : B_TFREEA], (kt - 1) & 1, lim))
-          return false;
-        tc_fence_after();
-        const uint32_t k_addr = sbase + (s ? OFF_K1 : OFF_K0);
-        const uint32_t q_addr = tile_b ? qb_addr : qa_addr;
-#pragma unroll
-        for (int ks = 0; ks < D / 16; ++ks)
-          mma_bf16_ss(tmem + (tile_b ? 128 : 0), kmajor_desc(k_addr, ks), kmajor_desc(q_addr, ks),
-                      IDESC_K_MAJOR, ks > 0);
-        mma_commit(&bar[tile_b ? B_TFULLB : B_TFULLA]);
-        if (tile_b || !has_b) mma_commit(&bar[B_KEMPTY0 + s]);  // K(kt) no longer read
-        return true;
-      };
-      auto issue_pv = [&](int kt, bool tile_b) -> bool {
-        if (!mbar_wait(&bar[tile_b ? B_PFULLB : B_PFULLA], kt & 1, lim)) return false;
-        if (!tile_b && !mbar_wait(&bar[B_VFULL0 + (kt & 1)], (kt >> 1) & 1, lim)) return false;
-        tc_fence_after();
-        const uint32_t v_addr = sbase + ((kt & 1) ? OFF_V1 : OFF_V0);
-#pragma unroll
-        for (int ks = 0; ks < BN / 16; ++ks)
-          mma_bf16_ss(tmem + (tile_b ? 384 : 256), mnmajor_desc(p_addr, ks),
-                      mnmajor_desc(v_addr, ks), IDESC_PV, (kt > 0 || ks > 0) ? 1u : 0u);
-        mma_commit(&bar[tile_b ? B_PFREEB : B_PFREEA]);
-        if (tile_b || !has_b) mma_commit(&bar[B_VEMPTY0 + (kt & 1)]);  // V(kt) no longer read
-        return true;
-      };
-      if (!aborted && !issue_st(0, false)) fail(p, aborted);
-      if (!aborted && has_b && !issue_st(0, true)) fail(p, aborted);
-      // S^T of the next tile is issued as soon as the softmax warps have read the
-      // current one out of TMEM (long before their P is ready), then the P V
-      // products of the current tile.
-      for (int kt = 0; kt < n_kt && !aborted; ++kt) {
-        if (kt + 1 < n_kt && !issue_st(kt + 1, false)) { fail(p, aborted); break; }
-        if (kt + 1 < n_kt && has_b && !issue_st(kt + 1, true)) { fail(p, aborted); break; }
-        if (!issue_pv(kt, false)) { fail(p, aborted); break; }
-        if (has_b && !issue_pv(kt, true)) { fail(p, aborted); break; }
-      }
-      mma_commit(&bar[B_OFULL]);
-      // drain: every MMA issued by this thread completes before TMEM is freed
-      mma_commit(&bar[B_DRAIN]);
-      mbar_wait(&bar[B_DRAIN], 0, 4000000000ull);
+      mbar_arrive(&bar[B_Q]);
     }
+    constexpr int RB = QTile<KV>::kRowBytes;
+    const int32_t *tpg = p.token_pos + (size_t)bg * p.N_C;
+    const uint8_t *kg = p.kq + (size_t)bg * p.N_C * RB;
+    const uint8_t *vg = p.vq + (size_t)bg * p.N_C * RB;
+    const __half *ksg = p.ksc + (size_t)bg * p.N_C;
+    const __half *vsg = p.vsc + (size_t)bg * p.N_C;
+    // L2 prefetch of a future tile's codes and scales (whole tiles only for the scales)
+    auto prefetch = [&](const uint8_t *codes, const __half *scales, int kt) {
+      if (ct != 0 || kt >= n_kt) return;
+      const int nv = min(BN, p.N_C - kt * BN);
+      bulk_prefetch_l2(codes + (size_t)kt * BN * RB, (uint32_t)(nv * RB));
+      const __half *sp = scales + (size_t)kt * BN;
+      if (nv == BN && (reinterpret_cast<uintptr_t>(sp) & 15u) == 0) bulk_prefetch_l2(sp, BN * 2);
+    };
+    // the stores of this warp reach the async proxy, then one arrival per warp
+    auto publish = [&](uint64_t *full) {
+      fence_proxy_async_smem();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(full);
+    };
+    // phase A: keys through the four-stage ring, with positions and scales
+    for (int kt = 0; kt < n_kt && !aborted; ++kt) {
+      const int stage = kt % kStagesA, n = kt / kStagesA;
+      if (n > 0 && !warp_wait(&bar[B_AEMPTY0 + stage], (n - 1) & 1, lim)) { fail(p, aborted); break; }
+      const int ahead = kt + kPrefetch;
+      if (ahead < n_kt) {
+        prefetch(kg, ksg, ahead);
+      } else {
+        prefetch(kg, ksg, ahead - n_kt);
+        prefetch(vg, vsg, ahead - n_kt);
+      }
+      const int nv = min(BN, p.N_C - kt * BN);
+      convert_tile<KV>(kg, nullptr, kt * BN, nv, sbase + slot_a(stage), false, ct);
+      write_rel(reinterpret_cast<float *>(smem + OFF_REL_A) + stage * BN, tpg, kt * BN, nv, p.P, ct,
+                kConvThreads);
+      float *ksd = reinterpret_cast<float *>(smem + OFF_KS_A) + stage * BN;
+      for (int e = ct; e < BN; e += kConvThreads)
+        ksd[e] = e < nv ? __half2float(ksg[kt * BN + e]) : 0.f;
+      publish(&bar[B_AFULL0 + stage]);
+    }
+    // phase B: K(s) then V(s - 1), the order in which the MMA issuer needs them
+    __half *ksb = reinterpret_cast<__half *>(smem + OFF_KSB);
+    for (int s2 = 0; s2 <= n_kt && !aborted; ++s2) {
+      if (s2 < n_kt) {
+        const int kt = s2, stage = kt & 1;
+        bool ok;
+        if (kt < 2) {
+          const int lu = last_use_a(stage, n_kt);
+          ok = lu < 0 || warp_wait(&bar[B_AEMPTY0 + stage], (lu / kStagesA) & 1, lim);
+        } else {
+          ok = warp_wait(&bar[B_KEMPTY0 + stage], ((kt >> 1) - 1) & 1, lim);
+        }
+        if (!ok) { fail(p, aborted); break; }
+        prefetch(kg, ksg, kt + kPrefetch);
+        const int nv = min(BN, p.N_C - kt * BN);
+        convert_tile<KV>(kg, nullptr, kt * BN, nv, sbase + (stage ? OFF_K1 : OFF_K0), false, ct);
+        write_rel(reinterpret_cast<float *>(tp_s) + stage * BN, tpg, kt * BN, nv, p.P, ct,
+                  kConvThreads);
+        for (int e = ct; e < BN; e += kConvThreads)
+          ksb[stage * BN + e] = e < nv ? ksg[kt * BN + e] : __float2half(0.f);
+        publish(&bar[B_KFULL0 + stage]);
+      }
+      if (s2 >= 1) {
+        const int kt = s2 - 1, vs = kt & 1, vn = kt >> 1;
+        // slots V0 / V1 serve as phase A K stages 2 / 3 until every phase A MMA is done
+        const bool ok = vn == 0 ? warp_wait(&bar[B_VGO], 0, lim)
+                                : warp_wait(&bar[B_VEMPTY0 + vs], (vn - 1) & 1, lim);
+        if (!ok) { fail(p, aborted); break; }
+        prefetch(vg, vsg, kt + kPrefetch);
+        const int nv = min(BN, p.N_C - kt * BN);
+        convert_tile<KV>(vg, vsg, kt * BN, nv, sbase + (vs ? OFF_V1 : OFF_V0), true, ct);
+        publish(&bar[B_VFULL0 + vs]);
+      }
+    }
+    // drain: the Q copy must land before exit
+    if (warp == 0 && lane == 0) mbar_wait(&bar[B_Q], 0, 4000000000ull);
     __syncwarp();
   }
   } else {
@@ -553,6 +812,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       tmem_ld32(sa + 64, *reinterpret_cast<uint32_t(*)[32]>(x + 64));
       tmem_ld32(sa + 96, *reinterpret_cast<uint32_t(*)[32]>(x + 96));
       tmem_wait_ld();
+      if constexpr (KV != H2OKV_BF16)
+        scale_row<BN>(x, reinterpret_cast<const float *>(smem + OFF_KS_A) + a * BN);
       if (masked) row_mask<BN>(x, rela, (float)(i0 + st));
       // S buffer and K stage (with its token positions) are free once read
       tc_fence_before();
@@ -587,6 +848,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (!warp_wait(&bar[B_KFULL0 + s], (kt >> 1) & 1, lim)) { fail(p, aborted); break; }
       tc_fence_after();
       const float relj = __int_as_float(tp_s[s * BN + st]);
+      // quantized caches: the slot's key scale joins the logit scale
+      const float c2j = KV == H2OKV_BF16
+                            ? c2
+                            : c2 * __half2float(reinterpret_cast<const __half *>(smem + OFF_KSB)[s * BN + st]);
       __syncwarp();
       if (lane == 0) mbar_arrive(&bar[B_KEMPTY0 + s]);
       // visible rows r of this tile: relj <= i0 + r, r < rmax
@@ -599,7 +864,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&bar[wg ? B_TFREEB : B_TFREEA]);
-      const float cs = slot_probs(r, lse_t, c2, rmin, rmax, full, pk);
+      const float cs = slot_probs(r, lse_t, c2j, rmin, rmax, full, pk);
       // the single P buffer goes a(kt) -> b(kt) -> a(kt+1): wait for the previous reader
       bool ok = true;
       if (wg == 1)
@@ -704,7 +969,8 @@ int encode_rows_map(CUtensorMap *map, const void *base, uint64_t rows, uint64_t 
 }  // namespace
 
 bool tc_path_supported(const h2okv_cache_desc &d) {
-  return d.head_dim == D && d.q_dtype == H2OKV_BF16 && d.kv_dtype == H2OKV_BF16;
+  return d.head_dim == D && d.q_dtype == H2OKV_BF16 &&
+         (d.kv_dtype == H2OKV_BF16 || d.kv_dtype == H2OKV_I8 || d.kv_dtype == H2OKV_I4);
 }
 
 void tc_plan(const h2okv_cache_desc &d, TcPlan *plan) {
@@ -713,50 +979,74 @@ void tc_plan(const h2okv_cache_desc &d, TcPlan *plan) {
   plan->max_splits = 0;
 }
 
+namespace {
+
+// Shared-memory opt-in and the register-allotment check, once per device and dtype.
+template <int KV>
+int prepare_kernel() {
+  static thread_local int ready_dev = -1;
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (ready_dev == dev) return H2OKV_OK;
+  cudaError_t e = cudaFuncSetAttribute(attn_tc_kernel<KV>,
+                                       cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmemBytes);
+  if (e != cudaSuccess)
+    return set_error(H2OKV_ERR_CUDA, "cudaFuncSetAttribute(attn_tc_kernel): %s",
+                     cudaGetErrorString(e));
+  cudaFuncAttributes fa;
+  e = cudaFuncGetAttributes(&fa, attn_tc_kernel<KV>);
+  if (e != cudaSuccess)
+    return set_error(H2OKV_ERR_CUDA, "cudaFuncGetAttributes(attn_tc_kernel): %s",
+                     cudaGetErrorString(e));
+  // the in-kernel register split assumes exactly this launch allotment
+  if (fa.numRegs != kLaunchRegs)
+    return set_error(H2OKV_ERR_UNSUPPORTED,
+                     "attn_tc_kernel built with %d registers per thread, expected %d", fa.numRegs,
+                     kLaunchRegs);
+  ready_dev = dev;
+  return H2OKV_OK;
+}
+
+template <int KV>
+int launch_kernel(int grid, const CUtensorMap &qmap, const CUtensorMap &kmap,
+                  const CUtensorMap &vmap, const TcParams &prm, cudaStream_t st) {
+  int rc = prepare_kernel<KV>();
+  if (rc) return rc;
+  attn_tc_kernel<KV><<<grid, kThreads, kSmemBytes, st>>>(qmap, kmap, vmap, prm);
+  return check_launch("attn_tc_kernel");
+}
+
+}  // namespace
+
 int launch_attn_tc(h2okv_cache *c, const void *q, int S, int64_t P, void *y, float *lse, float *w,
                    float *wq, cudaStream_t st) {
   const h2okv_cache_desc &d = c->desc;
   uint8_t *ws = reinterpret_cast<uint8_t *>(c->bufs.workspace);
+  const bool quant = d.kv_dtype != H2OKV_BF16;
   if (!c->tc.maps_ready) {
-    int rc = encode_rows_map(reinterpret_cast<CUtensorMap *>(c->tc.k_map), c->bufs.keys,
-                             (uint64_t)d.capacity, (uint64_t)d.batch * d.n_kv_heads);
-    if (rc) return rc;
-    rc = encode_rows_map(reinterpret_cast<CUtensorMap *>(c->tc.v_map), c->bufs.values,
-                         (uint64_t)d.capacity, (uint64_t)d.batch * d.n_kv_heads);
-    if (rc) return rc;
+    if (quant) {  // codes are read with plain loads: no maps for the cache
+      memset(c->tc.k_map, 0, sizeof(c->tc.k_map));
+      memset(c->tc.v_map, 0, sizeof(c->tc.v_map));
+    } else {
+      int rc = encode_rows_map(reinterpret_cast<CUtensorMap *>(c->tc.k_map), c->bufs.keys,
+                               (uint64_t)d.capacity, (uint64_t)d.batch * d.n_kv_heads);
+      if (rc) return rc;
+      rc = encode_rows_map(reinterpret_cast<CUtensorMap *>(c->tc.v_map), c->bufs.values,
+                           (uint64_t)d.capacity, (uint64_t)d.batch * d.n_kv_heads);
+      if (rc) return rc;
+    }
     c->tc.maps_ready = true;
   }
   CUtensorMap qmap;
   int rc = encode_rows_map(&qmap, q, (uint64_t)S, (uint64_t)d.batch * d.n_q_heads);
   if (rc) return rc;
 
-  static thread_local int configured_dev = -1;
-  int dev = 0;
-  cudaGetDevice(&dev);
-  if (configured_dev != dev) {
-    cudaError_t e = cudaFuncSetAttribute(attn_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         (int)kSmemBytes);
-    if (e != cudaSuccess)
-      return set_error(H2OKV_ERR_CUDA, "cudaFuncSetAttribute(attn_tc_kernel): %s",
-                       cudaGetErrorString(e));
-    configured_dev = dev;
-  }
-  static thread_local int checked_dev = -1;
-  if (checked_dev != dev) {
-    cudaFuncAttributes fa;
-    cudaError_t e = cudaFuncGetAttributes(&fa, attn_tc_kernel);
-    if (e != cudaSuccess)
-      return set_error(H2OKV_ERR_CUDA, "cudaFuncGetAttributes(attn_tc_kernel): %s",
-                       cudaGetErrorString(e));
-    // the in-kernel register split assumes exactly this launch allotment
-    if (fa.numRegs != kLaunchRegs)
-      return set_error(H2OKV_ERR_UNSUPPORTED,
-                       "attn_tc_kernel built with %d registers per thread, expected %d", fa.numRegs,
-                       kLaunchRegs);
-    checked_dev = dev;
-  }
   TcParams prm;
   prm.token_pos = c->bufs.token_pos;
+  prm.kq = reinterpret_cast<const uint8_t *>(c->bufs.keys);
+  prm.vq = reinterpret_cast<const uint8_t *>(c->bufs.values);
+  prm.ksc = reinterpret_cast<const __half *>(c->bufs.k_scales);
+  prm.vsc = reinterpret_cast<const __half *>(c->bufs.v_scales);
   prm.y = reinterpret_cast<__nv_bfloat16 *>(y);
   prm.lse_out = lse;
   prm.part_w = reinterpret_cast<float *>(ws + c->ws.part_w);
@@ -773,10 +1063,14 @@ int launch_attn_tc(h2okv_cache *c, const void *q, int S, int64_t P, void *y, flo
   prm.scale2 = (float)(1.4426950408889634 / 11.313708498984761);  // log2(e) / sqrt(128)
   prm.timeout_ns = c->wait_timeout_ns;
   const int grid = d.batch * d.n_kv_heads * prm.ctas_per_group;
-  attn_tc_kernel<<<grid, kThreads, kSmemBytes, st>>>(
-      qmap, *reinterpret_cast<const CUtensorMap *>(c->tc.k_map),
-      *reinterpret_cast<const CUtensorMap *>(c->tc.v_map), prm);
-  rc = check_launch("attn_tc_kernel");
+  const CUtensorMap &kmap = *reinterpret_cast<const CUtensorMap *>(c->tc.k_map);
+  const CUtensorMap &vmap = *reinterpret_cast<const CUtensorMap *>(c->tc.v_map);
+  switch (d.kv_dtype) {
+    case H2OKV_BF16: rc = launch_kernel<H2OKV_BF16>(grid, qmap, kmap, vmap, prm, st); break;
+    case H2OKV_I8: rc = launch_kernel<H2OKV_I8>(grid, qmap, kmap, vmap, prm, st); break;
+    case H2OKV_I4: rc = launch_kernel<H2OKV_I4>(grid, qmap, kmap, vmap, prm, st); break;
+    default: return set_error(H2OKV_ERR_UNSUPPORTED, "kv dtype on the tensor-core path");
+  }
   if (rc) return rc;
   dim3 rgrid((d.capacity + 255) / 256, d.batch * d.n_kv_heads);
   reduce_w_kernel<<<rgrid, 256, 0, st>>>(prm.part_w, w, wq, d.n_q_heads, d.n_kv_heads, prm.q_g,

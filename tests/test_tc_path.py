@@ -1,4 +1,4 @@
-"""Tensor-core path (head_dim 128, bf16 cache): parity with the oracle on every
+"""Tensor-core path (head_dim 128, bf16 / int8 / int4 cache): parity with the oracle on every
 chunk of small workloads whose shapes exercise the tiling -- several 128-slot
 and 128-row tiles, ragged slot and row tails, chunks shorter than a row tile,
 one-token chunks, a chunk as large as the cache, MHA and GQA, batch > 1."""
@@ -30,7 +30,23 @@ CASES = [
 ]
 
 
-@pytest.mark.parametrize("wl", CASES, ids=[w.name for w in CASES])
+# int8 / int4 caches: the loader warps dequantize while they load (exact integer
+# keys with the key scale on the logits, values multiplied by their scale)
+QCASES = [
+    tc("tc_i8_q4_c2048_s512", kv_dtype="i8"),
+    tc("tc_i4_q4_c2048_s512", kv_dtype="i4", seed=12),
+    tc("tc_i4_b2_q4_c1000_s300", kv_dtype="i4", B=2, Hq=4, Hk=1, capacity=1000, chunk=300,
+       seq_len=2100),
+    tc("tc_i8_s1", kv_dtype="i8", Hq=4, Hk=2, capacity=130, chunk=1, seq_len=150),
+    tc("tc_i8_s_eq_capacity", kv_dtype="i8", capacity=256, chunk=256, seq_len=768),
+    tc("tc_i4_mha_s300_odd_tiles", kv_dtype="i4", Hq=2, Hk=2, capacity=640, chunk=300,
+       seq_len=1500),
+    tc("tc_i8_s100_c700", kv_dtype="i8", Hq=4, Hk=1, capacity=700, chunk=100, seq_len=1200,
+       heavy_hitters=False),
+]
+
+
+@pytest.mark.parametrize("wl", CASES + QCASES, ids=[w.name for w in CASES + QCASES])
 def test_tc_workload_every_chunk(wl, cuda_device):
     run, n = run_and_check(wl, cuda_device)
     assert n == wl.n_chunks
