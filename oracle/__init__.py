@@ -16,11 +16,13 @@ path; see ``oracle/h2o_oracle.py`` for the per-function citations.
 from .h2o_oracle import (  # noqa: F401
     EMPTY_POS,
     QMAX,
+    SCORE_MODES,
     OracleCache,
     attend_head,
     dequantize_rows,
     pack_int4,
     quantize_rows,
     select_slots,
+    selection_keys,
     unpack_int4,
 )

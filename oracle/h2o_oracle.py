@@ -23,14 +23,25 @@ paper:
 * §3.1.1 "Variants of Heavy-Hitter Oracle": the H2O score of an entry is the
   cumulative sum of its attention weights while it sits in the cache (the
   paper's eq. (3), read as this); the entry with the lowest score is evicted.
-* §A.5.3: the buffer update is keys' = scatter(keys, index, key_new) (eq. (4)).
+* §A.5.3: the buffer update is keys' = scatter(keys, index, key_new) (eq. (4));
+  the delta encoding of an update is delta_key = gather(keys, index), from which
+  keys is rebuilt as scatter(keys', index, delta_key).
+* §3.1.1 also defines two score variants: h2o_orig selects the same slots for
+  every batch position by the score summed over b, and h2o_norm divides an
+  entry's score by its age t - t(b, h, j).
+* §3.2 / §A.5: eviction decisions are written to a replay log in the forward
+  pass and replayed by replay caches (insertion at given slots).
 * §2 "Related Work" and the library's feature list in §A.10: cache buffers may
   be quantized to 8 or 4 bits.  The paper gives no scheme; the oracle uses a
   symmetric per-(token, KV-head) absmax scheme with an fp16 scale (see
   ``quantize_rows``).
 
 Readings where the pages are silent (each one is listed again in the design
-notes): the GQA reduction of the summed weights is a SUM over the group's query
+notes): h2o_norm's time t (undefined in the pages) is P, the position of the
+chunk's first token, so an entry's age P - t(b, h, j) >= 1 counts the query
+positions that could attend to it; the normalised key is the float32 quotient
+float32(score) / float32(age), the same precision the kernel decides in;
+h2o_orig's summed score is accumulated in float32 in batch order; the GQA reduction of the summed weights is a SUM over the group's query
 heads; ties between equal scores go to the lowest slot index; chosen slots are
 filled in ascending slot order with the chunk's tokens in order; a new slot
 starts with score 0 and then accumulates its own chunk's weights; empty slots
@@ -138,6 +149,35 @@ def select_slots(scores: np.ndarray, token_pos: np.ndarray, n_new: int) -> np.nd
     return np.array(sorted(chosen), dtype=np.int64)
 
 
+SCORE_MODES = ("h2o", "h2o_norm", "h2o_orig")
+
+
+def selection_keys(mode: str, scores: np.ndarray, token_pos: np.ndarray, P: int) -> np.ndarray:
+    """Per-slot selection key [B, H_k, N_C] (float32) of a score variant (§3.1.1).
+
+    h2o:      the cumulative score itself.
+    h2o_norm: score / (t - t(b, h, j)) with t = P (a reading), in float32; empty
+              slots are taken first whatever their key, so their key is 0.
+    h2o_orig: sum over batch positions b of the scores (float32, b in order); the
+              same key, hence the same slots, for every b.
+    """
+    scores = np.asarray(scores, np.float32)
+    if mode == "h2o":
+        return scores.copy()
+    if mode == "h2o_norm":
+        occupied = token_pos != EMPTY_POS
+        age = np.where(occupied, P - np.asarray(token_pos, np.int64), 1).astype(np.float32)
+        if np.any(age[occupied] < 1):
+            raise ValueError("an occupied slot holds a token at or after the chunk start")
+        return np.where(occupied, scores / age, np.float32(0)).astype(np.float32)
+    if mode == "h2o_orig":
+        total = np.zeros(scores.shape[1:], np.float32)
+        for b in range(scores.shape[0]):
+            total = (total + scores[b]).astype(np.float32)
+        return np.broadcast_to(total, scores.shape).copy()
+    raise ValueError(f"unknown score mode {mode!r}")
+
+
 # --------------------------------------------------------------------------- #
 # SDPA with the token-position mask and summed weights (§A.1, §A.7).
 # --------------------------------------------------------------------------- #
@@ -217,23 +257,59 @@ class OracleCache:
         return self.v_store[b, g].astype(np.float64)
 
     # -- H2O score update, selection and overwrite ---------------------------
-    def evict_insert(self, w_prev, k_new, v_new, S, P):
+    def evict_insert(self, w_prev, k_new, v_new, S, P, mode="h2o", slots=None, delta=False):
         """Fold the previous chunk's summed weights into the scores, choose S
         slots per (b, h_k) and overwrite them with the chunk's keys/values.
 
         w_prev: [B, H_k, N_C] or None.  k_new, v_new: [B, H_k, S, d] float32
         values of the storage type (bf16-rounded for bf16/i8/i4 caches).
-        Returns the chosen slots [B, H_k, S] (ascending per (b, h_k)).
+        mode: the score variant that ranks occupied slots (``SCORE_MODES``).
+        slots: [B, H_k, S] slots to write instead of choosing them (replay of a
+        logged decision, §A.5); each (b, h_k) row must hold distinct slots.
+        delta: also return the rows the update overwrites (§A.5.3's
+        delta_key = gather(keys, index)), as a dict of arrays indexed like the
+        chunk: "keys", "values" (stored values, or codes and "k_scales",
+        "v_scales" for quantized caches) and "token_pos".
+        Returns the slots [B, H_k, S] (ascending per (b, h_k) when chosen here),
+        and the delta dict when ``delta`` is set.
         """
         if w_prev is not None:
             self.scores = (self.scores + np.asarray(w_prev, np.float32)).astype(np.float32)
-        slots = np.zeros((self.B, self.Hk, S), np.int64)
+        out = np.zeros((self.B, self.Hk, S), np.int64)
+        d = None
+        if delta:
+            shape = (self.B, self.Hk, S)
+            if self.quantized:
+                d = {"keys": np.zeros(shape + (self.d,), np.int8),
+                     "values": np.zeros(shape + (self.d,), np.int8),
+                     "k_scales": np.zeros(shape, np.float16), "v_scales": np.zeros(shape, np.float16)}
+            else:
+                d = {"keys": np.zeros(shape + (self.d,), np.float32),
+                     "values": np.zeros(shape + (self.d,), np.float32)}
+            d["token_pos"] = np.zeros(shape, np.int64)
         if S == 0:
-            return slots
+            return (out, d) if delta else out
+        if slots is None:
+            keys = selection_keys(mode, self.scores, self.token_pos, P)
         for b in range(self.B):
             for g in range(self.Hk):
-                chosen = select_slots(self.scores[b, g], self.token_pos[b, g], S)
-                slots[b, g] = chosen
+                if slots is None:
+                    chosen = select_slots(keys[b, g], self.token_pos[b, g], S)
+                else:
+                    chosen = np.asarray(slots[b, g], np.int64)
+                    if len(set(chosen.tolist())) != S or chosen.min() < 0 or chosen.max() >= self.N_C:
+                        raise ValueError("replayed slots must be distinct and inside the cache")
+                out[b, g] = chosen
+                if delta:
+                    if self.quantized:
+                        d["keys"][b, g] = self.k_codes[b, g, chosen]
+                        d["values"][b, g] = self.v_codes[b, g, chosen]
+                        d["k_scales"][b, g] = self.k_scales[b, g, chosen]
+                        d["v_scales"][b, g] = self.v_scales[b, g, chosen]
+                    else:
+                        d["keys"][b, g] = self.k_store[b, g, chosen]
+                        d["values"][b, g] = self.v_store[b, g, chosen]
+                    d["token_pos"][b, g] = self.token_pos[b, g, chosen]
                 kk = np.asarray(k_new[b, g], np.float32)
                 vv = np.asarray(v_new[b, g], np.float32)
                 if self.quantized:
@@ -249,7 +325,24 @@ class OracleCache:
                 self.token_pos[b, g, chosen] = P + np.arange(S)
                 self.scores[b, g, chosen] = 0.0
         self.n_filled = min(self.N_C, self.n_filled + S)
-        return slots
+        return (out, d) if delta else out
+
+    def restore(self, slots, d):
+        """Undo an update from its delta encoding: scatter the overwritten rows and
+        token positions back into ``slots`` (the recurrence of §A.5.3 played
+        backwards).  Scores are not restored."""
+        for b in range(self.B):
+            for g in range(self.Hk):
+                chosen = np.asarray(slots[b, g], np.int64)
+                if self.quantized:
+                    self.k_codes[b, g, chosen] = d["keys"][b, g]
+                    self.v_codes[b, g, chosen] = d["values"][b, g]
+                    self.k_scales[b, g, chosen] = d["k_scales"][b, g]
+                    self.v_scales[b, g, chosen] = d["v_scales"][b, g]
+                else:
+                    self.k_store[b, g, chosen] = d["keys"][b, g]
+                    self.v_store[b, g, chosen] = d["values"][b, g]
+                self.token_pos[b, g, chosen] = d["token_pos"][b, g]
 
     # -- SDPA over the cache with summed weights -----------------------------
     def attend(self, q, S, P):

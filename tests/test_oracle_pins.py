@@ -27,7 +27,7 @@ import pytest
 from scipy.special import logsumexp, softmax
 
 import oracle
-from oracle import EMPTY_POS, OracleCache, attend_head, quantize_rows, select_slots
+from oracle import EMPTY_POS, OracleCache, attend_head, quantize_rows, select_slots, selection_keys
 from oracle import h2o_oracle as ho
 
 GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
@@ -383,3 +383,171 @@ def test_t3_selection_brute_force_with(sel=select_slots):
         scores = rng.integers(0, 2, n).astype(np.float32)
         tp = np.arange(n)
         np.testing.assert_array_equal(sel(scores, tp, s), brute_force_select(scores, tp, s))
+
+
+# --------------------------------------------------------------------------- #
+# Score variants (§3.1.1), replay of logged decisions and the delta encoding of
+# an update (§A.5.3).
+# --------------------------------------------------------------------------- #
+def _golden_modes():
+    import json
+    import os
+    with open(os.path.join(os.path.dirname(__file__), "golden", "h2o_score_modes.json")) as f:
+        return json.load(f)
+
+
+def _tp(vals):
+    return np.array([EMPTY_POS if v == "empty" else v for v in vals], np.int64)
+
+
+def _select_mode(mode, scores, token_pos, P, S):
+    """Slots chosen by the oracle's cache for one chunk of a given variant."""
+    scores = np.asarray(scores, np.float32)
+    B = scores.shape[0]
+    n_c = scores.shape[-1]
+    c = OracleCache(B, 1, 1, 2, n_c, "f32")
+    c.load_state(token_pos=np.broadcast_to(token_pos, (B, 1, n_c)).copy(),
+                 scores=scores.reshape(B, 1, n_c), n_filled=n_c,
+                 keys=np.zeros((B, 1, n_c, 2), np.float32), values=np.zeros((B, 1, n_c, 2), np.float32))
+    kn = np.zeros((B, 1, S, 2), np.float32)
+    return c.evict_insert(None, kn, kn, S, P, mode=mode)[:, 0]
+
+
+def test_t7_score_variants_hand_derived():
+    g = _golden_modes()
+    for ex in g["h2o_norm"]:
+        tp = _tp(ex["token_pos"])
+        sc = np.array([ex["scores"]], np.float32)
+        keys = selection_keys("h2o_norm", sc[:, None], tp[None, None], ex["P"])[0, 0]
+        for j, k in enumerate(ex["keys"]):
+            if k != "empty":
+                assert keys[j] == np.float32(float(_frac(k)))
+        assert _select_mode("h2o_norm", sc, tp, ex["P"], ex["S"])[0].tolist() == ex["slots"]
+        assert _select_mode("h2o", sc, tp, ex["P"], ex["S"])[0].tolist() == ex["slots_h2o"]
+    for ex in g["h2o_orig"]:
+        tp = _tp(ex["token_pos"])
+        sc = np.array(ex["scores"], np.float32)
+        got = _select_mode("h2o_orig", sc, tp, 100, ex["S"])
+        for b in range(sc.shape[0]):
+            assert got[b].tolist() == ex["slots"]
+        per_b = _select_mode("h2o", sc, tp, 100, ex["S"])
+        assert [r.tolist() for r in per_b] == ex["slots_h2o"]
+
+
+def test_t7_score_variants_special_cases():
+    rng = np.random.default_rng(17)
+    for _ in range(50):
+        n_c, S = 12, 4
+        sc = rng.permutation(n_c).astype(np.float32)[None] + 1.0  # distinct scores
+        # every entry of the same age (a power of two): h2o_norm orders like h2o
+        tp = np.full(n_c, 3, np.int64)
+        a = _select_mode("h2o_norm", sc, tp, 3 + 8, S)
+        b = _select_mode("h2o", sc, tp, 3 + 8, S)
+        assert np.array_equal(a, b)
+        # one batch position, or identical rows: h2o_orig orders like h2o
+        assert np.array_equal(_select_mode("h2o_orig", sc, np.arange(n_c), 50, S),
+                              _select_mode("h2o", sc, np.arange(n_c), 50, S))
+        two = np.concatenate([sc, sc])
+        assert np.array_equal(_select_mode("h2o_orig", two, np.arange(n_c), 50, S)[0],
+                              _select_mode("h2o", sc, np.arange(n_c), 50, S)[0])
+
+
+def _brute(keys64, token_pos, S):
+    best = None
+    for sub in itertools.combinations(range(len(keys64)), S):
+        lst = sorted(((0, 0.0, j) if token_pos[j] == EMPTY_POS else (1, keys64[j], j)) for j in sub)
+        if best is None or lst < best[0]:
+            best = (lst, sub)
+    return sorted(best[1])
+
+
+def test_t7_score_variants_brute_force():
+    rng = np.random.default_rng(5)
+    for _ in range(200):
+        n_c, P = int(rng.integers(3, 9)), 40
+        S = int(rng.integers(1, n_c + 1))
+        tp = rng.integers(0, P, n_c).astype(np.int64)
+        tp[rng.random(n_c) < 0.2] = EMPTY_POS
+        # small integer scores: float32 sums are exact, quotients are compared in float64
+        sc = rng.integers(0, 6, (2, n_c)).astype(np.float32)
+        occ = tp != EMPTY_POS
+        norm64 = np.where(occ, sc[0].astype(np.float64) / np.where(occ, P - tp, 1), 0.0)
+        # compare where float32 rounding merges no two distinct float64 keys
+        if len(set(norm64[occ].tolist())) == len(set(np.float32(norm64[occ]).tolist())):
+            assert _select_mode("h2o_norm", sc[:1], tp, P, S)[0].tolist() == _brute(norm64, tp, S)
+        orig64 = sc[0].astype(np.float64) + sc[1]
+        got = _select_mode("h2o_orig", sc, tp, P, S)
+        assert got[0].tolist() == got[1].tolist() == _brute(orig64, tp, S)
+
+
+def test_t8_replay_reproduces_the_cache():
+    rng = np.random.default_rng(9)
+    for kv in ("f32", "i8", "i4"):
+        B, Hq, Hk, d, n_c = 2, 4, 2, 16, 20
+        a = OracleCache(B, Hq, Hk, d, n_c, kv)
+        r = OracleCache(B, Hq, Hk, d, n_c, kv)
+        P = 0
+        w = None
+        for S in (8, 8, 6, 8, 5, 8):
+            kn = _rand(rng, (B, Hk, S, d))
+            vn = _rand(rng, (B, Hk, S, d))
+            q = _rand(rng, (B, Hq, S, d))
+            slots = a.evict_insert(w, kn, vn, S, P, mode="h2o_norm" if P else "h2o")
+            r.evict_insert(w, kn, vn, S, P, slots=slots)
+            for name in ("token_pos", "scores") + (("k_codes", "v_codes", "k_scales", "v_scales")
+                                                    if kv != "f32" else ("k_store", "v_store")):
+                assert np.array_equal(getattr(a, name), getattr(r, name)), name
+            _, _, w, _ = a.attend(q, S, P)
+            w = w.astype(np.float32)
+            P += S
+
+
+def test_t9_delta_encoding_round_trip():
+    rng = np.random.default_rng(21)
+    for kv in ("f32", "bf16", "i8", "i4"):
+        B, Hq, Hk, d, n_c = 2, 2, 2, 8, 12
+        c = OracleCache(B, Hq, Hk, d, n_c, kv)
+        P = 0
+        w = None
+        for S in (6, 6, 5, 6, 6):
+            names = ("token_pos",) + (("k_codes", "v_codes", "k_scales", "v_scales")
+                                      if kv in ("i8", "i4") else ("k_store", "v_store"))
+            before = {n: getattr(c, n).copy() for n in names}
+            kn = _rand(rng, (B, Hk, S, d))
+            vn = _rand(rng, (B, Hk, S, d))
+            slots, dl = c.evict_insert(w, kn, vn, S, P, delta=True)
+            # the delta rows are the overwritten rows: gather(keys, index)
+            for b in range(B):
+                for g in range(Hk):
+                    src = "k_codes" if kv in ("i8", "i4") else "k_store"
+                    assert np.array_equal(dl["keys"][b, g], before[src][b, g, slots[b, g]])
+                    assert np.array_equal(dl["token_pos"][b, g], before["token_pos"][b, g, slots[b, g]])
+            after = {n: getattr(c, n).copy() for n in names}
+            c.restore(slots, dl)
+            for n in names:
+                assert np.array_equal(getattr(c, n), before[n]), n
+            # redo the update (the cache moves on)
+            c.restore(slots, {"keys": after[names[1]][np.arange(B)[:, None, None], np.arange(Hk)[None, :, None], slots],
+                              "values": after[names[2]][np.arange(B)[:, None, None], np.arange(Hk)[None, :, None], slots],
+                              "token_pos": after["token_pos"][np.arange(B)[:, None, None], np.arange(Hk)[None, :, None], slots],
+                              **({"k_scales": after["k_scales"][np.arange(B)[:, None, None], np.arange(Hk)[None, :, None], slots],
+                                  "v_scales": after["v_scales"][np.arange(B)[:, None, None], np.arange(Hk)[None, :, None], slots]}
+                                 if kv in ("i8", "i4") else {})})
+            for n in names:
+                assert np.array_equal(getattr(c, n), after[n]), n
+            q = _rand(rng, (B, Hq, S, d))
+            _, _, w, _ = c.attend(q, S, P)
+            w = w.astype(np.float32)
+            P += S
+
+
+def test_t7_planted_age_off_by_one_is_caught(monkeypatch):
+    import oracle.h2o_oracle as ho
+    good = ho.selection_keys
+
+    def age_plus_one(mode, scores, token_pos, P):
+        return good(mode, scores, token_pos, P + 1)
+
+    monkeypatch.setattr(ho, "selection_keys", age_plus_one)
+    with pytest.raises(AssertionError):
+        test_t7_score_variants_hand_derived()
