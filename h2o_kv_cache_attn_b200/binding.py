@@ -25,7 +25,10 @@ BUF_NAMES = ("keys", "values", "k_scales", "v_scales", "token_pos", "scores", "w
 EXPORTED = ("kv_cache_query_sizes", "kv_cache_create", "kv_cache_reset", "kv_cache_destroy",
             "kv_cache_get_fill", "kv_cache_set_fill", "kv_cache_quantize", "h2o_evict_insert",
             "attn_chunk_with_scoresum", "kv_cache_device_status", "kv_cache_set_wait_timeout",
-            "attn_chunk_with_scoresum_noalloc", "h2okv_last_error", "h2okv_abi_version")
+            "attn_chunk_with_scoresum_noalloc", "h2okv_last_error", "h2okv_abi_version",
+            "kv_cache_set_score_mode", "h2o_evict_insert_delta", "h2o_insert_at",
+            "kv_cache_restore")
+SCORE_MODE = {"h2o": 0, "h2o_norm": 1, "h2o_orig": 2}
 
 
 class H2OKVError(RuntimeError):
@@ -39,6 +42,12 @@ class CacheDesc(ctypes.Structure):
                 ("n_kv_heads", ctypes.c_int32), ("head_dim", ctypes.c_int32),
                 ("capacity", ctypes.c_int32), ("max_chunk", ctypes.c_int32),
                 ("q_dtype", ctypes.c_int32), ("kv_dtype", ctypes.c_int32)]
+
+
+class Delta(ctypes.Structure):
+    _fields_ = [("keys", ctypes.c_void_p), ("values", ctypes.c_void_p),
+                ("k_scales", ctypes.c_void_p), ("v_scales", ctypes.c_void_p),
+                ("token_pos", ctypes.c_void_p)]
 
 
 class CacheBuffers(ctypes.Structure):
@@ -80,6 +89,11 @@ def load() -> ctypes.CDLL:
         "kv_cache_set_wait_timeout": (ctypes.c_int, [vp, ctypes.c_uint64]),
         "attn_chunk_with_scoresum_noalloc": (ctypes.c_int, [ctypes.POINTER(CacheDesc), vp, vp, vp, vp,
                                                             vp, vp, i32, i64, vp, vp, vp, vp, vp]),
+        "kv_cache_set_score_mode": (ctypes.c_int, [vp, i32]),
+        "h2o_evict_insert_delta": (ctypes.c_int, [vp, vp, vp, vp, i32, i64, vp,
+                                                  ctypes.POINTER(Delta), vp]),
+        "h2o_insert_at": (ctypes.c_int, [vp, vp, vp, vp, i32, i64, vp, ctypes.POINTER(Delta), vp]),
+        "kv_cache_restore": (ctypes.c_int, [vp, vp, i32, ctypes.POINTER(Delta), vp]),
         "h2okv_last_error": (ctypes.c_char_p, []),
         "h2okv_abi_version": (i32, []),
     }
@@ -155,6 +169,33 @@ def kv_cache_quantize(kv_dtype: str, x: torch.Tensor, codes: torch.Tensor, scale
 def h2o_evict_insert(handle, w_prev, k_new, v_new, S: int, P: int, slots_out=None, stream=None):
     _check(load().h2o_evict_insert(handle, _ptr(w_prev), _ptr(k_new), _ptr(v_new), int(S), int(P),
                                    _ptr(slots_out), _stream(stream)))
+
+
+def kv_cache_set_score_mode(handle, mode: str):
+    _check(load().kv_cache_set_score_mode(handle, SCORE_MODE[mode]))
+
+
+def _delta(d):
+    """A Delta struct from a dict of tensors (keys, values, token_pos[, k_scales, v_scales])."""
+    if d is None:
+        return None
+    return ctypes.byref(Delta(_ptr(d["keys"]), _ptr(d["values"]), _ptr(d.get("k_scales")),
+                              _ptr(d.get("v_scales")), _ptr(d["token_pos"])))
+
+
+def h2o_evict_insert_delta(handle, w_prev, k_new, v_new, S: int, P: int, slots_out, delta,
+                           stream=None):
+    _check(load().h2o_evict_insert_delta(handle, _ptr(w_prev), _ptr(k_new), _ptr(v_new), int(S),
+                                         int(P), _ptr(slots_out), _delta(delta), _stream(stream)))
+
+
+def h2o_insert_at(handle, w_prev, k_new, v_new, S: int, P: int, slots_in, delta=None, stream=None):
+    _check(load().h2o_insert_at(handle, _ptr(w_prev), _ptr(k_new), _ptr(v_new), int(S), int(P),
+                                _ptr(slots_in), _delta(delta), _stream(stream)))
+
+
+def kv_cache_restore(handle, slots, S: int, delta, stream=None):
+    _check(load().kv_cache_restore(handle, _ptr(slots), int(S), _delta(delta), _stream(stream)))
 
 
 def attn_chunk_with_scoresum(handle, q, S: int, P: int, y_out, lse_out, w_out, wq_out=None,
@@ -277,6 +318,43 @@ class KVCache:
                     raise ValueError(f"k_new/v_new must be {want} {self.shape.q_dtype} on {self.device}")
         self._check_w(w_prev, allow_none=True)
         h2o_evict_insert(self.handle, w_prev, k_new, v_new, S, P, slots_out, stream)
+
+    def set_score_mode(self, mode: str):
+        kv_cache_set_score_mode(self.handle, mode)
+
+    def delta_buffers(self, S):
+        """Device buffers for the delta encoding of one chunk of S rows."""
+        s = self.shape
+        B, Hk = s.batch, s.n_kv_heads
+        row = self.keys.shape[-1]
+        d = {"keys": torch.empty((B, Hk, S, row), dtype=self.keys.dtype, device=self.device),
+             "values": torch.empty((B, Hk, S, row), dtype=self.keys.dtype, device=self.device),
+             "token_pos": torch.empty((B, Hk, S), dtype=torch.int32, device=self.device)}
+        if self.k_scales is not None:
+            d["k_scales"] = torch.empty((B, Hk, S), dtype=torch.float16, device=self.device)
+            d["v_scales"] = torch.empty((B, Hk, S), dtype=torch.float16, device=self.device)
+        return d
+
+    def evict_insert_delta(self, w_prev, k_new, v_new, S, P, slots_out, delta, stream=None):
+        self._check_kv(k_new, v_new, S)
+        self._check_w(w_prev, allow_none=True)
+        h2o_evict_insert_delta(self.handle, w_prev, k_new, v_new, S, P, slots_out, delta, stream)
+
+    def insert_at(self, w_prev, k_new, v_new, S, P, slots_in, delta=None, stream=None):
+        self._check_kv(k_new, v_new, S)
+        self._check_w(w_prev, allow_none=True)
+        if slots_in.dtype != torch.int32 or tuple(slots_in.shape) != (self.shape.batch, self.shape.n_kv_heads, S):
+            raise ValueError("slots_in must be int32 [B, H_k, S]")
+        h2o_insert_at(self.handle, w_prev, k_new, v_new, S, P, slots_in, delta, stream)
+
+    def restore(self, slots, S, delta, stream=None):
+        kv_cache_restore(self.handle, slots, S, delta, stream)
+
+    def _check_kv(self, k_new, v_new, S):
+        want = (self.shape.batch, self.shape.n_kv_heads, S, self.shape.head_dim)
+        for t in (k_new, v_new):
+            if tuple(t.shape) != want or t.dtype != _TORCH_Q[self.shape.q_dtype] or t.device != self.device:
+                raise ValueError(f"k_new/v_new must be {want} {self.shape.q_dtype} on {self.device}")
 
     def attend(self, q, S, P, y_out, lse_out, w_out, wq_out=None, stream=None):
         s = self.shape

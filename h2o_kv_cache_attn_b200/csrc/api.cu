@@ -153,6 +153,7 @@ int kv_cache_create(const h2okv_cache_desc *desc, const h2okv_cache_buffers *buf
   tc_plan(*desc, &c->tc);
   c->tc.maps_ready = false;
   c->wait_timeout_ns = kDefaultWaitTimeoutNs;
+  c->score_mode = H2OKV_SCORE_H2O;
   layout(*desc, c->tc, &c->ws);
   // The attention kernels read every slot and mask the empty ones arithmetically,
   // which needs finite values there: start from zeroed rows and scales.
@@ -263,10 +264,96 @@ int h2o_evict_insert(h2okv_cache *c, const float *w_prev, const void *k_new, con
   if (misaligned(k_new, 16) || misaligned(v_new, 16) || misaligned(w_prev, 4))
     return set_error(H2OKV_ERR_INVALID_ARG, "k_new and v_new must be 16-byte aligned");
   if (S == 0 && !w_prev) return H2OKV_OK;
-  int rc = launch_evict_insert(c, w_prev, k_new, v_new, S, P, slots_out, (cudaStream_t)stream);
+  int rc = launch_evict_insert(c, w_prev, k_new, v_new, S, P, slots_out, nullptr, nullptr,
+                               (cudaStream_t)stream);
   if (rc) return rc;
   c->n_filled = c->n_filled + S > c->desc.capacity ? c->desc.capacity : c->n_filled + S;
   return H2OKV_OK;
+}
+
+int kv_cache_set_score_mode(h2okv_cache *c, int32_t mode) {
+  g_err[0] = 0;
+  if (!c) return set_error(H2OKV_ERR_INVALID_ARG, "cache is NULL");
+  if (mode != H2OKV_SCORE_H2O && mode != H2OKV_SCORE_H2O_NORM && mode != H2OKV_SCORE_H2O_ORIG)
+    return set_error(H2OKV_ERR_INVALID_ARG, "unknown score mode %d", mode);
+  c->score_mode = mode;
+  return H2OKV_OK;
+}
+
+// Delta buffers: rows, token positions, and scales for quantized caches.
+static int check_delta(const h2okv_cache *c, const h2okv_delta *dl) {
+  if (!dl || !dl->keys || !dl->values || !dl->token_pos)
+    return set_error(H2OKV_ERR_INVALID_ARG, "delta keys, values and token_pos are required");
+  const bool quant = c->desc.kv_dtype == H2OKV_I8 || c->desc.kv_dtype == H2OKV_I4;
+  if (quant && (!dl->k_scales || !dl->v_scales))
+    return set_error(H2OKV_ERR_INVALID_ARG, "delta scales are required for I8/I4 caches");
+  if (misaligned(dl->keys, 16) || misaligned(dl->values, 16) || misaligned(dl->token_pos, 16) ||
+      (quant && (misaligned(dl->k_scales, 16) || misaligned(dl->v_scales, 16))))
+    return set_error(H2OKV_ERR_INVALID_ARG, "delta buffers must be 16-byte aligned");
+  return H2OKV_OK;
+}
+
+static int check_chunk(const h2okv_cache *c, const void *k_new, const void *v_new, int32_t S,
+                       int64_t P, const float *w_prev) {
+  if (S < 1 || S > c->desc.max_chunk || S > c->desc.capacity)
+    return set_error(H2OKV_ERR_INVALID_ARG, "S = %d outside [1, min(max_chunk %d, capacity %d)]",
+                     S, c->desc.max_chunk, c->desc.capacity);
+  if (P < 0 || P + S >= (int64_t)INT32_MAX)
+    return set_error(H2OKV_ERR_INVALID_ARG, "P = %lld out of range for int32 token positions",
+                     (long long)P);
+  if (!k_new || !v_new) return set_error(H2OKV_ERR_INVALID_ARG, "k_new and v_new are required");
+  if (misaligned(k_new, 16) || misaligned(v_new, 16) || misaligned(w_prev, 4))
+    return set_error(H2OKV_ERR_INVALID_ARG, "k_new and v_new must be 16-byte aligned");
+  return H2OKV_OK;
+}
+
+int h2o_evict_insert_delta(h2okv_cache *c, const float *w_prev, const void *k_new,
+                           const void *v_new, int32_t S, int64_t P, int32_t *slots_out,
+                           const h2okv_delta *delta, void *stream) {
+  g_err[0] = 0;
+  if (!c) return set_error(H2OKV_ERR_INVALID_ARG, "cache is NULL");
+  int rc = check_chunk(c, k_new, v_new, S, P, w_prev);
+  if (rc) return rc;
+  if (!slots_out) return set_error(H2OKV_ERR_INVALID_ARG, "slots_out is required with a delta");
+  rc = check_delta(c, delta);
+  if (rc) return rc;
+  rc = launch_evict_insert(c, w_prev, k_new, v_new, S, P, slots_out, nullptr, delta,
+                           (cudaStream_t)stream);
+  if (rc) return rc;
+  c->n_filled = c->n_filled + S > c->desc.capacity ? c->desc.capacity : c->n_filled + S;
+  return H2OKV_OK;
+}
+
+int h2o_insert_at(h2okv_cache *c, const float *w_prev, const void *k_new, const void *v_new,
+                  int32_t S, int64_t P, const int32_t *slots_in, const h2okv_delta *delta,
+                  void *stream) {
+  g_err[0] = 0;
+  if (!c) return set_error(H2OKV_ERR_INVALID_ARG, "cache is NULL");
+  int rc = check_chunk(c, k_new, v_new, S, P, w_prev);
+  if (rc) return rc;
+  if (!slots_in) return set_error(H2OKV_ERR_INVALID_ARG, "slots_in is required");
+  if (delta) {
+    rc = check_delta(c, delta);
+    if (rc) return rc;
+  }
+  rc = launch_evict_insert(c, w_prev, k_new, v_new, S, P, nullptr, slots_in, delta,
+                           (cudaStream_t)stream);
+  if (rc) return rc;
+  c->n_filled = c->n_filled + S > c->desc.capacity ? c->desc.capacity : c->n_filled + S;
+  return H2OKV_OK;
+}
+
+int kv_cache_restore(h2okv_cache *c, const int32_t *slots, int32_t S, const h2okv_delta *delta,
+                     void *stream) {
+  g_err[0] = 0;
+  if (!c) return set_error(H2OKV_ERR_INVALID_ARG, "cache is NULL");
+  if (S < 0 || S > c->desc.max_chunk || S > c->desc.capacity)
+    return set_error(H2OKV_ERR_INVALID_ARG, "S = %d outside [0, min(max_chunk, capacity)]", S);
+  if (S == 0) return H2OKV_OK;
+  if (!slots) return set_error(H2OKV_ERR_INVALID_ARG, "slots is required");
+  int rc = check_delta(c, delta);
+  if (rc) return rc;
+  return launch_restore(c, slots, S, delta, (cudaStream_t)stream);
 }
 
 int attn_chunk_with_scoresum(h2okv_cache *c, const void *q, int32_t S, int64_t P, void *y_out,

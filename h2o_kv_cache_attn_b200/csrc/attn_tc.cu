@@ -33,8 +33,9 @@
 // pipe compute the next logits while the softmax warps turn the current ones
 // into P.
 // Quantized caches (int8 / int4 codes with one fp16 scale per slot): warps 0, 2
-// and 3 replace the TMA producers and dequantize while they load (see
-// convert_tile): key tiles become exact bf16 integers and the key scale s_j
+// and 3 replace the TMA producers: one thread stages each tile of codes by a bulk
+// copy, all 96 dequantize it in place (see convert_i8 / convert_i4): key tiles
+// become exact bf16 integers and the key scale s_j
 // multiplies the logits of slot j (a column scale of S in phase A, a per-thread
 // factor in phase B), so scores and summed weights see the stored keys exactly;
 // value tiles are stored as bf16(code * scale).
@@ -60,7 +61,7 @@ constexpr int D = 128;         // head dim
 constexpr int kThreads = 384;  // 4 control warps + 2 softmax warpgroups
 constexpr int kPrefetch = 4;   // K / V tiles requested into L2 this many loads ahead
 constexpr int kRelFar = 1 << 20;  // relative position of a slot no row of the chunk sees
-constexpr float kMaskBias = 1073741824.f;  // 2^30: subtracted from a masked logit
+constexpr float kMaskBias = 1073741824.f;  // 2^30: a masked logit drops by this (base-2 units)
 // Register split between the warpgroups.  The launch allots 168 registers per
 // thread (384 x 168 = 64512); the control warpgroup drops to 88 and the two
 // softmax warpgroups rise to 208: 128 x 88 + 256 x 208 = 64512.
@@ -82,7 +83,7 @@ constexpr uint32_t OFF_LSE = OFF_TP + 2 * BN * 4;      // float [2 tiles][BM]
 constexpr uint32_t OFF_KSB = OFF_LSE + 2 * BM * 4;     // fp16 [2 stages][BN] phase B key scales
 constexpr uint32_t OFF_BAR = OFF_KSB + 2 * BN * 2;     // uint64 barriers
 constexpr int kStagesA = 4;  // phase A K ring: slots K0, K1, V0, V1 (V is unused in phase A)
-constexpr int NBAR = 25 + 2 * kStagesA;
+constexpr int NBAR = 25 + 2 * kStagesA + 5;
 constexpr uint32_t OFF_TMEM = OFF_BAR + NBAR * 8;
 constexpr uint32_t kSmemBytes = OFF_TMEM + 16;
 static_assert(kSmemBytes <= 232448, "shared memory budget");
@@ -102,6 +103,7 @@ __device__ __forceinline__ int last_use_a(int a, int n_kt) {
 
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t IDESC_K_MAJOR = idesc_bf16_f32(128, 128, false, false);
+constexpr uint32_t IDESC_K_MAJOR_F16 = idesc_f16_f32(128, 128, false, false);
 constexpr uint32_t IDESC_PV = idesc_bf16_f32(128, 128, true, true);
 
 struct TcParams {
@@ -127,8 +129,12 @@ enum {
   B_PFULLA, B_PFULLB, B_PFREEA, B_PFREEB,    // P buffer, handed a(kt) -> b(kt) -> a(kt+1)
   B_OFULL, B_DRAIN,                          // O complete; MMA drain before TMEM is freed
   B_VGO,                                     // every phase A MMA done: V may use slots V0 / V1
-  B_AFULL0, B_AEMPTY0 = B_AFULL0 + kStagesA  // phase A K ring (+ token positions)
+  B_AFULL0, B_AEMPTY0 = B_AFULL0 + kStagesA,  // phase A K ring (+ token positions)
+  B_LOADED0 = B_AEMPTY0 + kStagesA,          // quantized caches: codes staged in K0, K1, V0, V1
+  B_QREADY = B_LOADED0 + 4,                  // quantized caches: Q tiles converted to fp16
+  B_END = B_QREADY + 1
 };
+static_assert(B_END == NBAR, "barrier count");
 
 // K-major SW128 operand (rows x 128 columns as two 64-column halves): k-step ks
 // (16 columns) starts 32 bytes further inside a half.
@@ -164,11 +170,12 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
 constexpr int kPolyA = 0;
 constexpr int kPolyB = 0;
 
-// Online (max, sum) update of one row over N slots (base-2 units).
-// Masked logits (slot relative position rel_e > row index ri) drop by 2^30:
+// Masking of one row of raw logits: a masked logit (slot relative position rel_e >
+// row index ri) drops by mbias = 2^30 / (logit scale), i.e. by 2^30 in base-2 units;
 // nm = sat(rel_e - ri) is 1 for a masked slot, 0 for a visible one.
 template <int N>
-__device__ __forceinline__ void row_mask(uint32_t (&x)[N], const float *rel, float ri) {
+__device__ __forceinline__ void row_mask(uint32_t (&x)[N], const float *rel, float ri,
+                                         float mbias) {
 #pragma unroll
   for (int e = 0; e < N; e += 4) {
     const float4 r4 = *reinterpret_cast<const float4 *>(rel + e);
@@ -176,11 +183,12 @@ __device__ __forceinline__ void row_mask(uint32_t (&x)[N], const float *rel, flo
 #pragma unroll
     for (int q = 0; q < 4; ++q) {
       const float nm = fma_sat(rr[q], 1.f, -ri);
-      x[e + q] = __float_as_uint(fmaf(nm, -kMaskBias, __uint_as_float(x[e + q])));
+      x[e + q] = __float_as_uint(fmaf(nm, -mbias, __uint_as_float(x[e + q])));
     }
   }
 }
 
+// Online (max, sum) update of one row over N slots (base-2 units).
 template <int N>
 __device__ __forceinline__ void row_update(const uint32_t (&x)[N], float c2, float &m, float &l) {
   static_assert(N % 16 == 0, "row width");
@@ -278,24 +286,26 @@ __device__ __forceinline__ void store_p(uint32_t p_slot_row, int st, const uint3
 }
 
 // ---- quantized caches: dequantizing tile loads --------------------------------------
-// 96 converter threads (warps 0, 2, 3) read a 128-slot tile of codes with 16-byte
-// loads (a batch in flight per thread), turn every code into bf16 and store the
-// tile in the swizzled K-major layout the MMA reads (the bytes a TMA load of a
-// bf16 tile would produce: row j at 128 j, 16-byte chunk c at c ^ (j % 8), dims
-// 64..127 in the second 16 KiB half).  A code c becomes a float exactly as the
-// float whose bits are 0x4B0000uu (2^23 + u, u = c + 128 or c + 8 as an unsigned
-// byte) minus 2^23 + 128 (or + 8); |c| <= 127 is exact in bf16.  Value tiles are
-// multiplied by their slot's scale first (exact in float32, one rounding to bf16).
+// One loader thread copies a 128-slot tile of codes with a bulk copy into the upper
+// 16 KiB of the bf16 operand buffer it becomes; the 96 loader threads (warps 0, 2, 3)
+// then turn every code into bf16 in place and store the tile in the swizzled K-major
+// layout the MMA reads (the bytes a TMA load of a bf16 tile would produce: row j at
+// 128 j, 16-byte chunk c at c ^ (j % 8), dims 64..127 in the second 16 KiB half).
+// A code c becomes a float exactly as the float whose bits are 0x4B0000uu (2^23 + u,
+// u = c + 128 or c + 8 as an unsigned byte) minus 2^23 + 128 (or + 8); |c| <= 127
+// is exact in bf16.  Value tiles are multiplied by their slot's scale first (exact
+// in float32, one rounding to bf16).
 constexpr int kConvThreads = 96;
+constexpr uint32_t kStageOff = kHalfBytes;  // staged codes: upper half of the buffer
 template <int KV>
 struct QTile;
 template <>
 struct QTile<H2OKV_I8> {
-  static constexpr int kRowBytes = D, kChunksPerRow = D / 16;  // 16 codes per 16-byte chunk
+  static constexpr int kRowBytes = D;
 };
 template <>
 struct QTile<H2OKV_I4> {
-  static constexpr int kRowBytes = D / 2, kChunksPerRow = D / 32;  // 32 codes per chunk
+  static constexpr int kRowBytes = D / 2;
 };
 
 __device__ __forceinline__ float offset_byte_float(uint32_t u, uint32_t k) {
@@ -307,6 +317,14 @@ __device__ __forceinline__ void st_shared_v4(uint32_t addr, uint32_t a, uint32_t
   asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(a), "r"(b), "r"(c),
                "r"(d)
                : "memory");
+}
+__device__ __forceinline__ uint4 ld_shared_v4(uint32_t addr) {
+  uint4 v;
+  asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];"
+               : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+               : "r"(addr)
+               : "memory");
+  return v;
 }
 
 // 8 int8 codes (element 4i + k in byte k of word i) -> 4 bf16 pairs in element order
@@ -341,60 +359,159 @@ __device__ __forceinline__ void cvt_i4x8(uint32_t w, float2 s2, bool fold, uint3
   }
 }
 
-// Tile of slots slot0 .. slot0 + 127 (nv of them inside the cache; the rest are
-// written as zeros) into the bf16 operand at shared address dst.
-template <int KV>
-__device__ __forceinline__ void convert_tile(const uint8_t *__restrict__ codes,
-                                             const __half *__restrict__ scales, int slot0, int nv,
-                                             uint32_t dst, bool fold, int ct) {
-  using T = QTile<KV>;
-  constexpr int kChunks = BN * T::kChunksPerRow;
-  constexpr int kPer = (kChunks + kConvThreads - 1) / kConvThreads;
-  constexpr int kBatch = KV == H2OKV_I8 ? 3 : 2;  // loads in flight per thread (register budget of the loader warps)
+// Keys of quantized caches enter the logit MMAs as f16 (exact for |code| <= 127).
+// 8 int8 codes -> 4 f16 pairs in element order: the f16 with bits 0x64uu is 1024 + u.
+__device__ __forceinline__ void cvt_i8_f16x8(uint32_t w0, uint32_t w1, uint32_t (&o)[4]) {
+  const uint32_t u0 = w0 ^ 0x80808080u, u1 = w1 ^ 0x80808080u;
+  const uint32_t t[4] = {__byte_perm(u0, 0x64646464u, 0x4140u), __byte_perm(u0, 0x64646464u, 0x4342u),
+                         __byte_perm(u1, 0x64646464u, 0x4140u), __byte_perm(u1, 0x64646464u, 0x4342u)};
+  const __half2 off = __float2half2_rn(1152.f);  // 1024 + 128
 #pragma unroll
-  for (int r0 = 0; r0 < kPer; r0 += kBatch) {
-    uint4 w[kBatch];
-    float sc[kBatch];
+  for (int k = 0; k < 4; ++k) {
+    const __half2 h = __hsub2(*reinterpret_cast<const __half2 *>(&t[k]), off);
+    o[k] = *reinterpret_cast<const uint32_t *>(&h);
+  }
+}
+// 8 int4 codes (element n in nibble n) -> 4 f16 pairs in the order (0, 4) (1, 5) (2, 6)
+// (3, 7); the query tile's chunks are reordered the same way, so the dot products are
+// unchanged.
+__device__ __forceinline__ void cvt_i4_f16x8(uint32_t w, uint32_t (&o)[4]) {
+  const uint32_t u = w ^ 0x88888888u;
+  const __half2 off = __float2half2_rn(1032.f);  // 1024 + 8
 #pragma unroll
-    for (int b = 0; b < kBatch; ++b) {
-      const int ch = ct + kConvThreads * (r0 + b);
-      const int j = ch / T::kChunksPerRow, q = ch % T::kChunksPerRow;
-      w[b] = make_uint4(0u, 0u, 0u, 0u);
-      sc[b] = 0.f;
-      if (r0 + b < kPer && ch < kChunks && j < nv) {
-        w[b] = __ldg(reinterpret_cast<const uint4 *>(codes + (size_t)(slot0 + j) * T::kRowBytes) + q);
-        if (fold) sc[b] = __half2float(scales[slot0 + j]);
-      }
+  for (int k = 0; k < 4; ++k) {
+    const uint32_t t = ((u >> (4 * k)) & 0x000F000Fu) | 0x64006400u;
+    const __half2 h = __hsub2(*reinterpret_cast<const __half2 *>(&t), off);
+    o[k] = *reinterpret_cast<const uint32_t *>(&h);
+  }
+}
+
+// Exponent e of the power of two a query tile is divided by before it becomes f16:
+// its largest |q| (float bits maxbits) then lies in [2^14, 2^15).
+__device__ __forceinline__ int q_exponent(uint32_t maxbits) {
+  if (maxbits == 0u) return 0;
+  const int lg = (int)((maxbits >> 23) & 0xFFu) - 127;
+  return min(max(lg - 14, -100), 100);
+}
+__device__ __forceinline__ float exp2i(int e) { return __int_as_float((127 + e) << 23); }
+
+// int8 in place (keys to exact f16, values to bf16(code * scale)): the staged code
+// row j (128 bytes at kStageOff + 128 j) occupies the
+// bytes of bf16 row j of the upper half, so each warp owns whole rows (4 per pass: 8
+// lanes of 16 codes per row) and reads a pass's rows before any lane rewrites them;
+// no other warp's rows are touched.  w3 is this warp's index among the loader warps;
+// sv[i] is the value scale of this lane's row in pass i (values only).  Rows at or
+// past nv (outside the cache) are written as zeros.
+constexpr int kI8Passes = 11;  // 32 groups of 4 rows over 3 warps
+__device__ __forceinline__ void convert_i8(uint32_t buf, int nv, const float (&sv)[kI8Passes + 1],
+                                           bool fold, int w3, int lane) {
+  const int q = lane & 7;
+  constexpr int kU = 4;  // passes in flight
+#pragma unroll
+  for (int it = 0; it < kI8Passes; it += kU) {
+    uint4 w[kU];
+    int row[kU];
+    bool act[kU];
+#pragma unroll
+    for (int u = 0; u < kU; ++u) {
+      const int g = w3 + 3 * (it + u);
+      act[u] = it + u < kI8Passes && g < 32;
+      row[u] = 4 * g + (lane >> 3);
+      w[u] = make_uint4(0u, 0u, 0u, 0u);
+      if (act[u] && row[u] < nv) w[u] = ld_shared_v4(buf + kStageOff + row[u] * 128 + q * 16);
     }
+    __syncwarp();
 #pragma unroll
-    for (int b = 0; b < kBatch; ++b) {
-      const int ch = ct + kConvThreads * (r0 + b);
-      if (r0 + b >= kPer || ch >= kChunks) continue;
-      const int j = ch / T::kChunksPerRow, q = ch % T::kChunksPerRow;
-      const uint32_t sw = (uint32_t)(j & 7);
-      const float2 s2 = make_float2(sc[b], sc[b]);
+    for (int u = 0; u < kU; ++u) {
+      if (!act[u]) continue;
+      const float s1 = it + u < kI8Passes ? sv[it + u] : 0.f;
+      const float2 s2 = make_float2(s1, s1);
+      // dims 16q .. 16q + 15: half q / 4, 16-byte chunks 2 (q % 4) and 2 (q % 4) + 1
+      const uint32_t ra = buf + (uint32_t)(q >> 2) * kHalfBytes + (uint32_t)row[u] * 128;
+      const uint32_t sw = (uint32_t)(row[u] & 7), c0 = 2u * (uint32_t)(q & 3);
       uint32_t o[4];
-      if constexpr (KV == H2OKV_I8) {
-        // dims 16q .. 16q + 15: half q / 4, 16-byte chunks 2 (q % 4) and 2 (q % 4) + 1
-        const uint32_t row = dst + (uint32_t)(q >> 2) * kHalfBytes + (uint32_t)j * 128;
-        const uint32_t c0 = 2u * (uint32_t)(q & 3);
-        cvt_i8x8(w[b].x, w[b].y, s2, fold, o);
-        st_shared_v4(row + ((c0 ^ sw) << 4), o[0], o[1], o[2], o[3]);
-        cvt_i8x8(w[b].z, w[b].w, s2, fold, o);
-        st_shared_v4(row + (((c0 + 1) ^ sw) << 4), o[0], o[1], o[2], o[3]);
-      } else {
-        // dims 32q .. 32q + 31: half q / 2, 16-byte chunks 4 (q % 2) .. 4 (q % 2) + 3
-        const uint32_t row = dst + (uint32_t)(q >> 1) * kHalfBytes + (uint32_t)j * 128;
-        const uint32_t c0 = 4u * (uint32_t)(q & 1);
-        const uint32_t ws[4] = {w[b].x, w[b].y, w[b].z, w[b].w};
-#pragma unroll
-        for (int m = 0; m < 4; ++m) {
-          cvt_i4x8(ws[m], s2, fold, o);
-          st_shared_v4(row + (((c0 + m) ^ sw) << 4), o[0], o[1], o[2], o[3]);
-        }
-      }
+      if (fold) cvt_i8x8(w[u].x, w[u].y, s2, true, o); else cvt_i8_f16x8(w[u].x, w[u].y, o);
+      st_shared_v4(ra + ((c0 ^ sw) << 4), o[0], o[1], o[2], o[3]);
+      if (fold) cvt_i8x8(w[u].z, w[u].w, s2, true, o); else cvt_i8_f16x8(w[u].z, w[u].w, o);
+      st_shared_v4(ra + (((c0 + 1) ^ sw) << 4), o[0], o[1], o[2], o[3]);
     }
   }
+}
+
+// int4 in place: staged code rows are 64 bytes, so a bf16 row of the upper half
+// overlaps two code rows of other slots.  Every loader thread first reads all its
+// chunks (chunk ch = 32 codes of row ch / 4), the 96 threads meet at a named barrier,
+// then all write (keys to exact f16, values to bf16(code * scale)).  sv holds the
+// value scales of the chunks' rows (pairs).
+constexpr int kI4Per = 6;  // ceil(512 chunks / 96 threads)
+constexpr int kConvBar = 3;  // named barrier of the loader threads (0: CTA, 1-2: softmax)
+__device__ __forceinline__ void convert_i4_read(uint32_t buf, int nv, int ct, uint4 (&w)[kI4Per]) {
+#pragma unroll
+  for (int r = 0; r < kI4Per; ++r) {
+    const int ch = ct + kConvThreads * r;
+    w[r] = make_uint4(0u, 0u, 0u, 0u);
+    if (ch < BN * 4 && (ch >> 2) < nv) w[r] = ld_shared_v4(buf + kStageOff + ch * 16);
+  }
+}
+// (after every loader thread has read its chunks and met at the named barrier)
+__device__ __forceinline__ void convert_i4_write(uint32_t buf, const __half2 (&sv)[kI4Per / 2],
+                                                 bool fold, int ct, const uint4 (&w)[kI4Per]) {
+#pragma unroll
+  for (int r = 0; r < kI4Per; ++r) {
+    const int ch = ct + kConvThreads * r;
+    if (ch >= BN * 4) continue;
+    const int j = ch >> 2, q = ch & 3;
+    const float sc = fold ? ((r & 1) ? __high2float(sv[r / 2]) : __low2float(sv[r / 2])) : 0.f;
+    const float2 s2 = make_float2(sc, sc);
+    // dims 32q .. 32q + 31: half q / 2, 16-byte chunks 4 (q % 2) .. 4 (q % 2) + 3
+    const uint32_t ra = buf + (uint32_t)(q >> 1) * kHalfBytes + (uint32_t)j * 128;
+    const uint32_t sw = (uint32_t)(j & 7), c0 = 4u * (uint32_t)(q & 1);
+    const uint32_t ws[4] = {w[r].x, w[r].y, w[r].z, w[r].w};
+#pragma unroll
+    for (int m = 0; m < 4; ++m) {
+      uint32_t o[4];
+      if (fold) cvt_i4x8(ws[m], s2, true, o); else cvt_i4_f16x8(ws[m], o);
+      st_shared_v4(ra + (((c0 + m) ^ sw) << 4), o[0], o[1], o[2], o[3]);
+    }
+  }
+}
+
+// The loaders' sequence of tiles: phase A keys 0 .. n_kt - 1 (buffers K0, K1, V0, V1
+// in turn), then phase B K(0), K(1), V(0), K(2), V(1), ..., V(n_kt - 1): the order in
+// which the MMA issuer consumes them.  use = how many earlier tiles went to the buffer
+// (its LOADED barrier phase).
+struct LoadItem {
+  int kind;  // 0: phase A key tile, 1: phase B key tile, 2: value tile
+  int kt, buf, use;
+};
+__device__ __forceinline__ int uses_a(int b, int n_kt) {
+  return b < n_kt ? (n_kt - 1 - b) / kStagesA + 1 : 0;
+}
+__device__ __forceinline__ LoadItem load_item(int e, int n_kt) {
+  LoadItem x;
+  if (e < n_kt) {
+    x.kind = 0;
+    x.kt = e;
+    x.buf = e % kStagesA;
+    x.use = e / kStagesA;
+    return x;
+  }
+  const int r = e - n_kt;
+  if (r == 0) {
+    x.kind = 1;
+    x.kt = 0;
+  } else if (r & 1) {
+    const int s = (r + 1) >> 1;
+    x.kind = s < n_kt ? 1 : 2;
+    x.kt = s < n_kt ? s : n_kt - 1;
+  } else {
+    x.kind = 2;
+    x.kt = (r >> 1) - 1;
+  }
+  const int b = x.kt & 1;
+  x.buf = x.kind == 1 ? b : 2 + b;
+  x.use = uses_a(x.buf, n_kt) + (x.kt >> 1);
+  return x;
 }
 
 // Key scales times the raw logits of one row (phase A, quantized caches).
@@ -411,17 +528,6 @@ __device__ __forceinline__ void scale_row(uint32_t (&x)[N], const float *ks) {
     x[e + 1] = __float_as_uint(a.y);
     x[e + 2] = __float_as_uint(b.x);
     x[e + 3] = __float_as_uint(b.y);
-  }
-}
-
-// Relative token positions of a tile's slots (float; 2^20 for empty / outside
-// slots), written by the loader threads t = first, first + step, ...
-__device__ __forceinline__ void write_rel(float *dst, const int32_t *tpg, int slot0, int nv, int P,
-                                          int first, int step) {
-  for (int e = first; e < BN; e += step) {
-    const int64_t t = e < nv ? (int64_t)tpg[slot0 + e] : (int64_t)kEmptyPos;
-    const int64_t rel = t - (int64_t)P;
-    dst[e] = (float)(rel < -1 ? -1 : (rel > kRelFar ? kRelFar : rel));
   }
 }
 
@@ -485,6 +591,11 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(&bar[B_AFULL0 + i], kFullCount);
       mbar_init(&bar[B_AEMPTY0 + i], 1 + 4 * nwg);
     }
+    for (int i = 0; i < 4; ++i) mbar_init(&bar[B_LOADED0 + i], 1);
+    mbar_init(&bar[B_QREADY], kConvThreads / 32);
+    tmem_s[1] = 0;  // loader abort flag (quantized caches)
+    tmem_s[2] = 0;  // largest |q| of query tile a / b (float bits; quantized caches)
+    tmem_s[3] = 0;
     fence_mbar_init();
   }
   if (warp == 1) {
@@ -503,6 +614,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   tc_fence_after();
   const uint32_t tmem = *tmem_s;
   bool aborted = false;
+  // logits Q K^T: bf16 operands, or f16 for quantized caches (exact integer keys)
+  constexpr uint32_t kIdescS = KV == H2OKV_BF16 ? IDESC_K_MAJOR : IDESC_K_MAJOR_F16;
 
   if (warp < 4) {
   reg_dealloc<kCtrlRegs>();
@@ -510,7 +623,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     // ------------------------------------------------------------------ MMA issuer
     if (lane == 0) {
       const uint32_t qa_addr = sbase + OFF_QA, qb_addr = sbase + OFF_QB, p_addr = sbase + OFF_P;
-      if (!mbar_wait(&bar[B_Q], 0, lim)) fail(p, aborted);
+      if (!mbar_wait(&bar[KV == H2OKV_BF16 ? B_Q : B_QREADY], 0, lim)) fail(p, aborted);
       tc_fence_after();
       // phase A: S_a, S_b = Q_a K^T, Q_b K^T into the column pair of the tile parity
       for (int kt = 0; kt < n_kt && !aborted; ++kt) {
@@ -525,12 +638,12 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
         for (int ks = 0; ks < D / 16; ++ks)
           mma_bf16_ss(tmem + u * 256, kmajor_desc(qa_addr, ks), kmajor_desc(k_addr, ks),
-                      IDESC_K_MAJOR, ks > 0);
+                      kIdescS, ks > 0);
         if (has_b) {
 #pragma unroll
           for (int ks = 0; ks < D / 16; ++ks)
             mma_bf16_ss(tmem + u * 256 + 128, kmajor_desc(qb_addr, ks), kmajor_desc(k_addr, ks),
-                        IDESC_K_MAJOR, ks > 0);
+                        kIdescS, ks > 0);
         }
         mma_commit(&bar[B_SFULL0 + u]);
         mma_commit(&bar[B_AEMPTY0 + a]);
@@ -552,7 +665,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
         for (int ks = 0; ks < D / 16; ++ks)
           mma_bf16_ss(tmem + (tile_b ? 128 : 0), kmajor_desc(k_addr, ks), kmajor_desc(q_addr, ks),
-                      IDESC_K_MAJOR, ks > 0);
+                      kIdescS, ks > 0);
         mma_commit(&bar[tile_b ? B_TFULLB : B_TFULLA]);
         if (tile_b || !has_b) mma_commit(&bar[B_KEMPTY0 + s]);  // K(kt) no longer read
         return true;
@@ -697,7 +810,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
   } else {
     // --------------------------- loaders of quantized tiles (warps 0, 2, 3: 96 threads)
-    const int ct = warp == 0 ? lane : 32 * (warp - 1) + lane;
+    const int w3 = warp == 0 ? 0 : warp - 1;
+    const int ct = 32 * w3 + lane;
     if (warp == 0 && lane == 0) {
       mbar_expect_tx(&bar[B_Q], has_b ? 2 * kTileBytes : kTileBytes);
       tma_load_3d(smem + OFF_QA, &q_map, &bar[B_Q], 0, i0_a, bhq_a);
@@ -714,76 +828,232 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint8_t *vg = p.vq + (size_t)bg * p.N_C * RB;
     const __half *ksg = p.ksc + (size_t)bg * p.N_C;
     const __half *vsg = p.vsc + (size_t)bg * p.N_C;
-    // L2 prefetch of a future tile's codes and scales (whole tiles only for the scales)
-    auto prefetch = [&](const uint8_t *codes, const __half *scales, int kt) {
-      if (ct != 0 || kt >= n_kt) return;
-      const int nv = min(BN, p.N_C - kt * BN);
-      bulk_prefetch_l2(codes + (size_t)kt * BN * RB, (uint32_t)(nv * RB));
-      const __half *sp = scales + (size_t)kt * BN;
-      if (nv == BN && (reinterpret_cast<uintptr_t>(sp) & 15u) == 0) bulk_prefetch_l2(sp, BN * 2);
+    volatile uint32_t *abort_flag = tmem_s + 1;
+    __half *ksb = reinterpret_cast<__half *>(smem + OFF_KSB);
+    // The query tiles become f16 once: tile t is divided by 2^e_t so that its largest
+    // |q| lies in [2^14, 2^15) (the softmax warps multiply the logit scale by 2^e_t);
+    // for int4 caches the 8 elements of every 16-byte chunk take the keys' order.
+    {
+      const bool qok = warp_wait(&bar[B_Q], 0, lim);
+      if (!qok) {
+        fail(p, aborted);
+        if (lane == 0) *abort_flag = 1u;
+      }
+      const int nch = (has_b ? 2 : 1) * (int)(kTileBytes / 16);
+      uint32_t mx0 = 0u, mx1 = 0u;  // largest |bf16| bit pattern of tile a / b
+      if (qok) {
+        for (int ch = ct; ch < nch; ch += kConvThreads) {
+          const uint4 v = ld_shared_v4(sbase + OFF_QA + (uint32_t)ch * 16);
+          const uint32_t ws[4] = {v.x, v.y, v.z, v.w};
+          uint32_t m = 0u;
+#pragma unroll
+          for (int i = 0; i < 4; ++i) m = max(m, max(ws[i] & 0x7FFFu, (ws[i] >> 16) & 0x7FFFu));
+          if (ch < (int)(kTileBytes / 16)) mx0 = max(mx0, m); else mx1 = max(mx1, m);
+        }
+      }
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) {
+        mx0 = max(mx0, __shfl_xor_sync(0xffffffffu, mx0, o));
+        mx1 = max(mx1, __shfl_xor_sync(0xffffffffu, mx1, o));
+      }
+      if (lane == 0) {
+        atomicMax(const_cast<uint32_t *>(tmem_s) + 2, mx0 << 16);
+        atomicMax(const_cast<uint32_t *>(tmem_s) + 3, mx1 << 16);
+      }
+      named_bar_sync(kConvBar, kConvThreads);
+      if (*abort_flag) {
+        aborted = true;
+      } else {
+        const float f0 = exp2i(-q_exponent(tmem_s[2])), f1 = exp2i(-q_exponent(tmem_s[3]));
+        for (int ch = ct; ch < nch; ch += kConvThreads) {
+          const uint32_t addr = sbase + OFF_QA + (uint32_t)ch * 16;
+          const uint4 v = ld_shared_v4(addr);
+          const float f = ch < (int)(kTileBytes / 16) ? f0 : f1;
+          const uint32_t ws[4] = {v.x, v.y, v.z, v.w};
+          float e[8];
+#pragma unroll
+          for (int i = 0; i < 4; ++i) {
+            e[2 * i] = __uint_as_float(ws[i] << 16) * f;
+            e[2 * i + 1] = __uint_as_float(ws[i] & 0xFFFF0000u) * f;
+          }
+          uint32_t o[4];
+#pragma unroll
+          for (int i = 0; i < 4; ++i) {
+            const int lo = KV == H2OKV_I4 ? i : 2 * i, hi = KV == H2OKV_I4 ? i + 4 : 2 * i + 1;
+            const __half2 h = __floats2half2_rn(e[lo], e[hi]);
+            o[i] = *reinterpret_cast<const uint32_t *>(&h);
+          }
+          st_shared_v4(addr, o[0], o[1], o[2], o[3]);
+        }
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&bar[B_QREADY]);
+      }
+    }
+    const int E = aborted ? 0 : 3 * n_kt;
+    // The buffer a tile goes to is free once the previous tile in it has been consumed:
+    // the same conditions the TMA producers of a bf16 cache wait for.
+    auto free_cond = [&](const LoadItem &x, uint64_t *&fb, uint32_t &par) -> bool {
+      if (x.kind == 0) {
+        const int n = x.kt / kStagesA;
+        if (n == 0) return false;
+        fb = &bar[B_AEMPTY0 + x.buf];
+        par = (uint32_t)(n - 1) & 1u;
+      } else if (x.kind == 1) {
+        const int st = x.kt & 1;
+        if (x.kt < 2) {
+          const int lu = last_use_a(st, n_kt);
+          if (lu < 0) return false;
+          fb = &bar[B_AEMPTY0 + st];
+          par = (uint32_t)(lu / kStagesA) & 1u;
+        } else {
+          fb = &bar[B_KEMPTY0 + st];
+          par = (uint32_t)((x.kt >> 1) - 1) & 1u;
+        }
+      } else {
+        const int vn = x.kt >> 1;
+        fb = vn == 0 ? &bar[B_VGO] : &bar[B_VEMPTY0 + (x.kt & 1)];
+        par = vn == 0 ? 0u : (uint32_t)(vn - 1) & 1u;
+      }
+      return true;
     };
-    // the stores of this warp reach the async proxy, then one arrival per warp
-    auto publish = [&](uint64_t *full) {
+    int issued = 0;
+    uint32_t last_par = 0;  // per buffer b: bit 2b = a copy was issued, bit 2b + 1 = its parity
+    for (int e = 0; e < E; ++e) {
+      const LoadItem x = load_item(e, n_kt);
+      const int slot0 = x.kt * BN, nv = min(BN, p.N_C - slot0);
+      // one thread keeps the copies going: item e (waiting for its buffer) and, while
+      // their buffers are already free, the next two
+      if (ct == 0 && !aborted) {
+        while (issued < E && issued <= e + 2) {
+          const LoadItem y = load_item(issued, n_kt);
+          uint64_t *fb = nullptr;
+          uint32_t par = 0;
+          if (free_cond(y, fb, par)) {
+            const bool ready = issued == e ? mbar_wait(fb, par, lim) : mbar_test(fb, par);
+            if (!ready) {
+              if (issued == e) fail(p, aborted);
+              break;
+            }
+          }
+          const int y0 = y.kt * BN, ynv = min(BN, p.N_C - y0);
+          uint64_t *lb = &bar[B_LOADED0 + y.buf];
+          mbar_expect_tx(lb, (uint32_t)(ynv * RB));
+          bulk_load(smem + slot_a(y.buf) + kStageOff, (y.kind == 2 ? vg : kg) + (size_t)y0 * RB,
+                    (uint32_t)(ynv * RB), lb);
+          mbar_arrive(lb);
+          last_par = (last_par & ~(3u << (2 * y.buf))) |
+                     ((1u | (((uint32_t)y.use & 1u) << 1)) << (2 * y.buf));
+          ++issued;
+        }
+        // bring a later tile's codes, scales and positions into L2
+        const int ep = e + 6;
+        if (ep < E) {
+          const LoadItem z = load_item(ep, n_kt);
+          const int z0 = z.kt * BN, znv = min(BN, p.N_C - z0);
+          bulk_prefetch_l2((z.kind == 2 ? vg : kg) + (size_t)z0 * RB, (uint32_t)(znv * RB));
+          const __half *sp = (z.kind == 2 ? vsg : ksg) + z0;
+          if (znv == BN && (reinterpret_cast<uintptr_t>(sp) & 15u) == 0) bulk_prefetch_l2(sp, BN * 2);
+          if (z.kind != 2 && znv == BN && (reinterpret_cast<uintptr_t>(tpg + z0) & 15u) == 0)
+            bulk_prefetch_l2(tpg + z0, BN * 4);
+        }
+      }
+      // positions and scales of this tile, read from global memory while the codes travel
+      float relv[2], ksv[2];
+      __half ksh[2];
+#pragma unroll
+      for (int i = 0; i < 2; ++i) {
+        const int e2 = ct + kConvThreads * i;
+        relv[i] = (float)kRelFar;
+        ksv[i] = 0.f;
+        ksh[i] = __float2half(0.f);
+        if (x.kind != 2 && e2 < BN && e2 < nv) {
+          const int64_t rel = (int64_t)tpg[slot0 + e2] - (int64_t)p.P;
+          relv[i] = (float)(rel < -1 ? -1 : (rel > kRelFar ? kRelFar : rel));
+          ksh[i] = ksg[slot0 + e2];
+          ksv[i] = __half2float(ksh[i]);
+        }
+      }
+      float sv8[kI8Passes + 1] = {};
+      __half2 sv4[kI4Per / 2];
+      if constexpr (KV == H2OKV_I4) {
+#pragma unroll
+        for (int r = 0; r < kI4Per / 2; ++r) sv4[r] = __float2half2_rn(0.f);
+      }
+      if (x.kind == 2) {
+        if constexpr (KV == H2OKV_I8) {
+#pragma unroll
+          for (int i = 0; i <= kI8Passes; ++i) {
+            const int row = 4 * (w3 + 3 * i) + (lane >> 3);
+            sv8[i] = (i < kI8Passes && row < nv) ? __half2float(vsg[slot0 + row]) : 0.f;
+          }
+        } else {
+#pragma unroll
+          for (int r = 0; r < kI4Per; r += 2) {
+            const int row0 = (ct + kConvThreads * r) >> 2, row1 = (ct + kConvThreads * (r + 1)) >> 2;
+            sv4[r / 2] = __halves2half2(row0 < nv ? vsg[slot0 + row0] : __float2half(0.f),
+                                        row1 < nv ? vsg[slot0 + row1] : __float2half(0.f));
+          }
+        }
+      }
+      // the codes have landed (and the buffer's previous tile was consumed)
+      bool ok = !aborted && warp_wait(&bar[B_LOADED0 + x.buf], (uint32_t)x.use & 1u, lim);
+      if (!ok) fail(p, aborted);
+      uint4 w4[kI4Per];
+      if constexpr (KV == H2OKV_I4) {
+        // in place: every staged chunk is read before any is overwritten; the loaders
+        // meet at a named barrier (and leave the loop together after a failed wait)
+        if (!ok && lane == 0) *abort_flag = 1u;
+        if (ok) convert_i4_read(sbase + slot_a(x.buf), nv, ct, w4);
+        named_bar_sync(kConvBar, kConvThreads);
+        if (*abort_flag) {
+          aborted = true;
+          break;
+        }
+      } else {
+        if (!ok) break;
+      }
+      if (x.kind == 0) {
+        float *rd = reinterpret_cast<float *>(smem + OFF_REL_A) + x.buf * BN;
+        float *kd = reinterpret_cast<float *>(smem + OFF_KS_A) + x.buf * BN;
+#pragma unroll
+        for (int i = 0; i < 2; ++i) {
+          const int e2 = ct + kConvThreads * i;
+          if (e2 < BN) {
+            rd[e2] = relv[i];
+            kd[e2] = ksv[i];
+          }
+        }
+      } else if (x.kind == 1) {
+        float *rd = reinterpret_cast<float *>(tp_s) + x.buf * BN;
+#pragma unroll
+        for (int i = 0; i < 2; ++i) {
+          const int e2 = ct + kConvThreads * i;
+          if (e2 < BN) {
+            rd[e2] = relv[i];
+            ksb[x.buf * BN + e2] = ksh[i];
+          }
+        }
+      }
+      const uint32_t buf = sbase + slot_a(x.buf);
+      if constexpr (KV == H2OKV_I8)
+        convert_i8(buf, nv, sv8, x.kind == 2, w3, lane);
+      else
+        convert_i4_write(buf, sv4, x.kind == 2, ct, w4);
+      // the stores of this warp reach the async proxy, then one arrival per warp
       fence_proxy_async_smem();
       __syncwarp();
-      if (lane == 0) mbar_arrive(full);
-    };
-    // phase A: keys through the four-stage ring, with positions and scales
-    for (int kt = 0; kt < n_kt && !aborted; ++kt) {
-      const int stage = kt % kStagesA, n = kt / kStagesA;
-      if (n > 0 && !warp_wait(&bar[B_AEMPTY0 + stage], (n - 1) & 1, lim)) { fail(p, aborted); break; }
-      const int ahead = kt + kPrefetch;
-      if (ahead < n_kt) {
-        prefetch(kg, ksg, ahead);
-      } else {
-        prefetch(kg, ksg, ahead - n_kt);
-        prefetch(vg, vsg, ahead - n_kt);
-      }
-      const int nv = min(BN, p.N_C - kt * BN);
-      convert_tile<KV>(kg, nullptr, kt * BN, nv, sbase + slot_a(stage), false, ct);
-      write_rel(reinterpret_cast<float *>(smem + OFF_REL_A) + stage * BN, tpg, kt * BN, nv, p.P, ct,
-                kConvThreads);
-      float *ksd = reinterpret_cast<float *>(smem + OFF_KS_A) + stage * BN;
-      for (int e = ct; e < BN; e += kConvThreads)
-        ksd[e] = e < nv ? __half2float(ksg[kt * BN + e]) : 0.f;
-      publish(&bar[B_AFULL0 + stage]);
+      if (lane == 0)
+        mbar_arrive(x.kind == 0 ? &bar[B_AFULL0 + x.buf]
+                                : (x.kind == 1 ? &bar[B_KFULL0 + x.buf] : &bar[B_VFULL0 + x.buf - 2]));
     }
-    // phase B: K(s) then V(s - 1), the order in which the MMA issuer needs them
-    __half *ksb = reinterpret_cast<__half *>(smem + OFF_KSB);
-    for (int s2 = 0; s2 <= n_kt && !aborted; ++s2) {
-      if (s2 < n_kt) {
-        const int kt = s2, stage = kt & 1;
-        bool ok;
-        if (kt < 2) {
-          const int lu = last_use_a(stage, n_kt);
-          ok = lu < 0 || warp_wait(&bar[B_AEMPTY0 + stage], (lu / kStagesA) & 1, lim);
-        } else {
-          ok = warp_wait(&bar[B_KEMPTY0 + stage], ((kt >> 1) - 1) & 1, lim);
-        }
-        if (!ok) { fail(p, aborted); break; }
-        prefetch(kg, ksg, kt + kPrefetch);
-        const int nv = min(BN, p.N_C - kt * BN);
-        convert_tile<KV>(kg, nullptr, kt * BN, nv, sbase + (stage ? OFF_K1 : OFF_K0), false, ct);
-        write_rel(reinterpret_cast<float *>(tp_s) + stage * BN, tpg, kt * BN, nv, p.P, ct,
-                  kConvThreads);
-        for (int e = ct; e < BN; e += kConvThreads)
-          ksb[stage * BN + e] = e < nv ? ksg[kt * BN + e] : __float2half(0.f);
-        publish(&bar[B_KFULL0 + stage]);
-      }
-      if (s2 >= 1) {
-        const int kt = s2 - 1, vs = kt & 1, vn = kt >> 1;
-        // slots V0 / V1 serve as phase A K stages 2 / 3 until every phase A MMA is done
-        const bool ok = vn == 0 ? warp_wait(&bar[B_VGO], 0, lim)
-                                : warp_wait(&bar[B_VEMPTY0 + vs], (vn - 1) & 1, lim);
-        if (!ok) { fail(p, aborted); break; }
-        prefetch(vg, vsg, kt + kPrefetch);
-        const int nv = min(BN, p.N_C - kt * BN);
-        convert_tile<KV>(vg, vsg, kt * BN, nv, sbase + (vs ? OFF_V1 : OFF_V0), true, ct);
-        publish(&bar[B_VFULL0 + vs]);
-      }
+    // drain: the Q copy and the last copy into each buffer must land before exit
+    if (ct == 0) {
+      mbar_wait(&bar[B_Q], 0, 4000000000ull);
+      for (int b2 = 0; b2 < 4; ++b2)
+        if ((last_par >> (2 * b2)) & 1u)
+          mbar_wait(&bar[B_LOADED0 + b2], (last_par >> (2 * b2 + 1)) & 1u, 4000000000ull);
     }
-    // drain: the Q copy must land before exit
-    if (warp == 0 && lane == 0) mbar_wait(&bar[B_Q], 0, 4000000000ull);
     __syncwarp();
   }
   } else {
@@ -793,9 +1063,15 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int wg = (warp - 4) >> 2;  // 0: tile a, 1: tile b
     const int st = threadIdx.x - 128 * (1 + wg);  // row (phase A) or slot (phase B) in the tile
     const uint32_t lane_base = (uint32_t)(32 * (warp & 3)) << 16;
-    const float c2 = p.scale2;
+    float c2 = p.scale2;
+    if constexpr (KV != H2OKV_BF16) {
+      // the query tile was divided by 2^e before it became f16
+      if (!warp_wait(&bar[B_QREADY], 0, lim)) fail(p, aborted);
+      c2 *= exp2i(q_exponent(tmem_s[2 + wg]));
+    }
     const int i0 = wg ? i0_b : i0_a, bhq = wg ? bhq_b : bhq_a, t = wg ? t_b : t_a;
     float m = -INFINITY, l = 0.f;
+    const float mbias = kMaskBias / c2;
     uint32_t x[BN];
     for (int kt = 0; kt < n_kt && !aborted; ++kt) {
       const int u = kt & 1, a = kt % kStagesA;
@@ -814,7 +1090,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       tmem_wait_ld();
       if constexpr (KV != H2OKV_BF16)
         scale_row<BN>(x, reinterpret_cast<const float *>(smem + OFF_KS_A) + a * BN);
-      if (masked) row_mask<BN>(x, rela, (float)(i0 + st));
+      if (masked) row_mask<BN>(x, rela, (float)(i0 + st), mbias);
       // S buffer and K stage (with its token positions) are free once read
       tc_fence_before();
       __syncwarp();
@@ -828,7 +1104,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (lane == 0) mbar_arrive(&bar[B_AFREE]);
     // masked logits sit 2^30 below the visible ones: a row whose maximum is that
     // low sees no slot (lse = -inf, no weight, y = 0)
-    const bool seen = l > 0.f && m > -0.5f * kMaskBias * c2;
+    const bool seen = l > 0.f && m > -0.5f * kMaskBias;
     const float lse2 = seen ? m + lg2(l) : -INFINITY;
     float *lse_t = lse_s + wg * BM;  // holds -lse2 of the tile's rows
     lse_t[st] = seen ? -lse2 : -kMaskBias;

@@ -111,43 +111,66 @@ struct EvictArgs {
   uint8_t *keys, *values;
   __half *k_scales, *v_scales;
   int32_t *slots_out;
-  int N_C, S, P, mode, n_filled, d, slice;
+  const int32_t *slots_in;  // replay: the slots to write (mode 3)
+  uint8_t *dk, *dv;         // delta outputs (or null): overwritten rows [B][H_k][S][row bytes]
+  __half *dks, *dvs;        //   their scales (quantized caches)
+  int32_t *dpos;            //   their token positions [B][H_k][S]
+  int *status;              // device status word (replayed slot outside the cache)
+  int N_C, S, P, mode, n_filled, d, slice, score_mode, nbat, Hk;
   size_t row_bytes, in_row_bytes;
 };
 
 constexpr int kCopyUnroll = 8;   // 16-byte pieces per thread in flight in the row copy
 constexpr int kQuantUnroll = 4;  // rows per lane segment in flight in the row quantizer
 
-// Chunk rows k = rank + CL * m (m = 0 .. n_rows - 1) of this (b, h_k) go to slot slot_of(m).
+// The rows of one chunk row set: chunk rows k = rank + CL * m (m = 0 .. n_rows - 1) of
+// (batch row, KV head) at cache offset gbase (slots) and chunk offset rbase (rows) go to
+// slot slot_of(m) (negative: skipped).
+struct RowSet {
+  size_t gbase, rbase;
+};
+
 // f32 / bf16 caches: the key and value rows are cut into 16-byte pieces spread over the
 // whole CTA (consecutive threads take consecutive pieces of a row), and every thread loads
 // kCopyUnroll pieces before it stores any, so a launch waits on memory a few times in all
-// rather than once per row.
+// rather than once per row.  With delta outputs the same thread first reads the piece it
+// overwrites.
 template <typename SlotOf>
-__device__ __forceinline__ void copy_rows_cta(const EvictArgs &a, size_t bh, int rank, int CL,
+__device__ __forceinline__ void copy_rows_cta(const EvictArgs &a, RowSet rs, int rank, int CL,
                                               int n_rows, SlotOf slot_of) {
   const int C = (int)(a.row_bytes / 16);  // 16-byte pieces per row (row_bytes % 16 == 0)
   const int total = n_rows * 2 * C;
-  const size_t gbase = bh * (size_t)a.N_C;
+  const bool dl = a.dk != nullptr;
   for (int base = threadIdx.x; base < total; base += kEvThreads * kCopyUnroll) {
-    uint4 r[kCopyUnroll];
+    uint4 r[kCopyUnroll], old[kCopyUnroll];
     uint4 *dst[kCopyUnroll];
+    uint4 *ddst[kCopyUnroll];
 #pragma unroll
     for (int u = 0; u < kCopyUnroll; ++u) {
       const int e = base + u * kEvThreads;
       dst[u] = nullptr;
+      ddst[u] = nullptr;
       if (e < total) {
         const int c = e % C, rest = e / C, t = rest & 1, m = rest >> 1;
-        const size_t row = bh * (size_t)a.S + rank + (size_t)CL * m;
+        const size_t row = rs.rbase + rank + (size_t)CL * m;
         const uint8_t *src = (t ? a.v_new : a.k_new) + row * a.in_row_bytes;
         r[u] = __ldcs(reinterpret_cast<const uint4 *>(src) + c);
-        dst[u] = reinterpret_cast<uint4 *>((t ? a.values : a.keys) +
-                                           (gbase + (size_t)slot_of(m)) * a.row_bytes) + c;
+        const int slot = slot_of(m);
+        if (slot >= 0) {
+          dst[u] = reinterpret_cast<uint4 *>((t ? a.values : a.keys) +
+                                             (rs.gbase + (size_t)slot) * a.row_bytes) + c;
+          if (dl) {
+            old[u] = *dst[u];
+            ddst[u] = reinterpret_cast<uint4 *>((t ? a.dv : a.dk) + row * a.row_bytes) + c;
+          }
+        }
       }
     }
 #pragma unroll
-    for (int u = 0; u < kCopyUnroll; ++u)
+    for (int u = 0; u < kCopyUnroll; ++u) {
+      if (ddst[u]) *ddst[u] = old[u];
       if (dst[u]) *dst[u] = r[u];
+    }
   }
 }
 
@@ -155,9 +178,10 @@ __device__ __forceinline__ void copy_rows_cta(const EvictArgs &a, size_t bh, int
 // >= d / 8); lane i of a segment holds elements 8i .. 8i + 7 of the row.  A warp covers
 // 32 / L rows per pass and keeps kQuantUnroll passes in flight.  Per row, the same
 // arithmetic as the per-row quantizer: absmax, IEEE division by qmax, clamp to the fp16
-// range, round to fp16, then rint(x / scale) clamped to [-qmax, qmax].
+// range, round to fp16, then rint(x / scale) clamped to [-qmax, qmax].  With delta
+// outputs each lane first copies the codes (and lane 0 the scale) it overwrites.
 template <int KV, typename SlotOf>
-__device__ __forceinline__ void quantize_rows_cta(const EvictArgs &a, size_t bh, int rank, int CL,
+__device__ __forceinline__ void quantize_rows_cta(const EvictArgs &a, RowSet rs, int rank, int CL,
                                                   int n_rows, SlotOf slot_of) {
   constexpr int qmax = KV == H2OKV_I8 ? 127 : 7;
   const int G = a.d / 8;
@@ -166,18 +190,21 @@ __device__ __forceinline__ void quantize_rows_cta(const EvictArgs &a, size_t bh,
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const int seg = lane / L, li = lane % L, segs = 32 / L;
   const int items = n_rows * 2;  // (m, t): t = 0 key row, 1 value row
-  const size_t gbase = bh * (size_t)a.N_C;
+  const bool dl = a.dk != nullptr;
   for (int p0 = 0; (p0 * kEvWarps + warp) * segs < items; p0 += kQuantUnroll) {
     uint4 x[kQuantUnroll];
     bool ok[kQuantUnroll];
+    int slot[kQuantUnroll];
 #pragma unroll
     for (int u = 0; u < kQuantUnroll; ++u) {
       const int item = ((p0 + u) * kEvWarps + warp) * segs + seg;
       ok[u] = item < items && li < G;
       x[u] = make_uint4(0u, 0u, 0u, 0u);
+      slot[u] = -1;
       if (ok[u]) {
         const int t = item & 1, m = item >> 1;
-        const size_t row = bh * (size_t)a.S + rank + (size_t)CL * m;
+        slot[u] = slot_of(m);
+        const size_t row = rs.rbase + rank + (size_t)CL * m;
         const uint8_t *src = (t ? a.v_new : a.k_new) + row * a.in_row_bytes;
         x[u] = __ldcs(reinterpret_cast<const uint4 *>(src) + li);
       }
@@ -204,12 +231,22 @@ __device__ __forceinline__ void quantize_rows_cta(const EvictArgs &a, size_t bh,
 #pragma unroll
       for (int q = 0; q < 8; ++q)
         qc[q] = s > 0.f ? (int)fminf(fmaxf(rintf(v[q] / s), (float)-qmax), (float)qmax) : 0;
-      if (!ok[u]) continue;
+      if (!ok[u] || slot[u] < 0) continue;
       const int item = ((p0 + u) * kEvWarps + warp) * segs + seg;
       const int t = item & 1, m = item >> 1;
-      const size_t drow = gbase + (size_t)slot_of(m);
+      const size_t drow = rs.gbase + (size_t)slot[u];
+      const size_t crow = rs.rbase + rank + (size_t)CL * m;
       uint8_t *codes = (t ? a.values : a.keys) + drow * a.row_bytes;
-      if (li == 0) (t ? a.v_scales : a.k_scales)[drow] = hs;
+      __half *sdst = (t ? a.v_scales : a.k_scales) + drow;
+      if (dl) {
+        uint8_t *dcodes = (t ? a.dv : a.dk) + crow * a.row_bytes;
+        if (li == 0) (t ? a.dvs : a.dks)[crow] = *sdst;
+        if (KV == H2OKV_I8)
+          reinterpret_cast<uint2 *>(dcodes)[li] = reinterpret_cast<const uint2 *>(codes)[li];
+        else
+          reinterpret_cast<uint32_t *>(dcodes)[li] = reinterpret_cast<const uint32_t *>(codes)[li];
+      }
+      if (li == 0) *sdst = hs;
       if (KV == H2OKV_I8) {
         uint32_t lo = 0u, hi = 0u;
 #pragma unroll
@@ -229,13 +266,13 @@ __device__ __forceinline__ void quantize_rows_cta(const EvictArgs &a, size_t bh,
 }
 
 template <int KV, typename SlotOf>
-__device__ __forceinline__ void insert_rows_cta(const EvictArgs &a, size_t bh, int rank, int CL,
+__device__ __forceinline__ void insert_rows_cta(const EvictArgs &a, RowSet rs, int rank, int CL,
                                                 SlotOf slot_of) {
   const int n_rows = rank < a.S ? (a.S - rank + CL - 1) / CL : 0;
   if constexpr (KV == H2OKV_I8 || KV == H2OKV_I4)
-    quantize_rows_cta<KV>(a, bh, rank, CL, n_rows, slot_of);
+    quantize_rows_cta<KV>(a, rs, rank, CL, n_rows, slot_of);
   else
-    copy_rows_cta(a, bh, rank, CL, n_rows, slot_of);
+    copy_rows_cta(a, rs, rank, CL, n_rows, slot_of);
 }
 
 template <int IPT>
@@ -256,16 +293,34 @@ __device__ __forceinline__ void store_slice(float *dst, const float (&v)[IPT],
   }
 }
 
+// Slot j of a chunk row set receives chunk row k: bookkeeping of the slot (old token
+// position to the delta output, new token position, score 0, slot list).
+__device__ __forceinline__ void claim_slot(const EvictArgs &a, RowSet rs, int j, int k) {
+  const size_t gs = rs.gbase + (size_t)j, rk = rs.rbase + (size_t)k;
+  if (a.dpos) a.dpos[rk] = a.token_pos[gs];
+  a.token_pos[gs] = a.P + k;
+  a.scores[gs] = 0.f;
+  if (a.slots_out) a.slots_out[rk] = j;
+}
+
 // mode 0: fold w_prev only (S = 0); 1: fill slots n_filled.. (no occupied slot is
-// touched); 2: generic choice (empty slots first, then lowest scores).
+// touched); 2: generic choice (empty slots first, then lowest selection keys);
+// 3: replay (write the given slots).  One cluster per (batch row, KV head), or per KV
+// head for all batch rows together (score variant h2o_orig: nbat > 1).
 template <int KV, int IPT>
 __global__ void __launch_bounds__(kEvThreads) evict_kernel(const EvictArgs a) {
   namespace cg = cooperative_groups;
   cg::cluster_group cluster = cg::this_cluster();
   const int CL = (int)cluster.num_blocks();
   const int rank = (int)cluster.block_rank();
-  const int bh = blockIdx.x / CL;
+  const int gi = blockIdx.x / CL;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int nb = a.nbat;
+  const int b_first = nb > 1 ? 0 : gi / a.Hk, h = nb > 1 ? gi : gi % a.Hk;
+  auto rows_of = [&](int bb) {
+    const size_t bh = (size_t)(b_first + bb) * a.Hk + h;
+    return RowSet{bh * (size_t)a.N_C, bh * (size_t)a.S};
+  };
 
   __shared__ uint32_t hist[2][256];
   __shared__ uint32_t tot_bins[256];
@@ -274,77 +329,111 @@ __global__ void __launch_bounds__(kEvThreads) evict_kernel(const EvictArgs a) {
   __shared__ uint32_t cta_less, cta_eq;
   extern __shared__ int32_t rowslot[];  // [ceil(S / CL)]: slot of chunk row rank + CL * m
 
-  const size_t gbase = (size_t)bh * a.N_C;
   const int j0 = rank * a.slice + tid * IPT;
-  float sc[IPT], wp[IPT];
+  float sc[IPT], ksum[IPT];
   int32_t tp[IPT];
   uint32_t key[IPT];
   bool valid[IPT];
 #pragma unroll
   for (int i = 0; i < IPT; ++i) {
     valid[i] = j0 + i < a.N_C;
-    sc[i] = 0.f;
-    wp[i] = 0.f;
     tp[i] = kEmptyPos;
+    ksum[i] = 0.f;
   }
-  // 16-byte loads when this thread's slots are whole and aligned, else one by one
-  const bool vec = IPT % 4 == 0 && j0 + IPT <= a.N_C &&
-                   ((reinterpret_cast<uintptr_t>(a.scores + gbase + j0) |
-                     reinterpret_cast<uintptr_t>(a.token_pos + gbase + j0) |
-                     (a.w_prev ? reinterpret_cast<uintptr_t>(a.w_prev + gbase + j0) : 0u)) &
-                    15u) == 0u;
-  bool loaded = false;
-  if constexpr (IPT % 4 == 0) {
-    if (vec) {
-#pragma unroll
-      for (int i = 0; i < IPT; i += 4) {
-        *reinterpret_cast<float4 *>(&sc[i]) =
-            *reinterpret_cast<const float4 *>(a.scores + gbase + j0 + i);
-        if (a.w_prev)
-          *reinterpret_cast<float4 *>(&wp[i]) =
-              __ldcs(reinterpret_cast<const float4 *>(a.w_prev + gbase + j0 + i));
-        if (a.mode == 2)
-          *reinterpret_cast<int4 *>(&tp[i]) =
-              *reinterpret_cast<const int4 *>(a.token_pos + gbase + j0 + i);
-      }
-      loaded = true;
-    }
-  }
-  if (!loaded) {
+  // ---- fold w_prev into the scores of every batch row of this set ----------------
+  for (int bb = 0; bb < nb; ++bb) {
+    const size_t gbase = rows_of(bb).gbase;
+    float wp[IPT];
 #pragma unroll
     for (int i = 0; i < IPT; ++i) {
-      if (!valid[i]) continue;
-      sc[i] = a.scores[gbase + j0 + i];
-      if (a.w_prev) wp[i] = a.w_prev[gbase + j0 + i];
-      if (a.mode == 2) tp[i] = a.token_pos[gbase + j0 + i];
+      sc[i] = 0.f;
+      wp[i] = 0.f;
     }
-  }
+    const bool want_tp = bb == 0 && a.mode == 2;
+    // 16-byte loads when this thread's slots are whole and aligned, else one by one
+    const bool vec = IPT % 4 == 0 && j0 + IPT <= a.N_C &&
+                     ((reinterpret_cast<uintptr_t>(a.scores + gbase + j0) |
+                       reinterpret_cast<uintptr_t>(a.token_pos + gbase + j0) |
+                       (a.w_prev ? reinterpret_cast<uintptr_t>(a.w_prev + gbase + j0) : 0u)) &
+                      15u) == 0u;
+    bool loaded = false;
+    if constexpr (IPT % 4 == 0) {
+      if (vec) {
 #pragma unroll
-  for (int i = 0; i < IPT; ++i) {
-    if (a.w_prev) sc[i] = __fadd_rn(sc[i], wp[i]);
-    key[i] = (valid[i] && a.mode == 2 && tp[i] != kEmptyPos) ? order_key(sc[i]) : 0u;
-  }
-
-  if (a.mode != 2) {
-    // fold (and, while filling, the trivial slot choice n_filled + k)
+        for (int i = 0; i < IPT; i += 4) {
+          *reinterpret_cast<float4 *>(&sc[i]) =
+              *reinterpret_cast<const float4 *>(a.scores + gbase + j0 + i);
+          if (a.w_prev)
+            *reinterpret_cast<float4 *>(&wp[i]) =
+                __ldcs(reinterpret_cast<const float4 *>(a.w_prev + gbase + j0 + i));
+          if (want_tp)
+            *reinterpret_cast<int4 *>(&tp[i]) =
+                *reinterpret_cast<const int4 *>(a.token_pos + gbase + j0 + i);
+        }
+        loaded = true;
+      }
+    }
+    if (!loaded) {
+#pragma unroll
+      for (int i = 0; i < IPT; ++i) {
+        if (!valid[i]) continue;
+        sc[i] = a.scores[gbase + j0 + i];
+        if (a.w_prev) wp[i] = a.w_prev[gbase + j0 + i];
+        if (want_tp) tp[i] = a.token_pos[gbase + j0 + i];
+      }
+    }
 #pragma unroll
     for (int i = 0; i < IPT; ++i) {
-      const int j = j0 + i;
-      if (!valid[i]) continue;
-      const int k = j - a.n_filled;
-      if (a.mode == 1 && k >= 0 && k < a.S) {
-        sc[i] = 0.f;
-        if (!a.w_prev) a.scores[gbase + j] = 0.f;
-        a.token_pos[gbase + j] = a.P + k;
-        if (a.slots_out) a.slots_out[(size_t)bh * a.S + k] = j;
-      }
+      if (a.w_prev) sc[i] = __fadd_rn(sc[i], wp[i]);
+      ksum[i] = bb == 0 ? sc[i] : __fadd_rn(ksum[i], sc[i]);  // h2o_orig: batch order
     }
     if (a.w_prev) store_slice<IPT>(a.scores + gbase + j0, sc, valid, vec);
-    if (a.mode == 1) {
-      const int first = a.n_filled + rank;
-      insert_rows_cta<KV>(a, (size_t)bh, rank, CL, [&](int m) { return first + CL * m; });
+  }
+
+  if (a.mode == 1) {
+    // while filling: chunk row k takes slot n_filled + k (same slot for every batch row)
+#pragma unroll
+    for (int i = 0; i < IPT; ++i) {
+      const int k = j0 + i - a.n_filled;
+      if (valid[i] && k >= 0 && k < a.S)
+        for (int bb = 0; bb < nb; ++bb) claim_slot(a, rows_of(bb), j0 + i, k);
+    }
+    const int first = a.n_filled + rank;
+    for (int bb = 0; bb < nb; ++bb)
+      insert_rows_cta<KV>(a, rows_of(bb), rank, CL, [&](int m) { return first + CL * m; });
+    return;
+  }
+  if (a.mode == 3) {
+    // replay: every fold store of the cluster lands before a replayed slot is reset
+    cluster.sync();
+    for (int bb = 0; bb < nb; ++bb) {
+      const RowSet rs = rows_of(bb);
+      auto slot_of = [&](int m) -> int {
+        const int j = a.slots_in[rs.rbase + rank + (size_t)CL * m];
+        return (j >= 0 && j < a.N_C) ? j : -1;
+      };
+      for (int m = tid; rank + CL * m < a.S; m += kEvThreads) {
+        const int j = slot_of(m);
+        if (j < 0)
+          atomicExch(a.status, H2OKV_ERR_INVALID_ARG);
+        else
+          claim_slot(a, rs, j, rank + CL * m);
+      }
+      insert_rows_cta<KV>(a, rs, rank, CL, slot_of);
     }
     return;
+  }
+  if (a.mode != 2) return;
+
+  // ---- selection keys ----------------------------------------------------------------
+#pragma unroll
+  for (int i = 0; i < IPT; ++i) {
+    float kv = ksum[i];
+    if (a.score_mode == 1) {  // h2o_norm: score / (P - t(b, h, j)), age at least 1
+      const int age = max(a.P - tp[i], 1);
+      kv = __fdiv_rn(kv, (float)age);
+    }
+    key[i] = (valid[i] && tp[i] != kEmptyPos) ? order_key(kv) : 0u;
   }
 
   // ---- radix select of the S-th smallest key over the whole cluster --------------
@@ -436,18 +525,16 @@ __global__ void __launch_bounds__(kEvThreads) evict_kernel(const EvictArgs a) {
       ++eq_before;
     }
     if (take) {
-      sc[i] = 0.f;
-      a.token_pos[gbase + j] = a.P + (int)pos;
-      if (a.slots_out) a.slots_out[(size_t)bh * a.S + pos] = j;
+      for (int bb = 0; bb < nb; ++bb) claim_slot(a, rows_of(bb), j, (int)pos);
       int32_t *dst = cluster.map_shared_rank(rowslot, (int)(pos % (uint32_t)CL));
       dst[pos / (uint32_t)CL] = j;
     }
   }
-  store_slice<IPT>(a.scores + gbase + j0, sc, valid, vec);
   cluster.sync();  // rowslot lists complete
 
   // ---- insert the chunk's rows k = rank, rank + CL, ... -----------------------------
-  insert_rows_cta<KV>(a, (size_t)bh, rank, CL, [&](int m) { return rowslot[m]; });
+  for (int bb = 0; bb < nb; ++bb)
+    insert_rows_cta<KV>(a, rows_of(bb), rank, CL, [&](int m) { return rowslot[m]; });
 }
 
 template <int KV>
@@ -457,6 +544,38 @@ __global__ void __launch_bounds__(256)
   const int64_t row = (int64_t)blockIdx.x * 8 + (threadIdx.x >> 5);
   if (row >= n_rows) return;
   quantize_row_warp<KV>(x + row * d, d, codes + row * row_bytes, scales + row);
+}
+
+// Delta rows back into their slots (one warp per chunk row; 4-byte words).
+__global__ void __launch_bounds__(256)
+    restore_kernel(const int32_t *__restrict__ slots, int64_t n_rows, int S, int N_C,
+                   size_t row_bytes, const uint8_t *__restrict__ dk, const uint8_t *__restrict__ dv,
+                   const __half *__restrict__ dks, const __half *__restrict__ dvs,
+                   const int32_t *__restrict__ dpos, uint8_t *keys, uint8_t *values,
+                   __half *k_scales, __half *v_scales, int32_t *token_pos, int *status) {
+  const int64_t row = (int64_t)blockIdx.x * 8 + (threadIdx.x >> 5);
+  const int lane = threadIdx.x & 31;
+  if (row >= n_rows) return;
+  const int j = slots[row];
+  if (j < 0 || j >= N_C) {
+    if (lane == 0) atomicExch(status, H2OKV_ERR_INVALID_ARG);
+    return;
+  }
+  const size_t dst = (size_t)(row / S) * N_C + j;  // slot j of this row's (b, h_k)
+  const int words = (int)(row_bytes / 4);
+  const uint32_t *sk = reinterpret_cast<const uint32_t *>(dk + row * row_bytes);
+  const uint32_t *sv = reinterpret_cast<const uint32_t *>(dv + row * row_bytes);
+  uint32_t *tk = reinterpret_cast<uint32_t *>(keys + dst * row_bytes);
+  uint32_t *tv = reinterpret_cast<uint32_t *>(values + dst * row_bytes);
+  for (int w = lane; w < words; w += 32) {
+    tk[w] = sk[w];
+    tv[w] = sv[w];
+  }
+  if (lane == 0) {
+    if (k_scales && dks) k_scales[dst] = dks[row];
+    if (v_scales && dvs) v_scales[dst] = dvs[row];
+    token_pos[dst] = dpos[row];
+  }
 }
 
 __global__ void init_kernel(int32_t *__restrict__ token_pos, float *__restrict__ scores,
@@ -522,7 +641,8 @@ static int launch_evict_kv(const EvictArgs &a, int n_groups, int CL, int ipt, cu
 }
 
 int launch_evict_insert(h2okv_cache *c, const float *w_prev, const void *k_new, const void *v_new,
-                        int S, int64_t P, int32_t *slots_out, cudaStream_t st) {
+                        int S, int64_t P, int32_t *slots_out, const int32_t *slots_in,
+                        const h2okv_delta *delta, cudaStream_t st) {
   const h2okv_cache_desc &d = c->desc;
   EvictArgs a;
   a.scores = c->bufs.scores;
@@ -535,10 +655,22 @@ int launch_evict_insert(h2okv_cache *c, const float *w_prev, const void *k_new, 
   a.k_scales = reinterpret_cast<__half *>(c->bufs.k_scales);
   a.v_scales = reinterpret_cast<__half *>(c->bufs.v_scales);
   a.slots_out = slots_out;
+  a.slots_in = slots_in;
+  a.dk = delta ? reinterpret_cast<uint8_t *>(delta->keys) : nullptr;
+  a.dv = delta ? reinterpret_cast<uint8_t *>(delta->values) : nullptr;
+  a.dks = delta ? reinterpret_cast<__half *>(delta->k_scales) : nullptr;
+  a.dvs = delta ? reinterpret_cast<__half *>(delta->v_scales) : nullptr;
+  a.dpos = delta ? delta->token_pos : nullptr;
+  a.status = reinterpret_cast<int *>(reinterpret_cast<uint8_t *>(c->bufs.workspace) + c->ws.status);
   a.N_C = d.capacity;
   a.S = S;
   a.P = (int)P;
-  a.mode = S == 0 ? 0 : (c->n_filled + S <= d.capacity ? 1 : 2);
+  a.mode = S == 0 ? 0 : (slots_in ? 3 : (c->n_filled + S <= d.capacity ? 1 : 2));
+  a.score_mode = c->score_mode;
+  a.Hk = d.n_kv_heads;
+  // h2o_orig: one cluster per KV head selects for every batch row
+  const bool orig = c->score_mode == H2OKV_SCORE_H2O_ORIG && a.mode == 2;
+  a.nbat = orig ? d.batch : 1;
   a.n_filled = c->n_filled;
   a.d = d.head_dim;
   a.row_bytes = c->row_bytes;
@@ -548,7 +680,7 @@ int launch_evict_insert(h2okv_cache *c, const float *w_prev, const void *k_new, 
   int ipt = 1;
   while ((int64_t)CL * kEvThreads * ipt < d.capacity) ipt *= 2;
   a.slice = kEvThreads * ipt;
-  const int n_groups = d.batch * d.n_kv_heads;
+  const int n_groups = orig ? d.n_kv_heads : d.batch * d.n_kv_heads;
   switch (d.kv_dtype) {
     case H2OKV_F32: return launch_evict_kv<H2OKV_F32>(a, n_groups, CL, ipt, st);
     case H2OKV_BF16: return launch_evict_kv<H2OKV_BF16>(a, n_groups, CL, ipt, st);
@@ -570,6 +702,24 @@ int launch_quantize(int kv_dtype, const __nv_bfloat16 *x, int64_t n_rows, int d,
     quantize_kernel<H2OKV_I4><<<(unsigned)blocks, 256, 0, st>>>(
         x, n_rows, d, reinterpret_cast<uint8_t *>(codes), scales, rb);
   return check_launch("quantize_kernel");
+}
+
+int launch_restore(h2okv_cache *c, const int32_t *slots, int S, const h2okv_delta *delta,
+                   cudaStream_t st) {
+  const h2okv_cache_desc &d = c->desc;
+  const int64_t n_rows = (int64_t)d.batch * d.n_kv_heads * S;
+  if (n_rows == 0) return H2OKV_OK;
+  const bool quant = d.kv_dtype == H2OKV_I8 || d.kv_dtype == H2OKV_I4;
+  restore_kernel<<<(unsigned)((n_rows + 7) / 8), 256, 0, st>>>(
+      slots, n_rows, S, d.capacity, c->row_bytes, reinterpret_cast<const uint8_t *>(delta->keys),
+      reinterpret_cast<const uint8_t *>(delta->values),
+      quant ? reinterpret_cast<const __half *>(delta->k_scales) : nullptr,
+      quant ? reinterpret_cast<const __half *>(delta->v_scales) : nullptr, delta->token_pos,
+      reinterpret_cast<uint8_t *>(c->bufs.keys), reinterpret_cast<uint8_t *>(c->bufs.values),
+      reinterpret_cast<__half *>(c->bufs.k_scales), reinterpret_cast<__half *>(c->bufs.v_scales),
+      c->bufs.token_pos,
+      reinterpret_cast<int *>(reinterpret_cast<uint8_t *>(c->bufs.workspace) + c->ws.status));
+  return check_launch("restore_kernel");
 }
 
 }  // namespace h2okv

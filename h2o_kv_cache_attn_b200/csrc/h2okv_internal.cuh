@@ -45,6 +45,7 @@ struct h2okv_cache {
   h2okv::WorkspaceLayout ws;
   h2okv::TcPlan tc;
   uint64_t wait_timeout_ns;
+  int32_t score_mode;  // h2okv_score_mode
 };
 
 namespace h2okv {
@@ -66,7 +67,10 @@ inline size_t kv_row_bytes(int kv_dtype, int d) {
 // ---- launchers (return H2OKV_OK or an error code) -------------------------
 int launch_init_cache(h2okv_cache *c, cudaStream_t st);
 int launch_evict_insert(h2okv_cache *c, const float *w_prev, const void *k_new, const void *v_new,
-                        int S, int64_t P, int32_t *slots_out, cudaStream_t st);
+                        int S, int64_t P, int32_t *slots_out, const int32_t *slots_in,
+                        const h2okv_delta *delta, cudaStream_t st);
+int launch_restore(h2okv_cache *c, const int32_t *slots, int S, const h2okv_delta *delta,
+                   cudaStream_t st);
 int launch_quantize(int kv_dtype, const __nv_bfloat16 *x, int64_t n_rows, int d, void *codes,
                     __half *scales, cudaStream_t st);
 int launch_attn_simt(h2okv_cache *c, const void *q, int S, int64_t P, void *y, float *lse,

@@ -9,7 +9,9 @@ before SDPA runs):
   2. attn_chunk_with_scoresum: SDPA of the chunk's queries over the cache,
      returning y, the row log-sum-exp and the summed weights w.
 
-After the last chunk, h2o_evict_insert with S = 0 folds the last w in.
+After the last chunk, h2o_evict_insert with S = 0 folds the last w in.  A
+replay run (§3.2: decisions read back from a replay log) passes the logged slots
+to ``step`` and writes them with h2o_insert_at instead of step 1's choice.
 """
 
 from __future__ import annotations
@@ -45,8 +47,11 @@ class LayerRunner:
     def w_cur(self):
         return self.w[self.chunk_index % 2]
 
-    def step(self, q, k, v, stream=None):
-        """Process one chunk whose inputs are already on the device."""
+    def step(self, q, k, v, stream=None, slots_in=None):
+        """Process one chunk whose inputs are already on the device.  With
+        ``slots_in`` ([B, H_k, S] int32) the chunk is written to those slots
+        instead of the ones the policy would choose (replay of a logged
+        decision); the slots then returned are slots_in."""
         S = q.shape[2]
         y = self.y[:, :, :S] if S == self.wl.chunk else torch.empty_like(q)
         lse = None
@@ -55,7 +60,11 @@ class LayerRunner:
         if S != self.wl.chunk:
             y = y.contiguous()
         slots = self.slots[:, :, :S] if S == self.wl.chunk else torch.empty((self.wl.B, self.wl.Hk, S), dtype=torch.int32, device=self.device)
-        self.cache.evict_insert(self.w_prev(), k, v, S, self.P, slots, stream)
+        if slots_in is None:
+            self.cache.evict_insert(self.w_prev(), k, v, S, self.P, slots, stream)
+        else:
+            self.cache.insert_at(self.w_prev(), k, v, S, self.P, slots_in, None, stream)
+            slots = slots_in
         self.cache.attend(q, S, self.P, y, lse, self.w_cur(), self.wq, stream)
         self.last = (y, lse, self.w_cur(), self.wq, slots)
         self.chunk_index += 1

@@ -157,8 +157,9 @@ H2OKV_API int kv_cache_quantize(int32_t kv_dtype, const void *x_bf16, int64_t n_
  *   1. if w_prev != NULL: scores = float32(scores + w_prev)
  *      (w_prev: [B, H_k, N_C] float32, normally the previous chunk's w_out);
  *   2. choose S slots: empty slots first (lowest index first), then the
- *      occupied slots with the smallest (score, slot index) pairs -- lowest
- *      score, ties to the lowest index;
+ *      occupied slots with the smallest (key, slot index) pairs -- lowest key,
+ *      ties to the lowest index; the key is the score, or the variant set by
+ *      kv_cache_set_score_mode;
  *   3. chunk token k (position P + k) goes to the k-th smallest chosen slot:
  *      keys/values rows <- k_new/v_new row k (quantized for I8/I4),
  *      token_pos = P + k, scores = 0;
@@ -170,6 +171,66 @@ H2OKV_API int kv_cache_quantize(int32_t kv_dtype, const void *x_bf16, int64_t n_
 H2OKV_API int h2o_evict_insert(h2okv_cache *cache, const float *w_prev, const void *k_new,
                      const void *v_new, int32_t S, int64_t P, int32_t *slots_out,
                      void *stream);
+
+/* Score variant that ranks occupied slots in step 2 of h2o_evict_insert
+ * ("Learning how to Forget", §3.1.1 Variants of Heavy-Hitter Oracle):
+ *   H2OKV_SCORE_H2O       the cumulative score (default);
+ *   H2OKV_SCORE_H2O_NORM  score / (t - token_pos) with t = P, the first
+ *                         position of the chunk being inserted (the pages leave
+ *                         t undefined; this is the reading used), computed as an
+ *                         IEEE float32 quotient; an age below 1 counts as 1;
+ *   H2OKV_SCORE_H2O_ORIG  the score summed over the batch rows (float32, in
+ *                         batch order): every batch row evicts the same slots.
+ * Empty slots are taken first in every variant.  Host only; applies to the
+ * following calls. */
+enum h2okv_score_mode { H2OKV_SCORE_H2O = 0, H2OKV_SCORE_H2O_NORM = 1, H2OKV_SCORE_H2O_ORIG = 2 };
+H2OKV_API int kv_cache_set_score_mode(h2okv_cache *cache, int32_t mode);
+
+/* Delta encoding of one update (§A.5.3: for keys' = scatter(keys, index,
+ * key_new) it keeps delta_key = gather(keys, index), from which keys is rebuilt
+ * as scatter(keys', index, delta_key)).  Caller-owned device buffers, indexed
+ * like the chunk: keys, values [B, H_k, S, row bytes] in the cache's storage
+ * format (bytes as stored: f32 / bf16 values, int8 codes, packed int4 codes),
+ * k_scales, v_scales [B, H_k, S] fp16 (quantized caches, else NULL),
+ * token_pos [B, H_k, S] int32 (the overwritten token positions; INT32_MAX for a
+ * slot that was empty).  16-byte aligned. */
+typedef struct h2okv_delta {
+  void *keys;
+  void *values;
+  void *k_scales;
+  void *v_scales;
+  int32_t *token_pos;
+} h2okv_delta;
+
+/* h2o_evict_insert that also writes the delta encoding of the update: before
+ * chunk row k overwrites its slot, the slot's stored key/value row, scales and
+ * token position go to row k of `delta`.  slots_out is required (the index of
+ * the delta encoding).  Same arguments and errors as h2o_evict_insert; S >= 1. */
+H2OKV_API int h2o_evict_insert_delta(h2okv_cache *cache, const float *w_prev, const void *k_new,
+                                     const void *v_new, int32_t S, int64_t P, int32_t *slots_out,
+                                     const h2okv_delta *delta, void *stream);
+
+/* Replay of logged eviction decisions (§3.2 / §A.5: a replay cache acts like
+ * the cache, except that its decisions are read from the replay log):
+ * step 1 of h2o_evict_insert, then chunk row k goes to slots_in[b, h_k, k]
+ * (int32 [B, H_k, S], device) with token_pos = P + k and score 0.  The slots
+ * of one (b, h_k) must be distinct; a slot outside [0, N_C) is skipped and
+ * records H2OKV_ERR_INVALID_ARG in the device status word
+ * (kv_cache_device_status).  delta may be NULL, else it receives the delta
+ * encoding as in h2o_evict_insert_delta.  The fill level advances by S (capped
+ * at N_C), as for a log written by a cache that filled left to right. */
+H2OKV_API int h2o_insert_at(h2okv_cache *cache, const float *w_prev, const void *k_new,
+                            const void *v_new, int32_t S, int64_t P, const int32_t *slots_in,
+                            const h2okv_delta *delta, void *stream);
+
+/* Undo one update from its delta encoding (the recurrence of §A.5.3 played
+ * backwards): for every (b, h_k, k), the row, scales and token position of
+ * delta row k go back into slot slots[b, h_k, k].  Scores and the fill level
+ * are left as they are (set the fill level with kv_cache_set_fill).  Slots
+ * outside [0, N_C) are skipped and record H2OKV_ERR_INVALID_ARG in the device
+ * status word. */
+H2OKV_API int kv_cache_restore(h2okv_cache *cache, const int32_t *slots, int32_t S,
+                               const h2okv_delta *delta, void *stream);
 
 /* SDPA of one chunk of queries against the cache, with summed weights (§A.1,
  * §A.7).  For query head h (group g = h / q_g), row i (token P + i):

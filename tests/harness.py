@@ -95,12 +95,35 @@ def assert_lse_close(got, ref, what):
     assert np.all(err <= tol), f"{what}: max lse error {err.max():.3g}"
 
 
-def check_insert(wl, before, after, w_prev, k, v, S, P, slots_gpu, groups):
-    """Bit-exact check of the evict/insert step for the given (b, g) groups."""
+def oracle_head(wl: Workload, snap, g: int):
+    """An oracle cache for KV head g over every batch row (B = wl.B, H_k = 1)."""
+    oc = oracle.OracleCache(wl.B, wl.q_g, 1, wl.d, wl.capacity, wl.kv_dtype)
+    sl = (slice(None), slice(g, g + 1))
+    kw = dict(token_pos=snap["token_pos"][sl], scores=snap["scores"][sl], n_filled=snap["n_filled"])
+    if wl.kv_dtype in ("i8", "i4"):
+        kw.update(k_codes=snap["k_codes"][sl], v_codes=snap["v_codes"][sl],
+                  k_scales=snap["k_scales"][sl], v_scales=snap["v_scales"][sl])
+    else:
+        kw.update(keys=snap["keys"][sl], values=snap["values"][sl])
+    oc.load_state(**kw)
+    return oc
+
+
+def check_insert(wl, before, after, w_prev, k, v, S, P, slots_gpu, groups, mode="h2o"):
+    """Bit-exact check of the evict/insert step for the given (b, g) groups.
+    h2o_orig chooses for all batch rows of a KV head together: its oracle holds
+    every batch row of the head."""
     for (b, g) in groups:
-        oc = oracle_group(wl, before, b, g)
-        wp = None if w_prev is None else w_prev[b:b + 1, g:g + 1]
-        slots = oc.evict_insert(wp, k[b:b + 1, g:g + 1], v[b:b + 1, g:g + 1], S, P)
+        if mode == "h2o_orig":
+            oc = oracle_head(wl, before, g)
+            wp = None if w_prev is None else w_prev[:, g:g + 1]
+            slots = oc.evict_insert(wp, k[:, g:g + 1], v[:, g:g + 1], S, P, mode=mode)
+            oc = _row_of(oc, b)
+            slots = slots[b:b + 1]
+        else:
+            oc = oracle_group(wl, before, b, g)
+            wp = None if w_prev is None else w_prev[b:b + 1, g:g + 1]
+            slots = oc.evict_insert(wp, k[b:b + 1, g:g + 1], v[b:b + 1, g:g + 1], S, P, mode=mode)
         np.testing.assert_array_equal(slots_gpu[b, g], slots[0, 0], err_msg=f"slots b={b} g={g}")
         np.testing.assert_array_equal(after["token_pos"][b, g], oc.token_pos[0, 0])
         np.testing.assert_array_equal(after["scores"][b, g].view(np.uint32),
@@ -116,6 +139,20 @@ def check_insert(wl, before, after, w_prev, k, v, S, P, slots_gpu, groups):
             np.testing.assert_array_equal(after["keys"][b, g], oc.k_store[0, 0])
             np.testing.assert_array_equal(after["values"][b, g], oc.v_store[0, 0])
     return True
+
+
+class _Row:
+    """Batch row b of an oracle cache, as attributes shaped like a one-row cache."""
+
+    def __init__(self, oc, b):
+        for name in ("token_pos", "scores", "k_codes", "v_codes", "k_scales", "v_scales",
+                     "k_store", "v_store"):
+            if hasattr(oc, name):
+                setattr(self, name, getattr(oc, name)[b:b + 1])
+
+
+def _row_of(oc, b):
+    return _Row(oc, b)
 
 
 def check_attend(wl, after, q, S, P, y, lse, w, wq, groups):
@@ -134,12 +171,15 @@ def check_attend(wl, after, q, S, P, y, lse, w, wq, groups):
 
 
 def run_and_check(wl: Workload, device, check_chunks=None, groups=None, with_wq=True,
-                  source=None, on_chunk=None):
+                  source=None, on_chunk=None, mode="h2o"):
     """Run all chunks of one layer on the GPU; compare the chunks in
     ``check_chunks`` (None = all) for the (b, g) pairs in ``groups`` (None =
-    all) against the oracle re-seeded from the GPU state before each of them."""
+    all) against the oracle re-seeded from the GPU state before each of them.
+    ``mode``: the score variant of the eviction."""
     src = source or ChunkSource(wl, 0, "cpu")
     run = LayerRunner(wl, device, with_wq=with_wq)
+    if mode != "h2o":
+        run.cache.set_score_mode(mode)
     if groups is None:
         groups = [(b, g) for b in range(wl.B) for g in range(wl.Hk)]
     n_checked = 0
@@ -158,7 +198,7 @@ def run_and_check(wl: Workload, device, check_chunks=None, groups=None, with_wq=
             torch.cuda.synchronize()
             after = snapshot(run.cache)
             qn, kn, vn = to_np(q), to_np(k), to_np(v)
-            check_insert(wl, before, after, w_prev, kn, vn, S, P, to_np(slots), groups)
+            check_insert(wl, before, after, w_prev, kn, vn, S, P, to_np(slots), groups, mode=mode)
             check_attend(wl, after, qn, S, P, to_np(y), to_np(lse), to_np(w), to_np(wq), groups)
             n_checked += 1
         if on_chunk:
