@@ -166,6 +166,23 @@ def evict_bytes_chunk(wl, S):
     return per * wl.B * wl.Hk
 
 
+def split_schedule(wl, S, sms):
+    """Whether the library runs a chunk of S tokens with the split (persistent)
+    tensor-core schedule: the same rule as the library's (bf16 cache, an even number
+    of query tiles per KV group, the one-CTA-per-pair grid filling less than 95 % of
+    its last wave, at least 4 units per SM and 4 K/V tiles)."""
+    if wl.kv_dtype != "bf16" or wl.d != 128 or wl.q_dtype != "bf16":
+        return False
+    tiles = -(-S // 128)
+    n_qt = wl.q_g * tiles
+    if n_qt % 2:
+        return False
+    pairs = wl.B * wl.Hk * n_qt // 2
+    n_kt = -(-wl.capacity // 128)
+    waves = -(-pairs // sms)
+    return pairs / (waves * sms) < 0.95 and pairs * n_kt >= 4 * sms and n_kt >= 4
+
+
 # --------------------------------------------------------------------------- #
 def run_ours(args, wl, ws, rank, local):
     from h2o_kv_cache_attn_b200 import binding as hb
@@ -244,16 +261,22 @@ def run_ours(args, wl, ws, rank, local):
     # the tensor-core path serves head_dim 128 with a bf16, int8 or int4 cache and bf16
     # queries (the same rule as the library)
     tc_used = wl.d == 128 and wl.kv_dtype in ("bf16", "i8", "i4") and wl.q_dtype == "bf16"
-    # per chunk: one eviction launch, then two attention launches (tensor-core path:
-    # attention + reduction; CUDA-core path: two passes); plus the reset and the final fold
-    launches_per_step = wl.n_chunks * 3 + 2
+    # per chunk: one eviction launch, then the attention launches (fused tensor-core path:
+    # attention + reduction; split schedule: phase A, phase B, output and weight
+    # reductions; CUDA-core path: two passes); plus the reset and the final fold
+    sms = torch.cuda.get_device_properties(dev).multi_processor_count
+    n_split = sum(1 for c in range(wl.n_chunks) if split_schedule(wl, wl.chunk_len(c), sms))
+    launches_per_step = wl.n_chunks * 3 + 2 * n_split + 2
     per_launch_alg = at_flops_alg / len(at_ms)
     per_launch_ms = sum(at_ms) / len(at_ms)
     if tc_used:
         roof = {"bound": "tensor", "achieved": round(tflops_alg, 2), "peak": tc_peak,
                 "unit": "TFLOP/s", "frac": round(tflops_alg / tc_peak, 4),
                 "traffic": recorded_traffic("attn_tc_kernel"),
-                "kernel": "attention call per chunk (attn_tc_kernel + reduce_w_kernel)",
+                "kernel": ("attention call per chunk (attn_split_a_kernel + attn_split_b_kernel + "
+                           "reduce_o_kernel + reduce_w_kernel)") if n_split == wl.n_chunks else
+                          ("attention call per chunk (attn_tc_kernel + reduce_w_kernel)" if n_split == 0 else
+                           "attention call per chunk (split schedule on %d of %d chunks)" % (n_split, wl.n_chunks)),
                 "alg_flops_per_launch": per_launch_alg, "avg_launch_ms": round(per_launch_ms, 4),
                 "peak_kind": f"{pk_kind} bf16 dense, sustained (kernel timed inside a long step)"}
     else:

@@ -77,13 +77,13 @@ static void layout(const h2okv_cache_desc &d, const TcPlan &tc, WorkspaceLayout 
   off = align256(off + 4);
   ws->part_ml = ws->part_w = ws->part_o = off;
   if (tc.enabled) {
-    const size_t rows_pad = (size_t)tc.tiles_per_head * 128;
+    const size_t seg_rows = (size_t)tc.split_ctas * tc.max_seg * 2 * 128;
     ws->part_ml = off;
-    off = align256(off + (size_t)tc.max_splits * B * Hq * rows_pad * 8);
+    off = align256(off + seg_rows * 8);
     ws->part_w = off;
     off = align256(off + B * Hq * (size_t)tc.tiles_per_head * NC * 4);
     ws->part_o = off;
-    off = align256(off + (size_t)tc.max_splits * B * Hq * rows_pad * D * 4);
+    off = align256(off + seg_rows * D * 4);
   }
   ws->total = off;
 }

@@ -917,6 +917,45 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       return true;
     };
+    // per tile: slot positions relative to the chunk and key scales (threads ct and
+    // ct + 96 of the tile), and value scales of this lane's rows
+    struct Meta {
+      float rel[2];
+      __half2 ks;
+      __half2 sv[(kI8Passes + 2) / 2];
+    };
+    auto load_meta = [&](int e) -> Meta {
+      const LoadItem x = load_item(e, n_kt);
+      const int slot0 = x.kt * BN, nv = min(BN, p.N_C - slot0);
+      Meta m;
+      __half kh[2];
+#pragma unroll
+      for (int i = 0; i < 2; ++i) {
+        const int e2 = ct + kConvThreads * i;
+        m.rel[i] = (float)kRelFar;
+        kh[i] = __float2half(0.f);
+        if (x.kind != 2 && e2 < BN && e2 < nv) {
+          const int64_t rel = (int64_t)tpg[slot0 + e2] - (int64_t)p.P;
+          m.rel[i] = (float)(rel < -1 ? -1 : (rel > kRelFar ? kRelFar : rel));
+          kh[i] = ksg[slot0 + e2];
+        }
+      }
+      m.ks = __halves2half2(kh[0], kh[1]);
+      __half sh[2 * ((kI8Passes + 2) / 2)];
+#pragma unroll
+      for (int i = 0; i < 2 * ((kI8Passes + 2) / 2); ++i) {
+        int row = BN;
+        if (KV == H2OKV_I8)
+          row = i < kI8Passes ? 4 * (w3 + 3 * i) + (lane >> 3) : BN;
+        else
+          row = i < kI4Per ? (ct + kConvThreads * i) >> 2 : BN;
+        sh[i] = (x.kind == 2 && row < nv) ? vsg[slot0 + row] : __float2half(0.f);
+      }
+#pragma unroll
+      for (int i = 0; i < (kI8Passes + 2) / 2; ++i) m.sv[i] = __halves2half2(sh[2 * i], sh[2 * i + 1]);
+      return m;
+    };
+    Meta meta = E > 0 ? load_meta(0) : Meta{};
     int issued = 0;
     uint32_t last_par = 0;  // per buffer b: bit 2b = a copy was issued, bit 2b + 1 = its parity
     for (int e = 0; e < E; ++e) {
@@ -958,44 +997,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             bulk_prefetch_l2(tpg + z0, BN * 4);
         }
       }
-      // positions and scales of this tile, read from global memory while the codes travel
-      float relv[2], ksv[2];
-      __half ksh[2];
-#pragma unroll
-      for (int i = 0; i < 2; ++i) {
-        const int e2 = ct + kConvThreads * i;
-        relv[i] = (float)kRelFar;
-        ksv[i] = 0.f;
-        ksh[i] = __float2half(0.f);
-        if (x.kind != 2 && e2 < BN && e2 < nv) {
-          const int64_t rel = (int64_t)tpg[slot0 + e2] - (int64_t)p.P;
-          relv[i] = (float)(rel < -1 ? -1 : (rel > kRelFar ? kRelFar : rel));
-          ksh[i] = ksg[slot0 + e2];
-          ksv[i] = __half2float(ksh[i]);
-        }
-      }
-      float sv8[kI8Passes + 1] = {};
-      __half2 sv4[kI4Per / 2];
-      if constexpr (KV == H2OKV_I4) {
-#pragma unroll
-        for (int r = 0; r < kI4Per / 2; ++r) sv4[r] = __float2half2_rn(0.f);
-      }
-      if (x.kind == 2) {
-        if constexpr (KV == H2OKV_I8) {
-#pragma unroll
-          for (int i = 0; i <= kI8Passes; ++i) {
-            const int row = 4 * (w3 + 3 * i) + (lane >> 3);
-            sv8[i] = (i < kI8Passes && row < nv) ? __half2float(vsg[slot0 + row]) : 0.f;
-          }
-        } else {
-#pragma unroll
-          for (int r = 0; r < kI4Per; r += 2) {
-            const int row0 = (ct + kConvThreads * r) >> 2, row1 = (ct + kConvThreads * (r + 1)) >> 2;
-            sv4[r / 2] = __halves2half2(row0 < nv ? vsg[slot0 + row0] : __float2half(0.f),
-                                        row1 < nv ? vsg[slot0 + row1] : __float2half(0.f));
-          }
-        }
-      }
+      const Meta cur = meta;
       // the codes have landed (and the buffer's previous tile was consumed)
       bool ok = !aborted && warp_wait(&bar[B_LOADED0 + x.buf], (uint32_t)x.use & 1u, lim);
       if (!ok) fail(p, aborted);
@@ -1013,6 +1015,23 @@ __global__ void __launch_bounds__(kThreads, 1)
       } else {
         if (!ok) break;
       }
+      // the next tile's positions and scales are read while this one is converted
+      if (e + 1 < E) meta = load_meta(e + 1);
+      float relv[2], ksv[2];
+      __half ksh[2];
+#pragma unroll
+      for (int i = 0; i < 2; ++i) {
+        relv[i] = cur.rel[i];
+        ksh[i] = i ? __high2half(cur.ks) : __low2half(cur.ks);
+        ksv[i] = __half2float(ksh[i]);
+      }
+      float sv8[kI8Passes + 1];
+#pragma unroll
+      for (int i = 0; i <= kI8Passes; ++i)
+        sv8[i] = (i & 1) ? __high2float(cur.sv[i / 2]) : __low2float(cur.sv[i / 2]);
+      __half2 sv4[kI4Per / 2];
+#pragma unroll
+      for (int r = 0; r < kI4Per / 2; ++r) sv4[r] = cur.sv[r];
       if (x.kind == 0) {
         float *rd = reinterpret_cast<float *>(smem + OFF_REL_A) + x.buf * BN;
         float *kd = reinterpret_cast<float *>(smem + OFF_KS_A) + x.buf * BN;
@@ -1187,6 +1206,637 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
 }
 
+// ---- split scheduling (bf16 cache): the two passes as persistent kernels ----------
+// With one CTA per pair of query tiles, a grid of P pairs fills ceil(P / SMs) waves
+// and leaves SMs idle in the last one (P = 128 on 148 SMs: 14 % idle).  Here the
+// (pair, K/V tile) units are cut into G contiguous ranges of equal length, one per SM,
+// so a pair's slots may be spread over two or three CTAs ("segments").  Kernel A runs
+// phase A over each segment and stores the rows' partial (max, sum); kernel B combines
+// a pair's partials into the final row LSE, runs phase B over its segments and writes
+// y, or a partial O when the pair is split (the partials add up: P is already
+// normalised); a reduction sums the partial O's.  Requires an even number of query
+// tiles per KV group (every pair has two tiles).
+struct SplitParams {
+  TcParams t;
+  int G;            // CTAs (one per SM)
+  int max_seg;      // segments per CTA at most
+  long long U;      // units = pairs * n_kt
+  float2 *part_ml;  // [G][max_seg][2 tiles][BM] (max, sum), base-2 units
+  float *part_o;    // [G][max_seg][2 tiles][BM][D]
+};
+
+struct PairInfo {
+  int bg, bhq_a, bhq_b, i0_a, i0_b, t_a, t_b;
+};
+__device__ __forceinline__ PairInfo pair_info(int pidx, const TcParams &p) {
+  PairInfo r;
+  r.bg = pidx / p.ctas_per_group;
+  const int cpi = pidx - r.bg * p.ctas_per_group;
+  const int b = r.bg / p.Hk, g = r.bg - b * p.Hk;
+  const int qa = 2 * cpi, qb = qa + 1;
+  const int hl_a = qa / p.tiles, hl_b = qb / p.tiles;
+  r.t_a = qa - hl_a * p.tiles;
+  r.t_b = qb - hl_b * p.tiles;
+  r.bhq_a = b * p.Hq + g * p.q_g + hl_a;
+  r.bhq_b = b * p.Hq + g * p.q_g + hl_b;
+  r.i0_a = r.t_a * BM;
+  r.i0_b = r.t_b * BM;
+  return r;
+}
+
+// First unit of CTA c.
+__device__ __forceinline__ long long unit0(int c, const SplitParams &sp) {
+  return (sp.U * (long long)c) / sp.G;
+}
+// Segments of this CTA: pair p, tiles [kt0, kt1), and the segment's index in range
+// order (its slot in the partial buffers).  A range that starts inside a pair
+// processes that first piece last, so that every CTA sweeps its K/V tiles from tile 0
+// upwards at about the same time as the others: the tiles a group's CTAs share are
+// then read within a short window and stay in L2.
+struct SegIter {
+  long long u, u1;   // the rest of the range in natural order
+  long long f0, f1;  // the rotated first piece (empty if none)
+  long long ubase;   // first unit of the range
+  int n_kt;
+  __device__ __forceinline__ bool take(long long &a, long long b, int &p, int &kt0, int &kt1) {
+    p = (int)(a / n_kt);
+    kt0 = (int)(a - (long long)p * n_kt);
+    kt1 = (int)min((long long)n_kt, kt0 + (b - a));
+    a += kt1 - kt0;
+    return true;
+  }
+  __device__ __forceinline__ bool next(int &p, int &kt0, int &kt1, int &slot) {
+    if (u < u1) take(u, u1, p, kt0, kt1);
+    else if (f0 < f1) take(f0, f1, p, kt0, kt1);
+    else return false;
+    slot = p - (int)(ubase / n_kt);
+    return true;
+  }
+};
+__device__ __forceinline__ SegIter seg_iter(const SplitParams &sp) {
+  SegIter it;
+  it.n_kt = sp.t.n_kt;
+  it.ubase = unit0(blockIdx.x, sp);
+  it.u1 = unit0(blockIdx.x + 1, sp);
+  const long long kt0 = it.ubase % it.n_kt;
+  const long long first_end = min(it.u1, it.ubase + (it.n_kt - kt0));
+  if (kt0 > 0 && first_end < it.u1) {  // starts inside a pair and holds more
+    it.f0 = it.ubase;
+    it.f1 = first_end;
+    it.u = first_end;
+  } else {
+    it.f0 = it.f1 = 0;
+    it.u = it.ubase;
+  }
+  return it;
+}
+// CTAs whose ranges hold units of pair p: [c_first, c_last]; segment slot of p in c.
+__device__ __forceinline__ int cta_of_unit(long long x, const SplitParams &sp) {
+  // largest c with floor(U c / G) <= x
+  return (int)(((x + 1) * sp.G + sp.U - 1) / sp.U) - 1;
+}
+__device__ __forceinline__ int seg_slot(int p, int c, const SplitParams &sp) {
+  return p - (int)(unit0(c, sp) / sp.t.n_kt);
+}
+
+enum {
+  SA_Q = 0, SA_QFREE, SA_SFULL0, SA_SFULL1, SA_SFREE0, SA_SFREE1, SA_DRAIN,
+  SA_AFULL0, SA_AEMPTY0 = SA_AFULL0 + kStagesA, SA_END = SA_AEMPTY0 + kStagesA
+};
+static_assert(SA_END <= NBAR, "split A barriers");
+
+__global__ void __launch_bounds__(kThreads, 1)
+    attn_split_a_kernel(const __grid_constant__ CUtensorMap q_map,
+                        const __grid_constant__ CUtensorMap k_map, const SplitParams sp) {
+  extern __shared__ __align__(1024) uint8_t smem[];
+  const TcParams &p = sp.t;
+  const uint32_t sbase = smem_u32(smem);
+  if (sbase & 1023u) {
+    if (threadIdx.x == 0) atomicExch(p.status, H2OKV_ERR_CUDA);
+    return;
+  }
+  uint64_t *bar = reinterpret_cast<uint64_t *>(smem + OFF_BAR);
+  uint32_t *tmem_s = reinterpret_cast<uint32_t *>(smem + OFF_TMEM);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const uint64_t lim = p.timeout_ns;
+  if (threadIdx.x == 0) {
+    mbar_init(&bar[SA_Q], 1);
+    mbar_init(&bar[SA_QFREE], 1);
+    mbar_init(&bar[SA_DRAIN], 1);
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&bar[SA_SFULL0 + i], 1);
+      mbar_init(&bar[SA_SFREE0 + i], 8);
+    }
+    for (int i = 0; i < kStagesA; ++i) {
+      mbar_init(&bar[SA_AFULL0 + i], 1);
+      mbar_init(&bar[SA_AEMPTY0 + i], 1 + 8);
+    }
+    fence_mbar_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_s, kTmemCols);
+    tmem_relinquish();
+    tc_fence_before();
+  }
+  if (warp == 0 && lane == 0) {
+    prefetch_tensormap(&q_map);
+    prefetch_tensormap(&k_map);
+  }
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_s;
+  bool aborted = false;
+
+  if (warp < 4) {
+    reg_dealloc<kCtrlRegs>();
+    if (warp == 0) {
+      // ---------------------------------------- Q per segment, K tiles, token positions
+      SegIter si = seg_iter(sp);
+      int pidx, kt0, kt1, slot, sidx = 0, it = 0;
+      while (!aborted && si.next(pidx, kt0, kt1, slot)) {
+        const PairInfo pi = pair_info(pidx, p);
+        if (sidx > 0 && !warp_wait(&bar[SA_QFREE], (sidx - 1) & 1, lim)) { fail(p, aborted); break; }
+        if (lane == 0) {
+          mbar_expect_tx(&bar[SA_Q], 2 * kTileBytes);
+          tma_load_3d(smem + OFF_QA, &q_map, &bar[SA_Q], 0, pi.i0_a, pi.bhq_a);
+          tma_load_3d(smem + OFF_QA + kHalfBytes, &q_map, &bar[SA_Q], 64, pi.i0_a, pi.bhq_a);
+          tma_load_3d(smem + OFF_QB, &q_map, &bar[SA_Q], 0, pi.i0_b, pi.bhq_b);
+          tma_load_3d(smem + OFF_QB + kHalfBytes, &q_map, &bar[SA_Q], 64, pi.i0_b, pi.bhq_b);
+          mbar_arrive(&bar[SA_Q]);
+        }
+        const int32_t *tpg = p.token_pos + (size_t)pi.bg * p.N_C;
+        for (int kt = kt0; kt < kt1; ++kt, ++it) {
+          const int stage = it % kStagesA, n = it / kStagesA;
+          if (n > 0 && !warp_wait(&bar[SA_AEMPTY0 + stage], (n - 1) & 1, lim)) { fail(p, aborted); break; }
+          uint64_t *full = &bar[SA_AFULL0 + stage];
+          uint8_t *kdst = smem + slot_a(stage);
+          if (lane == 0) {
+            mbar_expect_tx(full, kTileBytes);
+            tma_load_3d(kdst, &k_map, full, 0, kt * BN, pi.bg);
+            tma_load_3d(kdst + kHalfBytes, &k_map, full, 64, kt * BN, pi.bg);
+            if (kt + kPrefetch < kt1) {
+              tma_prefetch_l2_3d(&k_map, 0, (kt + kPrefetch) * BN, pi.bg);
+              tma_prefetch_l2_3d(&k_map, 64, (kt + kPrefetch) * BN, pi.bg);
+            }
+          }
+          const int nv = min(BN, p.N_C - kt * BN);
+          float *rel = reinterpret_cast<float *>(smem + OFF_REL_A) + stage * BN;
+#pragma unroll
+          for (int e = lane; e < BN; e += 32) {
+            const int64_t t = e < nv ? (int64_t)tpg[kt * BN + e] : (int64_t)kEmptyPos;
+            const int64_t r = t - (int64_t)p.P;
+            rel[e] = (float)(r < -1 ? -1 : (r > kRelFar ? kRelFar : r));
+          }
+          __syncwarp();
+          if (lane == 0) mbar_arrive(full);
+        }
+        ++sidx;
+      }
+      // drain: the copies in flight land before exit
+      if (lane == 0 && sidx > 0) {
+        mbar_wait(&bar[SA_Q], (sidx - 1) & 1, 4000000000ull);
+        for (int k = it - 1; k >= 0 && k >= it - kStagesA; --k)
+          mbar_wait(&bar[SA_AFULL0 + k % kStagesA], (k / kStagesA) & 1, 4000000000ull);
+      }
+    } else if (warp == 1) {
+      // ------------------------------------------------------------------ MMA issuer
+      if (lane == 0) {
+        const uint32_t qa_addr = sbase + OFF_QA, qb_addr = sbase + OFF_QB;
+        SegIter si = seg_iter(sp);
+        int pidx, kt0, kt1, slot, sidx = 0, it = 0;
+        while (!aborted && si.next(pidx, kt0, kt1, slot)) {
+          if (!mbar_wait(&bar[SA_Q], sidx & 1, lim)) { fail(p, aborted); break; }
+          tc_fence_after();
+          for (int kt = kt0; kt < kt1; ++kt, ++it) {
+            const int a = it % kStagesA, u = it & 1;
+            if (!mbar_wait(&bar[SA_AFULL0 + a], (it / kStagesA) & 1, lim)) { fail(p, aborted); break; }
+            if (it >= 2 && !mbar_wait(&bar[SA_SFREE0 + u], ((it >> 1) - 1) & 1, lim)) {
+              fail(p, aborted);
+              break;
+            }
+            tc_fence_after();
+            const uint32_t k_addr = sbase + slot_a(a);
+#pragma unroll
+            for (int ks = 0; ks < D / 16; ++ks)
+              mma_bf16_ss(tmem + u * 256, kmajor_desc(qa_addr, ks), kmajor_desc(k_addr, ks),
+                          IDESC_K_MAJOR, ks > 0);
+#pragma unroll
+            for (int ks = 0; ks < D / 16; ++ks)
+              mma_bf16_ss(tmem + u * 256 + 128, kmajor_desc(qb_addr, ks), kmajor_desc(k_addr, ks),
+                          IDESC_K_MAJOR, ks > 0);
+            mma_commit(&bar[SA_SFULL0 + u]);
+            mma_commit(&bar[SA_AEMPTY0 + a]);
+          }
+          mma_commit(&bar[SA_QFREE]);  // this segment's Q tiles are no longer read
+          ++sidx;
+        }
+        mma_commit(&bar[SA_DRAIN]);
+        mbar_wait(&bar[SA_DRAIN], 0, 4000000000ull);
+      }
+      __syncwarp();
+    }
+  } else {
+    reg_alloc<kSoftRegs>();
+    // ---------------------------- online (max, sum) per row, one warpgroup per query tile
+    const int wg = (warp - 4) >> 2;
+    const int st = threadIdx.x - 128 * (1 + wg);
+    const uint32_t lane_base = (uint32_t)(32 * (warp & 3)) << 16;
+    const float c2 = p.scale2;
+    const float mbias = kMaskBias / c2;
+    SegIter si = seg_iter(sp);
+    int pidx, kt0, kt1, slot, sidx = 0, it = 0;
+    uint32_t x[BN];
+    while (!aborted && si.next(pidx, kt0, kt1, slot)) {
+      const PairInfo pi = pair_info(pidx, p);
+      const int i0 = wg ? pi.i0_b : pi.i0_a;
+      float m = -INFINITY, l = 0.f;
+      for (int kt = kt0; kt < kt1 && !aborted; ++kt, ++it) {
+        const int u = it & 1, a = it % kStagesA;
+        if (!warp_wait(&bar[SA_SFULL0 + u], (it >> 1) & 1, lim)) { fail(p, aborted); break; }
+        if (!warp_wait(&bar[SA_AFULL0 + a], (it / kStagesA) & 1, lim)) { fail(p, aborted); break; }
+        tc_fence_after();
+        const float *rela = reinterpret_cast<const float *>(smem + OFF_REL_A) + a * BN;
+        const float rv = fmax3(fmaxf(rela[lane], rela[lane + 32]), rela[lane + 64], rela[lane + 96]);
+        const bool masked = __any_sync(0xffffffffu, rv > (float)i0);
+        const uint32_t sa = tmem + lane_base + u * 256 + wg * 128;
+        tmem_ld32(sa, *reinterpret_cast<uint32_t(*)[32]>(x));
+        tmem_ld32(sa + 32, *reinterpret_cast<uint32_t(*)[32]>(x + 32));
+        tmem_ld32(sa + 64, *reinterpret_cast<uint32_t(*)[32]>(x + 64));
+        tmem_ld32(sa + 96, *reinterpret_cast<uint32_t(*)[32]>(x + 96));
+        tmem_wait_ld();
+        if (masked) row_mask<BN>(x, rela, (float)(i0 + st), mbias);
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) {
+          mbar_arrive(&bar[SA_SFREE0 + u]);
+          mbar_arrive(&bar[SA_AEMPTY0 + a]);
+        }
+        row_update<BN>(x, c2, m, l);
+      }
+      if (aborted) break;
+      sp.part_ml[((size_t)blockIdx.x * sp.max_seg + slot) * (2 * BM) + wg * BM + st] = make_float2(m, l);
+      ++sidx;
+    }
+    tc_fence_before();
+  }
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, kTmemCols);
+  }
+}
+
+enum {
+  SB_Q = 0, SB_QFREE, SB_KFULL0, SB_KFULL1, SB_KEMPTY0, SB_KEMPTY1, SB_VFULL0, SB_VFULL1,
+  SB_VEMPTY0, SB_VEMPTY1, SB_TFULLA, SB_TFULLB, SB_TFREEA, SB_TFREEB, SB_PFULLA, SB_PFULLB,
+  SB_PFREEA, SB_PFREEB, SB_OFULL, SB_OFREE, SB_DRAIN, SB_END
+};
+static_assert(SB_END <= NBAR, "split B barriers");
+
+__global__ void __launch_bounds__(kThreads, 1)
+    attn_split_b_kernel(const __grid_constant__ CUtensorMap q_map,
+                        const __grid_constant__ CUtensorMap k_map,
+                        const __grid_constant__ CUtensorMap v_map, const SplitParams sp) {
+  extern __shared__ __align__(1024) uint8_t smem[];
+  const TcParams &p = sp.t;
+  const uint32_t sbase = smem_u32(smem);
+  if (sbase & 1023u) {
+    if (threadIdx.x == 0) atomicExch(p.status, H2OKV_ERR_CUDA);
+    return;
+  }
+  int32_t *tp_s = reinterpret_cast<int32_t *>(smem + OFF_TP);
+  float *lse_s = reinterpret_cast<float *>(smem + OFF_LSE);
+  uint64_t *bar = reinterpret_cast<uint64_t *>(smem + OFF_BAR);
+  uint32_t *tmem_s = reinterpret_cast<uint32_t *>(smem + OFF_TMEM);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const uint64_t lim = p.timeout_ns;
+  if (threadIdx.x == 0) {
+    mbar_init(&bar[SB_Q], 1);
+    mbar_init(&bar[SB_QFREE], 1);
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&bar[SB_KFULL0 + i], 1);
+      mbar_init(&bar[SB_KEMPTY0 + i], 1 + 8);  // MMA commit + softmax warps (token positions)
+      mbar_init(&bar[SB_VFULL0 + i], 1);
+      mbar_init(&bar[SB_VEMPTY0 + i], 1);
+    }
+    mbar_init(&bar[SB_TFULLA], 1);
+    mbar_init(&bar[SB_TFULLB], 1);
+    mbar_init(&bar[SB_TFREEA], 4);
+    mbar_init(&bar[SB_TFREEB], 4);
+    mbar_init(&bar[SB_PFULLA], 4);
+    mbar_init(&bar[SB_PFULLB], 4);
+    mbar_init(&bar[SB_PFREEA], 1);
+    mbar_init(&bar[SB_PFREEB], 1);
+    mbar_init(&bar[SB_OFULL], 1);
+    mbar_init(&bar[SB_OFREE], 8);
+    mbar_init(&bar[SB_DRAIN], 1);
+    fence_mbar_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_s, kTmemCols);
+    tmem_relinquish();
+    tc_fence_before();
+  }
+  if (warp == 0 && lane == 0) {
+    prefetch_tensormap(&q_map);
+    prefetch_tensormap(&k_map);
+    prefetch_tensormap(&v_map);
+  }
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_s;
+  bool aborted = false;
+
+  if (warp < 4) {
+    reg_dealloc<kCtrlRegs>();
+    if (warp == 0) {
+      // ---------------------------------------- Q per segment, K tiles, token positions
+      SegIter si = seg_iter(sp);
+      int pidx, kt0, kt1, slot, sidx = 0, it = 0;
+      while (!aborted && si.next(pidx, kt0, kt1, slot)) {
+        const PairInfo pi = pair_info(pidx, p);
+        if (sidx > 0 && !warp_wait(&bar[SB_QFREE], (sidx - 1) & 1, lim)) { fail(p, aborted); break; }
+        if (lane == 0) {
+          mbar_expect_tx(&bar[SB_Q], 2 * kTileBytes);
+          tma_load_3d(smem + OFF_QA, &q_map, &bar[SB_Q], 0, pi.i0_a, pi.bhq_a);
+          tma_load_3d(smem + OFF_QA + kHalfBytes, &q_map, &bar[SB_Q], 64, pi.i0_a, pi.bhq_a);
+          tma_load_3d(smem + OFF_QB, &q_map, &bar[SB_Q], 0, pi.i0_b, pi.bhq_b);
+          tma_load_3d(smem + OFF_QB + kHalfBytes, &q_map, &bar[SB_Q], 64, pi.i0_b, pi.bhq_b);
+          mbar_arrive(&bar[SB_Q]);
+        }
+        const int32_t *tpg = p.token_pos + (size_t)pi.bg * p.N_C;
+        for (int kt = kt0; kt < kt1; ++kt, ++it) {
+          const int s = it & 1;
+          if (it >= 2 && !warp_wait(&bar[SB_KEMPTY0 + s], ((it >> 1) - 1) & 1, lim)) {
+            fail(p, aborted);
+            break;
+          }
+          uint64_t *full = &bar[SB_KFULL0 + s];
+          uint8_t *kdst = smem + (s ? OFF_K1 : OFF_K0);
+          if (lane == 0) {
+            mbar_expect_tx(full, kTileBytes);
+            tma_load_3d(kdst, &k_map, full, 0, kt * BN, pi.bg);
+            tma_load_3d(kdst + kHalfBytes, &k_map, full, 64, kt * BN, pi.bg);
+            if (kt + kPrefetch < kt1) {
+              tma_prefetch_l2_3d(&k_map, 0, (kt + kPrefetch) * BN, pi.bg);
+              tma_prefetch_l2_3d(&k_map, 64, (kt + kPrefetch) * BN, pi.bg);
+            }
+          }
+          const int nv = min(BN, p.N_C - kt * BN);
+          float *rel = reinterpret_cast<float *>(tp_s) + s * BN;
+#pragma unroll
+          for (int e = lane; e < BN; e += 32) {
+            const int64_t t = e < nv ? (int64_t)tpg[kt * BN + e] : (int64_t)kEmptyPos;
+            const int64_t r = t - (int64_t)p.P;
+            rel[e] = (float)(r < -1 ? -1 : (r > kRelFar ? kRelFar : r));
+          }
+          __syncwarp();
+          if (lane == 0) mbar_arrive(full);
+        }
+        ++sidx;
+      }
+      if (lane == 0 && sidx > 0) {
+        mbar_wait(&bar[SB_Q], (sidx - 1) & 1, 4000000000ull);
+        for (int k = it - 1; k >= 0 && k >= it - 2; --k)
+          mbar_wait(&bar[SB_KFULL0 + (k & 1)], (k >> 1) & 1, 4000000000ull);
+      }
+    } else if (warp == 2) {
+      // ------------------------------------------------------------------ V tiles
+      if (lane == 0) {
+        SegIter si = seg_iter(sp);
+        int pidx, kt0, kt1, slot, it = 0;
+        while (!aborted && si.next(pidx, kt0, kt1, slot)) {
+          const int bg = pidx / p.ctas_per_group;
+          for (int kt = kt0; kt < kt1; ++kt, ++it) {
+            const int vs = it & 1;
+            if (it >= 2 && !mbar_wait(&bar[SB_VEMPTY0 + vs], ((it >> 1) - 1) & 1, lim)) {
+              fail(p, aborted);
+              break;
+            }
+            uint8_t *vdst = smem + (vs ? OFF_V1 : OFF_V0);
+            mbar_expect_tx(&bar[SB_VFULL0 + vs], kTileBytes);
+            tma_load_3d(vdst, &v_map, &bar[SB_VFULL0 + vs], 0, kt * BN, bg);
+            tma_load_3d(vdst + kHalfBytes, &v_map, &bar[SB_VFULL0 + vs], 64, kt * BN, bg);
+            mbar_arrive(&bar[SB_VFULL0 + vs]);
+            if (kt + kPrefetch < kt1) {
+              tma_prefetch_l2_3d(&v_map, 0, (kt + kPrefetch) * BN, bg);
+              tma_prefetch_l2_3d(&v_map, 64, (kt + kPrefetch) * BN, bg);
+            }
+          }
+        }
+        for (int k = it - 1; k >= 0 && k >= it - 2; --k)
+          mbar_wait(&bar[SB_VFULL0 + (k & 1)], (k >> 1) & 1, 4000000000ull);
+      }
+      __syncwarp();
+    } else if (warp == 1) {
+      // ------------------------------------------------------------------ MMA issuer
+      if (lane == 0) {
+        const uint32_t qa_addr = sbase + OFF_QA, qb_addr = sbase + OFF_QB, p_addr = sbase + OFF_P;
+        // S^T_x(it) = K Q_x^T into columns 0 (a) / 128 (b); O_x += P_x V into 256 (a) / 384 (b)
+        auto issue_st = [&](int it, bool tile_b) -> bool {
+          const int s = it & 1;
+          if (!tile_b && !mbar_wait(&bar[SB_KFULL0 + s], (it >> 1) & 1, lim)) return false;
+          if (it >= 1 && !mbar_wait(&bar[tile_b ? SB_TFREEB : SB_TFREEA], (it - 1) & 1, lim))
+            return false;
+          tc_fence_after();
+          const uint32_t k_addr = sbase + (s ? OFF_K1 : OFF_K0);
+          const uint32_t q_addr = tile_b ? qb_addr : qa_addr;
+#pragma unroll
+          for (int ks = 0; ks < D / 16; ++ks)
+            mma_bf16_ss(tmem + (tile_b ? 128 : 0), kmajor_desc(k_addr, ks), kmajor_desc(q_addr, ks),
+                        IDESC_K_MAJOR, ks > 0);
+          mma_commit(&bar[tile_b ? SB_TFULLB : SB_TFULLA]);
+          if (tile_b) mma_commit(&bar[SB_KEMPTY0 + s]);
+          return true;
+        };
+        auto issue_pv = [&](int it, bool tile_b, bool first) -> bool {
+          if (!mbar_wait(&bar[tile_b ? SB_PFULLB : SB_PFULLA], it & 1, lim)) return false;
+          if (!tile_b && !mbar_wait(&bar[SB_VFULL0 + (it & 1)], (it >> 1) & 1, lim)) return false;
+          tc_fence_after();
+          const uint32_t v_addr = sbase + ((it & 1) ? OFF_V1 : OFF_V0);
+#pragma unroll
+          for (int ks = 0; ks < BN / 16; ++ks)
+            mma_bf16_ss(tmem + (tile_b ? 384 : 256), mnmajor_desc(p_addr, ks),
+                        mnmajor_desc(v_addr, ks), IDESC_PV, (!first || ks > 0) ? 1u : 0u);
+          mma_commit(&bar[tile_b ? SB_PFREEB : SB_PFREEA]);
+          if (tile_b) mma_commit(&bar[SB_VEMPTY0 + (it & 1)]);
+          return true;
+        };
+        SegIter si = seg_iter(sp);
+        int pidx, kt0, kt1, slot, sidx = 0, it = 0;
+        while (!aborted && si.next(pidx, kt0, kt1, slot)) {
+          const int n = kt1 - kt0;
+          if (!mbar_wait(&bar[SB_Q], sidx & 1, lim)) { fail(p, aborted); break; }
+          // the previous segment's O has been read out of TMEM
+          if (sidx > 0 && !mbar_wait(&bar[SB_OFREE], (sidx - 1) & 1, lim)) { fail(p, aborted); break; }
+          tc_fence_after();
+          bool ok = issue_st(it, false) && issue_st(it, true);
+          for (int j = 0; ok && j < n; ++j) {
+            if (j + 1 < n) ok = issue_st(it + j + 1, false) && issue_st(it + j + 1, true);
+            if (ok && j + 1 == n) mma_commit(&bar[SB_QFREE]);  // no later MMA of this segment reads Q
+            if (ok) ok = issue_pv(it + j, false, j == 0) && issue_pv(it + j, true, j == 0);
+          }
+          if (!ok) { fail(p, aborted); break; }
+          mma_commit(&bar[SB_OFULL]);
+          it += n;
+          ++sidx;
+        }
+        mma_commit(&bar[SB_DRAIN]);
+        mbar_wait(&bar[SB_DRAIN], 0, 4000000000ull);
+      }
+      __syncwarp();
+    }
+  } else {
+    reg_alloc<kSoftRegs>();
+    // ------------------------ per-slot probabilities, sums and epilogue, one warpgroup per tile
+    const int wg = (warp - 4) >> 2;
+    const int st = threadIdx.x - 128 * (1 + wg);
+    const uint32_t lane_base = (uint32_t)(32 * (warp & 3)) << 16;
+    const float c2 = p.scale2;
+    float *lse_t = lse_s + wg * BM;  // -lse2 of the tile's rows
+    const uint32_t p_row = sbase + OFF_P + (st >> 3) * 1024 + (st & 7) * 128;
+    SegIter si = seg_iter(sp);
+    int pidx, kt0, kt1, slot, sidx = 0, it = 0;
+    // every warp of the warpgroup meets the same named barriers in every segment, also
+    // after a failed wait (the work is then skipped), so none of them waits forever
+    while (si.next(pidx, kt0, kt1, slot)) {
+      const PairInfo pi = pair_info(pidx, p);
+      const int i0 = wg ? pi.i0_b : pi.i0_a, bhq = wg ? pi.bhq_b : pi.bhq_a, t = wg ? pi.t_b : pi.t_a;
+      // the final LSE of row st: combine the pair's partial (max, sum) in CTA order
+      const int c_first = cta_of_unit((long long)pidx * p.n_kt, sp);
+      const int c_last = cta_of_unit((long long)(pidx + 1) * p.n_kt - 1, sp);
+      float m = -INFINITY;
+      for (int c = c_first; c <= c_last; ++c)
+        m = fmaxf(m, sp.part_ml[((size_t)c * sp.max_seg + seg_slot(pidx, c, sp)) * (2 * BM) + wg * BM + st].x);
+      float l = 0.f;
+      if (m != -INFINITY)
+        for (int c = c_first; c <= c_last; ++c) {
+          const float2 ml = sp.part_ml[((size_t)c * sp.max_seg + seg_slot(pidx, c, sp)) * (2 * BM) + wg * BM + st];
+          l += ml.y * ex2(ml.x - m);
+        }
+      const bool seen = l > 0.f && m > -0.5f * kMaskBias;
+      const float lse2 = seen ? m + lg2(l) : -INFINITY;
+      named_bar_sync(1 + wg, 128);  // the previous segment's reads of lse_t are done
+      lse_t[st] = seen ? -lse2 : -kMaskBias;
+      if (p.lse_out && kt0 == 0 && i0 + st < p.S)
+        p.lse_out[(size_t)bhq * p.S + i0 + st] = lse2 * 0.69314718055994531f;
+      named_bar_sync(1 + wg, 128);
+      const int rmax = min(BM, p.S - i0);
+      float *pw = p.part_w + ((size_t)bhq * p.tiles + t) * p.N_C;
+      uint32_t pk[BM / 2];
+      for (int kt = kt0; kt < kt1 && !aborted; ++kt, ++it) {
+        const int s = it & 1;
+        const int j = kt * BN + st;
+        if (!warp_wait(&bar[wg ? SB_TFULLB : SB_TFULLA], it & 1, lim)) { fail(p, aborted); break; }
+        if (!warp_wait(&bar[SB_KFULL0 + s], (it >> 1) & 1, lim)) { fail(p, aborted); break; }
+        tc_fence_after();
+        const float relj = __int_as_float(tp_s[s * BN + st]);
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&bar[SB_KEMPTY0 + s]);
+        const float rmf = fminf(fmaxf(relj - (float)i0, 0.f), (float)BM);
+        const int rmin = (int)rmf;
+        const bool full = __all_sync(0xffffffffu, rmin == 0 && rmax == BM);
+        uint32_t r[BM];
+        tmem_ld128(tmem + lane_base + wg * 128, r);
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&bar[wg ? SB_TFREEB : SB_TFREEA]);
+        const float cs = slot_probs(r, lse_t, c2, rmin, rmax, full, pk);
+        // the single P buffer goes a(it) -> b(it) -> a(it + 1)
+        bool ok = true;
+        if (wg == 1)
+          ok = warp_wait(&bar[SB_PFREEA], it & 1, lim);
+        else if (it > 0)
+          ok = warp_wait(&bar[SB_PFREEB], (it - 1) & 1, lim);
+        if (!ok) { fail(p, aborted); break; }
+        store_p(p_row, st, pk);
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&bar[wg ? SB_PFULLB : SB_PFULLA]);
+        if (j < p.N_C) pw[j] = cs;
+      }
+      // epilogue of the segment: y, or this segment's share of O when the pair is split
+      if (!aborted && !warp_wait(&bar[SB_OFULL], sidx & 1, lim)) fail(p, aborted);
+      if (aborted) {
+        ++sidx;
+        continue;
+      }
+      tc_fence_after();
+      const bool whole = kt0 == 0 && kt1 == p.n_kt;
+      const int row_i = i0 + st;
+      __nv_bfloat16 *yrow = p.y + ((size_t)bhq * p.S + row_i) * D;
+      float *orow = sp.part_o + ((((size_t)blockIdx.x * sp.max_seg + slot) * 2 + wg) * BM + st) * D;
+      uint32_t o32[32];
+#pragma unroll
+      for (int cq = 0; cq < 4; ++cq) {
+        tmem_ld32(tmem + lane_base + 256 + wg * 128 + cq * 32, o32);
+        tmem_wait_ld();
+        if (whole) {
+          if (row_i < p.S) {
+            uint32_t o[16];
+#pragma unroll
+            for (int e = 0; e < 16; ++e)
+              o[e] = pack_bf16x2(__uint_as_float(o32[2 * e]), __uint_as_float(o32[2 * e + 1]));
+            uint4 *dst = reinterpret_cast<uint4 *>(yrow + cq * 32);
+#pragma unroll
+            for (int e = 0; e < 4; ++e)
+              dst[e] = make_uint4(o[4 * e], o[4 * e + 1], o[4 * e + 2], o[4 * e + 3]);
+          }
+        } else {
+          uint4 *dst = reinterpret_cast<uint4 *>(orow + cq * 32);
+#pragma unroll
+          for (int e = 0; e < 8; ++e)
+            dst[e] = make_uint4(o32[4 * e], o32[4 * e + 1], o32[4 * e + 2], o32[4 * e + 3]);
+        }
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&bar[SB_OFREE]);
+      ++sidx;
+    }
+    tc_fence_before();
+  }
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, kTmemCols);
+  }
+}
+
+// y of the pairs whose slots were split over several CTAs: the sum of their partial
+// O rows in CTA order.  One thread per 4 columns of one row (pair, tile, row, column
+// group), so that every load of the pass is in flight at once.
+__global__ void __launch_bounds__(256)
+    reduce_o_kernel(const SplitParams sp, int n_pairs) {
+  const TcParams &p = sp.t;
+  const long long e = (long long)blockIdx.x * blockDim.x + threadIdx.x;
+  const long long per_pair = 2LL * BM * (D / 4);
+  const int pidx = (int)(e / per_pair);
+  if (pidx >= n_pairs) return;
+  const int rem = (int)(e - (long long)pidx * per_pair);
+  const int wg = rem / (BM * (D / 4));
+  const int row = (rem / (D / 4)) % BM, c4 = rem % (D / 4);
+  const int c_first = cta_of_unit((long long)pidx * p.n_kt, sp);
+  const int c_last = cta_of_unit((long long)(pidx + 1) * p.n_kt - 1, sp);
+  if (c_first == c_last) return;  // written by its only CTA
+  const PairInfo pi = pair_info(pidx, p);
+  const int i0 = wg ? pi.i0_b : pi.i0_a, bhq = wg ? pi.bhq_b : pi.bhq_a;
+  if (i0 + row >= p.S) return;
+  float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+  for (int c = c_first; c <= c_last; ++c) {
+    const float4 v = __ldcs(reinterpret_cast<const float4 *>(
+        sp.part_o + ((((size_t)c * sp.max_seg + seg_slot(pidx, c, sp)) * 2 + wg) * BM + row) * D) + c4);
+    acc.x += v.x;
+    acc.y += v.y;
+    acc.z += v.z;
+    acc.w += v.w;
+  }
+  __nv_bfloat162 *dst =
+      reinterpret_cast<__nv_bfloat162 *>(p.y + ((size_t)bhq * p.S + i0 + row) * D + c4 * 4);
+  dst[0] = __floats2bfloat162_rn(acc.x, acc.y);
+  dst[1] = __floats2bfloat162_rn(acc.z, acc.w);
+}
+
 // w[b, g, j] = sum over the group's heads and row tiles of the partial sums;
 // wq[b, h, j] = sum over the head's row tiles.  Fixed summation order.
 __global__ void __launch_bounds__(256)
@@ -1249,10 +1899,48 @@ bool tc_path_supported(const h2okv_cache_desc &d) {
          (d.kv_dtype == H2OKV_BF16 || d.kv_dtype == H2OKV_I8 || d.kv_dtype == H2OKV_I4);
 }
 
+namespace {
+// Split scheduling pays when one CTA per pair of query tiles leaves many SMs idle in
+// the last wave; it needs two query tiles in every pair and a few tiles per CTA.
+struct SplitShape {
+  bool use;
+  long long U;
+  int max_seg;
+};
+SplitShape split_shape(const h2okv_cache_desc &d, int S, int G) {
+  SplitShape r{false, 0, 0};
+  if (G <= 0 || d.kv_dtype != H2OKV_BF16) return r;
+  const int tiles = (S + BM - 1) / BM;
+  const int n_qt = (d.n_q_heads / d.n_kv_heads) * tiles;
+  if (n_qt % 2) return r;
+  const long long pairs = (long long)d.batch * d.n_kv_heads * (n_qt / 2);
+  const int n_kt = (d.capacity + BN - 1) / BN;
+  r.U = pairs * n_kt;
+  const long long waves = (pairs + G - 1) / G;
+  const double fill = (double)pairs / (double)(waves * G);
+  if (fill >= 0.95 || r.U < 4LL * G || n_kt < 4) return r;
+  const long long per = (r.U + G - 1) / G;  // units of one CTA at most
+  r.max_seg = (int)((per + n_kt - 1) / n_kt) + 1;
+  r.use = true;
+  return r;
+}
+}  // namespace
+
 void tc_plan(const h2okv_cache_desc &d, TcPlan *plan) {
   plan->enabled = tc_path_supported(d);
   plan->tiles_per_head = (d.max_chunk + BM - 1) / BM;
-  plan->max_splits = 0;
+  plan->split_ctas = 0;
+  plan->max_seg = 0;
+  int dev = 0, sms = 0;
+  if (plan->enabled && cudaGetDevice(&dev) == cudaSuccess &&
+      cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) == cudaSuccess) {
+    const SplitShape sh = split_shape(d, d.max_chunk, sms);
+    if (sh.use) {
+      plan->split_ctas = sms;
+      plan->max_seg = sh.max_seg;
+    }
+  }
+  cudaGetLastError();  // a failed query (no device) is not an error here
 }
 
 namespace {
@@ -1279,6 +1967,27 @@ int prepare_kernel() {
     return set_error(H2OKV_ERR_UNSUPPORTED,
                      "attn_tc_kernel built with %d registers per thread, expected %d", fa.numRegs,
                      kLaunchRegs);
+  ready_dev = dev;
+  return H2OKV_OK;
+}
+
+// The same set-up for a split kernel.
+template <typename K>
+int prepare_split_kernel(K kernel, int &ready_dev, const char *name) {
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (ready_dev == dev) return H2OKV_OK;
+  cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       (int)kSmemBytes);
+  if (e != cudaSuccess)
+    return set_error(H2OKV_ERR_CUDA, "cudaFuncSetAttribute(%s): %s", name, cudaGetErrorString(e));
+  cudaFuncAttributes fa;
+  e = cudaFuncGetAttributes(&fa, kernel);
+  if (e != cudaSuccess)
+    return set_error(H2OKV_ERR_CUDA, "cudaFuncGetAttributes(%s): %s", name, cudaGetErrorString(e));
+  if (fa.numRegs != kLaunchRegs)
+    return set_error(H2OKV_ERR_UNSUPPORTED, "%s built with %d registers per thread, expected %d",
+                     name, fa.numRegs, kLaunchRegs);
   ready_dev = dev;
   return H2OKV_OK;
 }
@@ -1341,6 +2050,37 @@ int launch_attn_tc(h2okv_cache *c, const void *q, int S, int64_t P, void *y, flo
   const int grid = d.batch * d.n_kv_heads * prm.ctas_per_group;
   const CUtensorMap &kmap = *reinterpret_cast<const CUtensorMap *>(c->tc.k_map);
   const CUtensorMap &vmap = *reinterpret_cast<const CUtensorMap *>(c->tc.v_map);
+  // split scheduling: every SM gets the same share of (pair, K/V tile) units
+  const SplitShape sh = split_shape(d, S, c->tc.split_ctas);
+  if (sh.use && sh.max_seg <= c->tc.max_seg) {
+    static thread_local int ready_a = -1, ready_b = -1;
+    rc = prepare_split_kernel(attn_split_a_kernel, ready_a, "attn_split_a_kernel");
+    if (rc) return rc;
+    rc = prepare_split_kernel(attn_split_b_kernel, ready_b, "attn_split_b_kernel");
+    if (rc) return rc;
+    SplitParams sp;
+    sp.t = prm;
+    sp.G = c->tc.split_ctas;
+    sp.max_seg = c->tc.max_seg;
+    sp.U = sh.U;
+    sp.part_ml = reinterpret_cast<float2 *>(ws + c->ws.part_ml);
+    sp.part_o = reinterpret_cast<float *>(ws + c->ws.part_o);
+    attn_split_a_kernel<<<sp.G, kThreads, kSmemBytes, st>>>(qmap, kmap, sp);
+    rc = check_launch("attn_split_a_kernel");
+    if (rc) return rc;
+    attn_split_b_kernel<<<sp.G, kThreads, kSmemBytes, st>>>(qmap, kmap, vmap, sp);
+    rc = check_launch("attn_split_b_kernel");
+    if (rc) return rc;
+    const int n_pairs = grid;
+    const long long n_threads = (long long)n_pairs * 2 * BM * (D / 4);
+    reduce_o_kernel<<<(unsigned)((n_threads + 255) / 256), 256, 0, st>>>(sp, n_pairs);
+    rc = check_launch("reduce_o_kernel");
+    if (rc) return rc;
+    dim3 rgrid((d.capacity + 255) / 256, d.batch * d.n_kv_heads);
+    reduce_w_kernel<<<rgrid, 256, 0, st>>>(prm.part_w, w, wq, d.n_q_heads, d.n_kv_heads, prm.q_g,
+                                           d.capacity, prm.tiles, prm.tiles);
+    return check_launch("reduce_w_kernel");
+  }
   switch (d.kv_dtype) {
     case H2OKV_BF16: rc = launch_kernel<H2OKV_BF16>(grid, qmap, kmap, vmap, prm, st); break;
     case H2OKV_I8: rc = launch_kernel<H2OKV_I8>(grid, qmap, kmap, vmap, prm, st); break;

@@ -294,12 +294,14 @@ __device__ __forceinline__ void store_slice(float *dst, const float (&v)[IPT],
 }
 
 // Slot j of a chunk row set receives chunk row k: bookkeeping of the slot (old token
-// position to the delta output, new token position, score 0, slot list).
-__device__ __forceinline__ void claim_slot(const EvictArgs &a, RowSet rs, int j, int k) {
+// position to the delta output, new token position, score 0 unless the caller stores
+// the slice's scores afterwards, slot list).
+__device__ __forceinline__ void claim_slot(const EvictArgs &a, RowSet rs, int j, int k,
+                                           bool zero_score = true) {
   const size_t gs = rs.gbase + (size_t)j, rk = rs.rbase + (size_t)k;
   if (a.dpos) a.dpos[rk] = a.token_pos[gs];
   a.token_pos[gs] = a.P + k;
-  a.scores[gs] = 0.f;
+  if (zero_score) a.scores[gs] = 0.f;
   if (a.slots_out) a.slots_out[rk] = j;
 }
 
@@ -340,6 +342,10 @@ __global__ void __launch_bounds__(kEvThreads) evict_kernel(const EvictArgs a) {
     tp[i] = kEmptyPos;
     ksum[i] = 0.f;
   }
+  // one batch row choosing for itself: its folded scores are stored once, after the
+  // choice, with the chosen slots at 0 (the stores then overlap nothing else)
+  const bool defer_store = a.mode == 2 && nb == 1;
+  bool vec0 = false;
   // ---- fold w_prev into the scores of every batch row of this set ----------------
   for (int bb = 0; bb < nb; ++bb) {
     const size_t gbase = rows_of(bb).gbase;
@@ -387,7 +393,8 @@ __global__ void __launch_bounds__(kEvThreads) evict_kernel(const EvictArgs a) {
       if (a.w_prev) sc[i] = __fadd_rn(sc[i], wp[i]);
       ksum[i] = bb == 0 ? sc[i] : __fadd_rn(ksum[i], sc[i]);  // h2o_orig: batch order
     }
-    if (a.w_prev) store_slice<IPT>(a.scores + gbase + j0, sc, valid, vec);
+    if (a.w_prev && !defer_store) store_slice<IPT>(a.scores + gbase + j0, sc, valid, vec);
+    if (bb == 0) vec0 = vec;
   }
 
   if (a.mode == 1) {
@@ -525,11 +532,13 @@ __global__ void __launch_bounds__(kEvThreads) evict_kernel(const EvictArgs a) {
       ++eq_before;
     }
     if (take) {
-      for (int bb = 0; bb < nb; ++bb) claim_slot(a, rows_of(bb), j, (int)pos);
+      if (defer_store) sc[i] = 0.f;
+      for (int bb = 0; bb < nb; ++bb) claim_slot(a, rows_of(bb), j, (int)pos, !defer_store);
       int32_t *dst = cluster.map_shared_rank(rowslot, (int)(pos % (uint32_t)CL));
       dst[pos / (uint32_t)CL] = j;
     }
   }
+  if (defer_store) store_slice<IPT>(a.scores + rows_of(0).gbase + j0, sc, valid, vec0);
   cluster.sync();  // rowslot lists complete
 
   // ---- insert the chunk's rows k = rank, rank + CL, ... -----------------------------

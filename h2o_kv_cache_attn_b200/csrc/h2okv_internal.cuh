@@ -17,9 +17,9 @@ constexpr int kMaxCapacity = 65536;
 // Workspace carve-up of one cache (all offsets 256-byte aligned).
 struct WorkspaceLayout {
   size_t lse2;         // float [B*Hq*max_chunk]: base-2 log-sum-exp per query row
-  size_t part_ml;      // float2 [splits*B*Hq*rows_pad]: split-KV partial (max, sum) for pass 1
+  size_t part_ml;      // float2 [split CTAs * segments * 2 * 128]: partial (max, sum) per row
   size_t part_w;       // float [B*Hq*row_tiles*N_C]: per-row-tile summed weights (tensor-core path)
-  size_t part_o;       // float [splits*B*Hq*rows_pad*d]: split-KV partial outputs (tensor-core path)
+  size_t part_o;       // float [split CTAs * segments * 2 * 128 * d]: partial outputs
   size_t status;       // int32: device status word (0 = ok, else an H2OKV_ERR_* code)
   size_t total;
 };
@@ -27,7 +27,8 @@ struct WorkspaceLayout {
 struct TcPlan {          // launch plan of the tensor-core path
   bool enabled;
   int tiles_per_head;    // ceil(max_chunk / 128)
-  int max_splits;        // key splits the workspace is sized for
+  int split_ctas;        // CTAs of the split (persistent) kernels, 0 = split scheduling off
+  int max_seg;           // segments per CTA the split workspace is sized for
   bool maps_ready;       // k_map / v_map encoded
   alignas(64) unsigned char k_map[128];  // CUtensorMap over keys
   alignas(64) unsigned char v_map[128];  // CUtensorMap over values

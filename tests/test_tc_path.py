@@ -46,6 +46,22 @@ QCASES = [
 ]
 
 
+# Shapes whose one-CTA-per-pair grid would leave most SMs idle: the two passes run as
+# persistent kernels over equal shares of (pair, K/V tile) units, most pairs split over
+# several CTAs (partial LSE combined, partial outputs summed).
+SPLIT_CASES = [
+    tc("tc_split_c8192_s512", capacity=8192, chunk=512, seq_len=9216),
+    tc("tc_split_c8000_s300_ragged", capacity=8000, chunk=300, seq_len=8600),
+]
+
+
+@pytest.mark.parametrize("wl", SPLIT_CASES, ids=[w.name for w in SPLIT_CASES])
+def test_split_schedule(wl, cuda_device):
+    last = wl.n_chunks - 1
+    run, n = run_and_check(wl, cuda_device, check_chunks={0, last - 1, last})
+    assert n == 3
+
+
 @pytest.mark.parametrize("wl", CASES + QCASES, ids=[w.name for w in CASES + QCASES])
 def test_tc_workload_every_chunk(wl, cuda_device):
     run, n = run_and_check(wl, cuda_device)
