@@ -169,7 +169,7 @@ def evict_bytes_chunk(wl, S):
 def split_schedule(wl, S, sms):
     """Whether the library runs a chunk of S tokens with the split (persistent)
     tensor-core schedule: the same rule as the library's (bf16 cache, an even number
-    of query tiles per KV group, the one-CTA-per-pair grid filling less than 95 % of
+    of query tiles per KV group, the one-CTA-per-pair grid filling less than 75 % of
     its last wave, at least 4 units per SM and 4 K/V tiles)."""
     if wl.kv_dtype != "bf16" or wl.d != 128 or wl.q_dtype != "bf16":
         return False
@@ -180,7 +180,7 @@ def split_schedule(wl, S, sms):
     pairs = wl.B * wl.Hk * n_qt // 2
     n_kt = -(-wl.capacity // 128)
     waves = -(-pairs // sms)
-    return pairs / (waves * sms) < 0.95 and pairs * n_kt >= 4 * sms and n_kt >= 4
+    return pairs / (waves * sms) < 0.75 and pairs * n_kt >= 4 * sms and n_kt >= 4
 
 
 # --------------------------------------------------------------------------- #

@@ -67,6 +67,18 @@ constexpr float kMaskBias = 1073741824.f;  // 2^30: a masked logit drops by this
 // softmax warpgroups rise to 208: 128 x 88 + 256 x 208 = 64512.
 constexpr int kLaunchRegs = 168, kCtrlRegs = 88, kSoftRegs = 208;
 static_assert(128 * kCtrlRegs + 256 * kSoftRegs == kThreads * kLaunchRegs, "register split");
+// Quantized caches: 512 threads, warps 12-15 join the loaders.  Launch allotment 128
+// registers (512 x 128 = 65536); the control and loader warpgroups drop to 64, the
+// softmax warpgroups rise to 192: 256 x 64 + 256 x 192 = 65536.
+constexpr int kThreadsQ = 512;
+constexpr int kLaunchRegsQ = 128, kCtrlRegsQ = 64, kSoftRegsQ = 192;
+static_assert(256 * kCtrlRegsQ + 256 * kSoftRegsQ == kThreadsQ * kLaunchRegsQ, "register split");
+template <int KV>
+__host__ __device__ constexpr int threads_of() { return KV == H2OKV_BF16 ? kThreads : kThreadsQ; }
+template <int KV>
+__host__ __device__ constexpr int launch_regs_of() {
+  return KV == H2OKV_BF16 ? kLaunchRegs : kLaunchRegsQ;
+}
 constexpr uint32_t kTileBytes = BM * D * 2;  // 32 KiB (two 64-column swizzled halves)
 constexpr uint32_t kHalfBytes = kTileBytes / 2;
 
@@ -295,7 +307,8 @@ __device__ __forceinline__ void store_p(uint32_t p_slot_row, int st, const uint3
 // u = c + 128 or c + 8 as an unsigned byte) minus 2^23 + 128 (or + 8); |c| <= 127
 // is exact in bf16.  Value tiles are multiplied by their slot's scale first (exact
 // in float32, one rounding to bf16).
-constexpr int kConvThreads = 96;
+constexpr int kLoaderWarps = 7;  // warps 0, 2, 3 and 12-15
+constexpr int kConvThreads = 32 * kLoaderWarps;
 constexpr uint32_t kStageOff = kHalfBytes;  // staged codes: upper half of the buffer
 template <int KV>
 struct QTile;
@@ -402,7 +415,7 @@ __device__ __forceinline__ float exp2i(int e) { return __int_as_float((127 + e) 
 // no other warp's rows are touched.  w3 is this warp's index among the loader warps;
 // sv[i] is the value scale of this lane's row in pass i (values only).  Rows at or
 // past nv (outside the cache) are written as zeros.
-constexpr int kI8Passes = 11;  // 32 groups of 4 rows over 3 warps
+constexpr int kI8Passes = (32 + kLoaderWarps - 1) / kLoaderWarps;  // 32 groups of 4 rows
 __device__ __forceinline__ void convert_i8(uint32_t buf, int nv, const float (&sv)[kI8Passes + 1],
                                            bool fold, int w3, int lane) {
   const int q = lane & 7;
@@ -414,7 +427,7 @@ __device__ __forceinline__ void convert_i8(uint32_t buf, int nv, const float (&s
     bool act[kU];
 #pragma unroll
     for (int u = 0; u < kU; ++u) {
-      const int g = w3 + 3 * (it + u);
+      const int g = w3 + kLoaderWarps * (it + u);
       act[u] = it + u < kI8Passes && g < 32;
       row[u] = 4 * g + (lane >> 3);
       w[u] = make_uint4(0u, 0u, 0u, 0u);
@@ -443,7 +456,7 @@ __device__ __forceinline__ void convert_i8(uint32_t buf, int nv, const float (&s
 // chunks (chunk ch = 32 codes of row ch / 4), the 96 threads meet at a named barrier,
 // then all write (keys to exact f16, values to bf16(code * scale)).  sv holds the
 // value scales of the chunks' rows (pairs).
-constexpr int kI4Per = 6;  // ceil(512 chunks / 96 threads)
+constexpr int kI4Per = (BN * 4 + kConvThreads - 1) / kConvThreads;  // 512 chunks
 constexpr int kConvBar = 3;  // named barrier of the loader threads (0: CTA, 1-2: softmax)
 __device__ __forceinline__ void convert_i4_read(uint32_t buf, int nv, int ct, uint4 (&w)[kI4Per]) {
 #pragma unroll
@@ -454,7 +467,7 @@ __device__ __forceinline__ void convert_i4_read(uint32_t buf, int nv, int ct, ui
   }
 }
 // (after every loader thread has read its chunks and met at the named barrier)
-__device__ __forceinline__ void convert_i4_write(uint32_t buf, const __half2 (&sv)[kI4Per / 2],
+__device__ __forceinline__ void convert_i4_write(uint32_t buf, const __half2 (&sv)[(kI4Per + 1) / 2],
                                                  bool fold, int ct, const uint4 (&w)[kI4Per]) {
 #pragma unroll
   for (int r = 0; r < kI4Per; ++r) {
@@ -532,7 +545,7 @@ __device__ __forceinline__ void scale_row(uint32_t (&x)[N], const float *ks) {
 }
 
 template <int KV>
-__global__ void __launch_bounds__(kThreads, 1)
+__global__ void __launch_bounds__(threads_of<KV>(), 1)
     attn_tc_kernel(const __grid_constant__ CUtensorMap q_map,
                    const __grid_constant__ CUtensorMap k_map,
                    const __grid_constant__ CUtensorMap v_map, const TcParams p) {
@@ -617,8 +630,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   // logits Q K^T: bf16 operands, or f16 for quantized caches (exact integer keys)
   constexpr uint32_t kIdescS = KV == H2OKV_BF16 ? IDESC_K_MAJOR : IDESC_K_MAJOR_F16;
 
-  if (warp < 4) {
-  reg_dealloc<kCtrlRegs>();
+  if (warp < 4 || warp >= 12) {
+  reg_dealloc<KV == H2OKV_BF16 ? kCtrlRegs : kCtrlRegsQ>();
   if (warp == 1) {
     // ------------------------------------------------------------------ MMA issuer
     if (lane == 0) {
@@ -810,7 +823,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
   } else {
     // --------------------------- loaders of quantized tiles (warps 0, 2, 3: 96 threads)
-    const int w3 = warp == 0 ? 0 : warp - 1;
+    const int w3 = warp == 0 ? 0 : (warp < 4 ? warp - 1 : warp - 9);  // 0 .. kLoaderWarps - 1
     const int ct = 32 * w3 + lane;
     if (warp == 0 && lane == 0) {
       mbar_expect_tx(&bar[B_Q], has_b ? 2 * kTileBytes : kTileBytes);
@@ -946,7 +959,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int i = 0; i < 2 * ((kI8Passes + 2) / 2); ++i) {
         int row = BN;
         if (KV == H2OKV_I8)
-          row = i < kI8Passes ? 4 * (w3 + 3 * i) + (lane >> 3) : BN;
+          row = i < kI8Passes ? 4 * (w3 + kLoaderWarps * i) + (lane >> 3) : BN;
         else
           row = i < kI4Per ? (ct + kConvThreads * i) >> 2 : BN;
         sh[i] = (x.kind == 2 && row < nv) ? vsg[slot0 + row] : __float2half(0.f);
@@ -1029,9 +1042,9 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
       for (int i = 0; i <= kI8Passes; ++i)
         sv8[i] = (i & 1) ? __high2float(cur.sv[i / 2]) : __low2float(cur.sv[i / 2]);
-      __half2 sv4[kI4Per / 2];
+      __half2 sv4[(kI4Per + 1) / 2];
 #pragma unroll
-      for (int r = 0; r < kI4Per / 2; ++r) sv4[r] = cur.sv[r];
+      for (int r = 0; r < (kI4Per + 1) / 2; ++r) sv4[r] = cur.sv[r];
       if (x.kind == 0) {
         float *rd = reinterpret_cast<float *>(smem + OFF_REL_A) + x.buf * BN;
         float *kd = reinterpret_cast<float *>(smem + OFF_KS_A) + x.buf * BN;
@@ -1076,7 +1089,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     __syncwarp();
   }
   } else {
-  reg_alloc<kSoftRegs>();
+  reg_alloc<KV == H2OKV_BF16 ? kSoftRegs : kSoftRegsQ>();
   if (warp < 8 || has_b) {
     // -------------------------------------------- softmax / sums, one warpgroup per query tile
     const int wg = (warp - 4) >> 2;  // 0: tile a, 1: tile b
@@ -1901,7 +1914,10 @@ bool tc_path_supported(const h2okv_cache_desc &d) {
 
 namespace {
 // Split scheduling pays when one CTA per pair of query tiles leaves many SMs idle in
-// the last wave; it needs two query tiles in every pair and a few tiles per CTA.
+// the last wave (measured: a wave 86 % full runs as fast fused as split, since the
+// split kernels cost ~10 % more per unit); it needs two query tiles in every pair and
+// a few tiles per CTA.
+constexpr double kSplitFill = 0.75;
 struct SplitShape {
   bool use;
   long long U;
@@ -1918,7 +1934,7 @@ SplitShape split_shape(const h2okv_cache_desc &d, int S, int G) {
   r.U = pairs * n_kt;
   const long long waves = (pairs + G - 1) / G;
   const double fill = (double)pairs / (double)(waves * G);
-  if (fill >= 0.95 || r.U < 4LL * G || n_kt < 4) return r;
+  if (fill >= kSplitFill || r.U < 4LL * G || n_kt < 4) return r;
   const long long per = (r.U + G - 1) / G;  // units of one CTA at most
   r.max_seg = (int)((per + n_kt - 1) / n_kt) + 1;
   r.use = true;
@@ -1963,10 +1979,10 @@ int prepare_kernel() {
     return set_error(H2OKV_ERR_CUDA, "cudaFuncGetAttributes(attn_tc_kernel): %s",
                      cudaGetErrorString(e));
   // the in-kernel register split assumes exactly this launch allotment
-  if (fa.numRegs != kLaunchRegs)
+  if (fa.numRegs != launch_regs_of<KV>())
     return set_error(H2OKV_ERR_UNSUPPORTED,
                      "attn_tc_kernel built with %d registers per thread, expected %d", fa.numRegs,
-                     kLaunchRegs);
+                     launch_regs_of<KV>());
   ready_dev = dev;
   return H2OKV_OK;
 }
@@ -1997,7 +2013,7 @@ int launch_kernel(int grid, const CUtensorMap &qmap, const CUtensorMap &kmap,
                   const CUtensorMap &vmap, const TcParams &prm, cudaStream_t st) {
   int rc = prepare_kernel<KV>();
   if (rc) return rc;
-  attn_tc_kernel<KV><<<grid, kThreads, kSmemBytes, st>>>(qmap, kmap, vmap, prm);
+  attn_tc_kernel<KV><<<grid, threads_of<KV>(), kSmemBytes, st>>>(qmap, kmap, vmap, prm);
   return check_launch("attn_tc_kernel");
 }
 

@@ -135,12 +135,12 @@ struct RowSet {
 // kCopyUnroll pieces before it stores any, so a launch waits on memory a few times in all
 // rather than once per row.  With delta outputs the same thread first reads the piece it
 // overwrites.
-template <typename SlotOf>
+template <bool FULL, typename SlotOf>
 __device__ __forceinline__ void copy_rows_cta(const EvictArgs &a, RowSet rs, int rank, int CL,
                                               int n_rows, SlotOf slot_of) {
   const int C = (int)(a.row_bytes / 16);  // 16-byte pieces per row (row_bytes % 16 == 0)
   const int total = n_rows * 2 * C;
-  const bool dl = a.dk != nullptr;
+  const bool dl = FULL && a.dk != nullptr;
   for (int base = threadIdx.x; base < total; base += kEvThreads * kCopyUnroll) {
     uint4 r[kCopyUnroll], old[kCopyUnroll];
     uint4 *dst[kCopyUnroll];
@@ -180,7 +180,7 @@ __device__ __forceinline__ void copy_rows_cta(const EvictArgs &a, RowSet rs, int
 // arithmetic as the per-row quantizer: absmax, IEEE division by qmax, clamp to the fp16
 // range, round to fp16, then rint(x / scale) clamped to [-qmax, qmax].  With delta
 // outputs each lane first copies the codes (and lane 0 the scale) it overwrites.
-template <int KV, typename SlotOf>
+template <int KV, bool FULL, typename SlotOf>
 __device__ __forceinline__ void quantize_rows_cta(const EvictArgs &a, RowSet rs, int rank, int CL,
                                                   int n_rows, SlotOf slot_of) {
   constexpr int qmax = KV == H2OKV_I8 ? 127 : 7;
@@ -190,7 +190,7 @@ __device__ __forceinline__ void quantize_rows_cta(const EvictArgs &a, RowSet rs,
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const int seg = lane / L, li = lane % L, segs = 32 / L;
   const int items = n_rows * 2;  // (m, t): t = 0 key row, 1 value row
-  const bool dl = a.dk != nullptr;
+  const bool dl = FULL && a.dk != nullptr;
   for (int p0 = 0; (p0 * kEvWarps + warp) * segs < items; p0 += kQuantUnroll) {
     uint4 x[kQuantUnroll];
     bool ok[kQuantUnroll];
@@ -265,14 +265,14 @@ __device__ __forceinline__ void quantize_rows_cta(const EvictArgs &a, RowSet rs,
   }
 }
 
-template <int KV, typename SlotOf>
+template <int KV, bool FULL, typename SlotOf>
 __device__ __forceinline__ void insert_rows_cta(const EvictArgs &a, RowSet rs, int rank, int CL,
                                                 SlotOf slot_of) {
   const int n_rows = rank < a.S ? (a.S - rank + CL - 1) / CL : 0;
   if constexpr (KV == H2OKV_I8 || KV == H2OKV_I4)
-    quantize_rows_cta<KV>(a, rs, rank, CL, n_rows, slot_of);
+    quantize_rows_cta<KV, FULL>(a, rs, rank, CL, n_rows, slot_of);
   else
-    copy_rows_cta(a, rs, rank, CL, n_rows, slot_of);
+    copy_rows_cta<FULL>(a, rs, rank, CL, n_rows, slot_of);
 }
 
 template <int IPT>
@@ -296,10 +296,11 @@ __device__ __forceinline__ void store_slice(float *dst, const float (&v)[IPT],
 // Slot j of a chunk row set receives chunk row k: bookkeeping of the slot (old token
 // position to the delta output, new token position, score 0 unless the caller stores
 // the slice's scores afterwards, slot list).
+template <bool FULL>
 __device__ __forceinline__ void claim_slot(const EvictArgs &a, RowSet rs, int j, int k,
                                            bool zero_score = true) {
   const size_t gs = rs.gbase + (size_t)j, rk = rs.rbase + (size_t)k;
-  if (a.dpos) a.dpos[rk] = a.token_pos[gs];
+  if (FULL && a.dpos) a.dpos[rk] = a.token_pos[gs];
   a.token_pos[gs] = a.P + k;
   if (zero_score) a.scores[gs] = 0.f;
   if (a.slots_out) a.slots_out[rk] = j;
@@ -309,7 +310,9 @@ __device__ __forceinline__ void claim_slot(const EvictArgs &a, RowSet rs, int j,
 // touched); 2: generic choice (empty slots first, then lowest selection keys);
 // 3: replay (write the given slots).  One cluster per (batch row, KV head), or per KV
 // head for all batch rows together (score variant h2o_orig: nbat > 1).
-template <int KV, int IPT>
+// FULL: the general kernel (h2o_orig over several batch rows, replay, delta outputs); the
+// other instance is the plain per-(b, h_k) choice, built without those paths.
+template <int KV, int IPT, bool FULL>
 __global__ void __launch_bounds__(kEvThreads) evict_kernel(const EvictArgs a) {
   namespace cg = cooperative_groups;
   cg::cluster_group cluster = cg::this_cluster();
@@ -317,7 +320,7 @@ __global__ void __launch_bounds__(kEvThreads) evict_kernel(const EvictArgs a) {
   const int rank = (int)cluster.block_rank();
   const int gi = blockIdx.x / CL;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  const int nb = a.nbat;
+  const int nb = FULL ? a.nbat : 1;
   const int b_first = nb > 1 ? 0 : gi / a.Hk, h = nb > 1 ? gi : gi % a.Hk;
   auto rows_of = [&](int bb) {
     const size_t bh = (size_t)(b_first + bb) * a.Hk + h;
@@ -403,14 +406,14 @@ __global__ void __launch_bounds__(kEvThreads) evict_kernel(const EvictArgs a) {
     for (int i = 0; i < IPT; ++i) {
       const int k = j0 + i - a.n_filled;
       if (valid[i] && k >= 0 && k < a.S)
-        for (int bb = 0; bb < nb; ++bb) claim_slot(a, rows_of(bb), j0 + i, k);
+        for (int bb = 0; bb < nb; ++bb) claim_slot<FULL>(a, rows_of(bb), j0 + i, k);
     }
     const int first = a.n_filled + rank;
     for (int bb = 0; bb < nb; ++bb)
-      insert_rows_cta<KV>(a, rows_of(bb), rank, CL, [&](int m) { return first + CL * m; });
+      insert_rows_cta<KV, FULL>(a, rows_of(bb), rank, CL, [&](int m) { return first + CL * m; });
     return;
   }
-  if (a.mode == 3) {
+  if (FULL && a.mode == 3) {
     // replay: every fold store of the cluster lands before a replayed slot is reset
     cluster.sync();
     for (int bb = 0; bb < nb; ++bb) {
@@ -424,9 +427,9 @@ __global__ void __launch_bounds__(kEvThreads) evict_kernel(const EvictArgs a) {
         if (j < 0)
           atomicExch(a.status, H2OKV_ERR_INVALID_ARG);
         else
-          claim_slot(a, rs, j, rank + CL * m);
+          claim_slot<FULL>(a, rs, j, rank + CL * m);
       }
-      insert_rows_cta<KV>(a, rs, rank, CL, slot_of);
+      insert_rows_cta<KV, FULL>(a, rs, rank, CL, slot_of);
     }
     return;
   }
@@ -533,7 +536,7 @@ __global__ void __launch_bounds__(kEvThreads) evict_kernel(const EvictArgs a) {
     }
     if (take) {
       if (defer_store) sc[i] = 0.f;
-      for (int bb = 0; bb < nb; ++bb) claim_slot(a, rows_of(bb), j, (int)pos, !defer_store);
+      for (int bb = 0; bb < nb; ++bb) claim_slot<FULL>(a, rows_of(bb), j, (int)pos, !defer_store);
       int32_t *dst = cluster.map_shared_rank(rowslot, (int)(pos % (uint32_t)CL));
       dst[pos / (uint32_t)CL] = j;
     }
@@ -543,7 +546,7 @@ __global__ void __launch_bounds__(kEvThreads) evict_kernel(const EvictArgs a) {
 
   // ---- insert the chunk's rows k = rank, rank + CL, ... -----------------------------
   for (int bb = 0; bb < nb; ++bb)
-    insert_rows_cta<KV>(a, rows_of(bb), rank, CL, [&](int m) { return rowslot[m]; });
+    insert_rows_cta<KV, FULL>(a, rows_of(bb), rank, CL, [&](int m) { return rowslot[m]; });
 }
 
 template <int KV>
@@ -608,7 +611,7 @@ int launch_init_cache(h2okv_cache *c, cudaStream_t st) {
   return check_launch("init_kernel");
 }
 
-template <int KV, int IPT>
+template <int KV, int IPT, bool FULL>
 static int launch_evict_t(const EvictArgs &a, int n_groups, int CL, cudaStream_t st) {
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3((unsigned)(n_groups * CL));
@@ -623,28 +626,28 @@ static int launch_evict_t(const EvictArgs &a, int n_groups, int CL, cudaStream_t
   cfg.attrs = attr;
   cfg.numAttrs = 1;
   if (cfg.dynamicSmemBytes > 48 * 1024) {
-    cudaError_t e = cudaFuncSetAttribute(evict_kernel<KV, IPT>,
+    cudaError_t e = cudaFuncSetAttribute(evict_kernel<KV, IPT, FULL>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          (int)cfg.dynamicSmemBytes);
     if (e != cudaSuccess)
       return set_error(H2OKV_ERR_CUDA, "cudaFuncSetAttribute(evict_kernel): %s",
                        cudaGetErrorString(e));
   }
-  cudaError_t e = cudaLaunchKernelEx(&cfg, evict_kernel<KV, IPT>, a);
+  cudaError_t e = cudaLaunchKernelEx(&cfg, evict_kernel<KV, IPT, FULL>, a);
   if (e != cudaSuccess)
     return set_error(H2OKV_ERR_CUDA, "evict_kernel launch: %s", cudaGetErrorString(e));
   return check_launch("evict_kernel");
 }
 
-template <int KV>
+template <int KV, bool FULL>
 static int launch_evict_kv(const EvictArgs &a, int n_groups, int CL, int ipt, cudaStream_t st) {
   switch (ipt) {
-    case 1: return launch_evict_t<KV, 1>(a, n_groups, CL, st);
-    case 2: return launch_evict_t<KV, 2>(a, n_groups, CL, st);
-    case 4: return launch_evict_t<KV, 4>(a, n_groups, CL, st);
-    case 8: return launch_evict_t<KV, 8>(a, n_groups, CL, st);
-    case 16: return launch_evict_t<KV, 16>(a, n_groups, CL, st);
-    case 32: return launch_evict_t<KV, 32>(a, n_groups, CL, st);
+    case 1: return launch_evict_t<KV, 1, FULL>(a, n_groups, CL, st);
+    case 2: return launch_evict_t<KV, 2, FULL>(a, n_groups, CL, st);
+    case 4: return launch_evict_t<KV, 4, FULL>(a, n_groups, CL, st);
+    case 8: return launch_evict_t<KV, 8, FULL>(a, n_groups, CL, st);
+    case 16: return launch_evict_t<KV, 16, FULL>(a, n_groups, CL, st);
+    case 32: return launch_evict_t<KV, 32, FULL>(a, n_groups, CL, st);
   }
   return set_error(H2OKV_ERR_UNSUPPORTED, "capacity too large for the eviction kernel");
 }
@@ -690,11 +693,20 @@ int launch_evict_insert(h2okv_cache *c, const float *w_prev, const void *k_new, 
   while ((int64_t)CL * kEvThreads * ipt < d.capacity) ipt *= 2;
   a.slice = kEvThreads * ipt;
   const int n_groups = orig ? d.n_kv_heads : d.batch * d.n_kv_heads;
+  const bool full = orig || delta != nullptr || a.mode == 3;
   switch (d.kv_dtype) {
-    case H2OKV_F32: return launch_evict_kv<H2OKV_F32>(a, n_groups, CL, ipt, st);
-    case H2OKV_BF16: return launch_evict_kv<H2OKV_BF16>(a, n_groups, CL, ipt, st);
-    case H2OKV_I8: return launch_evict_kv<H2OKV_I8>(a, n_groups, CL, ipt, st);
-    case H2OKV_I4: return launch_evict_kv<H2OKV_I4>(a, n_groups, CL, ipt, st);
+    case H2OKV_F32:
+      return full ? launch_evict_kv<H2OKV_F32, true>(a, n_groups, CL, ipt, st)
+                  : launch_evict_kv<H2OKV_F32, false>(a, n_groups, CL, ipt, st);
+    case H2OKV_BF16:
+      return full ? launch_evict_kv<H2OKV_BF16, true>(a, n_groups, CL, ipt, st)
+                  : launch_evict_kv<H2OKV_BF16, false>(a, n_groups, CL, ipt, st);
+    case H2OKV_I8:
+      return full ? launch_evict_kv<H2OKV_I8, true>(a, n_groups, CL, ipt, st)
+                  : launch_evict_kv<H2OKV_I8, false>(a, n_groups, CL, ipt, st);
+    case H2OKV_I4:
+      return full ? launch_evict_kv<H2OKV_I4, true>(a, n_groups, CL, ipt, st)
+                  : launch_evict_kv<H2OKV_I4, false>(a, n_groups, CL, ipt, st);
   }
   return set_error(H2OKV_ERR_UNSUPPORTED, "kv dtype");
 }
