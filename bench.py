@@ -299,31 +299,62 @@ def run_ours(args, wl, ws, rank, local):
                launches=launches_per_step * args.steps)
 
     # ---- end to end through the public API, host buffers ----------------------
+    # Pinned host inputs in, y and w out, every chunk.  A copy stream moves chunk c + 1's
+    # inputs in and chunk c - 1's outputs out while chunk c computes (two device buffer
+    # sets; events order every reuse).  The timed region ends when the last output copy
+    # has landed.
     host = [(q.cpu().pin_memory(), k.cpu().pin_memory(), v.cpu().pin_memory()) for (q, k, v) in chunks]
     del chunks
-    q_d = torch.empty_like(host[0][0], device=dev)
-    k_d = torch.empty_like(host[0][1], device=dev)
-    v_d = torch.empty_like(host[0][2], device=dev)
-    y_h = torch.empty(host[0][0].shape, dtype=host[0][0].dtype).pin_memory()
-    w_h = torch.empty((wl.B, wl.Hk, wl.capacity), dtype=torch.float32).pin_memory()
+    qdb = [torch.empty_like(host[0][0], device=dev) for _ in range(2)]
+    kdb = [torch.empty_like(host[0][1], device=dev) for _ in range(2)]
+    vdb = [torch.empty_like(host[0][2], device=dev) for _ in range(2)]
+    ydb = [torch.empty_like(host[0][0], device=dev) for _ in range(2)]
+    y_h = [torch.empty(host[0][0].shape, dtype=host[0][0].dtype).pin_memory() for _ in range(2)]
+    w_h = [torch.empty((wl.B, wl.Hk, wl.capacity), dtype=torch.float32).pin_memory() for _ in range(2)]
     h2d = sum(t.numel() * t.element_size() for ch in host for t in ch)
-    d2h = wl.n_chunks * (y_h.numel() * y_h.element_size() + w_h.numel() * w_h.element_size())
+    d2h = sum(t.numel() * t.element_size() for (t, _, _) in host) + \
+        wl.n_chunks * (w_h[0].numel() * w_h[0].element_size())
+    cs = torch.cuda.Stream(dev)
+    ready = [torch.cuda.Event() for _ in range(2)]
+    consumed = [torch.cuda.Event() for _ in range(2)]
+    out_done = [torch.cuda.Event() for _ in range(2)]
 
     def e2e_step():
         runner.reset()
+        cs.wait_stream(stream)  # the previous step is done with both buffer sets
+        last = None
         for c, (qh, kh, vh) in enumerate(host):
             S = qh.shape[2]
-            qd, kd, vd = (q_d, k_d, v_d) if S == wl.chunk else (torch.empty_like(qh, device=dev),
-                                                               torch.empty_like(kh, device=dev),
-                                                               torch.empty_like(vh, device=dev))
-            qd.copy_(qh, non_blocking=True)
-            kd.copy_(kh, non_blocking=True)
-            vd.copy_(vh, non_blocking=True)
-            y, _, w, _, _ = runner.step(qd, kd, vd)
-            if S == wl.chunk:
-                y_h.copy_(y, non_blocking=True)
-            w_h.copy_(w, non_blocking=True)
+            b = c % 2
+            same = S == wl.chunk
+            qd, kd, vd, yd = (qdb[b], kdb[b], vdb[b], ydb[b]) if same else tuple(
+                torch.empty_like(t, device=dev) for t in (qh, kh, vh, qh))
+            with torch.cuda.stream(cs):
+                if c >= 2:
+                    cs.wait_event(consumed[b])  # chunk c - 2 no longer reads this input set
+                qd.copy_(qh, non_blocking=True)
+                kd.copy_(kh, non_blocking=True)
+                vd.copy_(vh, non_blocking=True)
+                ready[b].record(cs)
+            stream.wait_event(ready[b])
+            if c >= 2:
+                stream.wait_event(out_done[b])  # chunk c - 2's y and w have been copied out
+            runner.cache.evict_insert(runner.w_prev(), kd, vd, S, runner.P, None)
+            w = runner.w_cur()
+            runner.cache.attend(qd, S, runner.P, yd, None, w, None)
+            consumed[b].record(stream)
+            with torch.cuda.stream(cs):
+                cs.wait_event(consumed[b])
+                (y_h[b] if same else torch.empty(qh.shape, dtype=qh.dtype).pin_memory()).copy_(
+                    yd, non_blocking=True)
+                w_h[b].copy_(w, non_blocking=True)
+                out_done[b].record(cs)
+            last = out_done[b]
+            runner.chunk_index += 1
+            runner.P += S
         runner.finish()
+        if last is not None:
+            stream.wait_event(last)
 
     e2e_step()
     torch.cuda.synchronize()
