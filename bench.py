@@ -299,10 +299,10 @@ def run_ours(args, wl, ws, rank, local):
                launches=launches_per_step * args.steps)
 
     # ---- end to end through the public API, host buffers ----------------------
-    # Pinned host inputs in, y and w out, every chunk.  A copy stream moves chunk c + 1's
-    # inputs in and chunk c - 1's outputs out while chunk c computes (two device buffer
-    # sets; events order every reuse).  The timed region ends when the last output copy
-    # has landed.
+    # Pinned host inputs in, y and w out, every chunk.  One copy stream moves chunk c + 1's
+    # inputs in and another chunk c - 1's outputs out while chunk c computes (two device
+    # buffer sets; events order every reuse).  The timed region ends when the last output
+    # copy has landed.
     host = [(q.cpu().pin_memory(), k.cpu().pin_memory(), v.cpu().pin_memory()) for (q, k, v) in chunks]
     del chunks
     qdb = [torch.empty_like(host[0][0], device=dev) for _ in range(2)]
@@ -314,14 +314,15 @@ def run_ours(args, wl, ws, rank, local):
     h2d = sum(t.numel() * t.element_size() for ch in host for t in ch)
     d2h = sum(t.numel() * t.element_size() for (t, _, _) in host) + \
         wl.n_chunks * (w_h[0].numel() * w_h[0].element_size())
-    cs = torch.cuda.Stream(dev)
+    cs_in, cs_out = torch.cuda.Stream(dev), torch.cuda.Stream(dev)
     ready = [torch.cuda.Event() for _ in range(2)]
     consumed = [torch.cuda.Event() for _ in range(2)]
     out_done = [torch.cuda.Event() for _ in range(2)]
 
     def e2e_step():
         runner.reset()
-        cs.wait_stream(stream)  # the previous step is done with both buffer sets
+        stream.wait_stream(cs_out)  # the previous step's outputs have been copied out
+        cs_in.wait_stream(stream)  # the previous step is done with both input sets
         last = None
         for c, (qh, kh, vh) in enumerate(host):
             S = qh.shape[2]
@@ -329,13 +330,13 @@ def run_ours(args, wl, ws, rank, local):
             same = S == wl.chunk
             qd, kd, vd, yd = (qdb[b], kdb[b], vdb[b], ydb[b]) if same else tuple(
                 torch.empty_like(t, device=dev) for t in (qh, kh, vh, qh))
-            with torch.cuda.stream(cs):
+            with torch.cuda.stream(cs_in):
                 if c >= 2:
-                    cs.wait_event(consumed[b])  # chunk c - 2 no longer reads this input set
+                    cs_in.wait_event(consumed[b])  # chunk c - 2 no longer reads this input set
                 qd.copy_(qh, non_blocking=True)
                 kd.copy_(kh, non_blocking=True)
                 vd.copy_(vh, non_blocking=True)
-                ready[b].record(cs)
+                ready[b].record(cs_in)
             stream.wait_event(ready[b])
             if c >= 2:
                 stream.wait_event(out_done[b])  # chunk c - 2's y and w have been copied out
@@ -343,12 +344,12 @@ def run_ours(args, wl, ws, rank, local):
             w = runner.w_cur()
             runner.cache.attend(qd, S, runner.P, yd, None, w, None)
             consumed[b].record(stream)
-            with torch.cuda.stream(cs):
-                cs.wait_event(consumed[b])
+            with torch.cuda.stream(cs_out):
+                cs_out.wait_event(consumed[b])
                 (y_h[b] if same else torch.empty(qh.shape, dtype=qh.dtype).pin_memory()).copy_(
                     yd, non_blocking=True)
                 w_h[b].copy_(w, non_blocking=True)
-                out_done[b].record(cs)
+                out_done[b].record(cs_out)
             last = out_done[b]
             runner.chunk_index += 1
             runner.P += S
