@@ -19,6 +19,7 @@ from .h2o_oracle import (  # noqa: F401
     SCORE_MODES,
     OracleCache,
     attend_head,
+    attend_head_backward,
     dequantize_rows,
     pack_int4,
     quantize_rows,

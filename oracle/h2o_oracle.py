@@ -214,6 +214,30 @@ def attend_head(q: np.ndarray, keys: np.ndarray, values: np.ndarray,
     return y, lse, m
 
 
+def attend_head_backward(q: np.ndarray, keys: np.ndarray, values: np.ndarray,
+                         token_pos: np.ndarray, P: int, dy: np.ndarray):
+    """Gradients of one head's SDPA over the cache (§A.5: autograd through the
+    attention of each chunk; the cache policy itself is not differentiated).
+
+    For L = sum(dy * y) with y = m V, m = softmax_j(a), a_ij = q_i . k_j / sqrt(d)
+    (masked entries fixed at -inf): dV = m^T dy; dm = dy V^T;
+    da = m * (dm - rowsum(m * dm)); dq = da K / sqrt(d); dK = da^T q / sqrt(d).
+    Returns (dq [S, d], dk [N_C, d], dv [N_C, d]) in float64.
+    """
+    q = np.asarray(q, dtype=np.float64)
+    k = np.asarray(keys, dtype=np.float64)
+    v = np.asarray(values, dtype=np.float64)
+    dy = np.asarray(dy, dtype=np.float64)
+    d = q.shape[1]
+    _, _, m = attend_head(q, k, v, token_pos, P)
+    dv = m.T @ dy
+    dm = dy @ v.T
+    da = m * (dm - np.sum(m * dm, axis=1, keepdims=True))
+    dq = (da @ k) / math.sqrt(d)
+    dk = (da.T @ q) / math.sqrt(d)
+    return dq, dk, dv
+
+
 # --------------------------------------------------------------------------- #
 # One attention layer's cache, processed chunk by chunk (§3.1, §A.1, §A.5.3).
 # --------------------------------------------------------------------------- #
@@ -367,6 +391,26 @@ class OracleCache:
                     wq[b, h] = m.sum(axis=0)
                     w[b, g] += wq[b, h]
         return y, lse, w, wq
+
+    # -- gradients of the chunk's SDPA over the cache -------------------------
+    def attend_backward(self, q, dy, S, P):
+        """q, dy: [B, H_q, S, d].  Returns dq [B, H_q, S, d] and dk, dv
+        [B, H_k, N_C, d] (summed over the group's query heads), float64, with
+        respect to the stored (dequantized) keys and values."""
+        B, Hq, Hk, d, N_C = self.B, self.Hq, self.Hk, self.d, self.N_C
+        dq = np.zeros((B, Hq, S, d))
+        dk = np.zeros((B, Hk, N_C, d))
+        dv = np.zeros((B, Hk, N_C, d))
+        for b in range(B):
+            for g in range(Hk):
+                K, V = self.keys(b, g), self.values(b, g)
+                for r in range(self.q_g):
+                    h = g * self.q_g + r
+                    a, bk, bv = attend_head_backward(q[b, h], K, V, self.token_pos[b, g], P, dy[b, h])
+                    dq[b, h] = a
+                    dk[b, g] += bk
+                    dv[b, g] += bv
+        return dq, dk, dv
 
     # -- state transfer (re-seeding from another implementation) -------------
     def load_state(self, *, token_pos, scores, n_filled, keys=None, values=None,

@@ -27,7 +27,8 @@ import pytest
 from scipy.special import logsumexp, softmax
 
 import oracle
-from oracle import EMPTY_POS, OracleCache, attend_head, quantize_rows, select_slots, selection_keys
+from oracle import (EMPTY_POS, OracleCache, attend_head, attend_head_backward, quantize_rows,
+                    select_slots, selection_keys)
 from oracle import h2o_oracle as ho
 
 GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
@@ -551,3 +552,80 @@ def test_t7_planted_age_off_by_one_is_caught(monkeypatch):
     monkeypatch.setattr(ho, "selection_keys", age_plus_one)
     with pytest.raises(AssertionError):
         test_t7_score_variants_hand_derived()
+
+
+# --------------------------------------------------------------------------- #
+# Gradients of the chunk's SDPA over the cache (§A.5 autograd per chunk).
+# --------------------------------------------------------------------------- #
+def _loss(q, k, v, tp, P, dy):
+    y, _, _ = attend_head(q, k, v, tp, P)
+    return float(np.sum(y * dy))
+
+
+def test_t10_backward_matches_finite_differences():
+    """Central differences of L = sum(dy * y) along random directions: pins every
+    term of the analytic gradient without restating its formula."""
+    rng = np.random.default_rng(41)
+    for P, n_c, S, d in ((0, 9, 6, 5), (7, 12, 4, 8)):
+        q = rng.standard_normal((S, d))
+        k = rng.standard_normal((n_c, d))
+        v = rng.standard_normal((n_c, d))
+        tp = rng.integers(0, P + S, n_c).astype(np.int64)
+        tp[0] = 0  # every row sees at least one slot
+        tp[rng.random(n_c) < 0.2] = EMPTY_POS
+        tp[0] = 0
+        dy = rng.standard_normal((S, d))
+        dq, dk, dv = attend_head_backward(q, k, v, tp, P, dy)
+        h = 1e-6
+        for grad, which in ((dq, 0), (dk, 1), (dv, 2)):
+            for _ in range(3):
+                dirn = rng.standard_normal(grad.shape)
+                args = [q, k, v]
+                plus = [a.copy() for a in args]
+                minus = [a.copy() for a in args]
+                plus[which] = plus[which] + h * dirn
+                minus[which] = minus[which] - h * dirn
+                fd = (_loss(*plus, tp, P, dy) - _loss(*minus, tp, P, dy)) / (2 * h)
+                assert abs(fd - float(np.sum(grad * dirn))) <= 1e-6 * max(1.0, abs(fd))
+
+
+def test_t10_backward_closed_forms():
+    rng = np.random.default_rng(43)
+    d = 6
+    # one visible slot: y = v_0, so dv_0 = sum of dy, dq = 0, dk = 0
+    q = rng.standard_normal((3, d))
+    k = rng.standard_normal((4, d))
+    v = rng.standard_normal((4, d))
+    tp = np.array([0, EMPTY_POS, EMPTY_POS, EMPTY_POS])
+    dy = rng.standard_normal((3, d))
+    dq, dk, dv = attend_head_backward(q, k, v, tp, 5, dy)
+    assert np.allclose(dv[0], dy.sum(axis=0)) and np.allclose(dv[1:], 0)
+    assert np.allclose(dq, 0) and np.allclose(dk, 0)
+    # q = 0 (uniform weights over the visible slots): dk = 0, dv_j = sum_i dy_i / n_i
+    tp = np.array([0, 1, 2, 3])
+    q0 = np.zeros((4, d))
+    dq, dk, dv = attend_head_backward(q0, k, v, tp, 0, dy := rng.standard_normal((4, d)))
+    assert np.allclose(dk, 0)
+    want = np.zeros((4, d))
+    for i in range(4):
+        for j in range(i + 1):
+            want[j] += dy[i] / (i + 1)
+    assert np.allclose(dv, want)
+    # identical keys: every row's weights are uniform whatever q is, so dq = 0
+    kk = np.tile(rng.standard_normal((1, d)), (4, 1))
+    dq, _, _ = attend_head_backward(rng.standard_normal((4, d)), kk, v, tp, 0, dy)
+    assert np.allclose(dq, 0)
+
+
+def test_t10_cache_backward_sums_group_heads():
+    rng = np.random.default_rng(47)
+    c = OracleCache(1, 2, 1, 4, 6, "f32")
+    c.evict_insert(None, _rand(rng, (1, 1, 6, 4)), _rand(rng, (1, 1, 6, 4)), 6, 0)
+    q = _rand(rng, (1, 1, 6, 4))
+    dy = _rand(rng, (1, 1, 6, 4))
+    q2 = np.concatenate([q, q], axis=1)
+    dy2 = np.concatenate([dy, dy], axis=1)
+    dq, dk, dv = c.attend_backward(q2, dy2, 6, 0)
+    a, bk, bv = attend_head_backward(q[0, 0], c.keys(0, 0), c.values(0, 0), c.token_pos[0, 0], 0, dy[0, 0])
+    assert np.allclose(dk[0, 0], 2 * bk) and np.allclose(dv[0, 0], 2 * bv)
+    assert np.allclose(dq[0, 0], a) and np.allclose(dq[0, 1], a)
