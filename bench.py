@@ -298,6 +298,32 @@ def run_ours(args, wl, ws, rank, local):
     res = dict(value=value, ms_step=ms_step, roof=roof, extra=extra, clocks=clocks,
                launches=launches_per_step * args.steps)
 
+    # ---- gradients of the last chunk's SDPA (CUDA-core kernels), outside the step ----
+    # Algorithmic FLOPs: QK^T, dy V^T, dS K, dS^T Q, P^T dy = 10 * B * H_q * S * n_valid * d.
+    q_l = chunks[-1][0]
+    S_l = q_l.shape[2]
+    lse_l = torch.empty(q_l.shape[:3], dtype=torch.float32, device=dev)
+    y_l = torch.empty_like(q_l)
+    runner.cache.attend(q_l, S_l, runner.P - S_l, y_l, lse_l, runner.w[0], None)
+    g = torch.Generator(device=dev)
+    g.manual_seed(7)
+    dy_l = torch.randn(q_l.shape, generator=g, device=dev).to(q_l.dtype)
+    dq_l = torch.empty(q_l.shape, dtype=torch.float32, device=dev)
+    dk_l = torch.empty((wl.B, wl.Hk, wl.capacity, wl.d), dtype=torch.float32, device=dev)
+    dv_l = torch.empty_like(dk_l)
+    bwd_ms = []
+    for it in range(3):
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        runner.cache.attend_backward(q_l, dy_l, lse_l, S_l, runner.P - S_l, dq_l, dk_l, dv_l)
+        e1.record(stream)
+        torch.cuda.synchronize()
+        if it:
+            bwd_ms.append(e0.elapsed_time(e1))
+    bwd = statistics.median(bwd_ms)
+    res["extra"]["bwd_ms_per_chunk"] = round(bwd, 3)
+    res["extra"]["bwd_tflops_alg"] = round(10.0 * wl.B * wl.Hq * S_l * n_valid[-1] * wl.d / (bwd * 1e-3) / 1e12, 2)
+
     # ---- end to end through the public API, host buffers ----------------------
     # Pinned host inputs in, y and w out, every chunk.  One copy stream moves chunk c + 1's
     # inputs in and another chunk c - 1's outputs out while chunk c computes (two device

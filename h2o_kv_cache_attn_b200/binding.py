@@ -27,7 +27,7 @@ EXPORTED = ("kv_cache_query_sizes", "kv_cache_create", "kv_cache_reset", "kv_cac
             "attn_chunk_with_scoresum", "kv_cache_device_status", "kv_cache_set_wait_timeout",
             "attn_chunk_with_scoresum_noalloc", "h2okv_last_error", "h2okv_abi_version",
             "kv_cache_set_score_mode", "h2o_evict_insert_delta", "h2o_insert_at",
-            "kv_cache_restore")
+            "kv_cache_restore", "attn_chunk_backward")
 SCORE_MODE = {"h2o": 0, "h2o_norm": 1, "h2o_orig": 2}
 
 
@@ -94,6 +94,7 @@ def load() -> ctypes.CDLL:
                                                   ctypes.POINTER(Delta), vp]),
         "h2o_insert_at": (ctypes.c_int, [vp, vp, vp, vp, i32, i64, vp, ctypes.POINTER(Delta), vp]),
         "kv_cache_restore": (ctypes.c_int, [vp, vp, i32, ctypes.POINTER(Delta), vp]),
+        "attn_chunk_backward": (ctypes.c_int, [vp, vp, vp, vp, i32, i64, vp, vp, vp, vp]),
         "h2okv_last_error": (ctypes.c_char_p, []),
         "h2okv_abi_version": (i32, []),
     }
@@ -196,6 +197,11 @@ def h2o_insert_at(handle, w_prev, k_new, v_new, S: int, P: int, slots_in, delta=
 
 def kv_cache_restore(handle, slots, S: int, delta, stream=None):
     _check(load().kv_cache_restore(handle, _ptr(slots), int(S), _delta(delta), _stream(stream)))
+
+
+def attn_chunk_backward(handle, q, dy, lse, S: int, P: int, dq_out, dk_out, dv_out, stream=None):
+    _check(load().attn_chunk_backward(handle, _ptr(q), _ptr(dy), _ptr(lse), int(S), int(P),
+                                      _ptr(dq_out), _ptr(dk_out), _ptr(dv_out), _stream(stream)))
 
 
 def attn_chunk_with_scoresum(handle, q, S: int, P: int, y_out, lse_out, w_out, wq_out=None,
@@ -318,6 +324,16 @@ class KVCache:
                     raise ValueError(f"k_new/v_new must be {want} {self.shape.q_dtype} on {self.device}")
         self._check_w(w_prev, allow_none=True)
         h2o_evict_insert(self.handle, w_prev, k_new, v_new, S, P, slots_out, stream)
+
+    def attend_backward(self, q, dy, lse, S, P, dq_out, dk_out, dv_out, stream=None):
+        """Gradients of the chunk's SDPA (dq [B,H_q,S,d], dk/dv [B,H_k,N_C,d] float32)."""
+        s = self.shape
+        if tuple(dk_out.shape) != (s.batch, s.n_kv_heads, s.capacity, s.head_dim) or \
+                dk_out.dtype != torch.float32 or dv_out.shape != dk_out.shape or dv_out.dtype != torch.float32:
+            raise ValueError("dk_out/dv_out must be [B, H_k, N_C, d] float32")
+        if tuple(dq_out.shape) != (s.batch, s.n_q_heads, S, s.head_dim) or dq_out.dtype != torch.float32:
+            raise ValueError("dq_out must be [B, H_q, S, d] float32")
+        attn_chunk_backward(self.handle, q, dy, lse, S, P, dq_out, dk_out, dv_out, stream)
 
     def set_score_mode(self, mode: str):
         kv_cache_set_score_mode(self.handle, mode)

@@ -356,6 +356,24 @@ int kv_cache_restore(h2okv_cache *c, const int32_t *slots, int32_t S, const h2ok
   return launch_restore(c, slots, S, delta, (cudaStream_t)stream);
 }
 
+int attn_chunk_backward(h2okv_cache *c, const void *q, const void *dy, const float *lse, int32_t S,
+                        int64_t P, float *dq_out, float *dk_out, float *dv_out, void *stream) {
+  g_err[0] = 0;
+  if (!c) return set_error(H2OKV_ERR_INVALID_ARG, "cache is NULL");
+  if (S < 1 || S > c->desc.max_chunk)
+    return set_error(H2OKV_ERR_INVALID_ARG, "S = %d outside [1, max_chunk %d]", S,
+                     c->desc.max_chunk);
+  if (P < 0 || P + S >= (int64_t)INT32_MAX)
+    return set_error(H2OKV_ERR_INVALID_ARG, "P = %lld out of range for int32 token positions",
+                     (long long)P);
+  if (!q || !dy || !lse || !dq_out || !dk_out || !dv_out)
+    return set_error(H2OKV_ERR_INVALID_ARG, "q, dy, lse, dq_out, dk_out and dv_out are required");
+  if (misaligned(q, 16) || misaligned(dy, 16) || misaligned(lse, 4) || misaligned(dq_out, 16) ||
+      misaligned(dk_out, 16) || misaligned(dv_out, 16))
+    return set_error(H2OKV_ERR_INVALID_ARG, "q, dy and the outputs must be 16-byte aligned");
+  return launch_attn_backward(c, q, dy, lse, S, P, dq_out, dk_out, dv_out, (cudaStream_t)stream);
+}
+
 int attn_chunk_with_scoresum(h2okv_cache *c, const void *q, int32_t S, int64_t P, void *y_out,
                              float *lse_out, float *w_out, float *wq_out, void *stream) {
   g_err[0] = 0;

@@ -72,6 +72,8 @@ int launch_evict_insert(h2okv_cache *c, const float *w_prev, const void *k_new, 
                         const h2okv_delta *delta, cudaStream_t st);
 int launch_restore(h2okv_cache *c, const int32_t *slots, int S, const h2okv_delta *delta,
                    cudaStream_t st);
+int launch_attn_backward(h2okv_cache *c, const void *q, const void *dy, const float *lse, int S,
+                         int64_t P, float *dq, float *dk, float *dv, cudaStream_t st);
 int launch_quantize(int kv_dtype, const __nv_bfloat16 *x, int64_t n_rows, int d, void *codes,
                     __half *scales, cudaStream_t st);
 int launch_attn_simt(h2okv_cache *c, const void *q, int S, int64_t P, void *y, float *lse,

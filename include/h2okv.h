@@ -232,6 +232,23 @@ H2OKV_API int h2o_insert_at(h2okv_cache *cache, const float *w_prev, const void 
 H2OKV_API int kv_cache_restore(h2okv_cache *cache, const int32_t *slots, int32_t S,
                                const h2okv_delta *delta, void *stream);
 
+/* Gradients of one chunk's SDPA over the cache (§A.5: autograd runs over each
+ * chunk while the cache decisions are replayed; the cache policy itself is not
+ * differentiated).  With p_ij = exp(q_i.k_j/sqrt(d) - lse_i) on the visible
+ * slots (the mask of attn_chunk_with_scoresum), dP_ij = dy_i.v_j,
+ * D_i = sum_j p_ij dP_ij and dS_ij = p_ij (dP_ij - D_i):
+ *   dq_out[b,h,i]  = sum_j dS_ij k_j / sqrt(d)               [B, H_q, S, d] f32
+ *   dk_out[b,g,j]  = sum_{h in g, i} dS_ij q_i / sqrt(d)     [B, H_k, N_C, d] f32
+ *   dv_out[b,g,j]  = sum_{h in g, i} p_ij dy_i               [B, H_k, N_C, d] f32
+ * with respect to the stored (dequantized) keys and values; the outputs are
+ * overwritten.  q, dy: [B, H_q, S, d] in q_dtype; lse: [B, H_q, S] float32, the
+ * natural-log row log-sum-exp written by attn_chunk_with_scoresum for the same
+ * chunk and cache state.  CUDA cores; the workspace holds D.  Same S / P
+ * rules as attn_chunk_with_scoresum. */
+H2OKV_API int attn_chunk_backward(h2okv_cache *cache, const void *q, const void *dy,
+                                  const float *lse, int32_t S, int64_t P, float *dq_out,
+                                  float *dk_out, float *dv_out, void *stream);
+
 /* SDPA of one chunk of queries against the cache, with summed weights (§A.1,
  * §A.7).  For query head h (group g = h / q_g), row i (token P + i):
  *   a_ij = q_i . k_j / sqrt(d_h), -inf where P + i < token_pos[b, g, j];
