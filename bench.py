@@ -120,27 +120,29 @@ class ClockSampler:
 
 
 # --------------------------------------------------------------------------- #
-def kernel_source_hash():
+def kernel_source_hash(files=None):
+    """Hash of the CUDA sources a kernel is built from (all of csrc/ when files is
+    None); paths are relative to csrc/."""
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "h2o_kv_cache_attn_b200", "csrc")
-    for f in sorted(os.listdir(csrc)):
-        if not f.endswith((".cu", ".cuh")):
-            continue
-        with open(os.path.join(csrc, f), "rb") as fh:
-            h.update(f.encode() + fh.read())
+    if files is None:
+        files = sorted(f for f in os.listdir(csrc) if f.endswith((".cu", ".cuh")))
+    for f in files:
+        with open(os.path.normpath(os.path.join(csrc, f)), "rb") as fh:
+            h.update(os.path.basename(f).encode() + fh.read())
     return h.hexdigest()[:16]
 
 
 def recorded_traffic(kernel_name):
     """DRAM bytes per launch from the committed ncu summary, if it was taken on
-    the current kernel sources (else None)."""
+    the current sources of that kernel (else None)."""
     p = os.path.join(ROOT, "profiles", "dram_traffic.json")
     if not os.path.exists(p):
         return None
     with open(p) as f:
         d = json.load(f)
     e = d.get(kernel_name)
-    if not e or e.get("source_hash") != kernel_source_hash():
+    if not e or e.get("source_hash") != kernel_source_hash(e.get("sources")):
         return None
     return e.get("bytes_per_launch")
 
@@ -266,16 +268,20 @@ def run_ours(args, wl, ws, rank, local):
     # reductions; CUDA-core path: two passes); plus the reset and the final fold
     sms = torch.cuda.get_device_properties(dev).multi_processor_count
     n_split = sum(1 for c in range(wl.n_chunks) if split_schedule(wl, wl.chunk_len(c), sms))
-    launches_per_step = wl.n_chunks * 3 + 2 * n_split + 2
+    # bf16 caches outside the split schedule: attention pass + score-sum pass
+    two_pass = tc_used and wl.kv_dtype == "bf16" and os.environ.get("H2OKV_TC_FUSED") != "1"
+    launches_per_step = wl.n_chunks * 3 + 2 * n_split + 2 + (wl.n_chunks - n_split if two_pass else 0)
     per_launch_alg = at_flops_alg / len(at_ms)
     per_launch_ms = sum(at_ms) / len(at_ms)
     if tc_used:
         roof = {"bound": "tensor", "achieved": round(tflops_alg, 2), "peak": tc_peak,
                 "unit": "TFLOP/s", "frac": round(tflops_alg / tc_peak, 4),
-                "traffic": recorded_traffic("attn_tc_kernel"),
+                "traffic": recorded_traffic("attn_fwd_kernel" if two_pass and n_split == 0 else "attn_tc_kernel"),
                 "kernel": ("attention call per chunk (attn_split_a_kernel + attn_split_b_kernel + "
                            "reduce_o_kernel + reduce_w_kernel)") if n_split == wl.n_chunks else
-                          ("attention call per chunk (attn_tc_kernel + reduce_w_kernel)" if n_split == 0 else
+                          (("attention call per chunk (attn_fwd_kernel + scoresum_kernel + reduce_w_kernel)"
+                            if two_pass else "attention call per chunk (attn_tc_kernel + reduce_w_kernel)")
+                           if n_split == 0 else
                            "attention call per chunk (split schedule on %d of %d chunks)" % (n_split, wl.n_chunks)),
                 "alg_flops_per_launch": per_launch_alg, "avg_launch_ms": round(per_launch_ms, 4),
                 "peak_kind": f"{pk_kind} bf16 dense, sustained (kernel timed inside a long step)"}

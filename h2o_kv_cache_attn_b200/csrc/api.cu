@@ -75,7 +75,7 @@ static void layout(const h2okv_cache_desc &d, const TcPlan &tc, WorkspaceLayout 
   off = align256(off + B * Hq * S * 4);
   ws->status = off;
   off = align256(off + 4);
-  ws->part_ml = ws->part_w = ws->part_o = off;
+  ws->part_ml = ws->part_w = ws->part_o = ws->nlse = off;
   if (tc.enabled) {
     const size_t seg_rows = (size_t)tc.split_ctas * tc.max_seg * 2 * 128;
     ws->part_ml = off;
@@ -84,6 +84,8 @@ static void layout(const h2okv_cache_desc &d, const TcPlan &tc, WorkspaceLayout 
     off = align256(off + B * Hq * (size_t)tc.tiles_per_head * NC * 4);
     ws->part_o = off;
     off = align256(off + seg_rows * D * 4);
+    ws->nlse = off;
+    off = align256(off + B * Hq * (size_t)tc.tiles_per_head * 128 * 4);
   }
   ws->total = off;
 }

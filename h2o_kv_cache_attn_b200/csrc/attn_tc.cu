@@ -45,6 +45,7 @@
 // Per-(query tile, slot) sums go to a partial buffer; a small reduction kernel
 // sums them in a fixed order into w [B, H_k, N_C] and wq [B, H_q, N_C].
 #include <stdio.h>
+#include <stdlib.h>
 #include <string.h>
 
 #include "h2okv_internal.cuh"
@@ -125,6 +126,7 @@ struct TcParams {
   __nv_bfloat16 *y;          // [B*Hq][S][D]
   float *lse_out;            // [B*Hq][S] or null
   float *part_w;             // [B*Hq*tiles][N_C]
+  float *nlse;               // [B*Hq*tiles][BM]: -lse2 of every row (bf16 two-pass path)
   int *status;               // device status word (0 = ok)
   int Hq, Hk, q_g, N_C, S, P, tiles, n_kt, ctas_per_group;
   float scale2;  // log2(e) / sqrt(d)
@@ -1219,6 +1221,577 @@ __global__ void __launch_bounds__(threads_of<KV>(), 1)
   }
 }
 
+// ---- bf16 caches, two passes ------------------------------------------------------
+// Pass 1 (attn_fwd_kernel): attention of two query tiles against the cache with an
+// online softmax.  Per K/V tile: S = Q K^T into TMEM; the softmax warps read their
+// row, turn it into probabilities against a running reference maximum and write them
+// back over S as bf16 pairs; O += P V then takes P straight from TMEM (the A operand)
+// and V from shared memory.  Output: y, and -lse2 of every row for pass 2.
+// Pass 2 (scoresum_kernel): the logits again, transposed (S^T = K Q^T, slots on TMEM
+// lanes), normalised with the final row LSE and summed over the rows of each slot.
+// Neither pass stores P in shared memory; pass 2 reads no V.
+constexpr int kStagesF = 3;  // pass 1 K ring
+constexpr int kStagesS = 4;  // pass 2 K ring
+constexpr float kLazyMax = 8.f;  // the reference maximum moves only when exceeded by 2^8
+constexpr uint32_t F_OFF_QA = 0;
+constexpr uint32_t F_OFF_QB = kTileBytes;
+constexpr uint32_t F_OFF_K = 2 * kTileBytes;                      // [kStagesF] K tiles
+constexpr uint32_t F_OFF_V = F_OFF_K + kStagesF * kTileBytes;      // [2] V tiles
+constexpr uint32_t F_OFF_REL = F_OFF_V + 2 * kTileBytes;           // float [kStagesF][BN]
+constexpr uint32_t F_OFF_BAR = F_OFF_REL + kStagesF * BN * 4;
+enum {
+  F_Q = 0,
+  F_KFULL0, F_KEMPTY0 = F_KFULL0 + kStagesF,   // K ring (+ slot positions)
+  F_VFULL0 = F_KEMPTY0 + kStagesF, F_VEMPTY0 = F_VFULL0 + 2,  // V ring
+  F_SFULL0 = F_VEMPTY0 + 2,                    // S of tile a / b written
+  F_PFULL0 = F_SFULL0 + 2,                     // P of tile a / b written (O rescaled)
+  F_OFULL = F_PFULL0 + 2, F_DRAIN,
+  F_END
+};
+constexpr uint32_t F_OFF_TMEM = F_OFF_BAR + F_END * 8;
+constexpr uint32_t kSmemF = F_OFF_TMEM + 16;
+static_assert(kSmemF <= 232448, "pass 1 shared memory budget");
+// P (TMEM, K-major) x V (shared memory, MN-major)
+constexpr uint32_t IDESC_TS_PV = idesc_bf16_f32(128, 128, false, true);
+
+// Maximum of a row of raw logits (eight independent chains of three-input maxima).
+template <int N>
+__device__ __forceinline__ float row_max(const uint32_t (&x)[N]) {
+  float mx8[8];
+#pragma unroll
+  for (int q = 0; q < 8; ++q) mx8[q] = fmaxf(__uint_as_float(x[q]), __uint_as_float(x[q + 8]));
+#pragma unroll
+  for (int e = 16; e < N; e += 16) {
+#pragma unroll
+    for (int q = 0; q < 8; ++q)
+      mx8[q] = fmax3(mx8[q], __uint_as_float(x[e + q]), __uint_as_float(x[e + 8 + q]));
+  }
+  return fmax3(fmax3(mx8[0], mx8[1], mx8[2]), fmax3(mx8[3], mx8[4], mx8[5]),
+               fmaxf(mx8[6], mx8[7]));
+}
+
+// Slot positions of one K tile relative to the chunk start, as floats (row i of the
+// chunk sees the slot iff rel <= i; empty or out-of-cache slots: 2^20).  One warp.
+__device__ __forceinline__ void tile_positions(float *dst, const int32_t *tpg, int kt, int N_C,
+                                               int P, int lane) {
+  const int nv = min(BN, N_C - kt * BN);
+#pragma unroll
+  for (int e = lane; e < BN; e += 32) {
+    const int64_t t = e < nv ? (int64_t)tpg[kt * BN + e] : (int64_t)kEmptyPos;
+    const int64_t rel = t - (int64_t)P;
+    dst[e] = (float)(rel < -1 ? -1 : (rel > kRelFar ? kRelFar : rel));
+  }
+}
+
+__global__ void __launch_bounds__(kThreads, 1)
+    attn_fwd_kernel(const __grid_constant__ CUtensorMap q_map,
+                    const __grid_constant__ CUtensorMap k_map,
+                    const __grid_constant__ CUtensorMap v_map, const TcParams p) {
+  extern __shared__ __align__(1024) uint8_t smem[];
+  const uint32_t sbase = smem_u32(smem);
+  if (sbase & 1023u) {
+    if (threadIdx.x == 0) atomicExch(p.status, H2OKV_ERR_CUDA);
+    return;
+  }
+  float *rel_s = reinterpret_cast<float *>(smem + F_OFF_REL);
+  uint64_t *bar = reinterpret_cast<uint64_t *>(smem + F_OFF_BAR);
+  uint32_t *tmem_s = reinterpret_cast<uint32_t *>(smem + F_OFF_TMEM);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int bg = blockIdx.x / p.ctas_per_group;
+  const int c = blockIdx.x - bg * p.ctas_per_group;
+  const int b = bg / p.Hk, g = bg - b * p.Hk;
+  const int n_qt = p.q_g * p.tiles;
+  const int qa = 2 * c, qb = 2 * c + 1;
+  const bool has_b = qb < n_qt;
+  const int hl_a = qa / p.tiles, t_a = qa - hl_a * p.tiles;
+  const int hl_b = has_b ? qb / p.tiles : hl_a, t_b = has_b ? qb - hl_b * p.tiles : t_a;
+  const int bhq_a = b * p.Hq + g * p.q_g + hl_a, bhq_b = b * p.Hq + g * p.q_g + hl_b;
+  const int i0_a = t_a * BM, i0_b = t_b * BM;
+  const int n_kt = p.n_kt;
+  const uint64_t lim = p.timeout_ns;
+  const int nwg = has_b ? 2 : 1;
+  if (threadIdx.x == 0) {
+    mbar_init(&bar[F_Q], 1);
+    for (int i = 0; i < kStagesF; ++i) {
+      mbar_init(&bar[F_KFULL0 + i], 1);
+      mbar_init(&bar[F_KEMPTY0 + i], 1 + 4 * nwg);  // MMA commit + softmax warps (positions)
+    }
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&bar[F_VFULL0 + i], 1);
+      mbar_init(&bar[F_VEMPTY0 + i], 1);
+      mbar_init(&bar[F_SFULL0 + i], 1);
+      mbar_init(&bar[F_PFULL0 + i], 4);
+    }
+    mbar_init(&bar[F_OFULL], 1);
+    mbar_init(&bar[F_DRAIN], 1);
+    fence_mbar_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_s, kTmemCols);
+    tmem_relinquish();
+    tc_fence_before();
+  }
+  if (warp == 0 && lane == 0) {
+    prefetch_tensormap(&q_map);
+    prefetch_tensormap(&k_map);
+    prefetch_tensormap(&v_map);
+  }
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_s;
+  bool aborted = false;
+
+  if (warp < 4) {
+    reg_dealloc<kCtrlRegs>();
+    if (warp == 1) {
+      // ------------------------------------------------------------------ MMA issuer
+      // TMEM columns: S / P of tile a at 0, of tile b at 128; O of tile a at 256, b at 384.
+      if (lane == 0) {
+        const uint32_t qa_addr = sbase + F_OFF_QA, qb_addr = sbase + F_OFF_QB;
+        if (!mbar_wait(&bar[F_Q], 0, lim)) fail(p, aborted);
+        tc_fence_after();
+        // S_t(kt) = Q_t K(kt)^T.  Issued after P V of the previous tile of the same
+        // query tile: the tensor core runs one thread's MMAs in order, so P (which
+        // overlays S) is read before it is overwritten.
+        auto qk = [&](int kt, int t) -> bool {
+          const int s = kt % kStagesF;
+          if (!mbar_wait(&bar[F_KFULL0 + s], (kt / kStagesF) & 1, lim)) return false;
+          tc_fence_after();
+          const uint32_t k_addr = sbase + F_OFF_K + s * kTileBytes;
+          const uint32_t q_addr = t ? qb_addr : qa_addr;
+#pragma unroll
+          for (int ks = 0; ks < D / 16; ++ks)
+            mma_bf16_ss(tmem + t * 128, kmajor_desc(q_addr, ks), kmajor_desc(k_addr, ks),
+                        IDESC_K_MAJOR, ks > 0);
+          mma_commit(&bar[F_SFULL0 + t]);
+          if (t == 1 || !has_b) mma_commit(&bar[F_KEMPTY0 + s]);  // K(kt) no longer read
+          return true;
+        };
+        // O_t += P_t(kt) V(kt): A from TMEM (16 slots = 8 columns per k-step)
+        auto pv = [&](int kt, int t) -> bool {
+          if (!mbar_wait(&bar[F_PFULL0 + t], kt & 1, lim)) return false;
+          const int v = kt & 1;
+          if (t == 0 && !mbar_wait(&bar[F_VFULL0 + v], (kt >> 1) & 1, lim)) return false;
+          tc_fence_after();
+          const uint32_t v_addr = sbase + F_OFF_V + v * kTileBytes;
+#pragma unroll
+          for (int ks = 0; ks < BN / 16; ++ks)
+            mma_bf16_ts(tmem + 256 + t * 128, tmem + t * 128 + ks * 8, mnmajor_desc(v_addr, ks),
+                        IDESC_TS_PV, (kt > 0 || ks > 0) ? 1u : 0u);
+          if (t == 1 || !has_b) mma_commit(&bar[F_VEMPTY0 + v]);  // V(kt) no longer read
+          return true;
+        };
+        if (!aborted && !qk(0, 0)) fail(p, aborted);
+        if (!aborted && has_b && !qk(0, 1)) fail(p, aborted);
+        for (int kt = 0; kt < n_kt && !aborted; ++kt) {
+          if (!pv(kt, 0)) { fail(p, aborted); break; }
+          if (kt + 1 < n_kt && !qk(kt + 1, 0)) { fail(p, aborted); break; }
+          if (has_b) {
+            if (!pv(kt, 1)) { fail(p, aborted); break; }
+            if (kt + 1 < n_kt && !qk(kt + 1, 1)) { fail(p, aborted); break; }
+          }
+        }
+        mma_commit(&bar[F_OFULL]);
+        mma_commit(&bar[F_DRAIN]);
+        mbar_wait(&bar[F_DRAIN], 0, 4000000000ull);
+      }
+      __syncwarp();
+    } else if (warp == 0) {
+      // ----------------------------------------- producer of Q, K and slot positions
+      if (lane == 0) {
+        mbar_expect_tx(&bar[F_Q], has_b ? 2 * kTileBytes : kTileBytes);
+        tma_load_3d(smem + F_OFF_QA, &q_map, &bar[F_Q], 0, i0_a, bhq_a);
+        tma_load_3d(smem + F_OFF_QA + kHalfBytes, &q_map, &bar[F_Q], 64, i0_a, bhq_a);
+        if (has_b) {
+          tma_load_3d(smem + F_OFF_QB, &q_map, &bar[F_Q], 0, i0_b, bhq_b);
+          tma_load_3d(smem + F_OFF_QB + kHalfBytes, &q_map, &bar[F_Q], 64, i0_b, bhq_b);
+        }
+        mbar_arrive(&bar[F_Q]);
+      }
+      const int32_t *tpg = p.token_pos + (size_t)bg * p.N_C;
+      int issued = 0;
+      for (int kt = 0; kt < n_kt && !aborted; ++kt) {
+        const int s = kt % kStagesF, n = kt / kStagesF;
+        if (n > 0 && !warp_wait(&bar[F_KEMPTY0 + s], (n - 1) & 1, lim)) { fail(p, aborted); break; }
+        uint8_t *kdst = smem + F_OFF_K + s * kTileBytes;
+        if (lane == 0) {
+          mbar_expect_tx(&bar[F_KFULL0 + s], kTileBytes);
+          tma_load_3d(kdst, &k_map, &bar[F_KFULL0 + s], 0, kt * BN, bg);
+          tma_load_3d(kdst + kHalfBytes, &k_map, &bar[F_KFULL0 + s], 64, kt * BN, bg);
+          if (kt + kPrefetch < n_kt) {
+            tma_prefetch_l2_3d(&k_map, 0, (kt + kPrefetch) * BN, bg);
+            tma_prefetch_l2_3d(&k_map, 64, (kt + kPrefetch) * BN, bg);
+          }
+        }
+        tile_positions(rel_s + s * BN, tpg, kt, p.N_C, p.P, lane);
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&bar[F_KFULL0 + s]);
+        issued = kt + 1;
+      }
+      // drain: the last issued loads land before exit
+      if (lane == 0) {
+        mbar_wait(&bar[F_Q], 0, 4000000000ull);
+        for (int kt = issued - 1; kt >= 0 && kt >= issued - kStagesF; --kt)
+          mbar_wait(&bar[F_KFULL0 + kt % kStagesF], (kt / kStagesF) & 1, 4000000000ull);
+      }
+    } else if (warp == 2) {
+      // ------------------------------------------------------------------ producer of V
+      if (lane == 0) {
+        int issued = 0;
+        for (int kt = 0; kt < n_kt && !aborted; ++kt) {
+          const int v = kt & 1, n = kt >> 1;
+          if (n > 0 && !mbar_wait(&bar[F_VEMPTY0 + v], (n - 1) & 1, lim)) { fail(p, aborted); break; }
+          uint8_t *vdst = smem + F_OFF_V + v * kTileBytes;
+          mbar_expect_tx(&bar[F_VFULL0 + v], kTileBytes);
+          tma_load_3d(vdst, &v_map, &bar[F_VFULL0 + v], 0, kt * BN, bg);
+          tma_load_3d(vdst + kHalfBytes, &v_map, &bar[F_VFULL0 + v], 64, kt * BN, bg);
+          mbar_arrive(&bar[F_VFULL0 + v]);
+          if (kt + kPrefetch < n_kt) {
+            tma_prefetch_l2_3d(&v_map, 0, (kt + kPrefetch) * BN, bg);
+            tma_prefetch_l2_3d(&v_map, 64, (kt + kPrefetch) * BN, bg);
+          }
+          issued = kt + 1;
+        }
+        for (int kt = issued - 1; kt >= 0 && kt >= issued - 2; --kt)
+          mbar_wait(&bar[F_VFULL0 + (kt & 1)], (kt >> 1) & 1, 4000000000ull);
+      }
+      __syncwarp();
+    }
+  } else {
+    reg_alloc<kSoftRegs>();
+    const int t = (warp - 4) >> 2;  // 0: tile a, 1: tile b
+    if (t == 0 || has_b) {
+      // ------------------------------------- online softmax, one thread per query row
+      const int st = threadIdx.x - 128 * (1 + t);
+      const uint32_t lane_base = (uint32_t)(32 * (warp & 3)) << 16;
+      const uint32_t s_col = tmem + lane_base + t * 128, o_col = tmem + lane_base + 256 + t * 128;
+      const float c2 = p.scale2;
+      const int i0 = t ? i0_b : i0_a, bhq = t ? bhq_b : bhq_a, tt = t ? t_b : t_a;
+      const float mbias = kMaskBias / c2;
+      float m = -INFINITY, l = 0.f;  // reference maximum (base 2) and sum against it
+      uint32_t x[BN];
+      for (int kt = 0; kt < n_kt && !aborted; ++kt) {
+        const int s = kt % kStagesF;
+        if (!warp_wait(&bar[F_SFULL0 + t], kt & 1, lim)) { fail(p, aborted); break; }
+        if (!warp_wait(&bar[F_KFULL0 + s], (kt / kStagesF) & 1, lim)) { fail(p, aborted); break; }
+        tc_fence_after();
+        const float *rel = rel_s + s * BN;
+        const float rv = fmax3(fmaxf(rel[lane], rel[lane + 32]), rel[lane + 64], rel[lane + 96]);
+        const bool masked = __any_sync(0xffffffffu, rv > (float)i0);
+        tmem_ld32(s_col, *reinterpret_cast<uint32_t(*)[32]>(x));
+        tmem_ld32(s_col + 32, *reinterpret_cast<uint32_t(*)[32]>(x + 32));
+        tmem_ld32(s_col + 64, *reinterpret_cast<uint32_t(*)[32]>(x + 64));
+        tmem_ld32(s_col + 96, *reinterpret_cast<uint32_t(*)[32]>(x + 96));
+        tmem_wait_ld();
+        if (masked) row_mask<BN>(x, rel, (float)(i0 + st), mbias);
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&bar[F_KEMPTY0 + s]);
+        // the reference maximum follows the row maximum lazily: p <= 2^8 in between
+        const float mx = row_max<BN>(x) * c2;
+        const bool need = mx > m + kLazyMax;
+        if (__any_sync(0xffffffffu, need)) {
+          const float m_new = need ? mx : m;
+          const float f = ex2(m - m_new);  // 1 if unchanged, 0 from -inf
+          l *= f;
+          if (kt > 0) {
+            // O holds the sums of P V up to the previous tile: every MMA before S(kt)
+            // is complete, none after it is issued until this warp's P is written
+#pragma unroll 1
+            for (int cq = 0; cq < 4; ++cq) {
+              uint32_t o[32];
+              tmem_ld32(o_col + cq * 32, o);
+              tmem_wait_ld();
+#pragma unroll
+              for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * f);
+              tmem_st32(o_col + cq * 32, o);
+            }
+          }
+          m = m_new;
+        }
+        // probabilities against the reference maximum, packed to bf16 pairs over S
+        const float2 c2v = make_float2(c2, c2), negm = make_float2(-m, -m);
+        float2 acc[4];
+#pragma unroll
+        for (int q = 0; q < 4; ++q) acc[q] = make_float2(0.f, 0.f);
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+          uint32_t pk[32];
+#pragma unroll
+          for (int e = 0; e < 64; e += 2) {
+            const int ee = 64 * h + e;
+            const float2 a =
+                fma2(make_float2(__uint_as_float(x[ee]), __uint_as_float(x[ee + 1])), c2v, negm);
+            const float2 v = make_float2(ex2(a.x), ex2(a.y));
+            acc[(e >> 1) & 3] = add2(acc[(e >> 1) & 3], v);
+            pk[e >> 1] = pack_bf16x2(v.x, v.y);
+          }
+          tmem_st32(s_col + 32 * h, pk);
+        }
+        const float2 s01 = add2(acc[0], acc[1]), s23 = add2(acc[2], acc[3]);
+        const float2 s4 = add2(s01, s23);
+        l += s4.x + s4.y;
+        tmem_wait_st();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&bar[F_PFULL0 + t]);
+      }
+      // row results: -lse2 for pass 2, lse (natural log) on request, y = O / l
+      const bool seen = l > 0.f && m > -0.5f * kMaskBias;
+      const float lse2 = seen ? m + lg2(l) : -INFINITY;
+      const bool row_ok = i0 + st < p.S;
+      p.nlse[((size_t)bhq * p.tiles + tt) * BM + st] = seen ? -lse2 : -kMaskBias;
+      if (p.lse_out && row_ok) p.lse_out[(size_t)bhq * p.S + i0 + st] = lse2 * 0.69314718055994531f;
+      if (!aborted && !warp_wait(&bar[F_OFULL], 0, lim)) fail(p, aborted);
+      tc_fence_after();
+      if (!aborted) {
+        const float inv = seen ? 1.f / l : 0.f;
+        __nv_bfloat16 *yrow = p.y + ((size_t)bhq * p.S + i0 + st) * D;
+        uint32_t r[32];
+#pragma unroll
+        for (int cq = 0; cq < 4; ++cq) {
+          tmem_ld32(o_col + cq * 32, r);
+          tmem_wait_ld();
+          if (row_ok) {
+            uint32_t o[16];
+#pragma unroll
+            for (int e = 0; e < 16; ++e)
+              o[e] = pack_bf16x2(__uint_as_float(r[2 * e]) * inv, __uint_as_float(r[2 * e + 1]) * inv);
+            uint4 *dst = reinterpret_cast<uint4 *>(yrow + cq * 32);
+#pragma unroll
+            for (int e = 0; e < 4; ++e)
+              dst[e] = make_uint4(o[4 * e], o[4 * e + 1], o[4 * e + 2], o[4 * e + 3]);
+          }
+        }
+      }
+      tc_fence_before();
+    }
+  }
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, kTmemCols);
+  }
+}
+
+// Pass 2 shared memory: Q_a, Q_b, the K ring, slot positions, -lse2 of both tiles.
+constexpr uint32_t S_OFF_QA = 0;
+constexpr uint32_t S_OFF_QB = kTileBytes;
+constexpr uint32_t S_OFF_K = 2 * kTileBytes;                   // [kStagesS] K tiles
+constexpr uint32_t S_OFF_REL = S_OFF_K + kStagesS * kTileBytes;  // float [kStagesS][BN]
+constexpr uint32_t S_OFF_NLSE = S_OFF_REL + kStagesS * BN * 4;   // float [2][BM]
+constexpr uint32_t S_OFF_BAR = S_OFF_NLSE + 2 * BM * 4;
+enum {
+  G_Q = 0,
+  G_KFULL0, G_KEMPTY0 = G_KFULL0 + kStagesS,
+  G_SFULL0 = G_KEMPTY0 + kStagesS, G_SFREE0 = G_SFULL0 + 2,  // S^T pair, double buffered
+  G_DRAIN = G_SFREE0 + 2,
+  G_END
+};
+constexpr uint32_t S_OFF_TMEM = S_OFF_BAR + G_END * 8;
+constexpr uint32_t kSmemS = S_OFF_TMEM + 16;
+static_assert(kSmemS <= 232448, "pass 2 shared memory budget");
+
+// Sum over the rows of one tile of the normalised probabilities of one slot:
+// sum_r 2^(c2 s_r - lse2_r) over visible rows r (rmin <= r < rmax).
+__device__ __forceinline__ float slot_colsum(const uint32_t (&r)[BM], const float *nlse, float c2,
+                                             int rmin, int rmax, bool full) {
+  const float rminf = (float)rmin;
+  const float2 c2v = make_float2(c2, c2);
+  float2 acc[4];
+#pragma unroll
+  for (int q = 0; q < 4; ++q) acc[q] = make_float2(0.f, 0.f);
+#pragma unroll
+  for (int e = 0; e < BM; e += 2) {
+    const float2 nl = *reinterpret_cast<const float2 *>(nlse + e);
+    float2 a = fma2(make_float2(__uint_as_float(r[e]), __uint_as_float(r[e + 1])), c2v, nl);
+    if (!full) {  // rows before rmin are masked: nm = sat(rmin - row) is 1 there
+      const float2 nm = make_float2(fma_sat(rminf, 1.f, -(float)e), fma_sat(rminf, 1.f, -(float)(e + 1)));
+      a = fma2(nm, make_float2(-kMaskBias, -kMaskBias), a);
+    }
+    float2 v = make_float2(ex2(a.x), ex2(a.y));
+    if (rmax < BM) {  // rows past the chunk (last row tile only)
+      v.x = e < rmax ? v.x : 0.f;
+      v.y = e + 1 < rmax ? v.y : 0.f;
+    }
+    acc[(e >> 1) & 3] = add2(acc[(e >> 1) & 3], v);
+  }
+  const float2 s01 = add2(acc[0], acc[1]), s23 = add2(acc[2], acc[3]);
+  const float2 s4 = add2(s01, s23);
+  return s4.x + s4.y;
+}
+
+__global__ void __launch_bounds__(kThreads, 1)
+    scoresum_kernel(const __grid_constant__ CUtensorMap q_map,
+                    const __grid_constant__ CUtensorMap k_map, const TcParams p) {
+  extern __shared__ __align__(1024) uint8_t smem[];
+  const uint32_t sbase = smem_u32(smem);
+  if (sbase & 1023u) {
+    if (threadIdx.x == 0) atomicExch(p.status, H2OKV_ERR_CUDA);
+    return;
+  }
+  float *rel_s = reinterpret_cast<float *>(smem + S_OFF_REL);
+  float *nlse_s = reinterpret_cast<float *>(smem + S_OFF_NLSE);
+  uint64_t *bar = reinterpret_cast<uint64_t *>(smem + S_OFF_BAR);
+  uint32_t *tmem_s = reinterpret_cast<uint32_t *>(smem + S_OFF_TMEM);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int bg = blockIdx.x / p.ctas_per_group;
+  const int c = blockIdx.x - bg * p.ctas_per_group;
+  const int b = bg / p.Hk, g = bg - b * p.Hk;
+  const int n_qt = p.q_g * p.tiles;
+  const int qa = 2 * c, qb = 2 * c + 1;
+  const bool has_b = qb < n_qt;
+  const int hl_a = qa / p.tiles, t_a = qa - hl_a * p.tiles;
+  const int hl_b = has_b ? qb / p.tiles : hl_a, t_b = has_b ? qb - hl_b * p.tiles : t_a;
+  const int bhq_a = b * p.Hq + g * p.q_g + hl_a, bhq_b = b * p.Hq + g * p.q_g + hl_b;
+  const int i0_a = t_a * BM, i0_b = t_b * BM;
+  const int n_kt = p.n_kt;
+  const uint64_t lim = p.timeout_ns;
+  const int nwg = has_b ? 2 : 1;
+  if (threadIdx.x == 0) {
+    mbar_init(&bar[G_Q], 1);
+    for (int i = 0; i < kStagesS; ++i) {
+      mbar_init(&bar[G_KFULL0 + i], 1);
+      mbar_init(&bar[G_KEMPTY0 + i], 1 + 4 * nwg);
+    }
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&bar[G_SFULL0 + i], 1);
+      mbar_init(&bar[G_SFREE0 + i], 4 * nwg);
+    }
+    mbar_init(&bar[G_DRAIN], 1);
+    fence_mbar_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_s, kTmemCols);
+    tmem_relinquish();
+    tc_fence_before();
+  }
+  if (warp == 0 && lane == 0) {
+    prefetch_tensormap(&q_map);
+    prefetch_tensormap(&k_map);
+  }
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_s;
+  bool aborted = false;
+
+  if (warp < 4) {
+    reg_dealloc<kCtrlRegs>();
+    if (warp == 1) {
+      // ------------------------------------------------------------------ MMA issuer
+      // S^T_t(kt) = K(kt) Q_t^T into columns 256 (kt & 1) + 128 t
+      if (lane == 0) {
+        const uint32_t qa_addr = sbase + S_OFF_QA, qb_addr = sbase + S_OFF_QB;
+        if (!mbar_wait(&bar[G_Q], 0, lim)) fail(p, aborted);
+        tc_fence_after();
+        for (int kt = 0; kt < n_kt && !aborted; ++kt) {
+          const int s = kt % kStagesS, u = kt & 1;
+          if (!mbar_wait(&bar[G_KFULL0 + s], (kt / kStagesS) & 1, lim)) { fail(p, aborted); break; }
+          if (kt >= 2 && !mbar_wait(&bar[G_SFREE0 + u], ((kt >> 1) - 1) & 1, lim)) {
+            fail(p, aborted);
+            break;
+          }
+          tc_fence_after();
+          const uint32_t k_addr = sbase + S_OFF_K + s * kTileBytes;
+#pragma unroll
+          for (int ks = 0; ks < D / 16; ++ks)
+            mma_bf16_ss(tmem + u * 256, kmajor_desc(k_addr, ks), kmajor_desc(qa_addr, ks),
+                        IDESC_K_MAJOR, ks > 0);
+          if (has_b) {
+#pragma unroll
+            for (int ks = 0; ks < D / 16; ++ks)
+              mma_bf16_ss(tmem + u * 256 + 128, kmajor_desc(k_addr, ks), kmajor_desc(qb_addr, ks),
+                          IDESC_K_MAJOR, ks > 0);
+          }
+          mma_commit(&bar[G_SFULL0 + u]);
+          mma_commit(&bar[G_KEMPTY0 + s]);
+        }
+        mma_commit(&bar[G_DRAIN]);
+        mbar_wait(&bar[G_DRAIN], 0, 4000000000ull);
+      }
+      __syncwarp();
+    } else if (warp == 0) {
+      // ----------------------------------------- producer of Q, K and slot positions
+      if (lane == 0) {
+        mbar_expect_tx(&bar[G_Q], has_b ? 2 * kTileBytes : kTileBytes);
+        tma_load_3d(smem + S_OFF_QA, &q_map, &bar[G_Q], 0, i0_a, bhq_a);
+        tma_load_3d(smem + S_OFF_QA + kHalfBytes, &q_map, &bar[G_Q], 64, i0_a, bhq_a);
+        if (has_b) {
+          tma_load_3d(smem + S_OFF_QB, &q_map, &bar[G_Q], 0, i0_b, bhq_b);
+          tma_load_3d(smem + S_OFF_QB + kHalfBytes, &q_map, &bar[G_Q], 64, i0_b, bhq_b);
+        }
+        mbar_arrive(&bar[G_Q]);
+      }
+      const int32_t *tpg = p.token_pos + (size_t)bg * p.N_C;
+      int issued = 0;
+      for (int kt = 0; kt < n_kt && !aborted; ++kt) {
+        const int s = kt % kStagesS, n = kt / kStagesS;
+        if (n > 0 && !warp_wait(&bar[G_KEMPTY0 + s], (n - 1) & 1, lim)) { fail(p, aborted); break; }
+        uint8_t *kdst = smem + S_OFF_K + s * kTileBytes;
+        if (lane == 0) {
+          mbar_expect_tx(&bar[G_KFULL0 + s], kTileBytes);
+          tma_load_3d(kdst, &k_map, &bar[G_KFULL0 + s], 0, kt * BN, bg);
+          tma_load_3d(kdst + kHalfBytes, &k_map, &bar[G_KFULL0 + s], 64, kt * BN, bg);
+          if (kt + kPrefetch < n_kt) {
+            tma_prefetch_l2_3d(&k_map, 0, (kt + kPrefetch) * BN, bg);
+            tma_prefetch_l2_3d(&k_map, 64, (kt + kPrefetch) * BN, bg);
+          }
+        }
+        tile_positions(rel_s + s * BN, tpg, kt, p.N_C, p.P, lane);
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&bar[G_KFULL0 + s]);
+        issued = kt + 1;
+      }
+      if (lane == 0) {
+        mbar_wait(&bar[G_Q], 0, 4000000000ull);
+        for (int kt = issued - 1; kt >= 0 && kt >= issued - kStagesS; --kt)
+          mbar_wait(&bar[G_KFULL0 + kt % kStagesS], (kt / kStagesS) & 1, 4000000000ull);
+      }
+    }
+  } else {
+    reg_alloc<kSoftRegs>();
+    const int t = (warp - 4) >> 2;
+    if (t == 0 || has_b) {
+      // ------------------------------------- column sums, one thread per slot of a tile
+      const int st = threadIdx.x - 128 * (1 + t);
+      const uint32_t lane_base = (uint32_t)(32 * (warp & 3)) << 16;
+      const float c2 = p.scale2;
+      const int i0 = t ? i0_b : i0_a, bhq = t ? bhq_b : bhq_a, tt = t ? t_b : t_a;
+      float *nl = nlse_s + t * BM;
+      nl[st] = p.nlse[((size_t)bhq * p.tiles + tt) * BM + st];
+      named_bar_sync(1 + t, 128);
+      const int rmax = min(BM, p.S - i0);
+      float *pw = p.part_w + ((size_t)bhq * p.tiles + tt) * p.N_C;
+      for (int kt = 0; kt < n_kt && !aborted; ++kt) {
+        const int s = kt % kStagesS, u = kt & 1;
+        const int j = kt * BN + st;
+        if (!warp_wait(&bar[G_SFULL0 + u], (kt >> 1) & 1, lim)) { fail(p, aborted); break; }
+        if (!warp_wait(&bar[G_KFULL0 + s], (kt / kStagesS) & 1, lim)) { fail(p, aborted); break; }
+        tc_fence_after();
+        const float relj = rel_s[s * BN + st];
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&bar[G_KEMPTY0 + s]);
+        // visible rows r of this tile: relj <= i0 + r, r < rmax
+        const float rmf = fminf(fmaxf(relj - (float)i0, 0.f), (float)BM);
+        const int rmin = (int)rmf;
+        const bool full = __all_sync(0xffffffffu, rmin == 0 && rmax == BM);
+        uint32_t r[BM];
+        tmem_ld128(tmem + lane_base + u * 256 + t * 128, r);
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&bar[G_SFREE0 + u]);
+        const float cs = slot_colsum(r, nl, c2, rmin, rmax, full);
+        if (j < p.N_C) pw[j] = cs;
+      }
+      tc_fence_before();
+    }
+  }
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, kTmemCols);
+  }
+}
+
 // ---- split scheduling (bf16 cache): the two passes as persistent kernels ----------
 // With one CTA per pair of query tiles, a grid of P pairs fills ceil(P / SMs) waves
 // and leaves SMs idle in the last one (P = 128 on 148 SMs: 14 % idle).  Here the
@@ -1947,6 +2520,10 @@ void tc_plan(const h2okv_cache_desc &d, TcPlan *plan) {
   plan->tiles_per_head = (d.max_chunk + BM - 1) / BM;
   plan->split_ctas = 0;
   plan->max_seg = 0;
+  // bf16 caches: attention and score sums as two passes unless H2OKV_TC_FUSED=1 selects
+  // the single kernel that runs both phases per CTA
+  const char *fused = getenv("H2OKV_TC_FUSED");
+  plan->two_pass = !(fused && fused[0] == '1');
   int dev = 0, sms = 0;
   if (plan->enabled && cudaGetDevice(&dev) == cudaSuccess &&
       cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) == cudaSuccess) {
@@ -2008,6 +2585,27 @@ int prepare_split_kernel(K kernel, int &ready_dev, const char *name) {
   return H2OKV_OK;
 }
 
+// Shared-memory opt-in and register check of a bf16 two-pass kernel.
+template <typename K>
+int prepare_pass_kernel(K kernel, uint32_t smem_bytes, int &ready_dev, const char *name) {
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (ready_dev == dev) return H2OKV_OK;
+  cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       (int)smem_bytes);
+  if (e != cudaSuccess)
+    return set_error(H2OKV_ERR_CUDA, "cudaFuncSetAttribute(%s): %s", name, cudaGetErrorString(e));
+  cudaFuncAttributes fa;
+  e = cudaFuncGetAttributes(&fa, kernel);
+  if (e != cudaSuccess)
+    return set_error(H2OKV_ERR_CUDA, "cudaFuncGetAttributes(%s): %s", name, cudaGetErrorString(e));
+  if (fa.numRegs != kLaunchRegs)
+    return set_error(H2OKV_ERR_UNSUPPORTED, "%s built with %d registers per thread, expected %d",
+                     name, fa.numRegs, kLaunchRegs);
+  ready_dev = dev;
+  return H2OKV_OK;
+}
+
 template <int KV>
 int launch_kernel(int grid, const CUtensorMap &qmap, const CUtensorMap &kmap,
                   const CUtensorMap &vmap, const TcParams &prm, cudaStream_t st) {
@@ -2051,6 +2649,7 @@ int launch_attn_tc(h2okv_cache *c, const void *q, int S, int64_t P, void *y, flo
   prm.y = reinterpret_cast<__nv_bfloat16 *>(y);
   prm.lse_out = lse;
   prm.part_w = reinterpret_cast<float *>(ws + c->ws.part_w);
+  prm.nlse = reinterpret_cast<float *>(ws + c->ws.nlse);
   prm.status = reinterpret_cast<int *>(ws + c->ws.status);
   prm.Hq = d.n_q_heads;
   prm.Hk = d.n_kv_heads;
@@ -2091,6 +2690,24 @@ int launch_attn_tc(h2okv_cache *c, const void *q, int S, int64_t P, void *y, flo
     const long long n_threads = (long long)n_pairs * 2 * BM * (D / 4);
     reduce_o_kernel<<<(unsigned)((n_threads + 255) / 256), 256, 0, st>>>(sp, n_pairs);
     rc = check_launch("reduce_o_kernel");
+    if (rc) return rc;
+    dim3 rgrid((d.capacity + 255) / 256, d.batch * d.n_kv_heads);
+    reduce_w_kernel<<<rgrid, 256, 0, st>>>(prm.part_w, w, wq, d.n_q_heads, d.n_kv_heads, prm.q_g,
+                                           d.capacity, prm.tiles, prm.tiles);
+    return check_launch("reduce_w_kernel");
+  }
+  if (d.kv_dtype == H2OKV_BF16 && c->tc.two_pass) {
+    // attention with an online softmax, then the score sums against the final LSE
+    static thread_local int ready_f = -1, ready_s = -1;
+    rc = prepare_pass_kernel(attn_fwd_kernel, kSmemF, ready_f, "attn_fwd_kernel");
+    if (rc) return rc;
+    rc = prepare_pass_kernel(scoresum_kernel, kSmemS, ready_s, "scoresum_kernel");
+    if (rc) return rc;
+    attn_fwd_kernel<<<grid, kThreads, kSmemF, st>>>(qmap, kmap, vmap, prm);
+    rc = check_launch("attn_fwd_kernel");
+    if (rc) return rc;
+    scoresum_kernel<<<grid, kThreads, kSmemS, st>>>(qmap, kmap, prm);
+    rc = check_launch("scoresum_kernel");
     if (rc) return rc;
     dim3 rgrid((d.capacity + 255) / 256, d.batch * d.n_kv_heads);
     reduce_w_kernel<<<rgrid, 256, 0, st>>>(prm.part_w, w, wq, d.n_q_heads, d.n_kv_heads, prm.q_g,

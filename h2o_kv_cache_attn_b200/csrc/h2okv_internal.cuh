@@ -20,6 +20,7 @@ struct WorkspaceLayout {
   size_t part_ml;      // float2 [split CTAs * segments * 2 * 128]: partial (max, sum) per row
   size_t part_w;       // float [B*Hq*row_tiles*N_C]: per-row-tile summed weights (tensor-core path)
   size_t part_o;       // float [split CTAs * segments * 2 * 128 * d]: partial outputs
+  size_t nlse;         // float [B*Hq*row_tiles*128]: -lse2 per row of every row tile
   size_t status;       // int32: device status word (0 = ok, else an H2OKV_ERR_* code)
   size_t total;
 };
@@ -29,6 +30,7 @@ struct TcPlan {          // launch plan of the tensor-core path
   int tiles_per_head;    // ceil(max_chunk / 128)
   int split_ctas;        // CTAs of the split (persistent) kernels, 0 = split scheduling off
   int max_seg;           // segments per CTA the split workspace is sized for
+  bool two_pass;         // bf16: attention pass + score-sum pass (else the fused kernel)
   bool maps_ready;       // k_map / v_map encoded
   alignas(64) unsigned char k_map[128];  // CUtensorMap over keys
   alignas(64) unsigned char v_map[128];  // CUtensorMap over values

@@ -68,6 +68,19 @@ def test_tc_workload_every_chunk(wl, cuda_device):
     assert n == wl.n_chunks
 
 
+# bf16 caches run two passes (attention with an online softmax, then the score sums
+# against the final LSE); H2OKV_TC_FUSED=1 selects the single kernel that runs both
+# phases per CTA.  Both stay at parity.
+FUSED_CASES = [CASES[0], CASES[1], CASES[2], CASES[6]]
+
+
+@pytest.mark.parametrize("wl", FUSED_CASES, ids=[w.name for w in FUSED_CASES])
+def test_tc_fused_kernel(wl, cuda_device, monkeypatch):
+    monkeypatch.setenv("H2OKV_TC_FUSED", "1")
+    run, n = run_and_check(wl, cuda_device)
+    assert n == wl.n_chunks
+
+
 def test_forced_wait_timeout_reports_status_and_recovers(cuda_device):
     """Every device-side wait of the tensor-core kernel is bounded.  With the
     limit set to 0 the first wait that is not already complete gives up: the
