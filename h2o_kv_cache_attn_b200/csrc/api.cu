@@ -151,6 +151,7 @@ int kv_cache_create(const h2okv_cache_desc *desc, const h2okv_cache_buffers *buf
   c->bufs = *bufs;
   if (!quant) c->bufs.k_scales = c->bufs.v_scales = nullptr;
   c->n_filled = 0;
+  c->n_span = 0;
   c->row_bytes = kv_row_bytes(desc->kv_dtype, desc->head_dim);
   tc_plan(*desc, &c->tc);
   c->tc.maps_ready = false;
@@ -187,6 +188,7 @@ int kv_cache_reset(h2okv_cache *c, void *stream) {
   int rc = launch_init_cache(c, (cudaStream_t)stream);
   if (rc) return rc;
   c->n_filled = 0;
+  c->n_span = 0;
   return H2OKV_OK;
 }
 
@@ -231,6 +233,7 @@ int kv_cache_set_fill(h2okv_cache *c, int32_t n_filled) {
     return set_error(H2OKV_ERR_INVALID_ARG, "n_filled %d outside [0, %d]", n_filled,
                      c->desc.capacity);
   c->n_filled = n_filled;
+  c->n_span = c->desc.capacity;  // a state written directly may occupy any slot
   return H2OKV_OK;
 }
 
@@ -270,6 +273,8 @@ int h2o_evict_insert(h2okv_cache *c, const float *w_prev, const void *k_new, con
                                (cudaStream_t)stream);
   if (rc) return rc;
   c->n_filled = c->n_filled + S > c->desc.capacity ? c->desc.capacity : c->n_filled + S;
+  // the policy fills slots left to right before it evicts
+  if (c->n_filled > c->n_span) c->n_span = c->n_filled;
   return H2OKV_OK;
 }
 
@@ -323,6 +328,7 @@ int h2o_evict_insert_delta(h2okv_cache *c, const float *w_prev, const void *k_ne
                            (cudaStream_t)stream);
   if (rc) return rc;
   c->n_filled = c->n_filled + S > c->desc.capacity ? c->desc.capacity : c->n_filled + S;
+  if (c->n_filled > c->n_span) c->n_span = c->n_filled;
   return H2OKV_OK;
 }
 
@@ -342,6 +348,7 @@ int h2o_insert_at(h2okv_cache *c, const float *w_prev, const void *k_new, const 
                            (cudaStream_t)stream);
   if (rc) return rc;
   c->n_filled = c->n_filled + S > c->desc.capacity ? c->desc.capacity : c->n_filled + S;
+  c->n_span = c->desc.capacity;  // logged slots may lie anywhere
   return H2OKV_OK;
 }
 

@@ -1238,7 +1238,13 @@ constexpr uint32_t F_OFF_QB = kTileBytes;
 constexpr uint32_t F_OFF_K = 2 * kTileBytes;                      // [kStagesF] K tiles
 constexpr uint32_t F_OFF_V = F_OFF_K + kStagesF * kTileBytes;      // [2] V tiles
 constexpr uint32_t F_OFF_REL = F_OFF_V + 2 * kTileBytes;           // float [kStagesF][BN]
-constexpr uint32_t F_OFF_BAR = F_OFF_REL + kStagesF * BN * 4;
+// Per K stage, the slots that some row of the CTA may not see (position beyond the
+// first row of a query tile): int count, then up to kMaxCand (slot, position) pairs;
+// count -1 when there are more (the softmax then masks the whole row).
+constexpr int kMaxCand = 16;
+constexpr uint32_t F_OFF_CAND = F_OFF_REL + kStagesF * BN * 4;     // [kStagesF][1 + 2 kMaxCand]
+constexpr uint32_t kCandWords = 2 + 2 * kMaxCand;                  // count, pad, pairs
+constexpr uint32_t F_OFF_BAR = F_OFF_CAND + kStagesF * kCandWords * 4;
 enum {
   F_Q = 0,
   F_KFULL0, F_KEMPTY0 = F_KFULL0 + kStagesF,   // K ring (+ slot positions)
@@ -1268,6 +1274,26 @@ __device__ __forceinline__ float row_max(const uint32_t (&x)[N]) {
   }
   return fmax3(fmax3(mx8[0], mx8[1], mx8[2]), fmax3(mx8[3], mx8[4], mx8[5]),
                fmaxf(mx8[6], mx8[7]));
+}
+
+// Probabilities 2^(c2 x - m) of one row of raw logits, packed to bf16 pairs, and
+// their sum.
+__device__ __forceinline__ float row_probs(const uint32_t (&x)[BN], float c2, float m,
+                                           uint32_t (&pk)[BN / 2]) {
+  const float2 c2v = make_float2(c2, c2), negm = make_float2(-m, -m);
+  float2 acc[4];
+#pragma unroll
+  for (int q = 0; q < 4; ++q) acc[q] = make_float2(0.f, 0.f);
+#pragma unroll
+  for (int e = 0; e < BN; e += 2) {
+    const float2 a = fma2(make_float2(__uint_as_float(x[e]), __uint_as_float(x[e + 1])), c2v, negm);
+    const float2 v = make_float2(ex2(a.x), ex2(a.y));
+    acc[(e >> 1) & 3] = add2(acc[(e >> 1) & 3], v);
+    pk[e >> 1] = pack_bf16x2(v.x, v.y);
+  }
+  const float2 s01 = add2(acc[0], acc[1]), s23 = add2(acc[2], acc[3]);
+  const float2 s4 = add2(s01, s23);
+  return s4.x + s4.y;
 }
 
 // Slot positions of one K tile relative to the chunk start, as floats (row i of the
@@ -1367,29 +1393,52 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (t == 1 || !has_b) mma_commit(&bar[F_KEMPTY0 + s]);  // K(kt) no longer read
           return true;
         };
-        // O_t += P_t(kt) V(kt): A from TMEM (16 slots = 8 columns per k-step)
-        auto pv = [&](int kt, int t) -> bool {
-          if (!mbar_wait(&bar[F_PFULL0 + t], kt & 1, lim)) return false;
-          const int v = kt & 1;
-          if (t == 0 && !mbar_wait(&bar[F_VFULL0 + v], (kt >> 1) & 1, lim)) return false;
-          tc_fence_after();
-          const uint32_t v_addr = sbase + F_OFF_V + v * kTileBytes;
-#pragma unroll
-          for (int ks = 0; ks < BN / 16; ++ks)
-            mma_bf16_ts(tmem + 256 + t * 128, tmem + t * 128 + ks * 8, mnmajor_desc(v_addr, ks),
-                        IDESC_TS_PV, (kt > 0 || ks > 0) ? 1u : 0u);
-          if (t == 1 || !has_b) mma_commit(&bar[F_VEMPTY0 + v]);  // V(kt) no longer read
-          return true;
-        };
         if (!aborted && !qk(0, 0)) fail(p, aborted);
         if (!aborted && has_b && !qk(0, 1)) fail(p, aborted);
-        for (int kt = 0; kt < n_kt && !aborted; ++kt) {
-          if (!pv(kt, 0)) { fail(p, aborted); break; }
-          if (kt + 1 < n_kt && !qk(kt + 1, 0)) { fail(p, aborted); break; }
-          if (has_b) {
-            if (!pv(kt, 1)) { fail(p, aborted); break; }
-            if (kt + 1 < n_kt && !qk(kt + 1, 1)) { fail(p, aborted); break; }
+        // Then, per query tile and K/V tile: O_t += P_t(kt) V(kt) (A from TMEM, 16
+        // slots = 8 columns per k-step) and S_t(kt+1).  The two tiles are served in
+        // the order their P arrives: the barriers are polled, never waited on, so a
+        // tile that runs ahead (by as much as the K / V rings allow) never holds up
+        // the other.  The K and V stages are released by the second tile's commit.
+        int np0 = 0, np1 = has_b ? 0 : n_kt;  // next P V of tile a / b
+        uint64_t t_last = globaltimer();
+        while (!aborted && (np0 < n_kt || np1 < n_kt)) {
+          bool progressed = false;
+#pragma unroll
+          for (int t = 0; t < 2; ++t) {
+            const int kt = t ? np1 : np0;
+            if (kt >= n_kt) continue;
+            const bool more = kt + 1 < n_kt;
+            const int v = kt & 1, s1 = (kt + 1) % kStagesF;
+            if (!mbar_test(&bar[F_PFULL0 + t], kt & 1) ||
+                !mbar_test(&bar[F_VFULL0 + v], (kt >> 1) & 1) ||
+                (more && !mbar_test(&bar[F_KFULL0 + s1], ((kt + 1) / kStagesF) & 1)))
+              continue;
+            tc_fence_after();
+            const uint32_t v_addr = sbase + F_OFF_V + v * kTileBytes;
+#pragma unroll
+            for (int ks = 0; ks < BN / 16; ++ks)
+              mma_bf16_ts(tmem + 256 + t * 128, tmem + t * 128 + ks * 8, mnmajor_desc(v_addr, ks),
+                          IDESC_TS_PV, (kt > 0 || ks > 0) ? 1u : 0u);
+            // the other tile has issued its P V(kt) and S(kt+1) already
+            const bool second = (t ? np0 : np1) > kt;
+            if (second) mma_commit(&bar[F_VEMPTY0 + v]);  // V(kt) no longer read
+            if (more) {
+              const uint32_t k_addr = sbase + F_OFF_K + s1 * kTileBytes;
+              const uint32_t q_addr = t ? qb_addr : qa_addr;
+#pragma unroll
+              for (int ks = 0; ks < D / 16; ++ks)
+                mma_bf16_ss(tmem + t * 128, kmajor_desc(q_addr, ks), kmajor_desc(k_addr, ks),
+                            IDESC_K_MAJOR, ks > 0);
+              mma_commit(&bar[F_SFULL0 + t]);
+              if (second) mma_commit(&bar[F_KEMPTY0 + s1]);  // K(kt+1) no longer read
+            }
+            if (t) np1 = kt + 1; else np0 = kt + 1;
+            progressed = true;
           }
+          const uint64_t now = globaltimer();
+          if (progressed) t_last = now;
+          else if (now - t_last > lim) fail(p, aborted);
         }
         mma_commit(&bar[F_OFULL]);
         mma_commit(&bar[F_DRAIN]);
@@ -1424,6 +1473,31 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
         }
         tile_positions(rel_s + s * BN, tpg, kt, p.N_C, p.P, lane);
+        __syncwarp();
+        {
+          // slots invisible to the first row of a tile, compacted in slot order
+          const float thr = (float)min(i0_a, i0_b);
+          int32_t *cand = reinterpret_cast<int32_t *>(smem + F_OFF_CAND) + s * kCandWords;
+          int total = 0;
+#pragma unroll 1
+          for (int q = 0; q < 4; ++q)
+            total += __popc(__ballot_sync(0xffffffffu, rel_s[s * BN + lane + 32 * q] > thr));
+          if (total <= kMaxCand) {
+            int off = 0;
+#pragma unroll 1
+            for (int q = 0; q < 4; ++q) {
+              const float rq = rel_s[s * BN + lane + 32 * q];
+              const uint32_t bq = __ballot_sync(0xffffffffu, rq > thr);
+              if ((bq >> lane) & 1u) {
+                const int idx = off + __popc(bq & ((1u << lane) - 1u));
+                cand[2 + 2 * idx] = lane + 32 * q;
+                cand[3 + 2 * idx] = __float_as_int(rq);
+              }
+              off += __popc(bq);
+            }
+          }
+          if (lane == 0) cand[0] = total <= kMaxCand ? total : -1;
+        }
         __syncwarp();
         if (lane == 0) mbar_arrive(&bar[F_KFULL0 + s]);
         issued = kt + 1;
@@ -1476,18 +1550,43 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (!warp_wait(&bar[F_KFULL0 + s], (kt / kStagesF) & 1, lim)) { fail(p, aborted); break; }
         tc_fence_after();
         const float *rel = rel_s + s * BN;
-        const float rv = fmax3(fmaxf(rel[lane], rel[lane + 32]), rel[lane + 64], rel[lane + 96]);
-        const bool masked = __any_sync(0xffffffffu, rv > (float)i0);
+        const int32_t *cand = reinterpret_cast<const int32_t *>(smem + F_OFF_CAND) + s * kCandWords;
+        const int nc = cand[0];
+        if (nc > 0) {
+          // few slots to mask: lower them in TMEM before the row is read (a masked
+          // logit drops by 2^30 in base-2 units, as in row_mask)
+          const float ri = (float)(i0 + st);
+#pragma unroll 1
+          for (int q0 = 0; q0 < nc; q0 += 4) {
+            uint32_t cv[4];
+#pragma unroll
+            for (int q = 0; q < 4; ++q)
+              if (q0 + q < nc) cv[q] = tmem_ld1(s_col + cand[2 + 2 * (q0 + q)]);
+            tmem_wait_ld();
+#pragma unroll
+            for (int q = 0; q < 4; ++q)
+              if (q0 + q < nc) {
+                const float nm = fma_sat(__int_as_float(cand[3 + 2 * (q0 + q)]), 1.f, -ri);
+                tmem_st1(s_col + cand[2 + 2 * (q0 + q)],
+                         __float_as_uint(fmaf(nm, -mbias, __uint_as_float(cv[q]))));
+              }
+          }
+          tmem_wait_st();
+        }
+        const bool masked = nc < 0;  // too many: mask the whole row after reading it
         tmem_ld32(s_col, *reinterpret_cast<uint32_t(*)[32]>(x));
         tmem_ld32(s_col + 32, *reinterpret_cast<uint32_t(*)[32]>(x + 32));
         tmem_ld32(s_col + 64, *reinterpret_cast<uint32_t(*)[32]>(x + 64));
         tmem_ld32(s_col + 96, *reinterpret_cast<uint32_t(*)[32]>(x + 96));
         tmem_wait_ld();
         if (masked) row_mask<BN>(x, rel, (float)(i0 + st), mbias);
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&bar[F_KEMPTY0 + s]);
-        // the reference maximum follows the row maximum lazily: p <= 2^8 in between
+        // Probabilities against the reference maximum m, computed alongside the row
+        // maximum.  m follows the row maximum lazily (p <= 2^8 in between); when the
+        // maximum exceeds it by more than that (the first tile; rarely later) m moves,
+        // O and l are rescaled and the tile is done again from S, still in TMEM.
+        uint32_t pk[BN / 2];
         const float mx = row_max<BN>(x) * c2;
+        float ps = row_probs(x, c2, m, pk);
         const bool need = mx > m + kLazyMax;
         if (__any_sync(0xffffffffu, need)) {
           const float m_new = need ? mx : m;
@@ -1507,29 +1606,20 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
           }
           m = m_new;
+          tmem_ld32(s_col, *reinterpret_cast<uint32_t(*)[32]>(x));
+          tmem_ld32(s_col + 32, *reinterpret_cast<uint32_t(*)[32]>(x + 32));
+          tmem_ld32(s_col + 64, *reinterpret_cast<uint32_t(*)[32]>(x + 64));
+          tmem_ld32(s_col + 96, *reinterpret_cast<uint32_t(*)[32]>(x + 96));
+          tmem_wait_ld();
+          if (masked) row_mask<BN>(x, rel, (float)(i0 + st), mbias);
+          ps = row_probs(x, c2, m, pk);
         }
-        // probabilities against the reference maximum, packed to bf16 pairs over S
-        const float2 c2v = make_float2(c2, c2), negm = make_float2(-m, -m);
-        float2 acc[4];
-#pragma unroll
-        for (int q = 0; q < 4; ++q) acc[q] = make_float2(0.f, 0.f);
-#pragma unroll
-        for (int h = 0; h < 2; ++h) {
-          uint32_t pk[32];
-#pragma unroll
-          for (int e = 0; e < 64; e += 2) {
-            const int ee = 64 * h + e;
-            const float2 a =
-                fma2(make_float2(__uint_as_float(x[ee]), __uint_as_float(x[ee + 1])), c2v, negm);
-            const float2 v = make_float2(ex2(a.x), ex2(a.y));
-            acc[(e >> 1) & 3] = add2(acc[(e >> 1) & 3], v);
-            pk[e >> 1] = pack_bf16x2(v.x, v.y);
-          }
-          tmem_st32(s_col + 32 * h, pk);
-        }
-        const float2 s01 = add2(acc[0], acc[1]), s23 = add2(acc[2], acc[3]);
-        const float2 s4 = add2(s01, s23);
-        l += s4.x + s4.y;
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&bar[F_KEMPTY0 + s]);  // positions no longer read
+        // P over S (bf16 pairs), the A operand of O += P V
+        tmem_st32(s_col, *reinterpret_cast<uint32_t(*)[32]>(pk));
+        tmem_st32(s_col + 32, *reinterpret_cast<uint32_t(*)[32]>(pk + 32));
+        l += ps;
         tmem_wait_st();
         tc_fence_before();
         __syncwarp();
@@ -1573,12 +1663,11 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
 }
 
-// Pass 2 shared memory: Q_a, Q_b, the K ring, slot positions, -lse2 of both tiles.
+// Pass 2 shared memory: Q_a, Q_b, the K ring, -lse2 of both tiles.
 constexpr uint32_t S_OFF_QA = 0;
 constexpr uint32_t S_OFF_QB = kTileBytes;
 constexpr uint32_t S_OFF_K = 2 * kTileBytes;                   // [kStagesS] K tiles
-constexpr uint32_t S_OFF_REL = S_OFF_K + kStagesS * kTileBytes;  // float [kStagesS][BN]
-constexpr uint32_t S_OFF_NLSE = S_OFF_REL + kStagesS * BN * 4;   // float [2][BM]
+constexpr uint32_t S_OFF_NLSE = S_OFF_K + kStagesS * kTileBytes;  // float [2][BM]
 constexpr uint32_t S_OFF_BAR = S_OFF_NLSE + 2 * BM * 4;
 enum {
   G_Q = 0,
@@ -1592,9 +1681,11 @@ constexpr uint32_t kSmemS = S_OFF_TMEM + 16;
 static_assert(kSmemS <= 232448, "pass 2 shared memory budget");
 
 // Sum over the rows of one tile of the normalised probabilities of one slot:
-// sum_r 2^(c2 s_r - lse2_r) over visible rows r (rmin <= r < rmax).
+// sum_r 2^(c2 s_r - lse2_r) over visible rows r (rmin <= r < rmax).  MASK = false:
+// every row visible (rmin = 0, rmax = BM).
+template <bool MASK>
 __device__ __forceinline__ float slot_colsum(const uint32_t (&r)[BM], const float *nlse, float c2,
-                                             int rmin, int rmax, bool full) {
+                                             int rmin, int rmax) {
   const float rminf = (float)rmin;
   const float2 c2v = make_float2(c2, c2);
   float2 acc[4];
@@ -1604,12 +1695,12 @@ __device__ __forceinline__ float slot_colsum(const uint32_t (&r)[BM], const floa
   for (int e = 0; e < BM; e += 2) {
     const float2 nl = *reinterpret_cast<const float2 *>(nlse + e);
     float2 a = fma2(make_float2(__uint_as_float(r[e]), __uint_as_float(r[e + 1])), c2v, nl);
-    if (!full) {  // rows before rmin are masked: nm = sat(rmin - row) is 1 there
+    if constexpr (MASK) {  // rows before rmin are masked: nm = sat(rmin - row) is 1 there
       const float2 nm = make_float2(fma_sat(rminf, 1.f, -(float)e), fma_sat(rminf, 1.f, -(float)(e + 1)));
       a = fma2(nm, make_float2(-kMaskBias, -kMaskBias), a);
     }
     float2 v = make_float2(ex2(a.x), ex2(a.y));
-    if (rmax < BM) {  // rows past the chunk (last row tile only)
+    if constexpr (MASK) {  // rows past the chunk (last row tile only)
       v.x = e < rmax ? v.x : 0.f;
       v.y = e + 1 < rmax ? v.y : 0.f;
     }
@@ -1629,7 +1720,6 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (threadIdx.x == 0) atomicExch(p.status, H2OKV_ERR_CUDA);
     return;
   }
-  float *rel_s = reinterpret_cast<float *>(smem + S_OFF_REL);
   float *nlse_s = reinterpret_cast<float *>(smem + S_OFF_NLSE);
   uint64_t *bar = reinterpret_cast<uint64_t *>(smem + S_OFF_BAR);
   uint32_t *tmem_s = reinterpret_cast<uint32_t *>(smem + S_OFF_TMEM);
@@ -1651,7 +1741,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     mbar_init(&bar[G_Q], 1);
     for (int i = 0; i < kStagesS; ++i) {
       mbar_init(&bar[G_KFULL0 + i], 1);
-      mbar_init(&bar[G_KEMPTY0 + i], 1 + 4 * nwg);
+      mbar_init(&bar[G_KEMPTY0 + i], 1);  // the MMA's commit
     }
     for (int i = 0; i < 2; ++i) {
       mbar_init(&bar[G_SFULL0 + i], 1);
@@ -1721,7 +1811,6 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         mbar_arrive(&bar[G_Q]);
       }
-      const int32_t *tpg = p.token_pos + (size_t)bg * p.N_C;
       int issued = 0;
       for (int kt = 0; kt < n_kt && !aborted; ++kt) {
         const int s = kt % kStagesS, n = kt / kStagesS;
@@ -1735,10 +1824,8 @@ __global__ void __launch_bounds__(kThreads, 1)
             tma_prefetch_l2_3d(&k_map, 0, (kt + kPrefetch) * BN, bg);
             tma_prefetch_l2_3d(&k_map, 64, (kt + kPrefetch) * BN, bg);
           }
+          mbar_arrive(&bar[G_KFULL0 + s]);
         }
-        tile_positions(rel_s + s * BN, tpg, kt, p.N_C, p.P, lane);
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&bar[G_KFULL0 + s]);
         issued = kt + 1;
       }
       if (lane == 0) {
@@ -1761,26 +1848,31 @@ __global__ void __launch_bounds__(kThreads, 1)
       named_bar_sync(1 + t, 128);
       const int rmax = min(BM, p.S - i0);
       float *pw = p.part_w + ((size_t)bhq * p.tiles + tt) * p.N_C;
+      // each slot's token position, read one K tile ahead (empty / outside slots: far)
+      const int32_t *tpg = p.token_pos + (size_t)bg * p.N_C;
+      int32_t tp_next = st < p.N_C ? tpg[st] : kEmptyPos;
       for (int kt = 0; kt < n_kt && !aborted; ++kt) {
-        const int s = kt % kStagesS, u = kt & 1;
+        const int u = kt & 1;
         const int j = kt * BN + st;
+        const int32_t tp = tp_next;
+        if (kt + 1 < n_kt) tp_next = j + BN < p.N_C ? tpg[j + BN] : kEmptyPos;
         if (!warp_wait(&bar[G_SFULL0 + u], (kt >> 1) & 1, lim)) { fail(p, aborted); break; }
-        if (!warp_wait(&bar[G_KFULL0 + s], (kt / kStagesS) & 1, lim)) { fail(p, aborted); break; }
         tc_fence_after();
-        const float relj = rel_s[s * BN + st];
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&bar[G_KEMPTY0 + s]);
-        // visible rows r of this tile: relj <= i0 + r, r < rmax
-        const float rmf = fminf(fmaxf(relj - (float)i0, 0.f), (float)BM);
-        const int rmin = (int)rmf;
-        const bool full = __all_sync(0xffffffffu, rmin == 0 && rmax == BM);
+        // visible rows r of this tile: tp - P <= i0 + r, r < rmax.  A slot that no row
+        // of the tile sees (a later token of the chunk, an empty slot) sums to 0 and
+        // needs no masking; only slots first seen inside the tile do.
+        const int64_t rel = (int64_t)tp - (int64_t)p.P - (int64_t)i0;
+        const int rmin = rel <= 0 ? 0 : (rel >= BM ? BM : (int)rel);
+        const bool none = rmin >= rmax;
+        const bool full = __all_sync(0xffffffffu, (rmin == 0 || none) && rmax == BM);
         uint32_t r[BM];
         tmem_ld128(tmem + lane_base + u * 256 + t * 128, r);
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(&bar[G_SFREE0 + u]);
-        const float cs = slot_colsum(r, nl, c2, rmin, rmax, full);
-        if (j < p.N_C) pw[j] = cs;
+        const float cs = full ? slot_colsum<false>(r, nl, c2, 0, BM)
+                              : slot_colsum<true>(r, nl, c2, rmin, rmax);
+        if (j < p.N_C) pw[j] = none ? 0.f : cs;
       }
       tc_fence_before();
     }
@@ -2428,11 +2520,16 @@ __global__ void __launch_bounds__(256)
 __global__ void __launch_bounds__(256)
     reduce_w_kernel(const float *__restrict__ part_w, float *__restrict__ w,
                     float *__restrict__ wq, int Hq, int Hk, int q_g, int N_C, int tiles,
-                    int tiles_used) {
+                    int tiles_used, int n_cols) {
   const int bg = blockIdx.y;
   const int j = blockIdx.x * blockDim.x + threadIdx.x;
   if (j >= N_C) return;
   const int b = bg / Hk, g = bg - b * Hk;
+  if (j >= n_cols) {  // slots past the scanned span are empty: no weight
+    for (int hl = 0; hl < q_g && wq; ++hl) wq[(size_t)(b * Hq + g * q_g + hl) * N_C + j] = 0.f;
+    w[(size_t)bg * N_C + j] = 0.f;
+    return;
+  }
   float tot = 0.f;
   for (int hl = 0; hl < q_g; ++hl) {
     const int bhq = b * Hq + g * q_g + hl;
@@ -2659,6 +2756,7 @@ int launch_attn_tc(h2okv_cache *c, const void *q, int S, int64_t P, void *y, flo
   prm.P = (int)P;
   prm.tiles = (S + BM - 1) / BM;
   prm.n_kt = (d.capacity + BN - 1) / BN;
+  int n_cols = d.capacity;  // slots whose weights the kernels write
   prm.ctas_per_group = (prm.q_g * prm.tiles + 1) / 2;
   prm.scale2 = (float)(1.4426950408889634 / 11.313708498984761);  // log2(e) / sqrt(128)
   prm.timeout_ns = c->wait_timeout_ns;
@@ -2693,9 +2791,13 @@ int launch_attn_tc(h2okv_cache *c, const void *q, int S, int64_t P, void *y, flo
     if (rc) return rc;
     dim3 rgrid((d.capacity + 255) / 256, d.batch * d.n_kv_heads);
     reduce_w_kernel<<<rgrid, 256, 0, st>>>(prm.part_w, w, wq, d.n_q_heads, d.n_kv_heads, prm.q_g,
-                                           d.capacity, prm.tiles, prm.tiles);
+                                           d.capacity, prm.tiles, prm.tiles, n_cols);
     return check_launch("reduce_w_kernel");
   }
+  // outside the split schedule the kernels scan only the K/V tiles that may hold an
+  // occupied slot (the cache fills left to right)
+  prm.n_kt = (max(c->n_span, 1) + BN - 1) / BN;
+  n_cols = min(d.capacity, prm.n_kt * BN);
   if (d.kv_dtype == H2OKV_BF16 && c->tc.two_pass) {
     // attention with an online softmax, then the score sums against the final LSE
     static thread_local int ready_f = -1, ready_s = -1;
@@ -2711,7 +2813,7 @@ int launch_attn_tc(h2okv_cache *c, const void *q, int S, int64_t P, void *y, flo
     if (rc) return rc;
     dim3 rgrid((d.capacity + 255) / 256, d.batch * d.n_kv_heads);
     reduce_w_kernel<<<rgrid, 256, 0, st>>>(prm.part_w, w, wq, d.n_q_heads, d.n_kv_heads, prm.q_g,
-                                           d.capacity, prm.tiles, prm.tiles);
+                                           d.capacity, prm.tiles, prm.tiles, n_cols);
     return check_launch("reduce_w_kernel");
   }
   switch (d.kv_dtype) {
@@ -2723,7 +2825,7 @@ int launch_attn_tc(h2okv_cache *c, const void *q, int S, int64_t P, void *y, flo
   if (rc) return rc;
   dim3 rgrid((d.capacity + 255) / 256, d.batch * d.n_kv_heads);
   reduce_w_kernel<<<rgrid, 256, 0, st>>>(prm.part_w, w, wq, d.n_q_heads, d.n_kv_heads, prm.q_g,
-                                         d.capacity, prm.tiles, prm.tiles);
+                                         d.capacity, prm.tiles, prm.tiles, n_cols);
   return check_launch("reduce_w_kernel");
 }
 

@@ -44,6 +44,7 @@ struct h2okv_cache {
   h2okv_cache_desc desc;
   h2okv_cache_buffers bufs;
   int32_t n_filled;
+  int32_t n_span;  // every slot at or past this index is empty (the attention scans [0, n_span))
   size_t row_bytes;  // bytes of one stored key/value row
   h2okv::WorkspaceLayout ws;
   h2okv::TcPlan tc;

@@ -125,7 +125,10 @@ H2OKV_API int kv_cache_destroy(h2okv_cache *cache);
 
 /* Fill level bookkeeping: the number of occupied slots.  The library keeps it
  * on the host; set it after writing a cache state into the buffers directly
- * (occupied slots must then be exactly those with token_pos != INT32_MAX). */
+ * (occupied slots must then be exactly those with token_pos != INT32_MAX).
+ * While the eviction policy fills the cache left to right the attention scans
+ * only the slots filled so far; kv_cache_set_fill and h2o_insert_at make it
+ * scan every slot from then on (until kv_cache_reset). */
 H2OKV_API int kv_cache_get_fill(const h2okv_cache *cache, int32_t *n_filled);
 H2OKV_API int kv_cache_set_fill(h2okv_cache *cache, int32_t n_filled);
 
