@@ -1667,13 +1667,15 @@ __global__ void __launch_bounds__(kThreads, 1)
 constexpr uint32_t S_OFF_QA = 0;
 constexpr uint32_t S_OFF_QB = kTileBytes;
 constexpr uint32_t S_OFF_K = 2 * kTileBytes;                   // [kStagesS] K tiles
-constexpr uint32_t S_OFF_NLSE = S_OFF_K + kStagesS * kTileBytes;  // float [2][BM]
-constexpr uint32_t S_OFF_BAR = S_OFF_NLSE + 2 * BM * 4;
+constexpr uint32_t S_OFF_NLSE = S_OFF_K + kStagesS * kTileBytes;  // float [2 segments][2][BM]
+constexpr uint32_t S_OFF_BAR = S_OFF_NLSE + 4 * BM * 4;
 enum {
   G_Q = 0,
   G_KFULL0, G_KEMPTY0 = G_KFULL0 + kStagesS,
   G_SFULL0 = G_KEMPTY0 + kStagesS, G_SFREE0 = G_SFULL0 + 2,  // S^T pair, double buffered
-  G_DRAIN = G_SFREE0 + 2,
+  G_QFREE = G_SFREE0 + 2,                                     // Q of a segment no longer read
+  G_NL0,                                                      // -lse2 of tile a / b written
+  G_DRAIN = G_NL0 + 2,
   G_END
 };
 constexpr uint32_t S_OFF_TMEM = S_OFF_BAR + G_END * 8;
@@ -1683,8 +1685,8 @@ static_assert(kSmemS <= 232448, "pass 2 shared memory budget");
 // Sum over the rows of one tile of the normalised probabilities of one slot:
 // sum_r 2^(c2 s_r - lse2_r) over visible rows r (rmin <= r < rmax).  MASK = false:
 // every row visible (rmin = 0, rmax = BM).
-template <bool MASK>
-__device__ __forceinline__ float slot_colsum(const uint32_t (&r)[BM], const float *nlse, float c2,
+template <bool MASK, int N>
+__device__ __forceinline__ float slot_colsum(const uint32_t (&r)[N], const float *nlse, float c2,
                                              int rmin, int rmax) {
   const float rminf = (float)rmin;
   const float2 c2v = make_float2(c2, c2);
@@ -1692,7 +1694,7 @@ __device__ __forceinline__ float slot_colsum(const uint32_t (&r)[BM], const floa
 #pragma unroll
   for (int q = 0; q < 4; ++q) acc[q] = make_float2(0.f, 0.f);
 #pragma unroll
-  for (int e = 0; e < BM; e += 2) {
+  for (int e = 0; e < N; e += 2) {
     const float2 nl = *reinterpret_cast<const float2 *>(nlse + e);
     float2 a = fma2(make_float2(__uint_as_float(r[e]), __uint_as_float(r[e + 1])), c2v, nl);
     if constexpr (MASK) {  // rows before rmin are masked: nm = sat(rmin - row) is 1 there
@@ -1709,179 +1711,6 @@ __device__ __forceinline__ float slot_colsum(const uint32_t (&r)[BM], const floa
   const float2 s01 = add2(acc[0], acc[1]), s23 = add2(acc[2], acc[3]);
   const float2 s4 = add2(s01, s23);
   return s4.x + s4.y;
-}
-
-__global__ void __launch_bounds__(kThreads, 1)
-    scoresum_kernel(const __grid_constant__ CUtensorMap q_map,
-                    const __grid_constant__ CUtensorMap k_map, const TcParams p) {
-  extern __shared__ __align__(1024) uint8_t smem[];
-  const uint32_t sbase = smem_u32(smem);
-  if (sbase & 1023u) {
-    if (threadIdx.x == 0) atomicExch(p.status, H2OKV_ERR_CUDA);
-    return;
-  }
-  float *nlse_s = reinterpret_cast<float *>(smem + S_OFF_NLSE);
-  uint64_t *bar = reinterpret_cast<uint64_t *>(smem + S_OFF_BAR);
-  uint32_t *tmem_s = reinterpret_cast<uint32_t *>(smem + S_OFF_TMEM);
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int bg = blockIdx.x / p.ctas_per_group;
-  const int c = blockIdx.x - bg * p.ctas_per_group;
-  const int b = bg / p.Hk, g = bg - b * p.Hk;
-  const int n_qt = p.q_g * p.tiles;
-  const int qa = 2 * c, qb = 2 * c + 1;
-  const bool has_b = qb < n_qt;
-  const int hl_a = qa / p.tiles, t_a = qa - hl_a * p.tiles;
-  const int hl_b = has_b ? qb / p.tiles : hl_a, t_b = has_b ? qb - hl_b * p.tiles : t_a;
-  const int bhq_a = b * p.Hq + g * p.q_g + hl_a, bhq_b = b * p.Hq + g * p.q_g + hl_b;
-  const int i0_a = t_a * BM, i0_b = t_b * BM;
-  const int n_kt = p.n_kt;
-  const uint64_t lim = p.timeout_ns;
-  const int nwg = has_b ? 2 : 1;
-  if (threadIdx.x == 0) {
-    mbar_init(&bar[G_Q], 1);
-    for (int i = 0; i < kStagesS; ++i) {
-      mbar_init(&bar[G_KFULL0 + i], 1);
-      mbar_init(&bar[G_KEMPTY0 + i], 1);  // the MMA's commit
-    }
-    for (int i = 0; i < 2; ++i) {
-      mbar_init(&bar[G_SFULL0 + i], 1);
-      mbar_init(&bar[G_SFREE0 + i], 4 * nwg);
-    }
-    mbar_init(&bar[G_DRAIN], 1);
-    fence_mbar_init();
-  }
-  if (warp == 1) {
-    tmem_alloc(tmem_s, kTmemCols);
-    tmem_relinquish();
-    tc_fence_before();
-  }
-  if (warp == 0 && lane == 0) {
-    prefetch_tensormap(&q_map);
-    prefetch_tensormap(&k_map);
-  }
-  __syncthreads();
-  tc_fence_after();
-  const uint32_t tmem = *tmem_s;
-  bool aborted = false;
-
-  if (warp < 4) {
-    reg_dealloc<kCtrlRegs>();
-    if (warp == 1) {
-      // ------------------------------------------------------------------ MMA issuer
-      // S^T_t(kt) = K(kt) Q_t^T into columns 256 (kt & 1) + 128 t
-      if (lane == 0) {
-        const uint32_t qa_addr = sbase + S_OFF_QA, qb_addr = sbase + S_OFF_QB;
-        if (!mbar_wait(&bar[G_Q], 0, lim)) fail(p, aborted);
-        tc_fence_after();
-        for (int kt = 0; kt < n_kt && !aborted; ++kt) {
-          const int s = kt % kStagesS, u = kt & 1;
-          if (!mbar_wait(&bar[G_KFULL0 + s], (kt / kStagesS) & 1, lim)) { fail(p, aborted); break; }
-          if (kt >= 2 && !mbar_wait(&bar[G_SFREE0 + u], ((kt >> 1) - 1) & 1, lim)) {
-            fail(p, aborted);
-            break;
-          }
-          tc_fence_after();
-          const uint32_t k_addr = sbase + S_OFF_K + s * kTileBytes;
-#pragma unroll
-          for (int ks = 0; ks < D / 16; ++ks)
-            mma_bf16_ss(tmem + u * 256, kmajor_desc(k_addr, ks), kmajor_desc(qa_addr, ks),
-                        IDESC_K_MAJOR, ks > 0);
-          if (has_b) {
-#pragma unroll
-            for (int ks = 0; ks < D / 16; ++ks)
-              mma_bf16_ss(tmem + u * 256 + 128, kmajor_desc(k_addr, ks), kmajor_desc(qb_addr, ks),
-                          IDESC_K_MAJOR, ks > 0);
-          }
-          mma_commit(&bar[G_SFULL0 + u]);
-          mma_commit(&bar[G_KEMPTY0 + s]);
-        }
-        mma_commit(&bar[G_DRAIN]);
-        mbar_wait(&bar[G_DRAIN], 0, 4000000000ull);
-      }
-      __syncwarp();
-    } else if (warp == 0) {
-      // ----------------------------------------- producer of Q, K and slot positions
-      if (lane == 0) {
-        mbar_expect_tx(&bar[G_Q], has_b ? 2 * kTileBytes : kTileBytes);
-        tma_load_3d(smem + S_OFF_QA, &q_map, &bar[G_Q], 0, i0_a, bhq_a);
-        tma_load_3d(smem + S_OFF_QA + kHalfBytes, &q_map, &bar[G_Q], 64, i0_a, bhq_a);
-        if (has_b) {
-          tma_load_3d(smem + S_OFF_QB, &q_map, &bar[G_Q], 0, i0_b, bhq_b);
-          tma_load_3d(smem + S_OFF_QB + kHalfBytes, &q_map, &bar[G_Q], 64, i0_b, bhq_b);
-        }
-        mbar_arrive(&bar[G_Q]);
-      }
-      int issued = 0;
-      for (int kt = 0; kt < n_kt && !aborted; ++kt) {
-        const int s = kt % kStagesS, n = kt / kStagesS;
-        if (n > 0 && !warp_wait(&bar[G_KEMPTY0 + s], (n - 1) & 1, lim)) { fail(p, aborted); break; }
-        uint8_t *kdst = smem + S_OFF_K + s * kTileBytes;
-        if (lane == 0) {
-          mbar_expect_tx(&bar[G_KFULL0 + s], kTileBytes);
-          tma_load_3d(kdst, &k_map, &bar[G_KFULL0 + s], 0, kt * BN, bg);
-          tma_load_3d(kdst + kHalfBytes, &k_map, &bar[G_KFULL0 + s], 64, kt * BN, bg);
-          if (kt + kPrefetch < n_kt) {
-            tma_prefetch_l2_3d(&k_map, 0, (kt + kPrefetch) * BN, bg);
-            tma_prefetch_l2_3d(&k_map, 64, (kt + kPrefetch) * BN, bg);
-          }
-          mbar_arrive(&bar[G_KFULL0 + s]);
-        }
-        issued = kt + 1;
-      }
-      if (lane == 0) {
-        mbar_wait(&bar[G_Q], 0, 4000000000ull);
-        for (int kt = issued - 1; kt >= 0 && kt >= issued - kStagesS; --kt)
-          mbar_wait(&bar[G_KFULL0 + kt % kStagesS], (kt / kStagesS) & 1, 4000000000ull);
-      }
-    }
-  } else {
-    reg_alloc<kSoftRegs>();
-    const int t = (warp - 4) >> 2;
-    if (t == 0 || has_b) {
-      // ------------------------------------- column sums, one thread per slot of a tile
-      const int st = threadIdx.x - 128 * (1 + t);
-      const uint32_t lane_base = (uint32_t)(32 * (warp & 3)) << 16;
-      const float c2 = p.scale2;
-      const int i0 = t ? i0_b : i0_a, bhq = t ? bhq_b : bhq_a, tt = t ? t_b : t_a;
-      float *nl = nlse_s + t * BM;
-      nl[st] = p.nlse[((size_t)bhq * p.tiles + tt) * BM + st];
-      named_bar_sync(1 + t, 128);
-      const int rmax = min(BM, p.S - i0);
-      float *pw = p.part_w + ((size_t)bhq * p.tiles + tt) * p.N_C;
-      // each slot's token position, read one K tile ahead (empty / outside slots: far)
-      const int32_t *tpg = p.token_pos + (size_t)bg * p.N_C;
-      int32_t tp_next = st < p.N_C ? tpg[st] : kEmptyPos;
-      for (int kt = 0; kt < n_kt && !aborted; ++kt) {
-        const int u = kt & 1;
-        const int j = kt * BN + st;
-        const int32_t tp = tp_next;
-        if (kt + 1 < n_kt) tp_next = j + BN < p.N_C ? tpg[j + BN] : kEmptyPos;
-        if (!warp_wait(&bar[G_SFULL0 + u], (kt >> 1) & 1, lim)) { fail(p, aborted); break; }
-        tc_fence_after();
-        // visible rows r of this tile: tp - P <= i0 + r, r < rmax.  A slot that no row
-        // of the tile sees (a later token of the chunk, an empty slot) sums to 0 and
-        // needs no masking; only slots first seen inside the tile do.
-        const int64_t rel = (int64_t)tp - (int64_t)p.P - (int64_t)i0;
-        const int rmin = rel <= 0 ? 0 : (rel >= BM ? BM : (int)rel);
-        const bool none = rmin >= rmax;
-        const bool full = __all_sync(0xffffffffu, (rmin == 0 || none) && rmax == BM);
-        uint32_t r[BM];
-        tmem_ld128(tmem + lane_base + u * 256 + t * 128, r);
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&bar[G_SFREE0 + u]);
-        const float cs = full ? slot_colsum<false>(r, nl, c2, 0, BM)
-                              : slot_colsum<true>(r, nl, c2, rmin, rmax);
-        if (j < p.N_C) pw[j] = none ? 0.f : cs;
-      }
-      tc_fence_before();
-    }
-  }
-  __syncthreads();
-  if (warp == 1) {
-    tc_fence_after();
-    tmem_dealloc(tmem, kTmemCols);
-  }
 }
 
 // ---- split scheduling (bf16 cache): the two passes as persistent kernels ----------
@@ -1969,6 +1798,221 @@ __device__ __forceinline__ SegIter seg_iter(const SplitParams &sp) {
   return it;
 }
 // CTAs whose ranges hold units of pair p: [c_first, c_last]; segment slot of p in c.
+// Pass 2 over equal shares of the (pair, K tile) units: CTA c takes units
+// [U c / G, U (c + 1) / G) in segments of one pair each, so that all
+// SMs are busy whatever the number of pairs; each (row tile, slot) sum is written by
+// exactly one CTA.  With G = pairs every CTA takes one whole pair.
+__global__ void __launch_bounds__(kThreads, 1)
+    scoresum_kernel(const __grid_constant__ CUtensorMap q_map,
+                    const __grid_constant__ CUtensorMap k_map, const SplitParams sp) {
+  const TcParams &p = sp.t;
+  extern __shared__ __align__(1024) uint8_t smem[];
+  const uint32_t sbase = smem_u32(smem);
+  if (sbase & 1023u) {
+    if (threadIdx.x == 0) atomicExch(p.status, H2OKV_ERR_CUDA);
+    return;
+  }
+  float *nlse_s = reinterpret_cast<float *>(smem + S_OFF_NLSE);
+  uint64_t *bar = reinterpret_cast<uint64_t *>(smem + S_OFF_BAR);
+  uint32_t *tmem_s = reinterpret_cast<uint32_t *>(smem + S_OFF_TMEM);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int n_qt = p.q_g * p.tiles;
+  const uint64_t lim = p.timeout_ns;
+  if (threadIdx.x == 0) {
+    mbar_init(&bar[G_Q], 1);
+    for (int i = 0; i < kStagesS; ++i) {
+      mbar_init(&bar[G_KFULL0 + i], 1);
+      mbar_init(&bar[G_KEMPTY0 + i], 1);  // the MMA's commit
+    }
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&bar[G_SFULL0 + i], 1);
+      mbar_init(&bar[G_SFREE0 + i], 8);  // both softmax warpgroups, with or without a tile
+    }
+    mbar_init(&bar[G_QFREE], 1);
+    mbar_init(&bar[G_NL0], 4);
+    mbar_init(&bar[G_NL0 + 1], 4);
+    mbar_init(&bar[G_DRAIN], 1);
+    fence_mbar_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_s, kTmemCols);
+    tmem_relinquish();
+    tc_fence_before();
+  }
+  if (warp == 0 && lane == 0) {
+    prefetch_tensormap(&q_map);
+    prefetch_tensormap(&k_map);
+  }
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_s;
+  bool aborted = false;
+  // this CTA's units, in natural order (every K tile of pass 2 fits in L2)
+  const int n_kt = p.n_kt;
+  const int u_first = (int)((sp.U * blockIdx.x) / sp.G), u_last = (int)((sp.U * (blockIdx.x + 1)) / sp.G);
+  int pidx, kt0, kt1;
+  auto next = [&](int &u) -> bool {
+    if (u >= u_last) return false;
+    pidx = u / n_kt;
+    kt0 = u - pidx * n_kt;
+    kt1 = min(n_kt, kt0 + (u_last - u));
+    u += kt1 - kt0;
+    return true;
+  };
+
+  if (warp < 4) {
+    reg_dealloc<kCtrlRegs>();
+    if (warp == 1) {
+      // ------------------------------------------------------------------ MMA issuer
+      // S^T_t(i) = K Q_t^T of the CTA's i-th unit into columns 256 (i & 1) + 128 t
+      if (lane == 0) {
+        const uint32_t qa_addr = sbase + S_OFF_QA, qb_addr = sbase + S_OFF_QB;
+        int i = 0, seg = 0, u = u_first;
+        while (!aborted && next(u)) {
+          const bool has_b = 2 * (pidx % p.ctas_per_group) + 1 < n_qt;
+          if (!mbar_wait(&bar[G_Q], seg & 1, lim)) { fail(p, aborted); break; }
+          tc_fence_after();
+          for (int kt = kt0; kt < kt1 && !aborted; ++kt, ++i) {
+            const int s = i % kStagesS, u = i & 1;
+            if (!mbar_wait(&bar[G_KFULL0 + s], (i / kStagesS) & 1, lim)) { fail(p, aborted); break; }
+            if (i >= 2 && !mbar_wait(&bar[G_SFREE0 + u], ((i >> 1) - 1) & 1, lim)) {
+              fail(p, aborted);
+              break;
+            }
+            tc_fence_after();
+            const uint32_t k_addr = sbase + S_OFF_K + s * kTileBytes;
+#pragma unroll
+            for (int ks = 0; ks < D / 16; ++ks)
+              mma_bf16_ss(tmem + u * 256, kmajor_desc(k_addr, ks), kmajor_desc(qa_addr, ks),
+                          IDESC_K_MAJOR, ks > 0);
+            if (has_b) {
+#pragma unroll
+              for (int ks = 0; ks < D / 16; ++ks)
+                mma_bf16_ss(tmem + u * 256 + 128, kmajor_desc(k_addr, ks),
+                            kmajor_desc(qb_addr, ks), IDESC_K_MAJOR, ks > 0);
+            }
+            mma_commit(&bar[G_SFULL0 + u]);
+            mma_commit(&bar[G_KEMPTY0 + s]);
+          }
+          mma_commit(&bar[G_QFREE]);  // the segment's Q tiles no longer read
+          ++seg;
+        }
+        mma_commit(&bar[G_DRAIN]);
+        mbar_wait(&bar[G_DRAIN], 0, 4000000000ull);
+      }
+      __syncwarp();
+    } else if (warp == 0) {
+      // ---------------------------------------------- producer of Q (per segment) and K
+      if (lane == 0) {
+        int i = 0, seg = 0, u = u_first;
+        while (!aborted && next(u)) {
+          const PairInfo pi = pair_info(pidx, p);
+          const bool has_b = 2 * (pidx % p.ctas_per_group) + 1 < n_qt;
+          if (seg > 0 && !mbar_wait(&bar[G_QFREE], (seg - 1) & 1, lim)) { fail(p, aborted); break; }
+          mbar_expect_tx(&bar[G_Q], has_b ? 2 * kTileBytes : kTileBytes);
+          tma_load_3d(smem + S_OFF_QA, &q_map, &bar[G_Q], 0, pi.i0_a, pi.bhq_a);
+          tma_load_3d(smem + S_OFF_QA + kHalfBytes, &q_map, &bar[G_Q], 64, pi.i0_a, pi.bhq_a);
+          if (has_b) {
+            tma_load_3d(smem + S_OFF_QB, &q_map, &bar[G_Q], 0, pi.i0_b, pi.bhq_b);
+            tma_load_3d(smem + S_OFF_QB + kHalfBytes, &q_map, &bar[G_Q], 64, pi.i0_b, pi.bhq_b);
+          }
+          mbar_arrive(&bar[G_Q]);
+          for (int kt = kt0; kt < kt1 && !aborted; ++kt, ++i) {
+            const int s = i % kStagesS, n = i / kStagesS;
+            if (n > 0 && !mbar_wait(&bar[G_KEMPTY0 + s], (n - 1) & 1, lim)) { fail(p, aborted); break; }
+            uint8_t *kdst = smem + S_OFF_K + s * kTileBytes;
+            mbar_expect_tx(&bar[G_KFULL0 + s], kTileBytes);
+            tma_load_3d(kdst, &k_map, &bar[G_KFULL0 + s], 0, kt * BN, pi.bg);
+            tma_load_3d(kdst + kHalfBytes, &k_map, &bar[G_KFULL0 + s], 64, kt * BN, pi.bg);
+            if (kt + kPrefetch < kt1) {
+              tma_prefetch_l2_3d(&k_map, 0, (kt + kPrefetch) * BN, pi.bg);
+              tma_prefetch_l2_3d(&k_map, 64, (kt + kPrefetch) * BN, pi.bg);
+            }
+            mbar_arrive(&bar[G_KFULL0 + s]);
+          }
+          ++seg;
+        }
+        // drain: the last issued loads land before exit
+        if (seg > 0) mbar_wait(&bar[G_Q], (seg - 1) & 1, 4000000000ull);
+        for (int j = i - 1; j >= 0 && j >= i - kStagesS; --j)
+          mbar_wait(&bar[G_KFULL0 + j % kStagesS], (j / kStagesS) & 1, 4000000000ull);
+      }
+      __syncwarp();
+    }
+  } else {
+    reg_alloc<kSoftRegs>();
+    // ------------------------------------- column sums, one thread per slot of a tile
+    const int t = (warp - 4) >> 2;
+    const int st = threadIdx.x - 128 * (1 + t);
+    const uint32_t lane_base = (uint32_t)(32 * (warp & 3)) << 16;
+    const float c2 = p.scale2;
+    int i = 0, seg = 0, u = u_first;
+    while (!aborted && next(u)) {
+      const PairInfo pi = pair_info(pidx, p);
+      const bool active = t == 0 || 2 * (pidx % p.ctas_per_group) + 1 < n_qt;
+      const int i0 = t ? pi.i0_b : pi.i0_a, bhq = t ? pi.bhq_b : pi.bhq_a, tt = t ? pi.t_b : pi.t_a;
+      // -lse2 of the segment's rows, double buffered by segment: a warpgroup writes
+      // buffer seg & 1 only after all its threads have written (so finished reading)
+      // the other one
+      float *nl = nlse_s + ((seg & 1) * 2 + t) * BM;
+      if (active) nl[st] = p.nlse[((size_t)bhq * p.tiles + tt) * BM + st];
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&bar[G_NL0 + t]);
+      if (!warp_wait(&bar[G_NL0 + t], seg & 1, lim)) { fail(p, aborted); break; }
+      ++seg;
+      const int rmax = min(BM, p.S - i0);
+      float *pw = p.part_w + ((size_t)bhq * p.tiles + tt) * p.N_C;
+      // each slot's token position, read one K tile ahead (empty / outside slots: far)
+      const int32_t *tpg = p.token_pos + (size_t)pi.bg * p.N_C;
+      int32_t tp_next = kt0 * BN + st < p.N_C ? tpg[kt0 * BN + st] : kEmptyPos;
+      for (int kt = kt0; kt < kt1; ++kt, ++i) {
+        const int u = i & 1;
+        const int j = kt * BN + st;
+        const int32_t tp = tp_next;
+        if (kt + 1 < kt1) tp_next = j + BN < p.N_C ? tpg[j + BN] : kEmptyPos;
+        if (!warp_wait(&bar[G_SFULL0 + u], (i >> 1) & 1, lim)) { fail(p, aborted); break; }
+        tc_fence_after();
+        if (active) {
+          // visible rows r of this tile: tp - P <= i0 + r, r < rmax.  A slot that no row
+          // of the tile sees (a later token of the chunk, an empty slot) sums to 0 and
+          // needs no masking; only slots first seen inside the tile do.
+          const int64_t rel = (int64_t)tp - (int64_t)p.P - (int64_t)i0;
+          const int rmin = rel <= 0 ? 0 : (rel >= BM ? BM : (int)rel);
+          const bool none = rmin >= rmax;
+          const bool full = __all_sync(0xffffffffu, (rmin == 0 || none) && rmax == BM);
+          // the tile's 128 rows in two halves of 64 (fewer live registers)
+          const uint32_t ta = tmem + lane_base + u * 256 + t * 128;
+          float cs = 0.f;
+#pragma unroll
+          for (int h = 0; h < 2; ++h) {
+            uint32_t r[BM / 2];
+            tmem_ld32(ta + 64 * h, *reinterpret_cast<uint32_t(*)[32]>(r));
+            tmem_ld32(ta + 64 * h + 32, *reinterpret_cast<uint32_t(*)[32]>(r + 32));
+            tmem_wait_ld();
+            if (h == 1) {  // the S^T buffer is free once read
+              tc_fence_before();
+              __syncwarp();
+              if (lane == 0) mbar_arrive(&bar[G_SFREE0 + u]);
+            }
+            cs += full ? slot_colsum<false>(r, nl + 64 * h, c2, 0, BM / 2)
+                       : slot_colsum<true>(r, nl + 64 * h, c2, rmin - 64 * h, rmax - 64 * h);
+          }
+          if (j < p.N_C) pw[j] = none ? 0.f : cs;
+        } else {
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&bar[G_SFREE0 + u]);
+        }
+      }
+    }
+    tc_fence_before();
+  }
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, kTmemCols);
+  }
+}
+
 __device__ __forceinline__ int cta_of_unit(long long x, const SplitParams &sp) {
   // largest c with floor(U c / G) <= x
   return (int)(((x + 1) * sp.G + sp.U - 1) / sp.U) - 1;
@@ -2622,8 +2666,10 @@ void tc_plan(const h2okv_cache_desc &d, TcPlan *plan) {
   const char *fused = getenv("H2OKV_TC_FUSED");
   plan->two_pass = !(fused && fused[0] == '1');
   int dev = 0, sms = 0;
+  plan->sms = 0;
   if (plan->enabled && cudaGetDevice(&dev) == cudaSuccess &&
       cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) == cudaSuccess) {
+    plan->sms = sms;
     const SplitShape sh = split_shape(d, d.max_chunk, sms);
     if (sh.use) {
       plan->split_ctas = sms;
@@ -2808,7 +2854,12 @@ int launch_attn_tc(h2okv_cache *c, const void *q, int S, int64_t P, void *y, flo
     attn_fwd_kernel<<<grid, kThreads, kSmemF, st>>>(qmap, kmap, vmap, prm);
     rc = check_launch("attn_fwd_kernel");
     if (rc) return rc;
-    scoresum_kernel<<<grid, kThreads, kSmemS, st>>>(qmap, kmap, prm);
+    // the score sums over equal shares of (pair, K tile) units, one CTA per SM
+    SplitParams ss{};
+    ss.t = prm;
+    ss.U = (long long)grid * prm.n_kt;
+    ss.G = (int)min((long long)max(c->tc.sms, 1), ss.U);
+    scoresum_kernel<<<ss.G, kThreads, kSmemS, st>>>(qmap, kmap, ss);
     rc = check_launch("scoresum_kernel");
     if (rc) return rc;
     dim3 rgrid((d.capacity + 255) / 256, d.batch * d.n_kv_heads);

@@ -31,6 +31,7 @@ struct TcPlan {          // launch plan of the tensor-core path
   int split_ctas;        // CTAs of the split (persistent) kernels, 0 = split scheduling off
   int max_seg;           // segments per CTA the split workspace is sized for
   bool two_pass;         // bf16: attention pass + score-sum pass (else the fused kernel)
+  int sms;               // multiprocessors of the device (0 if unknown)
   bool maps_ready;       // k_map / v_map encoded
   alignas(64) unsigned char k_map[128];  // CUtensorMap over keys
   alignas(64) unsigned char v_map[128];  // CUtensorMap over values
