@@ -270,7 +270,18 @@ def run_ours(args, wl, ws, rank, local):
     n_split = sum(1 for c in range(wl.n_chunks) if split_schedule(wl, wl.chunk_len(c), sms))
     # bf16 caches outside the split schedule: attention pass + score-sum pass
     two_pass = tc_used and wl.kv_dtype == "bf16" and os.environ.get("H2OKV_TC_FUSED") != "1"
-    launches_per_step = wl.n_chunks * 3 + 2 * n_split + 2 + (wl.n_chunks - n_split if two_pass else 0)
+    # the two-pass path: attention, [combine of split pairs], score sums, reduction
+    pairs = wl.B * wl.Hk * ((wl.q_g * ((wl.chunk + 127) // 128) + 1) // 2)
+    if two_pass:
+        # pass 1 splits its scan (and a combine kernel merges the pieces) only when one
+        # CTA per pair leaves over a quarter of the SMs idle and the scan is long
+        fill = pairs / (((pairs + sms - 1) // sms) * sms)
+        n_combine = sum(1 for c in range(wl.n_chunks)
+                        if fill < 0.75 and -(-min(wl.capacity, (c + 1) * wl.chunk) // 128) >= 32)
+        n_split = 0
+        launches_per_step = wl.n_chunks * 4 + n_combine + 2
+    else:
+        launches_per_step = wl.n_chunks * 3 + 2 * n_split + 2
     per_launch_alg = at_flops_alg / len(at_ms)
     per_launch_ms = sum(at_ms) / len(at_ms)
     if tc_used:
@@ -279,7 +290,8 @@ def run_ours(args, wl, ws, rank, local):
                 "traffic": recorded_traffic("attn_fwd_kernel" if two_pass and n_split == 0 else "attn_tc_kernel"),
                 "kernel": ("attention call per chunk (attn_split_a_kernel + attn_split_b_kernel + "
                            "reduce_o_kernel + reduce_w_kernel)") if n_split == wl.n_chunks else
-                          (("attention call per chunk (attn_fwd_kernel + scoresum_kernel + reduce_w_kernel)"
+                          (("attention call per chunk (attn_fwd_kernel + %sscoresum_kernel + reduce_w_kernel)"
+                            % ("combine_fwd_kernel + " if n_combine else "")
                             if two_pass else "attention call per chunk (attn_tc_kernel + reduce_w_kernel)")
                            if n_split == 0 else
                            "attention call per chunk (split schedule on %d of %d chunks)" % (n_split, wl.n_chunks)),

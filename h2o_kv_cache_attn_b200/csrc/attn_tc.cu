@@ -1244,17 +1244,28 @@ constexpr uint32_t F_OFF_REL = F_OFF_V + 2 * kTileBytes;           // float [kSt
 constexpr int kMaxCand = 16;
 constexpr uint32_t F_OFF_CAND = F_OFF_REL + kStagesF * BN * 4;     // [kStagesF][1 + 2 kMaxCand]
 constexpr uint32_t kCandWords = 2 + 2 * kMaxCand;                  // count, pad, pairs
-constexpr uint32_t F_OFF_BAR = F_OFF_CAND + kStagesF * kCandWords * 4;
+// The CTA's segments (pair, first and end K/V tile, partial slot), listed once.
+constexpr int kMaxSegF = 15;
+constexpr uint32_t F_OFF_SEG = (F_OFF_CAND + kStagesF * kCandWords * 4 + 15) & ~15u;  // int4 [1 + kMaxSegF]
+static_assert(F_OFF_SEG % 16 == 0 && F_OFF_CAND % 16 == 0, "pass 1 shared memory alignment");
+constexpr uint32_t F_OFF_BAR = F_OFF_SEG + (1 + kMaxSegF) * 16;
 enum {
   F_Q = 0,
   F_KFULL0, F_KEMPTY0 = F_KFULL0 + kStagesF,   // K ring (+ slot positions)
   F_VFULL0 = F_KEMPTY0 + kStagesF, F_VEMPTY0 = F_VFULL0 + 2,  // V ring
   F_SFULL0 = F_VEMPTY0 + 2,                    // S of tile a / b written
   F_PFULL0 = F_SFULL0 + 2,                     // P of tile a / b written (O rescaled)
-  F_OFULL = F_PFULL0 + 2, F_DRAIN,
+  F_OFULL = F_PFULL0 + 2,                      // a segment's last P V done
+  F_OFREE,                                     // a segment's O read out by the softmax warps
+  F_QFREE,                                     // a segment's Q tiles no longer read
+  F_DRAIN,
   F_END
 };
 constexpr uint32_t F_OFF_TMEM = F_OFF_BAR + F_END * 8;
+// pass 1 register split: the softmax warps hold a row of logits and its packed
+// probabilities: 128 x 72 + 256 x 216 = 384 x 168
+constexpr int kCtrlRegsF = 72, kSoftRegsF = 216;
+static_assert(128 * kCtrlRegsF + 256 * kSoftRegsF == kThreads * kLaunchRegs, "pass 1 register split");
 constexpr uint32_t kSmemF = F_OFF_TMEM + 16;
 static_assert(kSmemF <= 232448, "pass 1 shared memory budget");
 // P (TMEM, K-major) x V (shared memory, MN-major)
@@ -1306,360 +1317,6 @@ __device__ __forceinline__ void tile_positions(float *dst, const int32_t *tpg, i
     const int64_t t = e < nv ? (int64_t)tpg[kt * BN + e] : (int64_t)kEmptyPos;
     const int64_t rel = t - (int64_t)P;
     dst[e] = (float)(rel < -1 ? -1 : (rel > kRelFar ? kRelFar : rel));
-  }
-}
-
-__global__ void __launch_bounds__(kThreads, 1)
-    attn_fwd_kernel(const __grid_constant__ CUtensorMap q_map,
-                    const __grid_constant__ CUtensorMap k_map,
-                    const __grid_constant__ CUtensorMap v_map, const TcParams p) {
-  extern __shared__ __align__(1024) uint8_t smem[];
-  const uint32_t sbase = smem_u32(smem);
-  if (sbase & 1023u) {
-    if (threadIdx.x == 0) atomicExch(p.status, H2OKV_ERR_CUDA);
-    return;
-  }
-  float *rel_s = reinterpret_cast<float *>(smem + F_OFF_REL);
-  uint64_t *bar = reinterpret_cast<uint64_t *>(smem + F_OFF_BAR);
-  uint32_t *tmem_s = reinterpret_cast<uint32_t *>(smem + F_OFF_TMEM);
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int bg = blockIdx.x / p.ctas_per_group;
-  const int c = blockIdx.x - bg * p.ctas_per_group;
-  const int b = bg / p.Hk, g = bg - b * p.Hk;
-  const int n_qt = p.q_g * p.tiles;
-  const int qa = 2 * c, qb = 2 * c + 1;
-  const bool has_b = qb < n_qt;
-  const int hl_a = qa / p.tiles, t_a = qa - hl_a * p.tiles;
-  const int hl_b = has_b ? qb / p.tiles : hl_a, t_b = has_b ? qb - hl_b * p.tiles : t_a;
-  const int bhq_a = b * p.Hq + g * p.q_g + hl_a, bhq_b = b * p.Hq + g * p.q_g + hl_b;
-  const int i0_a = t_a * BM, i0_b = t_b * BM;
-  const int n_kt = p.n_kt;
-  const uint64_t lim = p.timeout_ns;
-  const int nwg = has_b ? 2 : 1;
-  if (threadIdx.x == 0) {
-    mbar_init(&bar[F_Q], 1);
-    for (int i = 0; i < kStagesF; ++i) {
-      mbar_init(&bar[F_KFULL0 + i], 1);
-      mbar_init(&bar[F_KEMPTY0 + i], 1 + 4 * nwg);  // MMA commit + softmax warps (positions)
-    }
-    for (int i = 0; i < 2; ++i) {
-      mbar_init(&bar[F_VFULL0 + i], 1);
-      mbar_init(&bar[F_VEMPTY0 + i], 1);
-      mbar_init(&bar[F_SFULL0 + i], 1);
-      mbar_init(&bar[F_PFULL0 + i], 4);
-    }
-    mbar_init(&bar[F_OFULL], 1);
-    mbar_init(&bar[F_DRAIN], 1);
-    fence_mbar_init();
-  }
-  if (warp == 1) {
-    tmem_alloc(tmem_s, kTmemCols);
-    tmem_relinquish();
-    tc_fence_before();
-  }
-  if (warp == 0 && lane == 0) {
-    prefetch_tensormap(&q_map);
-    prefetch_tensormap(&k_map);
-    prefetch_tensormap(&v_map);
-  }
-  __syncthreads();
-  tc_fence_after();
-  const uint32_t tmem = *tmem_s;
-  bool aborted = false;
-
-  if (warp < 4) {
-    reg_dealloc<kCtrlRegs>();
-    if (warp == 1) {
-      // ------------------------------------------------------------------ MMA issuer
-      // TMEM columns: S / P of tile a at 0, of tile b at 128; O of tile a at 256, b at 384.
-      if (lane == 0) {
-        const uint32_t qa_addr = sbase + F_OFF_QA, qb_addr = sbase + F_OFF_QB;
-        if (!mbar_wait(&bar[F_Q], 0, lim)) fail(p, aborted);
-        tc_fence_after();
-        // S_t(kt) = Q_t K(kt)^T.  Issued after P V of the previous tile of the same
-        // query tile: the tensor core runs one thread's MMAs in order, so P (which
-        // overlays S) is read before it is overwritten.
-        auto qk = [&](int kt, int t) -> bool {
-          const int s = kt % kStagesF;
-          if (!mbar_wait(&bar[F_KFULL0 + s], (kt / kStagesF) & 1, lim)) return false;
-          tc_fence_after();
-          const uint32_t k_addr = sbase + F_OFF_K + s * kTileBytes;
-          const uint32_t q_addr = t ? qb_addr : qa_addr;
-#pragma unroll
-          for (int ks = 0; ks < D / 16; ++ks)
-            mma_bf16_ss(tmem + t * 128, kmajor_desc(q_addr, ks), kmajor_desc(k_addr, ks),
-                        IDESC_K_MAJOR, ks > 0);
-          mma_commit(&bar[F_SFULL0 + t]);
-          if (t == 1 || !has_b) mma_commit(&bar[F_KEMPTY0 + s]);  // K(kt) no longer read
-          return true;
-        };
-        if (!aborted && !qk(0, 0)) fail(p, aborted);
-        if (!aborted && has_b && !qk(0, 1)) fail(p, aborted);
-        // Then, per query tile and K/V tile: O_t += P_t(kt) V(kt) (A from TMEM, 16
-        // slots = 8 columns per k-step) and S_t(kt+1).  The two tiles are served in
-        // the order their P arrives: the barriers are polled, never waited on, so a
-        // tile that runs ahead (by as much as the K / V rings allow) never holds up
-        // the other.  The K and V stages are released by the second tile's commit.
-        int np0 = 0, np1 = has_b ? 0 : n_kt;  // next P V of tile a / b
-        uint64_t t_last = globaltimer();
-        while (!aborted && (np0 < n_kt || np1 < n_kt)) {
-          bool progressed = false;
-#pragma unroll
-          for (int t = 0; t < 2; ++t) {
-            const int kt = t ? np1 : np0;
-            if (kt >= n_kt) continue;
-            const bool more = kt + 1 < n_kt;
-            const int v = kt & 1, s1 = (kt + 1) % kStagesF;
-            if (!mbar_test(&bar[F_PFULL0 + t], kt & 1) ||
-                !mbar_test(&bar[F_VFULL0 + v], (kt >> 1) & 1) ||
-                (more && !mbar_test(&bar[F_KFULL0 + s1], ((kt + 1) / kStagesF) & 1)))
-              continue;
-            tc_fence_after();
-            const uint32_t v_addr = sbase + F_OFF_V + v * kTileBytes;
-#pragma unroll
-            for (int ks = 0; ks < BN / 16; ++ks)
-              mma_bf16_ts(tmem + 256 + t * 128, tmem + t * 128 + ks * 8, mnmajor_desc(v_addr, ks),
-                          IDESC_TS_PV, (kt > 0 || ks > 0) ? 1u : 0u);
-            // the other tile has issued its P V(kt) and S(kt+1) already
-            const bool second = (t ? np0 : np1) > kt;
-            if (second) mma_commit(&bar[F_VEMPTY0 + v]);  // V(kt) no longer read
-            if (more) {
-              const uint32_t k_addr = sbase + F_OFF_K + s1 * kTileBytes;
-              const uint32_t q_addr = t ? qb_addr : qa_addr;
-#pragma unroll
-              for (int ks = 0; ks < D / 16; ++ks)
-                mma_bf16_ss(tmem + t * 128, kmajor_desc(q_addr, ks), kmajor_desc(k_addr, ks),
-                            IDESC_K_MAJOR, ks > 0);
-              mma_commit(&bar[F_SFULL0 + t]);
-              if (second) mma_commit(&bar[F_KEMPTY0 + s1]);  // K(kt+1) no longer read
-            }
-            if (t) np1 = kt + 1; else np0 = kt + 1;
-            progressed = true;
-          }
-          const uint64_t now = globaltimer();
-          if (progressed) t_last = now;
-          else if (now - t_last > lim) fail(p, aborted);
-        }
-        mma_commit(&bar[F_OFULL]);
-        mma_commit(&bar[F_DRAIN]);
-        mbar_wait(&bar[F_DRAIN], 0, 4000000000ull);
-      }
-      __syncwarp();
-    } else if (warp == 0) {
-      // ----------------------------------------- producer of Q, K and slot positions
-      if (lane == 0) {
-        mbar_expect_tx(&bar[F_Q], has_b ? 2 * kTileBytes : kTileBytes);
-        tma_load_3d(smem + F_OFF_QA, &q_map, &bar[F_Q], 0, i0_a, bhq_a);
-        tma_load_3d(smem + F_OFF_QA + kHalfBytes, &q_map, &bar[F_Q], 64, i0_a, bhq_a);
-        if (has_b) {
-          tma_load_3d(smem + F_OFF_QB, &q_map, &bar[F_Q], 0, i0_b, bhq_b);
-          tma_load_3d(smem + F_OFF_QB + kHalfBytes, &q_map, &bar[F_Q], 64, i0_b, bhq_b);
-        }
-        mbar_arrive(&bar[F_Q]);
-      }
-      const int32_t *tpg = p.token_pos + (size_t)bg * p.N_C;
-      int issued = 0;
-      for (int kt = 0; kt < n_kt && !aborted; ++kt) {
-        const int s = kt % kStagesF, n = kt / kStagesF;
-        if (n > 0 && !warp_wait(&bar[F_KEMPTY0 + s], (n - 1) & 1, lim)) { fail(p, aborted); break; }
-        uint8_t *kdst = smem + F_OFF_K + s * kTileBytes;
-        if (lane == 0) {
-          mbar_expect_tx(&bar[F_KFULL0 + s], kTileBytes);
-          tma_load_3d(kdst, &k_map, &bar[F_KFULL0 + s], 0, kt * BN, bg);
-          tma_load_3d(kdst + kHalfBytes, &k_map, &bar[F_KFULL0 + s], 64, kt * BN, bg);
-          if (kt + kPrefetch < n_kt) {
-            tma_prefetch_l2_3d(&k_map, 0, (kt + kPrefetch) * BN, bg);
-            tma_prefetch_l2_3d(&k_map, 64, (kt + kPrefetch) * BN, bg);
-          }
-        }
-        tile_positions(rel_s + s * BN, tpg, kt, p.N_C, p.P, lane);
-        __syncwarp();
-        {
-          // slots invisible to the first row of a tile, compacted in slot order
-          const float thr = (float)min(i0_a, i0_b);
-          int32_t *cand = reinterpret_cast<int32_t *>(smem + F_OFF_CAND) + s * kCandWords;
-          int total = 0;
-#pragma unroll 1
-          for (int q = 0; q < 4; ++q)
-            total += __popc(__ballot_sync(0xffffffffu, rel_s[s * BN + lane + 32 * q] > thr));
-          if (total <= kMaxCand) {
-            int off = 0;
-#pragma unroll 1
-            for (int q = 0; q < 4; ++q) {
-              const float rq = rel_s[s * BN + lane + 32 * q];
-              const uint32_t bq = __ballot_sync(0xffffffffu, rq > thr);
-              if ((bq >> lane) & 1u) {
-                const int idx = off + __popc(bq & ((1u << lane) - 1u));
-                cand[2 + 2 * idx] = lane + 32 * q;
-                cand[3 + 2 * idx] = __float_as_int(rq);
-              }
-              off += __popc(bq);
-            }
-          }
-          if (lane == 0) cand[0] = total <= kMaxCand ? total : -1;
-        }
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&bar[F_KFULL0 + s]);
-        issued = kt + 1;
-      }
-      // drain: the last issued loads land before exit
-      if (lane == 0) {
-        mbar_wait(&bar[F_Q], 0, 4000000000ull);
-        for (int kt = issued - 1; kt >= 0 && kt >= issued - kStagesF; --kt)
-          mbar_wait(&bar[F_KFULL0 + kt % kStagesF], (kt / kStagesF) & 1, 4000000000ull);
-      }
-    } else if (warp == 2) {
-      // ------------------------------------------------------------------ producer of V
-      if (lane == 0) {
-        int issued = 0;
-        for (int kt = 0; kt < n_kt && !aborted; ++kt) {
-          const int v = kt & 1, n = kt >> 1;
-          if (n > 0 && !mbar_wait(&bar[F_VEMPTY0 + v], (n - 1) & 1, lim)) { fail(p, aborted); break; }
-          uint8_t *vdst = smem + F_OFF_V + v * kTileBytes;
-          mbar_expect_tx(&bar[F_VFULL0 + v], kTileBytes);
-          tma_load_3d(vdst, &v_map, &bar[F_VFULL0 + v], 0, kt * BN, bg);
-          tma_load_3d(vdst + kHalfBytes, &v_map, &bar[F_VFULL0 + v], 64, kt * BN, bg);
-          mbar_arrive(&bar[F_VFULL0 + v]);
-          if (kt + kPrefetch < n_kt) {
-            tma_prefetch_l2_3d(&v_map, 0, (kt + kPrefetch) * BN, bg);
-            tma_prefetch_l2_3d(&v_map, 64, (kt + kPrefetch) * BN, bg);
-          }
-          issued = kt + 1;
-        }
-        for (int kt = issued - 1; kt >= 0 && kt >= issued - 2; --kt)
-          mbar_wait(&bar[F_VFULL0 + (kt & 1)], (kt >> 1) & 1, 4000000000ull);
-      }
-      __syncwarp();
-    }
-  } else {
-    reg_alloc<kSoftRegs>();
-    const int t = (warp - 4) >> 2;  // 0: tile a, 1: tile b
-    if (t == 0 || has_b) {
-      // ------------------------------------- online softmax, one thread per query row
-      const int st = threadIdx.x - 128 * (1 + t);
-      const uint32_t lane_base = (uint32_t)(32 * (warp & 3)) << 16;
-      const uint32_t s_col = tmem + lane_base + t * 128, o_col = tmem + lane_base + 256 + t * 128;
-      const float c2 = p.scale2;
-      const int i0 = t ? i0_b : i0_a, bhq = t ? bhq_b : bhq_a, tt = t ? t_b : t_a;
-      const float mbias = kMaskBias / c2;
-      float m = -INFINITY, l = 0.f;  // reference maximum (base 2) and sum against it
-      uint32_t x[BN];
-      for (int kt = 0; kt < n_kt && !aborted; ++kt) {
-        const int s = kt % kStagesF;
-        if (!warp_wait(&bar[F_SFULL0 + t], kt & 1, lim)) { fail(p, aborted); break; }
-        if (!warp_wait(&bar[F_KFULL0 + s], (kt / kStagesF) & 1, lim)) { fail(p, aborted); break; }
-        tc_fence_after();
-        const float *rel = rel_s + s * BN;
-        const int32_t *cand = reinterpret_cast<const int32_t *>(smem + F_OFF_CAND) + s * kCandWords;
-        const int nc = cand[0];
-        if (nc > 0) {
-          // few slots to mask: lower them in TMEM before the row is read (a masked
-          // logit drops by 2^30 in base-2 units, as in row_mask)
-          const float ri = (float)(i0 + st);
-#pragma unroll 1
-          for (int q0 = 0; q0 < nc; q0 += 4) {
-            uint32_t cv[4];
-#pragma unroll
-            for (int q = 0; q < 4; ++q)
-              if (q0 + q < nc) cv[q] = tmem_ld1(s_col + cand[2 + 2 * (q0 + q)]);
-            tmem_wait_ld();
-#pragma unroll
-            for (int q = 0; q < 4; ++q)
-              if (q0 + q < nc) {
-                const float nm = fma_sat(__int_as_float(cand[3 + 2 * (q0 + q)]), 1.f, -ri);
-                tmem_st1(s_col + cand[2 + 2 * (q0 + q)],
-                         __float_as_uint(fmaf(nm, -mbias, __uint_as_float(cv[q]))));
-              }
-          }
-          tmem_wait_st();
-        }
-        const bool masked = nc < 0;  // too many: mask the whole row after reading it
-        tmem_ld32(s_col, *reinterpret_cast<uint32_t(*)[32]>(x));
-        tmem_ld32(s_col + 32, *reinterpret_cast<uint32_t(*)[32]>(x + 32));
-        tmem_ld32(s_col + 64, *reinterpret_cast<uint32_t(*)[32]>(x + 64));
-        tmem_ld32(s_col + 96, *reinterpret_cast<uint32_t(*)[32]>(x + 96));
-        tmem_wait_ld();
-        if (masked) row_mask<BN>(x, rel, (float)(i0 + st), mbias);
-        // Probabilities against the reference maximum m, computed alongside the row
-        // maximum.  m follows the row maximum lazily (p <= 2^8 in between); when the
-        // maximum exceeds it by more than that (the first tile; rarely later) m moves,
-        // O and l are rescaled and the tile is done again from S, still in TMEM.
-        uint32_t pk[BN / 2];
-        const float mx = row_max<BN>(x) * c2;
-        float ps = row_probs(x, c2, m, pk);
-        const bool need = mx > m + kLazyMax;
-        if (__any_sync(0xffffffffu, need)) {
-          const float m_new = need ? mx : m;
-          const float f = ex2(m - m_new);  // 1 if unchanged, 0 from -inf
-          l *= f;
-          if (kt > 0) {
-            // O holds the sums of P V up to the previous tile: every MMA before S(kt)
-            // is complete, none after it is issued until this warp's P is written
-#pragma unroll 1
-            for (int cq = 0; cq < 4; ++cq) {
-              uint32_t o[32];
-              tmem_ld32(o_col + cq * 32, o);
-              tmem_wait_ld();
-#pragma unroll
-              for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * f);
-              tmem_st32(o_col + cq * 32, o);
-            }
-          }
-          m = m_new;
-          tmem_ld32(s_col, *reinterpret_cast<uint32_t(*)[32]>(x));
-          tmem_ld32(s_col + 32, *reinterpret_cast<uint32_t(*)[32]>(x + 32));
-          tmem_ld32(s_col + 64, *reinterpret_cast<uint32_t(*)[32]>(x + 64));
-          tmem_ld32(s_col + 96, *reinterpret_cast<uint32_t(*)[32]>(x + 96));
-          tmem_wait_ld();
-          if (masked) row_mask<BN>(x, rel, (float)(i0 + st), mbias);
-          ps = row_probs(x, c2, m, pk);
-        }
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&bar[F_KEMPTY0 + s]);  // positions no longer read
-        // P over S (bf16 pairs), the A operand of O += P V
-        tmem_st32(s_col, *reinterpret_cast<uint32_t(*)[32]>(pk));
-        tmem_st32(s_col + 32, *reinterpret_cast<uint32_t(*)[32]>(pk + 32));
-        l += ps;
-        tmem_wait_st();
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&bar[F_PFULL0 + t]);
-      }
-      // row results: -lse2 for pass 2, lse (natural log) on request, y = O / l
-      const bool seen = l > 0.f && m > -0.5f * kMaskBias;
-      const float lse2 = seen ? m + lg2(l) : -INFINITY;
-      const bool row_ok = i0 + st < p.S;
-      p.nlse[((size_t)bhq * p.tiles + tt) * BM + st] = seen ? -lse2 : -kMaskBias;
-      if (p.lse_out && row_ok) p.lse_out[(size_t)bhq * p.S + i0 + st] = lse2 * 0.69314718055994531f;
-      if (!aborted && !warp_wait(&bar[F_OFULL], 0, lim)) fail(p, aborted);
-      tc_fence_after();
-      if (!aborted) {
-        const float inv = seen ? 1.f / l : 0.f;
-        __nv_bfloat16 *yrow = p.y + ((size_t)bhq * p.S + i0 + st) * D;
-        uint32_t r[32];
-#pragma unroll
-        for (int cq = 0; cq < 4; ++cq) {
-          tmem_ld32(o_col + cq * 32, r);
-          tmem_wait_ld();
-          if (row_ok) {
-            uint32_t o[16];
-#pragma unroll
-            for (int e = 0; e < 16; ++e)
-              o[e] = pack_bf16x2(__uint_as_float(r[2 * e]) * inv, __uint_as_float(r[2 * e + 1]) * inv);
-            uint4 *dst = reinterpret_cast<uint4 *>(yrow + cq * 32);
-#pragma unroll
-            for (int e = 0; e < 4; ++e)
-              dst[e] = make_uint4(o[4 * e], o[4 * e + 1], o[4 * e + 2], o[4 * e + 3]);
-          }
-        }
-      }
-      tc_fence_before();
-    }
-  }
-  __syncthreads();
-  if (warp == 1) {
-    tc_fence_after();
-    tmem_dealloc(tmem, kTmemCols);
   }
 }
 
@@ -1780,6 +1437,40 @@ struct SegIter {
     return true;
   }
 };
+// The same segments with 32-bit unit indices (pass 1 holds it in every role).
+struct SegIter32 {
+  int u, u1, f0, f1, ubase, n_kt;
+  __device__ __forceinline__ void take(int &a, int b, int &p, int &kt0, int &kt1) {
+    p = a / n_kt;
+    kt0 = a - p * n_kt;
+    kt1 = min(n_kt, kt0 + (b - a));
+    a += kt1 - kt0;
+  }
+  __device__ __forceinline__ bool next(int &p, int &kt0, int &kt1, int &slot) {
+    if (u < u1) take(u, u1, p, kt0, kt1);
+    else if (f0 < f1) take(f0, f1, p, kt0, kt1);
+    else return false;
+    slot = p - ubase / n_kt;
+    return true;
+  }
+};
+__device__ __forceinline__ SegIter32 seg_iter32(const SplitParams &sp) {
+  SegIter32 it;
+  it.n_kt = sp.t.n_kt;
+  it.ubase = (int)unit0(blockIdx.x, sp);
+  it.u1 = (int)unit0(blockIdx.x + 1, sp);
+  const int kt0 = it.ubase % it.n_kt;
+  const int first_end = min(it.u1, it.ubase + (it.n_kt - kt0));
+  if (kt0 > 0 && first_end < it.u1) {
+    it.f0 = it.ubase;
+    it.f1 = first_end;
+    it.u = first_end;
+  } else {
+    it.f0 = it.f1 = 0;
+    it.u = it.ubase;
+  }
+  return it;
+}
 __device__ __forceinline__ SegIter seg_iter(const SplitParams &sp) {
   SegIter it;
   it.n_kt = sp.t.n_kt;
@@ -2019,6 +1710,492 @@ __device__ __forceinline__ int cta_of_unit(long long x, const SplitParams &sp) {
 }
 __device__ __forceinline__ int seg_slot(int p, int c, const SplitParams &sp) {
   return p - (int)(unit0(c, sp) / sp.t.n_kt);
+}
+
+// Pass 1 over equal shares of the (pair, K/V tile) units, one CTA per SM: CTA c takes
+// units [U c / G, U (c + 1) / G) in segments of one pair each (SegIter order).  A
+// segment that covers a whole pair writes y and -lse2; the pieces of a pair split over
+// CTAs write their rows' (max, sum) and unnormalised O, which combine_fwd_kernel
+// merges.  With G = pairs every CTA takes one whole pair.
+__global__ void __launch_bounds__(kThreads, 1)
+    attn_fwd_kernel(const __grid_constant__ CUtensorMap q_map,
+                    const __grid_constant__ CUtensorMap k_map,
+                    const __grid_constant__ CUtensorMap v_map, const SplitParams sp) {
+  const TcParams &p = sp.t;
+  extern __shared__ __align__(1024) uint8_t smem[];
+  const uint32_t sbase = smem_u32(smem);
+  if (sbase & 1023u) {
+    if (threadIdx.x == 0) atomicExch(p.status, H2OKV_ERR_CUDA);
+    return;
+  }
+  float *rel_s = reinterpret_cast<float *>(smem + F_OFF_REL);
+  uint64_t *bar = reinterpret_cast<uint64_t *>(smem + F_OFF_BAR);
+  uint32_t *tmem_s = reinterpret_cast<uint32_t *>(smem + F_OFF_TMEM);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int n_qt = p.q_g * p.tiles;
+  const int n_kt = p.n_kt;
+  const uint64_t lim = p.timeout_ns;
+  int4 *segs = reinterpret_cast<int4 *>(smem + F_OFF_SEG);
+  if (threadIdx.x == 0) {
+    SegIter32 it = seg_iter32(sp);
+    int n = 0, pp, a0, a1, sl;
+    while (n < kMaxSegF && it.next(pp, a0, a1, sl)) segs[1 + n++] = make_int4(pp, a0, a1, sl);
+    segs[0].x = n;
+    mbar_init(&bar[F_Q], 1);
+    for (int i = 0; i < kStagesF; ++i) {
+      mbar_init(&bar[F_KFULL0 + i], 1);
+      mbar_init(&bar[F_KEMPTY0 + i], 1 + 8);  // MMA commit + all softmax warps (positions)
+    }
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&bar[F_VFULL0 + i], 1);
+      mbar_init(&bar[F_VEMPTY0 + i], 1);
+      mbar_init(&bar[F_SFULL0 + i], 1);
+      mbar_init(&bar[F_PFULL0 + i], 4);
+    }
+    mbar_init(&bar[F_OFULL], 1);
+    mbar_init(&bar[F_OFREE], 8);
+    mbar_init(&bar[F_QFREE], 1);
+    mbar_init(&bar[F_DRAIN], 1);
+    fence_mbar_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_s, kTmemCols);
+    tmem_relinquish();
+    tc_fence_before();
+  }
+  if (warp == 0 && lane == 0) {
+    prefetch_tensormap(&q_map);
+    prefetch_tensormap(&k_map);
+    prefetch_tensormap(&v_map);
+  }
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_s;
+  bool aborted = false;
+  const int nseg = segs[0].x;
+  int pidx, kt0, kt1, slot;
+  auto segment = [&](int sg) {
+    const int4 e = segs[1 + sg];
+    pidx = e.x;
+    kt0 = e.y;
+    kt1 = e.z;
+    slot = e.w;
+  };
+
+  if (warp < 4) {
+    reg_dealloc<kCtrlRegsF>();
+    if (warp == 1) {
+      // ------------------------------------------------------------------ MMA issuer
+      // TMEM columns: S / P of tile a at 0, of tile b at 128; O of tile a at 256, b at 384.
+      if (lane == 0) {
+        const uint32_t qa_addr = sbase + F_OFF_QA, qb_addr = sbase + F_OFF_QB;
+        int ibase = 0, nb_base = 0;  // units before this segment (all / tile b)
+        for (int seg = 0; seg < nseg && !aborted; ++seg) {
+          segment(seg);
+          const bool has_b = 2 * (pidx % p.ctas_per_group) + 1 < n_qt;
+          const int len = kt1 - kt0;
+          // S_t of the segment's first tile.  Every later S_t(kt+1) is issued after
+          // P_t(kt) V: the tensor core runs one thread's MMAs in order, so P (which
+          // overlays S) is read before it is overwritten.
+          if (!mbar_wait(&bar[F_Q], seg & 1, lim) ||
+              !mbar_wait(&bar[F_KFULL0 + ibase % kStagesF], (ibase / kStagesF) & 1, lim)) {
+            fail(p, aborted);
+            break;
+          }
+          tc_fence_after();
+          {
+            const uint32_t k_addr = sbase + F_OFF_K + (ibase % kStagesF) * kTileBytes;
+#pragma unroll
+            for (int t = 0; t < 2; ++t) {
+              if (t == 1 && !has_b) break;
+#pragma unroll
+              for (int ks = 0; ks < D / 16; ++ks)
+                mma_bf16_ss(tmem + t * 128, kmajor_desc(t ? qb_addr : qa_addr, ks),
+                            kmajor_desc(k_addr, ks), IDESC_K_MAJOR, ks > 0);
+              mma_commit(&bar[F_SFULL0 + t]);
+            }
+            mma_commit(&bar[F_KEMPTY0 + ibase % kStagesF]);  // first K no longer read
+          }
+          // O of the previous segment read out before the first P V overwrites it
+          if (seg > 0 && !mbar_wait(&bar[F_OFREE], (seg - 1) & 1, lim)) { fail(p, aborted); break; }
+          // Per query tile and K/V tile: O_t (+)= P_t V (A from TMEM, 16 slots = 8
+          // columns per k-step) and S_t of the next tile.  The tiles are served in the
+          // order their P arrives: the barriers are polled, never waited on, so a tile
+          // that runs ahead (as far as the K / V rings allow) never holds up the other.
+          // The K and V stages are released by the second tile's commit.
+          int np0 = 0, np1 = has_b ? 0 : len;  // next P V of tile a / b, within the segment
+          uint64_t t_last = globaltimer();
+          while (!aborted && (np0 < len || np1 < len)) {
+            bool progressed = false;
+#pragma unroll
+            for (int t = 0; t < 2; ++t) {
+              const int k = t ? np1 : np0;
+              if (k >= len) continue;
+              const int i = ibase + k;                        // unit index in the CTA
+              const int n = (t ? nb_base : ibase) + k;        // this tile's P count
+              const bool more = k + 1 < len;
+              const int v = i & 1, s1 = (i + 1) % kStagesF;
+              if (!mbar_test(&bar[F_PFULL0 + t], n & 1) ||
+                  !mbar_test(&bar[F_VFULL0 + v], (i >> 1) & 1) ||
+                  (more && !mbar_test(&bar[F_KFULL0 + s1], ((i + 1) / kStagesF) & 1)))
+                continue;
+              tc_fence_after();
+              const uint32_t v_addr = sbase + F_OFF_V + v * kTileBytes;
+#pragma unroll
+              for (int ks = 0; ks < BN / 16; ++ks)
+                mma_bf16_ts(tmem + 256 + t * 128, tmem + t * 128 + ks * 8, mnmajor_desc(v_addr, ks),
+                            IDESC_TS_PV, (k > 0 || ks > 0) ? 1u : 0u);
+              // the other tile has issued its P V and next S already
+              const bool second = (t ? np0 : np1) > k;
+              if (second) mma_commit(&bar[F_VEMPTY0 + v]);  // V no longer read
+              if (more) {
+                const uint32_t k_addr = sbase + F_OFF_K + s1 * kTileBytes;
+#pragma unroll
+                for (int ks = 0; ks < D / 16; ++ks)
+                  mma_bf16_ss(tmem + t * 128, kmajor_desc(t ? qb_addr : qa_addr, ks),
+                              kmajor_desc(k_addr, ks), IDESC_K_MAJOR, ks > 0);
+                mma_commit(&bar[F_SFULL0 + t]);
+                if (second) mma_commit(&bar[F_KEMPTY0 + s1]);  // K no longer read
+              }
+              if (t) np1 = k + 1; else np0 = k + 1;
+              progressed = true;
+            }
+            const uint64_t now = globaltimer();
+            if (progressed) t_last = now;
+            else if (now - t_last > lim) fail(p, aborted);
+          }
+          mma_commit(&bar[F_OFULL]);
+          mma_commit(&bar[F_QFREE]);  // the segment's Q tiles no longer read
+          ibase += len;
+          if (has_b) nb_base += len;
+        }
+        mma_commit(&bar[F_DRAIN]);
+        mbar_wait(&bar[F_DRAIN], 0, 4000000000ull);
+      }
+      __syncwarp();
+    } else if (warp == 0) {
+      // ------------------------- producer of Q (per segment), K and slot positions
+      int i = 0, seg = 0;
+      for (; seg < nseg && !aborted; ++seg) {
+        segment(seg);
+        const PairInfo pi = pair_info(pidx, p);
+        const bool has_b = 2 * (pidx % p.ctas_per_group) + 1 < n_qt;
+        if (seg > 0 && !warp_wait(&bar[F_QFREE], (seg - 1) & 1, lim)) { fail(p, aborted); break; }
+        if (lane == 0) {
+          mbar_expect_tx(&bar[F_Q], has_b ? 2 * kTileBytes : kTileBytes);
+          tma_load_3d(smem + F_OFF_QA, &q_map, &bar[F_Q], 0, pi.i0_a, pi.bhq_a);
+          tma_load_3d(smem + F_OFF_QA + kHalfBytes, &q_map, &bar[F_Q], 64, pi.i0_a, pi.bhq_a);
+          if (has_b) {
+            tma_load_3d(smem + F_OFF_QB, &q_map, &bar[F_Q], 0, pi.i0_b, pi.bhq_b);
+            tma_load_3d(smem + F_OFF_QB + kHalfBytes, &q_map, &bar[F_Q], 64, pi.i0_b, pi.bhq_b);
+          }
+          mbar_arrive(&bar[F_Q]);
+        }
+        const int32_t *tpg = p.token_pos + (size_t)pi.bg * p.N_C;
+        const float thr = (float)(has_b ? min(pi.i0_a, pi.i0_b) : pi.i0_a);
+        for (int kt = kt0; kt < kt1 && !aborted; ++kt, ++i) {
+          const int s = i % kStagesF, n = i / kStagesF;
+          if (n > 0 && !warp_wait(&bar[F_KEMPTY0 + s], (n - 1) & 1, lim)) { fail(p, aborted); break; }
+          uint8_t *kdst = smem + F_OFF_K + s * kTileBytes;
+          if (lane == 0) {
+            mbar_expect_tx(&bar[F_KFULL0 + s], kTileBytes);
+            tma_load_3d(kdst, &k_map, &bar[F_KFULL0 + s], 0, kt * BN, pi.bg);
+            tma_load_3d(kdst + kHalfBytes, &k_map, &bar[F_KFULL0 + s], 64, kt * BN, pi.bg);
+            if (kt + kPrefetch < kt1) {
+              tma_prefetch_l2_3d(&k_map, 0, (kt + kPrefetch) * BN, pi.bg);
+              tma_prefetch_l2_3d(&k_map, 64, (kt + kPrefetch) * BN, pi.bg);
+            }
+          }
+          tile_positions(rel_s + s * BN, tpg, kt, p.N_C, p.P, lane);
+          __syncwarp();
+          {
+            // slots invisible to the first row of a tile, compacted in slot order
+            int32_t *cand = reinterpret_cast<int32_t *>(smem + F_OFF_CAND) + s * kCandWords;
+            int total = 0;
+#pragma unroll 1
+            for (int q = 0; q < 4; ++q)
+              total += __popc(__ballot_sync(0xffffffffu, rel_s[s * BN + lane + 32 * q] > thr));
+            if (total <= kMaxCand) {
+              int off = 0;
+#pragma unroll 1
+              for (int q = 0; q < 4; ++q) {
+                const float rq = rel_s[s * BN + lane + 32 * q];
+                const uint32_t bq = __ballot_sync(0xffffffffu, rq > thr);
+                if ((bq >> lane) & 1u) {
+                  const int idx = off + __popc(bq & ((1u << lane) - 1u));
+                  cand[2 + 2 * idx] = lane + 32 * q;
+                  cand[3 + 2 * idx] = __float_as_int(rq);
+                }
+                off += __popc(bq);
+              }
+            }
+            if (lane == 0) cand[0] = total <= kMaxCand ? total : -1;
+          }
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&bar[F_KFULL0 + s]);
+        }
+      }
+      // drain: the last issued loads land before exit
+      if (lane == 0) {
+        if (seg > 0) mbar_wait(&bar[F_Q], (seg - 1) & 1, 4000000000ull);
+        for (int j = i - 1; j >= 0 && j >= i - kStagesF; --j)
+          mbar_wait(&bar[F_KFULL0 + j % kStagesF], (j / kStagesF) & 1, 4000000000ull);
+      }
+    } else if (warp == 2) {
+      // ------------------------------------------------------------------ producer of V
+      if (lane == 0) {
+        int i = 0;
+        for (int sg = 0; sg < nseg && !aborted; ++sg) {
+          segment(sg);
+          const int bg = pidx / p.ctas_per_group;
+          for (int kt = kt0; kt < kt1 && !aborted; ++kt, ++i) {
+            const int v = i & 1, n = i >> 1;
+            if (n > 0 && !mbar_wait(&bar[F_VEMPTY0 + v], (n - 1) & 1, lim)) { fail(p, aborted); break; }
+            uint8_t *vdst = smem + F_OFF_V + v * kTileBytes;
+            mbar_expect_tx(&bar[F_VFULL0 + v], kTileBytes);
+            tma_load_3d(vdst, &v_map, &bar[F_VFULL0 + v], 0, kt * BN, bg);
+            tma_load_3d(vdst + kHalfBytes, &v_map, &bar[F_VFULL0 + v], 64, kt * BN, bg);
+            mbar_arrive(&bar[F_VFULL0 + v]);
+            if (kt + kPrefetch < kt1) {
+              tma_prefetch_l2_3d(&v_map, 0, (kt + kPrefetch) * BN, bg);
+              tma_prefetch_l2_3d(&v_map, 64, (kt + kPrefetch) * BN, bg);
+            }
+          }
+        }
+        for (int j = i - 1; j >= 0 && j >= i - 2; --j)
+          mbar_wait(&bar[F_VFULL0 + (j & 1)], (j >> 1) & 1, 4000000000ull);
+      }
+      __syncwarp();
+    }
+  } else {
+    reg_alloc<kSoftRegsF>();
+    const int t = (warp - 4) >> 2;  // 0: tile a, 1: tile b
+    // ------------------------------------- online softmax, one thread per query row
+    const int st = threadIdx.x - 128 * (1 + t);
+    const uint32_t lane_base = (uint32_t)(32 * (warp & 3)) << 16;
+    const uint32_t s_col = tmem + lane_base + t * 128, o_col = tmem + lane_base + 256 + t * 128;
+    const float c2 = p.scale2;
+    const float mbias = kMaskBias / c2;
+    int i = 0, nt = 0;  // units of the CTA, units of this tile
+    for (int seg = 0; seg < nseg && !aborted; ++seg) {
+      segment(seg);
+      const PairInfo pi = pair_info(pidx, p);
+      const bool active = t == 0 || 2 * (pidx % p.ctas_per_group) + 1 < n_qt;
+      if (!active) {
+        // no tile b in this pair: keep the position ring's count
+        for (int kt = kt0; kt < kt1; ++kt, ++i) {
+          const int s = i % kStagesF;
+          if (!warp_wait(&bar[F_KFULL0 + s], (i / kStagesF) & 1, lim)) { fail(p, aborted); break; }
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&bar[F_KEMPTY0 + s]);
+        }
+        if (!aborted && !warp_wait(&bar[F_OFULL], seg & 1, lim)) fail(p, aborted);
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&bar[F_OFREE]);
+        continue;
+      }
+      const int i0 = t ? pi.i0_b : pi.i0_a, bhq = t ? pi.bhq_b : pi.bhq_a, tt = t ? pi.t_b : pi.t_a;
+      float m = -INFINITY, l = 0.f;  // reference maximum (base 2) and sum against it
+      uint32_t x[BN];
+      for (int kt = kt0; kt < kt1 && !aborted; ++kt, ++i, ++nt) {
+        const int s = i % kStagesF;
+        if (!warp_wait(&bar[F_SFULL0 + t], nt & 1, lim)) { fail(p, aborted); break; }
+        if (!warp_wait(&bar[F_KFULL0 + s], (i / kStagesF) & 1, lim)) { fail(p, aborted); break; }
+        tc_fence_after();
+        const float *rel = rel_s + s * BN;
+        const int32_t *cand = reinterpret_cast<const int32_t *>(smem + F_OFF_CAND) + s * kCandWords;
+        const int nc = cand[0];
+        if (nc > 0) {
+          // few slots to mask: lower them in TMEM before the row is read (a masked
+          // logit drops by 2^30 in base-2 units, as in row_mask)
+          const float ri = (float)(i0 + st);
+#pragma unroll 1
+          for (int q0 = 0; q0 < nc; q0 += 4) {
+            uint32_t cv[4];
+#pragma unroll
+            for (int q = 0; q < 4; ++q)
+              if (q0 + q < nc) cv[q] = tmem_ld1(s_col + cand[2 + 2 * (q0 + q)]);
+            tmem_wait_ld();
+#pragma unroll
+            for (int q = 0; q < 4; ++q)
+              if (q0 + q < nc) {
+                const float nm = fma_sat(__int_as_float(cand[3 + 2 * (q0 + q)]), 1.f, -ri);
+                tmem_st1(s_col + cand[2 + 2 * (q0 + q)],
+                         __float_as_uint(fmaf(nm, -mbias, __uint_as_float(cv[q]))));
+              }
+          }
+          tmem_wait_st();
+        }
+        const bool masked = nc < 0;  // too many: mask the whole row after reading it
+        tmem_ld32(s_col, *reinterpret_cast<uint32_t(*)[32]>(x));
+        tmem_ld32(s_col + 32, *reinterpret_cast<uint32_t(*)[32]>(x + 32));
+        tmem_ld32(s_col + 64, *reinterpret_cast<uint32_t(*)[32]>(x + 64));
+        tmem_ld32(s_col + 96, *reinterpret_cast<uint32_t(*)[32]>(x + 96));
+        tmem_wait_ld();
+        if (masked) row_mask<BN>(x, rel, (float)(i0 + st), mbias);
+        // Probabilities against the reference maximum m, computed alongside the row
+        // maximum.  m follows the row maximum lazily (p <= 2^8 in between); when the
+        // maximum exceeds it by more than that (the first tile; rarely later) m moves,
+        // O and l are rescaled and the tile is done again from S, still in TMEM.
+        uint32_t pk[BN / 2];
+        const float mx = row_max<BN>(x) * c2;
+        float ps = row_probs(x, c2, m, pk);
+        const bool need = mx > m + kLazyMax;
+        if (__any_sync(0xffffffffu, need)) {
+          const float m_new = need ? mx : m;
+          const float f = ex2(m - m_new);  // 1 if unchanged, 0 from -inf
+          l *= f;
+          if (kt > kt0) {
+            // O holds the sums of P V up to the previous tile: every MMA before S(kt)
+            // is complete, none after it is issued until this warp's P is written
+#pragma unroll 1
+            for (int cq = 0; cq < 4; ++cq) {
+              uint32_t o[32];
+              tmem_ld32(o_col + cq * 32, o);
+              tmem_wait_ld();
+#pragma unroll
+              for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * f);
+              tmem_st32(o_col + cq * 32, o);
+            }
+          }
+          m = m_new;
+          tmem_ld32(s_col, *reinterpret_cast<uint32_t(*)[32]>(x));
+          tmem_ld32(s_col + 32, *reinterpret_cast<uint32_t(*)[32]>(x + 32));
+          tmem_ld32(s_col + 64, *reinterpret_cast<uint32_t(*)[32]>(x + 64));
+          tmem_ld32(s_col + 96, *reinterpret_cast<uint32_t(*)[32]>(x + 96));
+          tmem_wait_ld();
+          if (masked) row_mask<BN>(x, rel, (float)(i0 + st), mbias);
+          ps = row_probs(x, c2, m, pk);
+        }
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&bar[F_KEMPTY0 + s]);  // positions no longer read
+        // P over S (bf16 pairs), the A operand of O += P V
+        tmem_st32(s_col, *reinterpret_cast<uint32_t(*)[32]>(pk));
+        tmem_st32(s_col + 32, *reinterpret_cast<uint32_t(*)[32]>(pk + 32));
+        l += ps;
+        tmem_wait_st();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&bar[F_PFULL0 + t]);
+      }
+      if (aborted) break;
+      // the segment's rows: y, -lse2 and lse for a whole pair, else the piece's
+      // (max, sum) and O for combine_fwd_kernel
+      const bool whole = kt0 == 0 && kt1 == n_kt;
+      const bool row_ok = i0 + st < p.S;
+      if (!warp_wait(&bar[F_OFULL], seg & 1, lim)) { fail(p, aborted); break; }
+      tc_fence_after();
+      if (whole) {
+        const bool seen = l > 0.f && m > -0.5f * kMaskBias;
+        const float lse2 = seen ? m + lg2(l) : -INFINITY;
+        p.nlse[((size_t)bhq * p.tiles + tt) * BM + st] = seen ? -lse2 : -kMaskBias;
+        if (p.lse_out && row_ok) p.lse_out[(size_t)bhq * p.S + i0 + st] = lse2 * 0.69314718055994531f;
+        const float inv = seen ? 1.f / l : 0.f;
+        __nv_bfloat16 *yrow = p.y + ((size_t)bhq * p.S + i0 + st) * D;
+        uint32_t r[32];
+#pragma unroll
+        for (int cq = 0; cq < 4; ++cq) {
+          tmem_ld32(o_col + cq * 32, r);
+          tmem_wait_ld();
+          if (row_ok) {
+            uint32_t o[16];
+#pragma unroll
+            for (int e = 0; e < 16; ++e)
+              o[e] = pack_bf16x2(__uint_as_float(r[2 * e]) * inv, __uint_as_float(r[2 * e + 1]) * inv);
+            uint4 *dst = reinterpret_cast<uint4 *>(yrow + cq * 32);
+#pragma unroll
+            for (int e = 0; e < 4; ++e)
+              dst[e] = make_uint4(o[4 * e], o[4 * e + 1], o[4 * e + 2], o[4 * e + 3]);
+          }
+        }
+      } else {
+        const size_t prow = (((size_t)blockIdx.x * sp.max_seg + slot) * 2 + t) * BM + st;
+        sp.part_ml[prow] = make_float2(m, l);
+        float4 *dst = reinterpret_cast<float4 *>(sp.part_o + prow * D);
+        uint32_t r[32];
+#pragma unroll
+        for (int cq = 0; cq < 4; ++cq) {
+          tmem_ld32(o_col + cq * 32, r);
+          tmem_wait_ld();
+#pragma unroll
+          for (int e = 0; e < 8; ++e)
+            dst[cq * 8 + e] = make_float4(__uint_as_float(r[4 * e]), __uint_as_float(r[4 * e + 1]),
+                                          __uint_as_float(r[4 * e + 2]), __uint_as_float(r[4 * e + 3]));
+        }
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&bar[F_OFREE]);  // O read out
+    }
+    tc_fence_before();
+  }
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, kTmemCols);
+  }
+}
+
+// The pieces of every pair that pass 1 split over CTAs: per row, with the pieces'
+// maxima m_i and sums l_i against them, m = max m_i, l = sum l_i 2^(m_i - m),
+// O = sum O_i 2^(m_i - m); y = O / l, lse2 = m + log2 l.  Grid (pairs, 32): a CTA
+// looks the pair's pieces up once; each thread takes one row and 4 columns.
+constexpr int kMaxPieces = 8;
+constexpr int kMinSplitTiles = 32;  // pass 1 is split over CTAs only for scans this long
+__global__ void __launch_bounds__(256)
+    combine_fwd_kernel(const SplitParams sp) {
+  const TcParams &p = sp.t;
+  const int pidx = blockIdx.x;
+  __shared__ int piece_row[kMaxPieces];  // first partial row of each piece
+  __shared__ int n_pieces;
+  if (threadIdx.x == 0) {
+    const int c_first = cta_of_unit((long long)pidx * p.n_kt, sp);
+    const int c_last = cta_of_unit((long long)(pidx + 1) * p.n_kt - 1, sp);
+    int n = 0;
+    for (int c = c_first; c <= c_last && n < kMaxPieces; ++c, ++n)
+      piece_row[n] = ((c * sp.max_seg + seg_slot(pidx, c, sp)) * 2) * BM;
+    n_pieces = c_last > c_first ? n : 0;  // a pair of one piece was written by its CTA
+  }
+  __syncthreads();
+  const int np = n_pieces;
+  if (np == 0) return;
+  const bool has_b = 2 * (pidx % p.ctas_per_group) + 1 < p.q_g * p.tiles;
+  const PairInfo pi = pair_info(pidx, p);
+  {
+    const int e = blockIdx.y * blockDim.x + threadIdx.x;  // < 2 * BM * (D / 4)
+    const int t = e / (BM * (D / 4));
+    const int row = (e / (D / 4)) % BM, c4 = e % (D / 4);
+    if (t == 1 && !has_b) return;
+    const int i0 = t ? pi.i0_b : pi.i0_a, bhq = t ? pi.bhq_b : pi.bhq_a, tt = t ? pi.t_b : pi.t_a;
+    float m = -INFINITY;
+    for (int q = 0; q < np; ++q) m = fmaxf(m, sp.part_ml[piece_row[q] + t * BM + row].x);
+    float l = 0.f;
+    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+    for (int q = 0; q < np; ++q) {
+      const size_t prow = (size_t)piece_row[q] + t * BM + row;
+      const float2 ml = sp.part_ml[prow];
+      const float w = m == -INFINITY ? 0.f : ex2(ml.x - m);
+      l += ml.y * w;
+      const float4 v = __ldcs(reinterpret_cast<const float4 *>(sp.part_o + prow * D) + c4);
+      acc.x += v.x * w;
+      acc.y += v.y * w;
+      acc.z += v.z * w;
+      acc.w += v.w * w;
+    }
+    const bool seen = l > 0.f && m > -0.5f * kMaskBias;
+    const float lse2 = seen ? m + lg2(l) : -INFINITY;
+    if (c4 == 0) {
+      p.nlse[((size_t)bhq * p.tiles + tt) * BM + row] = seen ? -lse2 : -kMaskBias;
+      if (p.lse_out && i0 + row < p.S)
+        p.lse_out[(size_t)bhq * p.S + i0 + row] = lse2 * 0.69314718055994531f;
+    }
+    if (i0 + row >= p.S) return;
+    const float inv = seen ? 1.f / l : 0.f;
+    __nv_bfloat162 *dst =
+        reinterpret_cast<__nv_bfloat162 *>(p.y + ((size_t)bhq * p.S + i0 + row) * D + c4 * 4);
+    dst[0] = __floats2bfloat162_rn(acc.x * inv, acc.y * inv);
+    dst[1] = __floats2bfloat162_rn(acc.z * inv, acc.w * inv);
+  }
 }
 
 enum {
@@ -2675,6 +2852,13 @@ void tc_plan(const h2okv_cache_desc &d, TcPlan *plan) {
       plan->split_ctas = sms;
       plan->max_seg = sh.max_seg;
     }
+    if (d.kv_dtype == H2OKV_BF16 && plan->two_pass) {
+      // pass 1 on every SM: a CTA holds at most ceil(pairs / SMs) + 2 segments
+      const long long pairs = (long long)d.batch * d.n_kv_heads *
+                              (((d.n_q_heads / d.n_kv_heads) * plan->tiles_per_head + 1) / 2);
+      plan->split_ctas = sms;
+      plan->max_seg = max(plan->max_seg, (int)((pairs + sms - 1) / sms) + 2);
+    }
   }
   cudaGetLastError();  // a failed query (no device) is not an error here
 }
@@ -2811,7 +2995,8 @@ int launch_attn_tc(h2okv_cache *c, const void *q, int S, int64_t P, void *y, flo
   const CUtensorMap &vmap = *reinterpret_cast<const CUtensorMap *>(c->tc.v_map);
   // split scheduling: every SM gets the same share of (pair, K/V tile) units
   const SplitShape sh = split_shape(d, S, c->tc.split_ctas);
-  if (sh.use && sh.max_seg <= c->tc.max_seg) {
+  // (the fused kernel's split schedule; the two-pass path splits its own work)
+  if (sh.use && sh.max_seg <= c->tc.max_seg && !(d.kv_dtype == H2OKV_BF16 && c->tc.two_pass)) {
     static thread_local int ready_a = -1, ready_b = -1;
     rc = prepare_split_kernel(attn_split_a_kernel, ready_a, "attn_split_a_kernel");
     if (rc) return rc;
@@ -2851,9 +3036,36 @@ int launch_attn_tc(h2okv_cache *c, const void *q, int S, int64_t P, void *y, flo
     if (rc) return rc;
     rc = prepare_pass_kernel(scoresum_kernel, kSmemS, ready_s, "scoresum_kernel");
     if (rc) return rc;
-    attn_fwd_kernel<<<grid, kThreads, kSmemF, st>>>(qmap, kmap, vmap, prm);
+    // attention over equal shares of (pair, K/V tile) units, one CTA per SM when the
+    // partial-result workspace holds every CTA's pieces, else one CTA per pair
+    SplitParams fs{};
+    fs.t = prm;
+    fs.U = (long long)grid * prm.n_kt;
+    fs.G = grid;
+    fs.max_seg = c->tc.max_seg;
+    fs.part_ml = reinterpret_cast<float2 *>(ws + c->ws.part_ml);
+    fs.part_o = reinterpret_cast<float *>(ws + c->ws.part_o);
+    const int G = (int)min((long long)c->tc.split_ctas, fs.U);
+    // Only when one CTA per pair leaves over a quarter of the SMs idle in the last wave,
+    // and the scan is long: otherwise the partial results' round trip and the K/V
+    // tiles that CTAs of a group no longer share in L2 cost more than the idle SMs.
+    const int sms = max(c->tc.sms, 1);
+    const double fill = (double)grid / (double)(((grid + sms - 1) / sms) * sms);
+    if (G > grid && prm.n_kt >= kMinSplitTiles && fill < kSplitFill) {
+      const long long per = (fs.U + G - 1) / G;
+      const long long segs = (per + prm.n_kt - 1) / prm.n_kt + 1;
+      // a pair spans at most ceil(n_kt / (per - 1)) + 1 CTAs
+      const long long pieces = per > 1 ? (prm.n_kt + per - 2) / (per - 1) + 1 : prm.n_kt;
+      if (segs <= c->tc.max_seg && segs <= kMaxSegF && pieces <= kMaxPieces) fs.G = G;
+    }
+    attn_fwd_kernel<<<fs.G, kThreads, kSmemF, st>>>(qmap, kmap, vmap, fs);
     rc = check_launch("attn_fwd_kernel");
     if (rc) return rc;
+    if (fs.G != grid) {
+      combine_fwd_kernel<<<dim3(grid, 2 * BM * (D / 4) / 256), 256, 0, st>>>(fs);
+      rc = check_launch("combine_fwd_kernel");
+      if (rc) return rc;
+    }
     // the score sums over equal shares of (pair, K tile) units, one CTA per SM
     SplitParams ss{};
     ss.t = prm;

@@ -46,9 +46,9 @@ QCASES = [
 ]
 
 
-# Shapes whose one-CTA-per-pair grid would leave most SMs idle: the two passes run as
-# persistent kernels over equal shares of (pair, K/V tile) units, most pairs split over
-# several CTAs (partial LSE combined, partial outputs summed).
+# Shapes whose one-CTA-per-pair grid would leave most SMs idle: the kernels run over
+# equal shares of (pair, K/V tile) units, most pairs split over several CTAs (partial
+# maxima, sums and outputs combined).
 SPLIT_CASES = [
     tc("tc_split_c8192_s512", capacity=8192, chunk=512, seq_len=9216),
     tc("tc_split_c8000_s300_ragged", capacity=8000, chunk=300, seq_len=8600),
@@ -57,6 +57,15 @@ SPLIT_CASES = [
 
 @pytest.mark.parametrize("wl", SPLIT_CASES, ids=[w.name for w in SPLIT_CASES])
 def test_split_schedule(wl, cuda_device):
+    last = wl.n_chunks - 1
+    run, n = run_and_check(wl, cuda_device, check_chunks={0, last - 1, last})
+    assert n == 3
+
+
+@pytest.mark.parametrize("wl", SPLIT_CASES, ids=[w.name for w in SPLIT_CASES])
+def test_split_schedule_fused_kernel(wl, cuda_device, monkeypatch):
+    """The fused kernel's own split schedule (phase A / phase B persistent kernels)."""
+    monkeypatch.setenv("H2OKV_TC_FUSED", "1")
     last = wl.n_chunks - 1
     run, n = run_and_check(wl, cuda_device, check_chunks={0, last - 1, last})
     assert n == 3
