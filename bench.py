@@ -133,16 +133,16 @@ def kernel_source_hash(files=None):
     return h.hexdigest()[:16]
 
 
-def recorded_traffic(kernel_name):
+def recorded_traffic(kernel_name, config):
     """DRAM bytes per launch from the committed ncu summary, if it was taken on
-    the current sources of that kernel (else None)."""
+    the current sources of that kernel and on this workload (else None)."""
     p = os.path.join(ROOT, "profiles", "dram_traffic.json")
     if not os.path.exists(p):
         return None
     with open(p) as f:
         d = json.load(f)
     e = d.get(kernel_name)
-    if not e or e.get("source_hash") != kernel_source_hash(e.get("sources")):
+    if not e or e.get("config") != config or e.get("source_hash") != kernel_source_hash(e.get("sources")):
         return None
     return e.get("bytes_per_launch")
 
@@ -287,7 +287,8 @@ def run_ours(args, wl, ws, rank, local):
     if tc_used:
         roof = {"bound": "tensor", "achieved": round(tflops_alg, 2), "peak": tc_peak,
                 "unit": "TFLOP/s", "frac": round(tflops_alg / tc_peak, 4),
-                "traffic": recorded_traffic("attn_fwd_kernel" if two_pass and n_split == 0 else "attn_tc_kernel"),
+                "traffic": recorded_traffic("attn_fwd_kernel" if two_pass and n_split == 0 else "attn_tc_kernel",
+                                            args.config),
                 "kernel": ("attention call per chunk (attn_split_a_kernel + attn_split_b_kernel + "
                            "reduce_o_kernel + reduce_w_kernel)") if n_split == wl.n_chunks else
                           (("attention call per chunk (attn_fwd_kernel + %sscoresum_kernel + reduce_w_kernel)"
@@ -301,7 +302,7 @@ def run_ours(args, wl, ws, rank, local):
         fma_peak = 148 * 128 * 2 * 1.965e9 / 1e12
         roof = {"bound": "alu", "achieved": round(tflops_alg, 2), "peak": round(fma_peak, 1),
                 "unit": "TFLOP/s", "frac": round(tflops_alg / fma_peak, 4),
-                "traffic": recorded_traffic("simt_attn_kernel"),
+                "traffic": recorded_traffic("simt_attn_kernel", args.config),
                 "kernel": "attention call per chunk, CUDA-core path (2 passes)",
                 "alg_flops_per_launch": per_launch_alg, "avg_launch_ms": round(per_launch_ms, 4),
                 "peak_kind": "derived: 148 SMs x 128 FP32 FMA/clk x 2 x 1965 MHz"}
