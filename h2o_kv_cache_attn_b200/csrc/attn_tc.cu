@@ -1336,6 +1336,12 @@ enum {
   G_END
 };
 constexpr uint32_t S_OFF_TMEM = S_OFF_BAR + G_END * 8;
+// pass 2: 4 control warps + 4 softmax warpgroups at 96 registers (640 x 96 = 61440); the
+// control warps drop to 64, the softmax warps (half a column of 64 logits at a time)
+// rise to 104: 128 x 64 + 512 x 104 = 61440
+constexpr int kThreadsS = 640;
+constexpr int kLaunchRegsS = 96, kCtrlRegsS = 64, kSoftRegsS = 104;
+static_assert(128 * kCtrlRegsS + 512 * kSoftRegsS == kThreadsS * kLaunchRegsS, "pass 2 register split");
 constexpr uint32_t kSmemS = S_OFF_TMEM + 16;
 static_assert(kSmemS <= 232448, "pass 2 shared memory budget");
 
@@ -1492,8 +1498,10 @@ __device__ __forceinline__ SegIter seg_iter(const SplitParams &sp) {
 // Pass 2 over equal shares of the (pair, K tile) units: CTA c takes units
 // [U c / G, U (c + 1) / G) in segments of one pair each, so that all
 // SMs are busy whatever the number of pairs; each (row tile, slot) sum is written by
-// exactly one CTA.  With G = pairs every CTA takes one whole pair.
-__global__ void __launch_bounds__(kThreads, 1)
+// exactly one CTA.  With G = pairs every CTA takes one whole pair.  Four softmax
+// warpgroups: (tile, S^T buffer parity), so that each takes every other K tile of its
+// query tile and four of them share each SM sub-partition's exponential unit.
+__global__ void __launch_bounds__(kThreadsS, 1)
     scoresum_kernel(const __grid_constant__ CUtensorMap q_map,
                     const __grid_constant__ CUtensorMap k_map, const SplitParams sp) {
   const TcParams &p = sp.t;
@@ -1520,8 +1528,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(&bar[G_SFREE0 + i], 8);  // both softmax warpgroups, with or without a tile
     }
     mbar_init(&bar[G_QFREE], 1);
-    mbar_init(&bar[G_NL0], 4);
-    mbar_init(&bar[G_NL0 + 1], 4);
+    mbar_init(&bar[G_NL0], 8);  // both warpgroups of a tile
+    mbar_init(&bar[G_NL0 + 1], 8);
     mbar_init(&bar[G_DRAIN], 1);
     fence_mbar_init();
   }
@@ -1552,7 +1560,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   };
 
   if (warp < 4) {
-    reg_dealloc<kCtrlRegs>();
+    reg_dealloc<kCtrlRegsS>();
     if (warp == 1) {
       // ------------------------------------------------------------------ MMA issuer
       // S^T_t(i) = K Q_t^T of the CTA's i-th unit into columns 256 (i & 1) + 128 t
@@ -1631,10 +1639,11 @@ __global__ void __launch_bounds__(kThreads, 1)
       __syncwarp();
     }
   } else {
-    reg_alloc<kSoftRegs>();
+    reg_alloc<kSoftRegsS>();
     // ------------------------------------- column sums, one thread per slot of a tile
-    const int t = (warp - 4) >> 2;
-    const int st = threadIdx.x - 128 * (1 + t);
+    const int wg = (warp - 4) >> 2;
+    const int t = wg & 1, par = wg >> 1;  // query tile; parity of the units (S^T buffer) taken
+    const int st = threadIdx.x & 127;
     const uint32_t lane_base = (uint32_t)(32 * (warp & 3)) << 16;
     const float c2 = p.scale2;
     int i = 0, seg = 0, u = u_first;
@@ -1646,22 +1655,27 @@ __global__ void __launch_bounds__(kThreads, 1)
       // buffer seg & 1 only after all its threads have written (so finished reading)
       // the other one
       float *nl = nlse_s + ((seg & 1) * 2 + t) * BM;
-      if (active) nl[st] = p.nlse[((size_t)bhq * p.tiles + tt) * BM + st];
+      if (active) nl[st] = p.nlse[((size_t)bhq * p.tiles + tt) * BM + st];  // both warpgroups: same value
       __syncwarp();
       if (lane == 0) mbar_arrive(&bar[G_NL0 + t]);
       if (!warp_wait(&bar[G_NL0 + t], seg & 1, lim)) { fail(p, aborted); break; }
       ++seg;
       const int rmax = min(BM, p.S - i0);
       float *pw = p.part_w + ((size_t)bhq * p.tiles + tt) * p.N_C;
-      // each slot's token position, read one K tile ahead (empty / outside slots: far)
+      // this warpgroup's K tiles: unit index i = i_seg + (kt - kt0) of parity par
+      const int i_seg = i;
+      i += kt1 - kt0;
+      const int kt_first = kt0 + ((par - i_seg) & 1);
+      // each slot's token position, read one of our K tiles ahead (empty / outside: far)
       const int32_t *tpg = p.token_pos + (size_t)pi.bg * p.N_C;
-      int32_t tp_next = kt0 * BN + st < p.N_C ? tpg[kt0 * BN + st] : kEmptyPos;
-      for (int kt = kt0; kt < kt1; ++kt, ++i) {
-        const int u = i & 1;
+      int32_t tp_next = kt_first < kt1 && kt_first * BN + st < p.N_C ? tpg[kt_first * BN + st] : kEmptyPos;
+      for (int kt = kt_first; kt < kt1; kt += 2) {
+        const int iu = i_seg + (kt - kt0);
+        const int u = iu & 1;
         const int j = kt * BN + st;
         const int32_t tp = tp_next;
-        if (kt + 1 < kt1) tp_next = j + BN < p.N_C ? tpg[j + BN] : kEmptyPos;
-        if (!warp_wait(&bar[G_SFULL0 + u], (i >> 1) & 1, lim)) { fail(p, aborted); break; }
+        if (kt + 2 < kt1) tp_next = j + 2 * BN < p.N_C ? tpg[j + 2 * BN] : kEmptyPos;
+        if (!warp_wait(&bar[G_SFULL0 + u], (iu >> 1) & 1, lim)) { fail(p, aborted); break; }
         tc_fence_after();
         if (active) {
           // visible rows r of this tile: tp - P <= i0 + r, r < rmax.  A slot that no row
@@ -2914,7 +2928,7 @@ int prepare_split_kernel(K kernel, int &ready_dev, const char *name) {
 
 // Shared-memory opt-in and register check of a bf16 two-pass kernel.
 template <typename K>
-int prepare_pass_kernel(K kernel, uint32_t smem_bytes, int &ready_dev, const char *name) {
+int prepare_pass_kernel(K kernel, uint32_t smem_bytes, int regs, int &ready_dev, const char *name) {
   int dev = 0;
   cudaGetDevice(&dev);
   if (ready_dev == dev) return H2OKV_OK;
@@ -2926,9 +2940,9 @@ int prepare_pass_kernel(K kernel, uint32_t smem_bytes, int &ready_dev, const cha
   e = cudaFuncGetAttributes(&fa, kernel);
   if (e != cudaSuccess)
     return set_error(H2OKV_ERR_CUDA, "cudaFuncGetAttributes(%s): %s", name, cudaGetErrorString(e));
-  if (fa.numRegs != kLaunchRegs)
+  if (fa.numRegs != regs)
     return set_error(H2OKV_ERR_UNSUPPORTED, "%s built with %d registers per thread, expected %d",
-                     name, fa.numRegs, kLaunchRegs);
+                     name, fa.numRegs, regs);
   ready_dev = dev;
   return H2OKV_OK;
 }
@@ -3032,9 +3046,9 @@ int launch_attn_tc(h2okv_cache *c, const void *q, int S, int64_t P, void *y, flo
   if (d.kv_dtype == H2OKV_BF16 && c->tc.two_pass) {
     // attention with an online softmax, then the score sums against the final LSE
     static thread_local int ready_f = -1, ready_s = -1;
-    rc = prepare_pass_kernel(attn_fwd_kernel, kSmemF, ready_f, "attn_fwd_kernel");
+    rc = prepare_pass_kernel(attn_fwd_kernel, kSmemF, kLaunchRegs, ready_f, "attn_fwd_kernel");
     if (rc) return rc;
-    rc = prepare_pass_kernel(scoresum_kernel, kSmemS, ready_s, "scoresum_kernel");
+    rc = prepare_pass_kernel(scoresum_kernel, kSmemS, kLaunchRegsS, ready_s, "scoresum_kernel");
     if (rc) return rc;
     // attention over equal shares of (pair, K/V tile) units, one CTA per SM when the
     // partial-result workspace holds every CTA's pieces, else one CTA per pair
@@ -3071,7 +3085,7 @@ int launch_attn_tc(h2okv_cache *c, const void *q, int S, int64_t P, void *y, flo
     ss.t = prm;
     ss.U = (long long)grid * prm.n_kt;
     ss.G = (int)min((long long)max(c->tc.sms, 1), ss.U);
-    scoresum_kernel<<<ss.G, kThreads, kSmemS, st>>>(qmap, kmap, ss);
+    scoresum_kernel<<<ss.G, kThreadsS, kSmemS, st>>>(qmap, kmap, ss);
     rc = check_launch("scoresum_kernel");
     if (rc) return rc;
     dim3 rgrid((d.capacity + 255) / 256, d.batch * d.n_kv_heads);
