@@ -53,9 +53,14 @@ SPLIT_CASES = [
     tc("tc_split_c8192_s512", capacity=8192, chunk=512, seq_len=9216),
     tc("tc_split_c8000_s300_ragged", capacity=8000, chunk=300, seq_len=8600),
 ]
+# an odd number of query tiles per KV group: the last pair of each group has no second
+# tile, so some segments run one tile (split attention pass, score sums, combination)
+SPLIT_ODD_CASES = [
+    tc("tc_split_mha_c8192_s300_odd_tiles", Hq=2, Hk=2, capacity=8192, chunk=300, seq_len=8900),
+]
 
 
-@pytest.mark.parametrize("wl", SPLIT_CASES, ids=[w.name for w in SPLIT_CASES])
+@pytest.mark.parametrize("wl", SPLIT_CASES + SPLIT_ODD_CASES, ids=[w.name for w in SPLIT_CASES + SPLIT_ODD_CASES])
 def test_split_schedule(wl, cuda_device):
     last = wl.n_chunks - 1
     run, n = run_and_check(wl, cuda_device, check_chunks={0, last - 1, last})
