@@ -18,6 +18,7 @@ from __future__ import annotations
 
 import argparse
 import hashlib
+import re
 import json
 import os
 import statistics
@@ -120,16 +121,24 @@ class ClockSampler:
 
 
 # --------------------------------------------------------------------------- #
+def strip_comments(code: str) -> str:
+    """C/C++ source without comments and blank lines, each line stripped (string
+    literals are kept as they are; none of the kernels' contains a comment marker)."""
+    code = re.sub(r"/\*.*?\*/", "", code, flags=re.S)
+    code = re.sub(r"//[^\n]*", "", code)
+    return "\n".join(line.strip() for line in code.splitlines() if line.strip())
+
+
 def kernel_source_hash(files=None):
-    """Hash of the CUDA sources a kernel is built from (all of csrc/ when files is
-    None); paths are relative to csrc/."""
+    """Hash of the code (comments excluded) of the CUDA sources a kernel is built from
+    (all of csrc/ when files is None); paths are relative to csrc/."""
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "h2o_kv_cache_attn_b200", "csrc")
     if files is None:
         files = sorted(f for f in os.listdir(csrc) if f.endswith((".cu", ".cuh")))
     for f in files:
-        with open(os.path.normpath(os.path.join(csrc, f)), "rb") as fh:
-            h.update(os.path.basename(f).encode() + fh.read())
+        with open(os.path.normpath(os.path.join(csrc, f)), encoding="utf-8") as fh:
+            h.update(os.path.basename(f).encode() + strip_comments(fh.read()).encode())
     return h.hexdigest()[:16]
 
 

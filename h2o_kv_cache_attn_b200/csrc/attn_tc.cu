@@ -4,41 +4,32 @@
 // per KV slot and summed over the q_g query heads of each GQA group; §4 / Table
 // 1 8- and 4-bit caches).
 //
-// One CTA owns two 128-row query tiles (a, b) of one KV group (two row tiles of
+// A CTA owns two 128-row query tiles (a, b) of one KV group (two row tiles of
 // one head, or the same rows of two heads); rows past S are zero-filled by TMA
-// and never written.  It streams the group's K/V twice, each 128-slot tile once
-// for both query tiles (half the bytes per FLOP of one tile per CTA):
+// and never written.  Each 128-slot K/V tile is read once for both query tiles.
+// The warp roles: warp 0 loads Q and K tiles (cp.async.bulk.tensor, no multicast)
+// and the slots' token positions, warp 2 loads V tiles, warp 1 allocates TMEM and
+// issues every MMA from one thread, warps 4-7 (tile a) and 8-11 (tile b) own TMEM
+// lanes 32(w%4)..32(w%4)+31 for the softmax, the column sums and the epilogue.
 //
-//   phase A  S = Q K^T (tcgen05.mma, M=128 rows, N=128 slots, K=128, fp32 in
-//            TMEM) for a and b; one softmax thread per row keeps the online
-//            max / sum of its rows of a and b -> base-2 log-sum-exp.
-//   phase B  S^T = K Q^T (M=128 slots, N=128 rows) for a and b: one thread per
-//            SLOT reads its 128 logits, forms p = exp2(s*log2e/sqrt(d) - lse2_i)
-//            with the FINAL row LSE, sums them in registers (the slot's summed
-//            weight over the tile's rows: no atomics, deterministic) and writes
-//            p as bf16 into shared memory (the MN-major A operand), then
-//            O += P V (A = P, B = V, both MN-major).  P is normalised already,
-//            so O needs no rescaling.  TMEM: S^T_a, S^T_b, O_a, O_b.
-//
-// Warp roles (384 threads): warp 0 loads Q and K tiles (cp.async.bulk.tensor, no
-// multicast) and turns the slots' token positions into positions relative to the
-// chunk (floats, for arithmetic masking) through a four-stage (phase A) and a
-// two-stage (phase B) ring, warp 2
-// loads V tiles through its own two-stage ring, warp 1 allocates TMEM and issues
-// every MMA from one thread, warps 4-7
-// (tile a) and 8-11 (tile b) softmax / column sums / epilogue (warp w owns
-// TMEM lanes 32(w%4)..32(w%4)+31).  The single P buffer is handed over
-// a(kt) -> b(kt) -> a(kt+1) through per-tile full / free barriers.
-// The MMA issue order S^T_a(kt+1), S^T_b(kt+1), PV_a(kt), PV_b(kt) lets the tensor
-// pipe compute the next logits while the softmax warps turn the current ones
-// into P.
-// Quantized caches (int8 / int4 codes with one fp16 scale per slot): warps 0, 2
-// and 3 replace the TMA producers: one thread stages each tile of codes by a bulk
-// copy, all 96 dequantize it in place (see convert_i8 / convert_i4): key tiles
-// become exact bf16 integers and the key scale s_j
-// multiplies the logits of slot j (a column scale of S in phase A, a per-thread
-// factor in phase B), so scores and summed weights see the stored keys exactly;
-// value tiles are stored as bf16(code * scale).
+// bf16 caches run two passes:
+//   attn_fwd_kernel   S = Q K^T (tcgen05.mma, M=128 rows, N=128 slots, fp32 in TMEM);
+//                     online softmax per row against a lazily moved reference
+//                     maximum; P written over S in TMEM as bf16 pairs; O += P V
+//                     with P read from TMEM (A) and V from shared memory (B).
+//                     Writes y and -lse2 per row (combine_fwd_kernel merges the
+//                     pieces of pairs split over CTAs).
+//   scoresum_kernel   S^T = K Q^T (M=128 slots, N=128 rows): one thread per SLOT
+//                     forms p = exp2(s*log2e/sqrt(d) - lse2_i) with the FINAL row
+//                     LSE and sums them in registers (no atomics, deterministic),
+//                     over equal shares of the (pair, K tile) units on every SM.
+// attn_tc_kernel runs both phases in one CTA (phase A: online max / sum -> LSE;
+// phase B: S^T with the final LSE, column sums, P in shared memory, O += P V) and
+// serves the int8 / int4 caches: there warps 0, 2, 3 and 12-15 replace the TMA
+// producers, stage each tile of codes by a bulk copy and dequantize it in place
+// (see convert_i8 / convert_i4): key tiles become exact f16 integers and the key
+// scale s_j multiplies the logits of slot j, so scores and summed weights see the
+// stored keys exactly; value tiles are stored as bf16(code * scale).
 // Every wait is bounded; a timeout sets the cache's device status word and the
 // CTA drains its copies and MMAs before freeing TMEM.
 //
@@ -1376,16 +1367,19 @@ __device__ __forceinline__ float slot_colsum(const uint32_t (&r)[N], const float
   return s4.x + s4.y;
 }
 
-// ---- split scheduling (bf16 cache): the two passes as persistent kernels ----------
+// ---- split scheduling: kernels over equal shares of the (pair, K/V tile) units ---
 // With one CTA per pair of query tiles, a grid of P pairs fills ceil(P / SMs) waves
 // and leaves SMs idle in the last one (P = 128 on 148 SMs: 14 % idle).  Here the
 // (pair, K/V tile) units are cut into G contiguous ranges of equal length, one per SM,
-// so a pair's slots may be spread over two or three CTAs ("segments").  Kernel A runs
+// so a pair's slots may be spread over two or three CTAs ("segments").  The score-sum
+// pass always runs this way (every slot sum is written by one CTA); the attention pass
+// when the grid would leave a quarter of the SMs idle (its split pairs' (max, sum, O)
+// pieces merged by combine_fwd_kernel).  The fused kernel's own split: kernel A runs
 // phase A over each segment and stores the rows' partial (max, sum); kernel B combines
 // a pair's partials into the final row LSE, runs phase B over its segments and writes
 // y, or a partial O when the pair is split (the partials add up: P is already
-// normalised); a reduction sums the partial O's.  Requires an even number of query
-// tiles per KV group (every pair has two tiles).
+// normalised); a reduction sums the partial O's.  The fused split requires an even
+// number of query tiles per KV group (every pair has two tiles).
 struct SplitParams {
   TcParams t;
   int G;            // CTAs (one per SM)
