@@ -1,0 +1,68 @@
+"""CPU checks of the measurement helpers behind the bench line: the DRAM traffic of
+the dominant kernel is reported only when the committed ncu record was taken on the
+same kernel code and the same workload, and the code hash ignores comments."""
+
+import json
+import os
+
+import pytest
+
+import bench
+
+
+def _fake_tree(tmp_path, kernel_src):
+    csrc = tmp_path / "h2o_kv_cache_attn_b200" / "csrc"
+    csrc.mkdir(parents=True)
+    (tmp_path / "include").mkdir()
+    (csrc / "k.cu").write_text(kernel_src)
+    (tmp_path / "include" / "h.h").write_text("int f(void);\n")
+    (tmp_path / "profiles").mkdir()
+    return ["k.cu", "../../include/h.h"]
+
+
+def test_strip_comments():
+    src = "int a; // one\n/* two\n three */ int b;\n\n   int c;  /* four */\n"
+    assert bench.strip_comments(src) == "int a;\nint b;\nint c;"
+
+
+def test_source_hash_ignores_comments_only(tmp_path, monkeypatch):
+    files = _fake_tree(tmp_path, "__global__ void k() { int x = 1; }\n")
+    monkeypatch.setattr(bench, "ROOT", str(tmp_path))
+    h0 = bench.kernel_source_hash(files)
+    (tmp_path / "h2o_kv_cache_attn_b200" / "csrc" / "k.cu").write_text(
+        "// a kernel\n/* its\n   description */\n__global__ void k() { int x = 1; }  // one\n\n")
+    assert bench.kernel_source_hash(files) == h0
+    (tmp_path / "h2o_kv_cache_attn_b200" / "csrc" / "k.cu").write_text(
+        "__global__ void k() { int x = 2; }\n")
+    assert bench.kernel_source_hash(files) != h0
+
+
+def test_recorded_traffic_requires_same_code_and_workload(tmp_path, monkeypatch):
+    files = _fake_tree(tmp_path, "__global__ void k() {}\n")
+    monkeypatch.setattr(bench, "ROOT", str(tmp_path))
+    rec = {"k": {"bytes_per_launch": 1234, "config": "128k", "sources": files,
+                 "source_hash": bench.kernel_source_hash(files)}}
+    (tmp_path / "profiles" / "dram_traffic.json").write_text(json.dumps(rec))
+    assert bench.recorded_traffic("k", "128k") == 1234
+    assert bench.recorded_traffic("k", "64k") is None        # another workload
+    assert bench.recorded_traffic("other", "128k") is None   # no record
+    (tmp_path / "h2o_kv_cache_attn_b200" / "csrc" / "k.cu").write_text("__global__ void k() { }\n;")
+    assert bench.recorded_traffic("k", "128k") is None       # the kernel's code changed
+
+
+def test_committed_traffic_record_matches_current_kernels():
+    """The record committed under profiles/ was taken on the kernel code as it stands."""
+    with open(os.path.join(bench.ROOT, "profiles", "dram_traffic.json")) as f:
+        rec = json.load(f)
+    assert "attn_fwd_kernel" in rec
+    for name, e in rec.items():
+        assert e["source_hash"] == bench.kernel_source_hash(e["sources"]), name
+        assert e["bytes_per_launch"] == e["dram_bytes_read"] + e["dram_bytes_write"]
+
+
+@pytest.mark.parametrize("config", ["128k", "64k"])
+def test_algorithmic_flops(config):
+    wl = bench.SHORT[config]
+    n = wl.capacity
+    assert bench.alg_flops_chunk(wl, n, wl.chunk) == 4.0 * wl.B * wl.Hq * wl.chunk * n * wl.d
+    assert bench.exec_flops_chunk(wl, n, wl.chunk) == 1.5 * bench.alg_flops_chunk(wl, n, wl.chunk)
