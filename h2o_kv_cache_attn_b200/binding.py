@@ -27,7 +27,7 @@ EXPORTED = ("kv_cache_query_sizes", "kv_cache_create", "kv_cache_reset", "kv_cac
             "attn_chunk_with_scoresum", "kv_cache_device_status", "kv_cache_set_wait_timeout",
             "attn_chunk_with_scoresum_noalloc", "h2okv_last_error", "h2okv_abi_version",
             "kv_cache_set_score_mode", "h2o_evict_insert_delta", "h2o_insert_at",
-            "kv_cache_restore", "attn_chunk_backward")
+            "kv_cache_restore", "attn_chunk_backward", "h2o_evict_insert_many")
 SCORE_MODE = {"h2o": 0, "h2o_norm": 1, "h2o_orig": 2}
 
 
@@ -95,6 +95,9 @@ def load() -> ctypes.CDLL:
         "h2o_insert_at": (ctypes.c_int, [vp, vp, vp, vp, i32, i64, vp, ctypes.POINTER(Delta), vp]),
         "kv_cache_restore": (ctypes.c_int, [vp, vp, i32, ctypes.POINTER(Delta), vp]),
         "attn_chunk_backward": (ctypes.c_int, [vp, vp, vp, vp, i32, i64, vp, vp, vp, vp]),
+        "h2o_evict_insert_many": (ctypes.c_int, [ctypes.POINTER(vp), i32, ctypes.POINTER(vp),
+                                                 ctypes.POINTER(vp), ctypes.POINTER(vp), i32, i64,
+                                                 ctypes.POINTER(vp), vp]),
         "h2okv_last_error": (ctypes.c_char_p, []),
         "h2okv_abi_version": (i32, []),
     }
@@ -170,6 +173,32 @@ def kv_cache_quantize(kv_dtype: str, x: torch.Tensor, codes: torch.Tensor, scale
 def h2o_evict_insert(handle, w_prev, k_new, v_new, S: int, P: int, slots_out=None, stream=None):
     _check(load().h2o_evict_insert(handle, _ptr(w_prev), _ptr(k_new), _ptr(v_new), int(S), int(P),
                                    _ptr(slots_out), _stream(stream)))
+
+
+def _ptr_array(items):
+    """A C array of void* from handles / tensors / None (None stays NULL), or NULL for None."""
+    if items is None:
+        return None
+    vals = []
+    for x in items:
+        if x is None:
+            vals.append(None)
+        elif isinstance(x, torch.Tensor):
+            vals.append(_ptr(x).value)
+        elif isinstance(x, ctypes.c_void_p):
+            vals.append(x.value)
+        else:
+            vals.append(int(x))
+    return (ctypes.c_void_p * len(vals))(*vals)
+
+
+def h2o_evict_insert_many(handles, w_prev, k_new, v_new, S: int, P: int, slots_out=None,
+                          stream=None):
+    """h2o_evict_insert on several caches of one shape in one call (lists of the
+    per-cache arguments; w_prev / slots_out may be None)."""
+    _check(load().h2o_evict_insert_many(_ptr_array(handles), len(handles), _ptr_array(w_prev),
+                                        _ptr_array(k_new), _ptr_array(v_new), int(S), int(P),
+                                        _ptr_array(slots_out), _stream(stream)))
 
 
 def kv_cache_set_score_mode(handle, mode: str):

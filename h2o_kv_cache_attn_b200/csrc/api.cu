@@ -75,6 +75,14 @@ static void layout(const h2okv_cache_desc &d, const TcPlan &tc, WorkspaceLayout 
   off = align256(off + B * Hq * S * 4);
   ws->status = off;
   off = align256(off + 4);
+  const size_t G = (size_t)d.batch * d.n_kv_heads;
+  ws->ev_hist = off;
+  off = align256(off + G * 2048 * 4);
+  ws->ev_arrive = off;
+  off = align256(off + G * 4);
+  ws->ev_zero_end = off;
+  ws->ev_slots = off;
+  off = align256(off + G * S * 4);
   ws->part_ml = ws->part_w = ws->part_o = ws->nlse = off;
   if (tc.enabled) {
     const size_t seg_rows = (size_t)tc.split_ctas * tc.max_seg * 2 * 128;
@@ -157,6 +165,14 @@ int kv_cache_create(const h2okv_cache_desc *desc, const h2okv_cache_buffers *buf
   c->tc.maps_ready = false;
   c->wait_timeout_ns = kDefaultWaitTimeoutNs;
   c->score_mode = H2OKV_SCORE_H2O;
+  {
+    int dev = 0, sms = 0;
+    c->sms = (cudaGetDevice(&dev) == cudaSuccess &&
+              cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) == cudaSuccess)
+                 ? sms
+                 : 0;
+    cudaGetLastError();
+  }
   layout(*desc, c->tc, &c->ws);
   // The attention kernels read every slot and mask the empty ones arithmetically,
   // which needs finite values there: start from zeroed rows and scales.
@@ -275,6 +291,50 @@ int h2o_evict_insert(h2okv_cache *c, const float *w_prev, const void *k_new, con
   c->n_filled = c->n_filled + S > c->desc.capacity ? c->desc.capacity : c->n_filled + S;
   // the policy fills slots left to right before it evicts
   if (c->n_filled > c->n_span) c->n_span = c->n_filled;
+  return H2OKV_OK;
+}
+
+int h2o_evict_insert_many(h2okv_cache *const *caches, int32_t n_caches,
+                          const float *const *w_prev, const void *const *k_new,
+                          const void *const *v_new, int32_t S, int64_t P,
+                          int32_t *const *slots_out, void *stream) {
+  g_err[0] = 0;
+  if (!caches || n_caches < 1) return set_error(H2OKV_ERR_INVALID_ARG, "no caches");
+  const h2okv_cache *c0 = caches[0];
+  if (!c0) return set_error(H2OKV_ERR_INVALID_ARG, "cache 0 is NULL");
+  if (S < 0 || S > c0->desc.max_chunk || S > c0->desc.capacity)
+    return set_error(H2OKV_ERR_INVALID_ARG, "S = %d outside [0, min(max_chunk %d, capacity %d)]",
+                     S, c0->desc.max_chunk, c0->desc.capacity);
+  if (P < 0 || P + S >= (int64_t)INT32_MAX)
+    return set_error(H2OKV_ERR_INVALID_ARG, "P = %lld out of range for int32 token positions",
+                     (long long)P);
+  if (S > 0 && (!k_new || !v_new))
+    return set_error(H2OKV_ERR_INVALID_ARG, "k_new and v_new are required when S > 0");
+  for (int i = 0; i < n_caches; ++i) {
+    const h2okv_cache *c = caches[i];
+    if (!c) return set_error(H2OKV_ERR_INVALID_ARG, "cache %d is NULL", i);
+    if (memcmp(&c->desc, &c0->desc, sizeof(c0->desc)) != 0 || c->n_filled != c0->n_filled ||
+        c->score_mode != c0->score_mode)
+      return set_error(H2OKV_ERR_INVALID_ARG,
+                       "cache %d differs from cache 0 in shape, fill level or score mode", i);
+    for (int j = 0; j < i; ++j)
+      if (caches[j] == c) return set_error(H2OKV_ERR_INVALID_ARG, "cache %d is listed twice", i);
+    if (S > 0 && (!k_new[i] || !v_new[i]))
+      return set_error(H2OKV_ERR_INVALID_ARG, "k_new[%d] / v_new[%d] is NULL", i, i);
+    if (S > 0 && (misaligned(k_new[i], 16) || misaligned(v_new[i], 16)))
+      return set_error(H2OKV_ERR_INVALID_ARG, "k_new and v_new must be 16-byte aligned");
+    if (w_prev && (!w_prev[i] || misaligned(w_prev[i], 4)))
+      return set_error(H2OKV_ERR_INVALID_ARG, "w_prev[%d] is NULL or misaligned", i);
+  }
+  if (S == 0 && !w_prev) return H2OKV_OK;
+  int rc = launch_evict_insert_many(caches, n_caches, w_prev, k_new, v_new, S, P, slots_out,
+                                    (cudaStream_t)stream);
+  if (rc) return rc;
+  for (int i = 0; i < n_caches; ++i) {
+    h2okv_cache *c = caches[i];
+    c->n_filled = c->n_filled + S > c->desc.capacity ? c->desc.capacity : c->n_filled + S;
+    if (c->n_filled > c->n_span) c->n_span = c->n_filled;
+  }
   return H2OKV_OK;
 }
 

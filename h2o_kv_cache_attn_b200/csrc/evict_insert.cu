@@ -4,34 +4,71 @@
 // §A.5.3 keys' = scatter(keys, index, key_new)), plus the 8/4-bit row
 // quantizer used on insert.
 //
-// One launch per call: evict_kernel runs a thread-block cluster of CL CTAs per
-// (b, h_k).  Each CTA holds a contiguous slice of the N_C slots in registers
-// (IPT consecutive slots per thread) and
-//   1. folds w_prev into the float32 scores and forms order-preserving uint32
-//      selection keys (0 for an empty slot, so empty slots come first);
-//   2. finds the S-th smallest key with a 4-pass, 8-bit radix select: each CTA
-//      builds a 256-bin histogram of its slice, the cluster sums them through
-//      distributed shared memory, every CTA picks the same bin;
-//   3. lists the chosen slots in slot order (token k -> k-th smallest slot):
-//      a block scan plus a cluster prefix of per-CTA counts gives each chosen
-//      slot its position; the slot of position k is sent to CTA k % CL;
-//   4. copies (or quantizes) the new key/value rows k = rank, rank + CL, ...
-//      into their slots.
-// While the cache is still filling (n_filled + S <= N_C) the slots are
-// n_filled + k and steps 2-3 are skipped.  No scratch memory in global memory.
-// The quantizer must agree bit for bit with an IEEE float32 reference: it uses
-// correctly rounded division, rintf and __float2half_rn only (this file is
-// never built with fast-math).
-#include <cooperative_groups.h>
+// One call = two launches on the caller's stream:
+//
+//   evict_select_kernel  C CTAs per group (a group is one (batch row, KV head),
+//     or one KV head over every batch row for the h2o_orig variant), each over
+//     a contiguous slice of the N_C slots:
+//       1. folds w_prev into the float32 scores and stores them; while the
+//          cache is filling (n_filled + S <= N_C) it also claims slots
+//          n_filled + k for the chunk rows k (token position, score 0);
+//       2. choosing: forms order-preserving uint32 selection keys (0 for an
+//          empty slot, so empty slots come first) and a 2048-bin histogram of
+//          their top 11 bits, adds it into the group's histogram in the
+//          workspace and counts itself in; the CTA that arrives last owns the
+//          rest of the choice: it finds the bin of the S-th smallest key,
+//          reads the group's keys back from L2 into shared memory, refines the
+//          threshold over bits 20..10 and 9..0 (two more histograms, only for
+//          keys in the chosen bins), lists the chosen slots in slot order with
+//          one block scan (ties at the threshold go to the lowest slots), and
+//          claims them; it leaves the histogram and counter at zero.
+//   evict_rows_kernel  launched as a programmatic dependent of the select
+//     kernel: it loads its first new key/value rows while the selection runs,
+//     then waits for it (griddepcontrol.wait) and writes (copies, or
+//     quantizes for 8/4-bit caches) every chunk row into its slot, with the
+//     overwritten row saved first for the delta encoding.
+//
+// A call over many caches of the same shape (independent layers) runs as the
+// same two launches over every (cache, group).  The quantizer must agree bit
+// for bit with an IEEE float32 reference: it uses correctly rounded division and
+// reciprocal, Markstein's correctly rounded quotient (quant_code) and __float2half_rn
+// only (this file is never built with fast-math).
+#include <mutex>
 
 #include "h2okv_internal.cuh"
+#include "tc_ptx.cuh"
 
 namespace h2okv {
 namespace {
+using namespace ptx;
 
-constexpr int kEvThreads = 256;   // threads per CTA of the eviction kernel
-constexpr int kEvictCluster = 8;  // CTAs per (b, h_k): a portable cluster size
-constexpr int kEvWarps = kEvThreads / 32;
+constexpr int kSelThreads = 512;  // threads of a select CTA
+constexpr int kTopBits = 11;  // bits of the first histogram (key bits 31..21)
+constexpr int kHistBins = 1 << kTopBits;
+constexpr int kMidBins = 2048;  // key bits 20..10
+constexpr int kLowBins = 1024;  // key bits 9..0
+constexpr int kSmemKeysMax = 32768;  // largest N_C whose keys the last CTA keeps in shared memory
+constexpr int kSlotListMax = 4096;   // chosen slots the last CTA lists in shared memory
+constexpr int kRowThreads = 256;     // threads of a row CTA
+constexpr int kRowWarps = kRowThreads / 32;
+constexpr int kCopyUnroll = 8;   // 16-byte pieces per thread in flight in the row copy
+constexpr int kQuantUnroll = 4;  // rows per lane segment in flight in the row quantizer
+
+// ---- quantizer arithmetic ------------------------------------------------------------
+// code = clamp(rint(x / s), -qmax, qmax) with x / s the correctly rounded float32
+// quotient, without a division per element: Markstein's division (P. Markstein, IBM J.
+// Res. Dev. 34(1), 1990): with y = RN(1/s) (one per row), q0 = RN(x y) is within one ulp
+// of x / s, r = x - s q0 is exact (one FMA), and RN(q0 + r y) is RN(x / s).  The
+// quotient is clamped first (which commutes with rounding to an integer for integer
+// bounds), then rounded to nearest-even by adding and removing 1.5 * 2^23 (exact for
+// |q| < 2^22).  For s > 0 only (scale 0 gives codes 0).
+__device__ __forceinline__ int quant_code(float x, float s, float y, float qmax) {
+  const float q0 = __fmul_rn(x, y);
+  const float r = __fmaf_rn(-q0, s, x);
+  float q = __fmaf_rn(r, y, q0);
+  q = fminf(fmaxf(q, -qmax), qmax);
+  return __float_as_int(__fadd_rn(q, 12582912.f)) - 0x4B400000;
+}
 
 // Unsigned key with the order of the float: -0 and +0 map to the same key;
 // every non-NaN score maps to a key >= 1 so that 0 can mark an empty slot.
@@ -41,33 +78,689 @@ __device__ __forceinline__ uint32_t order_key(float s) {
   return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
 }
 
-// Block-wide exclusive scan of one uint32 per thread (blockDim.x == kEvThreads).
-__device__ __forceinline__ uint32_t block_exclusive_scan(uint32_t v, uint32_t *warp_tot,
-                                                         uint32_t *total) {
+__device__ __forceinline__ void griddep_launch_dependents() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+__device__ __forceinline__ void griddep_wait() {
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+}
+
+// One cache of a call: its buffers, the caller's chunk buffers and its workspace.
+struct EvTarget {
+  float *scores;
+  const float *w_prev;
+  int32_t *token_pos;
+  const uint8_t *k_new, *v_new;
+  uint8_t *keys, *values;
+  __half *k_scales, *v_scales;
+  int32_t *slots_out;
+  const int32_t *slots_in;  // replay: the slots to write (mode 3)
+  uint8_t *dk, *dv;         // delta outputs (or null): overwritten rows [B][H_k][S][row bytes]
+  __half *dks, *dvs;        //   their scales (quantized caches)
+  int32_t *dpos;            //   their token positions [B][H_k][S]
+  uint32_t *hist;           // workspace: [groups][kHistBins] top-bit histograms, zero between calls
+  uint32_t *arrive;         // workspace: [groups] arrival counters, zero between calls
+  int32_t *slotlist;        // workspace: [groups][S] chosen slots in slot order (mode 2)
+  int *status;              // device status word (replayed slot outside the cache)
+};
+
+template <int NT>
+struct EvParams {
+  EvTarget t[NT];
+  int n_targets;
+  int G;            // groups per cache: B * H_k, or H_k (h2o_orig: every batch row together)
+  int nb;           // batch rows per group (1, or B for h2o_orig)
+  int Hk, N_C, S, P, n_filled, d;
+  int mode;         // 0 fold only (S = 0), 1 fill, 2 choose, 3 replay
+  int score_mode;   // h2okv_score_mode
+  int need_tp;      // the selection keys read token positions (empty slots, h2o_norm)
+  int vec;          // N_C % 4 == 0: 16-byte loads and stores of score / position vectors
+  int C;            // select CTAs per group
+  int slice;        // slots per select CTA (a multiple of 4)
+  int row_bytes, in_row_bytes;
+  uint64_t wait_ns;  // limit of the choose kernel's wait on its bulk copies
+};
+
+template <int NT>
+__device__ __forceinline__ size_t bh_of(const EvParams<NT> &p, int g, int bb) {
+  return p.nb > 1 ? (size_t)bb * p.Hk + g : (size_t)g;
+}
+
+// ---- vector helpers: 4 consecutive slots j4 .. j4+3 below `end` ------------------
+__device__ __forceinline__ void ld4(const float *base, int j4, int end, bool vec, float (&v)[4]) {
+  if (vec && j4 + 4 <= end) {
+    const float4 x = *reinterpret_cast<const float4 *>(base + j4);
+    v[0] = x.x; v[1] = x.y; v[2] = x.z; v[3] = x.w;
+  } else {
+#pragma unroll
+    for (int e = 0; e < 4; ++e) v[e] = j4 + e < end ? base[j4 + e] : 0.f;
+  }
+}
+__device__ __forceinline__ void ld4_cs(const float *base, int j4, int end, bool vec, float (&v)[4]) {
+  if (vec && j4 + 4 <= end) {
+    const float4 x = __ldcs(reinterpret_cast<const float4 *>(base + j4));
+    v[0] = x.x; v[1] = x.y; v[2] = x.z; v[3] = x.w;
+  } else {
+#pragma unroll
+    for (int e = 0; e < 4; ++e) v[e] = j4 + e < end ? __ldcs(base + j4 + e) : 0.f;
+  }
+}
+__device__ __forceinline__ void ld4i(const int32_t *base, int j4, int end, bool vec,
+                                     int32_t (&v)[4]) {
+  if (vec && j4 + 4 <= end) {
+    const int4 x = *reinterpret_cast<const int4 *>(base + j4);
+    v[0] = x.x; v[1] = x.y; v[2] = x.z; v[3] = x.w;
+  } else {
+#pragma unroll
+    for (int e = 0; e < 4; ++e) v[e] = j4 + e < end ? base[j4 + e] : kEmptyPos;
+  }
+}
+__device__ __forceinline__ void st4(float *base, int j4, int end, bool vec, const float (&v)[4]) {
+  if (vec && j4 + 4 <= end) {
+    *reinterpret_cast<float4 *>(base + j4) = make_float4(v[0], v[1], v[2], v[3]);
+  } else {
+#pragma unroll
+    for (int e = 0; e < 4; ++e)
+      if (j4 + e < end) base[j4 + e] = v[e];
+  }
+}
+
+// Shared-memory accesses by 32-bit shared addresses (explicit ld/st.shared).
+__device__ __forceinline__ int lds32(uint32_t a) {
+  int v;
+  asm volatile("ld.shared.u32 %0, [%1];" : "=r"(v) : "r"(a));
+  return v;
+}
+__device__ __forceinline__ void sts32(uint32_t a, int v) {
+  asm volatile("st.shared.u32 [%0], %1;" ::"r"(a), "r"(v) : "memory");
+}
+
+// Selection key of one slot from its (folded) score sum over the group's batch rows and
+// the token position of batch row 0.
+__device__ __forceinline__ uint32_t sel_key(float ksum, int32_t tp, int score_mode, int P) {
+  if (tp == kEmptyPos) return 0u;
+  if (score_mode == H2OKV_SCORE_H2O_NORM) {  // score / (P - t(b, h, j)), age at least 1
+    const int age = max(P - tp, 1);
+    ksum = __fdiv_rn(ksum, (float)age);
+  }
+  return order_key(ksum);
+}
+
+// Block-wide exclusive scan over NTHR threads (warp_tot: NTHR / 32 entries).
+template <int NTHR, typename T>
+__device__ __forceinline__ T block_exclusive_scan(T v, T *warp_tot) {
+  constexpr int kW = NTHR / 32;
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  uint32_t incl = v;
+  T incl = v;
 #pragma unroll
   for (int o = 1; o < 32; o <<= 1) {
-    uint32_t t = __shfl_up_sync(0xffffffffu, incl, o);
+    const T t = __shfl_up_sync(0xffffffffu, incl, o);
     if (lane >= o) incl += t;
   }
   if (lane == 31) warp_tot[warp] = incl;
   __syncthreads();
   if (warp == 0) {
-    uint32_t wv = lane < kEvWarps ? warp_tot[lane] : 0u;
-    uint32_t wincl = wv;
+    const T wv = lane < kW ? warp_tot[lane] : (T)0;
+    T wincl = wv;
 #pragma unroll
     for (int o = 1; o < 32; o <<= 1) {
-      uint32_t t = __shfl_up_sync(0xffffffffu, wincl, o);
+      const T t = __shfl_up_sync(0xffffffffu, wincl, o);
       if (lane >= o) wincl += t;
     }
-    if (lane < kEvWarps) warp_tot[lane] = wincl - wv;
-    if (lane == kEvWarps - 1) *total = wincl;
+    if (lane < kW) warp_tot[lane] = wincl - wv;
   }
   __syncthreads();
-  return warp_tot[warp] + incl - v;
+  const T r = warp_tot[warp] + incl - v;
+  __syncthreads();  // warp_tot may be reused right away
+  return r;
 }
-// ---- row quantizer ------------------------------------------------------------
+
+// The bin of hs[0 .. NBINS) that holds the kk-th smallest counted key (1-based): writes
+// res[0] = bin, res[1] = kk minus the keys in lower bins.
+template <int NTHR, int NBINS>
+__device__ __forceinline__ void find_bin(const uint32_t *hs, uint32_t kk, uint32_t *warp_tot,
+                                         uint32_t *res) {
+  constexpr int per = NBINS / NTHR;
+  const int t = threadIdx.x;
+  uint32_t loc = 0;
+#pragma unroll
+  for (int i = 0; i < per; ++i) loc += hs[t * per + i];
+  const uint32_t excl = block_exclusive_scan<NTHR, uint32_t>(loc, warp_tot);
+  if (excl < kk && kk <= excl + loc) {
+    uint32_t c = excl;
+#pragma unroll
+    for (int i = 0; i < per; ++i) {
+      const uint32_t h = hs[t * per + i];
+      if (c + h >= kk) {
+        res[0] = (uint32_t)(t * per + i);
+        res[1] = kk - c;
+        break;
+      }
+      c += h;
+    }
+  }
+  __syncthreads();
+}
+
+// Slot j of a group gets chunk row k: bookkeeping for every batch row of the group
+// (old position to the delta output, new position, score 0, slot list).
+template <int NT>
+__device__ __forceinline__ void claim(const EvParams<NT> &p, const EvTarget &T, int g, int j,
+                                      int k) {
+  for (int bb = 0; bb < p.nb; ++bb) {
+    const size_t bh = bh_of(p, g, bb);
+    const size_t gs = bh * p.N_C + j, rk = bh * p.S + k;
+    if (T.dpos) __stcg(T.dpos + rk, __ldcg(T.token_pos + gs));
+    __stcg(T.token_pos + gs, p.P + k);
+    __stcg(T.scores + gs, 0.f);
+    if (T.slots_out) __stcg(T.slots_out + rk, j);
+  }
+}
+
+// ---- fold kernel ---------------------------------------------------------------------
+// C CTAs per group, each over a slice of the slots: fold w_prev into the scores, claim
+// the fill slots (mode 1) and, for a choosing call (mode 2), add the slice's histogram of
+// the top 11 key bits into the group's histogram in the workspace.
+template <int NT>
+__global__ void __launch_bounds__(kSelThreads)
+    evict_fold_kernel(const __grid_constant__ EvParams<NT> p) {
+  griddep_launch_dependents();  // the choose / row kernel may be scheduled
+  const int unit = blockIdx.x / p.C, rank = blockIdx.x % p.C;
+  const int ti = unit / p.G, g = unit % p.G;
+  const EvTarget &T = p.t[ti];
+  const int tid = threadIdx.x;
+  const bool choose = p.mode == 2;
+  const bool vec = p.vec != 0;
+  __shared__ uint32_t hs[kHistBins];
+  if (choose) {
+    for (int i = tid; i < kHistBins; i += kSelThreads) hs[i] = 0u;
+    __syncthreads();
+  }
+  const int j_begin = rank * p.slice;
+  const int j_end = min(p.N_C, j_begin + p.slice);
+  const bool fold = T.w_prev != nullptr;
+  constexpr int U = 4;
+  const int stride = 4 * kSelThreads;
+  for (int j0 = j_begin + 4 * tid; j0 < j_end; j0 += stride * U) {
+    float ks[U][4];
+    int32_t tp[U][4];
+    for (int bb = 0; bb < p.nb; ++bb) {
+      const size_t base = bh_of(p, g, bb) * (size_t)p.N_C;
+      float sc[U][4], wp[U][4];
+#pragma unroll
+      for (int u = 0; u < U; ++u) {
+        const int j4 = j0 + stride * u;
+        ld4(T.scores + base, j4, j_end, vec, sc[u]);
+        if (fold) ld4_cs(T.w_prev + base, j4, j_end, vec, wp[u]);
+        if (bb == 0) {
+          if (choose && p.need_tp)
+            ld4i(T.token_pos + base, j4, j_end, vec, tp[u]);
+          else {
+#pragma unroll
+            for (int e = 0; e < 4; ++e) tp[u][e] = 0;
+          }
+        }
+      }
+#pragma unroll
+      for (int u = 0; u < U; ++u) {
+        const int j4 = j0 + stride * u;
+        if (j4 >= j_end) continue;
+        if (fold) {
+#pragma unroll
+          for (int e = 0; e < 4; ++e) sc[u][e] = __fadd_rn(sc[u][e], wp[u][e]);
+        }
+        bool store = fold;
+        if (p.mode == 1) {  // filling: chunk row k takes slot n_filled + k
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const int j = j4 + e, k = j - p.n_filled;
+            if (j < j_end && k >= 0 && k < p.S) {
+              sc[u][e] = 0.f;
+              store = true;
+              const size_t gs = base + j, rk = bh_of(p, g, bb) * p.S + k;
+              if (T.dpos) T.dpos[rk] = T.token_pos[gs];
+              T.token_pos[gs] = p.P + k;
+              if (T.slots_out) T.slots_out[rk] = j;
+            }
+          }
+        }
+        if (store) st4(T.scores + base, j4, j_end, vec, sc[u]);
+#pragma unroll
+        for (int e = 0; e < 4; ++e) ks[u][e] = bb == 0 ? sc[u][e] : __fadd_rn(ks[u][e], sc[u][e]);
+      }
+    }
+    if (choose) {
+#pragma unroll
+      for (int u = 0; u < U; ++u) {
+        const int j4 = j0 + stride * u;
+#pragma unroll
+        for (int e = 0; e < 4; ++e)
+          if (j4 + e < j_end)
+            atomicAdd(&hs[sel_key(ks[u][e], tp[u][e], p.score_mode, p.P) >> (32 - kTopBits)], 1u);
+      }
+    }
+  }
+  if (!choose) return;
+  __syncthreads();
+  uint32_t *gh = T.hist + (size_t)g * kHistBins;
+  for (int i = tid; i < kHistBins; i += kSelThreads) {
+    const uint32_t v = hs[i];
+    if (v) atomicAdd(gh + i, v);
+  }
+}
+
+// ---- choose kernel -------------------------------------------------------------------
+// One CTA per group (mode 2), launched as a programmatic dependent of the fold kernel.
+// It takes the group's histogram (and leaves zeros), finds the bin of the top 11 key bits
+// holding the S-th smallest key, and then works on two bitmasks over the slots: slots
+// whose key lies below that bin (all chosen) and slots whose key lies in it (the
+// candidates).  The threshold is refined over the candidates only (bits 20..10, 9..0),
+// the chosen candidates are added to the first mask (ties at the threshold: lowest slots
+// first), and each thread lists the chosen slots of its words in slot order after one
+// block scan of their counts.
+//   KM 2: the group's folded h2o scores are bulk-copied into shared memory (keys formed
+//         on read); KM 1: keys computed from L2 into shared memory (batch-row sums,
+//         positions, unaligned capacities); KM 0: keys read from L2 each time (N_C above
+//         what shared memory holds).
+constexpr int kChooseThreads = 1024;
+constexpr int kChooseWarps = kChooseThreads / 32;
+constexpr int kMaxWordsPerThread = 2;  // 32-slot words per thread: N_C <= 65536
+
+template <int NT>
+__device__ __forceinline__ uint32_t key_from_l2(const EvParams<NT> &p, const EvTarget &T, int g,
+                                                int j) {
+  float ks = 0.f;
+  for (int bb = 0; bb < p.nb; ++bb) {
+    const float sc = __ldcg(T.scores + bh_of(p, g, bb) * p.N_C + j);
+    ks = bb == 0 ? sc : __fadd_rn(ks, sc);
+  }
+  const int32_t tp = p.need_tp ? __ldcg(T.token_pos + bh_of(p, g, 0) * p.N_C + j) : 0;
+  return sel_key(ks, tp, p.score_mode, p.P);
+}
+
+template <int NT, int KM>
+__global__ void __launch_bounds__(kChooseThreads, 1)
+    evict_choose_kernel(const __grid_constant__ EvParams<NT> p) {
+  griddep_launch_dependents();  // the row kernel may start loading its inputs
+  const int ti = blockIdx.x / p.G, g = blockIdx.x % p.G;
+  const EvTarget &T = p.t[ti];
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  __shared__ uint32_t hs[kHistBins];
+  __shared__ uint32_t wscan[kChooseWarps];
+  __shared__ uint32_t res[4];
+  __shared__ __align__(8) uint64_t bar;
+  __shared__ uint32_t below_w[kChooseThreads * kMaxWordsPerThread];  // slots below the bin
+  __shared__ uint32_t cand_w[kChooseThreads * kMaxWordsPerThread];   // slots in the bin
+  extern __shared__ __align__(16) unsigned char dyn[];  // [kSlotListMax] slots, [N_C] keys
+  const uint32_t slist_a = smem_u32(dyn);
+  const uint32_t keys_a = slist_a + kSlotListMax * 4u;
+
+  const int n_words = (p.N_C + 31) >> 5;
+  if (KM == 2 && tid == 0) {
+    mbar_init(&bar, 1);
+    fence_mbar_init();
+  }
+  __syncthreads();
+  griddep_wait();  // the fold kernel's scores and histograms are complete
+  uint32_t *gh = T.hist + (size_t)g * kHistBins;
+  uint32_t hreg[kHistBins / kChooseThreads];
+#pragma unroll
+  for (int q = 0; q < kHistBins / kChooseThreads; ++q) hreg[q] = __ldcg(gh + tid + q * kChooseThreads);
+  if (KM == 2 && tid == 0) {
+    asm volatile("fence.proxy.async.global;" ::: "memory");
+    const uint32_t bytes = (uint32_t)p.N_C * 4u;
+    mbar_expect_tx(&bar, bytes);
+    const unsigned char *src =
+        reinterpret_cast<const unsigned char *>(T.scores + bh_of(p, g, 0) * p.N_C);
+    for (uint32_t off = 0; off < bytes; off += 16384u)
+      asm volatile(
+          "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
+          ::"r"(keys_a + off), "l"(src + off), "r"(bytes - off < 16384u ? bytes - off : 16384u),
+          "r"(smem_u32(&bar))
+          : "memory");
+    mbar_arrive(&bar);
+  }
+#pragma unroll
+  for (int q = 0; q < kHistBins / kChooseThreads; ++q) {
+    hs[tid + q * kChooseThreads] = hreg[q];
+    __stcg(gh + tid + q * kChooseThreads, 0u);
+  }
+  if (KM == 1) {
+#pragma unroll 1
+    for (int j = tid; j < p.N_C; j += kChooseThreads) sts32(keys_a + 4u * j, (int)key_from_l2(p, T, g, j));
+  }
+  __syncthreads();
+  // key of slot j
+#define KEY_AT(j)                                                                     \
+  (KM == 2 ? order_key(__int_as_float(lds32(keys_a + 4u * (uint32_t)(j))))            \
+           : KM == 1 ? (uint32_t)lds32(keys_a + 4u * (uint32_t)(j)) : key_from_l2(p, T, g, (j)))
+
+  // ---- the bin of the top 11 bits that holds the S-th smallest key -----------------------
+  find_bin<kChooseThreads, kHistBins>(hs, (uint32_t)p.S, wscan, res);
+  const uint32_t top = res[0];
+  uint32_t kk = res[1];
+  if (KM == 2) {
+    const bool ok = mbar_wait(&bar, 0, p.wait_ns);
+    if (__syncthreads_or(!ok)) {  // a copy that never lands: record it, drain, give up
+      if (tid == 0) {
+        atomicExch(T.status, H2OKV_ERR_TIMEOUT);
+        mbar_wait(&bar, 0, p.wait_ns);
+      }
+      __syncthreads();
+      return;
+    }
+  }
+
+  // ---- bitmasks: word w holds slots 32w .. 32w + 31, one per lane of a warp step --------
+#pragma unroll 4
+  for (int w = warp; w < n_words; w += kChooseWarps) {
+    const int j = 32 * w + lane;
+    const bool okj = j < p.N_C;
+    const uint32_t b = okj ? KEY_AT(j) >> (32 - kTopBits) : 0xffffffffu;
+    const uint32_t bm = __ballot_sync(0xffffffffu, b < top);
+    const uint32_t cm = __ballot_sync(0xffffffffu, b == top);
+    if (lane == 0) {
+      below_w[w] = bm;
+      cand_w[w] = cm;
+    }
+  }
+  for (int i = tid; i < kMidBins; i += kChooseThreads) hs[i] = 0u;
+  __syncthreads();
+
+  // ---- threshold: bits 20..10, then 9..0, of the candidates ------------------------------
+  // thread t owns words t * wpt .. t * wpt + wpt - 1 (slot order follows thread order)
+  const int wpt = (n_words + kChooseThreads - 1) / kChooseThreads;
+#pragma unroll
+  for (int q = 0; q < kMaxWordsPerThread; ++q) {
+    const int w = tid * wpt + q;
+    if (q >= wpt || w >= n_words) break;
+    for (uint32_t m = cand_w[w]; m; m &= m - 1u) {
+      const uint32_t key = KEY_AT(32 * w + __ffs(m) - 1);
+      atomicAdd(&hs[(key >> 10) & 2047u], 1u);
+    }
+  }
+  __syncthreads();
+  find_bin<kChooseThreads, kMidBins>(hs, kk, wscan, res);
+  const uint32_t pre = (top << 11) | res[0];  // key bits 31..10
+  kk = res[1];
+  for (int i = tid; i < kLowBins; i += kChooseThreads) hs[i] = 0u;
+  __syncthreads();
+#pragma unroll
+  for (int q = 0; q < kMaxWordsPerThread; ++q) {
+    const int w = tid * wpt + q;
+    if (q >= wpt || w >= n_words) break;
+    for (uint32_t m = cand_w[w]; m; m &= m - 1u) {
+      const uint32_t key = KEY_AT(32 * w + __ffs(m) - 1);
+      if ((key >> 10) == pre) atomicAdd(&hs[key & 1023u], 1u);
+    }
+  }
+  __syncthreads();
+  find_bin<kChooseThreads, kLowBins>(hs, kk, wscan, res);
+  const uint32_t Tk = (pre << 10) | res[0];  // take every key < Tk and the first k_eq keys == Tk
+  const uint32_t k_eq = res[1];
+
+  // ---- chosen words: below the bin, candidates < Tk, the first k_eq candidates == Tk -----
+  uint32_t lt[kMaxWordsPerThread], eq[kMaxWordsPerThread];
+  uint32_t n_eq = 0;
+#pragma unroll
+  for (int q = 0; q < kMaxWordsPerThread; ++q) {
+    lt[q] = 0u;
+    eq[q] = 0u;
+    const int w = tid * wpt + q;
+    if (q >= wpt || w >= n_words) continue;
+    lt[q] = below_w[w];
+    for (uint32_t m = cand_w[w]; m; m &= m - 1u) {
+      const int bit = __ffs(m) - 1;
+      const uint32_t key = KEY_AT(32 * w + bit);
+      if (key < Tk) lt[q] |= 1u << bit;
+      else if (key == Tk) eq[q] |= 1u << bit;
+    }
+    n_eq += __popc(eq[q]);
+  }
+  uint32_t eb = block_exclusive_scan<kChooseThreads, uint32_t>(n_eq, wscan);
+  uint32_t n_take = 0;
+#pragma unroll
+  for (int q = 0; q < kMaxWordsPerThread; ++q) {
+    for (uint32_t m = eq[q]; m && eb < k_eq; m &= m - 1u, ++eb) lt[q] |= m & (0u - m);
+    n_take += __popc(lt[q]);
+  }
+  uint32_t pos = block_exclusive_scan<kChooseThreads, uint32_t>(n_take, wscan);
+
+  // ---- the chosen slots in slot order ----------------------------------------------------
+  const bool list_smem = p.S <= kSlotListMax;
+  int32_t *slist = T.slotlist + (size_t)g * p.S;
+#pragma unroll
+  for (int q = 0; q < kMaxWordsPerThread; ++q) {
+    const int w = tid * wpt + q;
+    for (uint32_t m = lt[q]; m; m &= m - 1u, ++pos) {
+      const int j = 32 * w + __ffs(m) - 1;
+      if (list_smem) {
+        sts32(slist_a + 4u * pos, j);
+      } else {
+        __stcg(slist + pos, j);
+        claim(p, T, g, j, (int)pos);
+      }
+    }
+  }
+  if (list_smem) {
+    __syncthreads();
+#pragma unroll 1
+    for (int k = tid; k < p.S; k += kChooseThreads) {
+      const int j = lds32(slist_a + 4u * k);
+      __stcg(slist + k, j);
+      claim(p, T, g, j, k);
+    }
+  }
+}
+#undef KEY_AT
+
+// ---- row kernel ----------------------------------------------------------------------
+// blockIdx.y = row set = (cache, group, batch row in the group); blockIdx.x covers the
+// set's S chunk rows, key and value.
+template <int NT>
+struct RowSet {
+  const EvTarget *T;
+  size_t bh;        // (batch row, KV head) index of the set
+  int32_t *slist;   // the group's chosen slots (mode 2)
+};
+template <int NT>
+__device__ __forceinline__ RowSet<NT> row_set(const EvParams<NT> &p) {
+  const int set = blockIdx.y;
+  const int bb = set % p.nb, ug = set / p.nb;
+  const int g = ug % p.G, ti = ug / p.G;
+  RowSet<NT> r;
+  r.T = &p.t[ti];
+  r.bh = bh_of(p, g, bb);
+  r.slist = p.t[ti].slotlist + (size_t)g * p.S;
+  return r;
+}
+
+// Slot of chunk row k of a set (negative: skipped -- a replayed slot outside the cache).
+template <int NT>
+__device__ __forceinline__ int slot_of(const EvParams<NT> &p, const RowSet<NT> &rs, int k) {
+  if (p.mode == 1) return p.n_filled + k;
+  if (p.mode == 2) return __ldcg(rs.slist + k);
+  const int j = __ldg(rs.T->slots_in + rs.bh * p.S + k);
+  return (j >= 0 && j < p.N_C) ? j : -1;
+}
+
+// Replay: the bookkeeping of a logged slot (done once per chunk row, with its key row).
+template <int NT>
+__device__ __forceinline__ void replay_claim(const EvParams<NT> &p, const RowSet<NT> &rs, int k,
+                                             int j) {
+  const EvTarget &T = *rs.T;
+  if (j < 0) {
+    atomicExch(T.status, H2OKV_ERR_INVALID_ARG);
+    return;
+  }
+  const size_t gs = rs.bh * p.N_C + j, rk = rs.bh * p.S + k;
+  if (T.dpos) __stcg(T.dpos + rk, __ldcg(T.token_pos + gs));
+  __stcg(T.token_pos + gs, p.P + k);
+  __stcg(T.scores + gs, 0.f);
+}
+
+// f32 / bf16 caches: the set's rows are cut into 16-byte pieces (e = (2k + t) * PC + c),
+// consecutive threads take consecutive pieces, every thread keeps kCopyUnroll pieces in
+// flight.  The first pieces are loaded before the wait on the select kernel.
+template <int NT, bool DELTA>
+__device__ __forceinline__ void copy_rows(const EvParams<NT> &p) {
+  const RowSet<NT> rs = row_set(p);
+  const EvTarget &T = *rs.T;
+  const int PC = p.row_bytes / 16;
+  const int total = p.S * 2 * PC;
+  const int nthr = gridDim.x * kRowThreads;
+  const int first = blockIdx.x * kRowThreads + threadIdx.x;
+  const uint4 *src_k = reinterpret_cast<const uint4 *>(T.k_new + rs.bh * p.S * (size_t)p.in_row_bytes);
+  const uint4 *src_v = reinterpret_cast<const uint4 *>(T.v_new + rs.bh * p.S * (size_t)p.in_row_bytes);
+  uint4 *dst_k = reinterpret_cast<uint4 *>(T.keys + rs.bh * p.N_C * (size_t)p.row_bytes);
+  uint4 *dst_v = reinterpret_cast<uint4 *>(T.values + rs.bh * p.N_C * (size_t)p.row_bytes);
+  uint4 r[kCopyUnroll];
+  int rr[kCopyUnroll];  // 2k + t of each piece (-1: none)
+  int cc[kCopyUnroll];
+  auto load = [&](int base) {
+#pragma unroll
+    for (int u = 0; u < kCopyUnroll; ++u) {
+      const int e = base + u * nthr;
+      rr[u] = -1;
+      if (e < total) {
+        rr[u] = e / PC;
+        cc[u] = e - rr[u] * PC;
+        r[u] = __ldcs(((rr[u] & 1) ? src_v : src_k) + (size_t)(rr[u] >> 1) * PC + cc[u]);
+      }
+    }
+  };
+  load(first);
+  griddep_wait();
+  for (int base = first; base < total; base += nthr * kCopyUnroll) {
+    if (base != first) load(base);
+    int slot[kCopyUnroll];
+#pragma unroll
+    for (int u = 0; u < kCopyUnroll; ++u) slot[u] = rr[u] >= 0 ? slot_of(p, rs, rr[u] >> 1) : -1;
+#pragma unroll
+    for (int u = 0; u < kCopyUnroll; ++u) {
+      if (rr[u] < 0) continue;
+      const int k = rr[u] >> 1, t = rr[u] & 1;
+      if (p.mode == 3 && t == 0 && cc[u] == 0) replay_claim(p, rs, k, slot[u]);
+      if (slot[u] < 0) continue;
+      uint4 *dst = (t ? dst_v : dst_k) + (size_t)slot[u] * PC + cc[u];
+      if (DELTA && T.dk) {
+        uint4 *dd = reinterpret_cast<uint4 *>((t ? T.dv : T.dk) + (rs.bh * p.S + k) * (size_t)p.row_bytes);
+        __stcg(dd + cc[u], __ldcg(dst));
+      }
+      __stcg(dst, r[u]);
+    }
+  }
+}
+
+// int8 / int4 caches: one row per segment of L lanes (L = the smallest power of two
+// >= d / 8); lane i of a segment holds elements 8i .. 8i + 7 of the row.  Per row, the
+// same arithmetic as the per-row quantizer: absmax, IEEE division by qmax, clamp to the
+// fp16 range, round to fp16, then the code of quant_code.
+template <int NT, int KV, bool DELTA>
+__device__ __forceinline__ void quantize_rows(const EvParams<NT> &p) {
+  constexpr int qmax = KV == H2OKV_I8 ? 127 : 7;
+  const RowSet<NT> rs = row_set(p);
+  const EvTarget &T = *rs.T;
+  const int G8 = p.d / 8;
+  int L = 1;
+  while (L < G8) L <<= 1;
+  const int lane = threadIdx.x & 31;
+  const int seg = lane / L, li = lane % L, segs = 32 / L;
+  const int items = p.S * 2;  // (chunk row k, t) as 2k + t: t = 0 key row, 1 value row
+  const int W = gridDim.x * kRowWarps;
+  const int w0 = blockIdx.x * kRowWarps + (threadIdx.x >> 5);
+  const uint8_t *src_k = T.k_new + rs.bh * p.S * (size_t)p.in_row_bytes;
+  const uint8_t *src_v = T.v_new + rs.bh * p.S * (size_t)p.in_row_bytes;
+  uint4 xr[kQuantUnroll];
+  auto item_of = [&](int base, int u) { return ((base + u * W) * segs) + seg; };
+  auto load = [&](int base) {
+#pragma unroll
+    for (int u = 0; u < kQuantUnroll; ++u) {
+      const int it = item_of(base, u);
+      xr[u] = make_uint4(0u, 0u, 0u, 0u);
+      if (it < items && li < G8)
+        xr[u] = __ldcs(reinterpret_cast<const uint4 *>(((it & 1) ? src_v : src_k) +
+                                                        (size_t)(it >> 1) * p.in_row_bytes) + li);
+    }
+  };
+  load(w0);
+  griddep_wait();
+  for (int base = w0; base * segs < items; base += W * kQuantUnroll) {
+    if (base != w0) load(base);
+    int slot[kQuantUnroll];
+#pragma unroll
+    for (int u = 0; u < kQuantUnroll; ++u) {
+      const int it = item_of(base, u);
+      slot[u] = (it < items && li < G8) ? slot_of(p, rs, it >> 1) : -1;
+    }
+#pragma unroll
+    for (int u = 0; u < kQuantUnroll; ++u) {
+      const int it = item_of(base, u);
+      float v[8];
+      const __nv_bfloat162 *h2 = reinterpret_cast<const __nv_bfloat162 *>(&xr[u]);
+      float amax = 0.f;
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        const float2 f = __bfloat1622float2(h2[q]);
+        v[2 * q] = f.x;
+        v[2 * q + 1] = f.y;
+        amax = fmaxf(amax, fmaxf(fabsf(f.x), fabsf(f.y)));
+      }
+      for (int o = L >> 1; o > 0; o >>= 1)
+        amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
+      float rq = amax / (float)qmax;  // IEEE division
+      rq = fminf(rq, 65504.f);
+      const __half hs = __float2half_rn(rq);
+      const float s = __half2float(hs);
+      const float y = __frcp_rn(s);
+      int qc[8];
+#pragma unroll
+      for (int q = 0; q < 8; ++q) qc[q] = s > 0.f ? quant_code(v[q], s, y, (float)qmax) : 0;
+      if (it >= items || li >= G8) continue;
+      const int t = it & 1, k = it >> 1;
+      const int j = slot[u];
+      if (p.mode == 3 && t == 0 && li == 0) replay_claim(p, rs, k, j);
+      if (j < 0) continue;
+      const size_t drow = rs.bh * p.N_C + j, crow = rs.bh * p.S + k;
+      uint8_t *codes = (t ? T.values : T.keys) + drow * (size_t)p.row_bytes;
+      __half *sdst = (t ? T.v_scales : T.k_scales) + drow;
+      if (DELTA && T.dk) {
+        uint8_t *dcodes = (t ? T.dv : T.dk) + crow * (size_t)p.row_bytes;
+        if (li == 0) (t ? T.dvs : T.dks)[crow] = *sdst;
+        if (KV == H2OKV_I8)
+          reinterpret_cast<uint2 *>(dcodes)[li] = __ldcg(reinterpret_cast<const uint2 *>(codes) + li);
+        else
+          reinterpret_cast<uint32_t *>(dcodes)[li] =
+              __ldcg(reinterpret_cast<const unsigned int *>(codes) + li);
+      }
+      if (li == 0) *sdst = hs;
+      if (KV == H2OKV_I8) {
+        uint32_t lo = 0u, hi = 0u;
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          lo |= ((uint32_t)(qc[q] & 0xFF)) << (8 * q);
+          hi |= ((uint32_t)(qc[q + 4] & 0xFF)) << (8 * q);
+        }
+        __stcg(reinterpret_cast<uint2 *>(codes) + li, make_uint2(lo, hi));
+      } else {
+        uint32_t w = 0u;  // element 2i in the low nibble of byte i
+#pragma unroll
+        for (int q = 0; q < 8; ++q) w |= ((uint32_t)(qc[q] & 0xF)) << (4 * q);
+        __stcg(reinterpret_cast<unsigned int *>(codes) + li, w);
+      }
+    }
+  }
+}
+
+template <int NT, int KV, bool DELTA>
+__global__ void __launch_bounds__(kRowThreads) evict_rows_kernel(const __grid_constant__ EvParams<NT> p) {
+  if constexpr (KV == H2OKV_I8 || KV == H2OKV_I4)
+    quantize_rows<NT, KV, DELTA>(p);
+  else
+    copy_rows<NT, DELTA>(p);
+}
+
+// ---- per-row quantizer (kv_cache_quantize) ---------------------------------------------
 // One warp per row of d bf16 values; lane handles element pairs lane, lane+32, ...
 template <int KV>
 __device__ __forceinline__ void quantize_row_warp(const __nv_bfloat16 *__restrict__ x, int d,
@@ -87,12 +780,13 @@ __device__ __forceinline__ void quantize_row_warp(const __nv_bfloat16 *__restric
   const __half hs = __float2half_rn(r);
   const float s = __half2float(hs);
   if (lane == 0) *scale_out = hs;
+  const float y = __frcp_rn(s);
   for (int p = lane; p < d / 2; p += 32) {
     const float2 v = __bfloat1622float2(x2[p]);
     int qa = 0, qb = 0;
     if (s > 0.f) {
-      qa = (int)fminf(fmaxf(rintf(v.x / s), (float)-qmax), (float)qmax);
-      qb = (int)fminf(fmaxf(rintf(v.y / s), (float)-qmax), (float)qmax);
+      qa = quant_code(v.x, s, y, (float)qmax);
+      qb = quant_code(v.y, s, y, (float)qmax);
     }
     if (KV == H2OKV_I8) {
       out[2 * p] = (uint8_t)(int8_t)qa;
@@ -101,452 +795,6 @@ __device__ __forceinline__ void quantize_row_warp(const __nv_bfloat16 *__restric
       out[p] = (uint8_t)((qa & 0xF) | ((qb & 0xF) << 4));
     }
   }
-}
-
-struct EvictArgs {
-  float *scores;
-  const float *w_prev;
-  int32_t *token_pos;
-  const uint8_t *k_new, *v_new;
-  uint8_t *keys, *values;
-  __half *k_scales, *v_scales;
-  int32_t *slots_out;
-  const int32_t *slots_in;  // replay: the slots to write (mode 3)
-  uint8_t *dk, *dv;         // delta outputs (or null): overwritten rows [B][H_k][S][row bytes]
-  __half *dks, *dvs;        //   their scales (quantized caches)
-  int32_t *dpos;            //   their token positions [B][H_k][S]
-  int *status;              // device status word (replayed slot outside the cache)
-  int N_C, S, P, mode, n_filled, d, slice, score_mode, nbat, Hk;
-  size_t row_bytes, in_row_bytes;
-};
-
-constexpr int kCopyUnroll = 8;   // 16-byte pieces per thread in flight in the row copy
-constexpr int kQuantUnroll = 4;  // rows per lane segment in flight in the row quantizer
-
-// The rows of one chunk row set: chunk rows k = rank + CL * m (m = 0 .. n_rows - 1) of
-// (batch row, KV head) at cache offset gbase (slots) and chunk offset rbase (rows) go to
-// slot slot_of(m) (negative: skipped).
-struct RowSet {
-  size_t gbase, rbase;
-};
-
-// f32 / bf16 caches: the key and value rows are cut into 16-byte pieces spread over the
-// whole CTA (consecutive threads take consecutive pieces of a row), and every thread loads
-// kCopyUnroll pieces before it stores any, so a launch waits on memory a few times in all
-// rather than once per row.  With delta outputs the same thread first reads the piece it
-// overwrites.
-template <bool FULL, typename SlotOf>
-__device__ __forceinline__ void copy_rows_cta(const EvictArgs &a, RowSet rs, int rank, int CL,
-                                              int n_rows, SlotOf slot_of) {
-  const int C = (int)(a.row_bytes / 16);  // 16-byte pieces per row (row_bytes % 16 == 0)
-  const int total = n_rows * 2 * C;
-  const bool dl = FULL && a.dk != nullptr;
-  for (int base = threadIdx.x; base < total; base += kEvThreads * kCopyUnroll) {
-    uint4 r[kCopyUnroll], old[kCopyUnroll];
-    uint4 *dst[kCopyUnroll];
-    uint4 *ddst[kCopyUnroll];
-#pragma unroll
-    for (int u = 0; u < kCopyUnroll; ++u) {
-      const int e = base + u * kEvThreads;
-      dst[u] = nullptr;
-      ddst[u] = nullptr;
-      if (e < total) {
-        const int c = e % C, rest = e / C, t = rest & 1, m = rest >> 1;
-        const size_t row = rs.rbase + rank + (size_t)CL * m;
-        const uint8_t *src = (t ? a.v_new : a.k_new) + row * a.in_row_bytes;
-        r[u] = __ldcs(reinterpret_cast<const uint4 *>(src) + c);
-        const int slot = slot_of(m);
-        if (slot >= 0) {
-          dst[u] = reinterpret_cast<uint4 *>((t ? a.values : a.keys) +
-                                             (rs.gbase + (size_t)slot) * a.row_bytes) + c;
-          if (dl) {
-            old[u] = *dst[u];
-            ddst[u] = reinterpret_cast<uint4 *>((t ? a.dv : a.dk) + row * a.row_bytes) + c;
-          }
-        }
-      }
-    }
-#pragma unroll
-    for (int u = 0; u < kCopyUnroll; ++u) {
-      if (ddst[u]) *ddst[u] = old[u];
-      if (dst[u]) *dst[u] = r[u];
-    }
-  }
-}
-
-// int8 / int4 caches: one row per segment of L lanes (L = the smallest power of two
-// >= d / 8); lane i of a segment holds elements 8i .. 8i + 7 of the row.  A warp covers
-// 32 / L rows per pass and keeps kQuantUnroll passes in flight.  Per row, the same
-// arithmetic as the per-row quantizer: absmax, IEEE division by qmax, clamp to the fp16
-// range, round to fp16, then rint(x / scale) clamped to [-qmax, qmax].  With delta
-// outputs each lane first copies the codes (and lane 0 the scale) it overwrites.
-template <int KV, bool FULL, typename SlotOf>
-__device__ __forceinline__ void quantize_rows_cta(const EvictArgs &a, RowSet rs, int rank, int CL,
-                                                  int n_rows, SlotOf slot_of) {
-  constexpr int qmax = KV == H2OKV_I8 ? 127 : 7;
-  const int G = a.d / 8;
-  int L = 1;
-  while (L < G) L <<= 1;
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  const int seg = lane / L, li = lane % L, segs = 32 / L;
-  const int items = n_rows * 2;  // (m, t): t = 0 key row, 1 value row
-  const bool dl = FULL && a.dk != nullptr;
-  for (int p0 = 0; (p0 * kEvWarps + warp) * segs < items; p0 += kQuantUnroll) {
-    uint4 x[kQuantUnroll];
-    bool ok[kQuantUnroll];
-    int slot[kQuantUnroll];
-#pragma unroll
-    for (int u = 0; u < kQuantUnroll; ++u) {
-      const int item = ((p0 + u) * kEvWarps + warp) * segs + seg;
-      ok[u] = item < items && li < G;
-      x[u] = make_uint4(0u, 0u, 0u, 0u);
-      slot[u] = -1;
-      if (ok[u]) {
-        const int t = item & 1, m = item >> 1;
-        slot[u] = slot_of(m);
-        const size_t row = rs.rbase + rank + (size_t)CL * m;
-        const uint8_t *src = (t ? a.v_new : a.k_new) + row * a.in_row_bytes;
-        x[u] = __ldcs(reinterpret_cast<const uint4 *>(src) + li);
-      }
-    }
-#pragma unroll
-    for (int u = 0; u < kQuantUnroll; ++u) {
-      float v[8];
-      const __nv_bfloat162 *h2 = reinterpret_cast<const __nv_bfloat162 *>(&x[u]);
-      float amax = 0.f;
-#pragma unroll
-      for (int q = 0; q < 4; ++q) {
-        const float2 f = __bfloat1622float2(h2[q]);
-        v[2 * q] = f.x;
-        v[2 * q + 1] = f.y;
-        amax = fmaxf(amax, fmaxf(fabsf(f.x), fabsf(f.y)));
-      }
-      for (int o = L >> 1; o > 0; o >>= 1)
-        amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
-      float r = amax / (float)qmax;  // IEEE division
-      r = fminf(r, 65504.f);
-      const __half hs = __float2half_rn(r);
-      const float s = __half2float(hs);
-      int qc[8];
-#pragma unroll
-      for (int q = 0; q < 8; ++q)
-        qc[q] = s > 0.f ? (int)fminf(fmaxf(rintf(v[q] / s), (float)-qmax), (float)qmax) : 0;
-      if (!ok[u] || slot[u] < 0) continue;
-      const int item = ((p0 + u) * kEvWarps + warp) * segs + seg;
-      const int t = item & 1, m = item >> 1;
-      const size_t drow = rs.gbase + (size_t)slot[u];
-      const size_t crow = rs.rbase + rank + (size_t)CL * m;
-      uint8_t *codes = (t ? a.values : a.keys) + drow * a.row_bytes;
-      __half *sdst = (t ? a.v_scales : a.k_scales) + drow;
-      if (dl) {
-        uint8_t *dcodes = (t ? a.dv : a.dk) + crow * a.row_bytes;
-        if (li == 0) (t ? a.dvs : a.dks)[crow] = *sdst;
-        if (KV == H2OKV_I8)
-          reinterpret_cast<uint2 *>(dcodes)[li] = reinterpret_cast<const uint2 *>(codes)[li];
-        else
-          reinterpret_cast<uint32_t *>(dcodes)[li] = reinterpret_cast<const uint32_t *>(codes)[li];
-      }
-      if (li == 0) *sdst = hs;
-      if (KV == H2OKV_I8) {
-        uint32_t lo = 0u, hi = 0u;
-#pragma unroll
-        for (int q = 0; q < 4; ++q) {
-          lo |= ((uint32_t)(qc[q] & 0xFF)) << (8 * q);
-          hi |= ((uint32_t)(qc[q + 4] & 0xFF)) << (8 * q);
-        }
-        reinterpret_cast<uint2 *>(codes)[li] = make_uint2(lo, hi);
-      } else {
-        uint32_t w = 0u;  // element 2i in the low nibble of byte i
-#pragma unroll
-        for (int q = 0; q < 8; ++q) w |= ((uint32_t)(qc[q] & 0xF)) << (4 * q);
-        reinterpret_cast<uint32_t *>(codes)[li] = w;
-      }
-    }
-  }
-}
-
-template <int KV, bool FULL, typename SlotOf>
-__device__ __forceinline__ void insert_rows_cta(const EvictArgs &a, RowSet rs, int rank, int CL,
-                                                SlotOf slot_of) {
-  const int n_rows = rank < a.S ? (a.S - rank + CL - 1) / CL : 0;
-  if constexpr (KV == H2OKV_I8 || KV == H2OKV_I4)
-    quantize_rows_cta<KV, FULL>(a, rs, rank, CL, n_rows, slot_of);
-  else
-    copy_rows_cta<FULL>(a, rs, rank, CL, n_rows, slot_of);
-}
-
-template <int IPT>
-__device__ __forceinline__ void store_slice(float *dst, const float (&v)[IPT],
-                                            const bool (&valid)[IPT], bool vec) {
-  if constexpr (IPT % 4 == 0) {
-    if (vec) {
-#pragma unroll
-      for (int i = 0; i < IPT; i += 4)
-        *reinterpret_cast<float4 *>(dst + i) = make_float4(v[i], v[i + 1], v[i + 2], v[i + 3]);
-      return;
-    }
-  }
-  {
-#pragma unroll
-    for (int i = 0; i < IPT; ++i)
-      if (valid[i]) dst[i] = v[i];
-  }
-}
-
-// Slot j of a chunk row set receives chunk row k: bookkeeping of the slot (old token
-// position to the delta output, new token position, score 0 unless the caller stores
-// the slice's scores afterwards, slot list).
-template <bool FULL>
-__device__ __forceinline__ void claim_slot(const EvictArgs &a, RowSet rs, int j, int k,
-                                           bool zero_score = true) {
-  const size_t gs = rs.gbase + (size_t)j, rk = rs.rbase + (size_t)k;
-  if (FULL && a.dpos) a.dpos[rk] = a.token_pos[gs];
-  a.token_pos[gs] = a.P + k;
-  if (zero_score) a.scores[gs] = 0.f;
-  if (a.slots_out) a.slots_out[rk] = j;
-}
-
-// mode 0: fold w_prev only (S = 0); 1: fill slots n_filled.. (no occupied slot is
-// touched); 2: generic choice (empty slots first, then lowest selection keys);
-// 3: replay (write the given slots).  One cluster per (batch row, KV head), or per KV
-// head for all batch rows together (score variant h2o_orig: nbat > 1).
-// FULL: the general kernel (h2o_orig over several batch rows, replay, delta outputs); the
-// other instance is the plain per-(b, h_k) choice, built without those paths.
-template <int KV, int IPT, bool FULL>
-__global__ void __launch_bounds__(kEvThreads) evict_kernel(const EvictArgs a) {
-  namespace cg = cooperative_groups;
-  cg::cluster_group cluster = cg::this_cluster();
-  const int CL = (int)cluster.num_blocks();
-  const int rank = (int)cluster.block_rank();
-  const int gi = blockIdx.x / CL;
-  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  const int nb = FULL ? a.nbat : 1;
-  const int b_first = nb > 1 ? 0 : gi / a.Hk, h = nb > 1 ? gi : gi % a.Hk;
-  auto rows_of = [&](int bb) {
-    const size_t bh = (size_t)(b_first + bb) * a.Hk + h;
-    return RowSet{bh * (size_t)a.N_C, bh * (size_t)a.S};
-  };
-
-  __shared__ uint32_t hist[2][256];
-  __shared__ uint32_t tot_bins[256];
-  __shared__ uint32_t warp_tot[kEvWarps];
-  __shared__ uint32_t s_prefix, s_k, s_total;
-  __shared__ uint32_t cta_less, cta_eq;
-  extern __shared__ int32_t rowslot[];  // [ceil(S / CL)]: slot of chunk row rank + CL * m
-
-  const int j0 = rank * a.slice + tid * IPT;
-  float sc[IPT], ksum[IPT];
-  int32_t tp[IPT];
-  uint32_t key[IPT];
-  bool valid[IPT];
-#pragma unroll
-  for (int i = 0; i < IPT; ++i) {
-    valid[i] = j0 + i < a.N_C;
-    tp[i] = kEmptyPos;
-    ksum[i] = 0.f;
-  }
-  // one batch row choosing for itself: its folded scores are stored once, after the
-  // choice, with the chosen slots at 0 (the stores then overlap nothing else)
-  const bool defer_store = a.mode == 2 && nb == 1;
-  bool vec0 = false;
-  // ---- fold w_prev into the scores of every batch row of this set ----------------
-  for (int bb = 0; bb < nb; ++bb) {
-    const size_t gbase = rows_of(bb).gbase;
-    float wp[IPT];
-#pragma unroll
-    for (int i = 0; i < IPT; ++i) {
-      sc[i] = 0.f;
-      wp[i] = 0.f;
-    }
-    const bool want_tp = bb == 0 && a.mode == 2;
-    // 16-byte loads when this thread's slots are whole and aligned, else one by one
-    const bool vec = IPT % 4 == 0 && j0 + IPT <= a.N_C &&
-                     ((reinterpret_cast<uintptr_t>(a.scores + gbase + j0) |
-                       reinterpret_cast<uintptr_t>(a.token_pos + gbase + j0) |
-                       (a.w_prev ? reinterpret_cast<uintptr_t>(a.w_prev + gbase + j0) : 0u)) &
-                      15u) == 0u;
-    bool loaded = false;
-    if constexpr (IPT % 4 == 0) {
-      if (vec) {
-#pragma unroll
-        for (int i = 0; i < IPT; i += 4) {
-          *reinterpret_cast<float4 *>(&sc[i]) =
-              *reinterpret_cast<const float4 *>(a.scores + gbase + j0 + i);
-          if (a.w_prev)
-            *reinterpret_cast<float4 *>(&wp[i]) =
-                __ldcs(reinterpret_cast<const float4 *>(a.w_prev + gbase + j0 + i));
-          if (want_tp)
-            *reinterpret_cast<int4 *>(&tp[i]) =
-                *reinterpret_cast<const int4 *>(a.token_pos + gbase + j0 + i);
-        }
-        loaded = true;
-      }
-    }
-    if (!loaded) {
-#pragma unroll
-      for (int i = 0; i < IPT; ++i) {
-        if (!valid[i]) continue;
-        sc[i] = a.scores[gbase + j0 + i];
-        if (a.w_prev) wp[i] = a.w_prev[gbase + j0 + i];
-        if (want_tp) tp[i] = a.token_pos[gbase + j0 + i];
-      }
-    }
-#pragma unroll
-    for (int i = 0; i < IPT; ++i) {
-      if (a.w_prev) sc[i] = __fadd_rn(sc[i], wp[i]);
-      ksum[i] = bb == 0 ? sc[i] : __fadd_rn(ksum[i], sc[i]);  // h2o_orig: batch order
-    }
-    if (a.w_prev && !defer_store) store_slice<IPT>(a.scores + gbase + j0, sc, valid, vec);
-    if (bb == 0) vec0 = vec;
-  }
-
-  if (a.mode == 1) {
-    // while filling: chunk row k takes slot n_filled + k (same slot for every batch row)
-#pragma unroll
-    for (int i = 0; i < IPT; ++i) {
-      const int k = j0 + i - a.n_filled;
-      if (valid[i] && k >= 0 && k < a.S)
-        for (int bb = 0; bb < nb; ++bb) claim_slot<FULL>(a, rows_of(bb), j0 + i, k);
-    }
-    const int first = a.n_filled + rank;
-    for (int bb = 0; bb < nb; ++bb)
-      insert_rows_cta<KV, FULL>(a, rows_of(bb), rank, CL, [&](int m) { return first + CL * m; });
-    return;
-  }
-  if (FULL && a.mode == 3) {
-    // replay: every fold store of the cluster lands before a replayed slot is reset
-    cluster.sync();
-    for (int bb = 0; bb < nb; ++bb) {
-      const RowSet rs = rows_of(bb);
-      auto slot_of = [&](int m) -> int {
-        const int j = a.slots_in[rs.rbase + rank + (size_t)CL * m];
-        return (j >= 0 && j < a.N_C) ? j : -1;
-      };
-      for (int m = tid; rank + CL * m < a.S; m += kEvThreads) {
-        const int j = slot_of(m);
-        if (j < 0)
-          atomicExch(a.status, H2OKV_ERR_INVALID_ARG);
-        else
-          claim_slot<FULL>(a, rs, j, rank + CL * m);
-      }
-      insert_rows_cta<KV, FULL>(a, rs, rank, CL, slot_of);
-    }
-    return;
-  }
-  if (a.mode != 2) return;
-
-  // ---- selection keys ----------------------------------------------------------------
-#pragma unroll
-  for (int i = 0; i < IPT; ++i) {
-    float kv = ksum[i];
-    if (a.score_mode == 1) {  // h2o_norm: score / (P - t(b, h, j)), age at least 1
-      const int age = max(a.P - tp[i], 1);
-      kv = __fdiv_rn(kv, (float)age);
-    }
-    key[i] = (valid[i] && tp[i] != kEmptyPos) ? order_key(kv) : 0u;
-  }
-
-  // ---- radix select of the S-th smallest key over the whole cluster --------------
-  uint32_t prefix = 0u, pmask = 0u, kk = (uint32_t)a.S;
-  for (int pass = 0; pass < 4; ++pass) {
-    const int shift = 24 - 8 * pass;
-    uint32_t *h = hist[pass & 1];
-    h[tid] = 0u;
-    __syncthreads();
-#pragma unroll
-    for (int i = 0; i < IPT; ++i) {
-      const uint32_t bin =
-          (valid[i] && (key[i] & pmask) == prefix) ? (key[i] >> shift) & 255u : 0xffffffffu;
-      const uint32_t peers = __match_any_sync(0xffffffffu, bin);
-      if (bin != 0xffffffffu && lane == __ffs(peers) - 1) atomicAdd(&h[bin], __popc(peers));
-    }
-    cluster.sync();  // every CTA's histogram of this pass is complete
-    uint32_t sum = 0u;
-    for (int q = 0; q < CL; ++q) sum += cluster.map_shared_rank(h, q)[tid];
-    tot_bins[tid] = sum;
-    __syncthreads();
-    if (warp == 0) {
-      uint32_t loc[8], lsum = 0;
-#pragma unroll
-      for (int t = 0; t < 8; ++t) {
-        loc[t] = tot_bins[lane * 8 + t];
-        lsum += loc[t];
-      }
-      uint32_t incl = lsum;
-#pragma unroll
-      for (int o = 1; o < 32; o <<= 1) {
-        const uint32_t v = __shfl_up_sync(0xffffffffu, incl, o);
-        if (lane >= o) incl += v;
-      }
-      const uint32_t excl = incl - lsum;
-      if (excl < kk && kk <= incl) {
-        uint32_t c = excl;
-#pragma unroll
-        for (int t = 0; t < 8; ++t) {
-          if (c + loc[t] >= kk) {
-            s_prefix = prefix | ((uint32_t)(lane * 8 + t) << shift);
-            s_k = kk - c;
-            break;
-          }
-          c += loc[t];
-        }
-      }
-    }
-    __syncthreads();
-    prefix = s_prefix;
-    kk = s_k;
-    pmask |= 255u << shift;
-  }
-  const uint32_t T = prefix, k_eq = kk;  // take every key < T and the first k_eq keys == T
-
-  // ---- chosen slots in slot order ---------------------------------------------------
-  uint32_t nl = 0, ne = 0;
-#pragma unroll
-  for (int i = 0; i < IPT; ++i) {
-    nl += (valid[i] && key[i] < T) ? 1u : 0u;
-    ne += (valid[i] && key[i] == T) ? 1u : 0u;
-  }
-  // per-thread counts <= IPT and per-CTA totals <= kEvThreads * IPT < 65536: pack 16 + 16 bits
-  const uint32_t ex = block_exclusive_scan((nl << 16) | ne, warp_tot, &s_total);
-  if (tid == 0) {
-    cta_less = s_total >> 16;
-    cta_eq = s_total & 0xffffu;
-  }
-  cluster.sync();  // per-CTA totals visible to the cluster
-  uint32_t base_less = 0, base_eq = 0;
-  for (int q = 0; q < rank; ++q) {
-    base_less += *cluster.map_shared_rank(&cta_less, q);
-    base_eq += *cluster.map_shared_rank(&cta_eq, q);
-  }
-  uint32_t less_before = base_less + (ex >> 16), eq_before = base_eq + (ex & 0xffffu);
-#pragma unroll
-  for (int i = 0; i < IPT; ++i) {
-    if (!valid[i]) continue;
-    const int j = j0 + i;
-    bool take = false;
-    uint32_t pos = 0;
-    if (key[i] < T) {
-      take = true;
-      pos = less_before + min(eq_before, k_eq);
-      ++less_before;
-    } else if (key[i] == T) {
-      take = eq_before < k_eq;
-      pos = less_before + eq_before;
-      ++eq_before;
-    }
-    if (take) {
-      if (defer_store) sc[i] = 0.f;
-      for (int bb = 0; bb < nb; ++bb) claim_slot<FULL>(a, rows_of(bb), j, (int)pos, !defer_store);
-      int32_t *dst = cluster.map_shared_rank(rowslot, (int)(pos % (uint32_t)CL));
-      dst[pos / (uint32_t)CL] = j;
-    }
-  }
-  if (defer_store) store_slice<IPT>(a.scores + rows_of(0).gbase + j0, sc, valid, vec0);
-  cluster.sync();  // rowslot lists complete
-
-  // ---- insert the chunk's rows k = rank, rank + CL, ... -----------------------------
-  for (int bb = 0; bb < nb; ++bb)
-    insert_rows_cta<KV, FULL>(a, rows_of(bb), rank, CL, [&](int m) { return rowslot[m]; });
 }
 
 template <int KV>
@@ -599,116 +847,240 @@ __global__ void init_kernel(int32_t *__restrict__ token_pos, float *__restrict__
   }
 }
 
+// ---- launch --------------------------------------------------------------------------
+// Everything of a call that the caches share (they must agree on it).
+struct EvCall {
+  int mode, S, P, n_filled, score_mode;
+  bool orig, delta;
+};
+
+EvTarget target_of(h2okv_cache *c, const float *w_prev, const void *k_new, const void *v_new,
+                   int32_t *slots_out, const int32_t *slots_in, const h2okv_delta *delta) {
+  uint8_t *ws = reinterpret_cast<uint8_t *>(c->bufs.workspace);
+  EvTarget t;
+  t.scores = c->bufs.scores;
+  t.w_prev = w_prev;
+  t.token_pos = c->bufs.token_pos;
+  t.k_new = reinterpret_cast<const uint8_t *>(k_new);
+  t.v_new = reinterpret_cast<const uint8_t *>(v_new);
+  t.keys = reinterpret_cast<uint8_t *>(c->bufs.keys);
+  t.values = reinterpret_cast<uint8_t *>(c->bufs.values);
+  t.k_scales = reinterpret_cast<__half *>(c->bufs.k_scales);
+  t.v_scales = reinterpret_cast<__half *>(c->bufs.v_scales);
+  t.slots_out = slots_out;
+  t.slots_in = slots_in;
+  t.dk = delta ? reinterpret_cast<uint8_t *>(delta->keys) : nullptr;
+  t.dv = delta ? reinterpret_cast<uint8_t *>(delta->values) : nullptr;
+  t.dks = delta ? reinterpret_cast<__half *>(delta->k_scales) : nullptr;
+  t.dvs = delta ? reinterpret_cast<__half *>(delta->v_scales) : nullptr;
+  t.dpos = delta ? delta->token_pos : nullptr;
+  t.hist = reinterpret_cast<uint32_t *>(ws + c->ws.ev_hist);
+  t.arrive = reinterpret_cast<uint32_t *>(ws + c->ws.ev_arrive);
+  t.slotlist = reinterpret_cast<int32_t *>(ws + c->ws.ev_slots);
+  t.status = reinterpret_cast<int *>(ws + c->ws.status);
+  return t;
+}
+
+// Shared-memory opt-in of one choose kernel instance, once per device.
+template <int NT, int KM>
+int opt_in_choose() {
+  static std::mutex mu;
+  static bool done[64] = {};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64)
+    return set_error(H2OKV_ERR_CUDA, "cudaGetDevice failed");
+  std::lock_guard<std::mutex> lock(mu);
+  if (!done[dev]) {
+    cudaError_t e = cudaFuncSetAttribute(
+        evict_choose_kernel<NT, KM>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+        (int)(kSmemKeysMax * 4 + kSlotListMax * sizeof(int32_t)));
+    if (e != cudaSuccess)
+      return set_error(H2OKV_ERR_CUDA, "cudaFuncSetAttribute(evict_choose_kernel): %s",
+                       cudaGetErrorString(e));
+    done[dev] = true;
+  }
+  return H2OKV_OK;
+}
+
+template <int NT, int KV>
+int launch_rows(const EvParams<NT> &p, bool delta, int sms, cudaStream_t st) {
+  const long long sets = (long long)p.n_targets * p.G * p.nb;
+  long long work;  // independent units of one set (pieces, or lane segments)
+  int per_cta;
+  if (KV == H2OKV_I8 || KV == H2OKV_I4) {
+    int L = 1;
+    while (L < p.d / 8) L <<= 1;
+    work = (long long)p.S * 2;
+    per_cta = kRowWarps * (32 / L) * kQuantUnroll;
+  } else {
+    work = (long long)p.S * 2 * (p.row_bytes / 16);
+    per_cta = kRowThreads * kCopyUnroll;
+  }
+  if (work <= 0 || sets <= 0) return H2OKV_OK;
+  if (sets > 65535 || work >= (1LL << 30))
+    return set_error(H2OKV_ERR_UNSUPPORTED, "too many chunk rows in one eviction call");
+  // CTAs per set: every row of the call in flight in one round (CTAs are cheap; a CTA
+  // that looped over many rounds would wait on memory once per round)
+  const long long gx = (work + per_cta - 1) / per_cta;
+  if (gx > 65535) return set_error(H2OKV_ERR_UNSUPPORTED, "chunk too long for one eviction call");
+  (void)sms;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)gx, (unsigned)sets);
+  cfg.blockDim = dim3(kRowThreads);
+  cfg.dynamicSmemBytes = 0;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  cudaError_t e = delta ? cudaLaunchKernelEx(&cfg, evict_rows_kernel<NT, KV, true>, p)
+                        : cudaLaunchKernelEx(&cfg, evict_rows_kernel<NT, KV, false>, p);
+  if (e != cudaSuccess)
+    return set_error(H2OKV_ERR_CUDA, "evict_rows_kernel launch: %s", cudaGetErrorString(e));
+  return check_launch("evict_rows_kernel");
+}
+
+template <int NT>
+int launch_evict_t(h2okv_cache *const *caches, int n, const EvTarget *targets, const EvCall &call,
+                   cudaStream_t st) {
+  const h2okv_cache_desc &d = caches[0]->desc;
+  EvParams<NT> p;
+  for (int i = 0; i < n; ++i) p.t[i] = targets[i];
+  p.n_targets = n;
+  p.nb = call.orig ? d.batch : 1;
+  p.G = call.orig ? d.n_kv_heads : d.batch * d.n_kv_heads;
+  p.Hk = d.n_kv_heads;
+  p.N_C = d.capacity;
+  p.S = call.S;
+  p.P = call.P;
+  p.n_filled = call.n_filled;
+  p.d = d.head_dim;
+  p.mode = call.mode;
+  p.score_mode = call.score_mode;
+  p.need_tp = (call.n_filled < d.capacity || call.score_mode == H2OKV_SCORE_H2O_NORM) ? 1 : 0;
+  p.vec = d.capacity % 4 == 0 ? 1 : 0;
+  p.row_bytes = (int)caches[0]->row_bytes;
+  p.in_row_bytes = d.head_dim * (d.q_dtype == H2OKV_F32 ? 4 : 2);
+  p.wait_ns = caches[0]->wait_timeout_ns;
+  const int sms = caches[0]->sms > 0 ? caches[0]->sms : 148;
+  const int units = n * p.G;
+  // fold CTAs per group: about four per SM in all, slices of at least 2048 slots
+  const int by_sm = max(1, (4 * sms) / units);
+  const int by_len = max(1, (d.capacity + 2047) / 2048);
+  p.C = min(by_sm, by_len);
+  p.slice = ((d.capacity + p.C - 1) / p.C + 3) & ~3;
+  p.C = (d.capacity + p.slice - 1) / p.slice;
+  if ((long long)units * p.C > INT32_MAX)
+    return set_error(H2OKV_ERR_UNSUPPORTED, "too many groups in one eviction call");
+  evict_fold_kernel<NT><<<units * p.C, kSelThreads, 0, st>>>(p);
+  int rc = check_launch("evict_fold_kernel");
+  if (rc || p.mode == 0) return rc;
+  if (p.mode == 2) {
+    // key source of the choose kernel (see there)
+    const bool fits = d.capacity <= kSmemKeysMax;
+    const int km = !fits ? 0
+                   : (p.vec && p.nb == 1 && !p.need_tp && p.score_mode != H2OKV_SCORE_H2O_NORM) ? 2
+                                                                                            : 1;
+    const size_t smem = kSlotListMax * sizeof(int32_t) + (fits ? (size_t)d.capacity * 4 : 0);
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)units);
+    cfg.blockDim = dim3(kChooseThreads);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    cudaError_t e;
+    if (km == 2) {
+      rc = opt_in_choose<NT, 2>();
+      if (rc) return rc;
+      e = cudaLaunchKernelEx(&cfg, evict_choose_kernel<NT, 2>, p);
+    } else if (km == 1) {
+      rc = opt_in_choose<NT, 1>();
+      if (rc) return rc;
+      e = cudaLaunchKernelEx(&cfg, evict_choose_kernel<NT, 1>, p);
+    } else {
+      rc = opt_in_choose<NT, 0>();
+      if (rc) return rc;
+      e = cudaLaunchKernelEx(&cfg, evict_choose_kernel<NT, 0>, p);
+    }
+    if (e != cudaSuccess)
+      return set_error(H2OKV_ERR_CUDA, "evict_choose_kernel launch: %s", cudaGetErrorString(e));
+    rc = check_launch("evict_choose_kernel");
+    if (rc) return rc;
+  }
+  switch (d.kv_dtype) {
+    case H2OKV_F32: return launch_rows<NT, H2OKV_F32>(p, call.delta, sms, st);
+    case H2OKV_BF16: return launch_rows<NT, H2OKV_BF16>(p, call.delta, sms, st);
+    case H2OKV_I8: return launch_rows<NT, H2OKV_I8>(p, call.delta, sms, st);
+    case H2OKV_I4: return launch_rows<NT, H2OKV_I4>(p, call.delta, sms, st);
+  }
+  return set_error(H2OKV_ERR_UNSUPPORTED, "kv dtype");
+}
+
+constexpr int kMaxCachesPerLaunch = 48;
+
 }  // namespace
 
 int launch_init_cache(h2okv_cache *c, cudaStream_t st) {
   const size_t n = (size_t)c->desc.batch * c->desc.n_kv_heads * c->desc.capacity;
-  if (cudaMemsetAsync(reinterpret_cast<uint8_t *>(c->bufs.workspace) + c->ws.status, 0, 4, st) !=
-      cudaSuccess)
-    return set_error(H2OKV_ERR_CUDA, "cudaMemsetAsync(status) failed");
+  uint8_t *ws = reinterpret_cast<uint8_t *>(c->bufs.workspace);
+  if (cudaMemsetAsync(ws + c->ws.status, 0, 4, st) != cudaSuccess ||
+      cudaMemsetAsync(ws + c->ws.ev_hist, 0, c->ws.ev_zero_end - c->ws.ev_hist, st) != cudaSuccess)
+    return set_error(H2OKV_ERR_CUDA, "cudaMemsetAsync(workspace) failed");
   const int blocks = (int)((n + 255) / 256 < 4096 ? (n + 255) / 256 : 4096);
   init_kernel<<<blocks, 256, 0, st>>>(c->bufs.token_pos, c->bufs.scores, n);
   return check_launch("init_kernel");
 }
 
-template <int KV, int IPT, bool FULL>
-static int launch_evict_t(const EvictArgs &a, int n_groups, int CL, cudaStream_t st) {
-  cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3((unsigned)(n_groups * CL));
-  cfg.blockDim = dim3(kEvThreads);
-  cfg.dynamicSmemBytes = (size_t)((a.S + CL - 1) / CL) * 4;
-  cfg.stream = st;
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeClusterDimension;
-  attr[0].val.clusterDim.x = CL;
-  attr[0].val.clusterDim.y = 1;
-  attr[0].val.clusterDim.z = 1;
-  cfg.attrs = attr;
-  cfg.numAttrs = 1;
-  if (cfg.dynamicSmemBytes > 48 * 1024) {
-    cudaError_t e = cudaFuncSetAttribute(evict_kernel<KV, IPT, FULL>,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         (int)cfg.dynamicSmemBytes);
-    if (e != cudaSuccess)
-      return set_error(H2OKV_ERR_CUDA, "cudaFuncSetAttribute(evict_kernel): %s",
-                       cudaGetErrorString(e));
-  }
-  cudaError_t e = cudaLaunchKernelEx(&cfg, evict_kernel<KV, IPT, FULL>, a);
-  if (e != cudaSuccess)
-    return set_error(H2OKV_ERR_CUDA, "evict_kernel launch: %s", cudaGetErrorString(e));
-  return check_launch("evict_kernel");
-}
-
-template <int KV, bool FULL>
-static int launch_evict_kv(const EvictArgs &a, int n_groups, int CL, int ipt, cudaStream_t st) {
-  switch (ipt) {
-    case 1: return launch_evict_t<KV, 1, FULL>(a, n_groups, CL, st);
-    case 2: return launch_evict_t<KV, 2, FULL>(a, n_groups, CL, st);
-    case 4: return launch_evict_t<KV, 4, FULL>(a, n_groups, CL, st);
-    case 8: return launch_evict_t<KV, 8, FULL>(a, n_groups, CL, st);
-    case 16: return launch_evict_t<KV, 16, FULL>(a, n_groups, CL, st);
-    case 32: return launch_evict_t<KV, 32, FULL>(a, n_groups, CL, st);
-  }
-  return set_error(H2OKV_ERR_UNSUPPORTED, "capacity too large for the eviction kernel");
+// Mode of a call on a cache in this state.
+static int call_mode(const h2okv_cache *c, int S, const int32_t *slots_in) {
+  return S == 0 ? 0 : (slots_in ? 3 : (c->n_filled + S <= c->desc.capacity ? 1 : 2));
 }
 
 int launch_evict_insert(h2okv_cache *c, const float *w_prev, const void *k_new, const void *v_new,
                         int S, int64_t P, int32_t *slots_out, const int32_t *slots_in,
                         const h2okv_delta *delta, cudaStream_t st) {
-  const h2okv_cache_desc &d = c->desc;
-  EvictArgs a;
-  a.scores = c->bufs.scores;
-  a.w_prev = w_prev;
-  a.token_pos = c->bufs.token_pos;
-  a.k_new = reinterpret_cast<const uint8_t *>(k_new);
-  a.v_new = reinterpret_cast<const uint8_t *>(v_new);
-  a.keys = reinterpret_cast<uint8_t *>(c->bufs.keys);
-  a.values = reinterpret_cast<uint8_t *>(c->bufs.values);
-  a.k_scales = reinterpret_cast<__half *>(c->bufs.k_scales);
-  a.v_scales = reinterpret_cast<__half *>(c->bufs.v_scales);
-  a.slots_out = slots_out;
-  a.slots_in = slots_in;
-  a.dk = delta ? reinterpret_cast<uint8_t *>(delta->keys) : nullptr;
-  a.dv = delta ? reinterpret_cast<uint8_t *>(delta->values) : nullptr;
-  a.dks = delta ? reinterpret_cast<__half *>(delta->k_scales) : nullptr;
-  a.dvs = delta ? reinterpret_cast<__half *>(delta->v_scales) : nullptr;
-  a.dpos = delta ? delta->token_pos : nullptr;
-  a.status = reinterpret_cast<int *>(reinterpret_cast<uint8_t *>(c->bufs.workspace) + c->ws.status);
-  a.N_C = d.capacity;
-  a.S = S;
-  a.P = (int)P;
-  a.mode = S == 0 ? 0 : (slots_in ? 3 : (c->n_filled + S <= d.capacity ? 1 : 2));
-  a.score_mode = c->score_mode;
-  a.Hk = d.n_kv_heads;
-  // h2o_orig: one cluster per KV head selects for every batch row
-  const bool orig = c->score_mode == H2OKV_SCORE_H2O_ORIG && a.mode == 2;
-  a.nbat = orig ? d.batch : 1;
-  a.n_filled = c->n_filled;
-  a.d = d.head_dim;
-  a.row_bytes = c->row_bytes;
-  a.in_row_bytes = (size_t)d.head_dim * (d.q_dtype == H2OKV_F32 ? 4 : 2);
-  // cluster size and slots per thread: CL * kEvThreads * IPT >= N_C
-  const int CL = kEvictCluster;
-  int ipt = 1;
-  while ((int64_t)CL * kEvThreads * ipt < d.capacity) ipt *= 2;
-  a.slice = kEvThreads * ipt;
-  const int n_groups = orig ? d.n_kv_heads : d.batch * d.n_kv_heads;
-  const bool full = orig || delta != nullptr || a.mode == 3;
-  switch (d.kv_dtype) {
-    case H2OKV_F32:
-      return full ? launch_evict_kv<H2OKV_F32, true>(a, n_groups, CL, ipt, st)
-                  : launch_evict_kv<H2OKV_F32, false>(a, n_groups, CL, ipt, st);
-    case H2OKV_BF16:
-      return full ? launch_evict_kv<H2OKV_BF16, true>(a, n_groups, CL, ipt, st)
-                  : launch_evict_kv<H2OKV_BF16, false>(a, n_groups, CL, ipt, st);
-    case H2OKV_I8:
-      return full ? launch_evict_kv<H2OKV_I8, true>(a, n_groups, CL, ipt, st)
-                  : launch_evict_kv<H2OKV_I8, false>(a, n_groups, CL, ipt, st);
-    case H2OKV_I4:
-      return full ? launch_evict_kv<H2OKV_I4, true>(a, n_groups, CL, ipt, st)
-                  : launch_evict_kv<H2OKV_I4, false>(a, n_groups, CL, ipt, st);
+  EvCall call;
+  call.mode = call_mode(c, S, slots_in);
+  call.S = S;
+  call.P = (int)P;
+  call.n_filled = c->n_filled;
+  call.score_mode = c->score_mode;
+  // h2o_orig: one group per KV head chooses for every batch row
+  call.orig = c->score_mode == H2OKV_SCORE_H2O_ORIG && call.mode == 2;
+  call.delta = delta != nullptr;
+  const EvTarget t = target_of(c, w_prev, k_new, v_new, slots_out, slots_in, delta);
+  return launch_evict_t<1>(&c, 1, &t, call, st);
+}
+
+int launch_evict_insert_many(h2okv_cache *const *caches, int n, const float *const *w_prev,
+                             const void *const *k_new, const void *const *v_new, int S, int64_t P,
+                             int32_t *const *slots_out, cudaStream_t st) {
+  const h2okv_cache *c0 = caches[0];
+  EvCall call;
+  call.mode = call_mode(c0, S, nullptr);
+  call.S = S;
+  call.P = (int)P;
+  call.n_filled = c0->n_filled;
+  call.score_mode = c0->score_mode;
+  call.orig = c0->score_mode == H2OKV_SCORE_H2O_ORIG && call.mode == 2;
+  call.delta = false;
+  EvTarget t[kMaxCachesPerLaunch];
+  for (int base = 0; base < n; base += kMaxCachesPerLaunch) {
+    const int m = min(kMaxCachesPerLaunch, n - base);
+    for (int i = 0; i < m; ++i)
+      t[i] = target_of(caches[base + i], w_prev ? w_prev[base + i] : nullptr,
+                       k_new ? k_new[base + i] : nullptr, v_new ? v_new[base + i] : nullptr,
+                       slots_out ? slots_out[base + i] : nullptr, nullptr, nullptr);
+    const int rc = m == 1 ? launch_evict_t<1>(caches + base, 1, t, call, st)
+                          : launch_evict_t<kMaxCachesPerLaunch>(caches + base, m, t, call, st);
+    if (rc) return rc;
   }
-  return set_error(H2OKV_ERR_UNSUPPORTED, "kv dtype");
+  return H2OKV_OK;
 }
 
 int launch_quantize(int kv_dtype, const __nv_bfloat16 *x, int64_t n_rows, int d, void *codes,

@@ -22,6 +22,10 @@ struct WorkspaceLayout {
   size_t part_o;       // float [split CTAs * segments * 2 * 128 * d]: partial outputs
   size_t nlse;         // float [B*Hq*row_tiles*128]: -lse2 per row of every row tile
   size_t status;       // int32: device status word (0 = ok, else an H2OKV_ERR_* code)
+  size_t ev_hist;      // uint32 [B*H_k][2048]: top-bit key histograms of the eviction (zero between calls)
+  size_t ev_arrive;    // uint32 [B*H_k]: arrival counters of the eviction (zero between calls)
+  size_t ev_slots;     // int32 [B*H_k][max_chunk]: chosen slots in slot order
+  size_t ev_zero_end;  // [ev_hist, ev_zero_end) is zeroed on create and reset
   size_t total;
 };
 
@@ -51,6 +55,7 @@ struct h2okv_cache {
   h2okv::TcPlan tc;
   uint64_t wait_timeout_ns;
   int32_t score_mode;  // h2okv_score_mode
+  int32_t sms;         // multiprocessors of the device the cache was created on (0 if unknown)
 };
 
 namespace h2okv {
@@ -74,6 +79,9 @@ int launch_init_cache(h2okv_cache *c, cudaStream_t st);
 int launch_evict_insert(h2okv_cache *c, const float *w_prev, const void *k_new, const void *v_new,
                         int S, int64_t P, int32_t *slots_out, const int32_t *slots_in,
                         const h2okv_delta *delta, cudaStream_t st);
+int launch_evict_insert_many(h2okv_cache *const *caches, int n, const float *const *w_prev,
+                             const void *const *k_new, const void *const *v_new, int S, int64_t P,
+                             int32_t *const *slots_out, cudaStream_t st);
 int launch_restore(h2okv_cache *c, const int32_t *slots, int S, const h2okv_delta *delta,
                    cudaStream_t st);
 int launch_attn_backward(h2okv_cache *c, const void *q, const void *dy, const float *lse, int S,

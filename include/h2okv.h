@@ -175,6 +175,20 @@ H2OKV_API int h2o_evict_insert(h2okv_cache *cache, const float *w_prev, const vo
                      const void *v_new, int32_t S, int64_t P, int32_t *slots_out,
                      void *stream);
 
+/* h2o_evict_insert on n_caches caches at once: one pair of launches for every
+ * (cache, b, h_k), for independent layers that advance chunk by chunk in step
+ * (the layer loop of §A.5.1 run with every layer's chunk inputs at hand).
+ * Host arrays of n_caches entries: caches (distinct handles that agree in
+ * their description, fill level and score mode), w_prev (NULL array = no
+ * fold; else every entry non-NULL), k_new, v_new, slots_out (NULL array, or
+ * entries that may be NULL); each entry is what h2o_evict_insert takes for
+ * that cache.  Same S and P for every cache.  On an argument error nothing is
+ * enqueued; the caches' workspaces must not be in use by other calls. */
+H2OKV_API int h2o_evict_insert_many(h2okv_cache *const *caches, int32_t n_caches,
+                                    const float *const *w_prev, const void *const *k_new,
+                                    const void *const *v_new, int32_t S, int64_t P,
+                                    int32_t *const *slots_out, void *stream);
+
 /* Score variant that ranks occupied slots in step 2 of h2o_evict_insert
  * ("Learning how to Forget", §3.1.1 Variants of Heavy-Hitter Oracle):
  *   H2OKV_SCORE_H2O       the cumulative score (default);
@@ -281,13 +295,15 @@ H2OKV_API int attn_chunk_with_scoresum(h2okv_cache *cache, const void *q, int32_
  * (keys/values/scales/token_pos as in h2okv_cache_buffers; q, y_out, lse_out,
  * w_out, wq_out as in attn_chunk_with_scoresum), on the library's CUDA-core
  * kernels.
- *   - Limit: batch * n_q_heads * S <= 262144 rows; larger calls return
- *     H2OKV_ERR_INVALID_ARG without enqueuing anything.
+ *   - Limit: batch * n_q_heads * S <= 262144 rows (and batch * n_kv_heads <=
+ *     65535); larger calls return H2OKV_ERR_INVALID_ARG without enqueuing
+ *     anything.
  *   - The array (1 MiB) exists on every GPU that loads the library and is held
  *     until the process exits.
- *   - The first call on a device looks up the array's device address
- *     (cudaGetSymbolAddress) with that device current; make that first call
- *     before any stream capture.
+ *   - Every call looks up the array's device address (cudaGetSymbolAddress)
+ *     with the caller's device current, so the address always belongs to the
+ *     current context.  The first call on a device also loads the library's
+ *     device code there; make that first call before any stream capture.
  *   - Every call on a device shares the one array and leaves the last call's
  *     contents in it; calls whose work overlaps on the GPU (different streams,
  *     no ordering between them) race on it and give undefined results.

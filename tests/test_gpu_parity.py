@@ -105,6 +105,48 @@ def test_quantize_bit_exact(kind, d, cuda_device):
     np.testing.assert_array_equal(codes.cpu().numpy().view(np.uint8), rc.view(np.uint8))
 
 
+def _bf16_rows_up_to(anchors, d, seed):
+    """Rows of d bf16 values: element 0 is +-A (it sets the row's absmax, hence its
+    scale), the other d - 1 run through every finite bf16 value with |x| <= A."""
+    bits = np.arange(65536, dtype=np.uint32).astype(np.uint16)
+    allv = (bits.astype(np.uint32) << 16).view(np.float32)
+    allv = allv[np.isfinite(allv)]
+    rng = np.random.default_rng(seed)
+    rows = []
+    for a in anchors:
+        a = float(np.float32(torch.tensor(a).to(torch.bfloat16).float()))
+        vals = allv[np.abs(allv) <= a]
+        n = -(-len(vals) // (d - 1))
+        pad = np.resize(vals, n * (d - 1))
+        block = np.empty((n, d), np.float32)
+        block[:, 0] = a * rng.choice([-1.0, 1.0], size=n)
+        block[:, 1:] = pad.reshape(n, d - 1)
+        rows.append(block)
+    return np.concatenate(rows)
+
+
+@pytest.mark.parametrize("kind", ["i8", "i4"])
+def test_quantize_every_bf16_value(kind, cuda_device):
+    """Every finite bf16 value x, quantized in rows whose scale ranges over fp16
+    normals, subnormals, the 65504 clamp and rounding ties of x / scale: codes and
+    scales equal the oracle's (IEEE float32 division), bit for bit."""
+    anchors = [2.0 ** e * m for e in range(-20, 21, 3) for m in (1.0, 1.015625, 1.5, 1.9921875)]
+    anchors += [7.0, 127.0, 3.5, 63.5, 6.5e-6, 1e-7, 4.0e6, 1e9, 1e30, 3e38]
+    x = _bf16_rows_up_to(anchors, 128, seed=11)
+    xb = torch.from_numpy(x).to(torch.bfloat16)
+    n, d = x.shape
+    row = d // 2 if kind == "i4" else d
+    codes = torch.empty((n, row), dtype=torch.int8 if kind == "i8" else torch.uint8, device=cuda_device)
+    scales = torch.empty((n,), dtype=torch.float16, device=cuda_device)
+    hb.kv_cache_quantize(kind, xb.to(cuda_device), codes, scales)
+    torch.cuda.synchronize()
+    rc, rs = oracle.quantize_rows(xb.float().numpy(), kind)
+    if kind == "i4":
+        rc = oracle.pack_int4(rc)
+    np.testing.assert_array_equal(scales.cpu().numpy().view(np.uint16), rs.view(np.uint16))
+    np.testing.assert_array_equal(codes.cpu().numpy().view(np.uint8), rc.view(np.uint8))
+
+
 # ---------------------------------------------------------------------------
 # Eviction: bit-exact on tie-heavy score arrays, every capacity regime.
 # ---------------------------------------------------------------------------
