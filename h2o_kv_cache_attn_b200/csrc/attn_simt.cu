@@ -14,7 +14,6 @@
 // g is head g*q_g + r / S, chunk row r % S.
 #include <math.h>
 
-#include <mutex>
 
 #include "h2okv_internal.cuh"
 
@@ -282,6 +281,17 @@ int run(SimtArgs &a, int B, cudaStream_t st) {
 
 }  // namespace
 
+// The CUDA-core grid (row tiles of one (batch row, KV head), B * H_k) must fit the launch
+// limits; checked before anything is enqueued.
+static int simt_grid_check(int B, int Hk, int q_g, int S) {
+  const long long gx = ((long long)q_g * S + kRows - 1) / kRows;
+  const long long gy = (long long)B * Hk;
+  if (gy > 65535 || gx > INT32_MAX)
+    return set_error(H2OKV_ERR_INVALID_ARG,
+                     "batch * n_kv_heads = %lld (max 65535) or query rows per group too large", gy);
+  return H2OKV_OK;
+}
+
 int launch_attn_simt(h2okv_cache *c, const void *q, int S, int64_t P, void *y, float *lse,
                      float *w, float *wq, cudaStream_t st) {
   const h2okv_cache_desc &d = c->desc;
@@ -306,6 +316,8 @@ int launch_attn_simt(h2okv_cache *c, const void *q, int S, int64_t P, void *y, f
   a.P = (int)P;
   a.row_bytes = c->row_bytes;
   a.scale2 = (float)(1.4426950408889634 / sqrt((double)d.head_dim));
+  const int grc = simt_grid_check(d.batch, d.n_kv_heads, a.q_g, S);
+  if (grc) return grc;
 
   const size_t nw = (size_t)d.batch * d.n_kv_heads * d.capacity * 4;
   if (cudaMemsetAsync(w, 0, nw, st) != cudaSuccess ||
@@ -334,33 +346,20 @@ namespace {
 
 // B * H_q * S rows the array holds (1 MiB of float per device).
 constexpr size_t kNoAllocMaxRows = size_t(1) << 18;
-constexpr int kNoAllocMaxDevices = 64;
 
 static __device__ __align__(256) float g_noalloc_lse2[kNoAllocMaxRows];
 
-std::mutex g_noalloc_mu;
-float *g_noalloc_ptr[kNoAllocMaxDevices];
-
-// Device address of the array on the current device.  In host code the array's
-// name is only a host-side stand-in, so its device address is looked up once per
-// device (with that device current) and cached.
+// Device address of the array for the current device and context.  In host code the
+// array's name is only a host-side stand-in, so the address is looked up, with the
+// device current, on every call: a host-side query that allocates nothing, and that
+// stays right if the context is torn down and made again (the module then loads at a
+// new address).
 int noalloc_scratch(float **out) {
-  int dev = 0;
-  cudaError_t e = cudaGetDevice(&dev);
+  void *ptr = nullptr;
+  const cudaError_t e = cudaGetSymbolAddress(&ptr, g_noalloc_lse2);
   if (e != cudaSuccess)
-    return set_error(H2OKV_ERR_CUDA, "cudaGetDevice: %s", cudaGetErrorString(e));
-  if (dev < 0 || dev >= kNoAllocMaxDevices)
-    return set_error(H2OKV_ERR_UNSUPPORTED, "device ordinal %d above %d", dev,
-                     kNoAllocMaxDevices - 1);
-  std::lock_guard<std::mutex> lock(g_noalloc_mu);
-  if (!g_noalloc_ptr[dev]) {
-    void *ptr = nullptr;
-    e = cudaGetSymbolAddress(&ptr, g_noalloc_lse2);
-    if (e != cudaSuccess)
-      return set_error(H2OKV_ERR_CUDA, "cudaGetSymbolAddress(scratch): %s", cudaGetErrorString(e));
-    g_noalloc_ptr[dev] = static_cast<float *>(ptr);
-  }
-  *out = g_noalloc_ptr[dev];
+    return set_error(H2OKV_ERR_CUDA, "cudaGetSymbolAddress(scratch): %s", cudaGetErrorString(e));
+  *out = static_cast<float *>(ptr);
   return H2OKV_OK;
 }
 
@@ -392,6 +391,8 @@ extern "C" int attn_chunk_with_scoresum_noalloc(const h2okv_cache_desc *desc, co
     return set_error(H2OKV_ERR_INVALID_ARG,
                      "batch * n_q_heads * S = %zu exceeds the %zu rows of the static scratch", rows,
                      kNoAllocMaxRows);
+  rc = simt_grid_check(desc->batch, desc->n_kv_heads, desc->n_q_heads / desc->n_kv_heads, S);
+  if (rc) return rc;
   float *scratch = nullptr;
   rc = noalloc_scratch(&scratch);
   if (rc) return rc;
