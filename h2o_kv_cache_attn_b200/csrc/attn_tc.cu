@@ -169,12 +169,6 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   return *reinterpret_cast<uint32_t *>(&v);
 }
 
-// Exponentials: in every group of 8 consecutive elements the last kPolyA (phase A)
-// or kPolyB (phase B) go to the FMA-pipe polynomial exp2_poly2, the others to the
-// MUFU ex2 unit, so that neither unit alone bounds the softmax warps.
-constexpr int kPolyA = 0;
-constexpr int kPolyB = 0;
-
 // Masking of one row of raw logits: a masked logit (slot relative position rel_e >
 // row index ri) drops by mbias = 2^30 / (logit scale), i.e. by 2^30 in base-2 units;
 // nm = sat(rel_e - ri) is 1 for a masked slot, 0 for a visible one.
@@ -218,11 +212,7 @@ __device__ __forceinline__ void row_update(const uint32_t (&x)[N], float c2, flo
   for (int e = 0; e < N; e += 2) {
     const float2 a =
         fma2(make_float2(__uint_as_float(x[e]), __uint_as_float(x[e + 1])), c2v, negm);
-    float2 v;
-    if ((e & 7) >= 8 - kPolyA)
-      v = exp2_poly2(a);
-    else
-      v = make_float2(ex2(a.x), ex2(a.y));
+    const float2 v = make_float2(ex2(a.x), ex2(a.y));
     acc[(e >> 1) & 3] = add2(acc[(e >> 1) & 3], v);
   }
   const float2 s01 = add2(acc[0], acc[1]), s23 = add2(acc[2], acc[3]);
@@ -257,11 +247,7 @@ __device__ __forceinline__ float slot_probs(const uint32_t (&r)[BM], const float
       const float2 nm = make_float2(fma_sat(rminf, 1.f, -(float)e), fma_sat(rminf, 1.f, -(float)(e + 1)));
       a = fma2(nm, make_float2(-kMaskBias, -kMaskBias), a);
     }
-    float2 v;
-    if ((e & 7) >= 8 - kPolyB)
-      v = exp2_poly2(a);
-    else
-      v = make_float2(ex2(a.x), ex2(a.y));
+    float2 v = make_float2(ex2(a.x), ex2(a.y));
     if (rmax < BM) {  // rows past the chunk (last row tile only)
       v.x = e < rmax ? v.x : 0.f;
       v.y = e + 1 < rmax ? v.y : 0.f;

@@ -295,27 +295,6 @@ __device__ __forceinline__ float2 mul2(float2 a, float2 b) {
   return bits_f2(d);
 }
 
-// 2^x for a pair, on the FMA pipe: x = n + f with n = rint(x) (the 1.5 * 2^23
-// rounding constant), f in [-1/2, 1/2]; 2^f by a degree-4 polynomial (near-minimax
-// relative-error fit, exp2_poly_coeffs.py: max relative error 2.7e-6); 2^n by adding
-// n to the exponent field.  Inputs are clamped to [-126, +inf) so the exponent
-// never wraps; results below 2^-126 come out as tiny positives instead of 0.
-__device__ __forceinline__ float2 exp2_poly2(float2 x) {
-  x.x = fmaxf(x.x, -126.f);
-  x.y = fmaxf(x.y, -126.f);
-  const float2 magic = make_float2(12582912.f, 12582912.f);
-  const float2 t = add2(x, magic);
-  const float2 n = add2(t, make_float2(-12582912.f, -12582912.f));
-  const float2 f = fma2(n, make_float2(-1.f, -1.f), x);
-  float2 p = fma2(make_float2(0.009570101276040077f, 0.009570101276040077f), f,
-                  make_float2(0.05591786280274391f, 0.05591786280274391f));
-  p = fma2(p, f, make_float2(0.240247443318367f, 0.240247443318367f));
-  p = fma2(p, f, make_float2(0.6931217908859253f, 0.6931217908859253f));
-  p = fma2(p, f, make_float2(0.9999992847442627f, 0.9999992847442627f));
-  return make_float2(__uint_as_float(__float_as_uint(p.x) + (__float_as_uint(t.x) << 23)),
-                     __uint_as_float(__float_as_uint(p.y) + (__float_as_uint(t.y) << 23)));
-}
-
 // Two non-negative floats to packed bf16 (low half = lo), rounded to nearest with
 // ties away from zero, on the integer pipe.
 __device__ __forceinline__ uint32_t pack_bf16x2_int(float lo, float hi) {
