@@ -68,3 +68,23 @@ def test_algorithmic_flops(config):
     n = wl.capacity
     assert bench.alg_flops_chunk(wl, n, wl.chunk) == 4.0 * wl.B * wl.Hq * wl.chunk * n * wl.d
     assert bench.exec_flops_chunk(wl, n, wl.chunk) == 1.5 * bench.alg_flops_chunk(wl, n, wl.chunk)
+
+
+def test_launch_counts_follow_the_library_rules():
+    from h2o_kv_cache_attn_b200.configs import SHORT
+    assert bench.evict_launches(0, 0, 100) == 1          # fold only
+    assert bench.evict_launches(0, 64, 100) == 2         # filling: fold + rows
+    assert bench.evict_launches(64, 64, 100) == 3        # choosing: fold + choose + rows
+    wl = SHORT["128k"]
+    assert bench.attention_launches(wl, 1024, 32768, 148) == 3  # 128 pairs fill 86 % of a wave
+    assert bench.attention_launches(SHORT["tiny"], 128, 256, 148) == 2  # CUDA-core path
+
+
+def test_stack_flops_and_bytes_scale_with_layers():
+    from h2o_kv_cache_attn_b200.configs import SHORT
+    wl = SHORT["int4stack"]
+    one = bench.evict_bytes_chunk(wl, wl.chunk)
+    # per (b, h_k): 12 N_C + 4 S d + 2 S (row + scale) + 8 S bytes
+    per = 12 * 32768 + 4 * 2048 * 128 + 2 * 2048 * (64 + 2) + 8 * 2048
+    assert one == per * 4 * 8
+    assert bench.alg_flops_chunk(wl, 32768, 2048) == 4.0 * 4 * 32 * 2048 * 32768 * 128
