@@ -4,29 +4,25 @@
 // §A.5.3 keys' = scatter(keys, index, key_new)), plus the 8/4-bit row
 // quantizer used on insert.
 //
-// One call = two launches on the caller's stream:
+// One call = up to three launches on the caller's stream, chained by programmatic
+// dependent launch (each next kernel is scheduled early and waits for the previous
+// one with griddepcontrol.wait):
 //
-//   evict_select_kernel  C CTAs per group (a group is one (batch row, KV head),
-//     or one KV head over every batch row for the h2o_orig variant), each over
-//     a contiguous slice of the N_C slots:
-//       1. folds w_prev into the float32 scores and stores them; while the
-//          cache is filling (n_filled + S <= N_C) it also claims slots
-//          n_filled + k for the chunk rows k (token position, score 0);
-//       2. choosing: forms order-preserving uint32 selection keys (0 for an
-//          empty slot, so empty slots come first) and a 2048-bin histogram of
-//          their top 11 bits, adds it into the group's histogram in the
-//          workspace and counts itself in; the CTA that arrives last owns the
-//          rest of the choice: it finds the bin of the S-th smallest key,
-//          reads the group's keys back from L2 into shared memory, refines the
-//          threshold over bits 20..10 and 9..0 (two more histograms, only for
-//          keys in the chosen bins), lists the chosen slots in slot order with
-//          one block scan (ties at the threshold go to the lowest slots), and
-//          claims them; it leaves the histogram and counter at zero.
-//   evict_rows_kernel  launched as a programmatic dependent of the select
-//     kernel: it loads its first new key/value rows while the selection runs,
-//     then waits for it (griddepcontrol.wait) and writes (copies, or
-//     quantizes for 8/4-bit caches) every chunk row into its slot, with the
-//     overwritten row saved first for the delta encoding.
+//   evict_fold_kernel    C CTAs per group (a group is one (batch row, KV head), or one
+//     KV head over every batch row for the h2o_orig variant), each over a slice of
+//     the N_C slots: folds w_prev into the float32 scores and stores them; while the
+//     cache is filling (n_filled + S <= N_C) it claims slots n_filled + k for the
+//     chunk rows k; when choosing, it adds the slice's histogram of the top 11 bits
+//     of the order-preserving selection keys (0 for an empty slot, so empty slots
+//     come first) into the group's histogram in the workspace.
+//   evict_choose_kernel  (choosing only) one CTA per group: finds the bin of the
+//     S-th smallest key, marks the slots below it and in it (the candidates) in two
+//     bitmasks, refines the threshold over the candidates (bits 20..10, 9..0; ties
+//     go to the lowest slots) and lists the chosen slots in slot order.
+//   evict_rows_kernel    over every chunk row, key and value: loads the new rows
+//     while the earlier kernels run, then writes (copies, or quantizes for 8/4-bit
+//     caches) each into its slot, saving the overwritten row first for the delta
+//     encoding, and claims chosen or replayed slots (token position, score 0).
 //
 // A call over many caches of the same shape (independent layers) runs as the
 // same two launches over every (cache, group).  The quantizer must agree bit
@@ -48,7 +44,6 @@ constexpr int kHistBins = 1 << kTopBits;
 constexpr int kMidBins = 2048;  // key bits 20..10
 constexpr int kLowBins = 1024;  // key bits 9..0
 constexpr int kSmemKeysMax = 32768;  // largest N_C whose keys the last CTA keeps in shared memory
-constexpr int kSlotListMax = 4096;   // chosen slots the last CTA lists in shared memory
 constexpr int kRowThreads = 256;     // threads of a row CTA
 constexpr int kRowWarps = kRowThreads / 32;
 constexpr int kCopyUnroll = 8;   // 16-byte pieces per thread in flight in the row copy
@@ -175,6 +170,14 @@ __device__ __forceinline__ void sts32(uint32_t a, int v) {
   asm volatile("st.shared.u32 [%0], %1;" ::"r"(a), "r"(v) : "memory");
 }
 
+// hs[bin] += 1 for the calling lane: lanes (of those active together) that share a bin
+// add once, with their count.  Selection keys are often crowded into a few bins (scores
+// of one chunk's age are alike), where lane-by-lane atomics would serialize.
+__device__ __forceinline__ void hist_add(uint32_t *hs, uint32_t bin) {
+  const uint32_t peers = __match_any_sync(__activemask(), bin);
+  if ((threadIdx.x & 31) == __ffs(peers) - 1) atomicAdd(&hs[bin], __popc(peers));
+}
+
 // Selection key of one slot from its (folded) score sum over the group's batch rows and
 // the token position of batch row 0.
 __device__ __forceinline__ uint32_t sel_key(float ksum, int32_t tp, int score_mode, int P) {
@@ -240,21 +243,6 @@ __device__ __forceinline__ void find_bin(const uint32_t *hs, uint32_t kk, uint32
     }
   }
   __syncthreads();
-}
-
-// Slot j of a group gets chunk row k: bookkeeping for every batch row of the group
-// (old position to the delta output, new position, score 0, slot list).
-template <int NT>
-__device__ __forceinline__ void claim(const EvParams<NT> &p, const EvTarget &T, int g, int j,
-                                      int k) {
-  for (int bb = 0; bb < p.nb; ++bb) {
-    const size_t bh = bh_of(p, g, bb);
-    const size_t gs = bh * p.N_C + j, rk = bh * p.S + k;
-    if (T.dpos) __stcg(T.dpos + rk, __ldcg(T.token_pos + gs));
-    __stcg(T.token_pos + gs, p.P + k);
-    __stcg(T.scores + gs, 0.f);
-    if (T.slots_out) __stcg(T.slots_out + rk, j);
-  }
 }
 
 // ---- fold kernel ---------------------------------------------------------------------
@@ -336,7 +324,7 @@ __global__ void __launch_bounds__(kSelThreads)
 #pragma unroll
         for (int e = 0; e < 4; ++e)
           if (j4 + e < j_end)
-            atomicAdd(&hs[sel_key(ks[u][e], tp[u][e], p.score_mode, p.P) >> (32 - kTopBits)], 1u);
+            hist_add(hs, sel_key(ks[u][e], tp[u][e], p.score_mode, p.P) >> (32 - kTopBits));
       }
     }
   }
@@ -386,14 +374,14 @@ __global__ void __launch_bounds__(kChooseThreads, 1)
   const EvTarget &T = p.t[ti];
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   __shared__ uint32_t hs[kHistBins];
+  __shared__ uint32_t hs2[kMidBins];
   __shared__ uint32_t wscan[kChooseWarps];
   __shared__ uint32_t res[4];
   __shared__ __align__(8) uint64_t bar;
   __shared__ uint32_t below_w[kChooseThreads * kMaxWordsPerThread];  // slots below the bin
   __shared__ uint32_t cand_w[kChooseThreads * kMaxWordsPerThread];   // slots in the bin
-  extern __shared__ __align__(16) unsigned char dyn[];  // [kSlotListMax] slots, [N_C] keys
-  const uint32_t slist_a = smem_u32(dyn);
-  const uint32_t keys_a = slist_a + kSlotListMax * 4u;
+  extern __shared__ __align__(16) unsigned char dyn[];  // [N_C] scores or keys (KM 1, 2)
+  const uint32_t keys_a = smem_u32(dyn);
 
   const int n_words = (p.N_C + 31) >> 5;
   if (KM == 2 && tid == 0) {
@@ -451,36 +439,30 @@ __global__ void __launch_bounds__(kChooseThreads, 1)
     }
   }
 
-  // ---- bitmasks: word w holds slots 32w .. 32w + 31, one per lane of a warp step --------
+  // ---- bitmasks: word w holds slots 32w .. 32w + 31, one per lane of a warp step; the
+  // candidates' bits 20..10 are counted on the way (in a second histogram) -------------
+  for (int i = tid; i < kMidBins; i += kChooseThreads) hs2[i] = 0u;
+  __syncthreads();
 #pragma unroll 4
   for (int w = warp; w < n_words; w += kChooseWarps) {
     const int j = 32 * w + lane;
     const bool okj = j < p.N_C;
-    const uint32_t b = okj ? KEY_AT(j) >> (32 - kTopBits) : 0xffffffffu;
+    const uint32_t key = okj ? KEY_AT(j) : 0xffffffffu;
+    const uint32_t b = okj ? key >> (32 - kTopBits) : 0xffffffffu;
     const uint32_t bm = __ballot_sync(0xffffffffu, b < top);
     const uint32_t cm = __ballot_sync(0xffffffffu, b == top);
     if (lane == 0) {
       below_w[w] = bm;
       cand_w[w] = cm;
     }
+    if (b == top) hist_add(hs2, (key >> 10) & 2047u);
   }
-  for (int i = tid; i < kMidBins; i += kChooseThreads) hs[i] = 0u;
   __syncthreads();
 
   // ---- threshold: bits 20..10, then 9..0, of the candidates ------------------------------
   // thread t owns words t * wpt .. t * wpt + wpt - 1 (slot order follows thread order)
   const int wpt = (n_words + kChooseThreads - 1) / kChooseThreads;
-#pragma unroll
-  for (int q = 0; q < kMaxWordsPerThread; ++q) {
-    const int w = tid * wpt + q;
-    if (q >= wpt || w >= n_words) break;
-    for (uint32_t m = cand_w[w]; m; m &= m - 1u) {
-      const uint32_t key = KEY_AT(32 * w + __ffs(m) - 1);
-      atomicAdd(&hs[(key >> 10) & 2047u], 1u);
-    }
-  }
-  __syncthreads();
-  find_bin<kChooseThreads, kMidBins>(hs, kk, wscan, res);
+  find_bin<kChooseThreads, kMidBins>(hs2, kk, wscan, res);
   const uint32_t pre = (top << 11) | res[0];  // key bits 31..10
   kk = res[1];
   for (int i = tid; i < kLowBins; i += kChooseThreads) hs[i] = 0u;
@@ -491,7 +473,7 @@ __global__ void __launch_bounds__(kChooseThreads, 1)
     if (q >= wpt || w >= n_words) break;
     for (uint32_t m = cand_w[w]; m; m &= m - 1u) {
       const uint32_t key = KEY_AT(32 * w + __ffs(m) - 1);
-      if ((key >> 10) == pre) atomicAdd(&hs[key & 1023u], 1u);
+      if ((key >> 10) == pre) hist_add(hs, key & 1023u);
     }
   }
   __syncthreads();
@@ -526,30 +508,12 @@ __global__ void __launch_bounds__(kChooseThreads, 1)
   }
   uint32_t pos = block_exclusive_scan<kChooseThreads, uint32_t>(n_take, wscan);
 
-  // ---- the chosen slots in slot order ----------------------------------------------------
-  const bool list_smem = p.S <= kSlotListMax;
+  // ---- the chosen slots in slot order (the row kernel claims them) -----------------------
   int32_t *slist = T.slotlist + (size_t)g * p.S;
 #pragma unroll
   for (int q = 0; q < kMaxWordsPerThread; ++q) {
     const int w = tid * wpt + q;
-    for (uint32_t m = lt[q]; m; m &= m - 1u, ++pos) {
-      const int j = 32 * w + __ffs(m) - 1;
-      if (list_smem) {
-        sts32(slist_a + 4u * pos, j);
-      } else {
-        __stcg(slist + pos, j);
-        claim(p, T, g, j, (int)pos);
-      }
-    }
-  }
-  if (list_smem) {
-    __syncthreads();
-#pragma unroll 1
-    for (int k = tid; k < p.S; k += kChooseThreads) {
-      const int j = lds32(slist_a + 4u * k);
-      __stcg(slist + k, j);
-      claim(p, T, g, j, k);
-    }
+    for (uint32_t m = lt[q]; m; m &= m - 1u, ++pos) __stcg(slist + pos, 32 * w + __ffs(m) - 1);
   }
 }
 #undef KEY_AT
@@ -584,10 +548,11 @@ __device__ __forceinline__ int slot_of(const EvParams<NT> &p, const RowSet<NT> &
   return (j >= 0 && j < p.N_C) ? j : -1;
 }
 
-// Replay: the bookkeeping of a logged slot (done once per chunk row, with its key row).
+// The bookkeeping of a chosen (mode 2) or logged (mode 3) slot, once per chunk row with
+// its key row: old position to the delta output, new position, score 0, slot list out.
 template <int NT>
-__device__ __forceinline__ void replay_claim(const EvParams<NT> &p, const RowSet<NT> &rs, int k,
-                                             int j) {
+__device__ __forceinline__ void row_claim(const EvParams<NT> &p, const RowSet<NT> &rs, int k,
+                                          int j) {
   const EvTarget &T = *rs.T;
   if (j < 0) {
     atomicExch(T.status, H2OKV_ERR_INVALID_ARG);
@@ -597,6 +562,7 @@ __device__ __forceinline__ void replay_claim(const EvParams<NT> &p, const RowSet
   if (T.dpos) __stcg(T.dpos + rk, __ldcg(T.token_pos + gs));
   __stcg(T.token_pos + gs, p.P + k);
   __stcg(T.scores + gs, 0.f);
+  if (p.mode == 2 && T.slots_out) __stcg(T.slots_out + rk, j);
 }
 
 // f32 / bf16 caches: the set's rows are cut into 16-byte pieces (e = (2k + t) * PC + c),
@@ -640,7 +606,7 @@ __device__ __forceinline__ void copy_rows(const EvParams<NT> &p) {
     for (int u = 0; u < kCopyUnroll; ++u) {
       if (rr[u] < 0) continue;
       const int k = rr[u] >> 1, t = rr[u] & 1;
-      if (p.mode == 3 && t == 0 && cc[u] == 0) replay_claim(p, rs, k, slot[u]);
+      if (p.mode >= 2 && t == 0 && cc[u] == 0) row_claim(p, rs, k, slot[u]);
       if (slot[u] < 0) continue;
       uint4 *dst = (t ? dst_v : dst_k) + (size_t)slot[u] * PC + cc[u];
       if (DELTA && T.dk) {
@@ -719,7 +685,7 @@ __device__ __forceinline__ void quantize_rows(const EvParams<NT> &p) {
       if (it >= items || li >= G8) continue;
       const int t = it & 1, k = it >> 1;
       const int j = slot[u];
-      if (p.mode == 3 && t == 0 && li == 0) replay_claim(p, rs, k, j);
+      if (p.mode >= 2 && t == 0 && li == 0) row_claim(p, rs, k, j);
       if (j < 0) continue;
       const size_t drow = rs.bh * p.N_C + j, crow = rs.bh * p.S + k;
       uint8_t *codes = (t ? T.values : T.keys) + drow * (size_t)p.row_bytes;
@@ -893,7 +859,7 @@ int opt_in_choose() {
   if (!done[dev]) {
     cudaError_t e = cudaFuncSetAttribute(
         evict_choose_kernel<NT, KM>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-        (int)(kSmemKeysMax * 4 + kSlotListMax * sizeof(int32_t)));
+        (int)(kSmemKeysMax * 4));
     if (e != cudaSuccess)
       return set_error(H2OKV_ERR_CUDA, "cudaFuncSetAttribute(evict_choose_kernel): %s",
                        cudaGetErrorString(e));
@@ -982,7 +948,7 @@ int launch_evict_t(h2okv_cache *const *caches, int n, const EvTarget *targets, c
     const int km = !fits ? 0
                    : (p.vec && p.nb == 1 && !p.need_tp && p.score_mode != H2OKV_SCORE_H2O_NORM) ? 2
                                                                                             : 1;
-    const size_t smem = kSlotListMax * sizeof(int32_t) + (fits ? (size_t)d.capacity * 4 : 0);
+    const size_t smem = fits ? (size_t)d.capacity * 4 : 0;
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3((unsigned)units);
     cfg.blockDim = dim3(kChooseThreads);
