@@ -320,6 +320,8 @@ int run_bwd(const BwdArgs &a, int batch, cudaStream_t st) {
 int launch_attn_backward(h2okv_cache *c, const void *q, const void *dy, const float *lse, int S,
                          int64_t P, float *dq, float *dk, float *dv, cudaStream_t st) {
   const h2okv_cache_desc &d = c->desc;
+  // bf16 cache, d = 128: the tensor-core kernels (attn_bwd_tc.cu)
+  if (bwd_tc_supported(d)) return launch_attn_backward_tc(c, q, dy, lse, S, P, dq, dk, dv, st);
   BwdArgs a;
   a.q = q;
   a.dy = dy;

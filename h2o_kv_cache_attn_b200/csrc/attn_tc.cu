@@ -2757,12 +2757,14 @@ __global__ void __launch_bounds__(256)
   w[(size_t)bg * N_C + j] = tot;
 }
 
+}  // namespace
+
 typedef CUresult (*EncodeTiledFn)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *,
                                    const cuuint64_t *, const cuuint64_t *, const cuuint32_t *,
                                    const cuuint32_t *, CUtensorMapInterleave, CUtensorMapSwizzle,
                                    CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
 
-EncodeTiledFn encode_fn() {
+static EncodeTiledFn encode_fn() {
   static EncodeTiledFn fn = nullptr;
   if (!fn) {
     void *ptr = nullptr;
@@ -2790,7 +2792,24 @@ int encode_rows_map(CUtensorMap *map, const void *base, uint64_t rows, uint64_t 
   return H2OKV_OK;
 }
 
-}  // namespace
+
+int ensure_cache_maps(h2okv_cache *c) {
+  if (c->tc.maps_ready) return H2OKV_OK;
+  const h2okv_cache_desc &d = c->desc;
+  if (d.kv_dtype != H2OKV_BF16) {  // codes are read with plain loads: no maps for the cache
+    memset(c->tc.k_map, 0, sizeof(c->tc.k_map));
+    memset(c->tc.v_map, 0, sizeof(c->tc.v_map));
+  } else {
+    int rc = encode_rows_map(reinterpret_cast<CUtensorMap *>(c->tc.k_map), c->bufs.keys,
+                             (uint64_t)d.capacity, (uint64_t)d.batch * d.n_kv_heads);
+    if (rc) return rc;
+    rc = encode_rows_map(reinterpret_cast<CUtensorMap *>(c->tc.v_map), c->bufs.values,
+                         (uint64_t)d.capacity, (uint64_t)d.batch * d.n_kv_heads);
+    if (rc) return rc;
+  }
+  c->tc.maps_ready = true;
+  return H2OKV_OK;
+}
 
 bool tc_path_supported(const h2okv_cache_desc &d) {
   return d.head_dim == D && d.q_dtype == H2OKV_BF16 &&
@@ -2942,23 +2961,10 @@ int launch_attn_tc(h2okv_cache *c, const void *q, int S, int64_t P, void *y, flo
                    float *wq, cudaStream_t st) {
   const h2okv_cache_desc &d = c->desc;
   uint8_t *ws = reinterpret_cast<uint8_t *>(c->bufs.workspace);
-  const bool quant = d.kv_dtype != H2OKV_BF16;
-  if (!c->tc.maps_ready) {
-    if (quant) {  // codes are read with plain loads: no maps for the cache
-      memset(c->tc.k_map, 0, sizeof(c->tc.k_map));
-      memset(c->tc.v_map, 0, sizeof(c->tc.v_map));
-    } else {
-      int rc = encode_rows_map(reinterpret_cast<CUtensorMap *>(c->tc.k_map), c->bufs.keys,
-                               (uint64_t)d.capacity, (uint64_t)d.batch * d.n_kv_heads);
-      if (rc) return rc;
-      rc = encode_rows_map(reinterpret_cast<CUtensorMap *>(c->tc.v_map), c->bufs.values,
-                           (uint64_t)d.capacity, (uint64_t)d.batch * d.n_kv_heads);
-      if (rc) return rc;
-    }
-    c->tc.maps_ready = true;
-  }
+  int rc = ensure_cache_maps(c);
+  if (rc) return rc;
   CUtensorMap qmap;
-  int rc = encode_rows_map(&qmap, q, (uint64_t)S, (uint64_t)d.batch * d.n_q_heads);
+  rc = encode_rows_map(&qmap, q, (uint64_t)S, (uint64_t)d.batch * d.n_q_heads);
   if (rc) return rc;
 
   TcParams prm;

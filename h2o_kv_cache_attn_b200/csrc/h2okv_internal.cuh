@@ -1,6 +1,7 @@
 // Internal declarations shared by the library's translation units.
 #pragma once
 
+#include <cuda.h>
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
 #include <cuda_runtime.h>
@@ -94,5 +95,12 @@ bool tc_path_supported(const h2okv_cache_desc &d);
 int launch_attn_tc(h2okv_cache *c, const void *q, int S, int64_t P, void *y, float *lse, float *w,
                    float *wq, cudaStream_t st);
 void tc_plan(const h2okv_cache_desc &d, TcPlan *plan);
+// 3-D bf16 tensor map over [planes][rows][128] with a (64 x 128 x 1) box, 128-byte swizzle.
+int encode_rows_map(CUtensorMap *map, const void *base, uint64_t rows, uint64_t planes);
+// The cache's key / value tensor maps (bf16 caches), encoded once.
+int ensure_cache_maps(h2okv_cache *c);
+bool bwd_tc_supported(const h2okv_cache_desc &d);
+int launch_attn_backward_tc(h2okv_cache *c, const void *q, const void *dy, const float *lse, int S,
+                            int64_t P, float *dq, float *dk, float *dv, cudaStream_t st);
 
 }  // namespace h2okv
