@@ -1,12 +1,14 @@
 """A short, steady-state run of the hot path for profiler captures.
 
-``python -m h2o_kv_cache_attn_b200.profile_case [--config 128k] [--iters 3]``
+``python -m h2o_kv_cache_attn_b200.profile_case [--config 128k] [--iters 3] [--backward]``
 
 Fills one layer's cache directly (every slot occupied, random keys, values and
 scores), then runs ``--iters`` eviction chunks (h2o_evict_insert followed by
-attn_chunk_with_scoresum).  Only a handful of launches precede the measured
-ones, so a profiler can capture e.g. the second attention launch of a full
-128K-token / 32768-slot layer with the cache larger than L2.
+attn_chunk_with_scoresum), or with ``--backward`` one attention call (for the
+row log-sum-exp) and ``--iters`` calls of attn_chunk_backward on that chunk.
+Only a handful of launches precede the measured ones, so a profiler can capture
+e.g. the second attention launch of a full 128K-token / 32768-slot layer with
+the cache larger than L2.
 """
 
 from __future__ import annotations
@@ -23,6 +25,7 @@ def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--config", default="128k", choices=sorted(SHORT))
     ap.add_argument("--iters", type=int, default=3)
+    ap.add_argument("--backward", action="store_true")
     args = ap.parse_args()
     wl = SHORT[args.config]
     dev = torch.device("cuda:0")
@@ -49,6 +52,22 @@ def main():
     v = torch.randn((wl.B, wl.Hk, S, wl.d), generator=g, device=dev).to(kvt)
     run.P = wl.capacity
     run.chunk_index = 1  # the cache is full: the first w_prev is the zero buffer
+    if args.backward:
+        y = torch.empty_like(q)
+        lse = torch.empty(q.shape[:3], dtype=torch.float32, device=dev)
+        run.cache.attend(q, S, run.P, y, lse, run.w[0], None)
+        dy = torch.randn(q.shape, generator=g, device=dev).to(qt)
+        dq = torch.empty(q.shape, dtype=torch.float32, device=dev)
+        dk = torch.empty((wl.B, wl.Hk, wl.capacity, wl.d), dtype=torch.float32, device=dev)
+        dv = torch.empty_like(dk)
+        for _ in range(args.iters):
+            run.cache.attend_backward(q, dy, lse, S, run.P, dq, dk, dv)
+        torch.cuda.synchronize()
+        ok = bool(torch.isfinite(dq).all() and torch.isfinite(dk).all() and torch.isfinite(dv).all())
+        print(f"profile_case {wl.name}: {args.iters} backward calls, finite gradients: {ok}")
+        if not ok:
+            raise SystemExit("non-finite gradients")
+        return
     for _ in range(args.iters):
         run.step(q, k, v)
     torch.cuda.synchronize()

@@ -234,9 +234,20 @@ def _sampled(wl, n_extra_mid=1):
 @pytest.mark.parametrize("wl", [QWEN_64K, QWEN_128K, QWEN_INT8], ids=lambda w: w.name)
 def test_full_size_sampled(wl, cuda_device):
     src = ChunkSource(wl, 0, cuda_device)
-    run, n = run_and_check(wl, cuda_device, check_chunks=_sampled(wl), groups=[(0, 0), (0, 5)],
-                           with_wq=False, source=src)
+    run, n = run_and_check(wl, cuda_device, check_chunks=_sampled(wl),
+                           groups=[(0, 0), (0, 3), (0, 5), (0, 7)], with_wq=False, source=src)
     assert n == len(_sampled(wl))
+
+
+def test_full_size_128k_per_head_sums_sampled(cuda_device):
+    """The per-query-head summed weights (wq) of the 128K layer at full size, as the
+    bench's split and every-SM schedules produce them, on a fill and an eviction chunk."""
+    wl = QWEN_128K
+    src = ChunkSource(wl, 0, cuda_device)
+    n_fill = -(-wl.capacity // wl.chunk)
+    run, n = run_and_check(wl, cuda_device, check_chunks={n_fill - 1, n_fill + 5},
+                           groups=[(0, 2), (0, 6)], with_wq=True, source=src)
+    assert n == 2
 
 
 def test_full_size_int4_stack_one_layer_sampled(cuda_device):
