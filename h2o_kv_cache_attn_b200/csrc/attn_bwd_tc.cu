@@ -6,19 +6,24 @@
 //   dq_i = sum_j dS_ij k_j / sqrt(d),
 //   dk_j = sum over the group's heads and rows of dS_ij q_i / sqrt(d),
 //   dv_j = sum over the group's heads and rows of p_ij dy_i.
-// Two kernels, each with one loader warp (TMA, no multicast), one MMA warp and one
-// warpgroup whose threads own the 128 TMEM lanes:
+// Two kernels, each with one loader warp (TMA, no multicast), one MMA warp and two
+// warpgroups of lane warps: the warps w and w + 4 share TMEM lane quarter w mod 4 and
+// split the tile's columns in halves.
 //   bwd_dq_tc_kernel    one CTA per 128 packed rows of a group (row-stationary):
 //                       streams the group's K/V tiles twice.  Pass 1: S = Q K^T and
-//                       dP = dY V^T into TMEM, D_i summed in registers (one thread per
-//                       row).  Pass 2: S, dP again; dS written to TMEM (hi term over
-//                       S, lo term in spare columns); dQ += dS K with dS read from
-//                       TMEM.  Writes dq and D.
+//                       dP = dY V^T into one of two TMEM buffers (the next tile's
+//                       products run while the lanes read this one), D_i summed in
+//                       registers (one row per lane, each half over its 64 slots, the
+//                       halves added at the end).  Pass 2: S, dP again; dS written back
+//                       over S by 32-slot chunks (hi term, then lo term); dQ += dS K
+//                       with dS read from TMEM, a chunk's k-steps issued as soon as the
+//                       chunk is written.  Writes dq and D.
 //   bwd_dkdv_tc_kernel  one CTA per 128 slots of a group (slot-stationary): streams
 //                       every packed row tile of the group.  S^T = K Q^T and
-//                       dP^T = V dY^T into TMEM; one thread per slot forms P^T and dS^T
-//                       (written back over S^T / dP^T as hi and lo terms); dV += P^T dY
-//                       and dK += dS^T Q with P^T, dS^T read from TMEM.
+//                       dP^T = V dY^T into TMEM; one slot per lane forms P^T and dS^T
+//                       by 32-row chunks (written back over S^T / dP^T as hi and lo
+//                       terms); dV += P^T dY and dK += dS^T Q with P^T, dS^T read from
+//                       TMEM, again chunk by chunk.
 // Every output element is summed by one CTA in a fixed order (no atomics).  The
 // probabilities and dS enter the second products as two bf16 terms each (hi + lo,
 // one MMA per term): a single bf16 rounding of dS, amplified by the cancellation in
@@ -37,7 +42,8 @@ constexpr int BT = 128;                      // rows / slots per tile
 constexpr int HD = 128;                      // head dim
 constexpr uint32_t kTile = BT * HD * 2;      // one bf16 tile: two 64-column swizzled halves
 constexpr uint32_t kHalf = kTile / 2;
-constexpr int kThr = 192;                    // warp 0 loads, warp 1 MMAs, warps 2-5 lanes
+constexpr int kLaneWarps = 8;                // two warps per TMEM lane quarter
+constexpr int kThr = 64 + 32 * kLaneWarps;   // warp 0 loads, warp 1 MMAs, warps 2-9 lanes
 constexpr float kFar = 1048576.f;            // relative position no row of the chunk reaches
 constexpr uint32_t IDESC_KK = idesc_bf16_f32(128, 128, false, false);  // A, B K-major
 constexpr uint32_t IDESC_TM = idesc_bf16_f32(128, 128, false, true);   // A (TMEM), B MN-major
@@ -52,13 +58,18 @@ __device__ __forceinline__ uint64_t mdesc(uint32_t base, int ks) {
 }
 // Two values as bf16 pairs split in two terms: x = hi + lo up to 2^-17 |x|
 // (hi = bf16(x), lo = bf16(x - hi)); the products that take them run once per term.
-__device__ __forceinline__ void split2(float a, float b, uint32_t &hi, uint32_t &lo) {
-  const __nv_bfloat162 h = __floats2bfloat162_rn(a, b);
+__device__ __forceinline__ void split2(float2 x, uint32_t &hi, uint32_t &lo) {
+  const __nv_bfloat162 h = __floats2bfloat162_rn(x.x, x.y);
   const float2 hf = __bfloat1622float2(h);
-  const __nv_bfloat162 l = __floats2bfloat162_rn(a - hf.x, b - hf.y);
+  const float2 d = fma2(hf, make_float2(-1.f, -1.f), x);
+  const __nv_bfloat162 l = __floats2bfloat162_rn(d.x, d.y);
   hi = *reinterpret_cast<const uint32_t *>(&h);
   lo = *reinterpret_cast<const uint32_t *>(&l);
 }
+__device__ __forceinline__ float2 u2f2(uint32_t a, uint32_t b) {
+  return make_float2(__uint_as_float(a), __uint_as_float(b));
+}
+__device__ __forceinline__ float2 ex2_2(float2 x) { return make_float2(ex2(x.x), ex2(x.y)); }
 
 struct BwdTcParams {
   const int32_t *token_pos;  // [B*Hk][N_C]
@@ -88,11 +99,21 @@ __device__ __forceinline__ float rel_of(const int32_t *tpg, int j, int N_C, int 
 // ---- dq (and D) ----------------------------------------------------------------------
 constexpr uint32_t Q_OFF = 0, DY_OFF = kTile, K_OFF = 2 * kTile, V_OFF = 4 * kTile;
 constexpr uint32_t REL_OFF = 6 * kTile;                    // float [2 stages][BT]
-constexpr uint32_t QBAR_OFF = REL_OFF + 2 * BT * 4;
-enum { QB_Q = 0, QB_KF0, QB_KE0 = QB_KF0 + 2, QB_SF = QB_KE0 + 2, QB_SR, QB_PF, QB_DONE, QB_END };
+constexpr uint32_t RMAX_OFF = REL_OFF + 2 * BT * 4;        // float [2 stages][4]: max per 32 slots
+constexpr uint32_t DP_OFF = RMAX_OFF + 2 * 4 * 4;          // float [2 halves][BT]: partial D
+constexpr uint32_t QBAR_OFF = DP_OFF + 2 * BT * 4;
+enum {
+  QB_Q = 0, QB_KF0, QB_KE0 = QB_KF0 + 2, QB_SF0 = QB_KE0 + 2, QB_SR0 = QB_SF0 + 2,
+  QB_PF0 = QB_SR0 + 2, QB_DX = QB_PF0 + 2, QB_DONE, QB_END
+};
 constexpr uint32_t QTMEM_OFF = QBAR_OFF + QB_END * 8;
 constexpr uint32_t kSmemDq = QTMEM_OFF + 16;
 static_assert(kSmemDq + 1024 <= 232448, "dq shared memory budget");
+
+// TMEM column of the hi term of k-step kk (16 slots or rows) of a tile whose dS (or
+// P) was written back by 32-wide chunks: hi of chunk c in columns 32c .. 32c + 15,
+// lo 16 columns further.
+__device__ __forceinline__ uint32_t a_col(int kk) { return 32u * (kk >> 1) + 8u * (kk & 1); }
 
 __global__ void __launch_bounds__(kThr, 1)
     bwd_dq_tc_kernel(const __grid_constant__ CUtensorMap q_map,
@@ -104,6 +125,8 @@ __global__ void __launch_bounds__(kThr, 1)
   uint8_t *smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
   const uint32_t sbase = smem_u32(smem);
   float *rel_s = reinterpret_cast<float *>(smem + REL_OFF);
+  float *rmax_s = reinterpret_cast<float *>(smem + RMAX_OFF);
+  float *dpart = reinterpret_cast<float *>(smem + DP_OFF);
   uint64_t *bar = reinterpret_cast<uint64_t *>(smem + QBAR_OFF);
   uint32_t *tmem_s = reinterpret_cast<uint32_t *>(smem + QTMEM_OFF);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -118,11 +141,12 @@ __global__ void __launch_bounds__(kThr, 1)
     mbar_init(&bar[QB_Q], 1);
     for (int s = 0; s < 2; ++s) {
       mbar_init(&bar[QB_KF0 + s], 1);
-      mbar_init(&bar[QB_KE0 + s], 1 + 4);  // MMA commit + the lane warps (slot positions)
+      mbar_init(&bar[QB_KE0 + s], 1 + kLaneWarps);  // MMA commit + the lane warps (positions)
+      mbar_init(&bar[QB_SF0 + s], 1);
+      mbar_init(&bar[QB_SR0 + s], kLaneWarps);
+      mbar_init(&bar[QB_PF0 + s], kLaneWarps);
     }
-    mbar_init(&bar[QB_SF], 1);
-    mbar_init(&bar[QB_SR], 4);
-    mbar_init(&bar[QB_PF], 4);
+    mbar_init(&bar[QB_DX], kLaneWarps * 32);
     mbar_init(&bar[QB_DONE], 1);
     fence_mbar_init();
   }
@@ -151,7 +175,12 @@ __global__ void __launch_bounds__(kThr, 1)
     for (; it < n_it && !aborted; ++it) {
       const int s = it & 1, use = it >> 1, kt = it % n_kt;
       if (use > 0 && !wwait(&bar[QB_KE0 + s], (use - 1) & 1, lim)) { fail(p, aborted); break; }
-      for (int e = lane; e < BT; e += 32) rel_s[s * BT + e] = rel_of(tpg, kt * BT + e, p.N_C, p.P);
+      for (int c = 0; c < BT / 32; ++c) {
+        const float v = rel_of(tpg, kt * BT + 32 * c + lane, p.N_C, p.P);  // integer-valued
+        rel_s[s * BT + 32 * c + lane] = v;
+        const int m = __reduce_max_sync(0xffffffffu, (int)v);
+        if (lane == 0) rmax_s[s * 4 + c] = (float)m;
+      }
       __syncwarp();
       if (lane == 0) {
         mbar_expect_tx(&bar[QB_KF0 + s], 2 * kTile);
@@ -171,37 +200,87 @@ __global__ void __launch_bounds__(kThr, 1)
     // ------------------------------------------------------------------ MMA issuer
     if (lane == 0) {
       const uint32_t q_addr = sbase + Q_OFF, dy_addr = sbase + DY_OFF;
+      auto kv_addr = [&](int st, uint32_t off) { return sbase + off + st * kTile; };
+      auto issue_s = [&](int st, uint32_t col) {  // S = Q K^T
+#pragma unroll
+        for (int ks = 0; ks < HD / 16; ++ks)
+          mma_bf16_ss(tmem + col, kdesc(q_addr, ks), kdesc(kv_addr(st, K_OFF), ks), IDESC_KK, ks > 0);
+      };
+      auto issue_dp = [&](int st, uint32_t col) {  // dP = dY V^T
+#pragma unroll
+        for (int ks = 0; ks < HD / 16; ++ks)
+          mma_bf16_ss(tmem + col, kdesc(dy_addr, ks), kdesc(kv_addr(st, V_OFF), ks), IDESC_KK, ks > 0);
+      };
+      // dQ += dS K over the k-steps of chunk qq of both lane halves (slots 32 qq .. and
+      // 64 + 32 qq ..), dS read from TMEM at column xs (two bf16 per column)
+      auto dq_products = [&](int st, uint32_t xs, int qq, bool first) {
+        const uint32_t k_addr = kv_addr(st, K_OFF);
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          const int kk = 2 * qq + (u & 1) + 4 * (u >> 1);
+          mma_bf16_ts(tmem + 256, tmem + xs + a_col(kk), mdesc(k_addr, kk), IDESC_TM,
+                      (first && u == 0) ? 0u : 1u);
+        }
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          const int kk = 2 * qq + (u & 1) + 4 * (u >> 1);
+          mma_bf16_ts(tmem + 256, tmem + xs + a_col(kk) + 16, mdesc(k_addr, kk), IDESC_TM, 1u);
+        }
+      };
       if (!mbar_wait(&bar[QB_Q], 0, lim)) fail(p, aborted);
-      for (int it = 0; it < n_it && !aborted; ++it) {
-        const int s = it & 1, use = it >> 1;
-        const bool pass2 = it >= n_kt;
-        if (!mbar_wait(&bar[QB_KF0 + s], use & 1, lim)) { fail(p, aborted); break; }
-        // pass 1 holds no MMA behind the lanes' reads of S and dP: wait for them
-        if (it > 0 && it - 1 < n_kt && !mbar_wait(&bar[QB_SR], (it - 1) & 1, lim)) {
+      // Pass 1: S, dP of tile it into columns 256 (it & 1) ..; they were last read by
+      // the lanes in tile it - 2.
+      for (int it = 0; it < n_kt && !aborted; ++it) {
+        const int s = it & 1;
+        if (!mbar_wait(&bar[QB_KF0 + s], (it >> 1) & 1, lim)) { fail(p, aborted); break; }
+        if (it >= 2 && !mbar_wait(&bar[QB_SR0 + s], ((it - 2) >> 1) & 1, lim)) {
           fail(p, aborted);
           break;
         }
         tc_fence_after();
-        const uint32_t k_addr = sbase + K_OFF + s * kTile, v_addr = sbase + V_OFF + s * kTile;
-#pragma unroll
-        for (int ks = 0; ks < HD / 16; ++ks)
-          mma_bf16_ss(tmem, kdesc(q_addr, ks), kdesc(k_addr, ks), IDESC_KK, ks > 0);
-#pragma unroll
-        for (int ks = 0; ks < HD / 16; ++ks)
-          mma_bf16_ss(tmem + 128, kdesc(dy_addr, ks), kdesc(v_addr, ks), IDESC_KK, ks > 0);
-        mma_commit(&bar[QB_SF]);
-        if (pass2) {
-          // dQ += dS K: dS over S in TMEM (two bf16 per column, 8 columns per k-step)
-          if (!mbar_wait(&bar[QB_PF], (it - n_kt) & 1, lim)) { fail(p, aborted); break; }
+        issue_s(s, 256u * s);
+        issue_dp(s, 256u * s + 128);
+        mma_commit(&bar[QB_SF0 + s]);
+        mma_commit(&bar[QB_KE0 + s]);  // K, V of this stage no longer read
+      }
+      // Pass 2 (tile m = it - n_kt): S(m) in columns 0 or 384 (by the parity of m), dP
+      // at 128, dQ at 256.  Once the lanes have written the first chunk of dS(m), its
+      // products and S(m + 1) are issued; once they have read all of dP(m), dP(m + 1)
+      // and then the rest of dS(m)'s products, so the lanes wait only for dP.
+      if (!aborted) {
+        bool ok = true;
+        for (int j = n_kt - 1; ok && j >= 0 && j >= n_kt - 2; --j)
+          ok = mbar_wait(&bar[QB_SR0 + (j & 1)], (j >> 1) & 1, lim);
+        const int s0 = n_kt & 1;
+        if (ok) ok = mbar_wait(&bar[QB_KF0 + s0], (n_kt >> 1) & 1, lim);
+        if (!ok) {
+          fail(p, aborted);
+        } else {
           tc_fence_after();
-#pragma unroll
-          for (int ks = 0; ks < BT / 16; ++ks)
-            mma_bf16_ts(tmem + 256, tmem + ks * 8, mdesc(k_addr, ks), IDESC_TM,
-                        (it > n_kt || ks > 0) ? 1u : 0u);
-#pragma unroll
-          for (int ks = 0; ks < BT / 16; ++ks)
-            mma_bf16_ts(tmem + 256, tmem + 384 + ks * 8, mdesc(k_addr, ks), IDESC_TM, 1u);
+          issue_s(s0, 0);
+          issue_dp(s0, 128);
+          mma_commit(&bar[QB_SF0 + s0]);
         }
+      }
+      for (int m = 0; m < n_kt && !aborted; ++m) {
+        const int it = n_kt + m, s = it & 1;
+        const uint32_t xs = (m & 1) ? 384u : 0u;
+        const bool more = m + 1 < n_kt;
+        if (!mbar_wait(&bar[QB_PF0], m & 1, lim)) { fail(p, aborted); break; }
+        tc_fence_after();
+        dq_products(s, xs, 0, m == 0);
+        if (more) {
+          if (!mbar_wait(&bar[QB_KF0 + (s ^ 1)], ((it + 1) >> 1) & 1, lim)) { fail(p, aborted); break; }
+          tc_fence_after();
+          issue_s(s ^ 1, xs ^ 384u);
+        }
+        if (!mbar_wait(&bar[QB_PF0 + 1], m & 1, lim)) { fail(p, aborted); break; }
+        tc_fence_after();
+        if (more) {
+          issue_dp(s ^ 1, 128);
+          mma_commit(&bar[QB_SF0 + (s ^ 1)]);
+        }
+        dq_products(s, xs, 1, false);
         mma_commit(&bar[QB_KE0 + s]);  // K, V of this stage no longer read
       }
       mma_commit(&bar[QB_DONE]);
@@ -209,68 +288,112 @@ __global__ void __launch_bounds__(kThr, 1)
     }
     __syncwarp();
   } else {
-    // ------------------------------------------------- one thread per row (TMEM lane)
-    const int quarter = warp & 3;
+    // ----------------- one row per TMEM lane; two warps per lane quarter split the slots
+    const int half = (warp - 2) >> 2, quarter = warp & 3;
     const int r = 32 * quarter + lane;
     const uint32_t lb = (uint32_t)(32 * quarter) << 16;
     const bool row_ok = i0 + r < p.S;
     float lse2 = row_ok ? p.lse[(size_t)bhq * p.S + i0 + r] * 1.4426950408889634f : INFINITY;
     if (!(lse2 > -INFINITY && lse2 < INFINITY)) lse2 = INFINITY;  // sees nothing / past the chunk: p = 0
-    const float ri = (float)(i0 + r), c2 = p.c2;
+    const float ri = (float)(i0 + r), rowmin = (float)(i0 + 32 * quarter);
+    const float2 c22 = make_float2(p.c2, p.c2), nl22 = make_float2(-lse2, -lse2);
+    float2 Dacc2 = make_float2(0.f, 0.f);
     float Dacc = 0.f;
     for (int it = 0; it < n_it && !aborted; ++it) {
       const int s = it & 1, use = it >> 1;
       const bool pass2 = it >= n_kt;
-      if (!wwait(&bar[QB_SF], it & 1, lim)) { fail(p, aborted); break; }
+      if (!wwait(&bar[QB_SF0 + s], use & 1, lim)) { fail(p, aborted); break; }
       if (!wwait(&bar[QB_KF0 + s], use & 1, lim)) { fail(p, aborted); break; }
       tc_fence_after();
-      const float *rel = rel_s + s * BT;
-#pragma unroll 1
-      for (int h = 0; h < 2; ++h) {
+      const float *rel = rel_s + s * BT + 64 * half;  // this half's 64 slots
+      // a 32-slot chunk whose latest position is at or before the warp's first row is
+      // seen by every row of the warp: no mask
+      const bool vis0 = rmax_s[s * 4 + 2 * half] <= rowmin;
+      const bool vis1 = rmax_s[s * 4 + 2 * half + 1] <= rowmin;
+      if (!pass2) {
+        // D_i partial over this half's slots
+        const uint32_t cb = 256u * (uint32_t)s + 64u * half;
         uint32_t sv[64], dp[64];
-        tmem_ld32(tmem + lb + 64 * h, *reinterpret_cast<uint32_t(*)[32]>(sv));
-        tmem_ld32(tmem + lb + 64 * h + 32, *reinterpret_cast<uint32_t(*)[32]>(sv + 32));
-        tmem_ld32(tmem + lb + 128 + 64 * h, *reinterpret_cast<uint32_t(*)[32]>(dp));
-        tmem_ld32(tmem + lb + 128 + 64 * h + 32, *reinterpret_cast<uint32_t(*)[32]>(dp + 32));
+        tmem_ld32(tmem + lb + cb, *reinterpret_cast<uint32_t(*)[32]>(sv));
+        tmem_ld32(tmem + lb + cb + 32, *reinterpret_cast<uint32_t(*)[32]>(sv + 32));
+        tmem_ld32(tmem + lb + cb + 128, *reinterpret_cast<uint32_t(*)[32]>(dp));
+        tmem_ld32(tmem + lb + cb + 160, *reinterpret_cast<uint32_t(*)[32]>(dp + 32));
         tmem_wait_ld();
-        if (!pass2) {
+        if (vis0 && vis1) {
 #pragma unroll
-          for (int e = 0; e < 64; ++e) {
-            const float pe = rel[64 * h + e] <= ri ? ex2(__uint_as_float(sv[e]) * c2 - lse2) : 0.f;
-            Dacc = fmaf(pe, __uint_as_float(dp[e]), Dacc);
-          }
+          for (int e = 0; e < 64; e += 2)
+            Dacc2 = fma2(ex2_2(fma2(u2f2(sv[e], sv[e + 1]), c22, nl22)), u2f2(dp[e], dp[e + 1]), Dacc2);
         } else {
-          uint32_t hi[32], lo[32];
 #pragma unroll
           for (int e = 0; e < 64; e += 2) {
-            const float p0 = rel[64 * h + e] <= ri ? ex2(__uint_as_float(sv[e]) * c2 - lse2) : 0.f;
-            const float p1 =
-                rel[64 * h + e + 1] <= ri ? ex2(__uint_as_float(sv[e + 1]) * c2 - lse2) : 0.f;
-            split2(p0 * (__uint_as_float(dp[e]) - Dacc), p1 * (__uint_as_float(dp[e + 1]) - Dacc),
-                   hi[e >> 1], lo[e >> 1]);
+            float2 pr = ex2_2(fma2(u2f2(sv[e], sv[e + 1]), c22, nl22));
+            pr.x = rel[e] <= ri ? pr.x : 0.f;
+            pr.y = rel[e + 1] <= ri ? pr.y : 0.f;
+            Dacc2 = fma2(pr, u2f2(dp[e], dp[e + 1]), Dacc2);
           }
-          // dS of slots 64h .. 64h + 63: hi into columns 32h .. 32h + 31 (S there is
-          // read), lo into 384 + 32h ..
-          tmem_st32(tmem + lb + 32 * h, hi);
-          tmem_st32(tmem + lb + 384 + 32 * h, lo);
+        }
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) {
+          mbar_arrive(&bar[QB_SR0 + s]);
+          mbar_arrive(&bar[QB_KE0 + s]);  // slot positions no longer read
+        }
+        if (it == n_kt - 1) {
+          // D_i = the two halves' partial sums, added in a fixed order
+          dpart[half * BT + r] = Dacc2.x + Dacc2.y;
+          mbar_arrive(&bar[QB_DX]);
+          if (!wwait(&bar[QB_DX], 0, lim)) { fail(p, aborted); break; }
+          Dacc = dpart[r] + dpart[BT + r];
+          if (half == 0 && row_ok) p.D[(size_t)bhq * p.S + i0 + r] = Dacc;
+        }
+      } else {
+        // dS by 32-slot chunks, written back over the chunk's S columns (S(m) at column
+        // 0 or 384 by the parity of m = it - n_kt): hi term in the first 16, lo term in
+        // the next 16
+        const uint32_t xs = ((it - n_kt) & 1) ? 384u : 0u;
+        const float2 nD2 = make_float2(-Dacc, -Dacc);
+#pragma unroll 1
+        for (int qq = 0; qq < 2; ++qq) {
+          const uint32_t c0 = 64u * half + 32u * qq;
+          uint32_t sv[32], dp[32], hi[16], lo[16];
+          tmem_ld32(tmem + lb + xs + c0, sv);
+          tmem_ld32(tmem + lb + 128 + c0, dp);
+          tmem_wait_ld();
+          if (qq == 0 ? vis0 : vis1) {
+#pragma unroll
+            for (int e = 0; e < 32; e += 2) {
+              const float2 pr = ex2_2(fma2(u2f2(sv[e], sv[e + 1]), c22, nl22));
+              split2(mul2(pr, add2(u2f2(dp[e], dp[e + 1]), nD2)), hi[e >> 1], lo[e >> 1]);
+            }
+          } else {
+            const float *rq = rel + 32 * qq;
+#pragma unroll
+            for (int e = 0; e < 32; e += 2) {
+              float2 pr = ex2_2(fma2(u2f2(sv[e], sv[e + 1]), c22, nl22));
+              pr.x = rq[e] <= ri ? pr.x : 0.f;
+              pr.y = rq[e + 1] <= ri ? pr.y : 0.f;
+              split2(mul2(pr, add2(u2f2(dp[e], dp[e + 1]), nD2)), hi[e >> 1], lo[e >> 1]);
+            }
+          }
+          tmem_st16(tmem + lb + xs + c0, hi);
+          tmem_st16(tmem + lb + xs + c0 + 16, lo);
+          tmem_wait_st();
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) {
+            mbar_arrive(&bar[QB_PF0 + qq]);
+            if (qq == 1) mbar_arrive(&bar[QB_KE0 + s]);  // slot positions no longer read
+          }
         }
       }
-      if (pass2) tmem_wait_st();
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) {
-        mbar_arrive(&bar[pass2 ? QB_PF : QB_SR]);
-        mbar_arrive(&bar[QB_KE0 + s]);  // slot positions no longer read
-      }
-      if (it == n_kt - 1 && row_ok) p.D[(size_t)bhq * p.S + i0 + r] = Dacc;
     }
     if (!aborted && wwait(&bar[QB_DONE], 0, lim)) {
       tc_fence_after();
-      float *dst = p.dq + ((size_t)bhq * p.S + i0 + r) * HD;
+      float *dst = p.dq + ((size_t)bhq * p.S + i0 + r) * HD + 64 * half;
 #pragma unroll 1
-      for (int cq = 0; cq < 4; ++cq) {
+      for (int cq = 0; cq < 2; ++cq) {
         uint32_t o[32];
-        tmem_ld32(tmem + lb + 256 + 32 * cq, o);
+        tmem_ld32(tmem + lb + 256 + 64 * half + 32 * cq, o);
         tmem_wait_ld();
         if (row_ok) {
 #pragma unroll
@@ -294,9 +417,9 @@ __global__ void __launch_bounds__(kThr, 1)
 
 // ---- dk, dv --------------------------------------------------------------------------
 constexpr uint32_t KK_OFF = 0, KV_OFF = kTile, KQ_OFF = 2 * kTile, KDY_OFF = 4 * kTile;
-constexpr uint32_t ROWS_OFF = 6 * kTile;                     // float [2 stages][2][BT]: lse2, D
+constexpr uint32_t ROWS_OFF = 6 * kTile;                     // float [2 stages][2][BT]: -lse2, -D
 constexpr uint32_t KBAR_OFF = ROWS_OFF + 2 * 2 * BT * 4;
-enum { KB_KV = 0, KB_QF0, KB_QE0 = KB_QF0 + 2, KB_SF = KB_QE0 + 2, KB_PF, KB_DONE, KB_END };
+enum { KB_KV = 0, KB_QF0, KB_QE0 = KB_QF0 + 2, KB_SF = KB_QE0 + 2, KB_PF0, KB_DONE = KB_PF0 + 2, KB_END };
 constexpr uint32_t KTMEM_OFF = KBAR_OFF + KB_END * 8;
 constexpr uint32_t kSmemKv = KTMEM_OFF + 16;
 static_assert(kSmemKv + 1024 <= 232448, "dk/dv shared memory budget");
@@ -321,10 +444,10 @@ __global__ void __launch_bounds__(kThr, 1)
     mbar_init(&bar[KB_KV], 1);
     for (int s = 0; s < 2; ++s) {
       mbar_init(&bar[KB_QF0 + s], 1);
-      mbar_init(&bar[KB_QE0 + s], 1 + 4);  // MMA commit + the lane warps (lse2, D)
+      mbar_init(&bar[KB_QE0 + s], 1 + kLaneWarps);  // MMA commit + the lane warps (lse2, D)
+      mbar_init(&bar[KB_PF0 + s], kLaneWarps);
     }
     mbar_init(&bar[KB_SF], 1);
-    mbar_init(&bar[KB_PF], 4);
     mbar_init(&bar[KB_DONE], 1);
     fence_mbar_init();
   }
@@ -358,8 +481,8 @@ __global__ void __launch_bounds__(kThr, 1)
         const bool ok = i0 + r < p.S;
         float l2 = ok ? p.lse[(size_t)bhq * p.S + i0 + r] * 1.4426950408889634f : INFINITY;
         if (!(l2 > -INFINITY && l2 < INFINITY)) l2 = INFINITY;  // sees nothing / past the chunk: p = 0
-        rows_s[(s * 2 + 0) * BT + r] = l2;
-        rows_s[(s * 2 + 1) * BT + r] = ok ? p.D[(size_t)bhq * p.S + i0 + r] : 0.f;
+        rows_s[(s * 2 + 0) * BT + r] = -l2;
+        rows_s[(s * 2 + 1) * BT + r] = ok ? -p.D[(size_t)bhq * p.S + i0 + r] : 0.f;
       }
       __syncwarp();
       if (lane == 0) {
@@ -395,24 +518,36 @@ __global__ void __launch_bounds__(kThr, 1)
         for (int ks = 0; ks < HD / 16; ++ks)
           mma_bf16_ss(tmem + 128, kdesc(v_addr, ks), kdesc(dy_addr, ks), IDESC_KK, ks > 0);
         mma_commit(&bar[KB_SF]);
-        if (!mbar_wait(&bar[KB_PF], it & 1, lim)) { fail(p, aborted); break; }
-        tc_fence_after();
-        // dV += P^T dY, dK += dS^T Q (A from TMEM: hi terms at 0 / 128, lo terms at
-        // 64 / 192; B: the row tiles as MN-major operands)
+        // dV += P^T dY, dK += dS^T Q (A from TMEM: P^T terms in columns 0 .., dS^T terms
+        // in 128 ..; B: the row tiles as MN-major operands), the k-steps of each lane
+        // half's first 32 rows once PF0 completes, the rest after PF1
+        for (int qq = 0; qq < 2 && !aborted; ++qq) {
+          if (!mbar_wait(&bar[KB_PF0 + qq], it & 1, lim)) { fail(p, aborted); break; }
+          tc_fence_after();
 #pragma unroll
-        for (int ks = 0; ks < BT / 16; ++ks)
-          mma_bf16_ts(tmem + 256, tmem + ks * 8, mdesc(dy_addr, ks), IDESC_TM,
-                      (it > 0 || ks > 0) ? 1u : 0u);
+          for (int u = 0; u < 4; ++u) {
+            const int kk = 2 * qq + (u & 1) + 4 * (u >> 1);
+            mma_bf16_ts(tmem + 256, tmem + a_col(kk), mdesc(dy_addr, kk), IDESC_TM,
+                        (it > 0 || qq > 0 || u > 0) ? 1u : 0u);
+          }
 #pragma unroll
-        for (int ks = 0; ks < BT / 16; ++ks)
-          mma_bf16_ts(tmem + 256, tmem + 64 + ks * 8, mdesc(dy_addr, ks), IDESC_TM, 1u);
+          for (int u = 0; u < 4; ++u) {
+            const int kk = 2 * qq + (u & 1) + 4 * (u >> 1);
+            mma_bf16_ts(tmem + 256, tmem + a_col(kk) + 16, mdesc(dy_addr, kk), IDESC_TM, 1u);
+          }
 #pragma unroll
-        for (int ks = 0; ks < BT / 16; ++ks)
-          mma_bf16_ts(tmem + 384, tmem + 128 + ks * 8, mdesc(q_addr, ks), IDESC_TM,
-                      (it > 0 || ks > 0) ? 1u : 0u);
+          for (int u = 0; u < 4; ++u) {
+            const int kk = 2 * qq + (u & 1) + 4 * (u >> 1);
+            mma_bf16_ts(tmem + 384, tmem + 128 + a_col(kk), mdesc(q_addr, kk), IDESC_TM,
+                        (it > 0 || qq > 0 || u > 0) ? 1u : 0u);
+          }
 #pragma unroll
-        for (int ks = 0; ks < BT / 16; ++ks)
-          mma_bf16_ts(tmem + 384, tmem + 192 + ks * 8, mdesc(q_addr, ks), IDESC_TM, 1u);
+          for (int u = 0; u < 4; ++u) {
+            const int kk = 2 * qq + (u & 1) + 4 * (u >> 1);
+            mma_bf16_ts(tmem + 384, tmem + 128 + a_col(kk) + 16, mdesc(q_addr, kk), IDESC_TM, 1u);
+          }
+        }
+        if (aborted) break;
         mma_commit(&bar[KB_QE0 + s]);  // Q, dY of this stage no longer read
       }
       mma_commit(&bar[KB_DONE]);
@@ -420,13 +555,13 @@ __global__ void __launch_bounds__(kThr, 1)
     }
     __syncwarp();
   } else {
-    // ------------------------------------------------ one thread per slot (TMEM lane)
-    const int quarter = warp & 3;
+    // ---------------- one slot per TMEM lane; two warps per lane quarter split the rows
+    const int half = (warp - 2) >> 2, quarter = warp & 3;
     const int jl = 32 * quarter + lane;
     const int j = kt * BT + jl;
     const uint32_t lb = (uint32_t)(32 * quarter) << 16;
     const float rel = rel_of(p.token_pos + (size_t)bg * p.N_C, j, p.N_C, p.P);
-    const float c2 = p.c2;
+    const float2 c22 = make_float2(p.c2, p.c2);
     for (int it = 0; it < n_rt && !aborted; ++it) {
       const int s = it & 1, use = it >> 1;
       const int t = it % p.tiles, i0 = t * BT;
@@ -434,63 +569,67 @@ __global__ void __launch_bounds__(kThr, 1)
       if (!wwait(&bar[KB_QF0 + s], use & 1, lim)) { fail(p, aborted); break; }
       tc_fence_after();
       // row r of the tile sees this slot iff i0 + r >= rel; rows past the chunk have
-      // lse2 = +inf
+      // -lse2 = -inf
       const float rmin = rel - (float)i0;
-      const float *l2 = rows_s + (s * 2 + 0) * BT, *Dr = rows_s + (s * 2 + 1) * BT;
-      // by quarters of 32 rows (S^T columns 32q .. 32q + 31): hi terms of P^T into
-      // columns 16q .., of dS^T into 128 + 16q .. (all read already); lo terms into
-      // 64 + 16q .. and 192 + 16q .., written once quarter 2 (for q = 0, 1) or 3 (for
-      // q = 2, 3) has read those columns
-      uint32_t plo[4][16], dlo[4][16];
-#pragma unroll
-      for (int q = 0; q < 4; ++q) {
-        uint32_t sv[32], dp[32], phi[16], dhi[16];
-        tmem_ld32(tmem + lb + 32 * q, sv);
-        tmem_ld32(tmem + lb + 128 + 32 * q, dp);
+      const float *nl2 = rows_s + (s * 2 + 0) * BT, *nD = rows_s + (s * 2 + 1) * BT;
+      // by chunks of 32 rows (S^T columns r0 .. r0 + 31), written back over the
+      // chunk's own columns: P^T hi, lo in r0 .., r0 + 16 ..; dS^T hi, lo 128 further
+#pragma unroll 1
+      for (int qq = 0; qq < 2; ++qq) {
+        const int r0 = 64 * half + 32 * qq;
+        uint32_t sv[32], dp[32], phi[16], plo[16], dhi[16], dlo[16];
+        tmem_ld32(tmem + lb + r0, sv);
+        tmem_ld32(tmem + lb + 128 + r0, dp);
         tmem_wait_ld();
+        if (__all_sync(0xffffffffu, rmin <= (float)r0)) {  // every row sees every slot of the warp
 #pragma unroll
-        for (int e = 0; e < 32; e += 2) {
-          const int r = 32 * q + e;
-          const float p0 = (float)r >= rmin ? ex2(__uint_as_float(sv[e]) * c2 - l2[r]) : 0.f;
-          const float p1 = (float)(r + 1) >= rmin ? ex2(__uint_as_float(sv[e + 1]) * c2 - l2[r + 1]) : 0.f;
-          split2(p0, p1, phi[e >> 1], plo[q][e >> 1]);
-          split2(p0 * (__uint_as_float(dp[e]) - Dr[r]), p1 * (__uint_as_float(dp[e + 1]) - Dr[r + 1]),
-                 dhi[e >> 1], dlo[q][e >> 1]);
-        }
-        tmem_st16(tmem + lb + 16 * q, phi);
-        tmem_st16(tmem + lb + 128 + 16 * q, dhi);
-        if (q >= 2) {
+          for (int e = 0; e < 32; e += 2) {
+            const float2 pr =
+                ex2_2(fma2(u2f2(sv[e], sv[e + 1]), c22, *reinterpret_cast<const float2 *>(nl2 + r0 + e)));
+            split2(pr, phi[e >> 1], plo[e >> 1]);
+            split2(mul2(pr, add2(u2f2(dp[e], dp[e + 1]), *reinterpret_cast<const float2 *>(nD + r0 + e))),
+                   dhi[e >> 1], dlo[e >> 1]);
+          }
+        } else {
 #pragma unroll
-          for (int u = 2 * (q - 2); u < 2 * (q - 2) + 2; ++u) {
-            tmem_st16(tmem + lb + 64 + 16 * u, plo[u]);
-            tmem_st16(tmem + lb + 192 + 16 * u, dlo[u]);
+          for (int e = 0; e < 32; e += 2) {
+            const int r = r0 + e;
+            float2 pr = ex2_2(fma2(u2f2(sv[e], sv[e + 1]), c22, *reinterpret_cast<const float2 *>(nl2 + r)));
+            pr.x = (float)r >= rmin ? pr.x : 0.f;
+            pr.y = (float)(r + 1) >= rmin ? pr.y : 0.f;
+            split2(pr, phi[e >> 1], plo[e >> 1]);
+            split2(mul2(pr, add2(u2f2(dp[e], dp[e + 1]), *reinterpret_cast<const float2 *>(nD + r))),
+                   dhi[e >> 1], dlo[e >> 1]);
           }
         }
-      }
-      tmem_wait_st();
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) {
-        mbar_arrive(&bar[KB_PF]);
-        mbar_arrive(&bar[KB_QE0 + s]);  // lse2, D of this stage no longer read
+        tmem_st16(tmem + lb + r0, phi);
+        tmem_st16(tmem + lb + r0 + 16, plo);
+        tmem_st16(tmem + lb + 128 + r0, dhi);
+        tmem_st16(tmem + lb + 128 + r0 + 16, dlo);
+        tmem_wait_st();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) {
+          mbar_arrive(&bar[KB_PF0 + qq]);
+          if (qq == 1) mbar_arrive(&bar[KB_QE0 + s]);  // -lse2, -D of this stage no longer read
+        }
       }
     }
     if (!aborted && wwait(&bar[KB_DONE], 0, lim)) {
       tc_fence_after();
+      // half 0 writes dV, half 1 dK
       const bool ok = j < p.N_C;
-      float *dvr = p.dv + ((size_t)bg * p.N_C + j) * HD;
-      float *dkr = p.dk + ((size_t)bg * p.N_C + j) * HD;
+      float *dst = (half == 0 ? p.dv : p.dk) + ((size_t)bg * p.N_C + j) * HD;
+      const float f = half == 0 ? 1.f : p.rsd;
 #pragma unroll 1
-      for (int cq = 0; cq < 8; ++cq) {
+      for (int cq = 0; cq < 4; ++cq) {
         uint32_t o[32];
-        tmem_ld32(tmem + lb + 256 + 32 * cq, o);  // dV (cq < 4), then dK
+        tmem_ld32(tmem + lb + 256 + 128 * half + 32 * cq, o);
         tmem_wait_ld();
         if (ok) {
-          float *dst = cq < 4 ? dvr + 32 * cq : dkr + 32 * (cq - 4);
-          const float f = cq < 4 ? 1.f : p.rsd;
 #pragma unroll
           for (int e = 0; e < 8; ++e)
-            reinterpret_cast<float4 *>(dst)[e] =
+            reinterpret_cast<float4 *>(dst + 32 * cq)[e] =
                 make_float4(__uint_as_float(o[4 * e]) * f, __uint_as_float(o[4 * e + 1]) * f,
                             __uint_as_float(o[4 * e + 2]) * f, __uint_as_float(o[4 * e + 3]) * f);
         }

@@ -27,6 +27,9 @@ def wl_(name, **kw):
 CASES = [
     wl_("bwd_f32_d64", d=64, q_dtype="f32", kv_dtype="f32"),
     wl_("bwd_bf16_gqa_b2", B=2),
+    # tensor-core path: three row tiles and six slot tiles, both ragged; one slot tile
+    wl_("bwd_bf16_tiles", Hq=8, Hk=2, capacity=700, chunk=300, seq_len=1500),
+    wl_("bwd_bf16_one_tile", capacity=100, chunk=60, seq_len=300),
     wl_("bwd_i8", kv_dtype="i8"),
     wl_("bwd_i4_mha", Hq=2, Hk=2, kv_dtype="i4", capacity=260, chunk=90, seq_len=700),
 ]
