@@ -80,9 +80,9 @@ static void layout(const h2okv_cache_desc &d, const TcPlan &tc, WorkspaceLayout 
   off = align256(off + G * 2048 * 4);
   ws->ev_arrive = off;
   off = align256(off + G * 4);
-  ws->ev_zero_end = off;
   ws->ev_slots = off;
   off = align256(off + G * S * 4);
+  ws->ev_zero_end = off;
   ws->part_ml = ws->part_w = ws->part_o = ws->nlse = off;
   if (tc.enabled) {
     const size_t seg_rows = (size_t)tc.split_ctas * tc.max_seg * 2 * 128;

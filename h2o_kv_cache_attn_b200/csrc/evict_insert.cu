@@ -543,10 +543,7 @@ __device__ __forceinline__ RowSet<NT> row_set(const EvParams<NT> &p) {
 template <int NT>
 __device__ __forceinline__ int slot_of(const EvParams<NT> &p, const RowSet<NT> &rs, int k) {
   if (p.mode == 1) return p.n_filled + k;
-  if (p.mode == 2) {
-    const int j = __ldcg(rs.slist + k);
-    return (j >= 0 && j < p.N_C) ? j : -1;  // a list left incomplete by a timed-out choose
-  }
+  if (p.mode == 2) return __ldcg(rs.slist + k);  // in range: zeroed on create, written by choose
   const int j = __ldg(rs.T->slots_in + rs.bh * p.S + k);
   return (j >= 0 && j < p.N_C) ? j : -1;
 }

@@ -25,7 +25,8 @@ struct WorkspaceLayout {
   size_t status;       // int32: device status word (0 = ok, else an H2OKV_ERR_* code)
   size_t ev_hist;      // uint32 [B*H_k][2048]: top-bit key histograms of the eviction (zero between calls)
   size_t ev_arrive;    // uint32 [B*H_k]: arrival counters of the eviction (zero between calls)
-  size_t ev_slots;     // int32 [B*H_k][max_chunk]: chosen slots in slot order
+  size_t ev_slots;     // int32 [B*H_k][max_chunk]: chosen slots in slot order (zeroed on create
+                       //   and reset, so a list a timed-out choose left unfinished stays in range)
   size_t ev_zero_end;  // [ev_hist, ev_zero_end) is zeroed on create and reset
   size_t total;
 };
