@@ -260,8 +260,12 @@ H2OKV_API int kv_cache_restore(h2okv_cache *cache, const int32_t *slots, int32_t
  * with respect to the stored (dequantized) keys and values; the outputs are
  * overwritten.  q, dy: [B, H_q, S, d] in q_dtype; lse: [B, H_q, S] float32, the
  * natural-log row log-sum-exp written by attn_chunk_with_scoresum for the same
- * chunk and cache state.  CUDA cores; the workspace holds D.  Same S / P
- * rules as attn_chunk_with_scoresum. */
+ * chunk and cache state.  The workspace holds D.  Same S / P rules as
+ * attn_chunk_with_scoresum.  A bf16 cache with d_h = 128 and bf16 queries runs
+ * on the tensor cores (three kernels on `stream`, the probabilities and dS
+ * entering the second products as two bf16 terms each, hi + lo); every other
+ * combination on CUDA cores.  Every output element is summed in a fixed order
+ * (no atomics), so repeated calls give identical results. */
 H2OKV_API int attn_chunk_backward(h2okv_cache *cache, const void *q, const void *dy,
                                   const float *lse, int32_t S, int64_t P, float *dq_out,
                                   float *dk_out, float *dv_out, void *stream);
