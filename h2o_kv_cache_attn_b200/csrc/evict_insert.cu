@@ -47,7 +47,8 @@ constexpr int kSmemKeysMax = 32768;  // largest N_C whose keys the last CTA keep
 constexpr int kRowThreads = 256;     // threads of a row CTA
 constexpr int kRowWarps = kRowThreads / 32;
 constexpr int kCopyUnroll = 8;   // 16-byte pieces per thread in flight in the row copy
-constexpr int kQuantUnroll = 4;  // rows per lane segment in flight in the row quantizer
+constexpr int kQuantUnroll = 2;  // rows per lane segment in flight in the row quantizer
+constexpr int kQuantChunks = 4;  // 8-element chunks of a row per lane (up to)
 
 // ---- quantizer arithmetic ------------------------------------------------------------
 // code = clamp(rint(x / s), -qmax, qmax) with x / s the correctly rounded float32
@@ -63,6 +64,19 @@ __device__ __forceinline__ int quant_code(float x, float s, float y, float qmax)
   float q = __fmaf_rn(r, y, q0);
   q = fminf(fmaxf(q, -qmax), qmax);
   return __float_as_int(__fadd_rn(q, 12582912.f)) - 0x4B400000;
+}
+
+// The same for two elements with packed float32 arithmetic (each lane of an f32x2
+// operation is the IEEE float32 operation above); returns the bits of q + 1.5 * 2^23,
+// whose low byte (low nibble) is the int8 (int4) code in two's complement.
+__device__ __forceinline__ uint2 quant_bits2(float2 x, float s, float y, float qmax) {
+  const float2 q0 = mul2(x, make_float2(y, y));
+  const float2 r = fma2(q0, make_float2(-s, -s), x);
+  float2 q = fma2(r, make_float2(y, y), q0);
+  q.x = fminf(fmaxf(q.x, -qmax), qmax);
+  q.y = fminf(fmaxf(q.y, -qmax), qmax);
+  const float2 t = add2(q, make_float2(12582912.f, 12582912.f));
+  return make_uint2(__float_as_uint(t.x), __float_as_uint(t.y));
 }
 
 // Unsigned key with the order of the float: -0 and +0 map to the same key;
@@ -618,18 +632,28 @@ __device__ __forceinline__ void copy_rows(const EvParams<NT> &p) {
   }
 }
 
-// int8 / int4 caches: one row per segment of L lanes (L = the smallest power of two
-// >= d / 8); lane i of a segment holds elements 8i .. 8i + 7 of the row.  Per row, the
-// same arithmetic as the per-row quantizer: absmax, IEEE division by qmax, clamp to the
-// fp16 range, round to fp16, then the code of quant_code.
+// int8 / int4 caches: one row per segment of L lanes (L = the smallest power of two >=
+// d / 32); lane i of a segment holds the 8-element chunks i, i + L, ... (up to four) of
+// the row, so the per-row work (absmax reduction, IEEE division by qmax, fp16 scale,
+// correctly rounded reciprocal, addressing, the slot's bookkeeping) is shared by up to
+// 32 elements per lane.  Per row, the same arithmetic as the per-row quantizer:
+// absmax, IEEE division by qmax, clamp to the fp16 range, round to fp16, then the code
+// of quant_code (in pairs).
+__host__ __device__ __forceinline__ int quant_lanes(int d) {
+  const int g8 = d / 8;
+  const int need = (g8 + kQuantChunks - 1) / kQuantChunks;
+  int L = 1;
+  while (L < need) L <<= 1;
+  return L;
+}
+
 template <int NT, int KV, bool DELTA>
 __device__ __forceinline__ void quantize_rows(const EvParams<NT> &p) {
   constexpr int qmax = KV == H2OKV_I8 ? 127 : 7;
   const RowSet<NT> rs = row_set(p);
   const EvTarget &T = *rs.T;
   const int G8 = p.d / 8;
-  int L = 1;
-  while (L < G8) L <<= 1;
+  const int L = quant_lanes(p.d);
   const int lane = threadIdx.x & 31;
   const int seg = lane / L, li = lane % L, segs = 32 / L;
   const int items = p.S * 2;  // (chunk row k, t) as 2k + t: t = 0 key row, 1 value row
@@ -637,16 +661,20 @@ __device__ __forceinline__ void quantize_rows(const EvParams<NT> &p) {
   const int w0 = blockIdx.x * kRowWarps + (threadIdx.x >> 5);
   const uint8_t *src_k = T.k_new + rs.bh * p.S * (size_t)p.in_row_bytes;
   const uint8_t *src_v = T.v_new + rs.bh * p.S * (size_t)p.in_row_bytes;
-  uint4 xr[kQuantUnroll];
+  uint4 xr[kQuantUnroll][kQuantChunks];
   auto item_of = [&](int base, int u) { return ((base + u * W) * segs) + seg; };
   auto load = [&](int base) {
 #pragma unroll
     for (int u = 0; u < kQuantUnroll; ++u) {
       const int it = item_of(base, u);
-      xr[u] = make_uint4(0u, 0u, 0u, 0u);
-      if (it < items && li < G8)
-        xr[u] = __ldcs(reinterpret_cast<const uint4 *>(((it & 1) ? src_v : src_k) +
-                                                        (size_t)(it >> 1) * p.in_row_bytes) + li);
+      const uint4 *src = reinterpret_cast<const uint4 *>(((it & 1) ? src_v : src_k) +
+                                                         (size_t)(it >> 1) * p.in_row_bytes);
+#pragma unroll
+      for (int c = 0; c < kQuantChunks; ++c) {
+        const int ch = li + c * L;
+        xr[u][c] = make_uint4(0u, 0u, 0u, 0u);
+        if (it < items && ch < G8) xr[u][c] = __ldcs(src + ch);
+      }
     }
   };
   load(w0);
@@ -657,20 +685,20 @@ __device__ __forceinline__ void quantize_rows(const EvParams<NT> &p) {
 #pragma unroll
     for (int u = 0; u < kQuantUnroll; ++u) {
       const int it = item_of(base, u);
-      slot[u] = (it < items && li < G8) ? slot_of(p, rs, it >> 1) : -1;
+      slot[u] = it < items ? slot_of(p, rs, it >> 1) : -1;
     }
 #pragma unroll
     for (int u = 0; u < kQuantUnroll; ++u) {
       const int it = item_of(base, u);
-      float v[8];
-      const __nv_bfloat162 *h2 = reinterpret_cast<const __nv_bfloat162 *>(&xr[u]);
-      float amax = 0.f;
+      float amax = 0.f;  // the zero-filled chunks past the row do not change it
 #pragma unroll
-      for (int q = 0; q < 4; ++q) {
-        const float2 f = __bfloat1622float2(h2[q]);
-        v[2 * q] = f.x;
-        v[2 * q + 1] = f.y;
-        amax = fmaxf(amax, fmaxf(fabsf(f.x), fabsf(f.y)));
+      for (int c = 0; c < kQuantChunks; ++c) {
+        const __nv_bfloat162 *h2 = reinterpret_cast<const __nv_bfloat162 *>(&xr[u][c]);
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          const float2 f = __bfloat1622float2(h2[q]);
+          amax = fmaxf(amax, fmaxf(fabsf(f.x), fabsf(f.y)));
+        }
       }
       for (int o = L >> 1; o > 0; o >>= 1)
         amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
@@ -679,10 +707,8 @@ __device__ __forceinline__ void quantize_rows(const EvParams<NT> &p) {
       const __half hs = __float2half_rn(rq);
       const float s = __half2float(hs);
       const float y = __frcp_rn(s);
-      int qc[8];
-#pragma unroll
-      for (int q = 0; q < 8; ++q) qc[q] = s > 0.f ? quant_code(v[q], s, y, (float)qmax) : 0;
-      if (it >= items || li >= G8) continue;
+      const bool nz = s > 0.f;  // scale 0: every code 0
+      if (it >= items) continue;
       const int t = it & 1, k = it >> 1;
       const int j = slot[u];
       if (p.mode >= 2 && t == 0 && li == 0) row_claim(p, rs, k, j);
@@ -693,26 +719,41 @@ __device__ __forceinline__ void quantize_rows(const EvParams<NT> &p) {
       if (DELTA && T.dk) {
         uint8_t *dcodes = (t ? T.dv : T.dk) + crow * (size_t)p.row_bytes;
         if (li == 0) (t ? T.dvs : T.dks)[crow] = *sdst;
-        if (KV == H2OKV_I8)
-          reinterpret_cast<uint2 *>(dcodes)[li] = __ldcg(reinterpret_cast<const uint2 *>(codes) + li);
-        else
-          reinterpret_cast<uint32_t *>(dcodes)[li] =
-              __ldcg(reinterpret_cast<const unsigned int *>(codes) + li);
+#pragma unroll
+        for (int c = 0; c < kQuantChunks; ++c) {
+          const int ch = li + c * L;
+          if (ch >= G8) break;
+          if (KV == H2OKV_I8)
+            reinterpret_cast<uint2 *>(dcodes)[ch] = __ldcg(reinterpret_cast<const uint2 *>(codes) + ch);
+          else
+            reinterpret_cast<uint32_t *>(dcodes)[ch] =
+                __ldcg(reinterpret_cast<const unsigned int *>(codes) + ch);
+        }
       }
       if (li == 0) *sdst = hs;
-      if (KV == H2OKV_I8) {
-        uint32_t lo = 0u, hi = 0u;
 #pragma unroll
-        for (int q = 0; q < 4; ++q) {
-          lo |= ((uint32_t)(qc[q] & 0xFF)) << (8 * q);
-          hi |= ((uint32_t)(qc[q + 4] & 0xFF)) << (8 * q);
+      for (int c = 0; c < kQuantChunks; ++c) {
+        const int ch = li + c * L;
+        if (ch >= G8) break;
+        const __nv_bfloat162 *h2 = reinterpret_cast<const __nv_bfloat162 *>(&xr[u][c]);
+        uint2 bits[4];
+#pragma unroll
+        for (int q = 0; q < 4; ++q) bits[q] = quant_bits2(__bfloat1622float2(h2[q]), s, y, (float)qmax);
+        if (KV == H2OKV_I8) {
+          uint32_t lo = 0u, hi = 0u;  // code bytes: the low byte of each rounded value
+#pragma unroll
+          for (int q = 0; q < 2; ++q) {
+            lo |= ((bits[q].x & 0xFFu) | ((bits[q].y & 0xFFu) << 8)) << (16 * q);
+            hi |= ((bits[q + 2].x & 0xFFu) | ((bits[q + 2].y & 0xFFu) << 8)) << (16 * q);
+          }
+          __stcg(reinterpret_cast<uint2 *>(codes) + ch, nz ? make_uint2(lo, hi) : make_uint2(0u, 0u));
+        } else {
+          uint32_t w = 0u;  // element 2i in the low nibble of byte i
+#pragma unroll
+          for (int q = 0; q < 4; ++q)
+            w |= ((bits[q].x & 0xFu) | ((bits[q].y & 0xFu) << 4)) << (8 * q);
+          __stcg(reinterpret_cast<unsigned int *>(codes) + ch, nz ? w : 0u);
         }
-        __stcg(reinterpret_cast<uint2 *>(codes) + li, make_uint2(lo, hi));
-      } else {
-        uint32_t w = 0u;  // element 2i in the low nibble of byte i
-#pragma unroll
-        for (int q = 0; q < 8; ++q) w |= ((uint32_t)(qc[q] & 0xF)) << (4 * q);
-        __stcg(reinterpret_cast<unsigned int *>(codes) + li, w);
       }
     }
   }
@@ -874,10 +915,8 @@ int launch_rows(const EvParams<NT> &p, bool delta, int sms, cudaStream_t st) {
   long long work;  // independent units of one set (pieces, or lane segments)
   int per_cta;
   if (KV == H2OKV_I8 || KV == H2OKV_I4) {
-    int L = 1;
-    while (L < p.d / 8) L <<= 1;
     work = (long long)p.S * 2;
-    per_cta = kRowWarps * (32 / L) * kQuantUnroll;
+    per_cta = kRowWarps * (32 / quant_lanes(p.d)) * kQuantUnroll;
   } else {
     work = (long long)p.S * 2 * (p.row_bytes / 16);
     per_cta = kRowThreads * kCopyUnroll;
