@@ -264,7 +264,7 @@ __device__ __forceinline__ void find_bin(const uint32_t *hs, uint32_t kk, uint32
 // the fill slots (mode 1) and, for a choosing call (mode 2), add the slice's histogram of
 // the top 11 key bits into the group's histogram in the workspace.
 template <int NT>
-__global__ void __launch_bounds__(kSelThreads)
+__global__ void __launch_bounds__(kSelThreads, 2)
     evict_fold_kernel(const __grid_constant__ EvParams<NT> p) {
   griddep_launch_dependents();  // the choose / row kernel may be scheduled
   const int unit = blockIdx.x / p.C, rank = blockIdx.x % p.C;
@@ -281,7 +281,7 @@ __global__ void __launch_bounds__(kSelThreads)
   const int j_begin = rank * p.slice;
   const int j_end = min(p.N_C, j_begin + p.slice);
   const bool fold = T.w_prev != nullptr;
-  constexpr int U = 4;
+  constexpr int U = 2;
   const int stride = 4 * kSelThreads;
   for (int j0 = j_begin + 4 * tid; j0 < j_end; j0 += stride * U) {
     float ks[U][4];
