@@ -30,6 +30,8 @@ CASES = [
     # tensor-core path: three row tiles and six slot tiles, both ragged; one slot tile
     wl_("bwd_bf16_tiles", Hq=8, Hk=2, capacity=700, chunk=300, seq_len=1500),
     wl_("bwd_bf16_one_tile", capacity=100, chunk=60, seq_len=300),
+    # an odd number of packed row tiles (MHA, three tiles): the last D-kernel CTA has one
+    wl_("bwd_bf16_mha_odd_tiles", Hq=2, Hk=2, capacity=500, chunk=300, seq_len=900),
     wl_("bwd_i8", kv_dtype="i8"),
     wl_("bwd_i4_mha", Hq=2, Hk=2, kv_dtype="i4", capacity=260, chunk=90, seq_len=700),
 ]
