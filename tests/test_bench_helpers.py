@@ -88,3 +88,15 @@ def test_stack_flops_and_bytes_scale_with_layers():
     per = 12 * 32768 + 4 * 2048 * 128 + 2 * 2048 * (64 + 2) + 8 * 2048
     assert one == per * 4 * 8
     assert bench.alg_flops_chunk(wl, 32768, 2048) == 4.0 * 4 * 32 * 2048 * 32768 * 128
+
+
+def test_eviction_bytes_of_the_named_layers():
+    from h2o_kv_cache_attn_b200.configs import SHORT
+    # the 128K bf16 layer: 8 groups of 12 N_C + 4 S d + 2 S row + 8 S bytes = 11.6 MB per chunk
+    one = bench.evict_bytes_chunk(SHORT["128k"], 1024)
+    assert one == (12 * 32768 + 4 * 1024 * 128 + 2 * 1024 * 256 + 8 * 1024) * 8
+    assert round(one / 1e6, 1) == 11.6
+    # the 36-layer int4 stack: 1152 groups, about 1.99 GB per chunk
+    wl = SHORT["int4stack"]
+    assert round(bench.evict_bytes_chunk(wl, wl.chunk) * wl.layers / 1e9, 2) == 1.99
+
