@@ -7,7 +7,9 @@
 //   dq_i = sum_j dS_ij k_j / sqrt(d),
 //   dk_j = sum over the group's heads and rows of dS_ij q_i / sqrt(d),
 //   dv_j = sum over the group's heads and rows of p_ij dy_i.
-// lse is the forward's natural-log row log-sum-exp.  CUDA cores, float32:
+// lse is the forward's natural-log row log-sum-exp.  A bf16 cache with d = 128 and bf16
+// queries goes to the tensor-core kernels of attn_bwd_tc.cu; every other combination
+// runs here, on CUDA cores, in float32:
 //   bwd_rows_kernel   one CTA per 32 packed rows of a group: pass 1 finds D_i,
 //                     pass 2 accumulates dq_i (no atomics);
 //   bwd_slots_kernel  one CTA per 32 slots of a group: streams every packed row of
