@@ -25,10 +25,10 @@
 //     encoding, and claims chosen or replayed slots (token position, score 0).
 //
 // A call over many caches of the same shape (independent layers) runs as the
-// same three launches over every (cache, group) (up to 48 caches per launch).  The quantizer must agree bit
-// for bit with an IEEE float32 reference: it uses correctly rounded division and
-// reciprocal, Markstein's correctly rounded quotient (quant_code) and __float2half_rn
-// only (this file is never built with fast-math).
+// same three launches over every (cache, group), up to 48 caches per launch.  The
+// quantizer must agree bit for bit with an IEEE float32 reference: it uses correctly
+// rounded division and reciprocal, Markstein's correctly rounded quotient (quant_code)
+// and __float2half_rn only (this file is never built with fast-math).
 #include <mutex>
 
 #include "h2okv_internal.cuh"
